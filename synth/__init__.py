@@ -1,0 +1,175 @@
+"""Seeded synthetic inputs for the Hymba hybrid-head mixer.
+
+This module is shared by the CPU oracle, the tests and the benchmark. It holds
+no arithmetic of the mixer itself: it only draws random numbers with numpy's
+PCG64 generator (reproducible on any machine) and rounds them to the storage
+type of the layer (bf16 or fp32), so that every consumer sees identical values.
+
+Value recipe (Hymba-1.5B shapes from the 51cto article "Hymba-1.5B", section 2
+"模型架构非常巧妙": d_model 1600, 25 attention heads, 16 SSM states, GQA, RoPE;
+the distributions are those of the synthetic workloads):
+
+* X ~ N(0, 1); projection weights ~ N(0, 1/fan_in) (the second argument of N is a
+  variance); meta tokens ~ N(0, 0.02).
+* A_log = log(u), u ~ Uniform[1, 16] continuous, iid per (channel, state).
+* dt bias b = softplus^-1(dt), dt = exp(Uniform[ln 1e-3, ln 1e-1]) per channel.
+* conv taps ~ N(0, 1/d_conv), conv bias 0; D = 1; RMSNorm gains 1; beta1 = beta2 = 1.
+"""
+from __future__ import annotations
+
+import dataclasses
+from typing import Dict, List, Optional
+
+import numpy as np
+
+F32 = 0
+BF16 = 1
+
+
+@dataclasses.dataclass(frozen=True)
+class LayerCfg:
+    d_model: int
+    n_q_heads: int
+    n_kv_heads: int
+    head_dim: int
+    v_head_dim: int
+    d_inner: int
+    d_state: int
+    d_conv: int
+    dt_rank: int
+    n_meta: int
+    window: int            # <= 0: global (full causal) attention
+    is_kv_producer: int    # 1: computes its own K/V; 0: reads a producer's K/V
+    dtype: int             # F32 or BF16 (activations and big weights)
+    rope_base: float = 10000.0
+    rms_eps: float = 1e-6
+
+    @property
+    def n_in(self) -> int:
+        """Width of the fused input projection: [Q | K | V | x | z | dt_low | B | C]."""
+        kv = self.n_kv_heads * (self.head_dim + self.v_head_dim) if self.is_kv_producer else 0
+        return (self.n_q_heads * self.head_dim + kv + 2 * self.d_inner
+                + self.dt_rank + 2 * self.d_state)
+
+    def with_(self, **kw) -> "LayerCfg":
+        return dataclasses.replace(self, **kw)
+
+
+def tiny_layer_cfg() -> LayerCfg:
+    return LayerCfg(d_model=256, n_q_heads=4, n_kv_heads=2, head_dim=64, v_head_dim=128,
+                    d_inner=512, d_state=16, d_conv=4, dt_rank=16, n_meta=16, window=64,
+                    is_kv_producer=1, dtype=F32)
+
+
+def hymba15_layer_cfg(window: int = 1024, producer: int = 1) -> LayerCfg:
+    return LayerCfg(d_model=1600, n_q_heads=25, n_kv_heads=5, head_dim=64, v_head_dim=128,
+                    d_inner=3200, d_state=16, d_conv=4, dt_rank=100, n_meta=128,
+                    window=window, is_kv_producer=producer, dtype=BF16)
+
+
+# Workloads, named by what they are.
+WORKLOADS: Dict[str, dict] = {
+    # tiny fp32 layer: B=1, T=256 + 16 meta, window 64
+    "tiny_f32_b1_t256": dict(kind="prefill", cfg=tiny_layer_cfg(), B=1, T=256, seed=0),
+    # Hymba-1.5B-shaped SWA layer: B=1, T=2048 + 128 meta, window 1024
+    "hymba15_swa1024_b1_t2048": dict(kind="prefill", cfg=hymba15_layer_cfg(1024), B=1, T=2048, seed=1),
+    # the same shape as a global layer: B=4, T=8192 + 128 meta
+    "hymba15_global_b4_t8192": dict(kind="prefill", cfg=hymba15_layer_cfg(0), B=4, T=8192, seed=2),
+    # decode step of a KV-sharing layer pair: B=64, prompt 4096 + 128 meta, ring 1024
+    "hymba15_decode_pair_b64_p4096": dict(kind="decode_pair", cfg=hymba15_layer_cfg(1024), B=64,
+                                          T=4096, seed=3),
+    # 32-layer mixer stack: B=8, T=4096 + 128 meta; layers 0/15/31 global; pairs share KV
+    "hymba15_stack32_b8_t4096": dict(kind="stack", cfg=hymba15_layer_cfg(1024), B=8, T=4096,
+                                     seed=4, n_layers=32, global_layers=(0, 15, 31)),
+}
+
+
+def stack_layer_cfgs(base: LayerCfg, n_layers: int, global_layers) -> List[LayerCfg]:
+    """Layer configs of a KV-sharing stack: pairs (2i, 2i+1), even layers produce."""
+    out = []
+    for l in range(n_layers):
+        w = 0 if l in global_layers else base.window
+        out.append(base.with_(window=w, is_kv_producer=1 if l % 2 == 0 else 0))
+    return out
+
+
+def round_bf16(a) -> np.ndarray:
+    """Round to the nearest bf16 value (ties to even), returned as float32."""
+    a32 = np.ascontiguousarray(a, dtype=np.float32)
+    u = a32.view(np.uint32).astype(np.uint64)
+    u = ((u + (((u >> 16) & 1) + 0x7FFF)) >> 16) << 16
+    return u.astype(np.uint32).view(np.float32)
+
+
+def to_storage(a, dtype: int) -> np.ndarray:
+    """Values as stored on the device (float32 array holding bf16- or fp32-exact values)."""
+    return round_bf16(a) if dtype == BF16 else np.ascontiguousarray(a, dtype=np.float32)
+
+
+def _rng(*tags) -> np.random.Generator:
+    return np.random.default_rng([int(t) for t in tags])
+
+
+def _normal(rng, shape, var):
+    return rng.standard_normal(shape) * np.sqrt(var)
+
+
+def layer_weights(cfg: LayerCfg, seed: int) -> Dict[str, np.ndarray]:
+    """Random-init weights of one mixer layer, as float32 arrays of storage-exact values.
+
+    Big matrices follow the [out, in] convention: w_in [n_in, d_model],
+    w_dt [d_inner, dt_rank], w_out [d_model, d_inner].
+    """
+    d, di, N, r = cfg.d_model, cfg.d_inner, cfg.d_state, cfg.dt_rank
+    H, G, dh, dv = cfg.n_q_heads, cfg.n_kv_heads, cfg.head_dim, cfg.v_head_dim
+    blocks = [("q", H * dh), ("k", G * dh), ("v", G * dv), ("x", di), ("z", di),
+              ("dtl", r), ("B", N), ("C", N)]
+    rows = []
+    for i, (name, width) in enumerate(blocks):
+        blk = _normal(_rng(seed, 1, i), (width, d), 1.0 / d)
+        if name in ("k", "v") and not cfg.is_kv_producer:
+            continue
+        rows.append(blk)
+    w_in = np.concatenate(rows, axis=0)
+    dt = np.exp(_rng(seed, 2).uniform(np.log(1e-3), np.log(1e-1), size=di))
+    w = {
+        "w_in": to_storage(w_in, cfg.dtype),
+        "w_dt": to_storage(_normal(_rng(seed, 3), (di, r), 1.0 / r), cfg.dtype),
+        "b_dt": np.log(np.expm1(dt)).astype(np.float32),
+        "conv_w": _normal(_rng(seed, 4), (di, cfg.d_conv), 1.0 / cfg.d_conv).astype(np.float32),
+        "conv_b": np.zeros(di, np.float32),
+        "A_log": np.log(_rng(seed, 5).uniform(1.0, 16.0, size=(di, N))).astype(np.float32),
+        "D": np.ones(di, np.float32),
+        "norm_attn_w": np.ones(H * dv, np.float32),
+        "norm_ssm_w": np.ones(di, np.float32),
+        "beta1": np.ones(H * dv, np.float32),
+        "beta2": np.ones(di, np.float32),
+        "w_out": to_storage(_normal(_rng(seed, 6), (d, di), 1.0 / di), cfg.dtype),
+        "meta": to_storage(_normal(_rng(seed, 7), (cfg.n_meta, d), 0.02), cfg.dtype),
+    }
+    return w
+
+
+def layer_input(cfg: LayerCfg, B: int, T: int, seed: int, tag: int = 0) -> np.ndarray:
+    """User-token input X ~ N(0, 1), [B, T, d_model], storage-exact float32."""
+    return to_storage(_rng(seed, 100, tag).standard_normal((B, T, cfg.d_model)), cfg.dtype)
+
+
+def perturbed_weights(w: Dict[str, np.ndarray], cfg: LayerCfg, seed: int,
+                      scale: float = 0.5) -> Dict[str, np.ndarray]:
+    """Copy of w with the per-channel parameters (conv bias, D, gains, betas) drawn away
+    from their defaults, so that tests exercise every term of the layer."""
+    out = dict(w)
+    di = cfg.d_inner
+    g = _rng(seed, 9)
+    out["conv_b"] = (g.standard_normal(di) * 0.2).astype(np.float32)
+    out["D"] = (1.0 + g.standard_normal(di) * scale).astype(np.float32)
+    out["norm_attn_w"] = (1.0 + g.standard_normal(w["norm_attn_w"].shape) * scale).astype(np.float32)
+    out["norm_ssm_w"] = (1.0 + g.standard_normal(di) * scale).astype(np.float32)
+    out["beta1"] = (1.0 + g.standard_normal(w["beta1"].shape) * scale).astype(np.float32)
+    out["beta2"] = (1.0 + g.standard_normal(di) * scale).astype(np.float32)
+    return out
+
+
+def workload(name: str) -> dict:
+    return dict(WORKLOADS[name])

@@ -1,0 +1,146 @@
+"""Pins of the oracle's whole layer: decode-by-decode equals prefill (through the
+ring-buffer wrap), cross-layer KV sharing, fusion invariants, and the pages'
+printed cache sizes.
+
+Sources: "Hymba Guide", Cross-Layer KV Cache Sharing (a secondary layer reuses the
+primary layer's K and V with no new buffer); "Lecture 04", section 1 (the decode
+cache gains one K, V per token) and section 8 (kv_cache_gb, ssm_state_gb and their
+printed values); "Jamba: Hybrid SSM-Transformer", section 2 and the Worked Example.
+"""
+import json
+import os
+
+import numpy as np
+import pytest
+
+import oracle
+import synth
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "cache_sizes.json")
+
+
+def _pair(window=8, seed=21):
+    base = synth.tiny_layer_cfg().with_(window=window)
+    ca = base.with_(is_kv_producer=1)
+    cb = base.with_(is_kv_producer=0)
+    wa = synth.perturbed_weights(synth.layer_weights(ca, seed), ca, seed)
+    wb = synth.perturbed_weights(synth.layer_weights(cb, seed + 1), cb, seed + 1)
+    return ca, cb, wa, wb
+
+
+@pytest.mark.parametrize("window", [8, 0])
+def test_decode_by_decode_equals_prefill_pair(window):
+    """Prefill T0 tokens then decode the rest one at a time through a KV-sharing
+    pair (residual stack) equals prefilling all T tokens. With window 8 the ring
+    of 8 slots wraps several times."""
+    ca, cb, wa, wb = _pair(window)
+    B, T, T0 = 2, 30, 10
+    m = ca.n_meta
+    x = synth.layer_input(ca, B, T, 31)
+    # reference: the whole sequence at once
+    ra = oracle.mixer_prefill(ca, wa, x, residual=True)
+    rb = oracle.mixer_prefill(cb, wb, ra["y"], kv_shared=(ra["k"], ra["v"]), residual=True, x_has_meta=True)
+    # prefill T0, then decode
+    pa = oracle.mixer_prefill(ca, wa, x[:, :T0], residual=True)
+    pb = oracle.mixer_prefill(cb, wb, pa["y"], kv_shared=(pa["k"], pa["v"]), residual=True, x_has_meta=True)
+    cap = m + (window if window > 0 else T)
+    cache = oracle.cache_from_prefill(ca, pa["k"], pa["v"], cap)
+    ha, conva = pa["h"].copy(), pa["conv"].copy()
+    hb, convb = pb["h"].copy(), pb["conv"].copy()
+    for t in range(T0, T):
+        ya = oracle.mixer_decode(ca, wa, x[:, t], cache, ha, conva, residual=True)
+        yb = oracle.mixer_decode(cb, wb, ya, cache, hb, convb, residual=True)
+        np.testing.assert_allclose(ya, ra["y"][:, m + t], rtol=1e-10, atol=1e-10)
+        np.testing.assert_allclose(yb, rb["y"][:, m + t], rtol=1e-10, atol=1e-10)
+        assert list(cache["len"]) == [m + t + 1] * B
+    np.testing.assert_allclose(ha, ra["h"], rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(hb, rb["h"], rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(conva, ra["conv"], rtol=0, atol=1e-12)
+
+
+def test_ring_slots_closed_form():
+    """Meta positions keep slots 0..m-1; position p >= m goes to m + (p - m) mod R."""
+    m, R = 3, 4
+    got = [oracle.ring_slot(p, m, R) for p in range(13)]
+    assert got == [0, 1, 2, 3, 4, 5, 6, 3, 4, 5, 6, 3, 4]
+    cfg = synth.tiny_layer_cfg().with_(n_meta=m)
+    k = np.arange(13, dtype=np.float64).reshape(1, 1, 13, 1) * np.ones((1, 1, 13, 2))
+    c = oracle.cache_from_prefill(cfg, k, k, m + R)
+    np.testing.assert_array_equal(c["k"][0, 0, :, 0], [0, 1, 2, 11, 12, 9, 10])
+
+
+def test_kv_share_consumer_equals_producer_with_same_kv():
+    """A consumer reading K, V handed over from a producer (no K/V rows of its own)
+    equals the producer itself when the handed-over K, V are the producer's."""
+    cfg = synth.tiny_layer_cfg()
+    w = synth.perturbed_weights(synth.layer_weights(cfg, 41), cfg, 41)
+    x = synth.layer_input(cfg, 1, 20, 41)
+    rp = oracle.mixer_prefill(cfg, w, x)
+    cc = cfg.with_(is_kv_producer=0)
+    H, G, dh, dv, d = cfg.n_q_heads, cfg.n_kv_heads, cfg.head_dim, cfg.v_head_dim, cfg.d_model
+    wc = dict(w)
+    wc["w_in"] = np.concatenate([w["w_in"][:H * dh], w["w_in"][H * dh + G * (dh + dv):]], axis=0)
+    assert wc["w_in"].shape[0] == cc.n_in
+    rc = oracle.mixer_prefill(cc, wc, x, kv_shared=(rp["k"], rp["v"]))
+    np.testing.assert_allclose(rc["y"], rp["y"], rtol=1e-12, atol=1e-12)
+
+
+def test_rmsnorm_scale_invariance_and_unit_rms():
+    g = np.random.default_rng(51)
+    a = g.standard_normal((7, 33))
+    one = np.ones(33)
+    n = oracle.rms_norm(a, one, 0.0)
+    np.testing.assert_allclose(oracle.rms_norm(3.7 * a, one, 0.0), n, rtol=1e-13)
+    np.testing.assert_allclose(np.sqrt(np.mean(n * n, axis=1)), 1.0, rtol=1e-13)
+    gain = g.standard_normal(33)
+    np.testing.assert_allclose(oracle.rms_norm(a, gain, 0.0), gain * n, rtol=1e-13)
+
+
+def test_fuse_beta2_zero_drops_ssm_branch():
+    g = np.random.default_rng(52)
+    di = 12
+    w = {"norm_attn_w": g.standard_normal(di), "norm_ssm_w": g.standard_normal(di),
+         "beta1": g.standard_normal(di), "beta2": np.zeros(di)}
+    o = g.standard_normal((5, di))
+    u1 = oracle.fuse(o, g.standard_normal((5, di)), w, 1e-6)
+    u2 = oracle.fuse(o, g.standard_normal((5, di)) * 100.0, w, 1e-6)
+    np.testing.assert_array_equal(u1, u2)
+    # the average: equal branches with unit gains and betas give RMS(a)
+    w1 = {k: np.ones(di) for k in w}
+    np.testing.assert_allclose(oracle.fuse(o, o, w1, 0.0), oracle.rms_norm(o, np.ones(di), 0.0), rtol=1e-14)
+
+
+def test_cache_sizes_match_pages():
+    gold = json.load(open(GOLDEN))
+    ex = gold["jamba_worked_example"]
+    assert oracle.kv_cache_bytes(1, 8, 128, 1, 1, 2) == ex["bytes_per_token_layer"]
+    assert oracle.kv_cache_bytes(1, 8, 128, 1, 1, 1) == ex["elements_per_token_layer"]
+    assert oracle.kv_cache_bytes(32, 8, 128, 1, 1, 2) == ex["bytes_per_token_32_layers"]
+    assert oracle.kv_cache_bytes(32, 8, 128, 64000, 4, 2) == ex["dense_32_layers_bytes"]
+    assert oracle.kv_cache_bytes(4, 8, 128, 64000, 4, 2) == ex["hybrid_4_layers_bytes"]
+    code = gold["jamba_code_output"]
+    t = oracle.kv_cache_bytes(32, 8, 128, code["seq_len"], 1, 2) / 1024 ** 3
+    h = oracle.kv_cache_bytes(32 // 8, 8, 128, code["seq_len"], 1, 2) / 1024 ** 3
+    assert f"{t:.2f}" == code["transformer_gib_2dp"]
+    assert f"{h:.2f}" == code["hybrid_gib_2dp"]
+    assert f"{t / h:.1f}" == code["factor_1dp"]
+    lec = gold["lecture04_section8"]
+    dense70 = oracle.kv_cache_bytes(80, 8, 128, 128_000, 1, 2) / 1e9
+    state = oracle.ssm_state_bytes(64, 64 * 64, 128, 1, 2) / 1e9
+    dense7 = oracle.kv_cache_bytes(32, 8, 128, 128_000, 1, 2) / 1e9
+    assert round(dense70) == lec["dense70b_128k_gb_approx"]
+    assert round(state, 2) == lec["ssm_state_gb_approx"]
+    assert round(dense7) == lec["dense7b_128k_gb_approx"]
+    assert round(dense7 / state, -1) == lec["ratio_approx"]
+
+
+def test_layer_cache_bytes_formula():
+    """KV slots (meta + window) for a producer, fp32 state, conv state, lengths."""
+    cfg = synth.hymba15_layer_cfg(1024)
+    B = 64
+    kv = B * 5 * (128 + 1024) * (64 + 128) * 2
+    h = B * 3200 * 16 * 4
+    conv = B * 3200 * 4 * 2
+    assert oracle.layer_cache_bytes(cfg, B, 4096 + 128) == kv + h + conv + B * 4
+    g = cfg.with_(window=0)
+    assert oracle.layer_cache_bytes(g, B, 5000) == B * 5 * (128 + 5000) * 192 * 2 + h + conv + B * 4
