@@ -1,0 +1,413 @@
+"""Benchmark of the B200 Hymba hybrid-head mixer.
+
+One step = one hymba_mixer_prefill of the Hymba-1.5B-shaped SWA layer (B=1, T=2048
+user tokens + 128 meta tokens, window 1024, bf16): the fused projection with RoPE
+and K/V write, Delta projection, meta+window GQA attention, conv + selective scan,
+fusion epilogue and output projection. The decode step of the KV-sharing layer pair
+(B=64, 1024-slot ring + 128 meta, fp32 state [64, 3200, 16]) is timed the same way
+and reported under "decode".
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Under torchrun each rank runs its own replica (weak scaling, no collective on the
+data path); rank 0 prints one JSON line. --impl reference times the CPU oracle on a
+bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+WORKLOAD = "hymba15_swa1024_b1_t2048"
+DECODE_WORKLOAD = "hymba15_decode_pair_b64_p4096"
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return dict(hbm=d["hbm_gbs"], bf16=d["bf16_tflops"], bf16_sus=d["bf16_tflops_sustained"],
+                    src="measured")
+    return dict(hbm=6650.0, bf16=1590.0, bf16_sus=1400.0, src="fallback")
+
+
+class Clocks:
+    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{index}.csv")
+
+    def start(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.f.close()
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def visible_pairs(Tp, m, W):
+    i = np.arange(Tp)[:, None]
+    j = np.arange(Tp)[None, :]
+    vis = (j <= i) & ((j < m) | (i - j < W) if W > 0 else True)
+    return int(vis.sum())
+
+
+def prefill_work(cfg, B, T):
+    """Algorithmic FLOPs / bytes per launch of each prefill kernel."""
+    m, Tp = cfg.n_meta, cfg.n_meta + T
+    H, G, dh, dv, di, d, r = (cfg.n_q_heads, cfg.n_kv_heads, cfg.head_dim, cfg.v_head_dim,
+                              cfg.d_inner, cfg.d_model, cfg.dt_rank)
+    rows = B * Tp
+    pairs = visible_pairs(Tp, m, cfg.window)
+    return {
+        "gemm_in_proj": ("tensor", 2.0 * B * T * cfg.n_in * d),
+        "gemm_in_proj_meta": ("tensor", 2.0 * m * cfg.n_in * d),
+        "gemm_dt_proj": ("tensor", 2.0 * rows * di * r),
+        "attn_prefill": ("tensor", 2.0 * B * pairs * H * (dh + dv)),
+        "attn_prefill_simt": ("tensor", 2.0 * B * pairs * H * (dh + dv)),
+        # x (2 B) + Delta (4 B) read, y_pre (2 B) written per (row, channel); B, C per row
+        "conv_scan_prefill": ("hbm", rows * di * 8.0 + rows * 2 * 16 * 2.0),
+        # O, y_pre, z read, U written: 2 B each per (row, channel)
+        "fuse": ("hbm", rows * di * 8.0),
+        "gemm_out_proj": ("tensor", 2.0 * rows * d * di),
+    }
+
+
+def decode_work(cfg, B, cap):
+    """Algorithmic HBM bytes per launch of the decode kernels (2-byte K/V, fp32 state)."""
+    G, dh, dv, di = cfg.n_kv_heads, cfg.head_dim, cfg.v_head_dim, cfg.d_inner
+    return {
+        "attn_decode": ("hbm", B * G * cap * (dh + dv) * 2.0),
+        "ssm_decode": ("hbm", B * di * (16 * 4 * 2 + 4 * 4 * 2 + 4 + 2 + 2)),
+        "gemm_in_proj_decode": ("hbm", cfg.n_in * cfg.d_model * 2.0),
+        "gemm_out_proj_decode": ("hbm", cfg.d_model * di * 2.0),
+    }
+
+
+def cpu_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def oracle_sample(T_sample: int):
+    """Time the CPU oracle on the first T_sample tokens of the workload's sequence."""
+    import oracle
+    wl = synth.workload(WORKLOAD)
+    cfg = wl["cfg"]
+    w = synth.layer_weights(cfg, wl["seed"])
+    x = synth.layer_input(cfg, wl["B"], wl["T"], wl["seed"])[:, :T_sample]
+    t0 = time.perf_counter()
+    oracle.mixer_prefill(cfg, w, x)
+    dt = time.perf_counter() - t0
+    return x.shape[0] * x.shape[1] / dt, dt
+
+
+def run_reference(args, rank):
+    if rank != 0:
+        return
+    T_sample = 512
+    vals = []
+    for i in range(args.warmup + args.steps):
+        v, _ = oracle_sample(T_sample)
+        if i >= args.warmup:
+            vals.append(v)
+    v = statistics.median(vals)
+    wl = synth.workload(WORKLOAD)
+    sample = f"first {T_sample} of {wl['T']} user tokens of the B=1 sequence (+128 meta rows)"
+    print(json.dumps({
+        "impl": "reference", "metric": "hybrid-head mixer prefill tokens/s", "value": v,
+        "unit": "tokens/s", "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "higher_is_better": True, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "B": wl["B"], "T": wl["T"], "n_meta": 128, "window": 1024},
+        "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": cpu_cores(), "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }))
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-decode", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if args.impl == "reference":
+        return run_reference(args, rank)
+
+    import ctypes
+    import torch
+    import torch.distributed as dist
+    import hybrid_head_ssm_b200 as hy
+    from hybrid_head_ssm_b200 import runtime as rt
+
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(v):
+        if world == 1:
+            return v
+        t = torch.tensor([v], dtype=torch.float64, device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    pk = peaks()
+    wl = synth.workload(WORKLOAD)
+    cfg, B, T = wl["cfg"], wl["B"], wl["T"]
+    Tp = cfg.n_meta + T
+    w = synth.layer_weights(cfg, wl["seed"])
+    x_np = synth.layer_input(cfg, B, T, wl["seed"] + rank)
+    layer = rt.DeviceLayer(cfg, w)
+    x = rt.to_device(x_np, cfg)
+    y = torch.empty((B, Tp, cfg.d_model), dtype=torch.bfloat16, device="cuda")
+    kv = rt.KV(cfg, B, seq_cap=Tp)
+    ws = rt.workspace(cfg, B, T, hy.HYMBA_MODE_PREFILL)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")  # > 126 MB L2
+    stream = torch.cuda.current_stream()
+
+    def step():
+        rt.prefill(layer, x, T, kv, y, ws, None, 0)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+
+    # ---- timed region: K steps, L2 flushed between steps (outside the step events)
+    clocks = Clocks(local)
+    clocks.start()
+    hy.hymba_trace_enable(1)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    launches0 = hy.hymba_launch_count()
+    barrier()
+    torch.cuda.synchronize()
+    for i in range(args.steps):
+        flush.fill_(i & 0xFF)
+        ev[i][0].record(stream)
+        step()
+        ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    launches = hy.hymba_launch_count() - launches0
+    trace = hy.trace_collect()
+    hy.hymba_trace_enable(0)
+    clk = clocks.stop()
+    step_ms = [a.elapsed_time(b) for a, b in ev]
+    ms = max_over_ranks(sum(step_ms) / len(step_ms))
+    tokens = B * T * world
+    value = tokens / (ms * 1e-3)
+
+    # per-kernel times over the timed region
+    per = {}
+    for name, t in trace:
+        per.setdefault(name, []).append(t)
+    work = prefill_work(cfg, B, T)
+    kern = {n: {"launches": len(v), "avg_us": 1e3 * sum(v) / len(v), "share": sum(v) / max(sum(map(sum, per.values())), 1e-9)}
+            for n, v in per.items()}
+    dom = max(per, key=lambda n: sum(per[n]))
+    bound, units = work.get(dom, ("hbm", 0.0))
+    avg_s = sum(per[dom]) / len(per[dom]) * 1e-3
+    if bound == "tensor":
+        ach = units / avg_s / 1e12
+        roof = {"kernel": dom, "bound": "tensor", "achieved": ach, "peak": pk["bf16_sus"], "unit": "TFLOP/s",
+                "frac": ach / pk["bf16_sus"], "peak_kind": f"bf16 sustained, {pk['src']}"}
+    else:
+        ach = units / avg_s / 1e9
+        roof = {"kernel": dom, "bound": "hbm", "achieved": ach, "peak": pk["hbm"], "unit": "GB/s",
+                "frac": ach / pk["hbm"], "peak_kind": f"HBM copy, {pk['src']}"}
+    roof["traffic"] = None
+    for n, (bd, u) in work.items():
+        if n in per:
+            a = sum(per[n]) / len(per[n]) * 1e-3
+            kern[n]["achieved"] = u / a / (1e12 if bd == "tensor" else 1e9)
+            kern[n]["unit"] = "TFLOP/s" if bd == "tensor" else "GB/s"
+
+    # ---- end to end through the public API with host buffers
+    x_host = x.cpu().pin_memory()
+    y_host = torch.empty(y.shape, dtype=y.dtype).pin_memory()
+    e2e_ms = []
+    for i in range(args.warmup + args.steps):
+        flush.fill_(i & 0xFF)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        x.copy_(x_host, non_blocking=True)
+        step()
+        y_host.copy_(y, non_blocking=True)
+        b.record(stream)
+        torch.cuda.synchronize()
+        if i >= args.warmup:
+            e2e_ms.append(a.elapsed_time(b))
+    e2e_ms_step = max_over_ranks(sum(e2e_ms) / len(e2e_ms))
+
+    # ---- decode step of the KV-sharing pair (B=64, ring 1024 + 128 meta)
+    dec = None
+    if not args.no_decode:
+        dec = bench_decode(args, torch, hy, rt, max_over_ranks, barrier, world, pk, flush)
+
+    out = None
+    if rank == 0:
+        cpu = None
+        if world == 1 and not args.no_cpu_baseline:
+            v, dt = oracle_sample(T)
+            cpu = {"value": v, "unit": "tokens/s", "cores": cpu_cores(), "kind": "oracle",
+                   "sample": f"one full sequence of the workload (B=1, T={T} + 128 meta), {dt:.1f} s"}
+        out = {
+            "metric": "hybrid-head mixer prefill tokens/s", "value": value, "unit": "tokens/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic",
+            "config": {"workload": WORKLOAD, "B": B, "T": T, "n_meta": cfg.n_meta, "window": cfg.window,
+                       "d_model": cfg.d_model, "d_inner": cfg.d_inner, "per_rank_batch": B,
+                       "l2": "flushed between steps (256 MB write outside the step events)"},
+            "roofline": roof,
+            "cpu_baseline": cpu,
+            "e2e": {"value": tokens / (e2e_ms_step * 1e-3), "unit": "tokens/s",
+                    "h2d_bytes_per_step": x.numel() * x.element_size(),
+                    "d2h_bytes_per_step": y.numel() * y.element_size()},
+            "gpu_launches": int(launches),
+            "clocks": clk,
+            "kernels": kern,
+            "decode": dec,
+        }
+        print(json.dumps(out))
+    if world > 1:
+        dist.destroy_process_group()
+    return out
+
+
+def bench_decode(args, torch, hy, rt, max_over_ranks, barrier, world, pk, flush):
+    wl = synth.workload(DECODE_WORKLOAD)
+    ca = wl["cfg"]
+    cb = ca.with_(is_kv_producer=0)
+    B, T, seed = wl["B"], wl["T"], wl["seed"]
+    la = rt.DeviceLayer(ca, synth.layer_weights(ca, seed * 1000))
+    lb = rt.DeviceLayer(cb, synth.layer_weights(cb, seed * 1000 + 1))
+    cap = ca.n_meta + ca.window
+    Tp = ca.n_meta + T
+    import ctypes
+    kv = rt.KV(ca, B, seq_cap=Tp, cache_cap=cap)
+    kvb = hy.hymba_kv()
+    hy.check(hy.hymba_kv_share(ctypes.byref(kv.s), ctypes.byref(lb.c), ctypes.byref(kvb)))
+    sa, sb = rt.State(ca, B), rt.State(cb, B)
+    x = rt.to_device(synth.layer_input(ca, B, T, seed), ca)
+    ya = torch.empty((B, Tp, ca.d_model), dtype=torch.bfloat16, device="cuda")
+    yb = torch.empty_like(ya)
+    wsp = rt.workspace(ca, B, T, hy.HYMBA_MODE_PREFILL)
+    rt.prefill(la, x, T, kv, ya, wsp, sa, hy.HYMBA_ADD_RESIDUAL)
+    rt.prefill(lb, ya, T, kv, yb, wsp, sb, hy.HYMBA_X_HAS_META | hy.HYMBA_ADD_RESIDUAL, kv_struct_override=kvb)
+    del wsp, ya, yb
+    xt = rt.to_device(synth.layer_input(ca, B, 1, seed, tag=1)[:, 0], ca)
+    ha, hb = torch.empty_like(xt), torch.empty_like(xt)
+    wda = rt.workspace(ca, B, cap, hy.HYMBA_MODE_DECODE)
+    wdb = rt.workspace(cb, B, cap, hy.HYMBA_MODE_DECODE)
+    len0 = kv.len.clone()
+    stream = torch.cuda.current_stream()
+
+    def step():
+        rt.decode(la, xt, kv.s, sa, ha, wda, hy.HYMBA_ADD_RESIDUAL)
+        rt.decode(lb, ha, kvb, sb, hb, wdb, hy.HYMBA_ADD_RESIDUAL)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    hy.hymba_trace_enable(1)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    barrier()
+    torch.cuda.synchronize()
+    for i in range(args.steps):
+        flush.fill_(i & 0xFF)
+        ev[i][0].record(stream)
+        step()
+        ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    trace = hy.trace_collect()
+    hy.hymba_trace_enable(0)
+    ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in ev) / args.steps)
+    per = {}
+    for name, t in trace:
+        per.setdefault(name, []).append(t)
+    work = decode_work(ca, B, cap)
+    kern = {}
+    for n, v in per.items():
+        kern[n] = {"launches": len(v), "avg_us": 1e3 * sum(v) / len(v)}
+        if n in work:
+            a = sum(v) / len(v) * 1e-3
+            kern[n]["achieved_gbs"] = work[n][1] / a / 1e9
+            kern[n]["frac_hbm"] = kern[n]["achieved_gbs"] / pk["hbm"]
+    # the whole step's algorithmic bytes: both layers' weights, the shared KV read
+    # twice, state read+write twice
+    step_bytes = (2 * decode_work(ca, B, cap)["attn_decode"][1]
+                  + (ca.n_in + cb.n_in) * ca.d_model * 2.0 + 2 * ca.d_model * ca.d_inner * 2.0
+                  + 2 * decode_work(ca, B, cap)["ssm_decode"][1])
+    assert kv.len[0].item() >= len0[0].item()
+    return {"workload": DECODE_WORKLOAD, "tokens_per_s": B * world / (ms * 1e-3), "ms_per_step": ms,
+            "step_bytes": step_bytes, "step_gbs": step_bytes / (ms * 1e-3) / 1e9,
+            "step_frac_hbm": step_bytes / (ms * 1e-3) / 1e9 / pk["hbm"], "kernels": kern}
+
+
+if __name__ == "__main__":
+    main()

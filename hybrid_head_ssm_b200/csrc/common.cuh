@@ -1,0 +1,120 @@
+// Shared device helpers and the host-side launch context of libhymba.
+#pragma once
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <stdint.h>
+
+#include "../../include/hymba.h"
+
+namespace hymba {
+
+typedef __nv_bfloat16 bf16;
+typedef __half f16;
+
+// ---------------------------------------------------------------------------
+// host: launch context and tracing (defined in hymba_abi.cu)
+// ---------------------------------------------------------------------------
+struct Ctx {
+    cudaStream_t stream;
+    int* status;   // device status word of the current device
+    int sm_count;
+};
+
+void trace_before(const Ctx& ctx);
+// records the end event, counts the launch and checks the launch error; returns true on error
+bool trace_after(const Ctx& ctx, const char* name);
+
+#define HYMBA_LAUNCH(ctx, name, kernel, grid, block, smem, ...)                 \
+    do {                                                                        \
+        ::hymba::trace_before(ctx);                                             \
+        kernel<<<(grid), (block), (smem), (ctx).stream>>>(__VA_ARGS__);         \
+        if (::hymba::trace_after((ctx), (name))) return HYMBA_ERR_CUDA;         \
+    } while (0)
+
+static inline int ceil_div(long long a, long long b) { return (int)((a + b - 1) / b); }
+static inline long long round_up(long long a, long long b) { return (a + b - 1) / b * b; }
+
+// ---------------------------------------------------------------------------
+// device: dtype conversions, status word, fast exp2
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ float to_f(float v) { return v; }
+__device__ __forceinline__ float to_f(bf16 v) { return __bfloat162float(v); }
+__device__ __forceinline__ float to_f(f16 v) { return __half2float(v); }
+
+template <typename T> __device__ __forceinline__ T from_f(float v);
+template <> __device__ __forceinline__ float from_f<float>(float v) { return v; }
+template <> __device__ __forceinline__ bf16 from_f<bf16>(float v) { return __float2bfloat16_rn(v); }
+template <> __device__ __forceinline__ f16 from_f<f16>(float v) { return __float2half_rn(v); }
+
+__device__ __forceinline__ void set_status(int* status, int code) {
+    if (status) atomicCAS(status, 0, code);
+}
+
+// 2^x on the MUFU unit (ex2.approx, flush-to-zero).
+__device__ __forceinline__ float fast_exp2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+__device__ __forceinline__ float silu_f(float u) { return u / (1.0f + expf(-u)); }
+
+__device__ __forceinline__ float softplus_f(float u) {
+    return u > 20.0f ? u : log1pf(expf(u));
+}
+
+// Store n (<= 64) consecutive fp32 values as T at dst (16-byte vector stores when
+// the run is full and aligned).
+template <typename T>
+__device__ __forceinline__ void store_run(T* dst, const float* v, int n);
+
+template <>
+__device__ __forceinline__ void store_run<float>(float* dst, const float* v, int n) {
+    if (n == 64 && ((uintptr_t)dst & 15) == 0) {
+#pragma unroll
+        for (int i = 0; i < 64; i += 4)
+            *reinterpret_cast<float4*>(dst + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
+    } else {
+        for (int i = 0; i < n; ++i) dst[i] = v[i];
+    }
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+    __nv_bfloat162 p = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&p);
+}
+
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+    __half2 p = __floats2half2_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&p);
+}
+
+template <typename T>
+__device__ __forceinline__ uint32_t pack2(float lo, float hi);
+template <> __device__ __forceinline__ uint32_t pack2<bf16>(float lo, float hi) { return pack_bf16x2(lo, hi); }
+template <> __device__ __forceinline__ uint32_t pack2<f16>(float lo, float hi) { return pack_f16x2(lo, hi); }
+
+template <typename T>
+__device__ __forceinline__ void store_run16(T* dst, const float* v, int n) {
+    if (n == 64 && ((uintptr_t)dst & 15) == 0) {
+#pragma unroll
+        for (int i = 0; i < 64; i += 8) {
+            uint4 q;
+            q.x = pack2<T>(v[i], v[i + 1]);
+            q.y = pack2<T>(v[i + 2], v[i + 3]);
+            q.z = pack2<T>(v[i + 4], v[i + 5]);
+            q.w = pack2<T>(v[i + 6], v[i + 7]);
+            *reinterpret_cast<uint4*>(dst + i) = q;
+        }
+    } else {
+        for (int i = 0; i < n; ++i) dst[i] = from_f<T>(v[i]);
+    }
+}
+
+template <>
+__device__ __forceinline__ void store_run<bf16>(bf16* dst, const float* v, int n) { store_run16<bf16>(dst, v, n); }
+template <>
+__device__ __forceinline__ void store_run<f16>(f16* dst, const float* v, int n) { store_run16<f16>(dst, v, n); }
+
+}  // namespace hymba

@@ -1,0 +1,520 @@
+// The C ABI of libhymba.so: argument checks, workspace planning, and the order of
+// kernel launches of one mixer layer (prefill and decode). Every step of the layer
+// runs in the kernels of this library; this file only queues them on the caller's
+// stream.
+#include <algorithm>
+#include <atomic>
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+#include "kernels.h"
+
+namespace hymba {
+
+// ---------------------------------------------------------------------------
+// device status word (one per device that loads the library)
+// ---------------------------------------------------------------------------
+__device__ int g_status_word;
+
+static std::mutex g_mu;
+static int* g_status_ptr[64];
+static int g_sm_count[64];
+
+static int current_ctx(cudaStream_t stream, Ctx* ctx) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return HYMBA_ERR_CUDA;
+    if (!g_status_ptr[dev]) {
+        std::lock_guard<std::mutex> lk(g_mu);
+        if (!g_status_ptr[dev]) {
+            void* p = nullptr;
+            if (cudaGetSymbolAddress(&p, g_status_word) != cudaSuccess) return HYMBA_ERR_CUDA;
+            int sms = 0;
+            if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+                return HYMBA_ERR_CUDA;
+            g_sm_count[dev] = sms;
+            g_status_ptr[dev] = static_cast<int*>(p);
+        }
+    }
+    ctx->stream = stream;
+    ctx->status = g_status_ptr[dev];
+    ctx->sm_count = g_sm_count[dev];
+    return HYMBA_OK;
+}
+
+// ---------------------------------------------------------------------------
+// tracing and launch counting
+// ---------------------------------------------------------------------------
+struct TraceRec {
+    cudaEvent_t a, b;
+    const char* name;
+};
+static constexpr int kTracePool = 8192;
+static std::atomic<int> g_trace_on{0};
+static std::atomic<unsigned long long> g_launches{0};
+static std::vector<TraceRec> g_trace;
+static std::atomic<int> g_trace_used{0};
+static thread_local int t_trace_slot = -1;
+
+void trace_before(const Ctx& ctx) {
+    t_trace_slot = -1;
+    if (!g_trace_on.load(std::memory_order_relaxed)) return;
+    const int slot = g_trace_used.fetch_add(1);
+    if (slot >= (int)g_trace.size()) return;
+    t_trace_slot = slot;
+    cudaEventRecord(g_trace[slot].a, ctx.stream);
+}
+
+bool trace_after(const Ctx& ctx, const char* name) {
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    const cudaError_t err = cudaGetLastError();
+    if (t_trace_slot >= 0) {
+        g_trace[t_trace_slot].name = name;
+        cudaEventRecord(g_trace[t_trace_slot].b, ctx.stream);
+        t_trace_slot = -1;
+    }
+    return err != cudaSuccess;
+}
+
+// ---------------------------------------------------------------------------
+// configuration checks and workspace plan
+// ---------------------------------------------------------------------------
+static int check_cfg(const hymba_layer_cfg* c) {
+    if (!c) return HYMBA_ERR_INVALID_ARG;
+    if (c->d_model <= 0 || c->n_q_heads <= 0 || c->n_kv_heads <= 0 || c->d_inner <= 0 ||
+        c->dt_rank <= 0 || c->n_meta < 0 || (c->dtype != HYMBA_F32 && c->dtype != HYMBA_BF16) ||
+        !(c->rms_eps >= 0.f) || !(c->rope_base > 0.f))
+        return HYMBA_ERR_INVALID_ARG;
+    if (c->head_dim != 64 || c->d_state != 16 || c->d_conv != 4) return HYMBA_ERR_UNSUPPORTED;
+    if (c->n_q_heads % c->n_kv_heads) return HYMBA_ERR_UNSUPPORTED;
+    if (c->n_q_heads / c->n_kv_heads > 8) return HYMBA_ERR_UNSUPPORTED;
+    if (c->v_head_dim * c->n_q_heads != c->d_inner || c->v_head_dim != 128) return HYMBA_ERR_UNSUPPORTED;
+    if (c->d_model % 64 || c->d_inner % 64) return HYMBA_ERR_UNSUPPORTED;
+    return HYMBA_OK;
+}
+
+struct Cols {
+    int n_in, x, z, dtl, Bc, Cc;
+};
+
+static Cols columns(const hymba_layer_cfg* c) {
+    Cols k;
+    const int q = c->n_q_heads * c->head_dim;
+    const int kv = c->is_kv_producer ? c->n_kv_heads * (c->head_dim + c->v_head_dim) : 0;
+    k.x = q + kv;
+    k.z = k.x + c->d_inner;
+    k.dtl = k.z + c->d_inner;
+    k.Bc = k.dtl + c->dt_rank;
+    k.Cc = k.Bc + c->d_state;
+    k.n_in = k.Cc + c->d_state;
+    return k;
+}
+
+struct Plan {
+    size_t total = 0;
+    size_t rope = 0, P = 0, delta = 0, O = 0, ypre = 0, U = 0, wdt = 0, part = 0;
+    long long ldP = 0;
+    int rpad = 0, n_split = 1;
+};
+
+static size_t take(size_t* cur, size_t bytes) {
+    const size_t off = *cur;
+    *cur += (bytes + 255) / 256 * 256;
+    return off;
+}
+
+static int decode_splits(int cache_cap) { return ceil_div(cache_cap > 0 ? cache_cap : 1, 256); }
+
+static Plan plan(const hymba_layer_cfg* c, int B, int T, int mode) {
+    Plan p;
+    const size_t esz = c->dtype == HYMBA_BF16 ? 2 : 4;
+    const Cols k = columns(c);
+    const long long rows = mode == HYMBA_MODE_PREFILL ? (long long)B * (c->n_meta + T) : B;
+    const int di = c->d_inner;
+    p.ldP = round_up(k.n_in, 64);
+    p.rpad = (int)round_up(c->dt_rank, 64);
+    size_t cur = 0;
+    if (mode == HYMBA_MODE_PREFILL) p.rope = take(&cur, (size_t)(c->n_meta + T) * 32 * sizeof(float2));
+    p.P = take(&cur, rows * p.ldP * esz);
+    p.delta = take(&cur, rows * di * sizeof(float));
+    p.O = take(&cur, rows * (size_t)c->n_q_heads * c->v_head_dim * esz);
+    p.ypre = take(&cur, rows * di * esz);
+    p.U = take(&cur, rows * di * esz);
+    p.wdt = take(&cur, (size_t)di * p.rpad * esz);
+    if (mode == HYMBA_MODE_DECODE) {
+        p.n_split = decode_splits(T);
+        p.part = take(&cur, (size_t)B * c->n_q_heads * p.n_split * (c->v_head_dim + 2) * sizeof(float));
+    }
+    p.total = cur;
+    return p;
+}
+
+// ---------------------------------------------------------------------------
+// dispatch: tcgen05 for 16-bit operands, CUDA cores for fp32
+// ---------------------------------------------------------------------------
+template <typename TA, typename TO>
+static int gemm(const Ctx& ctx, const char* name, const TA* A, long long lda, const TA* W, long long ldw,
+                int M, int N, int K, const EpiArgs<TO>& e) {
+#ifdef HYMBA_WITH_TCGEN05
+    if constexpr (sizeof(TA) == 2) {
+        if (((uintptr_t)A & 15) == 0 && ((uintptr_t)W & 15) == 0 && lda % 8 == 0 && ldw % 8 == 0)
+            return launch_gemm_tc<TA, TO>(ctx, name, A, lda, W, ldw, M, N, K, e);
+    }
+#endif
+    return launch_gemm_simt<TA, TO>(ctx, name, A, lda, W, ldw, M, N, K, e);
+}
+
+template <typename I>
+static int attn_prefill(const Ctx& ctx, const I* P, long long ldP, const I* k, const I* v, int kcap,
+                        I* O, int B, int Tp, int H, int G, int dv, int n_meta, int window) {
+#ifdef HYMBA_WITH_TCGEN05_ATTN
+    if constexpr (sizeof(I) == 2) {
+        if (ldP % 8 == 0 && kcap % 8 == 0)
+            return launch_attn_prefill_tc(ctx, P, ldP, k, v, kcap, O, B, Tp, H, G, dv, n_meta, window);
+    }
+#endif
+    return launch_attn_prefill_simt<I>(ctx, P, ldP, k, v, kcap, O, B, Tp, H, G, dv, n_meta, window);
+}
+
+template <typename T>
+static EpiArgs<T> epi_base(int kind, int M, int N) {
+    EpiArgs<T> e;
+    memset(&e, 0, sizeof(e));
+    e.kind = kind;
+    e.M = M;
+    e.N = N;
+    return e;
+}
+
+// T: the layer's I/O and weight type (fp32 or bf16). I: its intermediate type
+// (fp32, or fp16 for bf16 layers: the projection, K/V, attention output and y_pre are
+// held in fp16, which has the same width as bf16 and a finer mantissa).
+template <typename T, typename I>
+static int prefill_impl(const Ctx& ctx, const hymba_layer_cfg* c, const hymba_layer_weights* w,
+                        const T* x, int B, int T_, int flags, T* y, hymba_kv* kv,
+                        hymba_ssm_state* st, char* ws) {
+    const Plan pl = plan(c, B, T_, HYMBA_MODE_PREFILL);
+    const Cols k = columns(c);
+    const int m = c->n_meta, Tp = m + T_, d = c->d_model, di = c->d_inner;
+    const int H = c->n_q_heads, G = c->n_kv_heads, dh = c->head_dim, dv = c->v_head_dim;
+    const long long rows = (long long)B * Tp;
+    const bool has_meta = flags & HYMBA_X_HAS_META;
+    float2* rope = reinterpret_cast<float2*>(ws + pl.rope);
+    I* P = reinterpret_cast<I*>(ws + pl.P);
+    float* delta = reinterpret_cast<float*>(ws + pl.delta);
+    I* O = reinterpret_cast<I*>(ws + pl.O);
+    I* ypre = reinterpret_cast<I*>(ws + pl.ypre);
+    T* U = reinterpret_cast<T*>(ws + pl.U);
+    I* wdt = reinterpret_cast<I*>(ws + pl.wdt);
+    I* k_seq = static_cast<I*>(kv->k_seq);
+    I* v_seq = static_cast<I*>(kv->v_seq);
+    int rc;
+
+    if ((rc = launch_rope_table(ctx, rope, Tp, dh, c->rope_base))) return rc;
+    // 1. fused input projection (+ RoPE, K/V scatter) ------------------------------
+    EpiArgs<I> ep = epi_base<I>(EPI_INPROJ, 0, k.n_in);
+    ep.B = B; ep.Tu = T_; ep.Tp = Tp; ep.n_meta = m;
+    ep.P = P; ep.ldP = pl.ldP;
+    ep.k_out = c->is_kv_producer ? k_seq : nullptr;
+    ep.v_out = c->is_kv_producer ? v_seq : nullptr;
+    ep.kcap = kv->seq_cap;
+    ep.H = H; ep.G = G; ep.dh = dh; ep.dv = dv;
+    ep.rope = rope;
+    const T* W_in = static_cast<const T*>(w->w_in);
+    if (has_meta) {
+        ep.row_mode = ROWS_DIRECT; ep.M = (int)rows;
+        if ((rc = gemm<T, I>(ctx, "gemm_in_proj", x, d, W_in, d, (int)rows, k.n_in, d, ep))) return rc;
+    } else {
+        if (m > 0) {
+            ep.row_mode = ROWS_META; ep.M = m;
+            if ((rc = gemm<T, I>(ctx, "gemm_in_proj_meta", static_cast<const T*>(w->meta), d, W_in, d, m, k.n_in, d, ep))) return rc;
+        }
+        ep.row_mode = ROWS_USER; ep.M = B * T_;
+        if ((rc = gemm<T, I>(ctx, "gemm_in_proj", x, d, W_in, d, B * T_, k.n_in, d, ep))) return rc;
+    }
+    // 2. Delta = softplus(dt_low W_dt^T + b_dt) ------------------------------------
+    if ((rc = launch_pad_copy<T, I>(ctx, static_cast<const T*>(w->w_dt), di, c->dt_rank, wdt, pl.rpad))) return rc;
+    EpiArgs<I> ed = epi_base<I>(EPI_DELTA, (int)rows, di);
+    ed.delta = delta; ed.b_dt = w->b_dt;
+    if ((rc = gemm<I, I>(ctx, "gemm_dt_proj", P + k.dtl, pl.ldP, wdt, pl.rpad, (int)rows, di, c->dt_rank, ed))) return rc;
+    // 3. attention heads ---------------------------------------------------------
+    if ((rc = attn_prefill<I>(ctx, P, pl.ldP, k_seq, v_seq, kv->seq_cap, O, B, Tp, H, G, dv, m, c->window)))
+        return rc;
+    // 4. Mamba heads ---------------------------------------------------------------
+    if ((rc = launch_conv_scan_prefill<I>(ctx, P, pl.ldP, k.x, k.Bc, k.Cc, delta, w->conv_w, w->conv_b,
+                                          w->A_log, w->D, ypre, st ? st->h : nullptr,
+                                          st ? st->conv : nullptr, B, Tp, di)))
+        return rc;
+    // 5. gate, norms, beta, average --------------------------------------------------
+    if ((rc = launch_fuse<I, T>(ctx, O, ypre, P, pl.ldP, k.z, w->norm_attn_w, w->norm_ssm_w, w->beta1,
+                                w->beta2, U, (int)rows, di, c->rms_eps, nullptr)))
+        return rc;
+    // 6. output projection (+ residual) -------------------------------------------------
+    EpiArgs<T> eo = epi_base<T>(EPI_OUT, (int)rows, d);
+    eo.y = y; eo.B = B; eo.Tu = T_; eo.Tp = Tp; eo.n_meta = m;
+    if (flags & HYMBA_ADD_RESIDUAL) {
+        eo.res_mode = has_meta ? 1 : 2;
+        eo.res_x = x;
+        eo.res_meta = static_cast<const T*>(w->meta);
+    }
+    if ((rc = gemm<T, T>(ctx, "gemm_out_proj", U, di, static_cast<const T*>(w->w_out), di, (int)rows, d, di, eo))) return rc;
+    // 7. decode cache of a producer ------------------------------------------------------
+    if (c->is_kv_producer && kv->k_cache) {
+        if ((rc = launch_cache_fill<I>(ctx, k_seq, v_seq, kv->seq_cap, static_cast<I*>(kv->k_cache),
+                                       static_cast<I*>(kv->v_cache), kv->cache_cap, kv->len, B, G, dh, dv, m, Tp)))
+            return rc;
+    }
+    return HYMBA_OK;
+}
+
+template <typename T, typename I>
+static int decode_impl(const Ctx& ctx, const hymba_layer_cfg* c, const hymba_layer_weights* w,
+                       const T* x, int B, int flags, T* y, hymba_kv* kv, hymba_ssm_state* st,
+                       char* ws) {
+    const Plan pl = plan(c, B, kv->cache_cap, HYMBA_MODE_DECODE);
+    const Cols k = columns(c);
+    const int m = c->n_meta, d = c->d_model, di = c->d_inner;
+    const int H = c->n_q_heads, G = c->n_kv_heads, dh = c->head_dim, dv = c->v_head_dim;
+    const int pos_offset = c->is_kv_producer ? 0 : -1;
+    I* P = reinterpret_cast<I*>(ws + pl.P);
+    float* delta = reinterpret_cast<float*>(ws + pl.delta);
+    I* O = reinterpret_cast<I*>(ws + pl.O);
+    I* ypre = reinterpret_cast<I*>(ws + pl.ypre);
+    T* U = reinterpret_cast<T*>(ws + pl.U);
+    I* wdt = reinterpret_cast<I*>(ws + pl.wdt);
+    float* part = reinterpret_cast<float*>(ws + pl.part);
+    I* k_cache = static_cast<I*>(kv->k_cache);
+    I* v_cache = static_cast<I*>(kv->v_cache);
+    int rc;
+    EpiArgs<I> ep = epi_base<I>(EPI_INPROJ, B, k.n_in);
+    ep.row_mode = ROWS_DECODE;
+    ep.B = B; ep.Tu = 1; ep.Tp = 1; ep.n_meta = m;
+    ep.P = P; ep.ldP = pl.ldP;
+    ep.k_out = c->is_kv_producer ? k_cache : nullptr;
+    ep.v_out = c->is_kv_producer ? v_cache : nullptr;
+    ep.kcap = kv->cache_cap;
+    ep.H = H; ep.G = G; ep.dh = dh; ep.dv = dv;
+    ep.pos = kv->len; ep.pos_offset = pos_offset;
+    ep.n_meta_ring = kv->cache_cap - m;
+    ep.rope_base = c->rope_base;
+    if ((rc = gemm<T, I>(ctx, "gemm_in_proj_decode", x, d, static_cast<const T*>(w->w_in), d, B, k.n_in, d, ep))) return rc;
+    if ((rc = launch_pad_copy<T, I>(ctx, static_cast<const T*>(w->w_dt), di, c->dt_rank, wdt, pl.rpad))) return rc;
+    EpiArgs<I> ed = epi_base<I>(EPI_DELTA, B, di);
+    ed.delta = delta; ed.b_dt = w->b_dt;
+    if ((rc = gemm<I, I>(ctx, "gemm_dt_proj_decode", P + k.dtl, pl.ldP, wdt, pl.rpad, B, di, c->dt_rank, ed))) return rc;
+    if ((rc = launch_attn_decode<I>(ctx, P, pl.ldP, k_cache, v_cache, kv->cache_cap, kv->len, pos_offset,
+                                    part, pl.n_split, O, B, H, G, dv, m, c->window)))
+        return rc;
+    if ((rc = launch_ssm_decode<I>(ctx, P, pl.ldP, k.x, k.Bc, k.Cc, delta, w->conv_w, w->conv_b, w->A_log,
+                                   w->D, st->h, st->conv, ypre, B, di)))
+        return rc;
+    if ((rc = launch_fuse<I, T>(ctx, O, ypre, P, pl.ldP, k.z, w->norm_attn_w, w->norm_ssm_w, w->beta1,
+                                w->beta2, U, B, di, c->rms_eps, c->is_kv_producer ? kv->len : nullptr)))
+        return rc;
+    EpiArgs<T> eo = epi_base<T>(EPI_OUT, B, d);
+    eo.y = y;
+    if (flags & HYMBA_ADD_RESIDUAL) { eo.res_mode = 1; eo.res_x = x; }
+    if ((rc = gemm<T, T>(ctx, "gemm_out_proj_decode", U, di, static_cast<const T*>(w->w_out), di, B, d, di, eo))) return rc;
+    return HYMBA_OK;
+}
+
+static int check_weights(const hymba_layer_cfg* c, const hymba_layer_weights* w) {
+    if (!w || !w->w_in || !w->w_dt || !w->b_dt || !w->conv_w || !w->conv_b || !w->A_log || !w->D ||
+        !w->norm_attn_w || !w->norm_ssm_w || !w->beta1 || !w->beta2 || !w->w_out)
+        return HYMBA_ERR_INVALID_ARG;
+    if (c->n_meta > 0 && !w->meta) return HYMBA_ERR_INVALID_ARG;
+    return HYMBA_OK;
+}
+
+static int kv_dtype(const hymba_layer_cfg* c) { return c->dtype == HYMBA_BF16 ? HYMBA_F16 : HYMBA_F32; }
+
+static int check_kv_shape(const hymba_layer_cfg* c, const hymba_kv* kv, int B) {
+    if (kv->batch != B || kv->n_meta != c->n_meta || kv->n_kv_heads != c->n_kv_heads ||
+        kv->head_dim != c->head_dim || kv->v_head_dim != c->v_head_dim || kv->dtype != kv_dtype(c))
+        return HYMBA_ERR_KV_INCOMPATIBLE;
+    return HYMBA_OK;
+}
+
+}  // namespace hymba
+
+using namespace hymba;
+
+extern "C" {
+
+size_t hymba_workspace_bytes(const hymba_layer_cfg* cfg, int B, int T, int mode) {
+    if (check_cfg(cfg) || B <= 0 || T <= 0 || (mode != HYMBA_MODE_PREFILL && mode != HYMBA_MODE_DECODE))
+        return 0;
+    return plan(cfg, B, T, mode).total;
+}
+
+int hymba_workspace_layout(const hymba_layer_cfg* cfg, int B, int T, int mode, int64_t* out, int n) {
+    if (check_cfg(cfg) || B <= 0 || T <= 0 || !out || n < 10) return HYMBA_ERR_INVALID_ARG;
+    const Plan p = plan(cfg, B, T, mode);
+    const int64_t v[10] = {(int64_t)p.total, (int64_t)p.P,    (int64_t)p.ldP, (int64_t)p.delta,
+                           (int64_t)p.O,     (int64_t)p.ypre, (int64_t)p.U,   (int64_t)p.rope,
+                           (int64_t)p.part,  (int64_t)p.n_split};
+    for (int i = 0; i < 10; ++i) out[i] = v[i];
+    return HYMBA_OK;
+}
+
+int hymba_mixer_prefill(const hymba_layer_cfg* cfg, const hymba_layer_weights* w, const void* x,
+                        int B, int T, int flags, void* y, hymba_kv* kv, hymba_ssm_state* st,
+                        void* workspace, size_t ws_bytes, void* stream) {
+    int rc = check_cfg(cfg);
+    if (rc) return rc;
+    if ((rc = check_weights(cfg, w))) return rc;
+    if (!x || !y || !kv || !workspace || B <= 0 || T <= 0 || (flags & ~3)) return HYMBA_ERR_INVALID_ARG;
+    if ((uintptr_t)workspace & 255) return HYMBA_ERR_INVALID_ARG;
+    if (!kv->k_seq || !kv->v_seq) return HYMBA_ERR_INVALID_ARG;
+    if ((rc = check_kv_shape(cfg, kv, B))) return rc;
+    const int Tp = cfg->n_meta + T;
+    if (kv->seq_cap < Tp) return HYMBA_ERR_KV_INCOMPATIBLE;
+    if (cfg->is_kv_producer && kv->k_cache) {
+        if (!kv->v_cache || !kv->len || kv->cache_cap <= cfg->n_meta) return HYMBA_ERR_INVALID_ARG;
+    }
+    if (st && (!st->h || !st->conv)) return HYMBA_ERR_INVALID_ARG;
+    if (y != x) {
+        const size_t xb = (size_t)B * ((flags & HYMBA_X_HAS_META) ? Tp : T) * cfg->d_model;
+        const size_t yb = (size_t)B * Tp * cfg->d_model;
+        const char* xs = static_cast<const char*>(x);
+        const char* ys = static_cast<const char*>(y);
+        const size_t es = cfg->dtype == HYMBA_BF16 ? 2 : 4;
+        if (xs < ys + yb * es && ys < xs + xb * es) return HYMBA_ERR_INVALID_ARG;
+    } else if (!(flags & HYMBA_X_HAS_META)) {
+        return HYMBA_ERR_INVALID_ARG;
+    }
+    if (ws_bytes < plan(cfg, B, T, HYMBA_MODE_PREFILL).total) return HYMBA_ERR_WORKSPACE_TOO_SMALL;
+    Ctx ctx;
+    if ((rc = current_ctx(static_cast<cudaStream_t>(stream), &ctx))) return rc;
+    char* ws = static_cast<char*>(workspace);
+    if (cfg->dtype == HYMBA_BF16)
+        return prefill_impl<bf16, f16>(ctx, cfg, w, static_cast<const bf16*>(x), B, T, flags,
+                                       static_cast<bf16*>(y), kv, st, ws);
+    return prefill_impl<float, float>(ctx, cfg, w, static_cast<const float*>(x), B, T, flags,
+                                      static_cast<float*>(y), kv, st, ws);
+}
+
+int hymba_mixer_decode(const hymba_layer_cfg* cfg, const hymba_layer_weights* w, const void* x_t,
+                       int B, int flags, void* y_t, hymba_kv* kv, hymba_ssm_state* st,
+                       void* workspace, size_t ws_bytes, void* stream) {
+    int rc = check_cfg(cfg);
+    if (rc) return rc;
+    if ((rc = check_weights(cfg, w))) return rc;
+    if (!x_t || !y_t || !kv || !st || !st->h || !st->conv || !workspace || B <= 0 ||
+        (flags & ~HYMBA_ADD_RESIDUAL))
+        return HYMBA_ERR_INVALID_ARG;
+    if ((uintptr_t)workspace & 255) return HYMBA_ERR_INVALID_ARG;
+    if (!kv->k_cache || !kv->v_cache || !kv->len || kv->cache_cap <= cfg->n_meta) return HYMBA_ERR_INVALID_ARG;
+    if ((rc = check_kv_shape(cfg, kv, B))) return rc;
+    if (ws_bytes < plan(cfg, B, kv->cache_cap, HYMBA_MODE_DECODE).total) return HYMBA_ERR_WORKSPACE_TOO_SMALL;
+    Ctx ctx;
+    if ((rc = current_ctx(static_cast<cudaStream_t>(stream), &ctx))) return rc;
+    char* ws = static_cast<char*>(workspace);
+    if (cfg->dtype == HYMBA_BF16)
+        return decode_impl<bf16, f16>(ctx, cfg, w, static_cast<const bf16*>(x_t), B, flags,
+                                      static_cast<bf16*>(y_t), kv, st, ws);
+    return decode_impl<float, float>(ctx, cfg, w, static_cast<const float*>(x_t), B, flags,
+                                     static_cast<float*>(y_t), kv, st, ws);
+}
+
+int hymba_kv_share(const hymba_kv* producer, const hymba_layer_cfg* consumer_cfg, hymba_kv* out) {
+    if (!producer || !consumer_cfg || !out) return HYMBA_ERR_INVALID_ARG;
+    int rc = check_cfg(consumer_cfg);
+    if (rc) return rc;
+    if (consumer_cfg->is_kv_producer) return HYMBA_ERR_INVALID_ARG;
+    if ((rc = check_kv_shape(consumer_cfg, producer, producer->batch))) return rc;
+    if (producer->k_cache) {
+        const int ring = producer->cache_cap - producer->n_meta;
+        if (consumer_cfg->window > 0 && consumer_cfg->window > ring) return HYMBA_ERR_KV_INCOMPATIBLE;
+        if (consumer_cfg->window <= 0 && producer->window > 0 && ring <= producer->window)
+            return HYMBA_ERR_KV_INCOMPATIBLE;
+    }
+    *out = *producer;
+    out->window = consumer_cfg->window;
+    return HYMBA_OK;
+}
+
+uint64_t hymba_kv_bytes(int n_attn_layers, int n_kv_heads, int head_dim, int v_head_dim,
+                        int64_t seq_len, int batch, int dtype_bytes) {
+    if (n_attn_layers < 0 || n_kv_heads < 0 || head_dim < 0 || v_head_dim < 0 || seq_len < 0 ||
+        batch < 0 || dtype_bytes < 0)
+        return 0;
+    return (uint64_t)batch * (uint64_t)seq_len * (uint64_t)n_attn_layers * (uint64_t)n_kv_heads *
+           (uint64_t)(head_dim + v_head_dim) * (uint64_t)dtype_bytes;
+}
+
+uint64_t hymba_ssm_state_bytes(int n_layers, int channels, int d_state, int batch, int dtype_bytes) {
+    if (n_layers < 0 || channels < 0 || d_state < 0 || batch < 0 || dtype_bytes < 0) return 0;
+    return (uint64_t)n_layers * channels * d_state * batch * dtype_bytes;
+}
+
+size_t hymba_cache_bytes(const hymba_layer_cfg* cfg, int B, int max_T) {
+    if (check_cfg(cfg) || B <= 0 || max_T <= 0) return 0;
+    const int esz = cfg->dtype == HYMBA_BF16 ? 2 : 4;
+    const int span = cfg->window > 0 ? cfg->window : max_T;
+    size_t kv = 0;
+    if (cfg->is_kv_producer)
+        kv = hymba_kv_bytes(1, cfg->n_kv_heads, cfg->head_dim, cfg->v_head_dim, cfg->n_meta + span, B, esz);
+    return kv + hymba_ssm_state_bytes(1, cfg->d_inner, cfg->d_state, B, 4) +
+           (size_t)B * cfg->d_inner * cfg->d_conv * 4 + (size_t)B * 4;
+}
+
+int hymba_get_device_status(void* stream) {
+    if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return HYMBA_ERR_CUDA;
+    Ctx ctx;
+    if (current_ctx(static_cast<cudaStream_t>(stream), &ctx)) return HYMBA_ERR_CUDA;
+    int v = 0;
+    if (cudaMemcpy(&v, ctx.status, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return HYMBA_ERR_CUDA;
+    const int zero = 0;
+    if (cudaMemcpy(ctx.status, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess) return HYMBA_ERR_CUDA;
+    return v;
+}
+
+const char* hymba_strerror(int code) {
+    switch (code) {
+        case HYMBA_OK: return "ok";
+        case HYMBA_ERR_INVALID_ARG: return "invalid argument";
+        case HYMBA_ERR_UNSUPPORTED: return "unsupported shape or dtype";
+        case HYMBA_ERR_WORKSPACE_TOO_SMALL: return "workspace too small";
+        case HYMBA_ERR_KV_INCOMPATIBLE: return "KV descriptor incompatible with the layer";
+        case HYMBA_ERR_CUDA: return "CUDA error";
+        case HYMBA_ERR_DEVICE_TIMEOUT: return "bounded device wait timed out";
+        case HYMBA_ERR_DEVICE_RANGE: return "device range check failed";
+        default: return "unknown status";
+    }
+}
+
+int hymba_trace_enable(int on) {
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (on && g_trace.empty()) {
+        g_trace.resize(kTracePool);
+        for (auto& r : g_trace) {
+            if (cudaEventCreate(&r.a) != cudaSuccess || cudaEventCreate(&r.b) != cudaSuccess)
+                return HYMBA_ERR_CUDA;
+            r.name = nullptr;
+        }
+    }
+    g_trace_used.store(0);
+    g_trace_on.store(on ? 1 : 0);
+    return HYMBA_OK;
+}
+
+int hymba_trace_collect(const char** names, float* ms, int max_records) {
+    if (cudaDeviceSynchronize() != cudaSuccess) return HYMBA_ERR_CUDA;
+    const int used = std::min(g_trace_used.load(), (int)g_trace.size());
+    int n = 0;
+    for (int i = 0; i < used && n < max_records; ++i) {
+        float t = 0.f;
+        if (!g_trace[i].name || cudaEventElapsedTime(&t, g_trace[i].a, g_trace[i].b) != cudaSuccess) continue;
+        if (names) names[n] = g_trace[i].name;
+        if (ms) ms[n] = t;
+        ++n;
+    }
+    for (int i = 0; i < used; ++i) g_trace[i].name = nullptr;
+    g_trace_used.store(0);
+    return n;
+}
+
+uint64_t hymba_launch_count(void) { return g_launches.load(); }
+
+}  // extern "C"

@@ -1,0 +1,73 @@
+// Host-side launchers of the library's kernels (one kernel per launcher).
+#pragma once
+#include "common.cuh"
+#include "epilogue.cuh"
+
+namespace hymba {
+
+// C = A B^T on CUDA cores (fp32 accumulate); A [M, K] (row stride lda), Bw [N, K]
+// (row stride ldb); the result goes through epi_run64.
+template <typename TA, typename TO>
+int launch_gemm_simt(const Ctx& ctx, const char* name, const TA* A, long long lda, const TA* Bw, long long ldb,
+                     int M, int N, int K, const EpiArgs<TO>& e);
+
+// C = A B^T on the tcgen05 tensor cores (bf16 or fp16 in, fp32 accumulate in TMEM).
+// Requirements: lda, ldb multiples of 8 elements, A and Bw 16-byte aligned.
+template <typename TA, typename TO>
+int launch_gemm_tc(const Ctx& ctx, const char* name, const TA* A, long long lda, const TA* Bw, long long ldb,
+                   int M, int N, int K, const EpiArgs<TO>& e);
+
+// Causal GQA attention over the meta prefix + window, CUDA cores.
+template <typename T>
+int launch_attn_prefill_simt(const Ctx& ctx, const T* P, long long ldP, const T* k_seq,
+                             const T* v_seq, int kcap, T* O, int B, int Tp, int H, int G,
+                             int dv, int n_meta, int window);
+
+// Causal GQA attention over the meta prefix + window, tcgen05 tensor cores (bf16).
+int launch_attn_prefill_tc(const Ctx& ctx, const f16* P, long long ldP, const f16* k_seq,
+                           const f16* v_seq, int kcap, f16* O, int B, int Tp, int H, int G,
+                           int dv, int n_meta, int window);
+
+// Depthwise causal conv + SiLU + selective scan over the T' rows of every sequence.
+template <typename T>
+int launch_conv_scan_prefill(const Ctx& ctx, const T* P, long long ldP, int col_x, int col_B,
+                             int col_C, const float* delta, const float* conv_w,
+                             const float* conv_b, const float* A_log, const float* D, T* ypre,
+                             float* h_out, float* conv_out, int B, int Tp, int di);
+
+// RMSNorm of both branches, SiLU(z) gate, beta scaling and average; one row per block.
+template <typename I, typename T>
+int launch_fuse(const Ctx& ctx, const I* O, const I* ypre, const I* P, long long ldP, int col_z,
+                const float* g_attn, const float* g_ssm, const float* beta1, const float* beta2,
+                T* U, int rows, int di, float eps, int* len_inc);
+
+// cos/sin table of RoPE for positions 0..Tp-1 (angles in double precision).
+int launch_rope_table(const Ctx& ctx, float2* tab, int Tp, int dh, float base);
+
+// Copy a [rows, cols] matrix into a zero-padded [rows, ld_dst] one of type TD.
+template <typename TS, typename TD>
+int launch_pad_copy(const Ctx& ctx, const TS* src, int rows, int cols, TD* dst, int ld_dst);
+
+// Fill the decode cache of a producer from its prefill sequence K/V and set len = Tp.
+template <typename T>
+int launch_cache_fill(const Ctx& ctx, const T* k_seq, const T* v_seq, int seq_cap, T* k_cache,
+                      T* v_cache, int cache_cap, int* len, int B, int G, int dh, int dv,
+                      int n_meta, int Tp);
+
+// Decode attention: one query per (sequence, head) over the cache; split over keys,
+// partial results in `part` [B, H, n_split, dv + 2] fp32, then combined into O.
+template <typename T>
+int launch_attn_decode(const Ctx& ctx, const T* P, long long ldP, const T* k_cache,
+                       const T* v_cache, int cache_cap, const int* len, int pos_offset,
+                       float* part, int n_split, T* O, int B, int H, int G, int dv, int n_meta,
+                       int window);
+
+// One SSM decode step per (sequence, channel): conv-state shift, conv, SiLU, scan
+// step on h in place, y_pre = C.h + D xc.
+template <typename T>
+int launch_ssm_decode(const Ctx& ctx, const T* P, long long ldP, int col_x, int col_B,
+                      int col_C, const float* delta, const float* conv_w, const float* conv_b,
+                      const float* A_log, const float* D, float* h, float* conv, T* ypre, int B,
+                      int di);
+
+}  // namespace hymba

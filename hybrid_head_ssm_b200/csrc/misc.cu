@@ -1,0 +1,79 @@
+// Small data-movement kernels around the mixer: the RoPE angle table, zero-padded
+// weight copies for TMA-aligned strides, and the decode-cache fill after a prefill.
+#include "kernels.h"
+
+namespace hymba {
+
+namespace {
+
+__global__ void rope_table_kernel(float2* tab, int Tp, int half, int dh, float base) {
+    const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    if (idx >= (long long)Tp * half) return;
+    const int p = (int)(idx / half), i = (int)(idx % half);
+    tab[idx] = rope_cs_at(p, i, dh, base);
+}
+
+template <typename TS, typename TD>
+__global__ void pad_copy_kernel(const TS* src, int rows, int cols, TD* dst, int ld_dst) {
+    const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    if (idx >= (long long)rows * ld_dst) return;
+    const int r = (int)(idx / ld_dst), c = (int)(idx % ld_dst);
+    dst[idx] = from_f<TD>(c < cols ? to_f(src[(long long)r * cols + c]) : 0.f);
+}
+
+// Slot of position p: meta positions keep their slot, the others wrap in a ring of
+// cache_cap - n_meta slots. Rows copied: meta positions and the newest ring-full.
+template <typename T>
+__global__ void cache_fill_kernel(const T* k_seq, const T* v_seq, int seq_cap, T* k_cache,
+                                  T* v_cache, int cache_cap, int* len, int G, int dh, int dv,
+                                  int n_meta, int Tp) {
+    const int ring = cache_cap - n_meta;
+    const int first_kept = max(n_meta, Tp - ring);
+    const int n_rows = min(n_meta, Tp) + max(0, Tp - first_kept);
+    const int b = blockIdx.z, g = blockIdx.y;
+    for (int ri = blockIdx.x; ri < n_rows; ri += gridDim.x) {
+        const int meta_rows = min(n_meta, Tp);
+        const int p = ri < meta_rows ? ri : first_kept + (ri - meta_rows);
+        const int slot = p < n_meta ? p : n_meta + (p - n_meta) % ring;
+        const long long src = ((long long)b * G + g) * seq_cap + p;
+        const long long dst = ((long long)b * G + g) * cache_cap + slot;
+        for (int e = threadIdx.x; e < dh; e += blockDim.x) k_cache[dst * dh + e] = k_seq[src * dh + e];
+        for (int e = threadIdx.x; e < dv; e += blockDim.x) v_cache[dst * dv + e] = v_seq[src * dv + e];
+    }
+    if (blockIdx.x == 0 && g == 0 && threadIdx.x == 0) len[b] = Tp;
+}
+
+}  // namespace
+
+int launch_rope_table(const Ctx& ctx, float2* tab, int Tp, int dh, float base) {
+    const long long n = (long long)Tp * (dh / 2);
+    HYMBA_LAUNCH(ctx, "rope_table", rope_table_kernel, ceil_div(n, 256), 256, 0, tab, Tp, dh / 2, dh, base);
+    return HYMBA_OK;
+}
+
+template <typename TS, typename TD>
+int launch_pad_copy(const Ctx& ctx, const TS* src, int rows, int cols, TD* dst, int ld_dst) {
+    const long long n = (long long)rows * ld_dst;
+    auto kern = pad_copy_kernel<TS, TD>;
+    HYMBA_LAUNCH(ctx, "pad_copy", kern, ceil_div(n, 256), 256, 0, src, rows, cols, dst, ld_dst);
+    return HYMBA_OK;
+}
+
+template <typename T>
+int launch_cache_fill(const Ctx& ctx, const T* k_seq, const T* v_seq, int seq_cap, T* k_cache,
+                      T* v_cache, int cache_cap, int* len, int B, int G, int dh, int dv, int n_meta,
+                      int Tp) {
+    dim3 grid(256, G, B);
+    HYMBA_LAUNCH(ctx, "cache_fill", cache_fill_kernel<T>, grid, 128, 0, k_seq, v_seq, seq_cap,
+                 k_cache, v_cache, cache_cap, len, G, dh, dv, n_meta, Tp);
+    return HYMBA_OK;
+}
+
+template int launch_pad_copy<float, float>(const Ctx&, const float*, int, int, float*, int);
+template int launch_pad_copy<bf16, f16>(const Ctx&, const bf16*, int, int, f16*, int);
+template int launch_cache_fill<float>(const Ctx&, const float*, const float*, int, float*, float*,
+                                      int, int*, int, int, int, int, int, int);
+template int launch_cache_fill<f16>(const Ctx&, const f16*, const f16*, int, f16*, f16*, int,
+                                    int*, int, int, int, int, int, int);
+
+}  // namespace hymba

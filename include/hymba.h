@@ -1,0 +1,252 @@
+/*
+ * hymba.h - C ABI of libhymba.so, the B200 (sm_100a) Hymba parallel hybrid-head mixer.
+ *
+ * What the library computes (one mixer layer; sources are cited by page title and
+ * section):
+ *   "Hymba Guide: NVIDIA Hybrid-Head Mamba & Attention SLM", section "Parallel
+ *   Hybrid-Head Layer Formulation": attention heads and Mamba (SSM) heads run in
+ *   parallel on the same input and one output projection W_o mixes them; section
+ *   "Learnable Meta-Tokens": n_meta learned rows are prepended to every sequence;
+ *   section "Cross-Layer KV Cache Sharing": a secondary layer reuses the K and V of
+ *   the primary layer with no new buffer.
+ *   "Jamba: Hybrid SSM-Transformer", How It Actually Works section 1: the selective
+ *   scan h_t = exp(Delta_t A) h_{t-1} + (Delta_t B_t) x_t, y_t = C_t h_t, and
+ *   softmax(Q K^T / sqrt(d_k)) V attention with GQA.
+ *   51cto "Hymba-1.5B" article, section 2: GQA + RoPE, sliding-window attention with
+ *   a few global layers, KV shared by pairs of layers.
+ *
+ * Per layer and sequence, with X^ = [meta; x] (T' = n_meta + T rows):
+ *   [Q K V x z dt_low B C] = X^ W_in^T                 one fused projection
+ *   Q, K <- RoPE (rotate-half, base rope_base), position of row i is i
+ *   O     = GQA softmax attention, key j visible to query i iff j <= i and
+ *           (j < n_meta or i - j < window); window <= 0 means global
+ *   xc    = SiLU(depthwise causal conv_{d_conv}(x) + conv_b)
+ *   Delta = softplus(dt_low W_dt^T + b_dt),  A = -exp(A_log)
+ *   h_t   = exp(Delta_t A) h_{t-1} + Delta_t B_t xc_t  (fp32 state)
+ *   Y     = (C_t . h_t + D xc_t) * SiLU(z_t)
+ *   U     = (beta1 * RMSNorm(O) + beta2 * RMSNorm(Y)) / 2
+ *   y     = U W_out^T (+ X^ when HYMBA_ADD_RESIDUAL)
+ *
+ * Conventions for every entry point:
+ *   - Every pointer marked "device" is device memory owned by the caller. The
+ *     library never allocates, frees or synchronises on the compute entry points;
+ *     all work is queued on `stream` (a cudaStream_t, NULL = legacy default stream).
+ *   - Tensors are dense row-major with the shapes given; "dtype" is the layer's
+ *     activation and weight type (HYMBA_F32 or HYMBA_BF16). Small per-channel
+ *     parameters are always fp32. Inside a bf16 layer, the projection, K/V,
+ *     attention output and pre-gate SSM output are held in fp16 (2 bytes like bf16,
+ *     8x finer rounding); accumulation is fp32 everywhere.
+ *   - Return value: HYMBA_OK (0) or a negative HYMBA_ERR_* code. Argument checks
+ *     happen on the host before any launch; a failed check queues no work. Errors
+ *     found on the device (bounded waits that time out, out-of-range positions)
+ *     are recorded in a per-device status word read by hymba_get_device_status().
+ *   - The functions keep no per-call global state and are safe to call from
+ *     several host threads on different streams (except the opt-in tracing).
+ */
+#ifndef HYMBA_H
+#define HYMBA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* status codes */
+#define HYMBA_OK                       0
+#define HYMBA_ERR_INVALID_ARG        (-1)  /* null pointer, non-positive size, bad flag */
+#define HYMBA_ERR_UNSUPPORTED        (-2)  /* shape or dtype outside what the kernels handle */
+#define HYMBA_ERR_WORKSPACE_TOO_SMALL (-3) /* ws_bytes < hymba_workspace_bytes(...) */
+#define HYMBA_ERR_KV_INCOMPATIBLE    (-4)  /* KV descriptor does not fit the layer */
+#define HYMBA_ERR_CUDA               (-5)  /* a CUDA call or launch failed */
+#define HYMBA_ERR_DEVICE_TIMEOUT     (-6)  /* a bounded device wait ran out (status word) */
+#define HYMBA_ERR_DEVICE_RANGE       (-7)  /* a device-side range check failed (status word) */
+
+/* dtypes: a layer is HYMBA_F32 or HYMBA_BF16; the K/V buffers of a bf16 layer hold
+ * HYMBA_F16 (same width as bf16, finer mantissa; see hymba_kv) */
+#define HYMBA_F32  0
+#define HYMBA_BF16 1
+#define HYMBA_F16  2
+
+/* flags of the mixer calls */
+#define HYMBA_X_HAS_META    1  /* x already holds the n_meta rows (a later layer of a stack) */
+#define HYMBA_ADD_RESIDUAL  2  /* y = X^ + mixer(X^) */
+
+/* workspace modes */
+#define HYMBA_MODE_PREFILL 0
+#define HYMBA_MODE_DECODE  1
+
+/* Shape and numerics of one mixer layer. The V head dim must equal
+ * d_inner / n_q_heads so that the two branches can be averaged (the concat
+ * formula of the Hymba Guide has no such constraint; averaging does).
+ * Supported: head_dim == 64; v_head_dim % 64 == 0; n_q_heads % n_kv_heads == 0;
+ * d_model, d_inner % 64 == 0; d_state == 16; d_conv == 4. */
+typedef struct hymba_layer_cfg {
+    int32_t d_model;
+    int32_t n_q_heads;
+    int32_t n_kv_heads;
+    int32_t head_dim;        /* Q/K head dim (64) */
+    int32_t v_head_dim;      /* = d_inner / n_q_heads */
+    int32_t d_inner;
+    int32_t d_state;
+    int32_t d_conv;
+    int32_t dt_rank;
+    int32_t n_meta;
+    int32_t window;          /* <= 0: global attention */
+    int32_t is_kv_producer;  /* 1: projects its own K, V; 0: reads a producer's */
+    int32_t dtype;           /* HYMBA_F32 or HYMBA_BF16 */
+    float   rope_base;
+    float   rms_eps;
+} hymba_layer_cfg;
+
+/* Weights of one layer (device pointers, caller-owned, read only). Big matrices
+ * use the [out, in] convention. n_in = H*dh + (producer ? G*(dh+dv) : 0)
+ * + 2*d_inner + dt_rank + 2*d_state, rows in the order Q | K | V | x | z |
+ * dt_low | B | C. */
+typedef struct hymba_layer_weights {
+    const void*  w_in;        /* [n_in, d_model]        dtype */
+    const void*  w_dt;        /* [d_inner, dt_rank]     dtype */
+    const float* b_dt;        /* [d_inner] */
+    const float* conv_w;      /* [d_inner, d_conv]      tap d_conv-1 meets the newest input */
+    const float* conv_b;      /* [d_inner] */
+    const float* A_log;       /* [d_inner, d_state]     A = -exp(A_log) */
+    const float* D;           /* [d_inner] */
+    const float* norm_attn_w; /* [n_q_heads*v_head_dim] RMSNorm gain of the attention branch */
+    const float* norm_ssm_w;  /* [d_inner]              RMSNorm gain of the SSM branch */
+    const float* beta1;       /* [n_q_heads*v_head_dim] */
+    const float* beta2;       /* [d_inner] */
+    const void*  w_out;       /* [d_model, d_inner]     dtype */
+    const void*  meta;        /* [n_meta, d_model]      dtype */
+} hymba_layer_weights;
+
+/* K/V of one producer layer and of the consumers that share it ("Hymba Guide",
+ * Cross-Layer KV Cache Sharing). Two parts, both caller-owned device memory:
+ *   - prefill sequence K/V: k_seq [batch, n_kv_heads, seq_cap, head_dim] and
+ *     v_seq [batch, n_kv_heads, seq_cap, v_head_dim]; position i of a sequence in
+ *     row i. A producer's prefill writes them (K after RoPE), a consumer's reads.
+ *     Required by prefill (seq_cap >= T'); unused by decode.
+ *   - decode cache: k_cache [batch, n_kv_heads, cache_cap, head_dim],
+ *     v_cache [batch, n_kv_heads, cache_cap, v_head_dim], len [batch] int32.
+ *     Slots 0..n_meta-1 hold the meta positions; position p >= n_meta lives in slot
+ *     n_meta + (p - n_meta) mod (cache_cap - n_meta), a ring. len[b] = positions
+ *     held so far (meta included). NULL k_cache: no decode cache. A producer's
+ *     prefill fills it (meta + the newest cache_cap - n_meta positions) and sets
+ *     len; a producer's decode appends one position and increments len; a
+ *     consumer's decode reads positions 0..len-1. */
+typedef struct hymba_kv {
+    void*    k_seq;
+    void*    v_seq;
+    int32_t  seq_cap;
+    void*    k_cache;
+    void*    v_cache;
+    int32_t* len;
+    int32_t  cache_cap;
+    int32_t  batch;
+    int32_t  n_meta;
+    int32_t  n_kv_heads;
+    int32_t  head_dim;
+    int32_t  v_head_dim;
+    int32_t  dtype;      /* HYMBA_F32 for fp32 layers, HYMBA_F16 for bf16 layers */
+    int32_t  window;     /* attention span of the producer (<= 0: global) */
+} hymba_kv;
+
+/* Recurrent state of one layer's Mamba heads (device, caller-owned):
+ * h [batch, d_inner, d_state] fp32; conv [batch, d_inner, d_conv] fp32 holding
+ * the last d_conv pre-conv inputs, oldest first. */
+typedef struct hymba_ssm_state {
+    float* h;
+    float* conv;
+} hymba_ssm_state;
+
+/* Prefill of B sequences of T user tokens through one layer.
+ *   x: device [B, T, d_model] dtype, or [B, n_meta+T, d_model] with HYMBA_X_HAS_META.
+ *   y: device [B, n_meta+T, d_model] dtype (meta rows included, so stacks compose).
+ *      y may equal x when HYMBA_X_HAS_META is set (in-place residual stacks);
+ *      otherwise y and x must not overlap.
+ *   kv: producer: k_seq/v_seq written (and the decode cache filled if k_cache);
+ *       consumer: k_seq/v_seq read (fill them with the producer's prefill first).
+ *   st: NULL, or the state to write: h and conv after the last row.
+ *   workspace: device scratch of at least hymba_workspace_bytes(cfg, B, T,
+ *       HYMBA_MODE_PREFILL) bytes, 256-byte aligned; contents are undefined after. */
+int hymba_mixer_prefill(const hymba_layer_cfg* cfg, const hymba_layer_weights* w,
+                        const void* x, int B, int T, int flags, void* y,
+                        hymba_kv* kv, hymba_ssm_state* st,
+                        void* workspace, size_t ws_bytes, void* stream);
+
+/* One decode step: one new token per sequence, all B sequences at the same position
+ * len[b] (producer) or len[b]-1 (consumer).
+ *   x_t: device [B, d_model]; y_t: device [B, d_model] (may equal x_t).
+ *   kv must hold a decode cache (k_cache, len); st is updated in place. A cache
+ *   whose ring is too short for the layer's span makes the step record
+ *   HYMBA_ERR_DEVICE_RANGE in the status word and write zeros for that row. */
+int hymba_mixer_decode(const hymba_layer_cfg* cfg, const hymba_layer_weights* w,
+                       const void* x_t, int B, int flags, void* y_t,
+                       hymba_kv* kv, hymba_ssm_state* st,
+                       void* workspace, size_t ws_bytes, void* stream);
+
+/* Cross-layer KV sharing: fill *consumer_out with the producer's buffers (pointer
+ * copies, no device work, no new memory). Fails with HYMBA_ERR_KV_INCOMPATIBLE
+ * when the consumer's KV shape differs, or when its attention span does not fit
+ * the producer's ring (an SWA consumer with window > cache_cap - n_meta, or a
+ * global consumer on a ring no longer than the producer's window). */
+int hymba_kv_share(const hymba_kv* producer, const hymba_layer_cfg* consumer_cfg,
+                   hymba_kv* consumer_out);
+
+/* Workspace bytes for one call (0 if the configuration is invalid). For
+ * HYMBA_MODE_DECODE, T is the cache_cap of the KV cache the step reads. */
+size_t hymba_workspace_bytes(const hymba_layer_cfg* cfg, int B, int T, int mode);
+
+/* Decode-state bytes of one layer for B sequences of up to max_T positions (meta
+ * included): KV slots (producer only; n_meta + window, or n_meta + max_T when
+ * global) * (head_dim + v_head_dim) * element size (2 for bf16 layers, whose K/V are
+ * fp16; 4 for fp32) * n_kv_heads * B, plus the fp32 SSM state, the fp32 conv state
+ * and the int32 lengths. */
+size_t hymba_cache_bytes(const hymba_layer_cfg* cfg, int B, int max_T);
+
+/* KV bytes over several attention layers ("Jamba: Hybrid SSM-Transformer",
+ * section 2 and Worked Example; "Lecture 04", section 8 kv_cache_gb):
+ * batch * seq_len * n_attn_layers * n_kv_heads * (head_dim + v_head_dim) * dtype_bytes. */
+uint64_t hymba_kv_bytes(int n_attn_layers, int n_kv_heads, int head_dim, int v_head_dim,
+                        int64_t seq_len, int batch, int dtype_bytes);
+
+/* SSM state bytes ("Lecture 04", section 8 ssm_state_gb):
+ * n_layers * channels * d_state * batch * dtype_bytes. */
+uint64_t hymba_ssm_state_bytes(int n_layers, int channels, int d_state, int batch,
+                               int dtype_bytes);
+
+/* Synchronises `stream`, then returns and clears the status word of the current
+ * device: HYMBA_OK, HYMBA_ERR_DEVICE_TIMEOUT or HYMBA_ERR_DEVICE_RANGE; or
+ * HYMBA_ERR_CUDA if the synchronisation itself failed. */
+int hymba_get_device_status(void* stream);
+
+/* Layout of the workspace of one call, for callers that inspect the stage outputs
+ * after a prefill (tests do): out[0] total bytes, out[1] byte offset of the
+ * projection P [rows, ld_p] dtype (columns Q | (K V, unused) | x | z | dt_low | B | C),
+ * out[2] ld_p in elements, out[3] offset of Delta [rows, d_inner] fp32, out[4] of the
+ * attention output O [rows, n_q_heads*v_head_dim] dtype, out[5] of y_pre = C.h + D xc
+ * [rows, d_inner] dtype (before the SiLU(z) gate), out[6] of the fused U [rows,
+ * d_inner] dtype, out[7] of the RoPE table, out[8] of the decode split partials,
+ * out[9] the decode split count. rows = B * (n_meta + T) for prefill, B for decode
+ * (where T is the cache_cap of the KV cache). Requires n >= 10. */
+int hymba_workspace_layout(const hymba_layer_cfg* cfg, int B, int T, int mode, int64_t* out, int n);
+
+/* Static description of a status code. */
+const char* hymba_strerror(int code);
+
+/* Opt-in per-kernel timing. While enabled, every kernel the library queues is
+ * bracketed by CUDA events on its own stream. hymba_trace_collect synchronises
+ * the device, writes up to max_records (name, milliseconds) pairs in launch order
+ * (names are static strings) and returns how many it wrote; records beyond the
+ * internal pool (8192) are dropped. Not thread-safe against concurrent
+ * enable/collect; calls in between may come from any thread. */
+int hymba_trace_enable(int on);
+int hymba_trace_collect(const char** names, float* ms, int max_records);
+
+/* Number of kernels the library has queued since load (all entry points). */
+uint64_t hymba_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* HYMBA_H */

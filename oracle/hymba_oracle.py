@@ -367,11 +367,12 @@ def ssm_state_bytes(n_layers: int, channels: int, d_state: int, batch: int, dtyp
 
 
 def layer_cache_bytes(cfg, batch: int, max_T: int) -> int:
-    """Decode cache of one producer layer: KV slots (meta + ring or full history),
-    fp32 SSM state, conv state (activation dtype) and the int32 lengths."""
+    """Decode cache of one producer layer: KV slots (meta + ring or full history) of
+    2-byte elements for a bf16 layer (4 for fp32), fp32 SSM state, fp32 conv state
+    and the int32 lengths."""
     esz = 2 if cfg.dtype == 1 else 4
     span = cfg.window if cfg.window > 0 else max_T
     cap = cfg.n_meta + span
     kv = batch * cfg.n_kv_heads * cap * (cfg.head_dim + cfg.v_head_dim) * esz if cfg.is_kv_producer else 0
     return (kv + ssm_state_bytes(1, cfg.d_inner, cfg.d_state, batch, 4)
-            + batch * cfg.d_inner * cfg.d_conv * esz + batch * 4)
+            + batch * cfg.d_inner * cfg.d_conv * 4 + batch * 4)

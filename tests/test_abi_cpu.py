@@ -1,0 +1,140 @@
+"""Host-side checks of the C ABI that need no GPU: the library loads, exports every
+function include/hymba.h declares, its host-only helpers agree with the oracle and
+the pages' printed cache sizes, and argument errors are caught before any launch."""
+import ctypes
+import json
+import os
+import re
+
+import pytest
+
+import oracle
+import synth
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def hy():
+    import hybrid_head_ssm_b200 as hy
+    return hy
+
+
+def _declared():
+    names = []
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            src = open(os.path.join(ROOT, "include", fn)).read()
+            src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+            names += re.findall(r"\b(hymba_\w+)\s*\(", src)
+    return sorted(set(names))
+
+
+def test_library_exports_every_declared_function(hy):
+    declared = _declared()
+    assert "hymba_mixer_prefill" in declared and "hymba_kv_share" in declared
+    lib = ctypes.CDLL(hy.LIB_PATH)
+    for n in declared:
+        assert hasattr(lib, n), n
+        assert n in hy.EXPORTS, n
+
+
+def test_kv_bytes_matches_pages(hy):
+    gold = json.load(open(os.path.join(ROOT, "tests", "golden", "cache_sizes.json")))
+    ex = gold["jamba_worked_example"]
+    assert hy.hymba_kv_bytes(32, 8, 128, 128, 64000, 4, 2) == ex["dense_32_layers_bytes"]
+    assert hy.hymba_kv_bytes(4, 8, 128, 128, 64000, 4, 2) == ex["hybrid_4_layers_bytes"]
+    assert hy.hymba_kv_bytes(1, 8, 128, 128, 1, 1, 2) == ex["bytes_per_token_layer"]
+    assert hy.hymba_ssm_state_bytes(64, 64 * 64, 128, 1, 2) == oracle.ssm_state_bytes(64, 4096, 128, 1, 2)
+    assert hy.hymba_kv_bytes(80, 8, 128, 128, 128000, 1, 2) == oracle.kv_cache_bytes(80, 8, 128, 128000, 1, 2)
+
+
+@pytest.mark.parametrize("window,producer", [(1024, 1), (0, 1), (1024, 0)])
+def test_cache_bytes_matches_oracle(hy, window, producer):
+    cfg = synth.hymba15_layer_cfg(window, producer)
+    c = hy.cfg_struct(cfg)
+    for B, T in [(1, 100), (64, 4224)]:
+        assert hy.hymba_cache_bytes(ctypes.byref(c), B, T) == oracle.layer_cache_bytes(cfg, B, T)
+
+
+def test_workspace_layout_is_consistent(hy):
+    cfg = synth.hymba15_layer_cfg(1024)
+    c = hy.cfg_struct(cfg)
+    lay = hy.workspace_layout(c, 1, 2048, hy.HYMBA_MODE_PREFILL)
+    assert lay["total"] == hy.hymba_workspace_bytes(ctypes.byref(c), 1, 2048, hy.HYMBA_MODE_PREFILL)
+    assert lay["ldP"] % 64 == 0 and lay["ldP"] >= cfg.n_in
+    offs = sorted(lay[k] for k in ("P", "delta", "O", "ypre", "U"))
+    assert all(o % 256 == 0 for o in offs)
+    assert len(set(offs)) == 5
+    dec = hy.workspace_layout(c, 64, 1152, hy.HYMBA_MODE_DECODE)
+    assert dec["n_split"] >= 1 and dec["part"] > 0
+
+
+def test_invalid_configs_rejected(hy):
+    base = synth.tiny_layer_cfg()
+    for bad in (base.with_(head_dim=32), base.with_(d_state=8), base.with_(n_kv_heads=3),
+                base.with_(v_head_dim=64), base.with_(dtype=7), base.with_(d_model=0)):
+        c = hy.cfg_struct(bad)
+        assert hy.hymba_workspace_bytes(ctypes.byref(c), 1, 10, 0) == 0
+        assert hy.hymba_cache_bytes(ctypes.byref(c), 1, 10) == 0
+
+
+def test_prefill_argument_errors_before_any_launch(hy):
+    cfg = synth.tiny_layer_cfg()
+    c = hy.cfg_struct(cfg)
+    w = hy.hymba_layer_weights()
+    kv = hy.hymba_kv()
+    rc = hy.hymba_mixer_prefill(ctypes.byref(c), ctypes.byref(w), None, 1, 10, 0, None, ctypes.byref(kv),
+                                None, None, 0, None)
+    assert rc == hy.HYMBA_ERR_INVALID_ARG
+    bad = hy.cfg_struct(cfg.with_(head_dim=48))
+    rc = hy.hymba_mixer_prefill(ctypes.byref(bad), ctypes.byref(w), None, 1, 10, 0, None, ctypes.byref(kv),
+                                None, None, 0, None)
+    assert rc == hy.HYMBA_ERR_UNSUPPORTED
+    # all pointers "present" (fake host addresses, never dereferenced) but workspace too small
+    fake = 1 << 20
+    wf = hy.hymba_layer_weights(*([fake] * 13))
+    kvf = hy.kv_struct(cfg, 1)
+    kvf.k_seq = kvf.v_seq = fake
+    kvf.seq_cap = cfg.n_meta + 10
+    rc = hy.hymba_mixer_prefill(ctypes.byref(c), ctypes.byref(wf), 1 << 24, 1, 10, 0, 1 << 28, ctypes.byref(kvf),
+                                None, 1 << 30, 256, None)
+    assert rc == hy.HYMBA_ERR_WORKSPACE_TOO_SMALL
+    kvf.seq_cap = 5
+    rc = hy.hymba_mixer_prefill(ctypes.byref(c), ctypes.byref(wf), 1 << 24, 1, 10, 0, 1 << 28, ctypes.byref(kvf),
+                                None, 1 << 30, 1 << 40, None)
+    assert rc == hy.HYMBA_ERR_KV_INCOMPATIBLE
+    # x and y overlap without the in-place form
+    kvf.seq_cap = cfg.n_meta + 10
+    rc = hy.hymba_mixer_prefill(ctypes.byref(c), ctypes.byref(wf), 1 << 24, 1, 10, 0, (1 << 24) + 64,
+                                ctypes.byref(kvf), None, 1 << 30, 1 << 40, None)
+    assert rc == hy.HYMBA_ERR_INVALID_ARG
+
+
+def test_kv_share_rules(hy):
+    prod_cfg = synth.tiny_layer_cfg().with_(window=8)
+    kv = hy.kv_struct(prod_cfg, 2)
+    kv.k_seq = kv.v_seq = 4096
+    kv.seq_cap = 100
+    out = hy.hymba_kv()
+    # consumer with the same span: fine, pointers copied
+    cons = hy.cfg_struct(prod_cfg.with_(is_kv_producer=0))
+    assert hy.hymba_kv_share(ctypes.byref(kv), ctypes.byref(cons), ctypes.byref(out)) == 0
+    assert out.k_seq == kv.k_seq and out.seq_cap == 100
+    # a producer config cannot be a consumer
+    assert hy.hymba_kv_share(ctypes.byref(kv), ctypes.byref(hy.cfg_struct(prod_cfg)), ctypes.byref(out)) == hy.HYMBA_ERR_INVALID_ARG
+    # decode ring of 8 slots: a window-16 consumer does not fit, a global one neither
+    kv.k_cache = kv.v_cache = kv.len = 8192
+    kv.cache_cap = prod_cfg.n_meta + 8
+    for w in (16, 0):
+        c2 = hy.cfg_struct(prod_cfg.with_(is_kv_producer=0, window=w))
+        assert hy.hymba_kv_share(ctypes.byref(kv), ctypes.byref(c2), ctypes.byref(out)) == hy.HYMBA_ERR_KV_INCOMPATIBLE
+    # a different KV head count is incompatible
+    c3 = hy.cfg_struct(prod_cfg.with_(is_kv_producer=0, n_kv_heads=4))
+    assert hy.hymba_kv_share(ctypes.byref(kv), ctypes.byref(c3), ctypes.byref(out)) == hy.HYMBA_ERR_KV_INCOMPATIBLE
+
+
+def test_strerror_covers_codes(hy):
+    for code in range(0, -8, -1):
+        assert hy.hymba_strerror(code).decode() != "unknown status"
+    assert hy.hymba_strerror(-99).decode() == "unknown status"

@@ -1,0 +1,197 @@
+"""GPU parity of hymba_mixer_prefill against the fp64 CPU oracle, element by element,
+through the C ABI. Stage outputs left in the workspace (projection, Delta, attention
+output, y_pre, fused U) are compared too, so a failure names the stage."""
+import ctypes
+
+import numpy as np
+import pytest
+
+import oracle
+import synth
+from gpu_helpers import assert_close, errors, to_np, torch_cuda
+
+pytestmark = pytest.mark.gpu
+
+
+def _run_prefill(cfg, w, x, *, kv_from=None, cache_cap=0, flags=0, state=True):
+    torch = torch_cuda()
+    import hybrid_head_ssm_b200 as hy
+    from hybrid_head_ssm_b200 import runtime as rt
+    B, T = x.shape[0], (x.shape[1] - cfg.n_meta if flags & hy.HYMBA_X_HAS_META else x.shape[1])
+    Tp = cfg.n_meta + T
+    layer = rt.DeviceLayer(cfg, w)
+    xd = rt.to_device(x, cfg)
+    yd = torch.empty((B, Tp, cfg.d_model), dtype=rt.act_dtype(cfg), device="cuda")
+    if kv_from is None:
+        kv = rt.KV(cfg, B, seq_cap=Tp, cache_cap=cache_cap)
+        kvs = kv.s
+    else:
+        kv = kv_from
+        kvs = hy.hymba_kv()
+        hy.check(hy.hymba_kv_share(ctypes.byref(kv_from.s), ctypes.byref(layer.c), ctypes.byref(kvs)))
+    st = rt.State(cfg, B) if state else None
+    ws = rt.workspace(cfg, B, T, hy.HYMBA_MODE_PREFILL)
+    ws.fill_(0xFF)  # garbage: every stage must write what it later reads
+    rt.prefill(layer, xd, T, kv, yd, ws, st, flags, kv_struct_override=kvs)
+    torch.cuda.synchronize()
+    assert hy.hymba_get_device_status(None) == 0
+    lay = hy.workspace_layout(layer.c, B, T, hy.HYMBA_MODE_PREFILL)
+    return dict(y=yd, kv=kv, st=st, ws=ws, lay=lay, layer=layer)
+
+
+def _ws_view(ws, off, shape, dtype):
+    import torch
+    n = int(np.prod(shape))
+    esz = torch.tensor([], dtype=dtype).element_size()
+    return ws[off:off + n * esz].view(dtype).view(*shape)
+
+
+def _check_stages(cfg, r, ref, B, Tp):
+    import torch
+    from hybrid_head_ssm_b200 import runtime as rt
+    lay, ws = r["lay"], r["ws"]
+    mdt = rt.mid_dtype(cfg)
+    di, H, dv = cfg.d_inner, cfg.n_q_heads, cfg.v_head_dim
+    delta = to_np(_ws_view(ws, lay["delta"], (B, Tp, di), torch.float32))
+    o = to_np(_ws_view(ws, lay["O"], (B, Tp, H * dv), mdt))
+    u = to_np(_ws_view(ws, lay["U"], (B, Tp, di), rt.act_dtype(cfg)))
+    tol = dict(max_abs=1e-4 if cfg.dtype == 0 else 6e-2, rel_l2=5e-3)
+    assert_close(delta, ref["delta"], cfg, "Delta", max_abs=tol["max_abs"])
+    assert_close(o, ref["o_attn"], cfg, "attention output", **tol)
+    assert_close(u, ref["u"], cfg, "fused U", max_abs=2e-4 if cfg.dtype == 0 else 1.5e-1, rel_l2=5e-3)
+
+
+@pytest.mark.parametrize("perturb", [False, True])
+def test_tiny_f32_layer(perturb):
+    """Tiny fp32 layer (B=1, T=256 + 16 meta, window 64): y and every stage <= 1e-4."""
+    wl = synth.workload("tiny_f32_b1_t256")
+    cfg = wl["cfg"]
+    w = synth.layer_weights(cfg, wl["seed"])
+    if perturb:
+        w = synth.perturbed_weights(w, cfg, 5)
+    x = synth.layer_input(cfg, wl["B"], wl["T"], wl["seed"])
+    ref = oracle.mixer_prefill(cfg, w, x)
+    r = _run_prefill(cfg, w, x)
+    B, Tp = wl["B"], cfg.n_meta + wl["T"]
+    assert_close(to_np(r["y"]), ref["y"], cfg, "y")
+    _check_stages(cfg, r, ref, B, Tp)
+    assert_close(to_np(r["kv"].k_seq), ref["k"], cfg, "K after RoPE")
+    assert_close(to_np(r["kv"].v_seq), ref["v"], cfg, "V")
+    assert_close(to_np(r["st"].h), ref["h"], cfg, "final SSM state")
+    assert_close(to_np(r["st"].conv), ref["conv"], cfg, "conv state", max_abs=1e-5)
+
+
+def test_tiny_f32_ragged_batch_and_tails():
+    """B=3, T=77 (not a multiple of any tile), window 5, n_meta 16: ragged tails
+    in the GEMM, attention and scan tiles."""
+    cfg = synth.tiny_layer_cfg().with_(window=5)
+    w = synth.perturbed_weights(synth.layer_weights(cfg, 8), cfg, 8)
+    x = synth.layer_input(cfg, 3, 77, 8)
+    ref = oracle.mixer_prefill(cfg, w, x)
+    r = _run_prefill(cfg, w, x)
+    assert_close(to_np(r["y"]), ref["y"], cfg, "y")
+    assert_close(to_np(r["st"].h), ref["h"], cfg, "final SSM state")
+
+
+def test_tiny_f32_global_and_no_meta():
+    """Global attention (window 0) and a layer without meta tokens."""
+    for kw in (dict(window=0), dict(n_meta=0, window=16)):
+        cfg = synth.tiny_layer_cfg().with_(**kw)
+        w = synth.layer_weights(cfg, 9)
+        x = synth.layer_input(cfg, 2, 50, 9)
+        ref = oracle.mixer_prefill(cfg, w, x)
+        r = _run_prefill(cfg, w, x)
+        assert_close(to_np(r["y"]), ref["y"], cfg, f"y {kw}")
+
+
+def test_tiny_f32_kv_share_and_residual_stack():
+    """Producer then consumer (hymba_kv_share, no K/V rows of its own), residual
+    stack with the consumer's input = the producer's output rows (meta included)."""
+    base = synth.tiny_layer_cfg().with_(window=12)
+    ca, cb = base, base.with_(is_kv_producer=0)
+    wa = synth.perturbed_weights(synth.layer_weights(ca, 21), ca, 21)
+    wb = synth.perturbed_weights(synth.layer_weights(cb, 22), cb, 22)
+    x = synth.layer_input(ca, 2, 40, 23)
+    ra = oracle.mixer_prefill(ca, wa, x, residual=True)
+    rb = oracle.mixer_prefill(cb, wb, ra["y"], kv_shared=(ra["k"], ra["v"]), residual=True, x_has_meta=True)
+    import hybrid_head_ssm_b200 as hy
+    ga = _run_prefill(ca, wa, x, flags=hy.HYMBA_ADD_RESIDUAL)
+    assert_close(to_np(ga["y"]), ra["y"], ca, "producer y")
+    # the consumer reads the GPU producer's K/V; its input is the GPU producer's output
+    from hybrid_head_ssm_b200 import runtime as rt
+    torch = torch_cuda()
+    lb = rt.DeviceLayer(cb, wb)
+    kvs = hy.hymba_kv()
+    hy.check(hy.hymba_kv_share(ctypes.byref(ga["kv"].s), ctypes.byref(lb.c), ctypes.byref(kvs)))
+    yb = ga["y"].clone()
+    ws = rt.workspace(cb, 2, 40, hy.HYMBA_MODE_PREFILL)
+    rt.prefill(lb, yb, 40, ga["kv"], yb, ws, None, hy.HYMBA_X_HAS_META | hy.HYMBA_ADD_RESIDUAL,
+               kv_struct_override=kvs)  # in place: y == x
+    torch.cuda.synchronize()
+    assert_close(to_np(yb), rb["y"], cb, "consumer y (in place)", max_abs=2e-4)
+
+
+def test_bf16_hymba15_swa_layer():
+    """Hymba-1.5B-shaped SWA layer, bf16, B=1, T=2048 + 128 meta: the full output."""
+    wl = synth.workload("hymba15_swa1024_b1_t2048")
+    cfg = wl["cfg"]
+    w = synth.layer_weights(cfg, wl["seed"])
+    x = synth.layer_input(cfg, wl["B"], wl["T"], wl["seed"])
+    ref = oracle.mixer_prefill(cfg, w, x)
+    r = _run_prefill(cfg, w, x)
+    mx, rl = assert_close(to_np(r["y"]), ref["y"], cfg, "y")
+    print(f"hymba15 swa layer: max abs {mx:.3e}, rel L2 {rl:.3e}")
+    _check_stages(cfg, r, ref, wl["B"], cfg.n_meta + wl["T"])
+    assert_close(to_np(r["st"].h), ref["h"], cfg, "final SSM state", max_abs=5e-2)
+
+
+def test_bf16_small_perturbed_layer():
+    """A small bf16 layer with every per-channel parameter away from its default,
+    ragged T, KV share to a consumer."""
+    cfg = synth.hymba15_layer_cfg(window=40).with_(d_model=256, n_q_heads=5, n_kv_heads=1,
+                                                   d_inner=640, dt_rank=24, n_meta=8)
+    w = synth.perturbed_weights(synth.layer_weights(cfg, 31), cfg, 31)
+    x = synth.layer_input(cfg, 2, 133, 31)
+    ref = oracle.mixer_prefill(cfg, w, x)
+    r = _run_prefill(cfg, w, x)
+    assert_close(to_np(r["y"]), ref["y"], cfg, "y")
+    cc = cfg.with_(is_kv_producer=0)
+    wc = synth.perturbed_weights(synth.layer_weights(cc, 32), cc, 32)
+    refc = oracle.mixer_prefill(cc, wc, x, kv_shared=(ref["k"], ref["v"]))
+    rc = _run_prefill(cc, wc, x, kv_from=r["kv"])
+    assert_close(to_np(rc["y"]), refc["y"], cc, "consumer y")
+
+
+def test_bf16_global_layer_b4_t8192_sampled_rows():
+    """Global layer, B=4, T=8192 + 128 meta, run in full on the GPU; the oracle
+    recomputes sequences 0 and 3 (rows are independent)."""
+    wl = synth.workload("hymba15_global_b4_t8192")
+    cfg = wl["cfg"]
+    w = synth.layer_weights(cfg, wl["seed"])
+    x = synth.layer_input(cfg, wl["B"], wl["T"], wl["seed"])
+    r = _run_prefill(cfg, w, x)
+    y = to_np(r["y"])
+    for b in (0, 3):
+        ref = oracle.mixer_prefill_row(cfg, w, x[b])
+        mx, rl = assert_close(y[b], ref["y"], cfg, f"y row {b}")
+        print(f"global layer row {b}: max abs {mx:.3e}, rel L2 {rl:.3e}")
+
+
+def test_prefill_fills_decode_ring_bit_exact():
+    """A producer's prefill with a ring smaller than the sequence copies the meta
+    rows and the newest positions into slot n_meta + (p - n_meta) mod R: compare
+    the cache with the prefill's own K/V rows, bit for bit."""
+    torch = torch_cuda()
+    cfg = synth.tiny_layer_cfg().with_(window=8)
+    w = synth.layer_weights(cfg, 3)
+    x = synth.layer_input(cfg, 2, 37, 3)
+    cap = cfg.n_meta + 8
+    r = _run_prefill(cfg, w, x, cache_cap=cap)
+    kv = r["kv"]
+    Tp = cfg.n_meta + 37
+    ks, vs = kv.k_seq.cpu(), kv.v_seq.cpu()
+    kc, vc = kv.k_cache.cpu(), kv.v_cache.cpu()
+    for p in list(range(cfg.n_meta)) + list(range(Tp - 8, Tp)):
+        s = oracle.ring_slot(p, cfg.n_meta, 8)
+        assert torch.equal(kc[:, :, s], ks[:, :, p]) and torch.equal(vc[:, :, s], vs[:, :, p]), p
+    assert kv.len.cpu().tolist() == [Tp, Tp]

@@ -140,7 +140,7 @@ def test_layer_cache_bytes_formula():
     B = 64
     kv = B * 5 * (128 + 1024) * (64 + 128) * 2
     h = B * 3200 * 16 * 4
-    conv = B * 3200 * 4 * 2
+    conv = B * 3200 * 4 * 4
     assert oracle.layer_cache_bytes(cfg, B, 4096 + 128) == kv + h + conv + B * 4
     g = cfg.with_(window=0)
     assert oracle.layer_cache_bytes(g, B, 5000) == B * 5 * (128 + 5000) * 192 * 2 + h + conv + B * 4
