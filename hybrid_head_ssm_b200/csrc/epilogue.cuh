@@ -92,7 +92,10 @@ __device__ void epi_run64(const EpiArgs<T>& e, int r, int c0, float* v) {
     if (e.row_mode == ROWS_DIRECT) { b0 = r / e.Tp; b1 = b0 + 1; t = r % e.Tp; }
     else if (e.row_mode == ROWS_META) { b0 = 0; b1 = e.B; t = r; }
     else if (e.row_mode == ROWS_USER) { b0 = r / e.Tu; b1 = b0 + 1; t = e.n_meta + r % e.Tu; }
-    else { b0 = r; b1 = r + 1; t = e.pos[r] + e.pos_offset; }
+    else {
+        b0 = r; b1 = r + 1; t = e.pos[r] + e.pos_offset;
+        if (t < 0) return;  // no position to write; the decode attention reports the range error
+    }
     const int qw = e.H * e.dh;
     const int kw = e.k_out ? e.G * e.dh : 0;
     const int vw = e.k_out ? e.G * e.dv : 0;
