@@ -352,14 +352,15 @@ def bench_decode(args, torch, hy, rt, max_over_ranks, barrier, world, pk, flush)
     kvb = hy.hymba_kv()
     hy.check(hy.hymba_kv_share(ctypes.byref(kv.s), ctypes.byref(lb.c), ctypes.byref(kvb)))
     sa, sb = rt.State(ca, B), rt.State(cb, B)
-    x = rt.to_device(synth.layer_input(ca, B, T, seed), ca)
-    ya = torch.empty((B, Tp, ca.d_model), dtype=torch.bfloat16, device="cuda")
+    fl = rt.stream_flags(ca)  # fp32 residual stream between the two bf16 layers
+    x = rt.to_device(synth.layer_input(ca, B, T, seed), ca, io_f32=True)
+    ya = torch.empty((B, Tp, ca.d_model), dtype=torch.float32, device="cuda")
     yb = torch.empty_like(ya)
     wsp = rt.workspace(ca, B, T, hy.HYMBA_MODE_PREFILL)
-    rt.prefill(la, x, T, kv, ya, wsp, sa, hy.HYMBA_ADD_RESIDUAL)
-    rt.prefill(lb, ya, T, kv, yb, wsp, sb, hy.HYMBA_X_HAS_META | hy.HYMBA_ADD_RESIDUAL, kv_struct_override=kvb)
+    rt.prefill(la, x, T, kv, ya, wsp, sa, fl)
+    rt.prefill(lb, ya, T, kv, yb, wsp, sb, hy.HYMBA_X_HAS_META | fl, kv_struct_override=kvb)
     del wsp, ya, yb
-    xt = rt.to_device(synth.layer_input(ca, B, 1, seed, tag=1)[:, 0], ca)
+    xt = rt.to_device(synth.layer_input(ca, B, 1, seed, tag=1)[:, 0], ca, io_f32=True)
     ha, hb = torch.empty_like(xt), torch.empty_like(xt)
     wda = rt.workspace(ca, B, cap, hy.HYMBA_MODE_DECODE)
     wdb = rt.workspace(cb, B, cap, hy.HYMBA_MODE_DECODE)
@@ -367,8 +368,8 @@ def bench_decode(args, torch, hy, rt, max_over_ranks, barrier, world, pk, flush)
     stream = torch.cuda.current_stream()
 
     def step():
-        rt.decode(la, xt, kv.s, sa, ha, wda, hy.HYMBA_ADD_RESIDUAL)
-        rt.decode(lb, ha, kvb, sb, hb, wdb, hy.HYMBA_ADD_RESIDUAL)
+        rt.decode(la, xt, kv.s, sa, ha, wda, fl)
+        rt.decode(lb, ha, kvb, sb, hb, wdb, fl)
 
     for _ in range(args.warmup):
         step()

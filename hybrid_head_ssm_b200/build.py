@@ -19,7 +19,7 @@ CSRC = os.path.join(PKG, "csrc")
 OBJ = os.path.join(PKG, "_build")
 LIB = os.path.join(PKG, "libhymba.so")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
-DEFINES: list = []
+DEFINES = ["-DHYMBA_WITH_TCGEN05"]
 
 
 def nvcc() -> str:
@@ -68,7 +68,7 @@ def build(verbose: bool = False, defines=None) -> str:
     with cf.ThreadPoolExecutor(max_workers=max(1, min(len(jobs), os.cpu_count() or 4))) as ex:
         list(ex.map(run, jobs))
     if jobs or _stale(LIB, objs):
-        run([cc] + ARCH + ["-shared", "-Xlinker", "--no-undefined", "-o", LIB] + objs + ["-lcuda"])
+        run([cc] + ARCH + ["-shared", "-Xlinker", "--no-undefined", "-o", LIB] + objs)
     return LIB
 
 

@@ -42,7 +42,8 @@ struct EpiArgs {
     T* y;                  // [M, N]
     int res_mode;          // 0: none; 1: residual = res_x row r; 2: residual = X^ row (meta or user)
     const T* res_x;
-    const T* res_meta;
+    const void* res_meta;  // [n_meta, N] of the layer's weight type
+    int res_meta_bf16;     // 1: res_meta is bf16; 0: it has type T
 };
 
 // RoPE on one 64-wide head run: pairs (i, i+32) rotated by (cos, sin).
@@ -80,9 +81,18 @@ __device__ void epi_run64(const EpiArgs<T>& e, int r, int c0, float* v) {
             for (int j = 0; j < n; ++j) v[j] += to_f(src[j]);
         } else if (e.res_mode == 2) {
             int b = r / e.Tp, t = r % e.Tp;
-            const T* src = t < e.n_meta ? e.res_meta + (long long)t * e.N
-                                        : e.res_x + ((long long)b * e.Tu + (t - e.n_meta)) * e.N;
-            for (int j = 0; j < n; ++j) v[j] += to_f(src[c0 + j]);
+            if (t < e.n_meta) {
+                if (e.res_meta_bf16) {
+                    const bf16* src = static_cast<const bf16*>(e.res_meta) + (long long)t * e.N + c0;
+                    for (int j = 0; j < n; ++j) v[j] += to_f(src[j]);
+                } else {
+                    const T* src = static_cast<const T*>(e.res_meta) + (long long)t * e.N + c0;
+                    for (int j = 0; j < n; ++j) v[j] += to_f(src[j]);
+                }
+            } else {
+                const T* src = e.res_x + ((long long)b * e.Tu + (t - e.n_meta)) * e.N + c0;
+                for (int j = 0; j < n; ++j) v[j] += to_f(src[j]);
+            }
         }
         store_run<T>(e.y + (long long)r * e.N + c0, v, n);
         return;

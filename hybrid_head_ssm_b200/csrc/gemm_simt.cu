@@ -80,6 +80,7 @@ INST(float, float)
 INST(bf16, f16)
 INST(f16, f16)
 INST(bf16, bf16)
+INST(bf16, float)
 #undef INST
 
 }  // namespace hymba

@@ -1,0 +1,269 @@
+// Projection GEMM C = A B^T on the 5th-generation tensor cores (tcgen05), used for
+// the fused input projection, the Delta projection and the output projection of the
+// mixer ("Hymba Guide", Parallel Hybrid-Head Layer Formulation: one projection
+// feeds both head families, one output projection mixes them).
+//
+// Persistent, warp-specialised kernel, one CTA per SM:
+//   warp 0      TMA producer: 128 x 64 A box and BN x 64 B box per k-block into a
+//               4-stage ring of 128-byte-swizzled shared-memory tiles;
+//   warp 1      TMEM allocator and MMA issuer (one thread): 4 x tcgen05.mma
+//               (128 x BN x 16) per k-block into a TMEM accumulator;
+//   warps 2..5  epilogue: tcgen05.ld of the accumulator (32 rows per warp) in runs of
+//               64 columns, then the layer's epilogue (RoPE, K/V scatter, softplus,
+//               residual) and the stores.
+// The accumulator is double-buffered in TMEM so the epilogue of one tile overlaps the
+// MMAs of the next. Every mbarrier wait is bounded; on timeout the CTA records
+// HYMBA_ERR_DEVICE_TIMEOUT, drains what it issued and exits.
+#include "kernels.h"
+#include "tc.cuh"
+
+namespace hymba {
+
+namespace tc {
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*,
+                                  CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
+                                  CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    if (!fn) {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    }
+    return fn;
+}
+
+bool make_tmap_2d(CUtensorMap* map, const void* base, bool is_bf16, uint64_t rows, uint64_t cols, uint64_t ld,
+                  uint32_t box_rows) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn || ((uintptr_t)base & 15) || (ld * 2) % 16) return false;
+    cuuint64_t dims[2] = {cols, rows};
+    cuuint64_t strides[1] = {ld * 2};
+    cuuint32_t box[2] = {64, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(map, is_bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2,
+                    const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                    CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+}  // namespace tc
+
+namespace {
+
+constexpr int BM = 128, BK = 64, STAGES = 4, NUM_THREADS = 192;
+
+template <int BN>
+struct GemmSmem {
+    alignas(1024) uint8_t a[STAGES][BM * BK * 2];
+    alignas(1024) uint8_t b[STAGES][BN * BK * 2];
+    uint64_t full[STAGES];
+    uint64_t empty[STAGES];
+    uint64_t tfull[2];
+    uint64_t tempty[2];
+    uint64_t drain;
+    uint32_t tmem_base;
+    int abort;
+};
+
+__device__ __forceinline__ void fail(volatile int* abort, int* status) {
+    *abort = 1;
+    set_status(status, HYMBA_ERR_DEVICE_TIMEOUT);
+}
+
+template <typename TA, typename TO, int BN>
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, int M, int N,
+               int K, EpiArgs<TO> e, int* status) {
+    extern __shared__ uint8_t smem_raw[];
+    GemmSmem<BN>& s = *reinterpret_cast<GemmSmem<BN>*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                                        ~static_cast<uintptr_t>(1023));
+    constexpr bool kBF16 = sizeof(TA) == 2 && std::is_same<TA, bf16>::value;
+    constexpr uint32_t IDESC = tc::idesc_f16(kBF16, BM, BN);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int num_m = (M + BM - 1) / BM, num_n = (N + BN - 1) / BN;
+    const int num_tiles = num_m * num_n, nk = (K + BK - 1) / BK;
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < STAGES; ++i) {
+            tc::mbar_init(&s.full[i], 1);
+            tc::mbar_init(&s.empty[i], 1);
+        }
+        for (int i = 0; i < 2; ++i) {
+            tc::mbar_init(&s.tfull[i], 1);
+            tc::mbar_init(&s.tempty[i], 128);
+        }
+        tc::mbar_init(&s.drain, 1);
+        s.abort = 0;
+        tc::fence_mbar_init();
+        tc::prefetch_tmap(&tmA);
+        tc::prefetch_tmap(&tmB);
+    }
+    if (warp == 1) {
+        tc::tmem_alloc(&s.tmem_base, 2 * BN);
+        tc::tmem_relinquish();
+    }
+    tc::tc_fence_before();
+    __syncthreads();
+    tc::tc_fence_after();
+    const uint32_t tmem = s.tmem_base;
+    volatile int* abort = &s.abort;
+
+    if (warp == 0) {
+        // ---------------- TMA producer ----------------
+        if (tc::elect_one()) {
+            int it = 0;
+            int issued_phase[STAGES];
+            for (int i = 0; i < STAGES; ++i) issued_phase[i] = -1;
+            for (int tile = blockIdx.x; tile < num_tiles && !*abort; tile += gridDim.x) {
+                const int m_blk = tile % num_m, n_blk = tile / num_m;
+                for (int kb = 0; kb < nk; ++kb, ++it) {
+                    const int st = it % STAGES;
+                    const uint32_t ph = (it / STAGES) & 1;
+                    if (!tc::mbar_wait(&s.empty[st], ph ^ 1, abort)) { fail(abort, status); break; }
+                    tc::mbar_arrive_expect_tx(&s.full[st], (BM + BN) * BK * 2);
+                    tc::tma_load_2d(s.a[st], &tmA, &s.full[st], kb * BK, m_blk * BM);
+                    tc::tma_load_2d(s.b[st], &tmB, &s.full[st], kb * BK, n_blk * BN);
+                    issued_phase[st] = (int)ph;
+                }
+            }
+            if (*abort) {
+                // let the copies this thread issued land before the CTA exits
+                int zero = 0;
+                for (int i = 0; i < STAGES; ++i)
+                    if (issued_phase[i] >= 0) tc::mbar_wait(&s.full[i], (uint32_t)issued_phase[i], &zero);
+            }
+        }
+    } else if (warp == 1) {
+        // ---------------- MMA issuer ----------------
+        if (tc::elect_one()) {
+            int it = 0, tcount = 0;
+            for (int tile = blockIdx.x; tile < num_tiles && !*abort; tile += gridDim.x, ++tcount) {
+                const int buf = tcount & 1;
+                const uint32_t tph = (tcount >> 1) & 1;
+                if (!tc::mbar_wait(&s.tempty[buf], tph ^ 1, abort)) { fail(abort, status); break; }
+                tc::tc_fence_after();
+                const uint32_t d = tmem + buf * BN;
+                bool ok = true;
+                for (int kb = 0; kb < nk; ++kb, ++it) {
+                    const int st = it % STAGES;
+                    const uint32_t ph = (it / STAGES) & 1;
+                    if (!tc::mbar_wait(&s.full[st], ph, abort)) { fail(abort, status); ok = false; break; }
+                    tc::tc_fence_after();
+                    const uint32_t a0 = tc::smem_u32(s.a[st]), b0 = tc::smem_u32(s.b[st]);
+#pragma unroll
+                    for (int kk = 0; kk < BK / 16; ++kk)
+                        tc::mma_f16_ss(d, tc::sdesc_k_sw128(a0 + kk * 32), tc::sdesc_k_sw128(b0 + kk * 32), IDESC,
+                                       (kb | kk) != 0);
+                    tc::mma_commit(&s.empty[st]);
+                }
+                if (!ok) break;
+                tc::mma_commit(&s.tfull[buf]);
+            }
+            // all MMAs issued by this thread have completed once `drain` flips
+            tc::mma_commit(&s.drain);
+            int zero = 0;
+            tc::mbar_wait(&s.drain, 0, &zero);
+        }
+    } else {
+        // ---------------- epilogue (warps 2..5 -> TMEM lane quadrants 2, 3, 0, 1) ----------------
+        const int q = warp & 3;
+        int tcount = 0;
+        for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++tcount) {
+            const int buf = tcount & 1;
+            const uint32_t tph = (tcount >> 1) & 1;
+            if (!tc::mbar_wait(&s.tfull[buf], tph, abort)) { fail(abort, status); break; }
+            tc::tc_fence_after();
+            const int m_blk = tile % num_m, n_blk = tile / num_m;
+            const int row = m_blk * BM + q * 32 + lane;
+#pragma unroll 1
+            for (int j = 0; j < BN / 64; ++j) {
+                uint32_t r0[32], r1[32];
+                const uint32_t taddr = tmem + ((uint32_t)(q * 32) << 16) + buf * BN + j * 64;
+                tc::tmem_ld32(taddr, r0);
+                tc::tmem_ld32(taddr + 32, r1);
+                tc::tmem_wait_ld();
+                float v[64];
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    v[i] = __uint_as_float(r0[i]);
+                    v[32 + i] = __uint_as_float(r1[i]);
+                }
+                epi_run64<TO>(e, row, n_blk * BN + j * 64, v);
+            }
+            tc::tc_fence_before();
+            tc::mbar_arrive(&s.tempty[buf]);
+        }
+    }
+    tc::tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc::tc_fence_after();
+        tc::tmem_dealloc(tmem, 2 * BN);
+    }
+}
+
+template <typename TA, typename TO, int BN>
+int launch_bn(const Ctx& ctx, const char* name, const TA* A, long long lda, const TA* Bw, long long ldb, int M,
+              int N, int K, const EpiArgs<TO>& e) {
+    constexpr bool kBF16 = std::is_same<TA, bf16>::value;
+    CUtensorMap ta, tb;
+    if (!tc::make_tmap_2d(&ta, A, kBF16, M, K, lda, BM)) return HYMBA_ERR_UNSUPPORTED;
+    if (!tc::make_tmap_2d(&tb, Bw, kBF16, N, K, ldb, BN)) return HYMBA_ERR_UNSUPPORTED;
+    const size_t smem = sizeof(GemmSmem<BN>) + 1024;
+    auto kern = gemm_tc_kernel<TA, TO, BN>;
+    static bool attr_set = false;
+    if (!attr_set) {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+            return HYMBA_ERR_CUDA;
+        attr_set = true;
+    }
+    const int tiles = ((M + BM - 1) / BM) * ((N + BN - 1) / BN);
+    const int grid = tiles < ctx.sm_count ? tiles : ctx.sm_count;
+    HYMBA_LAUNCH(ctx, name, kern, grid, NUM_THREADS, smem, ta, tb, M, N, K, e, ctx.status);
+    return HYMBA_OK;
+}
+
+}  // namespace
+
+// Tile width: the BN in {256, 128, 64} with the least estimated time, counting whole
+// waves of persistent CTAs and the lower operand reuse of narrow tiles.
+static int pick_bn(int M, int N, int sms) {
+    int best = 256;
+    double best_cost = 1e30;
+    for (int bn : {256, 128, 64}) {
+        const long long tiles = (long long)((M + BM - 1) / BM) * ((N + bn - 1) / bn);
+        const long long waves = (tiles + sms - 1) / sms;
+        const double cost = (double)waves * bn * (bn >= 128 ? 1.0 : 1.5);
+        if (cost < best_cost - 1e-9) { best_cost = cost; best = bn; }
+    }
+    return best;
+}
+
+template <typename TA, typename TO>
+int launch_gemm_tc(const Ctx& ctx, const char* name, const TA* A, long long lda, const TA* Bw, long long ldb,
+                   int M, int N, int K, const EpiArgs<TO>& e) {
+    if (M <= 0 || N <= 0) return HYMBA_OK;
+    switch (pick_bn(M, N, ctx.sm_count > 0 ? ctx.sm_count : 148)) {
+        case 256: return launch_bn<TA, TO, 256>(ctx, name, A, lda, Bw, ldb, M, N, K, e);
+        case 128: return launch_bn<TA, TO, 128>(ctx, name, A, lda, Bw, ldb, M, N, K, e);
+        default: return launch_bn<TA, TO, 64>(ctx, name, A, lda, Bw, ldb, M, N, K, e);
+    }
+}
+
+#define INST(TA, TO)                                                                                        \
+    template int launch_gemm_tc<TA, TO>(const Ctx&, const char*, const TA*, long long, const TA*, long long, \
+                                        int, int, int, const EpiArgs<TO>&);
+INST(bf16, f16)
+INST(f16, f16)
+INST(bf16, bf16)
+INST(bf16, float)
+#undef INST
+
+}  // namespace hymba

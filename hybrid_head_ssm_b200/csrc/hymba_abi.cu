@@ -5,6 +5,7 @@
 #include <algorithm>
 #include <atomic>
 #include <cstring>
+#include <type_traits>
 #include <mutex>
 #include <vector>
 
@@ -112,7 +113,7 @@ static Cols columns(const hymba_layer_cfg* c) {
 
 struct Plan {
     size_t total = 0;
-    size_t rope = 0, P = 0, delta = 0, O = 0, ypre = 0, U = 0, wdt = 0, part = 0;
+    size_t rope = 0, P = 0, delta = 0, O = 0, ypre = 0, U = 0, wdt = 0, part = 0, xcv = 0;
     long long ldP = 0;
     int rpad = 0, n_split = 1;
 };
@@ -141,6 +142,7 @@ static Plan plan(const hymba_layer_cfg* c, int B, int T, int mode) {
     p.ypre = take(&cur, rows * di * esz);
     p.U = take(&cur, rows * di * esz);
     p.wdt = take(&cur, (size_t)di * p.rpad * esz);
+    if (c->dtype == HYMBA_BF16) p.xcv = take(&cur, rows * c->d_model * 2);  // bf16 copy of fp32 input
     if (mode == HYMBA_MODE_DECODE) {
         p.n_split = decode_splits(T);
         p.part = take(&cur, (size_t)B * c->n_q_heads * p.n_split * (c->v_head_dim + 2) * sizeof(float));
@@ -189,9 +191,10 @@ static EpiArgs<T> epi_base(int kind, int M, int N) {
 // T: the layer's I/O and weight type (fp32 or bf16). I: its intermediate type
 // (fp32, or fp16 for bf16 layers: the projection, K/V, attention output and y_pre are
 // held in fp16, which has the same width as bf16 and a finer mantissa).
-template <typename T, typename I>
+// TIO: type of x and y (T, or fp32 for a bf16 layer in a fp32 residual stream).
+template <typename T, typename I, typename TIO>
 static int prefill_impl(const Ctx& ctx, const hymba_layer_cfg* c, const hymba_layer_weights* w,
-                        const T* x, int B, int T_, int flags, T* y, hymba_kv* kv,
+                        const TIO* x_io, int B, int T_, int flags, TIO* y, hymba_kv* kv,
                         hymba_ssm_state* st, char* ws) {
     const Plan pl = plan(c, B, T_, HYMBA_MODE_PREFILL);
     const Cols k = columns(c);
@@ -210,6 +213,15 @@ static int prefill_impl(const Ctx& ctx, const hymba_layer_cfg* c, const hymba_la
     I* v_seq = static_cast<I*>(kv->v_seq);
     int rc;
 
+    const T* x;
+    if constexpr (std::is_same<TIO, T>::value) {
+        x = x_io;
+    } else {
+        T* xc = reinterpret_cast<T*>(ws + pl.xcv);
+        const int xrows = B * (has_meta ? Tp : T_);
+        if ((rc = launch_pad_copy<TIO, T>(ctx, x_io, xrows, d, xc, d))) return rc;
+        x = xc;
+    }
     if ((rc = launch_rope_table(ctx, rope, Tp, dh, c->rope_base))) return rc;
     // 1. fused input projection (+ RoPE, K/V scatter) ------------------------------
     EpiArgs<I> ep = epi_base<I>(EPI_INPROJ, 0, k.n_in);
@@ -250,14 +262,15 @@ static int prefill_impl(const Ctx& ctx, const hymba_layer_cfg* c, const hymba_la
                                 w->beta2, U, (int)rows, di, c->rms_eps, nullptr)))
         return rc;
     // 6. output projection (+ residual) -------------------------------------------------
-    EpiArgs<T> eo = epi_base<T>(EPI_OUT, (int)rows, d);
+    EpiArgs<TIO> eo = epi_base<TIO>(EPI_OUT, (int)rows, d);
     eo.y = y; eo.B = B; eo.Tu = T_; eo.Tp = Tp; eo.n_meta = m;
     if (flags & HYMBA_ADD_RESIDUAL) {
         eo.res_mode = has_meta ? 1 : 2;
-        eo.res_x = x;
-        eo.res_meta = static_cast<const T*>(w->meta);
+        eo.res_x = x_io;
+        eo.res_meta = w->meta;
+        eo.res_meta_bf16 = std::is_same<T, bf16>::value;
     }
-    if ((rc = gemm<T, T>(ctx, "gemm_out_proj", U, di, static_cast<const T*>(w->w_out), di, (int)rows, d, di, eo))) return rc;
+    if ((rc = gemm<T, TIO>(ctx, "gemm_out_proj", U, di, static_cast<const T*>(w->w_out), di, (int)rows, d, di, eo))) return rc;
     // 7. decode cache of a producer ------------------------------------------------------
     if (c->is_kv_producer && kv->k_cache) {
         if ((rc = launch_cache_fill<I>(ctx, k_seq, v_seq, kv->seq_cap, static_cast<I*>(kv->k_cache),
@@ -267,9 +280,9 @@ static int prefill_impl(const Ctx& ctx, const hymba_layer_cfg* c, const hymba_la
     return HYMBA_OK;
 }
 
-template <typename T, typename I>
+template <typename T, typename I, typename TIO>
 static int decode_impl(const Ctx& ctx, const hymba_layer_cfg* c, const hymba_layer_weights* w,
-                       const T* x, int B, int flags, T* y, hymba_kv* kv, hymba_ssm_state* st,
+                       const TIO* x_io, int B, int flags, TIO* y, hymba_kv* kv, hymba_ssm_state* st,
                        char* ws) {
     const Plan pl = plan(c, B, kv->cache_cap, HYMBA_MODE_DECODE);
     const Cols k = columns(c);
@@ -286,6 +299,14 @@ static int decode_impl(const Ctx& ctx, const hymba_layer_cfg* c, const hymba_lay
     I* k_cache = static_cast<I*>(kv->k_cache);
     I* v_cache = static_cast<I*>(kv->v_cache);
     int rc;
+    const T* x;
+    if constexpr (std::is_same<TIO, T>::value) {
+        x = x_io;
+    } else {
+        T* xc = reinterpret_cast<T*>(ws + pl.xcv);
+        if ((rc = launch_pad_copy<TIO, T>(ctx, x_io, B, d, xc, d))) return rc;
+        x = xc;
+    }
     EpiArgs<I> ep = epi_base<I>(EPI_INPROJ, B, k.n_in);
     ep.row_mode = ROWS_DECODE;
     ep.B = B; ep.Tu = 1; ep.Tp = 1; ep.n_meta = m;
@@ -311,10 +332,10 @@ static int decode_impl(const Ctx& ctx, const hymba_layer_cfg* c, const hymba_lay
     if ((rc = launch_fuse<I, T>(ctx, O, ypre, P, pl.ldP, k.z, w->norm_attn_w, w->norm_ssm_w, w->beta1,
                                 w->beta2, U, B, di, c->rms_eps, c->is_kv_producer ? kv->len : nullptr)))
         return rc;
-    EpiArgs<T> eo = epi_base<T>(EPI_OUT, B, d);
+    EpiArgs<TIO> eo = epi_base<TIO>(EPI_OUT, B, d);
     eo.y = y;
-    if (flags & HYMBA_ADD_RESIDUAL) { eo.res_mode = 1; eo.res_x = x; }
-    if ((rc = gemm<T, T>(ctx, "gemm_out_proj_decode", U, di, static_cast<const T*>(w->w_out), di, B, d, di, eo))) return rc;
+    if (flags & HYMBA_ADD_RESIDUAL) { eo.res_mode = 1; eo.res_x = x_io; }
+    if ((rc = gemm<T, TIO>(ctx, "gemm_out_proj_decode", U, di, static_cast<const T*>(w->w_out), di, B, d, di, eo))) return rc;
     return HYMBA_OK;
 }
 
@@ -363,7 +384,8 @@ int hymba_mixer_prefill(const hymba_layer_cfg* cfg, const hymba_layer_weights* w
     int rc = check_cfg(cfg);
     if (rc) return rc;
     if ((rc = check_weights(cfg, w))) return rc;
-    if (!x || !y || !kv || !workspace || B <= 0 || T <= 0 || (flags & ~3)) return HYMBA_ERR_INVALID_ARG;
+    if (!x || !y || !kv || !workspace || B <= 0 || T <= 0 || (flags & ~7)) return HYMBA_ERR_INVALID_ARG;
+    if ((flags & HYMBA_IO_F32) && cfg->dtype != HYMBA_BF16) return HYMBA_ERR_INVALID_ARG;
     if ((uintptr_t)workspace & 255) return HYMBA_ERR_INVALID_ARG;
     if (!kv->k_seq || !kv->v_seq) return HYMBA_ERR_INVALID_ARG;
     if ((rc = check_kv_shape(cfg, kv, B))) return rc;
@@ -378,7 +400,7 @@ int hymba_mixer_prefill(const hymba_layer_cfg* cfg, const hymba_layer_weights* w
         const size_t yb = (size_t)B * Tp * cfg->d_model;
         const char* xs = static_cast<const char*>(x);
         const char* ys = static_cast<const char*>(y);
-        const size_t es = cfg->dtype == HYMBA_BF16 ? 2 : 4;
+        const size_t es = (cfg->dtype == HYMBA_BF16 && !(flags & HYMBA_IO_F32)) ? 2 : 4;
         if (xs < ys + yb * es && ys < xs + xb * es) return HYMBA_ERR_INVALID_ARG;
     } else if (!(flags & HYMBA_X_HAS_META)) {
         return HYMBA_ERR_INVALID_ARG;
@@ -387,11 +409,14 @@ int hymba_mixer_prefill(const hymba_layer_cfg* cfg, const hymba_layer_weights* w
     Ctx ctx;
     if ((rc = current_ctx(static_cast<cudaStream_t>(stream), &ctx))) return rc;
     char* ws = static_cast<char*>(workspace);
+    if (cfg->dtype == HYMBA_BF16 && (flags & HYMBA_IO_F32))
+        return prefill_impl<bf16, f16, float>(ctx, cfg, w, static_cast<const float*>(x), B, T, flags,
+                                              static_cast<float*>(y), kv, st, ws);
     if (cfg->dtype == HYMBA_BF16)
-        return prefill_impl<bf16, f16>(ctx, cfg, w, static_cast<const bf16*>(x), B, T, flags,
-                                       static_cast<bf16*>(y), kv, st, ws);
-    return prefill_impl<float, float>(ctx, cfg, w, static_cast<const float*>(x), B, T, flags,
-                                      static_cast<float*>(y), kv, st, ws);
+        return prefill_impl<bf16, f16, bf16>(ctx, cfg, w, static_cast<const bf16*>(x), B, T, flags,
+                                             static_cast<bf16*>(y), kv, st, ws);
+    return prefill_impl<float, float, float>(ctx, cfg, w, static_cast<const float*>(x), B, T, flags,
+                                             static_cast<float*>(y), kv, st, ws);
 }
 
 int hymba_mixer_decode(const hymba_layer_cfg* cfg, const hymba_layer_weights* w, const void* x_t,
@@ -401,8 +426,9 @@ int hymba_mixer_decode(const hymba_layer_cfg* cfg, const hymba_layer_weights* w,
     if (rc) return rc;
     if ((rc = check_weights(cfg, w))) return rc;
     if (!x_t || !y_t || !kv || !st || !st->h || !st->conv || !workspace || B <= 0 ||
-        (flags & ~HYMBA_ADD_RESIDUAL))
+        (flags & ~(HYMBA_ADD_RESIDUAL | HYMBA_IO_F32)))
         return HYMBA_ERR_INVALID_ARG;
+    if ((flags & HYMBA_IO_F32) && cfg->dtype != HYMBA_BF16) return HYMBA_ERR_INVALID_ARG;
     if ((uintptr_t)workspace & 255) return HYMBA_ERR_INVALID_ARG;
     if (!kv->k_cache || !kv->v_cache || !kv->len || kv->cache_cap <= cfg->n_meta) return HYMBA_ERR_INVALID_ARG;
     if ((rc = check_kv_shape(cfg, kv, B))) return rc;
@@ -410,11 +436,14 @@ int hymba_mixer_decode(const hymba_layer_cfg* cfg, const hymba_layer_weights* w,
     Ctx ctx;
     if ((rc = current_ctx(static_cast<cudaStream_t>(stream), &ctx))) return rc;
     char* ws = static_cast<char*>(workspace);
+    if (cfg->dtype == HYMBA_BF16 && (flags & HYMBA_IO_F32))
+        return decode_impl<bf16, f16, float>(ctx, cfg, w, static_cast<const float*>(x_t), B, flags,
+                                             static_cast<float*>(y_t), kv, st, ws);
     if (cfg->dtype == HYMBA_BF16)
-        return decode_impl<bf16, f16>(ctx, cfg, w, static_cast<const bf16*>(x_t), B, flags,
-                                      static_cast<bf16*>(y_t), kv, st, ws);
-    return decode_impl<float, float>(ctx, cfg, w, static_cast<const float*>(x_t), B, flags,
-                                     static_cast<float*>(y_t), kv, st, ws);
+        return decode_impl<bf16, f16, bf16>(ctx, cfg, w, static_cast<const bf16*>(x_t), B, flags,
+                                            static_cast<bf16*>(y_t), kv, st, ws);
+    return decode_impl<float, float, float>(ctx, cfg, w, static_cast<const float*>(x_t), B, flags,
+                                            static_cast<float*>(y_t), kv, st, ws);
 }
 
 int hymba_kv_share(const hymba_kv* producer, const hymba_layer_cfg* consumer_cfg, hymba_kv* out) {

@@ -88,5 +88,12 @@ def decode(layer: DeviceLayer, x_t: torch.Tensor, kv_s, state: State, y_t: torch
                              ws.data_ptr(), ws.numel(), current_stream_ptr()))
 
 
-def to_device(a: np.ndarray, cfg, device="cuda") -> torch.Tensor:
-    return torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).to(device=device, dtype=act_dtype(cfg))
+def to_device(a: np.ndarray, cfg, device="cuda", io_f32: bool = False) -> torch.Tensor:
+    dt = torch.float32 if io_f32 else act_dtype(cfg)
+    return torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).to(device=device, dtype=dt)
+
+
+def stream_flags(cfg) -> int:
+    """Flags of a layer inside a residual stack: fp32 residual stream for bf16 layers."""
+    from . import HYMBA_ADD_RESIDUAL, HYMBA_IO_F32
+    return HYMBA_ADD_RESIDUAL | (HYMBA_IO_F32 if cfg.dtype == HYMBA_BF16 else 0)

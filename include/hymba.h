@@ -72,6 +72,9 @@ extern "C" {
 /* flags of the mixer calls */
 #define HYMBA_X_HAS_META    1  /* x already holds the n_meta rows (a later layer of a stack) */
 #define HYMBA_ADD_RESIDUAL  2  /* y = X^ + mixer(X^) */
+#define HYMBA_IO_F32        4  /* bf16 layer with fp32 x, y: a residual stream kept in fp32
+                                  between stacked layers (the projection operand X^ is
+                                  rounded to bf16 inside; the residual add is fp32) */
 
 /* workspace modes */
 #define HYMBA_MODE_PREFILL 0
@@ -161,7 +164,8 @@ typedef struct hymba_ssm_state {
 
 /* Prefill of B sequences of T user tokens through one layer.
  *   x: device [B, T, d_model] dtype, or [B, n_meta+T, d_model] with HYMBA_X_HAS_META.
- *   y: device [B, n_meta+T, d_model] dtype (meta rows included, so stacks compose).
+ *   y: device [B, n_meta+T, d_model] dtype (meta rows included, so stacks compose);
+ *      x and y are fp32 instead when HYMBA_IO_F32 is set.
  *      y may equal x when HYMBA_X_HAS_META is set (in-place residual stacks);
  *      otherwise y and x must not overlap.
  *   kv: producer: k_seq/v_seq written (and the decode cache filled if k_cache);
@@ -176,7 +180,8 @@ int hymba_mixer_prefill(const hymba_layer_cfg* cfg, const hymba_layer_weights* w
 
 /* One decode step: one new token per sequence, all B sequences at the same position
  * len[b] (producer) or len[b]-1 (consumer).
- *   x_t: device [B, d_model]; y_t: device [B, d_model] (may equal x_t).
+ *   x_t: device [B, d_model]; y_t: device [B, d_model] (may equal x_t); fp32 with
+ *   HYMBA_IO_F32, else dtype. Flags: HYMBA_ADD_RESIDUAL, HYMBA_IO_F32.
  *   kv must hold a decode cache (k_cache, len); st is updated in place. A cache
  *   whose ring is too short for the layer's span makes the step record
  *   HYMBA_ERR_DEVICE_RANGE in the status word and write zeros for that row. */

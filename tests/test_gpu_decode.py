@@ -33,24 +33,27 @@ class _Pair:
         self.wda = rt.workspace(ca, B, cache_cap, hy.HYMBA_MODE_DECODE)
         self.wdb = rt.workspace(cb, B, cache_cap, hy.HYMBA_MODE_DECODE)
         self.Tprompt = Tprompt
+        # residual stream between the two layers: fp32 for bf16 layers
+        self.flags = rt.stream_flags(ca)
+        self.io_f32 = bool(self.flags & hy.HYMBA_IO_F32) or ca.dtype == 0
 
     def prefill(self, x):
         hy, rt, torch = self.hy, self.rt, self.torch
-        xd = rt.to_device(x, self.ca)
-        ya = torch.empty((self.B, self.ca.n_meta + self.Tprompt, self.ca.d_model), dtype=rt.act_dtype(self.ca), device="cuda")
-        rt.prefill(self.la, xd, self.Tprompt, self.kv, ya, self.wsa, self.sa, hy.HYMBA_ADD_RESIDUAL)
+        xd = rt.to_device(x, self.ca, io_f32=self.io_f32)
+        ya = torch.empty((self.B, self.ca.n_meta + self.Tprompt, self.ca.d_model), dtype=xd.dtype, device="cuda")
+        rt.prefill(self.la, xd, self.Tprompt, self.kv, ya, self.wsa, self.sa, self.flags)
         yb = torch.empty_like(ya)
         rt.prefill(self.lb, ya, self.Tprompt, self.kv, yb, self.wsb, self.sb,
-                   hy.HYMBA_X_HAS_META | hy.HYMBA_ADD_RESIDUAL, kv_struct_override=self.kvb)
+                   hy.HYMBA_X_HAS_META | self.flags, kv_struct_override=self.kvb)
         return ya, yb
 
     def step(self, x_t):
         hy, rt, torch = self.hy, self.rt, self.torch
-        xd = rt.to_device(x_t, self.ca)
+        xd = rt.to_device(x_t, self.ca, io_f32=self.io_f32)
         ya = torch.empty_like(xd)
         yb = torch.empty_like(xd)
-        rt.decode(self.la, xd, self.kv.s, self.sa, ya, self.wda, hy.HYMBA_ADD_RESIDUAL)
-        rt.decode(self.lb, ya, self.kvb, self.sb, yb, self.wdb, hy.HYMBA_ADD_RESIDUAL)
+        rt.decode(self.la, xd, self.kv.s, self.sa, ya, self.wda, self.flags)
+        rt.decode(self.lb, ya, self.kvb, self.sb, yb, self.wdb, self.flags)
         return ya, yb
 
 
