@@ -37,6 +37,7 @@ HYMBA_BF16 = 1
 HYMBA_F16 = 2
 HYMBA_X_HAS_META = 1
 HYMBA_ADD_RESIDUAL = 2
+HYMBA_IO_F32 = 4
 HYMBA_MODE_PREFILL = 0
 HYMBA_MODE_DECODE = 1
 

@@ -19,7 +19,7 @@ CSRC = os.path.join(PKG, "csrc")
 OBJ = os.path.join(PKG, "_build")
 LIB = os.path.join(PKG, "libhymba.so")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
-DEFINES = ["-DHYMBA_WITH_TCGEN05"]
+DEFINES = ["-DHYMBA_WITH_TCGEN05", "-DHYMBA_WITH_TCGEN05_ATTN"]
 
 
 def nvcc() -> str:

@@ -72,7 +72,18 @@ __device__ void epi_run64(const EpiArgs<T>& e, int r, int c0, float* v) {
     const int n = min(64, e.N - c0);
     if (e.kind == EPI_DELTA) {
         float* dst = e.delta + (long long)r * e.N + c0;
-        for (int j = 0; j < n; ++j) dst[j] = softplus_f(v[j] + e.b_dt[c0 + j]);
+        const float* bias = e.b_dt + c0;
+        if (n == 64 && (e.N & 3) == 0) {
+#pragma unroll
+            for (int j = 0; j < 64; j += 4) {
+                const float4 bb = *reinterpret_cast<const float4*>(bias + j);
+                *reinterpret_cast<float4*>(dst + j) =
+                    make_float4(softplus_f(v[j] + bb.x), softplus_f(v[j + 1] + bb.y), softplus_f(v[j + 2] + bb.z),
+                                softplus_f(v[j + 3] + bb.w));
+            }
+        } else {
+            for (int j = 0; j < n; ++j) dst[j] = softplus_f(v[j] + bias[j]);
+        }
         return;
     }
     if (e.kind == EPI_OUT) {

@@ -53,6 +53,21 @@ bool make_tmap_2d(CUtensorMap* map, const void* base, bool is_bf16, uint64_t row
     return r == CUDA_SUCCESS;
 }
 
+bool make_tmap_3d(CUtensorMap* map, const void* base, bool is_bf16, uint64_t planes, uint64_t rows,
+                  uint64_t cols, uint64_t ld, uint64_t plane_ld, uint32_t box_rows) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn || ((uintptr_t)base & 15) || (ld * 2) % 16 || (plane_ld * 2) % 16) return false;
+    cuuint64_t dims[3] = {cols, rows, planes};
+    cuuint64_t strides[2] = {ld * 2, plane_ld * 2};
+    cuuint32_t box[3] = {64, box_rows, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = fn(map, is_bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3,
+                    const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                    CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 }  // namespace tc
 
 namespace {
