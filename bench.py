@@ -133,6 +133,22 @@ def decode_work(cfg, B, cap):
     }
 
 
+def rank_inputs_seed(seed: int, rank: int) -> int:
+    """Weak scaling: every rank runs its own sequences, drawn from its own stream."""
+    return seed + rank
+
+
+def max_over_ranks(value: float, world: int, device: str) -> float:
+    """The slowest rank's time (every rank calls this collectively)."""
+    if world == 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 def cpu_cores():
     try:
         return len(os.sched_getaffinity(0))
@@ -208,19 +224,15 @@ def main():
         if world > 1:
             dist.barrier()
 
-    def max_over_ranks(v):
-        if world == 1:
-            return v
-        t = torch.tensor([v], dtype=torch.float64, device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+    def max_ranks(v):
+        return max_over_ranks(v, world, "cuda")
 
     pk = peaks()
     wl = synth.workload(WORKLOAD)
     cfg, B, T = wl["cfg"], wl["B"], wl["T"]
     Tp = cfg.n_meta + T
     w = synth.layer_weights(cfg, wl["seed"])
-    x_np = synth.layer_input(cfg, B, T, wl["seed"] + rank)
+    x_np = synth.layer_input(cfg, B, T, rank_inputs_seed(wl["seed"], rank))
     layer = rt.DeviceLayer(cfg, w)
     x = rt.to_device(x_np, cfg)
     y = torch.empty((B, Tp, cfg.d_model), dtype=torch.bfloat16, device="cuda")
@@ -256,7 +268,7 @@ def main():
     hy.hymba_trace_enable(0)
     clk = clocks.stop()
     step_ms = [a.elapsed_time(b) for a, b in ev]
-    ms = max_over_ranks(sum(step_ms) / len(step_ms))
+    ms = max_ranks(sum(step_ms) / len(step_ms))
     tokens = B * T * world
     value = tokens / (ms * 1e-3)
 
@@ -300,12 +312,12 @@ def main():
         torch.cuda.synchronize()
         if i >= args.warmup:
             e2e_ms.append(a.elapsed_time(b))
-    e2e_ms_step = max_over_ranks(sum(e2e_ms) / len(e2e_ms))
+    e2e_ms_step = max_ranks(sum(e2e_ms) / len(e2e_ms))
 
     # ---- decode step of the KV-sharing pair (B=64, ring 1024 + 128 meta)
     dec = None
     if not args.no_decode:
-        dec = bench_decode(args, torch, hy, rt, max_over_ranks, barrier, world, pk, flush)
+        dec = bench_decode(args, torch, hy, rt, max_ranks, barrier, world, pk, flush)
 
     out = None
     if rank == 0:

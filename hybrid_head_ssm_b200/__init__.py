@@ -18,7 +18,7 @@ LIB_PATH = os.path.join(_HERE, "libhymba.so")
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(
-        f"{LIB_PATH} is missing: build it with `python -m hybrid_head_ssm_b200.build` "
+        f"{LIB_PATH} is missing: build it with `python hybrid_head_ssm_b200/build.py` "
         "(the mixer has no non-CUDA implementation)")
 
 _lib = ctypes.CDLL(LIB_PATH)
@@ -83,6 +83,7 @@ _sig = {
                                          ctypes.c_int64, ctypes.c_int, ctypes.c_int]),
     "hymba_ssm_state_bytes": (ctypes.c_uint64, [ctypes.c_int] * 5),
     "hymba_get_device_status": (ctypes.c_int, [_vp]),
+    "hymba_get_device_diag": (ctypes.c_int, [_P(ctypes.c_int32), ctypes.c_int]),
     "hymba_strerror": (ctypes.c_char_p, [ctypes.c_int]),
     "hymba_trace_enable": (ctypes.c_int, [ctypes.c_int]),
     "hymba_trace_collect": (ctypes.c_int, [_P(ctypes.c_char_p), _P(ctypes.c_float), ctypes.c_int]),
@@ -113,6 +114,12 @@ def workspace_layout(cfg: hymba_layer_cfg, B: int, T: int, mode: int) -> dict:
     check(hymba_workspace_layout(ctypes.byref(cfg), B, T, mode, out, 10))
     keys = ("total", "P", "ldP", "delta", "O", "ypre", "U", "rope", "part", "n_split")
     return dict(zip(keys, list(out)))
+
+
+def device_diag():
+    out = (ctypes.c_int32 * 7)()
+    check(hymba_get_device_diag(out, 7))
+    return list(out)
 
 
 def trace_collect(max_records: int = 8192):

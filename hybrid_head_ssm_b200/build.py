@@ -1,6 +1,7 @@
 """Build libhymba.so in-tree with nvcc for sm_100a (B200).
 
-Run as `python -m hybrid_head_ssm_b200.build` (or through __graft_entry__.build()).
+Run as `python hybrid_head_ssm_b200/build.py` (or through __graft_entry__.build());
+`python -m` would import the package, which loads the library being built.
 Objects are rebuilt when a source or header is newer than the object; the shared
 library is relinked when any object changed. Needs no GPU.
 """

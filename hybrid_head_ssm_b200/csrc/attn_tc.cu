@@ -58,9 +58,9 @@ struct Blocks {
     }
 };
 
-__device__ __forceinline__ void fail(volatile int* abort, int* status) {
+__device__ __forceinline__ void fail(volatile int* abort, int* status, int role, int step, int bar) {
     *abort = 1;
-    set_status(status, HYMBA_ERR_DEVICE_TIMEOUT);
+    tc::record_timeout(status, role, step, bar);
 }
 
 __global__ void __launch_bounds__(NTHREADS, 1)
@@ -117,7 +117,7 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
             for (int j = 0; j < nblk; ++j) {
                 const int st = j & 1;
                 const uint32_t ph = (j >> 1) & 1;
-                if (!tc::mbar_wait(&s.kv_empty[st], ph ^ 1, abort)) { fail(abort, status); break; }
+                if (!tc::mbar_wait(&s.kv_empty[st], ph ^ 1, abort)) { fail(abort, status, 0, j, 1); break; }
                 int j0, rs, re;
                 blk.get(j, &j0, &rs, &re);
                 tc::mbar_arrive_expect_tx(&s.kv_full[st], KBLK * (DH + DV) * 2);
@@ -135,16 +135,14 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
         // ---------------- MMA issuer ----------------
         if (tc::elect_one()) {
             bool ok = tc::mbar_wait(&s.q_full, 0, abort);
-            if (!ok) fail(abort, status);
+            if (!ok) fail(abort, status, 1, 0, 0);
             const uint32_t qa = tc::smem_u32(s.q);
             for (int j = 0; ok && j <= nblk; ++j) {
                 if (j < nblk) {
                     const int st = j & 1;
                     const uint32_t ph = (j >> 1) & 1;
-                    if (!tc::mbar_wait(&s.kv_full[st], ph, abort) || !tc::mbar_wait(&s.s_free[st], ph ^ 1, abort)) {
-                        fail(abort, status);
-                        break;
-                    }
+                    if (!tc::mbar_wait(&s.kv_full[st], ph, abort)) { fail(abort, status, 1, j, 2); break; }
+                    if (!tc::mbar_wait(&s.s_free[st], ph ^ 1, abort)) { fail(abort, status, 1, j, 3); break; }
                     tc::tc_fence_after();
                     const uint32_t ka = tc::smem_u32(s.k[st]);
                     const uint32_t sd = tmem + 128 + st * 128;
@@ -156,7 +154,7 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
                 }
                 if (j >= 1) {
                     const int jj = j - 1, pb = jj & 1;
-                    if (!tc::mbar_wait(&s.p_full[pb], (jj >> 1) & 1, abort)) { fail(abort, status); break; }
+                    if (!tc::mbar_wait(&s.p_full[pb], (jj >> 1) & 1, abort)) { fail(abort, status, 1, jj, 4); break; }
                     tc::tc_fence_after();
                     const uint32_t pa = tc::smem_u32(s.p[pb][0]);
                     const uint32_t va = tc::smem_u32(s.v[pb][0]);
@@ -188,7 +186,13 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
             const int sb = j & 1;
             int j0, rs, re;
             blk.get(j, &j0, &rs, &re);
-            if (!tc::mbar_wait(&s.s_full[sb], (j >> 1) & 1, abort)) { fail(abort, status); ok = false; break; }
+            // tcgen05.ld/st are warp-collective: every decision that guards them is
+            // taken by the whole warp (__all_sync / __any_sync)
+            if (!__all_sync(0xffffffffu, tc::mbar_wait(&s.s_full[sb], (j >> 1) & 1, abort))) {
+                fail(abort, status, 2, j, 5);
+                ok = false;
+                break;
+            }
             tc::tc_fence_after();
             float sv[KBLK];
 #pragma unroll
@@ -222,36 +226,40 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
             }
             const float m_new = fmaxf(m_used, mx);
             // the P buffer of this block is free once PV[j-2] has completed
-            if (j >= 2 && !tc::mbar_wait(&s.pv_done[sb], ((j - 2) >> 1) & 1, abort)) {
-                fail(abort, status);
+            if (j >= 2 && !__all_sync(0xffffffffu, tc::mbar_wait(&s.pv_done[sb], ((j - 2) >> 1) & 1, abort))) {
+                fail(abort, status, 2, j, 6);
                 ok = false;
                 break;
             }
+            // rows whose running max grew by more than 2^8 move to the new max; their O row
+            // (PV[0..j-1]) is scaled by f in TMEM, the other rows of the warp by 1
+            float f = 1.f;
+            bool scale_o = false;
             if (m_new > m_used + RESCALE_LOG2) {
                 if (m_used != -INFINITY) {
-                    const float f = exp2f(m_used - m_new);
+                    f = exp2f(m_used - m_new);
                     l *= f;
-                    if (j >= 1) {
-                        // O holds PV[0..j-1]: wait for the last one, then rescale this row
-                        if (!tc::mbar_wait(&s.pv_done[(j - 1) & 1], ((j - 1) >> 1) & 1, abort)) {
-                            fail(abort, status);
-                            ok = false;
-                            break;
-                        }
-                        tc::tc_fence_after();
-#pragma unroll 1
-                        for (int c = 0; c < DV / 32; ++c) {
-                            uint32_t rr[32];
-                            tc::tmem_ld32(tmem + lane_base + c * 32, rr);
-                            tc::tmem_wait_ld();
-#pragma unroll
-                            for (int e = 0; e < 32; ++e) rr[e] = __float_as_uint(__uint_as_float(rr[e]) * f);
-                            tc::tmem_st32(tmem + lane_base + c * 32, rr);
-                        }
-                        tc::tmem_wait_st();
-                    }
+                    scale_o = j >= 1;
                 }
                 m_used = m_new;
+            }
+            if (__any_sync(0xffffffffu, scale_o)) {
+                if (!__all_sync(0xffffffffu, tc::mbar_wait(&s.pv_done[(j - 1) & 1], ((j - 1) >> 1) & 1, abort))) {
+                    fail(abort, status, 2, j, 7);
+                    ok = false;
+                    break;
+                }
+                tc::tc_fence_after();
+#pragma unroll 1
+                for (int c = 0; c < DV / 32; ++c) {
+                    uint32_t rr[32];
+                    tc::tmem_ld32(tmem + lane_base + c * 32, rr);
+                    tc::tmem_wait_ld();
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) rr[e] = __float_as_uint(__uint_as_float(rr[e]) * f);
+                    tc::tmem_st32(tmem + lane_base + c * 32, rr);
+                }
+                tc::tmem_wait_st();
             }
             const float mu = m_used == -INFINITY ? 0.f : m_used;
             uint8_t* prow = s.p[sb][0];
@@ -275,7 +283,7 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
             tc::tc_fence_before();
             tc::mbar_arrive(&s.p_full[sb]);
         }
-        if (ok && tc::mbar_wait(&s.o_done, 0, abort)) {
+        if (ok && __all_sync(0xffffffffu, tc::mbar_wait(&s.o_done, 0, abort))) {
             tc::tc_fence_after();
             const float inv = l > 0.f ? 1.f / l : 0.f;
             f16* orow = O + ((long long)b * Tp + i) * ((long long)H * DV) + h * DV;
@@ -297,7 +305,7 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
                 }
             }
         } else if (ok) {
-            fail(abort, status);
+            fail(abort, status, 2, nblk, 8);
         }
     }
     tc::tc_fence_before();

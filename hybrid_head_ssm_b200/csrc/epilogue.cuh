@@ -24,7 +24,7 @@ struct EpiArgs {
     int M, N;              // GEMM output extent
     int B, Tu, Tp, n_meta; // sequences, user tokens, layer rows per sequence, meta rows
     // EPI_INPROJ
-    T* P;                  // [B*T', ldP] projection (Q | (K V slots unused) | x | z | dt_low | B | C)
+    T* P;                  // [B*T', ldP] projection (Q | (K V slots unused) | x | z | B | C | dt_low)
     long long ldP;
     T* k_out;              // producer: K after RoPE [B, G, kcap, dh] (NULL: consumer)
     T* v_out;              // producer: V [B, G, kcap, dv]

@@ -2,83 +2,143 @@
 // RMSNorm of each branch over its full width, beta1 / beta2 scaling and average:
 //     Y = y_pre * SiLU(z),  U = (beta1 * g_a * O / rms(O) + beta2 * g_s * Y / rms(Y)) / 2
 // ("Hymba Guide", Parallel Hybrid-Head Layer Formulation: both families feed one
-// output projection; the normalise-scale-average form is the reading used here for
-// how they are combined). One block per row; the row is staged in shared memory so
-// HBM is read once and U written once.
+// output projection; normalise-scale-average is the reading used for how they are
+// combined). HBM-bound: per (row, channel) it reads O, y_pre and z and writes U once.
+//
+// 128 threads per row, two rows per 256-thread block; each thread keeps its share of
+// the row in registers between the two passes (sums of squares, then the output), and
+// moves 8 elements per 16-byte access.
 #include "kernels.h"
 
 namespace hymba {
 
 namespace {
 
-__device__ __forceinline__ float block_sum(float v, float* red) {
+constexpr int TPR = 128;                // threads per row
+constexpr int RPB = 2;                  // rows per block
+constexpr int VMAX = 4;                 // 8-element vectors per thread and array (d_inner <= 4096)
+
+template <typename I>
+__device__ __forceinline__ void load8(const I* p, float* v) {
+    if constexpr (sizeof(I) == 2) {
+        const uint4 u = *reinterpret_cast<const uint4*>(p);
+        const I* h = reinterpret_cast<const I*>(&u);
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    if (lane == 0) red[warp] = v;
-    __syncthreads();
-    float s = 0.f;
-    const int nw = blockDim.x >> 5;
-    for (int w = 0; w < nw; ++w) s += red[w];
-    __syncthreads();
-    return s;
+        for (int i = 0; i < 8; ++i) v[i] = to_f(h[i]);
+    } else {
+        const float4 a = *reinterpret_cast<const float4*>(p);
+        const float4 b = *reinterpret_cast<const float4*>(p + 4);
+        v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+        v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+    }
+}
+
+template <typename T>
+__device__ __forceinline__ void store8(T* p, const float* v) {
+    if constexpr (sizeof(T) == 2) {
+        uint4 u;
+        u.x = pack2<T>(v[0], v[1]);
+        u.y = pack2<T>(v[2], v[3]);
+        u.z = pack2<T>(v[4], v[5]);
+        u.w = pack2<T>(v[6], v[7]);
+        *reinterpret_cast<uint4*>(p) = u;
+    } else {
+        *reinterpret_cast<float4*>(p) = make_float4(v[0], v[1], v[2], v[3]);
+        *reinterpret_cast<float4*>(p + 4) = make_float4(v[4], v[5], v[6], v[7]);
+    }
+}
+
+__device__ __forceinline__ void load8f(const float* p, float* v) {
+    const float4 a = *reinterpret_cast<const float4*>(p);
+    const float4 b = *reinterpret_cast<const float4*>(p + 4);
+    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+    v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
 }
 
 template <typename I, typename T>
-__global__ void __launch_bounds__(256)
-fuse_kernel(const I* __restrict__ O, const I* __restrict__ ypre, const I* __restrict__ P,
-            long long ldP, int col_z, const float* __restrict__ g_attn,
-            const float* __restrict__ g_ssm, const float* __restrict__ beta1,
-            const float* __restrict__ beta2, T* __restrict__ U, int di, float eps, int* len_inc) {
-    extern __shared__ float sm[];
-    float* so = sm;
-    float* sy = sm + di;
-    __shared__ float red[32];
-    const long long row = blockIdx.x;
+__global__ void __launch_bounds__(TPR * RPB)
+fuse_kernel(const I* __restrict__ O, const I* __restrict__ ypre, const I* __restrict__ P, long long ldP, int col_z,
+            const float* __restrict__ g_attn, const float* __restrict__ g_ssm, const float* __restrict__ beta1,
+            const float* __restrict__ beta2, T* __restrict__ U, int rows, int di, float eps, int* len_inc) {
+    __shared__ float red[RPB][TPR / 32][2];
+    const int sub = threadIdx.x / TPR, t = threadIdx.x % TPR;
+    const long long row = (long long)blockIdx.x * RPB + sub;
+    const bool live = row < rows;
+    const int nvec = di / 8;
+    float o[VMAX][8], y[VMAX][8];
     float ss_o = 0.f, ss_y = 0.f;
-    for (int c = threadIdx.x; c < di; c += blockDim.x) {
-        const float o = to_f(O[row * di + c]);
-        const float z = to_f(P[row * ldP + col_z + c]);
-        const float y = to_f(ypre[row * di + c]) * silu_f(z);
-        so[c] = o;
-        sy[c] = y;
-        ss_o = fmaf(o, o, ss_o);
-        ss_y = fmaf(y, y, ss_y);
+#pragma unroll
+    for (int k = 0; k < VMAX; ++k) {
+        const int vi = t + k * TPR;
+        if (live && vi < nvec) {
+            const int c = vi * 8;
+            float z[8];
+            load8<I>(O + row * di + c, o[k]);
+            load8<I>(ypre + row * di + c, y[k]);
+            load8<I>(P + row * ldP + col_z + c, z);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                y[k][i] *= z[i] / (1.0f + __expf(-z[i]));
+                ss_o = fmaf(o[k][i], o[k][i], ss_o);
+                ss_y = fmaf(y[k][i], y[k][i], ss_y);
+            }
+        }
     }
-    ss_o = block_sum(ss_o, red);
-    ss_y = block_sum(ss_y, red);
-    const float ro = 1.0f / sqrtf(ss_o / di + eps);
-    const float ry = 1.0f / sqrtf(ss_y / di + eps);
-    for (int c = threadIdx.x; c < di; c += blockDim.x) {
-        const float u = 0.5f * (beta1[c] * g_attn[c] * so[c] * ro + beta2[c] * g_ssm[c] * sy[c] * ry);
-        U[row * di + c] = from_f<T>(u);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+        ss_o += __shfl_xor_sync(0xffffffffu, ss_o, off);
+        ss_y += __shfl_xor_sync(0xffffffffu, ss_y, off);
     }
-    if (len_inc && threadIdx.x == 0) len_inc[row] += 1;
+    if ((t & 31) == 0) {
+        red[sub][t >> 5][0] = ss_o;
+        red[sub][t >> 5][1] = ss_y;
+    }
+    __syncthreads();
+    ss_o = 0.f;
+    ss_y = 0.f;
+#pragma unroll
+    for (int w = 0; w < TPR / 32; ++w) {
+        ss_o += red[sub][w][0];
+        ss_y += red[sub][w][1];
+    }
+    const float ro = 0.5f / sqrtf(ss_o / di + eps);
+    const float ry = 0.5f / sqrtf(ss_y / di + eps);
+#pragma unroll
+    for (int k = 0; k < VMAX; ++k) {
+        const int vi = t + k * TPR;
+        if (live && vi < nvec) {
+            const int c = vi * 8;
+            float ga[8], gs[8], b1[8], b2[8], u[8];
+            load8f(g_attn + c, ga);
+            load8f(g_ssm + c, gs);
+            load8f(beta1 + c, b1);
+            load8f(beta2 + c, b2);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) u[i] = b1[i] * ga[i] * o[k][i] * ro + b2[i] * gs[i] * y[k][i] * ry;
+            store8<T>(U + row * di + c, u);
+        }
+    }
+    if (len_inc && live && t == 0) len_inc[row] += 1;
 }
 
 }  // namespace
 
 template <typename I, typename T>
 int launch_fuse(const Ctx& ctx, const I* O, const I* ypre, const I* P, long long ldP, int col_z,
-                const float* g_attn, const float* g_ssm, const float* beta1, const float* beta2,
-                T* U, int rows, int di, float eps, int* len_inc) {
+                const float* g_attn, const float* g_ssm, const float* beta1, const float* beta2, T* U, int rows,
+                int di, float eps, int* len_inc) {
     if (rows <= 0) return HYMBA_OK;
-    const size_t smem = (size_t)2 * di * sizeof(float);
+    if (di % 8 || di > VMAX * 8 * TPR || col_z % 8 || ldP % 8) return HYMBA_ERR_UNSUPPORTED;
     auto kern = fuse_kernel<I, T>;
-    if (smem > 48 * 1024) {
-        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
-            return HYMBA_ERR_CUDA;
-    }
-    HYMBA_LAUNCH(ctx, "fuse", kern, rows, 256, smem, O, ypre, P, ldP, col_z, g_attn, g_ssm, beta1,
-                 beta2, U, di, eps, len_inc);
+    HYMBA_LAUNCH(ctx, "fuse", kern, ceil_div(rows, RPB), TPR * RPB, 0, O, ypre, P, ldP, col_z, g_attn, g_ssm,
+                 beta1, beta2, U, rows, di, eps, len_inc);
     return HYMBA_OK;
 }
 
-template int launch_fuse<float, float>(const Ctx&, const float*, const float*, const float*, long long,
-                                       int, const float*, const float*, const float*, const float*,
-                                       float*, int, int, float, int*);
-template int launch_fuse<f16, bf16>(const Ctx&, const f16*, const f16*, const f16*, long long, int,
-                                    const float*, const float*, const float*, const float*, bf16*, int,
-                                    int, float, int*);
+template int launch_fuse<float, float>(const Ctx&, const float*, const float*, const float*, long long, int,
+                                       const float*, const float*, const float*, const float*, float*, int, int,
+                                       float, int*);
+template int launch_fuse<f16, bf16>(const Ctx&, const f16*, const f16*, const f16*, long long, int, const float*,
+                                    const float*, const float*, const float*, bf16*, int, int, float, int*);
 
 }  // namespace hymba

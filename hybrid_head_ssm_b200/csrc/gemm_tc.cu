@@ -87,9 +87,9 @@ struct GemmSmem {
     int abort;
 };
 
-__device__ __forceinline__ void fail(volatile int* abort, int* status) {
+__device__ __forceinline__ void fail(volatile int* abort, int* status, int role, int step, int bar) {
     *abort = 1;
-    set_status(status, HYMBA_ERR_DEVICE_TIMEOUT);
+    tc::record_timeout(status, role, step, bar);
 }
 
 template <typename TA, typename TO, int BN>
@@ -141,7 +141,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
                 for (int kb = 0; kb < nk; ++kb, ++it) {
                     const int st = it % STAGES;
                     const uint32_t ph = (it / STAGES) & 1;
-                    if (!tc::mbar_wait(&s.empty[st], ph ^ 1, abort)) { fail(abort, status); break; }
+                    if (!tc::mbar_wait(&s.empty[st], ph ^ 1, abort)) { fail(abort, status, 0, kb, 1); break; }
                     tc::mbar_arrive_expect_tx(&s.full[st], (BM + BN) * BK * 2);
                     tc::tma_load_2d(s.a[st], &tmA, &s.full[st], kb * BK, m_blk * BM);
                     tc::tma_load_2d(s.b[st], &tmB, &s.full[st], kb * BK, n_blk * BN);
@@ -162,14 +162,14 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
             for (int tile = blockIdx.x; tile < num_tiles && !*abort; tile += gridDim.x, ++tcount) {
                 const int buf = tcount & 1;
                 const uint32_t tph = (tcount >> 1) & 1;
-                if (!tc::mbar_wait(&s.tempty[buf], tph ^ 1, abort)) { fail(abort, status); break; }
+                if (!tc::mbar_wait(&s.tempty[buf], tph ^ 1, abort)) { fail(abort, status, 1, tcount, 4); break; }
                 tc::tc_fence_after();
                 const uint32_t d = tmem + buf * BN;
                 bool ok = true;
                 for (int kb = 0; kb < nk; ++kb, ++it) {
                     const int st = it % STAGES;
                     const uint32_t ph = (it / STAGES) & 1;
-                    if (!tc::mbar_wait(&s.full[st], ph, abort)) { fail(abort, status); ok = false; break; }
+                    if (!tc::mbar_wait(&s.full[st], ph, abort)) { fail(abort, status, 1, kb, 2); ok = false; break; }
                     tc::tc_fence_after();
                     const uint32_t a0 = tc::smem_u32(s.a[st]), b0 = tc::smem_u32(s.b[st]);
 #pragma unroll
@@ -193,7 +193,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
         for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++tcount) {
             const int buf = tcount & 1;
             const uint32_t tph = (tcount >> 1) & 1;
-            if (!tc::mbar_wait(&s.tfull[buf], tph, abort)) { fail(abort, status); break; }
+            // tcgen05.ld is warp-collective: the whole warp decides together
+            if (!__all_sync(0xffffffffu, tc::mbar_wait(&s.tfull[buf], tph, abort))) { fail(abort, status, 2, tcount, 3); break; }
             tc::tc_fence_after();
             const int m_blk = tile % num_m, n_blk = tile / num_m;
             const int row = m_blk * BM + q * 32 + lane;

@@ -3,6 +3,8 @@
 // runs in the kernels of this library; this file only queues them on the caller's
 // stream.
 #include <algorithm>
+#include <cstdio>
+#include <cstdlib>
 #include <atomic>
 #include <cstring>
 #include <type_traits>
@@ -16,7 +18,9 @@ namespace hymba {
 // ---------------------------------------------------------------------------
 // device status word (one per device that loads the library)
 // ---------------------------------------------------------------------------
-__device__ int g_status_word;
+// [0]: status code; [1..7]: where the first timed-out wait gave up (flag, block
+// x, y, z, role, step, barrier), for diagnosis.
+__device__ int g_status_word[8];
 
 static std::mutex g_mu;
 static int* g_status_ptr[64];
@@ -43,6 +47,8 @@ static int current_ctx(cudaStream_t stream, Ctx* ctx) {
     return HYMBA_OK;
 }
 
+int launch_context(cudaStream_t stream, Ctx* ctx) { return current_ctx(stream, ctx); }
+
 // ---------------------------------------------------------------------------
 // tracing and launch counting
 // ---------------------------------------------------------------------------
@@ -66,8 +72,28 @@ void trace_before(const Ctx& ctx) {
     cudaEventRecord(g_trace[slot].a, ctx.stream);
 }
 
+// HYMBA_SYNC_DEBUG=1: synchronise after every launch and log it to stderr (a
+// debugging aid: it serialises the host with the device).
+static int sync_debug() {
+    static int v = -1;
+    if (v < 0) {
+        const char* e = getenv("HYMBA_SYNC_DEBUG");
+        v = (e && e[0] == '1') ? 1 : 0;
+    }
+    return v;
+}
+
 bool trace_after(const Ctx& ctx, const char* name) {
     g_launches.fetch_add(1, std::memory_order_relaxed);
+    if (sync_debug()) {
+        fprintf(stderr, "[hymba] launched %s\n", name);
+        fflush(stderr);
+        const cudaError_t e2 = cudaStreamSynchronize(ctx.stream);
+        int st = 0;
+        cudaMemcpy(&st, ctx.status, sizeof(int), cudaMemcpyDeviceToHost);
+        fprintf(stderr, "[hymba] finished %s: %s, status %d\n", name, cudaGetErrorString(e2), st);
+        fflush(stderr);
+    }
     const cudaError_t err = cudaGetLastError();
     if (t_trace_slot >= 0) {
         g_trace[t_trace_slot].name = name;
@@ -104,10 +130,10 @@ static Cols columns(const hymba_layer_cfg* c) {
     const int kv = c->is_kv_producer ? c->n_kv_heads * (c->head_dim + c->v_head_dim) : 0;
     k.x = q + kv;
     k.z = k.x + c->d_inner;
-    k.dtl = k.z + c->d_inner;
-    k.Bc = k.dtl + c->dt_rank;
+    k.Bc = k.z + c->d_inner;
     k.Cc = k.Bc + c->d_state;
-    k.n_in = k.Cc + c->d_state;
+    k.dtl = k.Cc + c->d_state;
+    k.n_in = k.dtl + c->dt_rank;
     return k;
 }
 
@@ -497,6 +523,19 @@ int hymba_get_device_status(void* stream) {
     const int zero = 0;
     if (cudaMemcpy(ctx.status, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess) return HYMBA_ERR_CUDA;
     return v;
+}
+
+int hymba_get_device_diag(int32_t* out, int n) {
+    if (!out || n < 7) return HYMBA_ERR_INVALID_ARG;
+    if (cudaDeviceSynchronize() != cudaSuccess) return HYMBA_ERR_CUDA;
+    Ctx ctx;
+    if (current_ctx(nullptr, &ctx)) return HYMBA_ERR_CUDA;
+    int v[7] = {0};
+    if (cudaMemcpy(v, ctx.status + 1, sizeof(v), cudaMemcpyDeviceToHost) != cudaSuccess) return HYMBA_ERR_CUDA;
+    const int zero[7] = {0};
+    if (cudaMemcpy(ctx.status + 1, zero, sizeof(zero), cudaMemcpyHostToDevice) != cudaSuccess) return HYMBA_ERR_CUDA;
+    for (int i = 0; i < 7; ++i) out[i] = v[i];
+    return HYMBA_OK;
 }
 
 const char* hymba_strerror(int code) {

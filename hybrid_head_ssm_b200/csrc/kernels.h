@@ -5,6 +5,9 @@
 
 namespace hymba {
 
+// Launch context (stream, status word, SM count) of the current device.
+int launch_context(cudaStream_t stream, Ctx* ctx);
+
 // C = A B^T on CUDA cores (fp32 accumulate); A [M, K] (row stride lda), Bw [N, K]
 // (row stride ldb); the result goes through epi_run64.
 template <typename TA, typename TO>

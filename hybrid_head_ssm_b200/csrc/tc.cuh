@@ -62,9 +62,23 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
     return ok != 0;
 }
 
-// Cycles after which a wait gives up (about 1 s at the B200's clocks): a wait this
+// Cycles after which a wait gives up (about 0.1 s at the B200's clocks): a wait this
 // long means a protocol error, and the kernel exits instead of hanging the GPU.
-constexpr long long kWaitLimitCycles = 2000000000LL;
+constexpr long long kWaitLimitCycles = 200000000LL;
+
+// Record a timed-out wait: the status code, and (first one only) where it happened.
+__device__ __forceinline__ void record_timeout(int* status, int role, int step, int bar) {
+    if (!status) return;
+    atomicCAS(status, 0, HYMBA_ERR_DEVICE_TIMEOUT);
+    if (atomicCAS(status + 1, 0, 1) == 0) {
+        status[2] = blockIdx.x;
+        status[3] = blockIdx.y;
+        status[4] = blockIdx.z;
+        status[5] = role;
+        status[6] = step;
+        status[7] = bar;
+    }
+}
 
 // Bounded wait on an mbarrier phase. Returns false on timeout or when another role
 // of the block already aborted (*abort != 0).

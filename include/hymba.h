@@ -16,7 +16,7 @@
  *   a few global layers, KV shared by pairs of layers.
  *
  * Per layer and sequence, with X^ = [meta; x] (T' = n_meta + T rows):
- *   [Q K V x z dt_low B C] = X^ W_in^T                 one fused projection
+ *   [Q K V x z B C dt_low] = X^ W_in^T                 one fused projection
  *   Q, K <- RoPE (rotate-half, base rope_base), position of row i is i
  *   O     = GQA softmax attention, key j visible to query i iff j <= i and
  *           (j < n_meta or i - j < window); window <= 0 means global
@@ -105,8 +105,8 @@ typedef struct hymba_layer_cfg {
 
 /* Weights of one layer (device pointers, caller-owned, read only). Big matrices
  * use the [out, in] convention. n_in = H*dh + (producer ? G*(dh+dv) : 0)
- * + 2*d_inner + dt_rank + 2*d_state, rows in the order Q | K | V | x | z |
- * dt_low | B | C. */
+ * + 2*d_inner + 2*d_state + dt_rank, rows in the order Q | K | V | x | z | B | C |
+ * dt_low (B and C first so that their columns start on 16-byte boundaries). */
 typedef struct hymba_layer_weights {
     const void*  w_in;        /* [n_in, d_model]        dtype */
     const void*  w_dt;        /* [d_inner, dt_rank]     dtype */
@@ -225,9 +225,16 @@ uint64_t hymba_ssm_state_bytes(int n_layers, int channels, int d_state, int batc
  * HYMBA_ERR_CUDA if the synchronisation itself failed. */
 int hymba_get_device_status(void* stream);
 
+/* Where the first bounded device wait that ran out gave up (after a call reported
+ * HYMBA_ERR_DEVICE_TIMEOUT): out[0] 1 if a record exists, out[1..3] the block index
+ * (x, y, z), out[4] the role (0 TMA producer, 1 MMA issuer, 2 epilogue/softmax), out[5]
+ * the step (k-block or key block), out[6] the barrier. Synchronises the device and
+ * clears the record. Requires n >= 7. */
+int hymba_get_device_diag(int32_t* out, int n);
+
 /* Layout of the workspace of one call, for callers that inspect the stage outputs
  * after a prefill (tests do): out[0] total bytes, out[1] byte offset of the
- * projection P [rows, ld_p] dtype (columns Q | (K V, unused) | x | z | dt_low | B | C),
+ * projection P [rows, ld_p] dtype (columns Q | (K V, unused) | x | z | B | C | dt_low),
  * out[2] ld_p in elements, out[3] offset of Delta [rows, d_inner] fp32, out[4] of the
  * attention output O [rows, n_q_heads*v_head_dim] dtype, out[5] of y_pre = C.h + D xc
  * [rows, d_inner] dtype (before the SiLU(z) gate), out[6] of the fused U [rows,

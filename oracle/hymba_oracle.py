@@ -33,7 +33,7 @@ Readings taken where the pages are silent (each is listed in the design doc):
   width, scaled per channel by beta1 / beta2, and the two are averaged before
   W_o. The [Hymba Guide] formula concatenates instead; averaging needs equal
   widths, so the V head dim is d_inner / n_q_heads.
-* One input projection yields [Q | K | V | x | z | dt_low | B | C] in that order.
+* One input projection yields [Q | K | V | x | z | B | C | dt_low] in that order.
   A consumer (KV-sharing secondary) layer has no K, V rows.
 * RoPE is rotate-half with theta_i = base^(-2i/head_dim); meta tokens take
   positions 0..m-1 and user token t takes m + t; K is kept after RoPE.
@@ -205,8 +205,8 @@ def split_projection(cfg, p: np.ndarray) -> Dict[str, np.ndarray]:
     widths = [("q", H * dh)]
     if cfg.is_kv_producer:
         widths += [("k", G * dh), ("v", G * dv)]
-    widths += [("x", cfg.d_inner), ("z", cfg.d_inner), ("dtl", cfg.dt_rank),
-               ("B", cfg.d_state), ("C", cfg.d_state)]
+    widths += [("x", cfg.d_inner), ("z", cfg.d_inner), ("B", cfg.d_state), ("C", cfg.d_state),
+               ("dtl", cfg.dt_rank)]
     out, c = {}, 0
     for name, wd in widths:
         out[name] = p[:, c:c + wd]

@@ -46,7 +46,7 @@ class LayerCfg:
 
     @property
     def n_in(self) -> int:
-        """Width of the fused input projection: [Q | K | V | x | z | dt_low | B | C]."""
+        """Width of the fused input projection: [Q | K | V | x | z | B | C | dt_low]."""
         kv = self.n_kv_heads * (self.head_dim + self.v_head_dim) if self.is_kv_producer else 0
         return (self.n_q_heads * self.head_dim + kv + 2 * self.d_inner
                 + self.dt_rank + 2 * self.d_state)
@@ -122,11 +122,12 @@ def layer_weights(cfg: LayerCfg, seed: int) -> Dict[str, np.ndarray]:
     """
     d, di, N, r = cfg.d_model, cfg.d_inner, cfg.d_state, cfg.dt_rank
     H, G, dh, dv = cfg.n_q_heads, cfg.n_kv_heads, cfg.head_dim, cfg.v_head_dim
-    blocks = [("q", H * dh), ("k", G * dh), ("v", G * dv), ("x", di), ("z", di),
-              ("dtl", r), ("B", N), ("C", N)]
+    # row blocks of w_in in projection order; each block draws from its own stream
+    blocks = [("q", H * dh, 0), ("k", G * dh, 1), ("v", G * dv, 2), ("x", di, 3), ("z", di, 4),
+              ("B", N, 6), ("C", N, 7), ("dtl", r, 5)]
     rows = []
-    for i, (name, width) in enumerate(blocks):
-        blk = _normal(_rng(seed, 1, i), (width, d), 1.0 / d)
+    for name, width, tag in blocks:
+        blk = _normal(_rng(seed, 1, tag), (width, d), 1.0 / d)
         if name in ("k", "v") and not cfg.is_kv_producer:
             continue
         rows.append(blk)

@@ -34,7 +34,8 @@ def _run_prefill(cfg, w, x, *, kv_from=None, cache_cap=0, flags=0, state=True):
     ws.fill_(0xFF)  # garbage: every stage must write what it later reads
     rt.prefill(layer, xd, T, kv, yd, ws, st, flags, kv_struct_override=kvs)
     torch.cuda.synchronize()
-    assert hy.hymba_get_device_status(None) == 0
+    status = hy.hymba_get_device_status(None)
+    assert status == 0, (status, hy.device_diag())
     lay = hy.workspace_layout(layer.c, B, T, hy.HYMBA_MODE_PREFILL)
     return dict(y=yd, kv=kv, st=st, ws=ws, lay=lay, layer=layer)
 
@@ -55,8 +56,14 @@ def _check_stages(cfg, r, ref, B, Tp):
     delta = to_np(_ws_view(ws, lay["delta"], (B, Tp, di), torch.float32))
     o = to_np(_ws_view(ws, lay["O"], (B, Tp, H * dv), mdt))
     u = to_np(_ws_view(ws, lay["U"], (B, Tp, di), rt.act_dtype(cfg)))
+    ypre = to_np(_ws_view(ws, lay["ypre"], (B, Tp, di), mdt))
+    P = to_np(_ws_view(ws, lay["P"], (B, Tp, lay["ldP"]), mdt))
+    zc = cfg.n_q_heads * cfg.head_dim + (cfg.n_kv_heads * (cfg.head_dim + cfg.v_head_dim) if cfg.is_kv_producer else 0) + di
+    z = P[:, :, zc:zc + di]
     tol = dict(max_abs=1e-4 if cfg.dtype == 0 else 6e-2, rel_l2=5e-3)
     assert_close(delta, ref["delta"], cfg, "Delta", max_abs=tol["max_abs"])
+    assert_close(ypre * oracle.silu(z), ref["y_ssm"], cfg, "gated SSM output", max_abs=1e-4 if cfg.dtype == 0 else 2.5e-1,
+                 rel_l2=5e-3)
     assert_close(o, ref["o_attn"], cfg, "attention output", **tol)
     assert_close(u, ref["u"], cfg, "fused U", max_abs=2e-4 if cfg.dtype == 0 else 1.5e-1, rel_l2=5e-3)
 
