@@ -31,6 +31,7 @@ HYMBA_ERR_KV_INCOMPATIBLE = -4
 HYMBA_ERR_CUDA = -5
 HYMBA_ERR_DEVICE_TIMEOUT = -6
 HYMBA_ERR_DEVICE_RANGE = -7
+HYMBA_ERR_SCRATCH_LIMIT = -8
 
 HYMBA_F32 = 0
 HYMBA_BF16 = 1
@@ -88,6 +89,8 @@ _sig = {
     "hymba_trace_enable": (ctypes.c_int, [ctypes.c_int]),
     "hymba_trace_collect": (ctypes.c_int, [_P(ctypes.c_char_p), _P(ctypes.c_float), ctypes.c_int]),
     "hymba_launch_count": (ctypes.c_uint64, []),
+    "hymba_attn_decode_static": (ctypes.c_int, [_P(hymba_layer_cfg), _vp, ctypes.c_int64, _P(hymba_kv), _vp,
+                                                ctypes.c_int, _vp]),
 }
 EXPORTS = tuple(_sig)
 

@@ -62,6 +62,7 @@ extern "C" {
 #define HYMBA_ERR_CUDA               (-5)  /* a CUDA call or launch failed */
 #define HYMBA_ERR_DEVICE_TIMEOUT     (-6)  /* a bounded device wait ran out (status word) */
 #define HYMBA_ERR_DEVICE_RANGE       (-7)  /* a device-side range check failed (status word) */
+#define HYMBA_ERR_SCRATCH_LIMIT      (-8)  /* request larger than hymba_attn_decode_static's fixed scratch */
 
 /* dtypes: a layer is HYMBA_F32 or HYMBA_BF16; the K/V buffers of a bf16 layer hold
  * HYMBA_F16 (same width as bf16, finer mantissa; see hymba_kv) */
@@ -219,6 +220,33 @@ uint64_t hymba_kv_bytes(int n_attn_layers, int n_kv_heads, int head_dim, int v_h
  * n_layers * channels * d_state * batch * dtype_bytes. */
 uint64_t hymba_ssm_state_bytes(int n_layers, int channels, int d_state, int batch,
                                int dtype_bytes);
+
+/* Decode attention that allocates nothing and takes no workspace. The pages have no
+ * counterpart: this entry point exists for callers that cannot call cudaMalloc or
+ * hand the library a scratch buffer, for example a decode loop running inside
+ * another runtime that owns every device allocation through its own pool, or a
+ * latency-critical path where an allocation (which can synchronise the device) is
+ * not allowed.
+ *
+ * It computes the attention step of hymba_mixer_decode on its own: for every sequence
+ * b and query head, softmax attention of q[b] over the positions the decode cache
+ * holds, the newest being the query's own (position len[b] - 1), limited to the meta
+ * block plus the layer's window (or everything, for a global layer), with GQA.
+ *   q:  device [B, n_q_heads * head_dim], row stride ldq elements, after RoPE; element
+ *       type of the cache (fp16 for bf16 layers, fp32 for fp32 layers).
+ *   kv: a decode cache (k_cache, v_cache, len) as filled by prefill/decode.
+ *   o:  device [B, n_q_heads * v_head_dim], same element type.
+ * The partial results of its key splits live in one file-scope device array of 8 MiB
+ * (every GPU that loads the library holds it until the process exits). Requests with
+ * B * n_q_heads * ceil(cache_cap / 256) * (v_head_dim + 2) * 4 bytes above that return
+ * HYMBA_ERR_SCRATCH_LIMIT and queue no work. The first call on a device looks up the
+ * array's device address (with that device current); make that first call before any
+ * stream capture. All calls share the one array, and every call writes each partial
+ * before reading it, so nothing needs clearing between calls; but calls whose kernels
+ * overlap on the GPU (other streams, other host threads) race on it, so the caller
+ * must order them. */
+int hymba_attn_decode_static(const hymba_layer_cfg* cfg, const void* q, int64_t ldq, const hymba_kv* kv,
+                             void* o, int B, void* stream);
 
 /* Synchronises `stream`, then returns and clears the status word of the current
  * device: HYMBA_OK, HYMBA_ERR_DEVICE_TIMEOUT or HYMBA_ERR_DEVICE_RANGE; or

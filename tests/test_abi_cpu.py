@@ -135,6 +135,6 @@ def test_kv_share_rules(hy):
 
 
 def test_strerror_covers_codes(hy):
-    for code in range(0, -8, -1):
+    for code in range(0, -9, -1):
         assert hy.hymba_strerror(code).decode() != "unknown status"
     assert hy.hymba_strerror(-99).decode() == "unknown status"
