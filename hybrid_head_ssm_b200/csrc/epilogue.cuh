@@ -44,6 +44,11 @@ struct EpiArgs {
     const T* res_x;
     const void* res_meta;  // [n_meta, N] of the layer's weight type
     int res_meta_bf16;     // 1: res_meta is bf16; 0: it has type T
+    // in-projection GEMMs that also cover the meta rows: GEMM rows [0, meta_pad) are
+    // meta rows (valid below meta_M, written for every sequence), the rest follow
+    // row_mode after subtracting meta_pad
+    int meta_pad;
+    int meta_M;
 };
 
 // RoPE on one 64-wide head run: pairs (i, i+32) rotated by (cos, sin).
@@ -68,7 +73,16 @@ __device__ __forceinline__ float2 rope_cs_at(int p, int i, int dh, float base) {
 
 template <typename T>
 __device__ void epi_run64(const EpiArgs<T>& e, int r, int c0, float* v) {
-    if (r >= e.M || c0 >= e.N) return;
+    int mode = e.row_mode;
+    if (e.meta_pad > 0) {
+        if (r < e.meta_pad) {
+            if (r >= e.meta_M) return;
+            mode = ROWS_META;
+        } else {
+            r -= e.meta_pad;
+        }
+    }
+    if ((mode != ROWS_META && r >= e.M) || c0 >= e.N) return;
     const int n = min(64, e.N - c0);
     if (e.kind == EPI_DELTA) {
         float* dst = e.delta + (long long)r * e.N + c0;
@@ -78,11 +92,11 @@ __device__ void epi_run64(const EpiArgs<T>& e, int r, int c0, float* v) {
             for (int j = 0; j < 64; j += 4) {
                 const float4 bb = *reinterpret_cast<const float4*>(bias + j);
                 *reinterpret_cast<float4*>(dst + j) =
-                    make_float4(softplus_f(v[j] + bb.x), softplus_f(v[j + 1] + bb.y), softplus_f(v[j + 2] + bb.z),
-                                softplus_f(v[j + 3] + bb.w));
+                    make_float4(softplus_fast(v[j] + bb.x), softplus_fast(v[j + 1] + bb.y), softplus_fast(v[j + 2] + bb.z),
+                                softplus_fast(v[j + 3] + bb.w));
             }
         } else {
-            for (int j = 0; j < n; ++j) dst[j] = softplus_f(v[j] + bias[j]);
+            for (int j = 0; j < n; ++j) dst[j] = softplus_fast(v[j] + bias[j]);
         }
         return;
     }
@@ -110,9 +124,9 @@ __device__ void epi_run64(const EpiArgs<T>& e, int r, int c0, float* v) {
     }
     // EPI_INPROJ
     int b0, b1, t;
-    if (e.row_mode == ROWS_DIRECT) { b0 = r / e.Tp; b1 = b0 + 1; t = r % e.Tp; }
-    else if (e.row_mode == ROWS_META) { b0 = 0; b1 = e.B; t = r; }
-    else if (e.row_mode == ROWS_USER) { b0 = r / e.Tu; b1 = b0 + 1; t = e.n_meta + r % e.Tu; }
+    if (mode == ROWS_DIRECT) { b0 = r / e.Tp; b1 = b0 + 1; t = r % e.Tp; }
+    else if (mode == ROWS_META) { b0 = 0; b1 = e.B; t = r; }
+    else if (mode == ROWS_USER) { b0 = r / e.Tu; b1 = b0 + 1; t = e.n_meta + r % e.Tu; }
     else {
         b0 = r; b1 = r + 1; t = e.pos[r] + e.pos_offset;
         if (t < 0) return;  // no position to write; the decode attention reports the range error
@@ -121,7 +135,7 @@ __device__ void epi_run64(const EpiArgs<T>& e, int r, int c0, float* v) {
     const int kw = e.k_out ? e.G * e.dh : 0;
     const int vw = e.k_out ? e.G * e.dv : 0;
     if (c0 < qw + kw) {
-        if (e.row_mode == ROWS_DECODE) {
+        if (mode == ROWS_DECODE) {
             float2 cs[32];
 #pragma unroll 4
             for (int i = 0; i < 32; ++i) cs[i] = rope_cs_at(t, i, 64, e.rope_base);
@@ -134,16 +148,16 @@ __device__ void epi_run64(const EpiArgs<T>& e, int r, int c0, float* v) {
         if (c0 >= qw && c0 < qw + kw) {
             int g = (c0 - qw) / e.dh;
             int slot = t;
-            if (e.row_mode == ROWS_DECODE && t >= e.n_meta) slot = e.n_meta + (t - e.n_meta) % e.n_meta_ring;
+            if (mode == ROWS_DECODE && t >= e.n_meta) slot = e.n_meta + (t - e.n_meta) % e.n_meta_ring;
             store_run<T>(e.k_out + (((long long)b * e.G + g) * e.kcap + slot) * e.dh, v, 64);
         } else if (c0 >= qw + kw && c0 < qw + kw + vw) {
             int cv = c0 - qw - kw;
             int g = cv / e.dv, off = cv % e.dv;
             int slot = t;
-            if (e.row_mode == ROWS_DECODE && t >= e.n_meta) slot = e.n_meta + (t - e.n_meta) % e.n_meta_ring;
+            if (mode == ROWS_DECODE && t >= e.n_meta) slot = e.n_meta + (t - e.n_meta) % e.n_meta_ring;
             store_run<T>(e.v_out + (((long long)b * e.G + g) * e.kcap + slot) * e.dv + off, v, 64);
         } else {
-            long long row = e.row_mode == ROWS_DECODE ? b : (long long)b * e.Tp + t;
+            long long row = mode == ROWS_DECODE ? b : (long long)b * e.Tp + t;
             store_run<T>(e.P + row * e.ldP + c0, v, n);
         }
     }

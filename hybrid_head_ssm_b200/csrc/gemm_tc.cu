@@ -94,15 +94,18 @@ __device__ __forceinline__ void fail(volatile int* abort, int* status, int role,
 
 template <typename TA, typename TO, int BN>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
-gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, int M, int N,
-               int K, EpiArgs<TO> e, int* status) {
+gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+               const __grid_constant__ CUtensorMap tmA0, int M0, int M, int N, int K, EpiArgs<TO> e, int* status) {
     extern __shared__ uint8_t smem_raw[];
     GemmSmem<BN>& s = *reinterpret_cast<GemmSmem<BN>*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                         ~static_cast<uintptr_t>(1023));
     constexpr bool kBF16 = sizeof(TA) == 2 && std::is_same<TA, bf16>::value;
     constexpr uint32_t IDESC = tc::idesc_f16(kBF16, BM, BN);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int num_m = (M + BM - 1) / BM, num_n = (N + BN - 1) / BN;
+    // M-blocks [0, num_m0) come from the optional second operand A0 (M0 rows), the
+    // rest from A (M rows); the epilogue tells them apart by row index (EpiArgs::meta_pad)
+    const int num_m0 = (M0 + BM - 1) / BM;
+    const int num_m = num_m0 + (M + BM - 1) / BM, num_n = (N + BN - 1) / BN;
     const int num_tiles = num_m * num_n, nk = (K + BK - 1) / BK;
 
     if (threadIdx.x == 0) {
@@ -119,6 +122,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
         tc::fence_mbar_init();
         tc::prefetch_tmap(&tmA);
         tc::prefetch_tmap(&tmB);
+        if (M0 > 0) tc::prefetch_tmap(&tmA0);
     }
     if (warp == 1) {
         tc::tmem_alloc(&s.tmem_base, 2 * BN);
@@ -143,7 +147,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
                     const uint32_t ph = (it / STAGES) & 1;
                     if (!tc::mbar_wait(&s.empty[st], ph ^ 1, abort)) { fail(abort, status, 0, kb, 1); break; }
                     tc::mbar_arrive_expect_tx(&s.full[st], (BM + BN) * BK * 2);
-                    tc::tma_load_2d(s.a[st], &tmA, &s.full[st], kb * BK, m_blk * BM);
+                    if (m_blk < num_m0) tc::tma_load_2d(s.a[st], &tmA0, &s.full[st], kb * BK, m_blk * BM);
+                    else tc::tma_load_2d(s.a[st], &tmA, &s.full[st], kb * BK, (m_blk - num_m0) * BM);
                     tc::tma_load_2d(s.b[st], &tmB, &s.full[st], kb * BK, n_blk * BN);
                     issued_phase[st] = (int)ph;
                 }
@@ -227,11 +232,16 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
 
 template <typename TA, typename TO, int BN>
 int launch_bn(const Ctx& ctx, const char* name, const TA* A, long long lda, const TA* Bw, long long ldb, int M,
-              int N, int K, const EpiArgs<TO>& e) {
+              int N, int K, const EpiArgs<TO>& e, const TA* A0, int M0) {
     constexpr bool kBF16 = std::is_same<TA, bf16>::value;
-    CUtensorMap ta, tb;
+    CUtensorMap ta, tb, ta0;
     if (!tc::make_tmap_2d(&ta, A, kBF16, M, K, lda, BM)) return HYMBA_ERR_UNSUPPORTED;
     if (!tc::make_tmap_2d(&tb, Bw, kBF16, N, K, ldb, BN)) return HYMBA_ERR_UNSUPPORTED;
+    if (M0 > 0) {
+        if (!tc::make_tmap_2d(&ta0, A0, kBF16, M0, K, lda, BM)) return HYMBA_ERR_UNSUPPORTED;
+    } else {
+        ta0 = ta;
+    }
     const size_t smem = sizeof(GemmSmem<BN>) + 1024;
     auto kern = gemm_tc_kernel<TA, TO, BN>;
     static bool attr_set = false;
@@ -240,9 +250,12 @@ int launch_bn(const Ctx& ctx, const char* name, const TA* A, long long lda, cons
             return HYMBA_ERR_CUDA;
         attr_set = true;
     }
-    const int tiles = ((M + BM - 1) / BM) * ((N + BN - 1) / BN);
+    const int tiles = ((M0 + BM - 1) / BM + (M + BM - 1) / BM) * ((N + BN - 1) / BN);
     const int grid = tiles < ctx.sm_count ? tiles : ctx.sm_count;
-    HYMBA_LAUNCH(ctx, name, kern, grid, NUM_THREADS, smem, ta, tb, M, N, K, e, ctx.status);
+    EpiArgs<TO> e2 = e;
+    e2.meta_pad = ((M0 + BM - 1) / BM) * BM;
+    e2.meta_M = M0;
+    HYMBA_LAUNCH(ctx, name, kern, grid, NUM_THREADS, smem, ta, tb, ta0, M0, M, N, K, e2, ctx.status);
     return HYMBA_OK;
 }
 
@@ -264,18 +277,19 @@ static int pick_bn(int M, int N, int sms) {
 
 template <typename TA, typename TO>
 int launch_gemm_tc(const Ctx& ctx, const char* name, const TA* A, long long lda, const TA* Bw, long long ldb,
-                   int M, int N, int K, const EpiArgs<TO>& e) {
+                   int M, int N, int K, const EpiArgs<TO>& e, const TA* A0, int M0) {
     if (M <= 0 || N <= 0) return HYMBA_OK;
-    switch (pick_bn(M, N, ctx.sm_count > 0 ? ctx.sm_count : 148)) {
-        case 256: return launch_bn<TA, TO, 256>(ctx, name, A, lda, Bw, ldb, M, N, K, e);
-        case 128: return launch_bn<TA, TO, 128>(ctx, name, A, lda, Bw, ldb, M, N, K, e);
-        default: return launch_bn<TA, TO, 64>(ctx, name, A, lda, Bw, ldb, M, N, K, e);
+    if (M0 > 0 && (!A0 || ((uintptr_t)A0 & 15))) return HYMBA_ERR_INVALID_ARG;
+    switch (pick_bn(M + M0, N, ctx.sm_count > 0 ? ctx.sm_count : 148)) {
+        case 256: return launch_bn<TA, TO, 256>(ctx, name, A, lda, Bw, ldb, M, N, K, e, A0, M0);
+        case 128: return launch_bn<TA, TO, 128>(ctx, name, A, lda, Bw, ldb, M, N, K, e, A0, M0);
+        default: return launch_bn<TA, TO, 64>(ctx, name, A, lda, Bw, ldb, M, N, K, e, A0, M0);
     }
 }
 
 #define INST(TA, TO)                                                                                        \
     template int launch_gemm_tc<TA, TO>(const Ctx&, const char*, const TA*, long long, const TA*, long long, \
-                                        int, int, int, const EpiArgs<TO>&);
+                                        int, int, int, const EpiArgs<TO>&, const TA*, int);
 INST(bf16, f16)
 INST(f16, f16)
 INST(bf16, bf16)

@@ -263,12 +263,28 @@ static int prefill_impl(const Ctx& ctx, const hymba_layer_cfg* c, const hymba_la
         ep.row_mode = ROWS_DIRECT; ep.M = (int)rows;
         if ((rc = gemm<T, I>(ctx, "gemm_in_proj", x, d, W_in, d, (int)rows, k.n_in, d, ep))) return rc;
     } else {
-        if (m > 0) {
-            ep.row_mode = ROWS_META; ep.M = m;
-            if ((rc = gemm<T, I>(ctx, "gemm_in_proj_meta", static_cast<const T*>(w->meta), d, W_in, d, m, k.n_in, d, ep))) return rc;
+        bool fused = false;
+#ifdef HYMBA_WITH_TCGEN05
+        if constexpr (sizeof(T) == 2) {
+            if (((uintptr_t)x & 15) == 0 && ((uintptr_t)W_in & 15) == 0 && ((uintptr_t)w->meta & 15) == 0 &&
+                d % 8 == 0) {
+            // one launch: meta rows (projected once, written for every sequence) + user rows
+            ep.row_mode = ROWS_USER; ep.M = B * T_;
+            if ((rc = launch_gemm_tc<T, I>(ctx, "gemm_in_proj", x, d, W_in, d, B * T_, k.n_in, d, ep,
+                                           static_cast<const T*>(w->meta), m)))
+                return rc;
+            fused = true;
+            }
         }
-        ep.row_mode = ROWS_USER; ep.M = B * T_;
-        if ((rc = gemm<T, I>(ctx, "gemm_in_proj", x, d, W_in, d, B * T_, k.n_in, d, ep))) return rc;
+#endif
+        if (!fused) {
+            if (m > 0) {
+                ep.row_mode = ROWS_META; ep.M = m;
+                if ((rc = gemm<T, I>(ctx, "gemm_in_proj_meta", static_cast<const T*>(w->meta), d, W_in, d, m, k.n_in, d, ep))) return rc;
+            }
+            ep.row_mode = ROWS_USER; ep.M = B * T_;
+            if ((rc = gemm<T, I>(ctx, "gemm_in_proj", x, d, W_in, d, B * T_, k.n_in, d, ep))) return rc;
+        }
     }
     // 2. Delta = softplus(dt_low W_dt^T + b_dt) ------------------------------------
     if ((rc = launch_pad_copy<T, I>(ctx, static_cast<const T*>(w->w_dt), di, c->dt_rank, wdt, pl.rpad))) return rc;
@@ -548,6 +564,7 @@ const char* hymba_strerror(int code) {
         case HYMBA_ERR_CUDA: return "CUDA error";
         case HYMBA_ERR_DEVICE_TIMEOUT: return "bounded device wait timed out";
         case HYMBA_ERR_DEVICE_RANGE: return "device range check failed";
+        case HYMBA_ERR_SCRATCH_LIMIT: return "request exceeds the fixed scratch of hymba_attn_decode_static";
         default: return "unknown status";
     }
 }

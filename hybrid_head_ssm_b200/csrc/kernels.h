@@ -15,10 +15,12 @@ int launch_gemm_simt(const Ctx& ctx, const char* name, const TA* A, long long ld
                      int M, int N, int K, const EpiArgs<TO>& e);
 
 // C = A B^T on the tcgen05 tensor cores (bf16 or fp16 in, fp32 accumulate in TMEM).
-// Requirements: lda, ldb multiples of 8 elements, A and Bw 16-byte aligned.
+// Requirements: lda, ldb multiples of 8 elements, A and Bw 16-byte aligned. With A0
+// (M0 > 0 rows, same lda) the launch also covers A0's rows, handed to the epilogue
+// as meta rows (in-projection only): one launch for the meta and the user rows.
 template <typename TA, typename TO>
 int launch_gemm_tc(const Ctx& ctx, const char* name, const TA* A, long long lda, const TA* Bw, long long ldb,
-                   int M, int N, int K, const EpiArgs<TO>& e);
+                   int M, int N, int K, const EpiArgs<TO>& e, const TA* A0 = nullptr, int M0 = 0);
 
 // Causal GQA attention over the meta prefix + window, CUDA cores.
 template <typename T>
