@@ -73,16 +73,16 @@ __device__ __forceinline__ float2 rope_cs_at(int p, int i, int dh, float base) {
 
 template <typename T>
 __device__ void epi_run64(const EpiArgs<T>& e, int r, int c0, float* v) {
-    int mode = e.row_mode;
+    int mode = e.row_mode, M = e.M;
     if (e.meta_pad > 0) {
         if (r < e.meta_pad) {
-            if (r >= e.meta_M) return;
             mode = ROWS_META;
+            M = e.meta_M;
         } else {
             r -= e.meta_pad;
         }
     }
-    if ((mode != ROWS_META && r >= e.M) || c0 >= e.N) return;
+    if (r >= M || c0 >= e.N) return;
     const int n = min(64, e.N - c0);
     if (e.kind == EPI_DELTA) {
         float* dst = e.delta + (long long)r * e.N + c0;
