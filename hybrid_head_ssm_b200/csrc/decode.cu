@@ -27,15 +27,36 @@ __device__ __forceinline__ bool decode_span(int p, int n_meta, int window, int r
     return p >= 0 && span <= ring;
 }
 
+// 8 consecutive elements of a K or V row as fp32 (one or two 16-byte loads).
+template <typename T>
+__device__ __forceinline__ void load_row8(const T* p, float* v) {
+    if constexpr (sizeof(T) == 2) {
+        const uint4 u = __ldg(reinterpret_cast<const uint4*>(p));
+        const T* h = reinterpret_cast<const T*>(&u);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) v[i] = to_f(h[i]);
+    } else {
+        const float4 a = __ldg(reinterpret_cast<const float4*>(p));
+        const float4 b = __ldg(reinterpret_cast<const float4*>(p + 4));
+        v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+        v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+    }
+}
+
+constexpr int KGROUPS = 8;  // key groups of the PV phase (128 threads = 8 groups x 16 pieces of 8)
+
 template <typename T, int DV>
 __global__ void __launch_bounds__(128)
 attn_decode_kernel(const T* __restrict__ P, long long ldP, const T* __restrict__ k_cache,
                    const T* __restrict__ v_cache, int cap, const int* __restrict__ len,
                    int pos_offset, float* __restrict__ part, int n_split, int H, int G,
                    int n_meta, int window, int* status) {
-    __shared__ float qs[MAX_R][DH];
+    static_assert(DV == 16 * 8, "PV phase covers a V row with 16 pieces of 8");
+    __shared__ __align__(16) float qs[MAX_R][DH];
     __shared__ float ps[MAX_R][MAX_CHUNK];
+    __shared__ int slots[MAX_CHUNK];
     __shared__ float stat[MAX_R][2];
+    __shared__ __align__(16) float red[KGROUPS][MAX_R][DV];
     const int s = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
     const int R = H / G;
     const int tid = threadIdx.x;
@@ -54,22 +75,35 @@ attn_decode_kernel(const T* __restrict__ P, long long ldP, const T* __restrict__
         const int r = i / DH, e = i % DH;
         qs[r][e] = to_f(P[(long long)b * ldP + (g * R + r) * DH + e]) * (LOG2E * 0.125f);
     }
-    __syncthreads();
-    // scores: one key per thread
     for (int kk = tid; kk < nk; kk += blockDim.x) {
         const int idx = k0 + kk;
         const int j = idx < meta_n ? idx : lo + (idx - meta_n);
-        const int slot = j < n_meta ? j : n_meta + (j - n_meta) % ring;
-        const T* kr = k_cache + (kvbase + slot) * DH;
-        float kv[DH];
+        slots[kk] = j < n_meta ? j : n_meta + (j - n_meta) % ring;
+    }
+    __syncthreads();
+    // scores: one key per thread, its K row in 16-byte pieces, q broadcast from smem
+    for (int kk = tid; kk < nk; kk += blockDim.x) {
+        const T* kr = k_cache + (kvbase + slots[kk]) * DH;
+        float acc[MAX_R];
 #pragma unroll
-        for (int e = 0; e < DH; ++e) kv[e] = to_f(kr[e]);
-        for (int r = 0; r < R; ++r) {
-            float acc = 0.f;
+        for (int r = 0; r < MAX_R; ++r) acc[r] = 0.f;
 #pragma unroll
-            for (int e = 0; e < DH; ++e) acc = fmaf(qs[r][e], kv[e], acc);
-            ps[r][kk] = acc;
+        for (int e = 0; e < DH; e += 8) {
+            float kv[8];
+            load_row8<T>(kr + e, kv);
+#pragma unroll
+            for (int r = 0; r < MAX_R; ++r) {
+                if (r < R) {
+                    const float4 qa = *reinterpret_cast<const float4*>(&qs[r][e]);
+                    const float4 qb = *reinterpret_cast<const float4*>(&qs[r][e + 4]);
+                    acc[r] = fmaf(qa.x, kv[0], acc[r]); acc[r] = fmaf(qa.y, kv[1], acc[r]);
+                    acc[r] = fmaf(qa.z, kv[2], acc[r]); acc[r] = fmaf(qa.w, kv[3], acc[r]);
+                    acc[r] = fmaf(qb.x, kv[4], acc[r]); acc[r] = fmaf(qb.y, kv[5], acc[r]);
+                    acc[r] = fmaf(qb.z, kv[6], acc[r]); acc[r] = fmaf(qb.w, kv[7], acc[r]);
+                }
+            }
         }
+        for (int r = 0; r < R; ++r) ps[r][kk] = acc[r];
     }
     __syncthreads();
     // per-head max and sum over this split's keys: warp w handles heads w, w+4, ...
@@ -90,22 +124,41 @@ attn_decode_kernel(const T* __restrict__ P, long long ldP, const T* __restrict__
         if (lane == 0) { stat[r][0] = mx; stat[r][1] = sum; }
     }
     __syncthreads();
-    // P V: thread e of the V row
-    for (int e = tid; e < DV; e += blockDim.x) {
-        float acc[MAX_R];
+    // P V: thread (key group kg, piece eb) adds keys kg, kg + 8, ... for V elements eb*8..+7
+    {
+        const int eb = tid % 16, kg = tid / 16;
+        float acc[MAX_R][8];
 #pragma unroll
-        for (int r = 0; r < MAX_R; ++r) acc[r] = 0.f;
-        for (int kk = 0; kk < nk; ++kk) {
-            const int idx = k0 + kk;
-            const int j = idx < meta_n ? idx : lo + (idx - meta_n);
-            const int slot = j < n_meta ? j : n_meta + (j - n_meta) % ring;
-            const float v = to_f(v_cache[(kvbase + slot) * DV + e]);
+        for (int r = 0; r < MAX_R; ++r)
 #pragma unroll
-            for (int r = 0; r < MAX_R; ++r)
-                if (r < R) acc[r] = fmaf(ps[r][kk], v, acc[r]);
+            for (int i = 0; i < 8; ++i) acc[r][i] = 0.f;
+        for (int kk = kg; kk < nk; kk += KGROUPS) {
+            float v[8];
+            load_row8<T>(v_cache + (kvbase + slots[kk]) * DV + eb * 8, v);
+#pragma unroll
+            for (int r = 0; r < MAX_R; ++r) {
+                if (r < R) {
+                    const float pr = ps[r][kk];
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) acc[r][i] = fmaf(pr, v[i], acc[r][i]);
+                }
+            }
         }
-        for (int r = 0; r < R; ++r)
-            part[(((long long)b * H + g * R + r) * n_split + s) * (DV + 2) + e] = acc[r];
+#pragma unroll
+        for (int r = 0; r < MAX_R; ++r) {
+            if (r < R) {
+                *reinterpret_cast<float4*>(&red[kg][r][eb * 8]) = make_float4(acc[r][0], acc[r][1], acc[r][2], acc[r][3]);
+                *reinterpret_cast<float4*>(&red[kg][r][eb * 8 + 4]) = make_float4(acc[r][4], acc[r][5], acc[r][6], acc[r][7]);
+            }
+        }
+    }
+    __syncthreads();
+    for (int i = tid; i < R * DV; i += blockDim.x) {
+        const int r = i / DV, e = i % DV;
+        float sum = 0.f;
+#pragma unroll
+        for (int k = 0; k < KGROUPS; ++k) sum += red[k][r][e];
+        part[(((long long)b * H + g * R + r) * n_split + s) * (DV + 2) + e] = sum;
     }
     if (tid < R) {
         float* st = part + (((long long)b * H + g * R + tid) * n_split + s) * (DV + 2) + DV;

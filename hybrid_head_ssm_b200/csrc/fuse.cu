@@ -5,18 +5,19 @@
 // output projection; normalise-scale-average is the reading used for how they are
 // combined). HBM-bound: per (row, channel) it reads O, y_pre and z and writes U once.
 //
-// 128 threads per row, two rows per 256-thread block; each thread keeps its share of
-// the row in registers between the two passes (sums of squares, then the output), and
-// moves 8 elements per 16-byte access.
+// One row per 256-thread block; each thread keeps its (at most two) 8-element pieces
+// of the row in registers between the two passes (sums of squares, then the output),
+// moving 8 elements per 16-byte access. Few registers per thread keep many rows in
+// flight per SM, which is what an HBM-bound row kernel needs.
 #include "kernels.h"
 
 namespace hymba {
 
 namespace {
 
-constexpr int TPR = 128;                // threads per row
-constexpr int RPB = 2;                  // rows per block
-constexpr int VMAX = 4;                 // 8-element vectors per thread and array (d_inner <= 4096)
+constexpr int TPR = 256;                // threads per row
+constexpr int RPB = 1;                  // rows per block
+constexpr int VMAX = 2;                 // 8-element vectors per thread and array (d_inner <= 4096)
 
 template <typename I>
 __device__ __forceinline__ void load8(const I* p, float* v) {
@@ -56,7 +57,7 @@ __device__ __forceinline__ void load8f(const float* p, float* v) {
 }
 
 template <typename I, typename T>
-__global__ void __launch_bounds__(TPR * RPB)
+__global__ void __launch_bounds__(TPR * RPB, 4)
 fuse_kernel(const I* __restrict__ O, const I* __restrict__ ypre, const I* __restrict__ P, long long ldP, int col_z,
             const float* __restrict__ g_attn, const float* __restrict__ g_ssm, const float* __restrict__ beta1,
             const float* __restrict__ beta2, T* __restrict__ U, int rows, int di, float eps, int* len_inc) {

@@ -5,15 +5,14 @@
 // with A = -exp(A_log) per (channel, state) and the state in fp32 registers.
 //
 // One block per (8-channel group, sequence), 64 threads; thread (c, p) owns states 2p
-// and 2p+1 of channel c and updates both with packed f32x2 arithmetic, so one
-// recurrence step is two MUFU exp2 plus a handful of FMA-pipe instructions per thread,
-// and the only serial dependency is one FMA per state. Time is walked in chunks of 64
-// rows: x, Delta, B and C of the next chunk are copied into shared memory with cp.async
-// while the current chunk is scanned; the conv and its SiLU are done once per
-// (row, channel) when a chunk is unpacked. The C_t . h_t sum over the 8 threads of a
-// channel is deferred: every 8 steps a transpose-reduce (4 + 2 + 1 shuffles) leaves
-// thread p with the output of step p, so the reduction is off the recurrence's
-// critical path.
+// and 2p+1 of channel c and updates both with packed f32x2 arithmetic, so a recurrence
+// step is two MUFU exp2 and a few FMA-pipe instructions per thread, and the only serial
+// dependency is one FMA per state. Time is walked in chunks of 64 rows, each thread
+// staging one row with cp.async while the previous chunk is scanned:
+//   unpack   thread t: conv + SiLU of row t for the 8 channels, Delta * xc, B/C pairs;
+//   scan     thread (c, p): 64 steps, its partial C.h sums written to shared memory;
+//   reduce   thread t: y of row t = the 8 partial sums + D xc, one 16-byte store.
+// The sum over the threads of a channel is thus never on the recurrence's path.
 #include "kernels.h"
 
 namespace hymba {
@@ -23,9 +22,11 @@ namespace {
 constexpr int CPB = 8;   // channels per block
 constexpr int TPC = 8;   // threads per channel (2 states each)
 constexpr int NTH = CPB * TPC;
-constexpr int TC = 64;   // rows per chunk
+constexpr int TC = 64;   // rows per chunk (= threads: one row each when staging)
 constexpr int KC = 4;    // conv taps
+constexpr int PSTR = TC + 4;  // padded row of the partial-sum buffer
 constexpr float LOG2E = 1.4426950408889634f;
+static_assert(TC == NTH, "staging maps one row per thread");
 
 __device__ __forceinline__ float2 mul2(float2 a, float2 b) {
     uint64_t r;
@@ -58,35 +59,38 @@ struct Raw {  // one chunk as copied from global memory
     alignas(16) T c[TC][16];
 };
 
-// Queue the cp.async copies of rows [t0, t0 + TC) of sequence b (rows past Tp repeat
-// the last row; their results are never stored).
+// Thread t queues the copies of row t0 + t of the sequence (rows past Tp repeat the
+// last row; their results are never stored and their Delta is zeroed when unpacked).
 template <typename T>
-__device__ __forceinline__ void stage(Raw<T>& r, const T* P, long long ldP, int col_x, int col_B, int col_C,
-                                      const float* delta, int di, int c0, long long row0, int t0, int Tp) {
-    constexpr int XV = CPB * (int)sizeof(T) / 16;  // 16-byte pieces per row of x
-    constexpr int BV = 16 * (int)sizeof(T) / 16;   // ... of B (and of C)
-    constexpr int DVp = CPB * 4 / 16;              // ... of Delta
-    constexpr int PER_ROW = XV + DVp + 2 * BV;
-    for (int i = threadIdx.x; i < TC * PER_ROW; i += NTH) {
-        const int tt = i / PER_ROW, k = i % PER_ROW;
-        const long long row = row0 + min(t0 + tt, Tp - 1);
-        const T* prow = P + row * ldP;
-        if (k < XV) {
-            cp_async16(reinterpret_cast<char*>(&r.x[tt][0]) + 16 * k,
-                       reinterpret_cast<const char*>(prow + col_x + c0) + 16 * k);
-        } else if (k < XV + DVp) {
-            const int q = k - XV;
-            cp_async16(reinterpret_cast<char*>(&r.d[tt][0]) + 16 * q,
-                       reinterpret_cast<const char*>(delta + row * di + c0) + 16 * q);
-        } else if (k < XV + DVp + BV) {
-            const int q = k - XV - DVp;
-            cp_async16(reinterpret_cast<char*>(&r.b[tt][0]) + 16 * q, reinterpret_cast<const char*>(prow + col_B) + 16 * q);
-        } else {
-            const int q = k - XV - DVp - BV;
-            cp_async16(reinterpret_cast<char*>(&r.c[tt][0]) + 16 * q, reinterpret_cast<const char*>(prow + col_C) + 16 * q);
-        }
+__device__ __forceinline__ void stage_row(Raw<T>& r, const T* P, long long ldP, int col_x, int col_B, int col_C,
+                                          const float* delta, int di, int c0, long long row0, int t0, int Tp) {
+    const int tt = threadIdx.x;
+    const long long row = row0 + min(t0 + tt, Tp - 1);
+    const T* prow = P + row * ldP;
+    constexpr int XV = CPB * (int)sizeof(T) / 16;
+    constexpr int BV = 16 * (int)sizeof(T) / 16;
+#pragma unroll
+    for (int k = 0; k < XV; ++k)
+        cp_async16(reinterpret_cast<char*>(&r.x[tt][0]) + 16 * k, reinterpret_cast<const char*>(prow + col_x + c0) + 16 * k);
+#pragma unroll
+    for (int k = 0; k < CPB * 4 / 16; ++k)
+        cp_async16(reinterpret_cast<char*>(&r.d[tt][0]) + 16 * k,
+                   reinterpret_cast<const char*>(delta + row * di + c0) + 16 * k);
+#pragma unroll
+    for (int k = 0; k < BV; ++k) {
+        cp_async16(reinterpret_cast<char*>(&r.b[tt][0]) + 16 * k, reinterpret_cast<const char*>(prow + col_B) + 16 * k);
+        cp_async16(reinterpret_cast<char*>(&r.c[tt][0]) + 16 * k, reinterpret_cast<const char*>(prow + col_C) + 16 * k);
     }
 }
+
+template <typename T>
+struct ScanSmem {
+    Raw<T> raw[2];
+    alignas(16) float2 dd[TC][CPB];            // (Delta, Delta * xc)
+    alignas(16) float4 bc[TC][TPC];            // (B_2p, B_2p+1, C_2p, C_2p+1)
+    alignas(16) float xd[TC][CPB];             // D * xc
+    alignas(16) float part[CPB][TPC][PSTR];    // partial C.h sums
+};
 
 template <typename T>
 __global__ void __launch_bounds__(NTH)
@@ -95,13 +99,16 @@ conv_scan_prefill_kernel(const T* __restrict__ P, long long ldP, int col_x, int 
                          const float* __restrict__ conv_b, const float* __restrict__ A_log,
                          const float* __restrict__ Dp, T* __restrict__ ypre, float* __restrict__ h_out,
                          float* __restrict__ conv_out, int Tp, int di) {
-    __shared__ Raw<T> raw[2];
-    __shared__ float2 dd[TC][CPB];   // (Delta, Delta * xc)
-    __shared__ float4 bc[TC][TPC];   // (B_2p, B_2p+1, C_2p, C_2p+1)
-    __shared__ float xd[TC][CPB];    // D * xc
-    __shared__ float ys[TC][CPB];
+    extern __shared__ __align__(16) uint8_t scan_smem[];
+    ScanSmem<T>& sm = *reinterpret_cast<ScanSmem<T>*>(scan_smem);
+    Raw<T>* raw = sm.raw;
+    float2 (*dd)[CPB] = sm.dd;
+    float4 (*bc)[TPC] = sm.bc;
+    float (*xd)[CPB] = sm.xd;
+    float (*part)[TPC][PSTR] = sm.part;
     __shared__ float halo[KC - 1][CPB];
     __shared__ float wconv[CPB][KC + 1];
+    __shared__ float dch[CPB];
 
     const int b = blockIdx.y, c0 = blockIdx.x * CPB;
     const int tid = threadIdx.x, cl = tid / TPC, p = tid % TPC, c = c0 + cl;
@@ -112,105 +119,100 @@ conv_scan_prefill_kernel(const T* __restrict__ P, long long ldP, int col_x, int 
     if (tid < CPB) {
         for (int k = 0; k < KC; ++k) wconv[tid][k] = conv_w[(long long)(c0 + tid) * KC + k];
         wconv[tid][KC] = conv_b[c0 + tid];
+        dch[tid] = Dp[c0 + tid];
     }
     float2 h = make_float2(0.f, 0.f);
     const int nchunk = (Tp + TC - 1) / TC;
 
-    stage<T>(raw[0], P, ldP, col_x, col_B, col_C, delta, di, c0, row0, 0, Tp);
+    stage_row<T>(raw[0], P, ldP, col_x, col_B, col_C, delta, di, c0, row0, 0, Tp);
     cp_async_commit();
     for (int k = 0; k < nchunk; ++k) {
         const int t0 = k * TC, nt = min(TC, Tp - t0);
-        if (k + 1 < nchunk)
-            stage<T>(raw[(k + 1) & 1], P, ldP, col_x, col_B, col_C, delta, di, c0, row0, t0 + TC, Tp);
+        if (k + 1 < nchunk) stage_row<T>(raw[(k + 1) & 1], P, ldP, col_x, col_B, col_C, delta, di, c0, row0, t0 + TC, Tp);
         cp_async_commit();
         cp_async_wait1();
-        __syncthreads();
-        Raw<T>& r = raw[k & 1];
-        // unpack: conv + SiLU per (row, channel), B/C to fp32 pairs
-        for (int i = tid; i < TC * CPB; i += NTH) {
-            const int tt = i / CPB, cc = i % CPB;
-            float acc = wconv[cc][KC];
+        __syncthreads();  // chunk k staged; previous chunk's reduce done
+        const Raw<T>& r = raw[k & 1];
+        {
+            // unpack row tid
+            const int tt = tid;
+            float xs[KC][CPB];
 #pragma unroll
             for (int q = 0; q < KC; ++q) {
                 const int src = tt - (KC - 1) + q;
-                const float xv = src >= 0 ? to_f(r.x[src][cc]) : halo[src + KC - 1][cc];
-                acc = fmaf(wconv[cc][q], xv, acc);
+#pragma unroll
+                for (int cc = 0; cc < CPB; ++cc) xs[q][cc] = src >= 0 ? to_f(r.x[src][cc]) : halo[src + KC - 1][cc];
             }
-            const float xc = silu_f(acc);
-            // rows past the end of the sequence get Delta = 0: exp2(0) = 1 and a zero
-            // input leave the state exactly as it is after the last row
-            const float d = tt < nt ? r.d[tt][cc] : 0.f;
-            dd[tt][cc] = make_float2(d, d * xc);
-            xd[tt][cc] = Dp[c0 + cc] * xc;
+#pragma unroll
+            for (int cc = 0; cc < CPB; ++cc) {
+                float acc = wconv[cc][KC];
+#pragma unroll
+                for (int q = 0; q < KC; ++q) acc = fmaf(wconv[cc][q], xs[q][cc], acc);
+                const float xc = acc / (1.0f + __expf(-acc));
+                // rows past the end of the sequence get Delta = 0: exp2(0) = 1 and a zero
+                // input leave the state exactly as it is after the last row
+                const float d = tt < nt ? r.d[tt][cc] : 0.f;
+                dd[tt][cc] = make_float2(d, d * xc);
+                xd[tt][cc] = dch[cc] * xc;
+            }
+#pragma unroll
+            for (int q = 0; q < TPC; ++q)
+                bc[tt][q] = make_float4(to_f(r.b[tt][2 * q]), to_f(r.b[tt][2 * q + 1]), to_f(r.c[tt][2 * q]),
+                                        to_f(r.c[tt][2 * q + 1]));
+            if (k + 1 == nchunk && conv_out && tt < KC) {
+                // conv state: the last KC inputs of the sequence, oldest first
+                const int src = nt - KC + tt;
+#pragma unroll
+                for (int cc = 0; cc < CPB; ++cc)
+                    conv_out[((long long)b * di + c0 + cc) * KC + tt] =
+                        src >= 0 ? to_f(r.x[src][cc]) : (src + KC - 1 >= 0 ? halo[src + KC - 1][cc] : 0.f);
+            }
         }
-        for (int i = tid; i < TC * TPC; i += NTH) {
-            const int tt = i / TPC, q = i % TPC;
-            bc[tt][q] = make_float4(to_f(r.b[tt][2 * q]), to_f(r.b[tt][2 * q + 1]), to_f(r.c[tt][2 * q]),
-                                    to_f(r.c[tt][2 * q + 1]));
-        }
-        __syncthreads();
+        __syncthreads();  // unpacked; halo readers done
         if (k + 1 < nchunk && tid < (KC - 1) * CPB) {
             const int q = tid / CPB, cc = tid % CPB;
             halo[q][cc] = to_f(r.x[TC - (KC - 1) + q][cc]);
         }
-        if (k + 1 == nchunk && conv_out && tid < KC * CPB) {
-            // conv state: the last KC inputs of the sequence, oldest first
-            const int q = tid / CPB, cc = tid % CPB;
-            const int src = nt - KC + q;
-            conv_out[((long long)b * di + c0 + cc) * KC + q] =
-                src >= 0 ? to_f(r.x[src][cc]) : (src + KC - 1 >= 0 ? halo[src + KC - 1][cc] : 0.f);
-        }
-        // scan: 8 steps at a time, then the deferred C.h reduction
+        // scan the chunk: partial sums of 4 steps go to shared memory together
 #pragma unroll 1
-        for (int t8 = 0; t8 < TC; t8 += 8) {
-            float yp[8];
+        for (int t4 = 0; t4 < TC; t4 += 16) {
+            float yp[16];
 #pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                const float2 dv = dd[t8 + u][cl];
-                const float4 q = bc[t8 + u][p];
+            for (int u = 0; u < 16; ++u) {
+                const float2 dv = dd[t4 + u][cl];
+                const float4 q = bc[t4 + u][p];
                 const float2 arg = mul2(make_float2(dv.x, dv.x), A2);
                 const float2 a = make_float2(fast_exp2(arg.x), fast_exp2(arg.y));
                 h = fma2(a, h, mul2(make_float2(dv.y, dv.y), make_float2(q.x, q.y)));
                 const float2 ch = mul2(make_float2(q.z, q.w), h);
                 yp[u] = ch.x + ch.y;
             }
-            // transpose-reduce over the 8 threads of the channel: thread p ends with step p
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const bool hi = p & 4;
-                const float send = hi ? yp[i] : yp[i + 4];
-                const float keep = hi ? yp[i + 4] : yp[i];
-                yp[i] = keep + __shfl_xor_sync(0xffffffffu, send, 4);
-            }
-#pragma unroll
-            for (int i = 0; i < 2; ++i) {
-                const bool hi = p & 2;
-                const float send = hi ? yp[i] : yp[i + 2];
-                const float keep = hi ? yp[i + 2] : yp[i];
-                yp[i] = keep + __shfl_xor_sync(0xffffffffu, send, 2);
-            }
-            {
-                const bool hi = p & 1;
-                const float send = hi ? yp[0] : yp[1];
-                const float keep = hi ? yp[1] : yp[0];
-                yp[0] = keep + __shfl_xor_sync(0xffffffffu, send, 1);
-            }
-            ys[t8 + p][cl] = yp[0] + xd[t8 + p][cl];
+            for (int u = 0; u < 16; u += 4)
+                *reinterpret_cast<float4*>(&part[cl][p][t4 + u]) = make_float4(yp[u], yp[u + 1], yp[u + 2], yp[u + 3]);
         }
-        __syncthreads();
-        // store the chunk: one row of 8 channels per thread
-        for (int tt = tid; tt < nt; tt += NTH) {
+        __syncthreads();  // partial sums complete
+        if (tid < nt) {
+            const int tt = tid;
+            float y[CPB];
+#pragma unroll
+            for (int cc = 0; cc < CPB; ++cc) {
+                float s = xd[tt][cc];
+#pragma unroll
+                for (int q = 0; q < TPC; ++q) s += part[cc][q][tt];
+                y[cc] = s;
+            }
             T* dst = ypre + (row0 + t0 + tt) * di + c0;
             if constexpr (sizeof(T) == 2) {
                 uint4 v;
-                v.x = pack2<T>(ys[tt][0], ys[tt][1]);
-                v.y = pack2<T>(ys[tt][2], ys[tt][3]);
-                v.z = pack2<T>(ys[tt][4], ys[tt][5]);
-                v.w = pack2<T>(ys[tt][6], ys[tt][7]);
+                v.x = pack2<T>(y[0], y[1]);
+                v.y = pack2<T>(y[2], y[3]);
+                v.z = pack2<T>(y[4], y[5]);
+                v.w = pack2<T>(y[6], y[7]);
                 *reinterpret_cast<uint4*>(dst) = v;
             } else {
-                *reinterpret_cast<float4*>(dst) = make_float4(ys[tt][0], ys[tt][1], ys[tt][2], ys[tt][3]);
-                *reinterpret_cast<float4*>(dst + 4) = make_float4(ys[tt][4], ys[tt][5], ys[tt][6], ys[tt][7]);
+                *reinterpret_cast<float4*>(dst) = make_float4(y[0], y[1], y[2], y[3]);
+                *reinterpret_cast<float4*>(dst + 4) = make_float4(y[4], y[5], y[6], y[7]);
             }
         }
     }
@@ -230,8 +232,16 @@ int launch_conv_scan_prefill(const Ctx& ctx, const T* P, long long ldP, int col_
                              const float* D, T* ypre, float* h_out, float* conv_out, int B, int Tp, int di) {
     if (di % CPB || (col_x % 8) || (col_B % 8) || (col_C % 8) || (ldP % 8)) return HYMBA_ERR_UNSUPPORTED;
     dim3 grid(di / CPB, B);
-    HYMBA_LAUNCH(ctx, "conv_scan_prefill", conv_scan_prefill_kernel<T>, grid, NTH, 0, P, ldP, col_x, col_B, col_C,
-                 delta, conv_w, conv_b, A_log, D, ypre, h_out, conv_out, Tp, di);
+    const size_t smem = sizeof(ScanSmem<T>);
+    auto kern = conv_scan_prefill_kernel<T>;
+    static bool attr_set = false;
+    if (!attr_set) {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+            return HYMBA_ERR_CUDA;
+        attr_set = true;
+    }
+    HYMBA_LAUNCH(ctx, "conv_scan_prefill", kern, grid, NTH, smem, P, ldP, col_x, col_B, col_C, delta, conv_w, conv_b,
+                 A_log, D, ypre, h_out, conv_out, Tp, di);
     return HYMBA_OK;
 }
 
