@@ -141,5 +141,7 @@ template int launch_fuse<float, float>(const Ctx&, const float*, const float*, c
                                        float, int*);
 template int launch_fuse<f16, bf16>(const Ctx&, const f16*, const f16*, const f16*, long long, int, const float*,
                                     const float*, const float*, const float*, bf16*, int, int, float, int*);
+template int launch_fuse<f16, f16>(const Ctx&, const f16*, const f16*, const f16*, long long, int, const float*,
+                                   const float*, const float*, const float*, f16*, int, int, float, int*);
 
 }  // namespace hymba

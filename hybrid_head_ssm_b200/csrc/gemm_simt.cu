@@ -81,6 +81,7 @@ INST(bf16, f16)
 INST(f16, f16)
 INST(bf16, bf16)
 INST(bf16, float)
+INST(f16, float)
 #undef INST
 
 }  // namespace hymba

@@ -140,6 +140,7 @@ static Cols columns(const hymba_layer_cfg* c) {
 struct Plan {
     size_t total = 0;
     size_t rope = 0, P = 0, delta = 0, O = 0, ypre = 0, U = 0, wdt = 0, part = 0, xcv = 0;
+    size_t win16 = 0, meta16 = 0, wout16 = 0;
     long long ldP = 0;
     int rpad = 0, n_split = 1;
 };
@@ -168,7 +169,15 @@ static Plan plan(const hymba_layer_cfg* c, int B, int T, int mode) {
     p.ypre = take(&cur, rows * di * esz);
     p.U = take(&cur, rows * di * esz);
     p.wdt = take(&cur, (size_t)di * p.rpad * esz);
-    if (c->dtype == HYMBA_BF16) p.xcv = take(&cur, rows * c->d_model * 2);  // bf16 copy of fp32 input
+    if (c->dtype == HYMBA_BF16) {
+        p.xcv = take(&cur, rows * c->d_model * 2);  // 16-bit copy of an fp32 input
+        if (mode == HYMBA_MODE_PREFILL) {
+            // fp16 copies of the projection weights for fp32-stream calls
+            p.win16 = take(&cur, (size_t)k.n_in * c->d_model * 2);
+            p.meta16 = take(&cur, (size_t)c->n_meta * c->d_model * 2);
+            p.wout16 = take(&cur, (size_t)c->d_model * di * 2);
+        }
+    }
     if (mode == HYMBA_MODE_DECODE) {
         p.n_split = decode_splits(T);
         p.part = take(&cur, (size_t)B * c->n_q_heads * p.n_split * (c->v_head_dim + 2) * sizeof(float));
@@ -218,10 +227,17 @@ static EpiArgs<T> epi_base(int kind, int M, int N) {
 // (fp32, or fp16 for bf16 layers: the projection, K/V, attention output and y_pre are
 // held in fp16, which has the same width as bf16 and a finer mantissa).
 // TIO: type of x and y (T, or fp32 for a bf16 layer in a fp32 residual stream).
+// A bf16 layer in an fp32 residual stream takes the operands of its in- and
+// output projections in fp16: the stream and U are rounded to fp16 (8x finer than
+// bf16) and W_in, meta and W_out are converted per call (exact for all but the
+// tiniest weights). The stream's values at depth are several times larger than the
+// first layer's, and the attention scores they feed are correspondingly sharper.
 template <typename T, typename I, typename TIO>
 static int prefill_impl(const Ctx& ctx, const hymba_layer_cfg* c, const hymba_layer_weights* w,
                         const TIO* x_io, int B, int T_, int flags, TIO* y, hymba_kv* kv,
                         hymba_ssm_state* st, char* ws) {
+    constexpr bool kF16Ops = std::is_same<T, bf16>::value && std::is_same<TIO, float>::value;
+    using TA = typename std::conditional<kF16Ops, f16, T>::type;
     const Plan pl = plan(c, B, T_, HYMBA_MODE_PREFILL);
     const Cols k = columns(c);
     const int m = c->n_meta, Tp = m + T_, d = c->d_model, di = c->d_inner;
@@ -233,20 +249,30 @@ static int prefill_impl(const Ctx& ctx, const hymba_layer_cfg* c, const hymba_la
     float* delta = reinterpret_cast<float*>(ws + pl.delta);
     I* O = reinterpret_cast<I*>(ws + pl.O);
     I* ypre = reinterpret_cast<I*>(ws + pl.ypre);
-    T* U = reinterpret_cast<T*>(ws + pl.U);
+    TA* U = reinterpret_cast<TA*>(ws + pl.U);
     I* wdt = reinterpret_cast<I*>(ws + pl.wdt);
     I* k_seq = static_cast<I*>(kv->k_seq);
     I* v_seq = static_cast<I*>(kv->v_seq);
     int rc;
 
-    const T* x;
-    if constexpr (std::is_same<TIO, T>::value) {
-        x = x_io;
-    } else {
-        T* xc = reinterpret_cast<T*>(ws + pl.xcv);
+    const TA *x, *W_in, *meta, *W_out;
+    if constexpr (kF16Ops) {
+        TA* xc = reinterpret_cast<TA*>(ws + pl.xcv);
+        TA* wi = reinterpret_cast<TA*>(ws + pl.win16);
+        TA* mt = reinterpret_cast<TA*>(ws + pl.meta16);
+        TA* wo = reinterpret_cast<TA*>(ws + pl.wout16);
         const int xrows = B * (has_meta ? Tp : T_);
-        if ((rc = launch_pad_copy<TIO, T>(ctx, x_io, xrows, d, xc, d))) return rc;
-        x = xc;
+        if ((rc = launch_pad_copy<TIO, TA>(ctx, x_io, xrows, d, xc, d))) return rc;
+        if ((rc = launch_pad_copy<T, TA>(ctx, static_cast<const T*>(w->w_in), k.n_in, d, wi, d))) return rc;
+        if (m > 0 && !has_meta && (rc = launch_pad_copy<T, TA>(ctx, static_cast<const T*>(w->meta), m, d, mt, d)))
+            return rc;
+        if ((rc = launch_pad_copy<T, TA>(ctx, static_cast<const T*>(w->w_out), d, di, wo, di))) return rc;
+        x = xc; W_in = wi; meta = mt; W_out = wo;
+    } else {
+        x = x_io;
+        W_in = static_cast<const T*>(w->w_in);
+        meta = static_cast<const T*>(w->meta);
+        W_out = static_cast<const T*>(w->w_out);
     }
     if ((rc = launch_rope_table(ctx, rope, Tp, dh, c->rope_base))) return rc;
     // 1. fused input projection (+ RoPE, K/V scatter) ------------------------------
@@ -258,32 +284,30 @@ static int prefill_impl(const Ctx& ctx, const hymba_layer_cfg* c, const hymba_la
     ep.kcap = kv->seq_cap;
     ep.H = H; ep.G = G; ep.dh = dh; ep.dv = dv;
     ep.rope = rope;
-    const T* W_in = static_cast<const T*>(w->w_in);
     if (has_meta) {
         ep.row_mode = ROWS_DIRECT; ep.M = (int)rows;
-        if ((rc = gemm<T, I>(ctx, "gemm_in_proj", x, d, W_in, d, (int)rows, k.n_in, d, ep))) return rc;
+        if ((rc = gemm<TA, I>(ctx, "gemm_in_proj", x, d, W_in, d, (int)rows, k.n_in, d, ep))) return rc;
     } else {
         bool fused = false;
 #ifdef HYMBA_WITH_TCGEN05
-        if constexpr (sizeof(T) == 2) {
-            if (((uintptr_t)x & 15) == 0 && ((uintptr_t)W_in & 15) == 0 && ((uintptr_t)w->meta & 15) == 0 &&
+        if constexpr (sizeof(TA) == 2) {
+            if (((uintptr_t)x & 15) == 0 && ((uintptr_t)W_in & 15) == 0 && ((uintptr_t)meta & 15) == 0 &&
                 d % 8 == 0) {
-            // one launch: meta rows (projected once, written for every sequence) + user rows
-            ep.row_mode = ROWS_USER; ep.M = B * T_;
-            if ((rc = launch_gemm_tc<T, I>(ctx, "gemm_in_proj", x, d, W_in, d, B * T_, k.n_in, d, ep,
-                                           static_cast<const T*>(w->meta), m)))
-                return rc;
-            fused = true;
+                // one launch: meta rows (projected once, written for every sequence) + user rows
+                ep.row_mode = ROWS_USER; ep.M = B * T_;
+                if ((rc = launch_gemm_tc<TA, I>(ctx, "gemm_in_proj", x, d, W_in, d, B * T_, k.n_in, d, ep, meta, m)))
+                    return rc;
+                fused = true;
             }
         }
 #endif
         if (!fused) {
             if (m > 0) {
                 ep.row_mode = ROWS_META; ep.M = m;
-                if ((rc = gemm<T, I>(ctx, "gemm_in_proj_meta", static_cast<const T*>(w->meta), d, W_in, d, m, k.n_in, d, ep))) return rc;
+                if ((rc = gemm<TA, I>(ctx, "gemm_in_proj_meta", meta, d, W_in, d, m, k.n_in, d, ep))) return rc;
             }
             ep.row_mode = ROWS_USER; ep.M = B * T_;
-            if ((rc = gemm<T, I>(ctx, "gemm_in_proj", x, d, W_in, d, B * T_, k.n_in, d, ep))) return rc;
+            if ((rc = gemm<TA, I>(ctx, "gemm_in_proj", x, d, W_in, d, B * T_, k.n_in, d, ep))) return rc;
         }
     }
     // 2. Delta = softplus(dt_low W_dt^T + b_dt) ------------------------------------
@@ -300,8 +324,8 @@ static int prefill_impl(const Ctx& ctx, const hymba_layer_cfg* c, const hymba_la
                                           st ? st->conv : nullptr, B, Tp, di)))
         return rc;
     // 5. gate, norms, beta, average --------------------------------------------------
-    if ((rc = launch_fuse<I, T>(ctx, O, ypre, P, pl.ldP, k.z, w->norm_attn_w, w->norm_ssm_w, w->beta1,
-                                w->beta2, U, (int)rows, di, c->rms_eps, nullptr)))
+    if ((rc = launch_fuse<I, TA>(ctx, O, ypre, P, pl.ldP, k.z, w->norm_attn_w, w->norm_ssm_w, w->beta1,
+                                 w->beta2, U, (int)rows, di, c->rms_eps, nullptr)))
         return rc;
     // 6. output projection (+ residual) -------------------------------------------------
     EpiArgs<TIO> eo = epi_base<TIO>(EPI_OUT, (int)rows, d);
@@ -312,7 +336,7 @@ static int prefill_impl(const Ctx& ctx, const hymba_layer_cfg* c, const hymba_la
         eo.res_meta = w->meta;
         eo.res_meta_bf16 = std::is_same<T, bf16>::value;
     }
-    if ((rc = gemm<T, TIO>(ctx, "gemm_out_proj", U, di, static_cast<const T*>(w->w_out), di, (int)rows, d, di, eo))) return rc;
+    if ((rc = gemm<TA, TIO>(ctx, "gemm_out_proj", U, di, W_out, di, (int)rows, d, di, eo))) return rc;
     // 7. decode cache of a producer ------------------------------------------------------
     if (c->is_kv_producer && kv->k_cache) {
         if ((rc = launch_cache_fill<I>(ctx, k_seq, v_seq, kv->seq_cap, static_cast<I*>(kv->k_cache),

@@ -71,6 +71,7 @@ int launch_cache_fill(const Ctx& ctx, const T* k_seq, const T* v_seq, int seq_ca
 
 template int launch_pad_copy<float, float>(const Ctx&, const float*, int, int, float*, int);
 template int launch_pad_copy<float, bf16>(const Ctx&, const float*, int, int, bf16*, int);
+template int launch_pad_copy<float, f16>(const Ctx&, const float*, int, int, f16*, int);
 template int launch_pad_copy<bf16, f16>(const Ctx&, const bf16*, int, int, f16*, int);
 template int launch_cache_fill<float>(const Ctx&, const float*, const float*, int, float*, float*,
                                       int, int*, int, int, int, int, int, int);

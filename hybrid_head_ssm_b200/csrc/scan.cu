@@ -148,7 +148,7 @@ conv_scan_prefill_kernel(const T* __restrict__ P, long long ldP, int col_x, int 
                 float acc = wconv[cc][KC];
 #pragma unroll
                 for (int q = 0; q < KC; ++q) acc = fmaf(wconv[cc][q], xs[q][cc], acc);
-                const float xc = acc / (1.0f + __expf(-acc));
+                const float xc = __fdividef(acc, 1.0f + __expf(-acc));
                 // rows past the end of the sequence get Delta = 0: exp2(0) = 1 and a zero
                 // input leave the state exactly as it is after the last row
                 const float d = tt < nt ? r.d[tt][cc] : 0.f;
@@ -173,23 +173,45 @@ conv_scan_prefill_kernel(const T* __restrict__ P, long long ldP, int col_x, int 
             const int q = tid / CPB, cc = tid % CPB;
             halo[q][cc] = to_f(r.x[TC - (KC - 1) + q][cc]);
         }
-        // scan the chunk: partial sums of 4 steps go to shared memory together
-#pragma unroll 1
-        for (int t4 = 0; t4 < TC; t4 += 16) {
-            float yp[16];
+        // scan the chunk in groups of 8 steps, software-pipelined: the shared-memory
+        // operands of group g+1 are loaded while group g's exp2s and FMAs run, so each
+        // step waits only on its own recurrence FMA
+        {
+            constexpr int GS = 8;
+            float2 dvb[2][GS];
+            float4 qb[2][GS];
 #pragma unroll
-            for (int u = 0; u < 16; ++u) {
-                const float2 dv = dd[t4 + u][cl];
-                const float4 q = bc[t4 + u][p];
-                const float2 arg = mul2(make_float2(dv.x, dv.x), A2);
-                const float2 a = make_float2(fast_exp2(arg.x), fast_exp2(arg.y));
-                h = fma2(a, h, mul2(make_float2(dv.y, dv.y), make_float2(q.x, q.y)));
-                const float2 ch = mul2(make_float2(q.z, q.w), h);
-                yp[u] = ch.x + ch.y;
+            for (int u = 0; u < GS; ++u) {
+                dvb[0][u] = dd[u][cl];
+                qb[0][u] = bc[u][p];
             }
 #pragma unroll
-            for (int u = 0; u < 16; u += 4)
-                *reinterpret_cast<float4*>(&part[cl][p][t4 + u]) = make_float4(yp[u], yp[u + 1], yp[u + 2], yp[u + 3]);
+            for (int g8 = 0; g8 < TC / GS; ++g8) {
+                const int cur = g8 & 1;
+                if (g8 + 1 < TC / GS) {
+#pragma unroll
+                    for (int u = 0; u < GS; ++u) {
+                        dvb[cur ^ 1][u] = dd[(g8 + 1) * GS + u][cl];
+                        qb[cur ^ 1][u] = bc[(g8 + 1) * GS + u][p];
+                    }
+                }
+                float2 a[GS];
+#pragma unroll
+                for (int u = 0; u < GS; ++u) {
+                    const float2 arg = mul2(make_float2(dvb[cur][u].x, dvb[cur][u].x), A2);
+                    a[u] = make_float2(fast_exp2(arg.x), fast_exp2(arg.y));
+                }
+                float yp[GS];
+#pragma unroll
+                for (int u = 0; u < GS; ++u) {
+                    const float4 q = qb[cur][u];
+                    h = fma2(a[u], h, mul2(make_float2(dvb[cur][u].y, dvb[cur][u].y), make_float2(q.x, q.y)));
+                    const float2 ch = mul2(make_float2(q.z, q.w), h);
+                    yp[u] = ch.x + ch.y;
+                }
+                *reinterpret_cast<float4*>(&part[cl][p][g8 * GS]) = make_float4(yp[0], yp[1], yp[2], yp[3]);
+                *reinterpret_cast<float4*>(&part[cl][p][g8 * GS + 4]) = make_float4(yp[4], yp[5], yp[6], yp[7]);
+            }
         }
         __syncthreads();  // partial sums complete
         if (tid < nt) {
