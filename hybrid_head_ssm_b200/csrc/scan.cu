@@ -5,42 +5,33 @@
 // with A = -exp(A_log) per (channel, state) and the state in fp32 registers.
 //
 // One block per (8-channel group, sequence), 64 threads; thread (c, p) owns states 2p
-// and 2p+1 of channel c and updates both with packed f32x2 arithmetic, so a recurrence
-// step is two MUFU exp2 and a few FMA-pipe instructions per thread, and the only serial
-// dependency is one FMA per state. Time is walked in chunks of 64 rows, each thread
-// staging one row with cp.async while the previous chunk is scanned:
-//   unpack   thread t: conv + SiLU of row t for the 8 channels, Delta * xc, B/C pairs;
-//   scan     thread (c, p): 64 steps, its partial C.h sums written to shared memory;
+// and 2p+1 of channel c and updates both with packed f32x2 arithmetic (__ffma2_rn and
+// friends), so a recurrence step is two MUFU exp2 and four FMA-pipe instructions, and
+// the only serial dependency is one FFMA2 per step. Time is walked in chunks of 64
+// rows; while a chunk is processed the next one is staged with cp.async:
+//   unpack   thread t: conv + SiLU of row t for the 8 channels (as 4 channel pairs),
+//            (Delta, Delta, Delta*xc, Delta*xc) quads and (B, B, C, C) quads, so the
+//            scan reads each operand pair ready-made with one 16-byte load;
+//   scan     thread (c, p): 64 steps, its partial C.h sum of each step to shared memory;
 //   reduce   thread t: y of row t = the 8 partial sums + D xc, one 16-byte store.
-// The sum over the threads of a channel is thus never on the recurrence's path.
+// The chunk's x rows sit after three halo rows (the previous chunk's last three rows,
+// zero before the sequence), so the causal conv needs no branches. Shared-memory rows
+// are padded so that the unpack's per-row stores spread over all banks.
 #include "kernels.h"
 
 namespace hymba {
 
 namespace {
 
-constexpr int CPB = 8;   // channels per block
-constexpr int TPC = 8;   // threads per channel (2 states each)
+constexpr int CPB = 8;             // channels per block
+constexpr int TPC = 8;             // threads per channel (2 states each)
 constexpr int NTH = CPB * TPC;
-constexpr int TC = 64;   // rows per chunk (= threads: one row each when staging)
-constexpr int KC = 4;    // conv taps
-constexpr int PSTR = TC + 4;  // padded row of the partial-sum buffer
+constexpr int TC = 64;             // rows per chunk (one row per thread in unpack and reduce)
+constexpr int KC = 4;              // conv taps
+constexpr int GS = 4;              // steps per software-pipelined group of the scan
+constexpr int PCS = TC * TPC + 8;  // channel stride of the partial-sum buffer (floats)
 constexpr float LOG2E = 1.4426950408889634f;
-static_assert(TC == NTH, "staging maps one row per thread");
-
-__device__ __forceinline__ float2 mul2(float2 a, float2 b) {
-    uint64_t r;
-    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(*reinterpret_cast<uint64_t*>(&a)), "l"(*reinterpret_cast<uint64_t*>(&b)));
-    return *reinterpret_cast<float2*>(&r);
-}
-__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
-    uint64_t r;
-    asm("fma.rn.f32x2 %0, %1, %2, %3;"
-        : "=l"(r)
-        : "l"(*reinterpret_cast<uint64_t*>(&a)), "l"(*reinterpret_cast<uint64_t*>(&b)),
-          "l"(*reinterpret_cast<uint64_t*>(&c)));
-    return *reinterpret_cast<float2*>(&r);
-}
+static_assert(TC == NTH, "unpack and reduce map one row per thread");
 
 __device__ __forceinline__ void cp_async16(void* dst, const void* src) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(static_cast<uint32_t>(__cvta_generic_to_shared(dst))),
@@ -51,46 +42,83 @@ __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commi
 __device__ __forceinline__ void cp_async_wait1() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
 __device__ __forceinline__ void cp_async_wait0() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
 
+__device__ __forceinline__ float rcp_approx(float x) {
+    float y;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+__device__ __forceinline__ float2 exp2_pair(float2 a) { return make_float2(fast_exp2(a.x), fast_exp2(a.y)); }
+
 template <typename T>
 struct Raw {  // one chunk as copied from global memory
-    alignas(16) T x[TC][CPB];
+    alignas(16) T x[TC + KC - 1][CPB];   // rows 0..2: the three rows before the chunk
     alignas(16) float d[TC][CPB];
     alignas(16) T b[TC][16];
     alignas(16) T c[TC][16];
 };
 
-// Thread t queues the copies of row t0 + t of the sequence (rows past Tp repeat the
-// last row; their results are never stored and their Delta is zeroed when unpacked).
-template <typename T>
-__device__ __forceinline__ void stage_row(Raw<T>& r, const T* P, long long ldP, int col_x, int col_B, int col_C,
-                                          const float* delta, int di, int c0, long long row0, int t0, int Tp) {
-    const int tt = threadIdx.x;
-    const long long row = row0 + min(t0 + tt, Tp - 1);
-    const T* prow = P + row * ldP;
-    constexpr int XV = CPB * (int)sizeof(T) / 16;
-    constexpr int BV = 16 * (int)sizeof(T) / 16;
-#pragma unroll
-    for (int k = 0; k < XV; ++k)
-        cp_async16(reinterpret_cast<char*>(&r.x[tt][0]) + 16 * k, reinterpret_cast<const char*>(prow + col_x + c0) + 16 * k);
-#pragma unroll
-    for (int k = 0; k < CPB * 4 / 16; ++k)
-        cp_async16(reinterpret_cast<char*>(&r.d[tt][0]) + 16 * k,
-                   reinterpret_cast<const char*>(delta + row * di + c0) + 16 * k);
-#pragma unroll
-    for (int k = 0; k < BV; ++k) {
-        cp_async16(reinterpret_cast<char*>(&r.b[tt][0]) + 16 * k, reinterpret_cast<const char*>(prow + col_B) + 16 * k);
-        cp_async16(reinterpret_cast<char*>(&r.c[tt][0]) + 16 * k, reinterpret_cast<const char*>(prow + col_C) + 16 * k);
-    }
-}
-
 template <typename T>
 struct ScanSmem {
     Raw<T> raw[2];
-    alignas(16) float2 dd[TC][CPB];            // (Delta, Delta * xc)
-    alignas(16) float4 bc[TC][TPC];            // (B_2p, B_2p+1, C_2p, C_2p+1)
-    alignas(16) float xd[TC][CPB];             // D * xc
-    alignas(16) float part[CPB][TPC][PSTR];    // partial C.h sums
+    alignas(16) float4 dd[TC][CPB + 1];      // (Delta, Delta, Delta*xc, Delta*xc), padded rows
+    alignas(16) float4 bc[TC][TPC + 1];      // (B_2p, B_2p+1, C_2p, C_2p+1), padded rows
+    alignas(16) float xd[TC][12];            // D * xc (8 used), padded rows
+    alignas(16) float part[CPB * PCS];       // [channel][row][p] partial C.h sums
+    alignas(16) float2 w2[KC + 2][CPB / 2];  // conv taps, conv bias and D as channel pairs
 };
+
+// 8 consecutive values as 4 float pairs
+template <typename T>
+__device__ __forceinline__ void load8x2(const T* p, float2* v) {
+    if constexpr (sizeof(T) == 2) {
+        const uint4 u = *reinterpret_cast<const uint4*>(p);
+        v[0] = __half22float2(*reinterpret_cast<const __half2*>(&u.x));
+        v[1] = __half22float2(*reinterpret_cast<const __half2*>(&u.y));
+        v[2] = __half22float2(*reinterpret_cast<const __half2*>(&u.z));
+        v[3] = __half22float2(*reinterpret_cast<const __half2*>(&u.w));
+    } else {
+        const float4 a = reinterpret_cast<const float4*>(p)[0];
+        const float4 b = reinterpret_cast<const float4*>(p)[1];
+        v[0] = make_float2(a.x, a.y);
+        v[1] = make_float2(a.z, a.w);
+        v[2] = make_float2(b.x, b.y);
+        v[3] = make_float2(b.z, b.w);
+    }
+}
+
+// Queue the copies of rows t0 .. t0+TC-1 of the sequence (rows past Tp repeat the last
+// row; their results are never stored and their Delta is zeroed when unpacked).
+template <typename T>
+__device__ __forceinline__ void stage_chunk(Raw<T>& r, const T* P, long long ldP, int col_x, int col_B, int col_C,
+                                            const float* delta, int di, int c0, long long row0, int t0, int Tp) {
+    constexpr int XV = CPB * (int)sizeof(T) / 16;  // 16-byte pieces per row
+    constexpr int DV = CPB * 4 / 16;
+    constexpr int BV = 16 * (int)sizeof(T) / 16;
+    const int tid = threadIdx.x;
+#pragma unroll
+    for (int j = tid; j < TC * XV; j += NTH) {
+        const int rr = j / XV, k = j % XV;
+        const long long row = row0 + min(t0 + rr, Tp - 1);
+        cp_async16(reinterpret_cast<char*>(&r.x[rr + KC - 1][0]) + 16 * k,
+                   reinterpret_cast<const char*>(P + row * ldP + col_x + c0) + 16 * k);
+    }
+#pragma unroll
+    for (int j = tid; j < TC * DV; j += NTH) {
+        const int rr = j / DV, k = j % DV;
+        const long long row = row0 + min(t0 + rr, Tp - 1);
+        cp_async16(reinterpret_cast<char*>(&r.d[rr][0]) + 16 * k,
+                   reinterpret_cast<const char*>(delta + row * di + c0) + 16 * k);
+    }
+#pragma unroll
+    for (int j = tid; j < TC * BV; j += NTH) {
+        const int rr = j / BV, k = j % BV;
+        const long long row = row0 + min(t0 + rr, Tp - 1);
+        cp_async16(reinterpret_cast<char*>(&r.b[rr][0]) + 16 * k,
+                   reinterpret_cast<const char*>(P + row * ldP + col_B) + 16 * k);
+        cp_async16(reinterpret_cast<char*>(&r.c[rr][0]) + 16 * k,
+                   reinterpret_cast<const char*>(P + row * ldP + col_C) + 16 * k);
+    }
+}
 
 template <typename T>
 __global__ void __launch_bounds__(NTH)
@@ -101,130 +129,139 @@ conv_scan_prefill_kernel(const T* __restrict__ P, long long ldP, int col_x, int 
                          float* __restrict__ conv_out, int Tp, int di) {
     extern __shared__ __align__(16) uint8_t scan_smem[];
     ScanSmem<T>& sm = *reinterpret_cast<ScanSmem<T>*>(scan_smem);
-    Raw<T>* raw = sm.raw;
-    float2 (*dd)[CPB] = sm.dd;
-    float4 (*bc)[TPC] = sm.bc;
-    float (*xd)[CPB] = sm.xd;
-    float (*part)[TPC][PSTR] = sm.part;
-    __shared__ float halo[KC - 1][CPB];
-    __shared__ float wconv[CPB][KC + 1];
-    __shared__ float dch[CPB];
-
     const int b = blockIdx.y, c0 = blockIdx.x * CPB;
-    const int tid = threadIdx.x, cl = tid / TPC, p = tid % TPC, c = c0 + cl;
+    const int tid = threadIdx.x, cl = tid / TPC, p = tid % TPC;
     const long long row0 = (long long)b * Tp;
-    const float2 A2 = make_float2(-expf(A_log[(long long)c * 16 + 2 * p]) * LOG2E,
-                                  -expf(A_log[(long long)c * 16 + 2 * p + 1]) * LOG2E);
-    if (tid < (KC - 1) * CPB) halo[tid / CPB][tid % CPB] = 0.f;
-    if (tid < CPB) {
-        for (int k = 0; k < KC; ++k) wconv[tid][k] = conv_w[(long long)(c0 + tid) * KC + k];
-        wconv[tid][KC] = conv_b[c0 + tid];
-        dch[tid] = Dp[c0 + tid];
+    // A * log2(e) for the thread's two states: exp(Delta A) = exp2(Delta * A2)
+    const float2 A2 = make_float2(-expf(A_log[(long long)(c0 + cl) * 16 + 2 * p]) * LOG2E,
+                                  -expf(A_log[(long long)(c0 + cl) * 16 + 2 * p + 1]) * LOG2E);
+    if (tid < (KC + 2) * (CPB / 2)) {
+        const int q = tid / (CPB / 2), j = tid % (CPB / 2);
+        const int ca = c0 + 2 * j, cb = ca + 1;
+        float2 v;
+        if (q < KC) v = make_float2(conv_w[(long long)ca * KC + q], conv_w[(long long)cb * KC + q]);
+        else if (q == KC) v = make_float2(conv_b[ca], conv_b[cb]);
+        else v = make_float2(Dp[ca], Dp[cb]);
+        sm.w2[q][j] = v;
     }
+    if (tid < (KC - 1) * CPB) sm.raw[0].x[tid / CPB][tid % CPB] = from_f<T>(0.f);
     float2 h = make_float2(0.f, 0.f);
     const int nchunk = (Tp + TC - 1) / TC;
 
-    stage_row<T>(raw[0], P, ldP, col_x, col_B, col_C, delta, di, c0, row0, 0, Tp);
+    stage_chunk<T>(sm.raw[0], P, ldP, col_x, col_B, col_C, delta, di, c0, row0, 0, Tp);
     cp_async_commit();
     for (int k = 0; k < nchunk; ++k) {
         const int t0 = k * TC, nt = min(TC, Tp - t0);
-        if (k + 1 < nchunk) stage_row<T>(raw[(k + 1) & 1], P, ldP, col_x, col_B, col_C, delta, di, c0, row0, t0 + TC, Tp);
+        if (k + 1 < nchunk)
+            stage_chunk<T>(sm.raw[(k + 1) & 1], P, ldP, col_x, col_B, col_C, delta, di, c0, row0, t0 + TC, Tp);
         cp_async_commit();
         cp_async_wait1();
         __syncthreads();  // chunk k staged; previous chunk's reduce done
-        const Raw<T>& r = raw[k & 1];
+        const Raw<T>& r = sm.raw[k & 1];
         {
-            // unpack row tid
-            const int tt = tid;
-            float xs[KC][CPB];
+            // unpack row t
+            const int t = tid;
+            float2 acc[CPB / 2];
+#pragma unroll
+            for (int j = 0; j < CPB / 2; ++j) acc[j] = sm.w2[KC][j];
 #pragma unroll
             for (int q = 0; q < KC; ++q) {
-                const int src = tt - (KC - 1) + q;
+                float2 xv[CPB / 2];
+                load8x2<T>(&r.x[t + q][0], xv);
 #pragma unroll
-                for (int cc = 0; cc < CPB; ++cc) xs[q][cc] = src >= 0 ? to_f(r.x[src][cc]) : halo[src + KC - 1][cc];
+                for (int j = 0; j < CPB / 2; ++j) acc[j] = __ffma2_rn(sm.w2[q][j], xv[j], acc[j]);
             }
+            const float4 da = *reinterpret_cast<const float4*>(&r.d[t][0]);
+            const float4 db = *reinterpret_cast<const float4*>(&r.d[t][4]);
+            // rows past the end of the sequence get Delta = 0: exp2(0) = 1 and a zero
+            // input leave the state exactly as it is after the last row
+            const float keep = t < nt ? 1.f : 0.f;
+            const float2 dl[CPB / 2] = {make_float2(da.x, da.y), make_float2(da.z, da.w), make_float2(db.x, db.y),
+                                        make_float2(db.z, db.w)};
+            float2 xdv[CPB / 2];
 #pragma unroll
-            for (int cc = 0; cc < CPB; ++cc) {
-                float acc = wconv[cc][KC];
-#pragma unroll
-                for (int q = 0; q < KC; ++q) acc = fmaf(wconv[cc][q], xs[q][cc], acc);
-                const float xc = __fdividef(acc, 1.0f + __expf(-acc));
-                // rows past the end of the sequence get Delta = 0: exp2(0) = 1 and a zero
-                // input leave the state exactly as it is after the last row
-                const float d = tt < nt ? r.d[tt][cc] : 0.f;
-                dd[tt][cc] = make_float2(d, d * xc);
-                xd[tt][cc] = dch[cc] * xc;
+            for (int j = 0; j < CPB / 2; ++j) {
+                // SiLU(u) = u / (1 + exp(-u))
+                const float2 e = exp2_pair(__fmul2_rn(acc[j], make_float2(-LOG2E, -LOG2E)));
+                const float2 den = __fadd2_rn(e, make_float2(1.f, 1.f));
+                const float2 xc = __fmul2_rn(acc[j], make_float2(rcp_approx(den.x), rcp_approx(den.y)));
+                const float2 d = __fmul2_rn(dl[j], make_float2(keep, keep));
+                const float2 dv = __fmul2_rn(d, xc);
+                sm.dd[t][2 * j] = make_float4(d.x, d.x, dv.x, dv.x);
+                sm.dd[t][2 * j + 1] = make_float4(d.y, d.y, dv.y, dv.y);
+                xdv[j] = __fmul2_rn(sm.w2[KC + 1][j], xc);
             }
+            *reinterpret_cast<float4*>(&sm.xd[t][0]) = make_float4(xdv[0].x, xdv[0].y, xdv[1].x, xdv[1].y);
+            *reinterpret_cast<float4*>(&sm.xd[t][4]) = make_float4(xdv[2].x, xdv[2].y, xdv[3].x, xdv[3].y);
+            float2 bv[8], cv[8];
+            load8x2<T>(&r.b[t][0], bv);
+            load8x2<T>(&r.b[t][8], bv + 4);
+            load8x2<T>(&r.c[t][0], cv);
+            load8x2<T>(&r.c[t][8], cv + 4);
 #pragma unroll
-            for (int q = 0; q < TPC; ++q)
-                bc[tt][q] = make_float4(to_f(r.b[tt][2 * q]), to_f(r.b[tt][2 * q + 1]), to_f(r.c[tt][2 * q]),
-                                        to_f(r.c[tt][2 * q + 1]));
-            if (k + 1 == nchunk && conv_out && tt < KC) {
-                // conv state: the last KC inputs of the sequence, oldest first
-                const int src = nt - KC + tt;
-#pragma unroll
-                for (int cc = 0; cc < CPB; ++cc)
-                    conv_out[((long long)b * di + c0 + cc) * KC + tt] =
-                        src >= 0 ? to_f(r.x[src][cc]) : (src + KC - 1 >= 0 ? halo[src + KC - 1][cc] : 0.f);
-            }
+            for (int q = 0; q < TPC; ++q) sm.bc[t][q] = make_float4(bv[q].x, bv[q].y, cv[q].x, cv[q].y);
         }
-        __syncthreads();  // unpacked; halo readers done
-        if (k + 1 < nchunk && tid < (KC - 1) * CPB) {
+        if (k + 1 < nchunk) {
+            if (tid < KC - 1) {
+                // halo of the next chunk: this chunk's last three rows of x (the next
+                // chunk's copies write rows 3.. of that buffer only)
+                const uint4* src = reinterpret_cast<const uint4*>(&r.x[TC + tid][0]);
+                uint4* dst = reinterpret_cast<uint4*>(&sm.raw[(k + 1) & 1].x[tid][0]);
+#pragma unroll
+                for (int i = 0; i < CPB * (int)sizeof(T) / 16; ++i) dst[i] = src[i];
+            }
+        } else if (conv_out && tid < KC * CPB) {
+            // conv state: the last KC inputs of the sequence, oldest first (zero rows
+            // stand before the sequence start)
             const int q = tid / CPB, cc = tid % CPB;
-            halo[q][cc] = to_f(r.x[TC - (KC - 1) + q][cc]);
+            conv_out[((long long)b * di + c0 + cc) * KC + q] = to_f(r.x[nt - 1 + q][cc]);
         }
-        // scan the chunk in groups of 8 steps, software-pipelined: the shared-memory
-        // operands of group g+1 are loaded while group g's exp2s and FMAs run, so each
-        // step waits only on its own recurrence FMA
+        __syncthreads();  // unpacked
         {
-            constexpr int GS = 8;
-            float2 dvb[2][GS];
-            float4 qb[2][GS];
+            // scan in groups of GS steps; the next group's operands load while the
+            // current group's exp2s and FMAs run
+            float* pw = sm.part + cl * PCS + p;
+            float4 qd[2][GS], qb[2][GS];
 #pragma unroll
             for (int u = 0; u < GS; ++u) {
-                dvb[0][u] = dd[u][cl];
-                qb[0][u] = bc[u][p];
+                qd[0][u] = sm.dd[u][cl];
+                qb[0][u] = sm.bc[u][p];
             }
 #pragma unroll
-            for (int g8 = 0; g8 < TC / GS; ++g8) {
-                const int cur = g8 & 1;
-                if (g8 + 1 < TC / GS) {
+            for (int g = 0; g < TC / GS; ++g) {
+                const int cur = g & 1;
+                if (g + 1 < TC / GS) {
 #pragma unroll
                     for (int u = 0; u < GS; ++u) {
-                        dvb[cur ^ 1][u] = dd[(g8 + 1) * GS + u][cl];
-                        qb[cur ^ 1][u] = bc[(g8 + 1) * GS + u][p];
+                        qd[cur ^ 1][u] = sm.dd[(g + 1) * GS + u][cl];
+                        qb[cur ^ 1][u] = sm.bc[(g + 1) * GS + u][p];
                     }
                 }
                 float2 a[GS];
 #pragma unroll
-                for (int u = 0; u < GS; ++u) {
-                    const float2 arg = mul2(make_float2(dvb[cur][u].x, dvb[cur][u].x), A2);
-                    a[u] = make_float2(fast_exp2(arg.x), fast_exp2(arg.y));
-                }
-                float yp[GS];
+                for (int u = 0; u < GS; ++u) a[u] = exp2_pair(__fmul2_rn(make_float2(qd[cur][u].x, qd[cur][u].y), A2));
 #pragma unroll
                 for (int u = 0; u < GS; ++u) {
                     const float4 q = qb[cur][u];
-                    h = fma2(a[u], h, mul2(make_float2(dvb[cur][u].y, dvb[cur][u].y), make_float2(q.x, q.y)));
-                    const float2 ch = mul2(make_float2(q.z, q.w), h);
-                    yp[u] = ch.x + ch.y;
+                    h = __ffma2_rn(a[u], h, __fmul2_rn(make_float2(qd[cur][u].z, qd[cur][u].w), make_float2(q.x, q.y)));
+                    const float2 ch = __fmul2_rn(make_float2(q.z, q.w), h);
+                    pw[(g * GS + u) * TPC] = ch.x + ch.y;
                 }
-                *reinterpret_cast<float4*>(&part[cl][p][g8 * GS]) = make_float4(yp[0], yp[1], yp[2], yp[3]);
-                *reinterpret_cast<float4*>(&part[cl][p][g8 * GS + 4]) = make_float4(yp[4], yp[5], yp[6], yp[7]);
             }
         }
         __syncthreads();  // partial sums complete
         if (tid < nt) {
-            const int tt = tid;
+            const int t = tid;
             float y[CPB];
 #pragma unroll
             for (int cc = 0; cc < CPB; ++cc) {
-                float s = xd[tt][cc];
-#pragma unroll
-                for (int q = 0; q < TPC; ++q) s += part[cc][q][tt];
-                y[cc] = s;
+                const float4 a = *reinterpret_cast<const float4*>(sm.part + cc * PCS + t * TPC);
+                const float4 e = *reinterpret_cast<const float4*>(sm.part + cc * PCS + t * TPC + 4);
+                const float2 s = __fadd2_rn(__fadd2_rn(make_float2(a.x, a.y), make_float2(a.z, a.w)),
+                                            __fadd2_rn(make_float2(e.x, e.y), make_float2(e.z, e.w)));
+                y[cc] = (s.x + s.y) + sm.xd[t][cc];
             }
-            T* dst = ypre + (row0 + t0 + tt) * di + c0;
+            T* dst = ypre + (row0 + t0 + t) * di + c0;
             if constexpr (sizeof(T) == 2) {
                 uint4 v;
                 v.x = pack2<T>(y[0], y[1]);
@@ -240,7 +277,7 @@ conv_scan_prefill_kernel(const T* __restrict__ P, long long ldP, int col_x, int 
     }
     cp_async_wait0();
     if (h_out) {
-        float* dst = h_out + ((long long)b * di + c) * 16 + 2 * p;
+        float* dst = h_out + ((long long)b * di + c0 + cl) * 16 + 2 * p;
         dst[0] = h.x;
         dst[1] = h.y;
     }
