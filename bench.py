@@ -19,6 +19,7 @@ import argparse
 import json
 import os
 import statistics
+import threading
 import subprocess
 import sys
 import time
@@ -44,54 +45,79 @@ def peaks():
 
 
 class Clocks:
-    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
+    """SM clocks and clock-event (throttle) reasons sampled through NVML every 2 ms
+    while the timed region is open (read-only queries; no setting is touched). The
+    samples also go to gpurun_out/clocks_rank<i>.csv."""
 
-    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = (("hw_slowdown", "nvmlClocksEventReasonHwSlowdown"),
+               ("hw_thermal_slowdown", "nvmlClocksEventReasonHwThermalSlowdown"),
+               ("sw_thermal_slowdown", "nvmlClocksEventReasonSwThermalSlowdown"),
+               ("sw_power_cap", "nvmlClocksEventReasonSwPowerCap"))
 
-    def __init__(self, index: int):
-        self.index = index
-        self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{index}.csv")
+    def __init__(self, cuda_index: int):
+        self.cuda_index = cuda_index
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{cuda_index}.csv")
+        self.samples = []
+        self.thread = None
+        self.open = threading.Event()
+        self.done = threading.Event()
+
+    def _handle(self, nv):
+        try:
+            pr = torch.cuda.get_device_properties(self.cuda_index)
+            return nv.nvmlDeviceGetHandleByPciBusId(
+                f"{pr.pci_domain_id:08X}:{pr.pci_bus_id:02X}:{pr.pci_device_id:02X}.0".encode())
+        except Exception:
+            return nv.nvmlDeviceGetHandleByIndex(self.cuda_index)
+
+    def _run(self, nv, hd, masks):
+        while not self.done.is_set():
+            if self.open.is_set():
+                try:
+                    sm = nv.nvmlDeviceGetClockInfo(hd, nv.NVML_CLOCK_SM)
+                    mx = nv.nvmlDeviceGetMaxClockInfo(hd, nv.NVML_CLOCK_SM)
+                    rs = nv.nvmlDeviceGetCurrentClocksEventReasons(hd)
+                    self.samples.append((time.time(), sm, mx, rs, [n for n, m in masks if rs & m]))
+                except Exception:
+                    pass
+            time.sleep(0.002)
 
     def start(self):
         try:
-            os.makedirs(os.path.dirname(self.path), exist_ok=True)
-            self.f = open(self.path, "w")
-            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}",
-                                          "--format=csv,noheader,nounits", "-lms", "200"],
-                                         stdout=self.f, stderr=subprocess.DEVNULL)
+            import pynvml as nv
+            nv.nvmlInit()
+            hd = self._handle(nv)
+            masks = [(n, getattr(nv, attr)) for n, attr in self.REASONS]
         except Exception:
-            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._run, args=(nv, hd, masks), daemon=True)
+        self.thread.start()
+
+    def begin(self):
+        self.open.set()
+
+    def end(self):
+        self.open.clear()
 
     def stop(self):
-        if self.proc is None:
+        if self.thread is None:
             return None
-        self.proc.terminate()
+        self.done.set()
+        self.thread.join(timeout=5)
         try:
-            self.proc.wait(timeout=5)
-        except Exception:
-            self.proc.kill()
-        self.f.close()
-        sm, mx, reasons = [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for line in open(self.path):
-            parts = [p.strip() for p in line.split(",")]
-            if len(parts) < 9:
-                continue
-            try:
-                sm.append(float(parts[1]))
-                mx.append(float(parts[2]))
-            except ValueError:
-                continue
-            for n, v in zip(names, parts[5:9]):
-                if v.lower().startswith("active"):
-                    reasons.add(n)
-        if not sm:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            with open(self.path, "w") as f:
+                f.write("time,sm_mhz,sm_max_mhz,reasons_mask,reasons\n")
+                for t, sm, mx, rs, names in self.samples:
+                    f.write(f"{t:.4f},{sm},{mx},{rs:#x},{'|'.join(names)}\n")
+        except OSError:
+            pass
+        if not self.samples:
             return None
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
-                "samples": len(sm)}
+        reasons = sorted({n for *_, names in self.samples for n in names})
+        return {"sm_mhz": statistics.median(s[1] for s in self.samples),
+                "sm_max_mhz": max(s[2] for s in self.samples), "reasons": reasons,
+                "samples": len(self.samples), "source": "NVML, 2 ms, timed region only"}
 
 
 def visible_pairs(Tp, m, W):
@@ -256,12 +282,14 @@ def main():
     launches0 = hy.hymba_launch_count()
     barrier()
     torch.cuda.synchronize()
+    clocks.begin()
     for i in range(args.steps):
         flush.fill_(i & 0xFF)
         ev[i][0].record(stream)
         step()
         ev[i][1].record(stream)
     torch.cuda.synchronize()
+    clocks.end()
     barrier()
     launches = hy.hymba_launch_count() - launches0
     trace = hy.trace_collect()

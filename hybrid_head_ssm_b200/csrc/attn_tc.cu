@@ -4,16 +4,27 @@
 // plus a sliding window or the whole causal history (51cto Hymba-1.5B article,
 // section 2). Key j is visible to query i iff j <= i and (j < n_meta or i - j < W).
 //
-// One CTA per (128-query tile, query head, sequence), 6 warps:
-//   warp 0      TMA: the Q tile once, then K (128 keys x 64) and V (128 keys x 128, two
-//               64-wide panels) of each visible key block into a 2-stage ring;
+// One CTA per (128-query tile, query head, sequence), 10 warps:
+//   warp 0      TMA, two producer lanes: lane 0 the Q tile once, then K (128 keys x 64)
+//               of each visible key block into a 3-stage ring that frees a stage as soon
+//               as its S MMA completes; lane 1 V (128 keys x 128, two 64-wide panels)
+//               into a 2-stage ring freed by the PV MMA. K of later blocks thus never
+//               waits for an earlier PV;
 //   warp 1      MMA issuer: S_j = Q K_j^T (128 x 128 x 64) into one of two TMEM S buffers,
-//               then O += P_j V_j (128 x 128 x 128) into the TMEM O accumulator;
-//   warps 2..5  softmax, one query row per thread: S_j from TMEM, scale and mask, running
-//               max; P_j = 2^(s - m) in fp16 into a 128-byte-swizzled shared-memory tile
-//               (the A operand of the PV MMA); O is rescaled in TMEM only when the
-//               running max grows by more than 2^8, so most blocks need no rescale.
-//               At the end O / l is written in fp16.
+//               O += P_j V_j (128 x 128 x 128) into the TMEM O accumulator once the
+//               softmax of block j is done, and right after it S_{j+2}: the tensor pipe
+//               works on PV_j and S_{j+2} while the softmax of block j+1 runs;
+//   warps 2..9  softmax, two threads per query row (warps w and w+4 read the same TMEM
+//               lane quadrant, columns 0..63 and 64..127 of S_j): scale and mask, row max
+//               (the two halves exchange theirs through shared memory each block);
+//               P_j = 2^(s - m) in fp16 into a 128-byte-swizzled shared-memory tile (the A
+//               operand of the PV MMA, one 64-column panel per half); O is rescaled in
+//               TMEM only when the running max grows by more than 2^8, so most blocks
+//               need no rescale. At the end O / l is written in fp16.
+// The exp2s are the softmax's throughput limit (MUFU: 16 instructions per clock per SM
+// against 128 x 128 elements per block): they run two per instruction on fp16 pairs
+// (P is fp16 for the PV MMA anyway), max and sum use independent partial chains, and
+// masking is one branch-free interval test per key.
 // Only key blocks that hold visible keys are visited: the meta blocks and the blocks of
 // [max(n_meta, i0 - W + 1), i_last]. Operands are fp16 (the layer's intermediate type).
 #include "kernels.h"
@@ -23,20 +34,26 @@ namespace hymba {
 
 namespace {
 
-constexpr int QT = 128, KBLK = 128, DH = 64, DV = 128, NTHREADS = 192;
+constexpr int QT = 128, KBLK = 128, DH = 64, DV = 128, NTHREADS = 320;
+constexpr int NSOFT = 256;  // softmax threads: two per query row
+constexpr int KST = 3;      // K ring stages (a stage frees when its S MMA completes)
+constexpr int VST = 2;      // V ring stages (a stage frees when its PV MMA completes)
 constexpr float LOG2E = 1.4426950408889634f;
 constexpr float RESCALE_LOG2 = 8.0f;
 
 struct AttnSmem {
     alignas(1024) uint8_t q[QT * DH * 2];
-    alignas(1024) uint8_t k[2][KBLK * DH * 2];
-    alignas(1024) uint8_t v[2][2][KBLK * 64 * 2];
+    alignas(1024) uint8_t k[KST][KBLK * DH * 2];
+    alignas(1024) uint8_t v[VST][2][KBLK * 64 * 2];
     alignas(1024) uint8_t p[2][2][QT * 64 * 2];
     uint64_t q_full;
-    uint64_t kv_full[2], kv_empty[2];
+    uint64_t k_full[KST], k_empty[KST];
+    uint64_t v_full[VST], v_empty[VST];
     uint64_t s_full[2], s_free[2];
     uint64_t p_full[2], pv_done[2];
     uint64_t o_done, drain;
+    float xmax[2][2][QT];  // [block parity][half][row] partial row maxima
+    float xsum[2][QT];     // [half][row] partial row sums
     uint32_t tmem_base;
     int abort;
 };
@@ -57,6 +74,13 @@ struct Blocks {
         else { *j0 = lo + (j - n_meta_blk) * KBLK; *rs = lo; *re = hi; }
     }
 };
+
+// 2^x for both halves of an fp16 pair, one MUFU instruction
+__device__ __forceinline__ uint32_t exp2_f16x2(uint32_t x) {
+    uint32_t y;
+    asm("ex2.approx.f16x2 %0, %1;" : "=r"(y) : "r"(x));
+    return y;
+}
 
 __device__ __forceinline__ void fail(volatile int* abort, int* status, int role, int step, int bar) {
     *abort = 1;
@@ -81,12 +105,18 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
 
     if (threadIdx.x == 0) {
         tc::mbar_init(&s.q_full, 1);
+        for (int i = 0; i < KST; ++i) {
+            tc::mbar_init(&s.k_full[i], 1);
+            tc::mbar_init(&s.k_empty[i], 1);
+        }
+        for (int i = 0; i < VST; ++i) {
+            tc::mbar_init(&s.v_full[i], 1);
+            tc::mbar_init(&s.v_empty[i], 1);
+        }
         for (int i = 0; i < 2; ++i) {
-            tc::mbar_init(&s.kv_full[i], 1);
-            tc::mbar_init(&s.kv_empty[i], 1);
             tc::mbar_init(&s.s_full[i], 1);
-            tc::mbar_init(&s.s_free[i], 128);
-            tc::mbar_init(&s.p_full[i], 128);
+            tc::mbar_init(&s.s_free[i], NSOFT);
+            tc::mbar_init(&s.p_full[i], NSOFT);
             tc::mbar_init(&s.pv_done[i], 1);
         }
         tc::mbar_init(&s.o_done, 1);
@@ -108,28 +138,44 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
     volatile int* abort = &s.abort;
 
     if (warp == 0) {
-        // ---------------- TMA producer ----------------
-        if (tc::elect_one()) {
-            int zero = 0;
-            int last_phase[2] = {-1, -1};
+        // ---------------- TMA producers: lane 0 loads Q and the K blocks, lane 1 the V blocks ----------------
+        int zero = 0;
+        if (lane == 0) {
+            int last_phase[KST];
+            for (int i = 0; i < KST; ++i) last_phase[i] = -1;
             tc::mbar_arrive_expect_tx(&s.q_full, QT * DH * 2);
             tc::tma_load_3d(s.q, &tmQ, &s.q_full, h * DH, i0, b);
             for (int j = 0; j < nblk; ++j) {
-                const int st = j & 1;
-                const uint32_t ph = (j >> 1) & 1;
-                if (!tc::mbar_wait(&s.kv_empty[st], ph ^ 1, abort)) { fail(abort, status, 0, j, 1); break; }
+                const int st = j % KST;
+                const uint32_t ph = (j / KST) & 1;
+                if (!tc::mbar_wait(&s.k_empty[st], ph ^ 1, abort)) { fail(abort, status, 0, j, 1); break; }
                 int j0, rs, re;
                 blk.get(j, &j0, &rs, &re);
-                tc::mbar_arrive_expect_tx(&s.kv_full[st], KBLK * (DH + DV) * 2);
-                tc::tma_load_3d(s.k[st], &tmK, &s.kv_full[st], 0, j0, bg);
-                tc::tma_load_3d(s.v[st][0], &tmV, &s.kv_full[st], 0, j0, bg);
-                tc::tma_load_3d(s.v[st][1], &tmV, &s.kv_full[st], 64, j0, bg);
+                tc::mbar_arrive_expect_tx(&s.k_full[st], KBLK * DH * 2);
+                tc::tma_load_3d(s.k[st], &tmK, &s.k_full[st], 0, j0, bg);
                 last_phase[st] = (int)ph;
             }
             tc::mbar_wait(&s.q_full, 0, &zero);
             if (*abort)
-                for (int i = 0; i < 2; ++i)
-                    if (last_phase[i] >= 0) tc::mbar_wait(&s.kv_full[i], (uint32_t)last_phase[i], &zero);
+                for (int i = 0; i < KST; ++i)
+                    if (last_phase[i] >= 0) tc::mbar_wait(&s.k_full[i], (uint32_t)last_phase[i], &zero);
+        } else if (lane == 1) {
+            int last_phase[VST];
+            for (int i = 0; i < VST; ++i) last_phase[i] = -1;
+            for (int j = 0; j < nblk; ++j) {
+                const int st = j % VST;
+                const uint32_t ph = (j / VST) & 1;
+                if (!tc::mbar_wait(&s.v_empty[st], ph ^ 1, abort)) { fail(abort, status, 0, j, 9); break; }
+                int j0, rs, re;
+                blk.get(j, &j0, &rs, &re);
+                tc::mbar_arrive_expect_tx(&s.v_full[st], KBLK * DV * 2);
+                tc::tma_load_3d(s.v[st][0], &tmV, &s.v_full[st], 0, j0, bg);
+                tc::tma_load_3d(s.v[st][1], &tmV, &s.v_full[st], 64, j0, bg);
+                last_phase[st] = (int)ph;
+            }
+            if (*abort)
+                for (int i = 0; i < VST; ++i)
+                    if (last_phase[i] >= 0) tc::mbar_wait(&s.v_full[i], (uint32_t)last_phase[i], &zero);
         }
     } else if (warp == 1) {
         // ---------------- MMA issuer ----------------
@@ -137,36 +183,42 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
             bool ok = tc::mbar_wait(&s.q_full, 0, abort);
             if (!ok) fail(abort, status, 1, 0, 0);
             const uint32_t qa = tc::smem_u32(s.q);
-            for (int j = 0; ok && j <= nblk; ++j) {
-                if (j < nblk) {
-                    const int st = j & 1;
-                    const uint32_t ph = (j >> 1) & 1;
-                    if (!tc::mbar_wait(&s.kv_full[st], ph, abort)) { fail(abort, status, 1, j, 2); break; }
-                    if (!tc::mbar_wait(&s.s_free[st], ph ^ 1, abort)) { fail(abort, status, 1, j, 3); break; }
-                    tc::tc_fence_after();
-                    const uint32_t ka = tc::smem_u32(s.k[st]);
-                    const uint32_t sd = tmem + 128 + st * 128;
+            // S_j = Q K_j^T into S buffer j & 1; issued two blocks ahead of the PV that
+            // follows the same block's softmax, so the tensor pipe computes S_{j+2} and
+            // PV_j while the softmax of block j+1 runs
+            auto issue_s = [&](int j) -> bool {
+                const int kst = j % KST, sb = j & 1;
+                if (!tc::mbar_wait(&s.k_full[kst], (j / KST) & 1, abort)) { fail(abort, status, 1, j, 2); return false; }
+                if (!tc::mbar_wait(&s.s_free[sb], ((j >> 1) & 1) ^ 1, abort)) { fail(abort, status, 1, j, 3); return false; }
+                tc::tc_fence_after();
+                const uint32_t ka = tc::smem_u32(s.k[kst]);
+                const uint32_t sd = tmem + 128 + sb * 128;
 #pragma unroll
-                    for (int kk = 0; kk < DH / 16; ++kk)
-                        tc::mma_f16_ss(sd, tc::sdesc_k_sw128(qa + kk * 32), tc::sdesc_k_sw128(ka + kk * 32), IDESC_S,
-                                       kk > 0);
-                    tc::mma_commit(&s.s_full[st]);
-                }
-                if (j >= 1) {
-                    const int jj = j - 1, pb = jj & 1;
-                    if (!tc::mbar_wait(&s.p_full[pb], (jj >> 1) & 1, abort)) { fail(abort, status, 1, jj, 4); break; }
-                    tc::tc_fence_after();
-                    const uint32_t pa = tc::smem_u32(s.p[pb][0]);
-                    const uint32_t va = tc::smem_u32(s.v[pb][0]);
+                for (int kk = 0; kk < DH / 16; ++kk)
+                    tc::mma_f16_ss(sd, tc::sdesc_k_sw128(qa + kk * 32), tc::sdesc_k_sw128(ka + kk * 32), IDESC_S,
+                                   kk > 0);
+                tc::mma_commit(&s.s_full[sb]);
+                tc::mma_commit(&s.k_empty[kst]);
+                return true;
+            };
+            for (int j = 0; ok && j < 2 && j < nblk; ++j) ok = issue_s(j);
+            for (int j = 0; ok && j < nblk; ++j) {
+                // O += P_j V_j
+                const int pb = j & 1, vst = j % VST;
+                if (!tc::mbar_wait(&s.p_full[pb], (j >> 1) & 1, abort)) { fail(abort, status, 1, j, 4); break; }
+                if (!tc::mbar_wait(&s.v_full[vst], (j / VST) & 1, abort)) { fail(abort, status, 1, j, 10); break; }
+                tc::tc_fence_after();
+                const uint32_t pa = tc::smem_u32(s.p[pb][0]);
+                const uint32_t va = tc::smem_u32(s.v[vst][0]);
 #pragma unroll
-                    for (int kk = 0; kk < KBLK / 16; ++kk) {
-                        const uint64_t ad = tc::sdesc_k_sw128(pa + (kk >> 2) * (QT * 128) + (kk & 3) * 32);
-                        const uint64_t bd = tc::sdesc_mn_sw128(va + kk * 2048, KBLK * 128);
-                        tc::mma_f16_ss(tmem, ad, bd, IDESC_PV, (jj > 0 || kk > 0));
-                    }
-                    tc::mma_commit(&s.pv_done[pb]);
-                    tc::mma_commit(&s.kv_empty[pb]);
+                for (int kk = 0; kk < KBLK / 16; ++kk) {
+                    const uint64_t ad = tc::sdesc_k_sw128(pa + (kk >> 2) * (QT * 128) + (kk & 3) * 32);
+                    const uint64_t bd = tc::sdesc_mn_sw128(va + kk * 2048, KBLK * 128);
+                    tc::mma_f16_ss(tmem, ad, bd, IDESC_PV, (j > 0 || kk > 0));
                 }
+                tc::mma_commit(&s.pv_done[pb]);
+                tc::mma_commit(&s.v_empty[vst]);
+                if (j + 2 < nblk && !issue_s(j + 2)) break;
             }
             tc::mma_commit(&s.o_done);
             tc::mma_commit(&s.drain);
@@ -174,65 +226,86 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
             tc::mbar_wait(&s.drain, 0, &zero);
         }
     } else {
-        // ---------------- softmax + output (warps 2..5 -> TMEM lane quadrants 2, 3, 0, 1) ----------------
+        // ---------------- softmax + output (warps 2..9 -> TMEM lane quadrants warp % 4) ----------------
         const int q = warp & 3;
-        const int r = q * 32 + lane;  // row within the tile
+        const int half = (warp - 2) >> 2;  // columns half*64 .. half*64+63 of S, P and O
+        const int r = q * 32 + lane;       // row within the tile
         const int i = i0 + r;
         const uint32_t lane_base = (uint32_t)(q * 32) << 16;
+        const uint32_t col0 = (uint32_t)half * 64;
         const float scale = LOG2E * 0.125f;  // log2(e) / sqrt(64)
         float m_used = -INFINITY, l = 0.f;
         bool ok = true;
+        // The two halves of a row meet at a named barrier once per block and once at the
+        // end. A failed wait never skips those barriers: the failing warp stops its work
+        // (ok = false, and the abort flag makes every later wait return at once) but
+        // still walks all nblk blocks, so both warps of a pair pass the same barriers.
         for (int j = 0; j < nblk; ++j) {
             const int sb = j & 1;
             int j0, rs, re;
             blk.get(j, &j0, &rs, &re);
             // tcgen05.ld/st are warp-collective: every decision that guards them is
             // taken by the whole warp (__all_sync / __any_sync)
-            if (!__all_sync(0xffffffffu, tc::mbar_wait(&s.s_full[sb], (j >> 1) & 1, abort))) {
+            if (ok && !__all_sync(0xffffffffu, tc::mbar_wait(&s.s_full[sb], (j >> 1) & 1, abort))) {
                 fail(abort, status, 2, j, 5);
                 ok = false;
-                break;
             }
-            tc::tc_fence_after();
-            float sv[KBLK];
-#pragma unroll
-            for (int c = 0; c < KBLK / 32; ++c) {
-                uint32_t rr[32];
-                tc::tmem_ld32(tmem + lane_base + 128 + sb * 128 + c * 32, rr);
-                tc::tmem_wait_ld();
-#pragma unroll
-                for (int e = 0; e < 32; ++e) sv[c * 32 + e] = __uint_as_float(rr[e]);
-            }
-            tc::tc_fence_before();
-            tc::mbar_arrive(&s.s_free[sb]);
-            // scale, mask, block max
-            const bool row_full = j0 >= rs && j0 + KBLK <= re && j0 + KBLK - 1 <= i &&
-                                  (j0 + KBLK <= n_meta || window <= 0 || i - j0 < window);
+            float sv[64];
             float mx = -INFINITY;
-            if (row_full) {
+            const int jb = j0 + (int)col0;
+            if (ok) {
+                tc::tc_fence_after();
+                {
+                    uint32_t ra[32], rb[32];
+                    tc::tmem_ld32(tmem + lane_base + 128 + sb * 128 + col0, ra);
+                    tc::tmem_ld32(tmem + lane_base + 128 + sb * 128 + col0 + 32, rb);
+                    tc::tmem_wait_ld();
 #pragma unroll
-                for (int c = 0; c < KBLK; ++c) {
-                    sv[c] *= scale;
-                    mx = fmaxf(mx, sv[c]);
+                    for (int e = 0; e < 32; ++e) {
+                        sv[e] = __uint_as_float(ra[e]);
+                        sv[32 + e] = __uint_as_float(rb[e]);
+                    }
                 }
-            } else {
+                tc::tc_fence_before();
+                tc::mbar_arrive(&s.s_free[sb]);
+                // mask, then the half-row max of the raw scores (the scale is positive). The
+                // keys row i sees in this block form one interval [a, e): the meta range
+                // [0, meta_end) or the window range [lo, hi), cut at i (causal) and, for
+                // window blocks, at i - W + 1; the test is one unsigned compare per key.
+                int a = rs, e = min(re, i + 1);
+                if (rs >= n_meta && window > 0) a = max(a, i - window + 1);
+                if (a > jb || e < jb + 64) {
+                    const unsigned span = e > a ? (unsigned)(e - a) : 0u;
 #pragma unroll
-                for (int c = 0; c < KBLK; ++c) {
-                    const int jk = j0 + c;
-                    const bool vis = jk >= rs && jk < re && jk <= i && (jk < n_meta || window <= 0 || i - jk < window);
-                    sv[c] = vis ? sv[c] * scale : -INFINITY;
-                    mx = fmaxf(mx, sv[c]);
+                    for (int c = 0; c < 64; ++c)
+                        sv[c] = (unsigned)(jb + c - a) < span ? sv[c] : -INFINITY;
                 }
+                float mx8[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) mx8[e] = sv[e];
+#pragma unroll
+                for (int c = 8; c < 64; c += 8)
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) mx8[e] = fmaxf(mx8[e], sv[c + e]);
+                mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                           fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
             }
+            // the row max over both halves: exchange through shared memory (double
+            // buffered by block parity, so a partner one block ahead never overwrites a
+            // value still to be read)
+            s.xmax[sb][half][r] = mx;
+            asm volatile("bar.sync %0, 64;" ::"r"(1 + q) : "memory");
+            if (!ok) continue;
+            mx = fmaxf(mx, s.xmax[sb][half ^ 1][r]) * scale;
             const float m_new = fmaxf(m_used, mx);
             // the P buffer of this block is free once PV[j-2] has completed
             if (j >= 2 && !__all_sync(0xffffffffu, tc::mbar_wait(&s.pv_done[sb], ((j - 2) >> 1) & 1, abort))) {
                 fail(abort, status, 2, j, 6);
                 ok = false;
-                break;
+                continue;
             }
             // rows whose running max grew by more than 2^8 move to the new max; their O row
-            // (PV[0..j-1]) is scaled by f in TMEM, the other rows of the warp by 1
+            // (PV[0..j-1]) is scaled by f in TMEM, each half its 64 columns
             float f = 1.f;
             bool scale_o = false;
             if (m_new > m_used + RESCALE_LOG2) {
@@ -247,50 +320,57 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
                 if (!__all_sync(0xffffffffu, tc::mbar_wait(&s.pv_done[(j - 1) & 1], ((j - 1) >> 1) & 1, abort))) {
                     fail(abort, status, 2, j, 7);
                     ok = false;
-                    break;
+                    continue;
                 }
                 tc::tc_fence_after();
 #pragma unroll 1
-                for (int c = 0; c < DV / 32; ++c) {
+                for (int c = 0; c < 2; ++c) {
                     uint32_t rr[32];
-                    tc::tmem_ld32(tmem + lane_base + c * 32, rr);
+                    tc::tmem_ld32(tmem + lane_base + col0 + c * 32, rr);
                     tc::tmem_wait_ld();
 #pragma unroll
                     for (int e = 0; e < 32; ++e) rr[e] = __float_as_uint(__uint_as_float(rr[e]) * f);
-                    tc::tmem_st32(tmem + lane_base + c * 32, rr);
+                    tc::tmem_st32(tmem + lane_base + col0 + c * 32, rr);
                 }
                 tc::tmem_wait_st();
             }
+            // P = 2^(s * scale - m) straight in fp16 pairs: the argument is rounded to fp16
+            // and exponentiated two at a time on the MUFU unit (P is stored in fp16 for the
+            // PV MMA in any case); it is at most 2^8 (the rescale threshold), far inside
+            // fp16's range. The row sum adds the same fp16 values in fp32.
             const float mu = m_used == -INFINITY ? 0.f : m_used;
-            uint8_t* prow = s.p[sb][0];
+            const float2 sc2 = make_float2(scale, scale), nmu2 = make_float2(-mu, -mu);
+            uint8_t* prow = s.p[sb][half] + r * 128;
+            float2 l4[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
-            for (int c8 = 0; c8 < KBLK / 8; ++c8) {
-                float pv[8];
+            for (int c8 = 0; c8 < 8; ++c8) {
+                uint32_t pk[4];
 #pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    pv[e] = fast_exp2(sv[c8 * 8 + e] - mu);
-                    l += pv[e];
+                for (int e = 0; e < 4; ++e) {
+                    const float2 x = __ffma2_rn(make_float2(sv[c8 * 8 + 2 * e], sv[c8 * 8 + 2 * e + 1]), sc2, nmu2);
+                    pk[e] = exp2_f16x2(pack_f16x2(x.x, x.y));
+                    l4[e] = __fadd2_rn(l4[e], __half22float2(*reinterpret_cast<const __half2*>(&pk[e])));
                 }
-                uint4 pk;
-                pk.x = pack_f16x2(pv[0], pv[1]);
-                pk.y = pack_f16x2(pv[2], pv[3]);
-                pk.z = pack_f16x2(pv[4], pv[5]);
-                pk.w = pack_f16x2(pv[6], pv[7]);
-                const int panel = c8 >> 3, ch = c8 & 7;
-                *reinterpret_cast<uint4*>(prow + panel * (QT * 128) + r * 128 + ((ch ^ (r & 7)) << 4)) = pk;
+                *reinterpret_cast<uint4*>(prow + ((c8 ^ (r & 7)) << 4)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
             }
+            const float2 l2 = __fadd2_rn(__fadd2_rn(l4[0], l4[1]), __fadd2_rn(l4[2], l4[3]));
+            l += l2.x + l2.y;
             tc::fence_proxy_async_smem();
             tc::tc_fence_before();
             tc::mbar_arrive(&s.p_full[sb]);
         }
+        // the row sum over both halves
+        s.xsum[half][r] = l;
+        asm volatile("bar.sync %0, 64;" ::"r"(1 + q) : "memory");
+        l += s.xsum[half ^ 1][r];
         if (ok && __all_sync(0xffffffffu, tc::mbar_wait(&s.o_done, 0, abort))) {
             tc::tc_fence_after();
             const float inv = l > 0.f ? 1.f / l : 0.f;
-            f16* orow = O + ((long long)b * Tp + i) * ((long long)H * DV) + h * DV;
+            f16* orow = O + ((long long)b * Tp + i) * ((long long)H * DV) + h * DV + col0;
 #pragma unroll 1
-            for (int c = 0; c < DV / 32; ++c) {
+            for (int c = 0; c < 2; ++c) {
                 uint32_t rr[32];
-                tc::tmem_ld32(tmem + lane_base + c * 32, rr);
+                tc::tmem_ld32(tmem + lane_base + col0 + c * 32, rr);
                 tc::tmem_wait_ld();
                 if (i < Tp) {
 #pragma unroll
