@@ -88,6 +88,7 @@ _sig = {
     "hymba_strerror": (ctypes.c_char_p, [ctypes.c_int]),
     "hymba_trace_enable": (ctypes.c_int, [ctypes.c_int]),
     "hymba_trace_collect": (ctypes.c_int, [_P(ctypes.c_char_p), _P(ctypes.c_float), ctypes.c_int]),
+    "hymba_trace_only": (ctypes.c_int, [ctypes.c_char_p]),
     "hymba_launch_count": (ctypes.c_uint64, []),
     "hymba_attn_decode_static": (ctypes.c_int, [_P(hymba_layer_cfg), _vp, ctypes.c_int64, _P(hymba_kv), _vp,
                                                 ctypes.c_int, _vp]),

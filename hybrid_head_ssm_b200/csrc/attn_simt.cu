@@ -19,6 +19,7 @@ __global__ void __launch_bounds__(256)
 attn_prefill_simt_kernel(const T* __restrict__ P, long long ldP, const T* __restrict__ kseq,
                          const T* __restrict__ vseq, int kcap, T* __restrict__ O, int Tp, int H,
                          int G, int n_meta, int window, float scale_log2) {
+    griddep_sync();
     __shared__ float Ks[KT][DH + 1];
     __shared__ float Vs[KT][DV + 1];
     const int i0 = blockIdx.x * QT, h = blockIdx.y, b = blockIdx.z;

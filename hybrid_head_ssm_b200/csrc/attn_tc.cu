@@ -134,6 +134,9 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
     tc::tc_fence_before();
     __syncthreads();
     tc::tc_fence_after();
+    // setup above touches no global memory; everything below may read the previous
+    // kernel's output
+    griddep_sync();
     const uint32_t tmem = s.tmem_base;  // O: columns 0..127, S buffers: 128..255, 256..383
     volatile int* abort = &s.abort;
 

@@ -5,6 +5,8 @@
 #include <cuda_fp16.h>
 #include <stdint.h>
 
+#include <utility>
+
 #include "../../include/hymba.h"
 
 namespace hymba {
@@ -21,15 +23,39 @@ struct Ctx {
     int sm_count;
 };
 
-void trace_before(const Ctx& ctx);
+// records the start event when tracing covers this kernel
+void trace_before(const Ctx& ctx, const char* name);
 // records the end event, counts the launch and checks the launch error; returns true on error
 bool trace_after(const Ctx& ctx, const char* name);
 
-#define HYMBA_LAUNCH(ctx, name, kernel, grid, block, smem, ...)                 \
-    do {                                                                        \
-        ::hymba::trace_before(ctx);                                             \
-        kernel<<<(grid), (block), (smem), (ctx).stream>>>(__VA_ARGS__);         \
-        if (::hymba::trace_after((ctx), (name))) return HYMBA_ERR_CUDA;         \
+// Every kernel of the library is launched with programmatic stream serialization
+// (programmatic dependent launch): its CTAs may start while the previous kernel on the
+// stream drains, run their setup (barrier init, TMEM allocation, tensor-map prefetch)
+// and then block in griddep_wait() until that kernel has completed and its writes are
+// visible. Each kernel calls griddep_wait() before its first global memory access and
+// then griddep_launch_dependents(), so the next kernel can be scheduled as SMs free up.
+template <typename... KArgs, typename... Args>
+static inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                                     cudaStream_t stream, Args&&... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
+#define HYMBA_LAUNCH(ctx, name, kernel, grid, block, smem, ...)                                  \
+    do {                                                                                         \
+        ::hymba::trace_before((ctx), (name));                                                    \
+        const cudaError_t launch_err_ =                                                          \
+            ::hymba::launch_pdl(kernel, dim3(grid), dim3(block), (size_t)(smem), (ctx).stream, __VA_ARGS__); \
+        if (::hymba::trace_after((ctx), (name)) || launch_err_ != cudaSuccess) return HYMBA_ERR_CUDA; \
     } while (0)
 
 static inline int ceil_div(long long a, long long b) { return (int)((a + b - 1) / b); }
@@ -46,6 +72,15 @@ template <typename T> __device__ __forceinline__ T from_f(float v);
 template <> __device__ __forceinline__ float from_f<float>(float v) { return v; }
 template <> __device__ __forceinline__ bf16 from_f<bf16>(float v) { return __float2bfloat16_rn(v); }
 template <> __device__ __forceinline__ f16 from_f<f16>(float v) { return __float2half_rn(v); }
+
+// Wait for the previous kernel on the stream (programmatic dependent launch), then let
+// the next one be scheduled. A no-op pair when the kernel was launched without it.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void griddep_sync() {
+    griddep_wait();
+    griddep_launch_dependents();
+}
 
 __device__ __forceinline__ void set_status(int* status, int code) {
     if (status) atomicCAS(status, 0, code);
@@ -86,7 +121,9 @@ __device__ __forceinline__ void store_run<float>(float* dst, const float* v, int
         for (int i = 0; i < 64; i += 4)
             *reinterpret_cast<float4*>(dst + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
     } else {
-        for (int i = 0; i < n; ++i) dst[i] = v[i];
+#pragma unroll
+        for (int i = 0; i < 64; ++i)
+            if (i < n) dst[i] = v[i];
     }
 }
 
@@ -118,7 +155,9 @@ __device__ __forceinline__ void store_run16(T* dst, const float* v, int n) {
             *reinterpret_cast<uint4*>(dst + i) = q;
         }
     } else {
-        for (int i = 0; i < n; ++i) dst[i] = from_f<T>(v[i]);
+#pragma unroll
+        for (int i = 0; i < 64; ++i)
+            if (i < n) dst[i] = from_f<T>(v[i]);
     }
 }
 

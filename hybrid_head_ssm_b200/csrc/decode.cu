@@ -51,6 +51,7 @@ attn_decode_kernel(const T* __restrict__ P, long long ldP, const T* __restrict__
                    const T* __restrict__ v_cache, int cap, const int* __restrict__ len,
                    int pos_offset, float* __restrict__ part, int n_split, int H, int G,
                    int n_meta, int window, int* status) {
+    griddep_sync();
     static_assert(DV == 16 * 8, "PV phase covers a V row with 16 pieces of 8");
     __shared__ __align__(16) float qs[MAX_R][DH];
     __shared__ float ps[MAX_R][MAX_CHUNK];
@@ -170,6 +171,7 @@ attn_decode_kernel(const T* __restrict__ P, long long ldP, const T* __restrict__
 template <typename T, int DV>
 __global__ void __launch_bounds__(DV)
 attn_decode_combine_kernel(const float* __restrict__ part, int n_split, T* __restrict__ O, int H) {
+    griddep_sync();
     const int h = blockIdx.x, b = blockIdx.y, e = threadIdx.x;
     const float* base = part + ((long long)b * H + h) * n_split * (DV + 2);
     float M = -INFINITY;
@@ -193,6 +195,7 @@ ssm_decode_kernel(const T* __restrict__ P, long long ldP, int col_x, int col_B, 
                   const float* __restrict__ conv_b, const float* __restrict__ A_log,
                   const float* __restrict__ Dp, float* __restrict__ h, float* __restrict__ conv,
                   T* __restrict__ ypre, int B, int di) {
+    griddep_sync();
     constexpr int NS = 16, KC = 4;
     const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
     if (idx >= (long long)B * di) return;

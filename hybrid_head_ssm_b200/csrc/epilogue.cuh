@@ -71,8 +71,45 @@ __device__ __forceinline__ float2 rope_cs_at(int p, int i, int dh, float base) {
     return make_float2((float)c, (float)s);
 }
 
+// v[0..n) += the residual run at src (16-byte loads when the run is full and aligned);
+// every index into v is a compile-time constant, so v stays in registers
+template <typename S>
+__device__ __forceinline__ void add_residual64(float* v, const S* src, int n) {
+    constexpr int PER = 16 / (int)sizeof(S);
+    if (n == 64 && (reinterpret_cast<uintptr_t>(src) & 15) == 0) {
+#pragma unroll
+        for (int j = 0; j < 64; j += PER) {
+            const uint4 u = *reinterpret_cast<const uint4*>(src + j);
+            const S* q = reinterpret_cast<const S*>(&u);
+#pragma unroll
+            for (int k = 0; k < PER; ++k) v[j + k] += to_f(q[k]);
+        }
+    } else {
+#pragma unroll
+        for (int j = 0; j < 64; ++j)
+            if (j < n) v[j] += to_f(src[j]);
+    }
+}
+
+// Where one row's run of (up to) 64 output columns goes: `count` copies `stride` bytes
+// apart (a meta row of the in-projection is written once per sequence), `nbytes` valid
+// bytes of elements of `esz` bytes (fp32 Delta, otherwise the output type).
+struct RunDst {
+    char* p;
+    long long stride;
+    int count;
+    int nbytes;
+    int esz;
+};
+
+// Everything the epilogue does to one run except the store: bias + softplus (Delta),
+// residual (output projection), RoPE (Q and K of the in-projection), and the run's
+// destination. count = 0 when the row has nothing to write.
 template <typename T>
-__device__ void epi_run64(const EpiArgs<T>& e, int r, int c0, float* v) {
+__device__ __forceinline__ RunDst epi_prepare64(const EpiArgs<T>& e, int r, int c0, float* v) {
+    // the element size depends on the launch only (the staged store relies on it being
+    // the same in every lane, rows without output included)
+    RunDst d{nullptr, 0, 0, 0, e.kind == EPI_DELTA ? 4 : (int)sizeof(T)};
     int mode = e.row_mode, M = e.M;
     if (e.meta_pad > 0) {
         if (r < e.meta_pad) {
@@ -82,45 +119,49 @@ __device__ void epi_run64(const EpiArgs<T>& e, int r, int c0, float* v) {
             r -= e.meta_pad;
         }
     }
-    if (r >= M || c0 >= e.N) return;
+    if (r >= M || c0 >= e.N) return d;
     const int n = min(64, e.N - c0);
     if (e.kind == EPI_DELTA) {
-        float* dst = e.delta + (long long)r * e.N + c0;
         const float* bias = e.b_dt + c0;
         if (n == 64 && (e.N & 3) == 0) {
+            float4 bb[16];
 #pragma unroll
-            for (int j = 0; j < 64; j += 4) {
-                const float4 bb = *reinterpret_cast<const float4*>(bias + j);
-                *reinterpret_cast<float4*>(dst + j) =
-                    make_float4(softplus_fast(v[j] + bb.x), softplus_fast(v[j + 1] + bb.y), softplus_fast(v[j + 2] + bb.z),
-                                softplus_fast(v[j + 3] + bb.w));
+            for (int j = 0; j < 16; ++j) bb[j] = reinterpret_cast<const float4*>(bias)[j];
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+                v[4 * j] = softplus_fast(v[4 * j] + bb[j].x);
+                v[4 * j + 1] = softplus_fast(v[4 * j + 1] + bb[j].y);
+                v[4 * j + 2] = softplus_fast(v[4 * j + 2] + bb[j].z);
+                v[4 * j + 3] = softplus_fast(v[4 * j + 3] + bb[j].w);
             }
         } else {
-            for (int j = 0; j < n; ++j) dst[j] = softplus_fast(v[j] + bias[j]);
+#pragma unroll
+            for (int j = 0; j < 64; ++j)
+                if (j < n) v[j] = softplus_fast(v[j] + bias[j]);
         }
-        return;
+        d.p = reinterpret_cast<char*>(e.delta + (long long)r * e.N + c0);
+        d.count = 1;
+        d.nbytes = n * 4;
+        return d;
     }
     if (e.kind == EPI_OUT) {
         if (e.res_mode == 1) {
-            const T* src = e.res_x + (long long)r * e.N + c0;
-            for (int j = 0; j < n; ++j) v[j] += to_f(src[j]);
+            add_residual64(v, e.res_x + (long long)r * e.N + c0, n);
         } else if (e.res_mode == 2) {
             int b = r / e.Tp, t = r % e.Tp;
             if (t < e.n_meta) {
-                if (e.res_meta_bf16) {
-                    const bf16* src = static_cast<const bf16*>(e.res_meta) + (long long)t * e.N + c0;
-                    for (int j = 0; j < n; ++j) v[j] += to_f(src[j]);
-                } else {
-                    const T* src = static_cast<const T*>(e.res_meta) + (long long)t * e.N + c0;
-                    for (int j = 0; j < n; ++j) v[j] += to_f(src[j]);
-                }
+                if (e.res_meta_bf16)
+                    add_residual64(v, static_cast<const bf16*>(e.res_meta) + (long long)t * e.N + c0, n);
+                else
+                    add_residual64(v, static_cast<const T*>(e.res_meta) + (long long)t * e.N + c0, n);
             } else {
-                const T* src = e.res_x + ((long long)b * e.Tu + (t - e.n_meta)) * e.N + c0;
-                for (int j = 0; j < n; ++j) v[j] += to_f(src[j]);
+                add_residual64(v, e.res_x + ((long long)b * e.Tu + (t - e.n_meta)) * e.N + c0, n);
             }
         }
-        store_run<T>(e.y + (long long)r * e.N + c0, v, n);
-        return;
+        d.p = reinterpret_cast<char*>(e.y + (long long)r * e.N + c0);
+        d.count = 1;
+        d.nbytes = n * (int)sizeof(T);
+        return d;
     }
     // EPI_INPROJ
     int b0, b1, t;
@@ -129,7 +170,7 @@ __device__ void epi_run64(const EpiArgs<T>& e, int r, int c0, float* v) {
     else if (mode == ROWS_USER) { b0 = r / e.Tu; b1 = b0 + 1; t = e.n_meta + r % e.Tu; }
     else {
         b0 = r; b1 = r + 1; t = e.pos[r] + e.pos_offset;
-        if (t < 0) return;  // no position to write; the decode attention reports the range error
+        if (t < 0) return d;  // no position to write; the decode attention reports the range error
     }
     const int qw = e.H * e.dh;
     const int kw = e.k_out ? e.G * e.dh : 0;
@@ -144,22 +185,101 @@ __device__ void epi_run64(const EpiArgs<T>& e, int r, int c0, float* v) {
             rope_run64(v, e.rope + (long long)t * 32);
         }
     }
-    for (int b = b0; b < b1; ++b) {
-        if (c0 >= qw && c0 < qw + kw) {
-            int g = (c0 - qw) / e.dh;
-            int slot = t;
-            if (mode == ROWS_DECODE && t >= e.n_meta) slot = e.n_meta + (t - e.n_meta) % e.n_meta_ring;
-            store_run<T>(e.k_out + (((long long)b * e.G + g) * e.kcap + slot) * e.dh, v, 64);
-        } else if (c0 >= qw + kw && c0 < qw + kw + vw) {
-            int cv = c0 - qw - kw;
-            int g = cv / e.dv, off = cv % e.dv;
-            int slot = t;
-            if (mode == ROWS_DECODE && t >= e.n_meta) slot = e.n_meta + (t - e.n_meta) % e.n_meta_ring;
-            store_run<T>(e.v_out + (((long long)b * e.G + g) * e.kcap + slot) * e.dv + off, v, 64);
-        } else {
-            long long row = mode == ROWS_DECODE ? b : (long long)b * e.Tp + t;
-            store_run<T>(e.P + row * e.ldP + c0, v, n);
+    d.count = b1 - b0;
+    if (c0 >= qw && c0 < qw + kw) {
+        const int g = (c0 - qw) / e.dh;
+        int slot = t;
+        if (mode == ROWS_DECODE && t >= e.n_meta) slot = e.n_meta + (t - e.n_meta) % e.n_meta_ring;
+        d.p = reinterpret_cast<char*>(e.k_out + (((long long)b0 * e.G + g) * e.kcap + slot) * e.dh);
+        d.stride = (long long)e.G * e.kcap * e.dh * (long long)sizeof(T);
+        d.nbytes = 64 * (int)sizeof(T);
+    } else if (c0 >= qw + kw && c0 < qw + kw + vw) {
+        const int cv = c0 - qw - kw;
+        const int g = cv / e.dv, off = cv % e.dv;
+        int slot = t;
+        if (mode == ROWS_DECODE && t >= e.n_meta) slot = e.n_meta + (t - e.n_meta) % e.n_meta_ring;
+        d.p = reinterpret_cast<char*>(e.v_out + (((long long)b0 * e.G + g) * e.kcap + slot) * e.dv + off);
+        d.stride = (long long)e.G * e.kcap * e.dv * (long long)sizeof(T);
+        d.nbytes = 64 * (int)sizeof(T);
+    } else {
+        const long long row = mode == ROWS_DECODE ? b0 : (long long)b0 * e.Tp + t;
+        d.p = reinterpret_cast<char*>(e.P + row * e.ldP + c0);
+        d.stride = (long long)e.Tp * e.ldP * (long long)sizeof(T);
+        d.nbytes = n * (int)sizeof(T);
+    }
+    return d;
+}
+
+// One thread stores its own row's run (CUDA-core GEMM).
+template <typename T>
+__device__ void epi_run64(const EpiArgs<T>& e, int r, int c0, float* v) {
+    const RunDst d = epi_prepare64<T>(e, r, c0, v);
+    for (int b = 0; b < d.count; ++b) {
+        char* p = d.p + b * d.stride;
+        if (d.esz == 4) store_run<float>(reinterpret_cast<float*>(p), v, d.nbytes / 4);
+        else store_run<T>(reinterpret_cast<T*>(p), v, d.nbytes / (int)sizeof(T));
+    }
+}
+
+// Shared-memory staging of one warp's 32 rows: 128 bytes per row and unit, rows padded
+// to 144 bytes so that both the per-row writes and the per-segment reads are free of
+// bank conflicts.
+constexpr int kStageRow = 144;
+constexpr int kStageWarpBytes = 32 * kStageRow;
+
+// Warp-collective store of the 32 rows' runs (lane l holds row l's values and RunDst):
+// each 128-byte unit (32 fp32 or 64 16-bit values) goes through shared memory so that
+// eight lanes write one row's 128 contiguous bytes with 16-byte stores, instead of each
+// lane writing its own row (32 rows, 32 cache lines per store instruction).
+template <typename T>
+__device__ __forceinline__ void epi_store_staged(const RunDst& d, const float* v, uint8_t* stage, RunDst* info, int lane) {
+    const int units = d.esz == 4 ? 2 : 1;  // esz is the same in every lane (one kind per launch)
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        if (h >= units) break;
+        uint4* srow = reinterpret_cast<uint4*>(stage + lane * kStageRow);
+        if (d.esz == 4) {
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+                srow[i] = make_uint4(__float_as_uint(v[h * 32 + 4 * i]), __float_as_uint(v[h * 32 + 4 * i + 1]),
+                                     __float_as_uint(v[h * 32 + 4 * i + 2]), __float_as_uint(v[h * 32 + 4 * i + 3]));
+        } else if constexpr (sizeof(T) == 2) {
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+                srow[i] = make_uint4(pack2<T>(v[8 * i], v[8 * i + 1]), pack2<T>(v[8 * i + 2], v[8 * i + 3]),
+                                     pack2<T>(v[8 * i + 4], v[8 * i + 5]), pack2<T>(v[8 * i + 6], v[8 * i + 7]));
         }
+        RunDst di = d;
+        di.p += h * 128;
+        di.nbytes = min(max(d.nbytes - h * 128, 0), 128);
+        if (di.nbytes == 0) di.count = 0;
+        info[lane] = di;
+        __syncwarp();
+#pragma unroll 1
+        for (int it = 0; it < 8; ++it) {
+            const int row = it * 4 + (lane >> 3), off = (lane & 7) * 16;
+            const RunDst ri = info[row];
+            if (ri.count > 0 && off < ri.nbytes) {
+                const uint4 val = *reinterpret_cast<const uint4*>(stage + row * kStageRow + off);
+                const bool vec = off + 16 <= ri.nbytes && ((reinterpret_cast<uintptr_t>(ri.p) | (uintptr_t)ri.stride) & 15) == 0;
+                for (int b = 0; b < ri.count; ++b) {
+                    char* dst = ri.p + b * ri.stride + off;
+                    if (vec) {
+                        *reinterpret_cast<uint4*>(dst) = val;
+                    } else {
+                        const uint8_t* src = reinterpret_cast<const uint8_t*>(&val);
+                        const int nb = min(16, ri.nbytes - off);
+                        if (ri.esz == 4)
+                            for (int k = 0; k < nb; k += 4)
+                                *reinterpret_cast<uint32_t*>(dst + k) = *reinterpret_cast<const uint32_t*>(src + k);
+                        else
+                            for (int k = 0; k < nb; k += 2)
+                                *reinterpret_cast<uint16_t*>(dst + k) = *reinterpret_cast<const uint16_t*>(src + k);
+                    }
+                }
+            }
+        }
+        __syncwarp();
     }
 }
 

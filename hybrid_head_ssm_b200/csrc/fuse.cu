@@ -61,6 +61,7 @@ __global__ void __launch_bounds__(TPR * RPB, 4)
 fuse_kernel(const I* __restrict__ O, const I* __restrict__ ypre, const I* __restrict__ P, long long ldP, int col_z,
             const float* __restrict__ g_attn, const float* __restrict__ g_ssm, const float* __restrict__ beta1,
             const float* __restrict__ beta2, T* __restrict__ U, int rows, int di, float eps, int* len_inc) {
+    griddep_sync();
     __shared__ float red[RPB][TPR / 32][2];
     const int sub = threadIdx.x / TPR, t = threadIdx.x % TPR;
     const long long row = (long long)blockIdx.x * RPB + sub;

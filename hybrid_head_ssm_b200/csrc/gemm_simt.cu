@@ -13,6 +13,7 @@ template <typename TA, typename TO>
 __global__ void __launch_bounds__(256)
 gemm_simt_kernel(const TA* __restrict__ A, long long lda, const TA* __restrict__ Bw, long long ldb,
                  int M, int N, int K, EpiArgs<TO> e) {
+    griddep_sync();
     __shared__ float As[TK][TM + 4];
     __shared__ float Bs[TK][TN + 4];
     __shared__ float Cs[TM][TN + 1];

@@ -83,6 +83,8 @@ struct GemmSmem {
     uint64_t tfull[2];
     uint64_t tempty[2];
     uint64_t drain;
+    alignas(16) uint8_t stage[4][kStageWarpBytes];  // epilogue warps' store staging
+    RunDst info[4][32];
     uint32_t tmem_base;
     int abort;
 };
@@ -131,6 +133,9 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     tc::tc_fence_before();
     __syncthreads();
     tc::tc_fence_after();
+    // setup above touches no global memory; everything below may read the previous
+    // kernel's output
+    griddep_sync();
     const uint32_t tmem = s.tmem_base;
     volatile int* abort = &s.abort;
 
@@ -216,7 +221,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
                     v[i] = __uint_as_float(r0[i]);
                     v[32 + i] = __uint_as_float(r1[i]);
                 }
-                epi_run64<TO>(e, row, n_blk * BN + j * 64, v);
+                const RunDst d = epi_prepare64<TO>(e, row, n_blk * BN + j * 64, v);
+                epi_store_staged<TO>(d, v, s.stage[q], s.info[q], lane);
             }
             tc::tc_fence_before();
             tc::mbar_arrive(&s.tempty[buf]);

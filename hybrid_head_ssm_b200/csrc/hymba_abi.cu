@@ -63,9 +63,12 @@ static std::vector<TraceRec> g_trace;
 static std::atomic<int> g_trace_used{0};
 static thread_local int t_trace_slot = -1;
 
-void trace_before(const Ctx& ctx) {
+static char g_trace_only[64] = {0};  // non-empty: trace only launches of this name
+
+void trace_before(const Ctx& ctx, const char* name) {
     t_trace_slot = -1;
     if (!g_trace_on.load(std::memory_order_relaxed)) return;
+    if (g_trace_only[0] && strcmp(g_trace_only, name) != 0) return;
     const int slot = g_trace_used.fetch_add(1);
     if (slot >= (int)g_trace.size()) return;
     t_trace_slot = slot;
@@ -605,6 +608,14 @@ int hymba_trace_enable(int on) {
     }
     g_trace_used.store(0);
     g_trace_on.store(on ? 1 : 0);
+    return HYMBA_OK;
+}
+
+int hymba_trace_only(const char* name) {
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (name && strlen(name) >= sizeof(g_trace_only)) return HYMBA_ERR_INVALID_ARG;
+    if (name) strcpy(g_trace_only, name);
+    else g_trace_only[0] = 0;
     return HYMBA_OK;
 }
 

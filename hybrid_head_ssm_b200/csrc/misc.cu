@@ -7,6 +7,7 @@ namespace hymba {
 namespace {
 
 __global__ void rope_table_kernel(float2* tab, int Tp, int half, int dh, float base) {
+    griddep_sync();
     const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
     if (idx >= (long long)Tp * half) return;
     const int p = (int)(idx / half), i = (int)(idx % half);
@@ -15,6 +16,7 @@ __global__ void rope_table_kernel(float2* tab, int Tp, int half, int dh, float b
 
 template <typename TS, typename TD>
 __global__ void pad_copy_kernel(const TS* src, int rows, int cols, TD* dst, int ld_dst) {
+    griddep_sync();
     const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
     if (idx >= (long long)rows * ld_dst) return;
     const int r = (int)(idx / ld_dst), c = (int)(idx % ld_dst);
@@ -27,6 +29,7 @@ template <typename T>
 __global__ void cache_fill_kernel(const T* k_seq, const T* v_seq, int seq_cap, T* k_cache,
                                   T* v_cache, int cache_cap, int* len, int G, int dh, int dv,
                                   int n_meta, int Tp) {
+    griddep_sync();
     const int ring = cache_cap - n_meta;
     const int first_kept = max(n_meta, Tp - ring);
     const int n_rows = min(n_meta, Tp) + max(0, Tp - first_kept);

@@ -127,6 +127,7 @@ conv_scan_prefill_kernel(const T* __restrict__ P, long long ldP, int col_x, int 
                          const float* __restrict__ conv_b, const float* __restrict__ A_log,
                          const float* __restrict__ Dp, T* __restrict__ ypre, float* __restrict__ h_out,
                          float* __restrict__ conv_out, int Tp, int di) {
+    griddep_sync();
     extern __shared__ __align__(16) uint8_t scan_smem[];
     ScanSmem<T>& sm = *reinterpret_cast<ScanSmem<T>*>(scan_smem);
     const int b = blockIdx.y, c0 = blockIdx.x * CPB;

@@ -283,6 +283,13 @@ const char* hymba_strerror(int code);
 int hymba_trace_enable(int on);
 int hymba_trace_collect(const char** names, float* ms, int max_records);
 
+/* Restrict tracing to the launches of one kernel name (as reported by
+ * hymba_trace_collect; at most 63 characters), or trace every launch again with
+ * NULL. Events between launches serialise the device-side overlap of consecutive
+ * kernels, so a timing run traces only the kernel it reports. Returns
+ * HYMBA_ERR_INVALID_ARG for a longer name. */
+int hymba_trace_only(const char* name);
+
 /* Number of kernels the library has queued since load (all entry points). */
 uint64_t hymba_launch_count(void);
 
