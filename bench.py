@@ -65,80 +65,103 @@ def roofline_entry(name, bound, units, avg_s, pk, sm_count, sm_mhz):
             "frac": ach / pk["hbm"], "peak_kind": f"HBM copy, {pk['src']}"}
 
 
-class Clocks:
-    """SM clocks and clock-event (throttle) reasons sampled through NVML every 2 ms
-    while the timed region is open (read-only queries; no setting is touched). The
-    samples also go to gpurun_out/clocks_rank<i>.csv."""
+CLOCK_SAMPLER = r"""
+import sys, time
+import pynvml as nv
+nv.nvmlInit()
+bus, index, path, stop = sys.argv[1], int(sys.argv[2]), sys.argv[3], sys.argv[4]
+try:
+    h = nv.nvmlDeviceGetHandleByPciBusId(bus.encode())
+except Exception:
+    h = nv.nvmlDeviceGetHandleByIndex(index)
+import os
+with open(path, "w", buffering=1) as f:
+    f.write("time,sm_mhz,sm_max_mhz,reasons_mask\n")
+    mx = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
+    n = 0
+    while True:
+        f.write(f"{time.time():.6f},{nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)},{mx},"
+                f"{nv.nvmlDeviceGetCurrentClocksEventReasons(h)}\n")
+        n += 1
+        if n % 64 == 0 and os.path.exists(stop):
+            break
+        time.sleep(0.0005)
+"""
 
-    REASONS = (("hw_slowdown", "nvmlClocksEventReasonHwSlowdown"),
-               ("hw_thermal_slowdown", "nvmlClocksEventReasonHwThermalSlowdown"),
-               ("sw_thermal_slowdown", "nvmlClocksEventReasonSwThermalSlowdown"),
-               ("sw_power_cap", "nvmlClocksEventReasonSwPowerCap"))
+
+class Clocks:
+    """SM clocks and clock-event (throttle) reasons through NVML (read-only queries; no
+    setting is touched), polled about every millisecond by a separate process so that
+    the polling does not compete with this one; only the samples taken while the timed
+    region is open (wall clock) are reported. The samples go to
+    gpurun_out/clocks_rank<i>.csv."""
+
+    REASONS = (("hw_slowdown", 0x8), ("hw_thermal_slowdown", 0x40), ("sw_thermal_slowdown", 0x20),
+               ("sw_power_cap", 0x4))
 
     def __init__(self, cuda_index: int):
         self.cuda_index = cuda_index
         self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{cuda_index}.csv")
-        self.samples = []
-        self.thread = None
-        self.open = threading.Event()
-        self.done = threading.Event()
-
-    def _handle(self, nv):
-        try:
-            pr = torch.cuda.get_device_properties(self.cuda_index)
-            return nv.nvmlDeviceGetHandleByPciBusId(
-                f"{pr.pci_domain_id:08X}:{pr.pci_bus_id:02X}:{pr.pci_device_id:02X}.0".encode())
-        except Exception:
-            return nv.nvmlDeviceGetHandleByIndex(self.cuda_index)
-
-    def _run(self, nv, hd, masks):
-        while not self.done.is_set():
-            if self.open.is_set():
-                try:
-                    sm = nv.nvmlDeviceGetClockInfo(hd, nv.NVML_CLOCK_SM)
-                    mx = nv.nvmlDeviceGetMaxClockInfo(hd, nv.NVML_CLOCK_SM)
-                    rs = nv.nvmlDeviceGetCurrentClocksEventReasons(hd)
-                    self.samples.append((time.time(), sm, mx, rs, [n for n, m in masks if rs & m]))
-                except Exception:
-                    pass
-            time.sleep(0.002)
+        self.stop_path = self.path + ".stop"
+        self.proc = None
+        self.t0 = self.t1 = None
 
     def start(self):
         try:
-            import pynvml as nv
-            nv.nvmlInit()
-            hd = self._handle(nv)
-            masks = [(n, getattr(nv, attr)) for n, attr in self.REASONS]
+            import pynvml  # noqa: F401
+            import torch
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            if os.path.exists(self.stop_path):
+                os.remove(self.stop_path)
+            pr = torch.cuda.get_device_properties(self.cuda_index)
+            bus = f"{pr.pci_domain_id:08X}:{pr.pci_bus_id:02X}:{pr.pci_device_id:02X}.0"
+            self.err = open(self.path + ".err", "w")
+            self.proc = subprocess.Popen([sys.executable, "-c", CLOCK_SAMPLER, bus, str(self.cuda_index), self.path,
+                                          self.stop_path], stdout=subprocess.DEVNULL, stderr=self.err)
+            # wait for the first samples so that the timed region is covered
+            for _ in range(400):
+                if os.path.exists(self.path) and sum(1 for _ in open(self.path)) > 3:
+                    break
+                time.sleep(0.01)
         except Exception:
-            return
-        self.thread = threading.Thread(target=self._run, args=(nv, hd, masks), daemon=True)
-        self.thread.start()
+            self.proc = None
 
     def begin(self):
-        self.open.set()
+        self.t0 = time.time()
 
     def end(self):
-        self.open.clear()
+        self.t1 = time.time()
 
     def stop(self):
-        if self.thread is None:
+        if self.proc is None:
             return None
-        self.done.set()
-        self.thread.join(timeout=5)
+        time.sleep(0.01)
+        open(self.stop_path, "w").close()
         try:
-            os.makedirs(os.path.dirname(self.path), exist_ok=True)
-            with open(self.path, "w") as f:
-                f.write("time,sm_mhz,sm_max_mhz,reasons_mask,reasons\n")
-                for t, sm, mx, rs, names in self.samples:
-                    f.write(f"{t:.4f},{sm},{mx},{rs:#x},{'|'.join(names)}\n")
-        except OSError:
-            pass
-        if not self.samples:
+            self.proc.wait(timeout=10)
+        except Exception:
+            self.proc.kill()
+        os.remove(self.stop_path)
+        rows = []
+        for line in open(self.path).read().splitlines()[1:]:
+            try:
+                t, sm, mx, rs = line.split(",")
+                rows.append((float(t), float(sm), float(mx), int(rs)))
+            except ValueError:
+                continue
+        inside = [r for r in rows if self.t0 is not None and self.t0 <= r[0] <= self.t1]
+        source = "NVML, separate process polling about every 1 ms, timed region only"
+        if not inside and rows and self.t0 is not None:
+            # region shorter than the polling interval: the samples just before and after it
+            before = [r for r in rows if r[0] < self.t0][-1:]
+            after = [r for r in rows if r[0] > self.t1][:1]
+            inside = before + after
+            source = "NVML, the samples adjacent to a timed region shorter than the polling interval"
+        if not inside:
             return None
-        reasons = sorted({n for *_, names in self.samples for n in names})
-        return {"sm_mhz": statistics.median(s[1] for s in self.samples),
-                "sm_max_mhz": max(s[2] for s in self.samples), "reasons": reasons,
-                "samples": len(self.samples), "source": "NVML, 2 ms, timed region only"}
+        reasons = sorted({n for r in inside for n, m in self.REASONS if r[3] & m})
+        return {"sm_mhz": statistics.median(r[1] for r in inside), "sm_max_mhz": max(r[2] for r in inside),
+                "reasons": reasons, "samples": len(inside), "source": source}
 
 
 def visible_pairs(Tp, m, W):
@@ -290,9 +313,11 @@ def main():
     flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")  # > 126 MB L2
     stream = torch.cuda.current_stream()
 
-    def step():
-        rt.prefill(layer, x, T, kv, y, ws, None, 0)
+    def step(xin=None, yout=None):
+        rt.prefill(layer, x if xin is None else xin, T, kv, y if yout is None else yout, ws, None, 0)
 
+    clocks = Clocks(local)
+    clocks.start()
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
@@ -335,8 +360,6 @@ def main():
     dom = max(per, key=lambda n: sum(per[n]))
 
     # ---- timed region: K steps; only the dominant kernel is bracketed by events
-    clocks = Clocks(local)
-    clocks.start()
     launches0 = hy.hymba_launch_count()
     step_ms, trace_dom = run_steps(args.steps, traced_only=dom, timed=True)
     launches = hy.hymba_launch_count() - launches0
@@ -357,22 +380,49 @@ def main():
             r = roofline_entry(n, bd, u, sum(per[n]) / len(per[n]) * 1e-3, pk, sm_count, sm_mhz)
             kern[n]["achieved"], kern[n]["unit"], kern[n]["frac"] = r["achieved"], r["unit"], r["frac"]
 
-    # ---- end to end through the public API with host buffers
+    # ---- end to end through the public API with host buffers: each step uploads its
+    # input from pinned host memory, runs the layer and downloads the output; uploads,
+    # compute and downloads go on three streams with two device buffer sets, so step
+    # i+1's upload and step i-1's download overlap step i's compute. Timed with device
+    # events from the first upload to the last download.
     x_host = x.cpu().pin_memory()
-    y_host = torch.empty(y.shape, dtype=y.dtype).pin_memory()
-    e2e_ms = []
-    for i in range(args.warmup + args.steps):
-        flush.fill_(i & 0xFF)
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record(stream)
-        x.copy_(x_host, non_blocking=True)
-        step()
-        y_host.copy_(y, non_blocking=True)
-        b.record(stream)
+    y_host = [torch.empty(y.shape, dtype=y.dtype).pin_memory() for _ in range(2)]
+    xs, ys = [x, torch.empty_like(x)], [y, torch.empty_like(y)]
+    up, down = torch.cuda.Stream(), torch.cuda.Stream()
+
+    def e2e_run(n):
+        ev = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
+        t_start, t_end = ev(), ev()
+        uploaded = [torch.cuda.Event(), torch.cuda.Event()]
+        computed = [torch.cuda.Event(), torch.cuda.Event()]
+        downloaded = [torch.cuda.Event(), torch.cuda.Event()]
+        used = [False, False]
         torch.cuda.synchronize()
-        if i >= args.warmup:
-            e2e_ms.append(a.elapsed_time(b))
-    e2e_ms_step = max_ranks(sum(e2e_ms) / len(e2e_ms))
+        t_start.record(up)
+        for i in range(n):
+            k = i & 1
+            with torch.cuda.stream(up):
+                if used[k]:
+                    up.wait_event(computed[k])  # the compute of step i-2 has read xs[k]
+                xs[k].copy_(x_host, non_blocking=True)
+                uploaded[k].record(up)
+            stream.wait_event(uploaded[k])
+            if used[k]:
+                stream.wait_event(downloaded[k])  # ys[k] of step i-2 is on the host
+            step(xs[k], ys[k])
+            computed[k].record(stream)
+            with torch.cuda.stream(down):
+                down.wait_event(computed[k])
+                y_host[k].copy_(ys[k], non_blocking=True)
+                downloaded[k].record(down)
+            used[k] = True
+        down.wait_event(computed[(n - 1) & 1])
+        t_end.record(down)
+        torch.cuda.synchronize()
+        return t_start.elapsed_time(t_end) / n
+
+    e2e_run(args.warmup)
+    e2e_ms_step = max_ranks(e2e_run(args.steps))
 
     # ---- decode step of the KV-sharing pair (B=64, ring 1024 + 128 meta)
     dec = None
