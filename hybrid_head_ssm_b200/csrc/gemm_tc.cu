@@ -72,9 +72,11 @@ bool make_tmap_3d(CUtensorMap* map, const void* base, bool is_bf16, uint64_t pla
 
 namespace {
 
-constexpr int BM = 128, BK = 64, STAGES = 4, NUM_THREADS = 192;
+constexpr int BM = 128, BK = 64, NUM_THREADS = 192;
 
-template <int BN>
+// STAGES-deep operand ring; GEMMs of at most two k-blocks use two stages, which leaves
+// room for two CTAs per SM (their epilogues, the bulk of such a GEMM, then overlap)
+template <int BN, int STAGES>
 struct GemmSmem {
     alignas(1024) uint8_t a[STAGES][BM * BK * 2];
     alignas(1024) uint8_t b[STAGES][BN * BK * 2];
@@ -94,12 +96,12 @@ __device__ __forceinline__ void fail(volatile int* abort, int* status, int role,
     tc::record_timeout(status, role, step, bar);
 }
 
-template <typename TA, typename TO, int BN>
-__global__ void __launch_bounds__(NUM_THREADS, 1)
+template <typename TA, typename TO, int BN, int STAGES>
+__global__ void __launch_bounds__(NUM_THREADS, STAGES == 2 ? 2 : 1)
 gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                const __grid_constant__ CUtensorMap tmA0, int M0, int M, int N, int K, EpiArgs<TO> e, int* status) {
     extern __shared__ uint8_t smem_raw[];
-    GemmSmem<BN>& s = *reinterpret_cast<GemmSmem<BN>*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+    GemmSmem<BN, STAGES>& s = *reinterpret_cast<GemmSmem<BN, STAGES>*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                         ~static_cast<uintptr_t>(1023));
     constexpr bool kBF16 = sizeof(TA) == 2 && std::is_same<TA, bf16>::value;
     constexpr uint32_t IDESC = tc::idesc_f16(kBF16, BM, BN);
@@ -236,7 +238,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     }
 }
 
-template <typename TA, typename TO, int BN>
+template <typename TA, typename TO, int BN, int STAGES>
 int launch_bn(const Ctx& ctx, const char* name, const TA* A, long long lda, const TA* Bw, long long ldb, int M,
               int N, int K, const EpiArgs<TO>& e, const TA* A0, int M0) {
     constexpr bool kBF16 = std::is_same<TA, bf16>::value;
@@ -248,8 +250,8 @@ int launch_bn(const Ctx& ctx, const char* name, const TA* A, long long lda, cons
     } else {
         ta0 = ta;
     }
-    const size_t smem = sizeof(GemmSmem<BN>) + 1024;
-    auto kern = gemm_tc_kernel<TA, TO, BN>;
+    const size_t smem = sizeof(GemmSmem<BN, STAGES>) + 1024;
+    auto kern = gemm_tc_kernel<TA, TO, BN, STAGES>;
     static bool attr_set = false;
     if (!attr_set) {
         if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
@@ -257,7 +259,8 @@ int launch_bn(const Ctx& ctx, const char* name, const TA* A, long long lda, cons
         attr_set = true;
     }
     const int tiles = ((M0 + BM - 1) / BM + (M + BM - 1) / BM) * ((N + BN - 1) / BN);
-    const int grid = tiles < ctx.sm_count ? tiles : ctx.sm_count;
+    const int slots = ctx.sm_count * (STAGES == 2 ? 2 : 1);
+    const int grid = tiles < slots ? tiles : slots;
     EpiArgs<TO> e2 = e;
     e2.meta_pad = ((M0 + BM - 1) / BM) * BM;
     e2.meta_M = M0;
@@ -290,9 +293,13 @@ int launch_gemm_tc(const Ctx& ctx, const char* name, const TA* A, long long lda,
     if (M <= 0 || N <= 0) return HYMBA_OK;
     if (M0 > 0 && (!A0 || ((uintptr_t)A0 & 15))) return HYMBA_ERR_INVALID_ARG;
     switch (pick_bn(M + M0, N, ctx.sm_count > 0 ? ctx.sm_count : 148)) {
-        case 256: return launch_bn<TA, TO, 256>(ctx, name, A, lda, Bw, ldb, M, N, K, e, A0, M0);
-        case 128: return launch_bn<TA, TO, 128>(ctx, name, A, lda, Bw, ldb, M, N, K, e, A0, M0);
-        default: return launch_bn<TA, TO, 64>(ctx, name, A, lda, Bw, ldb, M, N, K, e, A0, M0);
+        case 256: return launch_bn<TA, TO, 256, 4>(ctx, name, A, lda, Bw, ldb, M, N, K, e, A0, M0);
+        case 128:
+            if (K <= 2 * BK) return launch_bn<TA, TO, 128, 2>(ctx, name, A, lda, Bw, ldb, M, N, K, e, A0, M0);
+            return launch_bn<TA, TO, 128, 4>(ctx, name, A, lda, Bw, ldb, M, N, K, e, A0, M0);
+        default:
+            if (K <= 2 * BK) return launch_bn<TA, TO, 64, 2>(ctx, name, A, lda, Bw, ldb, M, N, K, e, A0, M0);
+            return launch_bn<TA, TO, 64, 4>(ctx, name, A, lda, Bw, ldb, M, N, K, e, A0, M0);
     }
 }
 
