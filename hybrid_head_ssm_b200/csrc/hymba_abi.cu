@@ -277,7 +277,10 @@ static int prefill_impl(const Ctx& ctx, const hymba_layer_cfg* c, const hymba_la
         meta = static_cast<const T*>(w->meta);
         W_out = static_cast<const T*>(w->w_out);
     }
-    if ((rc = launch_rope_table(ctx, rope, Tp, dh, c->rope_base))) return rc;
+    // RoPE table and the padded 16-bit W_dt of step 2, one launch
+    if ((rc = launch_prefill_prep<T, I>(ctx, rope, Tp, dh, c->rope_base, static_cast<const T*>(w->w_dt), di,
+                                        c->dt_rank, wdt, pl.rpad)))
+        return rc;
     // 1. fused input projection (+ RoPE, K/V scatter) ------------------------------
     EpiArgs<I> ep = epi_base<I>(EPI_INPROJ, 0, k.n_in);
     ep.B = B; ep.Tu = T_; ep.Tp = Tp; ep.n_meta = m;
@@ -314,7 +317,6 @@ static int prefill_impl(const Ctx& ctx, const hymba_layer_cfg* c, const hymba_la
         }
     }
     // 2. Delta = softplus(dt_low W_dt^T + b_dt) ------------------------------------
-    if ((rc = launch_pad_copy<T, I>(ctx, static_cast<const T*>(w->w_dt), di, c->dt_rank, wdt, pl.rpad))) return rc;
     EpiArgs<I> ed = epi_base<I>(EPI_DELTA, (int)rows, di);
     ed.delta = delta; ed.b_dt = w->b_dt;
     if ((rc = gemm<I, I>(ctx, "gemm_dt_proj", P + k.dtl, pl.ldP, wdt, pl.rpad, (int)rows, di, c->dt_rank, ed))) return rc;

@@ -46,8 +46,12 @@ int launch_fuse(const Ctx& ctx, const I* O, const I* ypre, const I* P, long long
                 const float* g_attn, const float* g_ssm, const float* beta1, const float* beta2,
                 T* U, int rows, int di, float eps, int* len_inc);
 
-// cos/sin table of RoPE for positions 0..Tp-1 (angles in double precision).
-int launch_rope_table(const Ctx& ctx, float2* tab, int Tp, int dh, float base);
+
+// The RoPE table and the zero-padded 16-bit copy of W_dt [rows, cols] -> [rows, ld_dst],
+// in one launch.
+template <typename TS, typename TD>
+int launch_prefill_prep(const Ctx& ctx, float2* tab, int Tp, int dh, float base, const TS* w, int rows, int cols,
+                        TD* wdst, int ld_dst);
 
 // Copy a [rows, cols] matrix into a zero-padded [rows, ld_dst] one of type TD.
 template <typename TS, typename TD>

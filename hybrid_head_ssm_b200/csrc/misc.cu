@@ -1,18 +1,11 @@
-// Small data-movement kernels around the mixer: the RoPE angle table, zero-padded
-// weight copies for TMA-aligned strides, and the decode-cache fill after a prefill.
+// Small data-movement kernels around the mixer: the RoPE angle table with the padded
+// W_dt copy of a prefill, zero-padded weight copies for TMA-aligned strides, and the
+// decode-cache fill after a prefill.
 #include "kernels.h"
 
 namespace hymba {
 
 namespace {
-
-__global__ void rope_table_kernel(float2* tab, int Tp, int half, int dh, float base) {
-    griddep_sync();
-    const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-    if (idx >= (long long)Tp * half) return;
-    const int p = (int)(idx / half), i = (int)(idx % half);
-    tab[idx] = rope_cs_at(p, i, dh, base);
-}
 
 template <typename TS, typename TD>
 __global__ void pad_copy_kernel(const TS* src, int rows, int cols, TD* dst, int ld_dst) {
@@ -21,6 +14,25 @@ __global__ void pad_copy_kernel(const TS* src, int rows, int cols, TD* dst, int 
     if (idx >= (long long)rows * ld_dst) return;
     const int r = (int)(idx / ld_dst), c = (int)(idx % ld_dst);
     dst[idx] = from_f<TD>(c < cols ? to_f(src[(long long)r * cols + c]) : 0.f);
+}
+
+// The two small inputs of a prefill in one launch: blocks [0, nb_rope) fill the RoPE
+// table, the rest copy W_dt into its zero-padded 16-bit form.
+template <typename TS, typename TD>
+__global__ void prefill_prep_kernel(float2* tab, int Tp, int half, int dh, float base, int nb_rope, const TS* w,
+                                    int rows, int cols, TD* wdst, int ld_dst) {
+    griddep_sync();
+    if ((int)blockIdx.x < nb_rope) {
+        const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+        if (idx >= (long long)Tp * half) return;
+        const int p = (int)(idx / half), i = (int)(idx % half);
+        tab[idx] = rope_cs_at(p, i, dh, base);
+    } else {
+        const long long idx = (long long)(blockIdx.x - nb_rope) * blockDim.x + threadIdx.x;
+        if (idx >= (long long)rows * ld_dst) return;
+        const int r = (int)(idx / ld_dst), c = (int)(idx % ld_dst);
+        wdst[idx] = from_f<TD>(c < cols ? to_f(w[(long long)r * cols + c]) : 0.f);
+    }
 }
 
 // Slot of position p: meta positions keep their slot, the others wrap in a ring of
@@ -48,17 +60,22 @@ __global__ void cache_fill_kernel(const T* k_seq, const T* v_seq, int seq_cap, T
 
 }  // namespace
 
-int launch_rope_table(const Ctx& ctx, float2* tab, int Tp, int dh, float base) {
-    const long long n = (long long)Tp * (dh / 2);
-    HYMBA_LAUNCH(ctx, "rope_table", rope_table_kernel, ceil_div(n, 256), 256, 0, tab, Tp, dh / 2, dh, base);
-    return HYMBA_OK;
-}
-
 template <typename TS, typename TD>
 int launch_pad_copy(const Ctx& ctx, const TS* src, int rows, int cols, TD* dst, int ld_dst) {
     const long long n = (long long)rows * ld_dst;
     auto kern = pad_copy_kernel<TS, TD>;
     HYMBA_LAUNCH(ctx, "pad_copy", kern, ceil_div(n, 256), 256, 0, src, rows, cols, dst, ld_dst);
+    return HYMBA_OK;
+}
+
+template <typename TS, typename TD>
+int launch_prefill_prep(const Ctx& ctx, float2* tab, int Tp, int dh, float base, const TS* w, int rows, int cols,
+                        TD* wdst, int ld_dst) {
+    const int nb_rope = ceil_div((long long)Tp * (dh / 2), 256);
+    const int nb_pad = ceil_div((long long)rows * ld_dst, 256);
+    auto kern = prefill_prep_kernel<TS, TD>;
+    HYMBA_LAUNCH(ctx, "prefill_prep", kern, nb_rope + nb_pad, 256, 0, tab, Tp, dh / 2, dh, base, nb_rope, w, rows,
+                 cols, wdst, ld_dst);
     return HYMBA_OK;
 }
 
@@ -76,6 +93,9 @@ template int launch_pad_copy<float, float>(const Ctx&, const float*, int, int, f
 template int launch_pad_copy<float, bf16>(const Ctx&, const float*, int, int, bf16*, int);
 template int launch_pad_copy<float, f16>(const Ctx&, const float*, int, int, f16*, int);
 template int launch_pad_copy<bf16, f16>(const Ctx&, const bf16*, int, int, f16*, int);
+template int launch_prefill_prep<float, float>(const Ctx&, float2*, int, int, float, const float*, int, int, float*,
+                                               int);
+template int launch_prefill_prep<bf16, f16>(const Ctx&, float2*, int, int, float, const bf16*, int, int, f16*, int);
 template int launch_cache_fill<float>(const Ctx&, const float*, const float*, int, float*, float*,
                                       int, int*, int, int, int, int, int, int);
 template int launch_cache_fill<f16>(const Ctx&, const f16*, const f16*, int, f16*, f16*, int,
