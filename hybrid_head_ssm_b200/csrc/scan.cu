@@ -10,15 +10,20 @@
 //       two MUFU exp2 and four FMA-pipe instructions and the only serial dependency is
 //       one FFMA2; each step's partial C.h sum goes to shared memory;
 //   helper warps (64 threads, two per row): cp.async staging of the rows, conv + SiLU,
-//       the operand quads (Delta, Delta, Delta*xc, Delta*xc) and (B, B, C, C) that the
-//       scan reads with one 16-byte load each, and the reduction y = sum of the 8 partial
-//       sums + D xc.
+//       the scan's operands and the reduction y = sum of the 8 partial sums + D xc.
+// The scan warps are bound by shared-memory bandwidth (a 16-byte load costs four
+// wavefronts even when it is a broadcast), so the operands are packed for the fewest
+// wavefronts per step: one 16-byte (Delta_t, Delta_t xc_t, Delta_t+1, Delta_t+1 xc_t+1)
+// load serves two steps, and B_2p, B_2p+1, C_2p, C_2p+1 stay the fp16 values of the
+// projection (one 8-byte load, converted in registers).
 // Time is walked in chunks of 32 rows with one block barrier per chunk: while the scan
 // warps scan chunk k, the helpers stage chunk k+2, reduce chunk k-1 and unpack chunk
 // k+1, so the recurrence never waits for the preparation or the reduction. Raw rows are
 // triple-buffered, operands and partial sums double-buffered. A chunk's x rows sit after
 // three halo rows (the previous chunk's last three, zero before the sequence), so the
 // causal conv needs no branches; shared-memory rows are padded against bank conflicts.
+#include <type_traits>
+
 #include "kernels.h"
 
 namespace hymba {
@@ -60,11 +65,16 @@ struct Raw {
     alignas(16) T c[TC][16];
 };
 
+// (B_2p, B_2p+1, C_2p, C_2p+1) of a row: fp16 inputs keep their four halves (8 bytes,
+// converted in the scan), fp32 inputs four floats
+template <typename T>
+using BcEl = typename std::conditional<sizeof(T) == 2, uint2, float4>::type;
+
 template <typename T>
 struct Smem {
     Raw<T> raw[NRAW];
-    alignas(16) float4 dd[2][TC][CPB + 1];
-    alignas(16) float4 bc[2][TC][TPC + 1];
+    alignas(16) float4 dd[2][TC / 2][CPB + 1];  // (d_t, dv_t, d_t+1, dv_t+1) per row pair
+    alignas(16) BcEl<T> bc[2][TC][TPC + 1];
     alignas(16) float xd[2][TC][12];
     alignas(16) float part[2][CPB * PCS];
     alignas(16) float2 w2[KC + 2][CPB / 2];
@@ -124,8 +134,8 @@ __device__ __forceinline__ void stage_chunk(Raw<T>& r, int h, const T* P, long l
 }
 
 // Helper thread h: unpack row h >> 1 of the chunk in r, for channels (and state pairs)
-// 4 * (h & 1) .. +3: conv + SiLU, (Delta, Delta, Delta*xc, Delta*xc) quads, D xc and
-// (B, B, C, C) quads into operand buffer `buf`.
+// 4 * (h & 1) .. +3: conv + SiLU, the (Delta, Delta*xc) pairs, D xc and the B/C quads
+// into operand buffer `buf`.
 template <typename T>
 __device__ __forceinline__ void unpack_chunk(Smem<T>& sm, const Raw<T>& r, int buf, int h, int nt) {
     const int t = h >> 1, hf = h & 1;
@@ -147,16 +157,26 @@ __device__ __forceinline__ void unpack_chunk(Smem<T>& sm, const Raw<T>& r, int b
         const float2 den = __fadd2_rn(e, make_float2(1.f, 1.f));
         const float2 xc = __fmul2_rn(acc[j], make_float2(rcp_approx(den.x), rcp_approx(den.y)));
         const float2 dv = __fmul2_rn(dl[j], xc);
-        sm.dd[buf][t][4 * hf + 2 * j] = make_float4(dl[j].x, dl[j].x, dv.x, dv.x);
-        sm.dd[buf][t][4 * hf + 2 * j + 1] = make_float4(dl[j].y, dl[j].y, dv.y, dv.y);
+        float2* d2 = reinterpret_cast<float2*>(&sm.dd[buf][t >> 1][0]) + (t & 1);
+        d2[2 * (4 * hf + 2 * j)] = make_float2(dl[j].x, dv.x);
+        d2[2 * (4 * hf + 2 * j + 1)] = make_float2(dl[j].y, dv.y);
         xdv[j] = __fmul2_rn(sm.w2[KC + 1][2 * hf + j], xc);
     }
     *reinterpret_cast<float4*>(&sm.xd[buf][t][4 * hf]) = make_float4(xdv[0].x, xdv[0].y, xdv[1].x, xdv[1].y);
-    float2 bv[4], cv[4];
-    load8x2<T>(&r.b[t][8 * hf], bv);
-    load8x2<T>(&r.c[t][8 * hf], cv);
+    if constexpr (sizeof(T) == 2) {
+        const uint4 bw = *reinterpret_cast<const uint4*>(&r.b[t][8 * hf]);
+        const uint4 cw = *reinterpret_cast<const uint4*>(&r.c[t][8 * hf]);
+        sm.bc[buf][t][4 * hf + 0] = make_uint2(bw.x, cw.x);
+        sm.bc[buf][t][4 * hf + 1] = make_uint2(bw.y, cw.y);
+        sm.bc[buf][t][4 * hf + 2] = make_uint2(bw.z, cw.z);
+        sm.bc[buf][t][4 * hf + 3] = make_uint2(bw.w, cw.w);
+    } else {
+        float2 bv[4], cv[4];
+        load8x2<T>(&r.b[t][8 * hf], bv);
+        load8x2<T>(&r.c[t][8 * hf], cv);
 #pragma unroll
-    for (int q = 0; q < 4; ++q) sm.bc[buf][t][4 * hf + q] = make_float4(bv[q].x, bv[q].y, cv[q].x, cv[q].y);
+        for (int q = 0; q < 4; ++q) sm.bc[buf][t][4 * hf + q] = make_float4(bv[q].x, bv[q].y, cv[q].x, cv[q].y);
+    }
 }
 
 // Helper thread h: y of row h >> 1 for channels 4 * (h & 1) .. +3 = the 8 partial C.h
@@ -237,30 +257,44 @@ conv_scan_prefill_kernel(const T* __restrict__ P, long long ldP, int col_x, int 
         const int buf = k & 1;
         if (scanner) {
             float* pw = sm.part[buf] + cl * PCS + p;
-            float4 qd[2][GS], qb[2][GS];
+            float4 qd[2][GS / 2];
+            BcEl<T> qb[2][GS];
 #pragma unroll
-            for (int u = 0; u < GS; ++u) {
-                qd[0][u] = sm.dd[buf][u][cl];
-                qb[0][u] = sm.bc[buf][u][p];
-            }
+            for (int u = 0; u < GS; ++u) qb[0][u] = sm.bc[buf][u][p];
+#pragma unroll
+            for (int u = 0; u < GS / 2; ++u) qd[0][u] = sm.dd[buf][u][cl];
 #pragma unroll
             for (int g = 0; g < TC / GS; ++g) {
                 const int cur = g & 1;
                 if (g + 1 < TC / GS) {
 #pragma unroll
-                    for (int u = 0; u < GS; ++u) {
-                        qd[cur ^ 1][u] = sm.dd[buf][(g + 1) * GS + u][cl];
-                        qb[cur ^ 1][u] = sm.bc[buf][(g + 1) * GS + u][p];
-                    }
+                    for (int u = 0; u < GS; ++u) qb[cur ^ 1][u] = sm.bc[buf][(g + 1) * GS + u][p];
+#pragma unroll
+                    for (int u = 0; u < GS / 2; ++u) qd[cur ^ 1][u] = sm.dd[buf][(g + 1) * (GS / 2) + u][cl];
+                }
+                float dstep[GS], dvstep[GS];
+#pragma unroll
+                for (int u = 0; u < GS / 2; ++u) {
+                    dstep[2 * u] = qd[cur][u].x;
+                    dvstep[2 * u] = qd[cur][u].y;
+                    dstep[2 * u + 1] = qd[cur][u].z;
+                    dvstep[2 * u + 1] = qd[cur][u].w;
                 }
                 float2 a[GS];
 #pragma unroll
-                for (int u = 0; u < GS; ++u) a[u] = exp2_pair(__fmul2_rn(make_float2(qd[cur][u].x, qd[cur][u].y), A2));
+                for (int u = 0; u < GS; ++u) a[u] = exp2_pair(__fmul2_rn(make_float2(dstep[u], dstep[u]), A2));
 #pragma unroll
                 for (int u = 0; u < GS; ++u) {
-                    const float4 q = qb[cur][u];
-                    hs = __ffma2_rn(a[u], hs, __fmul2_rn(make_float2(qd[cur][u].z, qd[cur][u].w), make_float2(q.x, q.y)));
-                    const float2 ch = __fmul2_rn(make_float2(q.z, q.w), hs);
+                    float2 Bq, Cq;
+                    if constexpr (sizeof(T) == 2) {
+                        Bq = __half22float2(*reinterpret_cast<const __half2*>(&qb[cur][u].x));
+                        Cq = __half22float2(*reinterpret_cast<const __half2*>(&qb[cur][u].y));
+                    } else {
+                        Bq = make_float2(qb[cur][u].x, qb[cur][u].y);
+                        Cq = make_float2(qb[cur][u].z, qb[cur][u].w);
+                    }
+                    hs = __ffma2_rn(a[u], hs, __fmul2_rn(make_float2(dvstep[u], dvstep[u]), Bq));
+                    const float2 ch = __fmul2_rn(Cq, hs);
                     pw[(g * GS + u) * TPC] = ch.x + ch.y;
                 }
             }
