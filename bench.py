@@ -16,6 +16,7 @@ bounded sample of the same workload.
 from __future__ import annotations
 
 import argparse
+import hashlib
 import json
 import os
 import statistics
@@ -45,6 +46,21 @@ def peaks():
         return dict(hbm=d["hbm_gbs"], bf16=d["bf16_tflops"], bf16_sus=d["bf16_tflops_sustained"],
                     sm_mhz=d.get("sm_max_mhz", 1965.0), src="measured")
     return dict(hbm=6650.0, bf16=1590.0, bf16_sus=1400.0, sm_mhz=1965.0, src="fallback")
+
+
+def kernel_traffic(name, workload):
+    """DRAM bytes per launch of a kernel from the committed ncu record (profiles/), or
+    None when there is none for this workload or the kernel's source changed since."""
+    try:
+        rec = json.load(open(os.path.join(ROOT, "profiles", "dram_traffic.json"))).get(name)
+        if not rec or rec.get("workload") != workload:
+            return None
+        src = open(os.path.join(ROOT, rec["kernel_source"]), "rb").read()
+        if hashlib.sha1(src).hexdigest() != rec["kernel_source_sha1"]:
+            return None
+        return rec["bytes_per_launch"]
+    except (OSError, ValueError, KeyError):
+        return None
 
 
 def roofline_entry(name, bound, units, avg_s, pk, sm_count, sm_mhz):
@@ -374,7 +390,9 @@ def main():
     bound, units = work.get(dom, ("hbm", 0.0))
     roof = roofline_entry(dom, bound, units, sum(dom_t) / len(dom_t) * 1e-3, pk, sm_count, sm_mhz)
     roof["launches_timed"] = len(dom_t)
-    roof["traffic"] = None
+    roof["traffic"] = kernel_traffic(dom, WORKLOAD)
+    if roof["traffic"] is not None:
+        roof["traffic_unit"] = "bytes per launch (ncu dram__bytes_read.sum + dram__bytes_write.sum)"
     for n, (bd, u) in work.items():
         if n in per:
             r = roofline_entry(n, bd, u, sum(per[n]) / len(per[n]) * 1e-3, pk, sm_count, sm_mhz)
