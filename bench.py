@@ -272,7 +272,8 @@ def run_reference(args, rank):
     print(json.dumps({
         "impl": "reference", "metric": "hybrid-head mixer prefill tokens/s", "value": v,
         "unit": "tokens/s", "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
-        "higher_is_better": True, "dtype": "f64", "data": "synthetic",
+        "ms_per_step": 1e3 * T_sample / v, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f64", "data": "synthetic",
         "config": {"workload": WORKLOAD, "B": wl["B"], "T": wl["T"], "n_meta": 128, "window": 1024},
         "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": cpu_cores(), "kind": "oracle",
                          "sample": sample},
