@@ -82,25 +82,26 @@ attn_decode_kernel(const T* __restrict__ P, long long ldP, const T* __restrict__
         slots[kk] = j < n_meta ? j : n_meta + (j - n_meta) % ring;
     }
     __syncthreads();
-    // scores: one key per thread, its K row in 16-byte pieces, q broadcast from smem
+    // scores: one key per thread, its K row (128 bytes) loaded whole before any use so
+    // that all eight 16-byte loads are in flight together; q broadcast from smem
     for (int kk = tid; kk < nk; kk += blockDim.x) {
         const T* kr = k_cache + (kvbase + slots[kk]) * DH;
+        float kv[DH];
+#pragma unroll
+        for (int e = 0; e < DH; e += 8) load_row8<T>(kr + e, kv + e);
         float acc[MAX_R];
 #pragma unroll
         for (int r = 0; r < MAX_R; ++r) acc[r] = 0.f;
 #pragma unroll
-        for (int e = 0; e < DH; e += 8) {
-            float kv[8];
-            load_row8<T>(kr + e, kv);
+        for (int e = 0; e < DH; e += 4) {
 #pragma unroll
             for (int r = 0; r < MAX_R; ++r) {
                 if (r < R) {
                     const float4 qa = *reinterpret_cast<const float4*>(&qs[r][e]);
-                    const float4 qb = *reinterpret_cast<const float4*>(&qs[r][e + 4]);
-                    acc[r] = fmaf(qa.x, kv[0], acc[r]); acc[r] = fmaf(qa.y, kv[1], acc[r]);
-                    acc[r] = fmaf(qa.z, kv[2], acc[r]); acc[r] = fmaf(qa.w, kv[3], acc[r]);
-                    acc[r] = fmaf(qb.x, kv[4], acc[r]); acc[r] = fmaf(qb.y, kv[5], acc[r]);
-                    acc[r] = fmaf(qb.z, kv[6], acc[r]); acc[r] = fmaf(qb.w, kv[7], acc[r]);
+                    acc[r] = fmaf(qa.x, kv[e], acc[r]);
+                    acc[r] = fmaf(qa.y, kv[e + 1], acc[r]);
+                    acc[r] = fmaf(qa.z, kv[e + 2], acc[r]);
+                    acc[r] = fmaf(qa.w, kv[e + 3], acc[r]);
                 }
             }
         }
@@ -133,15 +134,33 @@ attn_decode_kernel(const T* __restrict__ P, long long ldP, const T* __restrict__
         for (int r = 0; r < MAX_R; ++r)
 #pragma unroll
             for (int i = 0; i < 8; ++i) acc[r][i] = 0.f;
-        for (int kk = kg; kk < nk; kk += KGROUPS) {
-            float v[8];
-            load_row8<T>(v_cache + (kvbase + slots[kk]) * DV + eb * 8, v);
+        // four keys per round, their V pieces loaded before any is used, so that four
+        // loads per thread are in flight instead of one
+        constexpr int U = 4;
+        for (int kk0 = kg; kk0 < nk; kk0 += KGROUPS * U) {
+            float v[U][8];
 #pragma unroll
-            for (int r = 0; r < MAX_R; ++r) {
-                if (r < R) {
-                    const float pr = ps[r][kk];
+            for (int u = 0; u < U; ++u) {
+                const int kk = kk0 + u * KGROUPS;
+                if (kk < nk) {
+                    load_row8<T>(v_cache + (kvbase + slots[kk]) * DV + eb * 8, v[u]);
+                } else {
 #pragma unroll
-                    for (int i = 0; i < 8; ++i) acc[r][i] = fmaf(pr, v[i], acc[r][i]);
+                    for (int i = 0; i < 8; ++i) v[u][i] = 0.f;
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const int kk = kk0 + u * KGROUPS;
+                if (kk < nk) {
+#pragma unroll
+                    for (int r = 0; r < MAX_R; ++r) {
+                        if (r < R) {
+                            const float pr = ps[r][kk];
+#pragma unroll
+                            for (int i = 0; i < 8; ++i) acc[r][i] = fmaf(pr, v[u][i], acc[r][i]);
+                        }
+                    }
                 }
             }
         }
@@ -201,21 +220,49 @@ ssm_decode_kernel(const T* __restrict__ P, long long ldP, int col_x, int col_B, 
     if (idx >= (long long)B * di) return;
     const int b = (int)(idx / di), c = (int)(idx % di);
     const T* prow = P + (long long)b * ldP;
-    // shift the new input into the conv state (oldest first), then convolve
-    float* cst = conv + idx * KC;
-    float cs[KC];
-#pragma unroll
-    for (int k = 0; k < KC - 1; ++k) cs[k] = cst[k + 1];
-    cs[KC - 1] = to_f(prow[col_x + c]);
+    // shift the new input into the conv state (oldest first), then convolve; every
+    // per-channel and per-row vector below is read with 16-byte loads
+    float4* cst = reinterpret_cast<float4*>(conv + idx * KC);
+    const float4 c4 = *cst;
+    const float cs[KC] = {c4.y, c4.z, c4.w, to_f(prow[col_x + c])};
+    const float4 w4 = *reinterpret_cast<const float4*>(conv_w + (long long)c * KC);
     float acc = conv_b[c];
-#pragma unroll
-    for (int k = 0; k < KC; ++k) {
-        acc = fmaf(conv_w[(long long)c * KC + k], cs[k], acc);
-        cst[k] = cs[k];
-    }
+    acc = fmaf(w4.x, cs[0], acc);
+    acc = fmaf(w4.y, cs[1], acc);
+    acc = fmaf(w4.z, cs[2], acc);
+    acc = fmaf(w4.w, cs[3], acc);
+    *cst = make_float4(cs[0], cs[1], cs[2], cs[3]);
     const float xc = silu_f(acc);
     const float d = delta[idx];
     const float dx = d * xc;
+    float Bv[NS], Cv[NS], Al[NS];
+    if constexpr (sizeof(T) == 2) {
+#pragma unroll
+        for (int k = 0; k < 2; ++k) {
+            const uint4 ub = *reinterpret_cast<const uint4*>(prow + col_B + 8 * k);
+            const uint4 uc = *reinterpret_cast<const uint4*>(prow + col_C + 8 * k);
+            const T* hb = reinterpret_cast<const T*>(&ub);
+            const T* hc = reinterpret_cast<const T*>(&uc);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                Bv[8 * k + i] = to_f(hb[i]);
+                Cv[8 * k + i] = to_f(hc[i]);
+            }
+        }
+    } else {
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const float4 fb = *reinterpret_cast<const float4*>(prow + col_B + 4 * k);
+            const float4 fc = *reinterpret_cast<const float4*>(prow + col_C + 4 * k);
+            Bv[4 * k] = fb.x; Bv[4 * k + 1] = fb.y; Bv[4 * k + 2] = fb.z; Bv[4 * k + 3] = fb.w;
+            Cv[4 * k] = fc.x; Cv[4 * k + 1] = fc.y; Cv[4 * k + 2] = fc.z; Cv[4 * k + 3] = fc.w;
+        }
+    }
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        const float4 a4 = *reinterpret_cast<const float4*>(A_log + (long long)c * NS + 4 * k);
+        Al[4 * k] = a4.x; Al[4 * k + 1] = a4.y; Al[4 * k + 2] = a4.z; Al[4 * k + 3] = a4.w;
+    }
     float4* hp = reinterpret_cast<float4*>(h + idx * NS);
     float hv[NS];
 #pragma unroll
@@ -226,9 +273,10 @@ ssm_decode_kernel(const T* __restrict__ P, long long ldP, int col_x, int col_B, 
     float y = 0.f;
 #pragma unroll
     for (int n = 0; n < NS; ++n) {
-        const float a = fast_exp2(d * (-expf(A_log[(long long)c * NS + n]) * LOG2E));
-        hv[n] = fmaf(a, hv[n], dx * to_f(prow[col_B + n]));
-        y = fmaf(to_f(prow[col_C + n]), hv[n], y);
+        // exp(Delta A) with A = -exp(A_log): exp2(-Delta * 2^(A_log log2 e) * log2 e)
+        const float a = fast_exp2(-d * fast_exp2(Al[n] * LOG2E) * LOG2E);
+        hv[n] = fmaf(a, hv[n], dx * Bv[n]);
+        y = fmaf(Cv[n], hv[n], y);
     }
 #pragma unroll
     for (int q = 0; q < NS / 4; ++q) hp[q] = make_float4(hv[4 * q], hv[4 * q + 1], hv[4 * q + 2], hv[4 * q + 3]);
@@ -260,6 +308,12 @@ int launch_ssm_decode(const Ctx& ctx, const T* P, long long ldP, int col_x, int 
                       const float* A_log, const float* D, float* h, float* conv, T* ypre, int B,
                       int di) {
     const long long n = (long long)B * di;
+    // 16-byte loads: the B/C columns of every projection row, conv taps, A_log and conv state
+    constexpr int V = 16 / (int)sizeof(T);
+    if (ldP % V || col_B % V || col_C % V || (reinterpret_cast<uintptr_t>(conv_w) & 15) ||
+        (reinterpret_cast<uintptr_t>(A_log) & 15) || (reinterpret_cast<uintptr_t>(conv) & 15) ||
+        (reinterpret_cast<uintptr_t>(h) & 15) || (reinterpret_cast<uintptr_t>(P) & 15))
+        return HYMBA_ERR_UNSUPPORTED;
     HYMBA_LAUNCH(ctx, "ssm_decode", ssm_decode_kernel<T>, ceil_div(n, 128), 128, 0, P, ldP, col_x,
                  col_B, col_C, delta, conv_w, conv_b, A_log, D, h, conv, ypre, B, di);
     return HYMBA_OK;

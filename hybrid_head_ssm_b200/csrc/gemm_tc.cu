@@ -299,6 +299,10 @@ int launch_gemm_tc(const Ctx& ctx, const char* name, const TA* A, long long lda,
             return launch_bn<TA, TO, 128, 4>(ctx, name, A, lda, Bw, ldb, M, N, K, e, A0, M0);
         default:
             if (K <= 2 * BK) return launch_bn<TA, TO, 64, 2>(ctx, name, A, lda, Bw, ldb, M, N, K, e, A0, M0);
+            // one row block streaming a long K (decode): a deeper ring keeps more weight
+            // tiles in flight per CTA
+            if (M + M0 <= BM && K > 4 * BK)
+                return launch_bn<TA, TO, 64, 8>(ctx, name, A, lda, Bw, ldb, M, N, K, e, A0, M0);
             return launch_bn<TA, TO, 64, 4>(ctx, name, A, lda, Bw, ldb, M, N, K, e, A0, M0);
     }
 }
