@@ -45,7 +45,13 @@ __device__ __forceinline__ void load_row8(const T* p, float* v) {
 
 constexpr int KGROUPS = 8;  // key groups of the PV phase (128 threads = 8 groups x 16 pieces of 8)
 
-template <typename T, int DV>
+// One block per (key split, KV head, sequence) serves the R query heads of the KV head.
+// Scores: four lanes per key, each holding its 16 dimensions of the R queries in
+// registers and reading 32 bytes of the K row, joined by two shuffles per head. P V:
+// thread (key group, 8-dimension piece) walks its keys four at a time with the V pieces
+// loaded ahead of use and all R heads' weights read as two 16-byte loads per key
+// (P stored [key][head]); the products are packed f32x2 FMAs.
+template <typename T, int DV, int R>
 __global__ void __launch_bounds__(128)
 attn_decode_kernel(const T* __restrict__ P, long long ldP, const T* __restrict__ k_cache,
                    const T* __restrict__ v_cache, int cap, const int* __restrict__ len,
@@ -53,14 +59,13 @@ attn_decode_kernel(const T* __restrict__ P, long long ldP, const T* __restrict__
                    int n_meta, int window, int* status) {
     griddep_sync();
     static_assert(DV == 16 * 8, "PV phase covers a V row with 16 pieces of 8");
-    __shared__ __align__(16) float qs[MAX_R][DH];
-    __shared__ float ps[MAX_R][MAX_CHUNK];
+    static_assert(R >= 1 && R <= 8, "query heads per KV head");
+    __shared__ __align__(16) float ps[MAX_CHUNK][8];
     __shared__ int slots[MAX_CHUNK];
-    __shared__ float stat[MAX_R][2];
-    __shared__ __align__(16) float red[KGROUPS][MAX_R][DV];
+    __shared__ float stat[R][2];
+    __shared__ __align__(16) float red[KGROUPS][R][DV];
     const int s = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
-    const int R = H / G;
-    const int tid = threadIdx.x;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int p = len[b] + pos_offset;
     const int ring = cap - n_meta;
     int meta_n, lo;
@@ -72,53 +77,68 @@ attn_decode_kernel(const T* __restrict__ P, long long ldP, const T* __restrict__
     const int nk = k1 - k0;
     const long long kvbase = ((long long)b * G + g) * cap;
 
-    for (int i = tid; i < R * DH; i += blockDim.x) {
-        const int r = i / DH, e = i % DH;
-        qs[r][e] = to_f(P[(long long)b * ldP + (g * R + r) * DH + e]) * (LOG2E * 0.125f);
-    }
     for (int kk = tid; kk < nk; kk += blockDim.x) {
         const int idx = k0 + kk;
         const int j = idx < meta_n ? idx : lo + (idx - meta_n);
         slots[kk] = j < n_meta ? j : n_meta + (j - n_meta) % ring;
     }
+    // this lane's quarter of the head dimension (16 of 64) for the R queries, scaled by
+    // log2(e) / sqrt(64)
+    const int qq = lane & 3, kl = lane >> 2;
+    float2 qr[R][8];
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+        float qv[16];
+        const T* qp = P + (long long)b * ldP + (g * R + r) * DH + 16 * qq;
+        load_row8<T>(qp, qv);
+        load_row8<T>(qp + 8, qv + 8);
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+            qr[r][i] = make_float2(qv[2 * i] * (LOG2E * 0.125f), qv[2 * i + 1] * (LOG2E * 0.125f));
+    }
     __syncthreads();
-    // scores: one key per thread, its K row (128 bytes) loaded whole before any use so
-    // that all eight 16-byte loads are in flight together; q broadcast from smem
-    for (int kk = tid; kk < nk; kk += blockDim.x) {
-        const T* kr = k_cache + (kvbase + slots[kk]) * DH;
-        float kv[DH];
+    // scores: warp w takes keys w*8 .. w*8+7 of every 32, lane (key kl, quarter qq)
+    for (int kb = warp * 8; kb < nk; kb += 32) {
+        const int kk = kb + kl;
+        float2 acc[R];
 #pragma unroll
-        for (int e = 0; e < DH; e += 8) load_row8<T>(kr + e, kv + e);
-        float acc[MAX_R];
+        for (int r = 0; r < R; ++r) acc[r] = make_float2(0.f, 0.f);
+        if (kk < nk) {
+            const T* kr = k_cache + (kvbase + slots[kk]) * DH + 16 * qq;
+            float kv[16];
+            load_row8<T>(kr, kv);
+            load_row8<T>(kr + 8, kv + 8);
 #pragma unroll
-        for (int r = 0; r < MAX_R; ++r) acc[r] = 0.f;
+            for (int i = 0; i < 8; ++i) {
+                const float2 k2 = make_float2(kv[2 * i], kv[2 * i + 1]);
 #pragma unroll
-        for (int e = 0; e < DH; e += 4) {
-#pragma unroll
-            for (int r = 0; r < MAX_R; ++r) {
-                if (r < R) {
-                    const float4 qa = *reinterpret_cast<const float4*>(&qs[r][e]);
-                    acc[r] = fmaf(qa.x, kv[e], acc[r]);
-                    acc[r] = fmaf(qa.y, kv[e + 1], acc[r]);
-                    acc[r] = fmaf(qa.z, kv[e + 2], acc[r]);
-                    acc[r] = fmaf(qa.w, kv[e + 3], acc[r]);
-                }
+                for (int r = 0; r < R; ++r) acc[r] = __ffma2_rn(qr[r][i], k2, acc[r]);
             }
         }
-        for (int r = 0; r < R; ++r) ps[r][kk] = acc[r];
+        float sc[R];
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+            float a = acc[r].x + acc[r].y;
+            a += __shfl_xor_sync(0xffffffffu, a, 1);
+            a += __shfl_xor_sync(0xffffffffu, a, 2);
+            sc[r] = a;
+        }
+        if (kk < nk && qq == 0) {
+#pragma unroll
+            for (int r = 0; r < R; ++r) ps[kk][r] = sc[r];
+        }
     }
     __syncthreads();
     // per-head max and sum over this split's keys: warp w handles heads w, w+4, ...
-    const int warp = tid >> 5, lane = tid & 31;
     for (int r = warp; r < R; r += 4) {
         float mx = -INFINITY;
-        for (int kk = lane; kk < nk; kk += 32) mx = fmaxf(mx, ps[r][kk]);
+        for (int kk = lane; kk < nk; kk += 32) mx = fmaxf(mx, ps[kk][r]);
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
         float sum = 0.f;
         for (int kk = lane; kk < nk; kk += 32) {
-            const float e = exp2f(ps[r][kk] - mx);
-            ps[r][kk] = e;
+            const float e = exp2f(ps[kk][r] - mx);
+            ps[kk][r] = e;
             sum += e;
         }
 #pragma unroll
@@ -129,13 +149,11 @@ attn_decode_kernel(const T* __restrict__ P, long long ldP, const T* __restrict__
     // P V: thread (key group kg, piece eb) adds keys kg, kg + 8, ... for V elements eb*8..+7
     {
         const int eb = tid % 16, kg = tid / 16;
-        float acc[MAX_R][8];
+        float2 acc[R][4];
 #pragma unroll
-        for (int r = 0; r < MAX_R; ++r)
+        for (int r = 0; r < R; ++r)
 #pragma unroll
-            for (int i = 0; i < 8; ++i) acc[r][i] = 0.f;
-        // four keys per round, their V pieces loaded before any is used, so that four
-        // loads per thread are in flight instead of one
+            for (int i = 0; i < 4; ++i) acc[r][i] = make_float2(0.f, 0.f);
         constexpr int U = 4;
         for (int kk0 = kg; kk0 < nk; kk0 += KGROUPS * U) {
             float v[U][8];
@@ -153,23 +171,23 @@ attn_decode_kernel(const T* __restrict__ P, long long ldP, const T* __restrict__
             for (int u = 0; u < U; ++u) {
                 const int kk = kk0 + u * KGROUPS;
                 if (kk < nk) {
+                    const float4 pa = *reinterpret_cast<const float4*>(&ps[kk][0]);
+                    const float4 pb = *reinterpret_cast<const float4*>(&ps[kk][4]);
+                    const float pw[8] = {pa.x, pa.y, pa.z, pa.w, pb.x, pb.y, pb.z, pb.w};
 #pragma unroll
-                    for (int r = 0; r < MAX_R; ++r) {
-                        if (r < R) {
-                            const float pr = ps[r][kk];
+                    for (int r = 0; r < R; ++r) {
+                        const float2 pr = make_float2(pw[r], pw[r]);
 #pragma unroll
-                            for (int i = 0; i < 8; ++i) acc[r][i] = fmaf(pr, v[u][i], acc[r][i]);
-                        }
+                        for (int i = 0; i < 4; ++i)
+                            acc[r][i] = __ffma2_rn(pr, make_float2(v[u][2 * i], v[u][2 * i + 1]), acc[r][i]);
                     }
                 }
             }
         }
 #pragma unroll
-        for (int r = 0; r < MAX_R; ++r) {
-            if (r < R) {
-                *reinterpret_cast<float4*>(&red[kg][r][eb * 8]) = make_float4(acc[r][0], acc[r][1], acc[r][2], acc[r][3]);
-                *reinterpret_cast<float4*>(&red[kg][r][eb * 8 + 4]) = make_float4(acc[r][4], acc[r][5], acc[r][6], acc[r][7]);
-            }
+        for (int r = 0; r < R; ++r) {
+            *reinterpret_cast<float4*>(&red[kg][r][eb * 8]) = make_float4(acc[r][0].x, acc[r][0].y, acc[r][1].x, acc[r][1].y);
+            *reinterpret_cast<float4*>(&red[kg][r][eb * 8 + 4]) = make_float4(acc[r][2].x, acc[r][2].y, acc[r][3].x, acc[r][3].y);
         }
     }
     __syncthreads();
@@ -293,7 +311,21 @@ int launch_attn_decode(const Ctx& ctx, const T* P, long long ldP, const T* k_cac
     if (H / G > MAX_R || dv != 128) return HYMBA_ERR_UNSUPPORTED;
     if ((cache_cap + n_split - 1) / n_split > MAX_CHUNK) return HYMBA_ERR_INVALID_ARG;
     dim3 grid(n_split, G, B);
-    auto k1 = attn_decode_kernel<T, 128>;
+    // 16-byte loads of q, K and V rows
+    if ((reinterpret_cast<uintptr_t>(P) | reinterpret_cast<uintptr_t>(k_cache) | reinterpret_cast<uintptr_t>(v_cache)) & 15 ||
+        ldP % (16 / (long long)sizeof(T)))
+        return HYMBA_ERR_UNSUPPORTED;
+    void (*k1)(const T*, long long, const T*, const T*, int, const int*, int, float*, int, int, int, int, int, int*);
+    switch (H / G) {
+        case 1: k1 = attn_decode_kernel<T, 128, 1>; break;
+        case 2: k1 = attn_decode_kernel<T, 128, 2>; break;
+        case 3: k1 = attn_decode_kernel<T, 128, 3>; break;
+        case 4: k1 = attn_decode_kernel<T, 128, 4>; break;
+        case 5: k1 = attn_decode_kernel<T, 128, 5>; break;
+        case 6: k1 = attn_decode_kernel<T, 128, 6>; break;
+        case 7: k1 = attn_decode_kernel<T, 128, 7>; break;
+        default: k1 = attn_decode_kernel<T, 128, 8>; break;
+    }
     HYMBA_LAUNCH(ctx, "attn_decode", k1, grid, 128, 0, P, ldP, k_cache, v_cache, cache_cap, len,
                  pos_offset, part, n_split, H, G, n_meta, window, ctx.status);
     dim3 g2(H, B);
