@@ -30,7 +30,8 @@ struct EpiArgs {
     T* v_out;              // producer: V [B, G, kcap, dv]
     int kcap;
     int H, G, dh, dv;
-    const float2* rope;    // [T', dh/2] (cos, sin) of position * theta_i (prefill)
+    const float2* rope;    // prefill: [T', dh/2] (cos, sin) of position * theta_i; decode: [B, dh/2] for
+                           // each sequence's new position (computed on the fly when null)
     const int* pos;        // decode: [B] positions held (len); the new token sits at pos[b] + pos_offset
     int pos_offset;        // decode: 0 for a producer (appends), -1 for a consumer
     int n_meta_ring;       // decode: ring length (cache_cap - n_meta)
@@ -177,10 +178,14 @@ __device__ __forceinline__ RunDst epi_prepare64(const EpiArgs<T>& e, int r, int 
     const int vw = e.k_out ? e.G * e.dv : 0;
     if (c0 < qw + kw) {
         if (mode == ROWS_DECODE) {
-            float2 cs[32];
+            if (e.rope) {
+                rope_run64(v, e.rope + (long long)r * 32);  // the step's table, one row per sequence
+            } else {
+                float2 cs[32];
 #pragma unroll 4
-            for (int i = 0; i < 32; ++i) cs[i] = rope_cs_at(t, i, 64, e.rope_base);
-            rope_run64(v, cs);
+                for (int i = 0; i < 32; ++i) cs[i] = rope_cs_at(t, i, 64, e.rope_base);
+                rope_run64(v, cs);
+            }
         } else {
             rope_run64(v, e.rope + (long long)t * 32);
         }

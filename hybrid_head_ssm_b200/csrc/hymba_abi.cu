@@ -165,7 +165,8 @@ static Plan plan(const hymba_layer_cfg* c, int B, int T, int mode) {
     p.ldP = round_up(k.n_in, 64);
     p.rpad = (int)round_up(c->dt_rank, 64);
     size_t cur = 0;
-    if (mode == HYMBA_MODE_PREFILL) p.rope = take(&cur, (size_t)(c->n_meta + T) * 32 * sizeof(float2));
+    // RoPE table: prefill, one row per position; decode, one row per sequence
+    p.rope = take(&cur, (size_t)(mode == HYMBA_MODE_PREFILL ? c->n_meta + T : B) * 32 * sizeof(float2));
     p.P = take(&cur, rows * p.ldP * esz);
     p.delta = take(&cur, rows * di * sizeof(float));
     p.O = take(&cur, rows * (size_t)c->n_q_heads * c->v_head_dim * esz);
@@ -389,8 +390,13 @@ static int decode_impl(const Ctx& ctx, const hymba_layer_cfg* c, const hymba_lay
     ep.pos = kv->len; ep.pos_offset = pos_offset;
     ep.n_meta_ring = kv->cache_cap - m;
     ep.rope_base = c->rope_base;
+    // RoPE table of the new positions and the padded 16-bit W_dt, one launch
+    float2* rope = reinterpret_cast<float2*>(ws + pl.rope);
+    if ((rc = launch_decode_prep<T, I>(ctx, rope, kv->len, pos_offset, B, dh, c->rope_base,
+                                       static_cast<const T*>(w->w_dt), di, c->dt_rank, wdt, pl.rpad)))
+        return rc;
+    ep.rope = rope;
     if ((rc = gemm<T, I>(ctx, "gemm_in_proj_decode", x, d, static_cast<const T*>(w->w_in), d, B, k.n_in, d, ep))) return rc;
-    if ((rc = launch_pad_copy<T, I>(ctx, static_cast<const T*>(w->w_dt), di, c->dt_rank, wdt, pl.rpad))) return rc;
     EpiArgs<I> ed = epi_base<I>(EPI_DELTA, B, di);
     ed.delta = delta; ed.b_dt = w->b_dt;
     if ((rc = gemm<I, I>(ctx, "gemm_dt_proj_decode", P + k.dtl, pl.ldP, wdt, pl.rpad, B, di, c->dt_rank, ed))) return rc;

@@ -53,6 +53,12 @@ template <typename TS, typename TD>
 int launch_prefill_prep(const Ctx& ctx, float2* tab, int Tp, int dh, float base, const TS* w, int rows, int cols,
                         TD* wdst, int ld_dst);
 
+// The RoPE table of a decode step's new positions ([B, dh/2] (cos, sin)) and the
+// zero-padded 16-bit copy of W_dt, in one launch.
+template <typename TS, typename TD>
+int launch_decode_prep(const Ctx& ctx, float2* tab, const int* len, int pos_offset, int B, int dh, float base,
+                       const TS* w, int rows, int cols, TD* wdst, int ld_dst);
+
 // Copy a [rows, cols] matrix into a zero-padded [rows, ld_dst] one of type TD.
 template <typename TS, typename TD>
 int launch_pad_copy(const Ctx& ctx, const TS* src, int rows, int cols, TD* dst, int ld_dst);

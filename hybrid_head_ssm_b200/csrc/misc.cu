@@ -35,6 +35,28 @@ __global__ void prefill_prep_kernel(float2* tab, int Tp, int half, int dh, float
     }
 }
 
+// The small inputs of a decode step in one launch: blocks [0, nb_rope) fill the RoPE
+// table of each sequence's new position (len[b] + pos_offset; rows without a valid
+// position get the identity rotation, their outputs are never written), the rest copy
+// W_dt into its zero-padded 16-bit form.
+template <typename TS, typename TD>
+__global__ void decode_prep_kernel(float2* tab, const int* len, int pos_offset, int B, int half, int dh, float base,
+                                   int nb_rope, const TS* w, int rows, int cols, TD* wdst, int ld_dst) {
+    griddep_sync();
+    if ((int)blockIdx.x < nb_rope) {
+        const int idx = blockIdx.x * blockDim.x + threadIdx.x;
+        if (idx >= B * half) return;
+        const int b = idx / half, i = idx % half;
+        const int p = len[b] + pos_offset;
+        tab[idx] = p >= 0 ? rope_cs_at(p, i, dh, base) : make_float2(1.f, 0.f);
+    } else {
+        const long long idx = (long long)(blockIdx.x - nb_rope) * blockDim.x + threadIdx.x;
+        if (idx >= (long long)rows * ld_dst) return;
+        const int r = (int)(idx / ld_dst), c = (int)(idx % ld_dst);
+        wdst[idx] = from_f<TD>(c < cols ? to_f(w[(long long)r * cols + c]) : 0.f);
+    }
+}
+
 // Slot of position p: meta positions keep their slot, the others wrap in a ring of
 // cache_cap - n_meta slots. Rows copied: meta positions and the newest ring-full.
 template <typename T>
@@ -79,6 +101,17 @@ int launch_prefill_prep(const Ctx& ctx, float2* tab, int Tp, int dh, float base,
     return HYMBA_OK;
 }
 
+template <typename TS, typename TD>
+int launch_decode_prep(const Ctx& ctx, float2* tab, const int* len, int pos_offset, int B, int dh, float base,
+                       const TS* w, int rows, int cols, TD* wdst, int ld_dst) {
+    const int nb_rope = ceil_div((long long)B * (dh / 2), 256);
+    const int nb_pad = ceil_div((long long)rows * ld_dst, 256);
+    auto kern = decode_prep_kernel<TS, TD>;
+    HYMBA_LAUNCH(ctx, "decode_prep", kern, nb_rope + nb_pad, 256, 0, tab, len, pos_offset, B, dh / 2, dh, base,
+                 nb_rope, w, rows, cols, wdst, ld_dst);
+    return HYMBA_OK;
+}
+
 template <typename T>
 int launch_cache_fill(const Ctx& ctx, const T* k_seq, const T* v_seq, int seq_cap, T* k_cache,
                       T* v_cache, int cache_cap, int* len, int B, int G, int dh, int dv, int n_meta,
@@ -96,6 +129,10 @@ template int launch_pad_copy<bf16, f16>(const Ctx&, const bf16*, int, int, f16*,
 template int launch_prefill_prep<float, float>(const Ctx&, float2*, int, int, float, const float*, int, int, float*,
                                                int);
 template int launch_prefill_prep<bf16, f16>(const Ctx&, float2*, int, int, float, const bf16*, int, int, f16*, int);
+template int launch_decode_prep<float, float>(const Ctx&, float2*, const int*, int, int, int, float, const float*,
+                                              int, int, float*, int);
+template int launch_decode_prep<bf16, f16>(const Ctx&, float2*, const int*, int, int, int, float, const bf16*, int, int,
+                                           f16*, int);
 template int launch_cache_fill<float>(const Ctx&, const float*, const float*, int, float*, float*,
                                       int, int*, int, int, int, int, int, int);
 template int launch_cache_fill<f16>(const Ctx&, const f16*, const f16*, int, f16*, f16*, int,
