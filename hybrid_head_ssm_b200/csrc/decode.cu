@@ -225,80 +225,248 @@ attn_decode_combine_kernel(const float* __restrict__ part, int n_split, T* __res
     O[((long long)b * H + h) * DV + e] = from_f<T>(den > 0.f ? num / den : 0.f);
 }
 
-template <typename T>
-__global__ void __launch_bounds__(128)
+constexpr int SSM_WARPS = 4;   // warps per block
+constexpr int SSM_RPT = 2;     // sequences per thread: rows warp and warp + 4 of the block's 8
+constexpr int SSM_ROWS = SSM_WARPS * SSM_RPT;
+constexpr int SSM_CH = 32;     // channels per block, one per lane
+constexpr int SSM_PAIRS = 128; // W_dt column pairs staged per pass (dt_rank <= 256 in one pass)
+constexpr int SSM_WLD = 4;     // 16-byte W_dt loads per thread in the wide staging (32 rows x <= 64 pairs)
+constexpr int SSM_XLD = 4;     // 4-byte dt_low loads per thread in the wide staging (8 rows x <= 64 pairs)
+
+// A pair of adjacent W_dt entries of one channel as held in shared memory: the raw
+// bits of two bf16 (exact on unpacking), or two floats.
+template <typename TW> struct WSlot { using type = float2; };
+template <> struct WSlot<bf16> { using type = uint32_t; };
+__device__ __forceinline__ float2 wunpack(float2 v) { return v; }
+__device__ __forceinline__ float2 wunpack(uint32_t v) {
+    return make_float2(__uint_as_float(v << 16), __uint_as_float(v & 0xffff0000u));
+}
+__device__ __forceinline__ float2 wpack(float lo, float hi) { return make_float2(lo, hi); }
+__device__ __forceinline__ uint32_t wpack(bf16 lo, bf16 hi) {
+    return (uint32_t)__bfloat16_as_ushort(lo) | ((uint32_t)__bfloat16_as_ushort(hi) << 16);
+}
+__device__ __forceinline__ float2 x2float(uint32_t v) {  // an fp16 pair
+    __half2 h;
+    memcpy(&h, &v, 4);
+    return __half22float2(h);
+}
+
+// One decode step of the selective SSM for (sequence b, channel c), with the Delta
+// projection of the new token folded in: Delta = softplus(dt_low . W_dt[c] + b_dt[c])
+// ("Hymba Guide", Parallel Hybrid-Head Layer Formulation: the SSM heads take Delta,
+// B, C from the shared input projection). Block = 8 sequences x 32 channels, each
+// thread one channel of two sequences (the W_dt row and the per-channel constants are
+// read once for both). The block's 32 rows of W_dt and 8 dt_low rows are staged in
+// shared memory (rows padded to an odd number of slots, so that the per-lane row reads
+// hit distinct banks); with 16-bit operands and an even dt_rank <= 128 the staging is
+// a few wide loads per thread, all in flight together, and the loads of h go out
+// before the dot products.
+template <typename T, typename TW>
+__global__ void __launch_bounds__(SSM_WARPS * 32, 6)
 ssm_decode_kernel(const T* __restrict__ P, long long ldP, int col_x, int col_B, int col_C,
-                  const float* __restrict__ delta, const float* __restrict__ conv_w,
-                  const float* __restrict__ conv_b, const float* __restrict__ A_log,
-                  const float* __restrict__ Dp, float* __restrict__ h, float* __restrict__ conv,
-                  T* __restrict__ ypre, int B, int di) {
+                  int col_dtl, const TW* __restrict__ w_dt, const float* __restrict__ b_dt, int r,
+                  int wide, const float* __restrict__ conv_w, const float* __restrict__ conv_b,
+                  const float* __restrict__ A_log, const float* __restrict__ Dp,
+                  float* __restrict__ h, float* __restrict__ conv, T* __restrict__ ypre, int B,
+                  int di) {
     griddep_sync();
+    using Slot = typename WSlot<TW>::type;
     constexpr int NS = 16, KC = 4;
-    const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-    if (idx >= (long long)B * di) return;
-    const int b = (int)(idx / di), c = (int)(idx % di);
-    const T* prow = P + (long long)b * ldP;
-    // shift the new input into the conv state (oldest first), then convolve; every
-    // per-channel and per-row vector below is read with 16-byte loads
-    float4* cst = reinterpret_cast<float4*>(conv + idx * KC);
-    const float4 c4 = *cst;
-    const float cs[KC] = {c4.y, c4.z, c4.w, to_f(prow[col_x + c])};
-    const float4 w4 = *reinterpret_cast<const float4*>(conv_w + (long long)c * KC);
-    float acc = conv_b[c];
-    acc = fmaf(w4.x, cs[0], acc);
-    acc = fmaf(w4.y, cs[1], acc);
-    acc = fmaf(w4.z, cs[2], acc);
-    acc = fmaf(w4.w, cs[3], acc);
-    *cst = make_float4(cs[0], cs[1], cs[2], cs[3]);
-    const float xc = silu_f(acc);
-    const float d = delta[idx];
-    const float dx = d * xc;
-    float Bv[NS], Cv[NS], Al[NS];
-    if constexpr (sizeof(T) == 2) {
+    extern __shared__ __align__(16) unsigned char ssm_smem[];
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int c0 = blockIdx.x * SSM_CH, b0 = blockIdx.y * SSM_ROWS;
+    const int c = c0 + lane;
+    const bool cok = c < di;
+    int bs[SSM_RPT];
+    bool ok[SSM_RPT];
 #pragma unroll
-        for (int k = 0; k < 2; ++k) {
-            const uint4 ub = *reinterpret_cast<const uint4*>(prow + col_B + 8 * k);
-            const uint4 uc = *reinterpret_cast<const uint4*>(prow + col_C + 8 * k);
-            const T* hb = reinterpret_cast<const T*>(&ub);
-            const T* hc = reinterpret_cast<const T*>(&uc);
+    for (int u = 0; u < SSM_RPT; ++u) {
+        bs[u] = b0 + warp + u * SSM_WARPS;
+        ok[u] = cok && bs[u] < B;
+    }
+    // the state rows: the longest loads, independent of Delta, issued ahead of the dot
+    // products (which run while they are in flight)
+    float hv[SSM_RPT][NS];
+    auto load_h = [&]() {
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                Bv[8 * k + i] = to_f(hb[i]);
-                Cv[8 * k + i] = to_f(hc[i]);
+        for (int u = 0; u < SSM_RPT; ++u) {
+            const float4* hp = reinterpret_cast<const float4*>(h + ((long long)bs[u] * di + c) * NS);
+#pragma unroll
+            for (int q = 0; q < NS / 4; ++q) {
+                const float4 t = ok[u] ? hp[q] : make_float4(0.f, 0.f, 0.f, 0.f);
+                hv[u][4 * q] = t.x; hv[u][4 * q + 1] = t.y; hv[u][4 * q + 2] = t.z; hv[u][4 * q + 3] = t.w;
             }
         }
-    } else {
+    };
+    const int npairs = (r + 1) / 2;
+    const int cp = min(npairs, SSM_PAIRS);
+    const int RS = cp | 1;
+    Slot* Ws = reinterpret_cast<Slot*>(ssm_smem);
+    float2* xs = reinterpret_cast<float2*>(ssm_smem + ((SSM_CH * RS * sizeof(Slot) + 15) & ~size_t(15)));
+    float2 dacc[SSM_RPT];
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            const float4 fb = *reinterpret_cast<const float4*>(prow + col_B + 4 * k);
-            const float4 fc = *reinterpret_cast<const float4*>(prow + col_C + 4 * k);
-            Bv[4 * k] = fb.x; Bv[4 * k + 1] = fb.y; Bv[4 * k + 2] = fb.z; Bv[4 * k + 3] = fb.w;
-            Cv[4 * k] = fc.x; Cv[4 * k + 1] = fc.y; Cv[4 * k + 2] = fc.z; Cv[4 * k + 3] = fc.w;
+    for (int u = 0; u < SSM_RPT; ++u) dacc[u] = make_float2(0.f, 0.f);
+    if constexpr (sizeof(TW) == 2) {
+        if (wide) {
+            // one pass: the block's W_dt rows are one contiguous run of 32 * r entries
+            // (16-byte aligned), the dt_low rows r/2 fp16 pairs each
+            const int n4 = SSM_CH * npairs / 4;
+            const uint4* wsrc = reinterpret_cast<const uint4*>(w_dt + (long long)c0 * r);
+            uint4 wb[SSM_WLD];
+#pragma unroll
+            for (int k = 0; k < SSM_WLD; ++k)
+                if (tid + k * SSM_WARPS * 32 < n4) wb[k] = __ldg(wsrc + tid + k * SSM_WARPS * 32);
+            const int nx = SSM_ROWS * npairs;
+            uint32_t xb[SSM_XLD];
+#pragma unroll
+            for (int k = 0; k < SSM_XLD; ++k) {
+                const int i = tid + k * SSM_WARPS * 32;
+                xb[k] = 0u;
+                if (i < nx) {
+                    const int row = i / npairs, q = i - row * npairs;
+                    if (b0 + row < B)
+                        xb[k] = *reinterpret_cast<const uint32_t*>(P + (long long)(b0 + row) * ldP + col_dtl + 2 * q);
+                }
+            }
+#pragma unroll
+            for (int k = 0; k < SSM_WLD; ++k) {
+                const int i4 = tid + k * SSM_WARPS * 32;
+                if (i4 < n4) {
+                    int row = (4 * i4) / npairs, q = 4 * i4 - row * npairs;
+                    const uint32_t wv[4] = {wb[k].x, wb[k].y, wb[k].z, wb[k].w};
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        Ws[row * RS + q] = wv[j];
+                        if (++q == npairs) { q = 0; ++row; }
+                    }
+                }
+            }
+#pragma unroll
+            for (int k = 0; k < SSM_XLD; ++k) {
+                const int i = tid + k * SSM_WARPS * 32;
+                if (i < nx) {
+                    const int row = i / npairs, q = i - row * npairs;
+                    xs[row * cp + q] = x2float(xb[k]);
+                }
+            }
+            __syncthreads();
+            load_h();
+#pragma unroll 4
+            for (int q = 0; q < npairs; ++q) {
+                const float2 wv = wunpack(Ws[lane * RS + q]);
+#pragma unroll
+                for (int u = 0; u < SSM_RPT; ++u)
+                    dacc[u] = __ffma2_rn(wv, xs[(warp + u * SSM_WARPS) * cp + q], dacc[u]);
+            }
         }
     }
+    if (!(sizeof(TW) == 2 && wide)) {
+        // general staging: any dt_rank and weight type, in passes of SSM_PAIRS pairs
+        load_h();
+        const TW wz = from_f<TW>(0.f);
+        for (int q0 = 0; q0 < npairs; q0 += cp) {
+            const int nq = min(cp, npairs - q0);
+            if (q0) __syncthreads();
+            for (int cc = warp; cc < SSM_CH; cc += SSM_WARPS) {
+                const int ch = c0 + cc;
+                for (int q = lane; q < nq; q += 32) {
+                    const int j = 2 * (q0 + q);
+                    TW lo = wz, hi = wz;
+                    if (ch < di) {
+                        lo = w_dt[(long long)ch * r + j];
+                        if (j + 1 < r) hi = w_dt[(long long)ch * r + j + 1];
+                    }
+                    Ws[cc * RS + q] = wpack(lo, hi);
+                }
+            }
+            for (int row = warp; row < SSM_ROWS; row += SSM_WARPS) {
+                for (int q = lane; q < nq; q += 32) {
+                    const int j = 2 * (q0 + q);
+                    float lo = 0.f, hi = 0.f;
+                    if (b0 + row < B) {
+                        const T* xr = P + (long long)(b0 + row) * ldP + col_dtl;
+                        lo = to_f(xr[j]);
+                        if (j + 1 < r) hi = to_f(xr[j + 1]);
+                    }
+                    xs[row * cp + q] = make_float2(lo, hi);
+                }
+            }
+            __syncthreads();
+            for (int q = 0; q < nq; ++q) {
+                const float2 wv = wunpack(Ws[lane * RS + q]);
+#pragma unroll
+                for (int u = 0; u < SSM_RPT; ++u)
+                    dacc[u] = __ffma2_rn(wv, xs[(warp + u * SSM_WARPS) * cp + q], dacc[u]);
+            }
+        }
+    }
+    if (!cok) return;
+    // per-channel constants, shared by the thread's sequences
+    const float4 w4 = *reinterpret_cast<const float4*>(conv_w + (long long)c * KC);
+    const float cb = conv_b[c], bdt = b_dt[c], Dc = Dp[c];
+    float Ae[NS];  // -exp(A_log) log2(e): exp(Delta A) = exp2(Delta Ae)
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
         const float4 a4 = *reinterpret_cast<const float4*>(A_log + (long long)c * NS + 4 * k);
-        Al[4 * k] = a4.x; Al[4 * k + 1] = a4.y; Al[4 * k + 2] = a4.z; Al[4 * k + 3] = a4.w;
-    }
-    float4* hp = reinterpret_cast<float4*>(h + idx * NS);
-    float hv[NS];
-#pragma unroll
-    for (int q = 0; q < NS / 4; ++q) {
-        float4 t = hp[q];
-        hv[4 * q] = t.x; hv[4 * q + 1] = t.y; hv[4 * q + 2] = t.z; hv[4 * q + 3] = t.w;
-    }
-    float y = 0.f;
-#pragma unroll
-    for (int n = 0; n < NS; ++n) {
-        // exp(Delta A) with A = -exp(A_log): exp2(-Delta * 2^(A_log log2 e) * log2 e)
-        const float a = fast_exp2(-d * fast_exp2(Al[n] * LOG2E) * LOG2E);
-        hv[n] = fmaf(a, hv[n], dx * Bv[n]);
-        y = fmaf(Cv[n], hv[n], y);
+        Ae[4 * k] = -fast_exp2(a4.x * LOG2E) * LOG2E;
+        Ae[4 * k + 1] = -fast_exp2(a4.y * LOG2E) * LOG2E;
+        Ae[4 * k + 2] = -fast_exp2(a4.z * LOG2E) * LOG2E;
+        Ae[4 * k + 3] = -fast_exp2(a4.w * LOG2E) * LOG2E;
     }
 #pragma unroll
-    for (int q = 0; q < NS / 4; ++q) hp[q] = make_float4(hv[4 * q], hv[4 * q + 1], hv[4 * q + 2], hv[4 * q + 3]);
-    ypre[idx] = from_f<T>(fmaf(Dp[c], xc, y));
+    for (int u = 0; u < SSM_RPT; ++u) {
+        if (!ok[u]) continue;
+        const long long idx = (long long)bs[u] * di + c;
+        const T* prow = P + (long long)bs[u] * ldP;
+        const float d = softplus_fast(dacc[u].x + dacc[u].y + bdt);
+        // shift the new input into the conv state (oldest first), then convolve
+        float4* cst = reinterpret_cast<float4*>(conv + idx * KC);
+        const float4 c4 = *cst;
+        const float cs[KC] = {c4.y, c4.z, c4.w, to_f(prow[col_x + c])};
+        float acc = cb;
+        acc = fmaf(w4.x, cs[0], acc);
+        acc = fmaf(w4.y, cs[1], acc);
+        acc = fmaf(w4.z, cs[2], acc);
+        acc = fmaf(w4.w, cs[3], acc);
+        *cst = make_float4(cs[0], cs[1], cs[2], cs[3]);
+        const float xc = silu_f(acc);
+        const float dx = d * xc;
+        float Bv[NS], Cv[NS];
+        if constexpr (sizeof(T) == 2) {
+#pragma unroll
+            for (int k = 0; k < 2; ++k) {
+                const uint4 ub = *reinterpret_cast<const uint4*>(prow + col_B + 8 * k);
+                const uint4 uc = *reinterpret_cast<const uint4*>(prow + col_C + 8 * k);
+                const T* hb = reinterpret_cast<const T*>(&ub);
+                const T* hc = reinterpret_cast<const T*>(&uc);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    Bv[8 * k + i] = to_f(hb[i]);
+                    Cv[8 * k + i] = to_f(hc[i]);
+                }
+            }
+        } else {
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const float4 fb = *reinterpret_cast<const float4*>(prow + col_B + 4 * k);
+                const float4 fc = *reinterpret_cast<const float4*>(prow + col_C + 4 * k);
+                Bv[4 * k] = fb.x; Bv[4 * k + 1] = fb.y; Bv[4 * k + 2] = fb.z; Bv[4 * k + 3] = fb.w;
+                Cv[4 * k] = fc.x; Cv[4 * k + 1] = fc.y; Cv[4 * k + 2] = fc.z; Cv[4 * k + 3] = fc.w;
+            }
+        }
+        float y = 0.f;
+#pragma unroll
+        for (int n = 0; n < NS; ++n) {
+            const float a = fast_exp2(d * Ae[n]);
+            hv[u][n] = fmaf(a, hv[u][n], dx * Bv[n]);
+            y = fmaf(Cv[n], hv[u][n], y);
+        }
+        float4* hp = reinterpret_cast<float4*>(h + idx * NS);
+#pragma unroll
+        for (int q = 0; q < NS / 4; ++q)
+            hp[q] = make_float4(hv[u][4 * q], hv[u][4 * q + 1], hv[u][4 * q + 2], hv[u][4 * q + 3]);
+        ypre[idx] = from_f<T>(fmaf(Dc, xc, y));
+    }
 }
 
 }  // namespace
@@ -328,26 +496,41 @@ int launch_attn_decode(const Ctx& ctx, const T* P, long long ldP, const T* k_cac
     }
     HYMBA_LAUNCH(ctx, "attn_decode", k1, grid, 128, 0, P, ldP, k_cache, v_cache, cache_cap, len,
                  pos_offset, part, n_split, H, G, n_meta, window, ctx.status);
+    if (!O) return HYMBA_OK;  // the caller merges the splits itself
     dim3 g2(H, B);
     auto k2 = attn_decode_combine_kernel<T, 128>;
     HYMBA_LAUNCH(ctx, "attn_decode_combine", k2, g2, 128, 0, part, n_split, O, H);
     return HYMBA_OK;
 }
 
-template <typename T>
+template <typename T, typename TW>
 int launch_ssm_decode(const Ctx& ctx, const T* P, long long ldP, int col_x, int col_B, int col_C,
-                      const float* delta, const float* conv_w, const float* conv_b,
-                      const float* A_log, const float* D, float* h, float* conv, T* ypre, int B,
-                      int di) {
-    const long long n = (long long)B * di;
+                      int col_dtl, const TW* w_dt, const float* b_dt, int dt_rank,
+                      const float* conv_w, const float* conv_b, const float* A_log, const float* D,
+                      float* h, float* conv, T* ypre, int B, int di) {
+    if (B <= 0) return HYMBA_OK;
+    if (dt_rank <= 0) return HYMBA_ERR_INVALID_ARG;
     // 16-byte loads: the B/C columns of every projection row, conv taps, A_log and conv state
     constexpr int V = 16 / (int)sizeof(T);
     if (ldP % V || col_B % V || col_C % V || (reinterpret_cast<uintptr_t>(conv_w) & 15) ||
         (reinterpret_cast<uintptr_t>(A_log) & 15) || (reinterpret_cast<uintptr_t>(conv) & 15) ||
         (reinterpret_cast<uintptr_t>(h) & 15) || (reinterpret_cast<uintptr_t>(P) & 15))
         return HYMBA_ERR_UNSUPPORTED;
-    HYMBA_LAUNCH(ctx, "ssm_decode", ssm_decode_kernel<T>, ceil_div(n, 128), 128, 0, P, ldP, col_x,
-                 col_B, col_C, delta, conv_w, conv_b, A_log, D, h, conv, ypre, B, di);
+    using Slot = typename WSlot<TW>::type;
+    const int npairs = (dt_rank + 1) / 2;
+    const int cp = npairs < SSM_PAIRS ? npairs : SSM_PAIRS;
+    const size_t smem = ((SSM_CH * (size_t)(cp | 1) * sizeof(Slot) + 15) & ~size_t(15)) +
+                        (size_t)SSM_ROWS * cp * sizeof(float2);
+    // one-pass wide staging: 16-bit W_dt with even dt_rank <= 128 (so the block's run of
+    // 32 rows is 16-byte aligned and a whole number of 16-byte pieces, d_inner being a
+    // multiple of 32), 4-byte dt_low pairs
+    const int wide = sizeof(TW) == 2 && dt_rank % 2 == 0 && npairs <= SSM_PAIRS && di % SSM_CH == 0 &&
+                     (reinterpret_cast<uintptr_t>(w_dt) & 15) == 0 && col_dtl % 2 == 0 &&
+                     SSM_CH * npairs / 4 <= SSM_WLD * SSM_WARPS * 32 && SSM_ROWS * npairs <= SSM_XLD * SSM_WARPS * 32;
+    dim3 grid(ceil_div(di, SSM_CH), ceil_div(B, SSM_ROWS));
+    HYMBA_LAUNCH(ctx, "ssm_decode", (ssm_decode_kernel<T, TW>), grid, SSM_WARPS * 32, smem, P, ldP, col_x,
+                 col_B, col_C, col_dtl, w_dt, b_dt, dt_rank, wide, conv_w, conv_b, A_log, D, h, conv, ypre, B,
+                 di);
     return HYMBA_OK;
 }
 
@@ -357,11 +540,11 @@ template int launch_attn_decode<float>(const Ctx&, const float*, long long, cons
 template int launch_attn_decode<f16>(const Ctx&, const f16*, long long, const f16*, const f16*,
                                      int, const int*, int, float*, int, f16*, int, int, int, int,
                                      int, int);
-template int launch_ssm_decode<float>(const Ctx&, const float*, long long, int, int, int,
-                                      const float*, const float*, const float*, const float*,
-                                      const float*, float*, float*, float*, int, int);
-template int launch_ssm_decode<f16>(const Ctx&, const f16*, long long, int, int, int,
-                                    const float*, const float*, const float*, const float*,
-                                    const float*, float*, float*, f16*, int, int);
+template int launch_ssm_decode<float, float>(const Ctx&, const float*, long long, int, int, int, int,
+                                             const float*, const float*, int, const float*, const float*,
+                                             const float*, const float*, float*, float*, float*, int, int);
+template int launch_ssm_decode<f16, bf16>(const Ctx&, const f16*, long long, int, int, int, int,
+                                          const bf16*, const float*, int, const float*, const float*,
+                                          const float*, const float*, float*, float*, f16*, int, int);
 
 }  // namespace hymba

@@ -9,6 +9,11 @@
 // of the row in registers between the two passes (sums of squares, then the output),
 // moving 8 elements per 16-byte access. Few registers per thread keep many rows in
 // flight per SM, which is what an HBM-bound row kernel needs.
+//
+// Decode variant (SPLIT): the attention output arrives as the split-KV partials of the
+// decode attention (per head and key split: unnormalised sum of p v, the split's
+// max logit and sum of p) and is merged here, piece by piece, with the usual
+// rescaling by exp2(m_s - max_s m_s).
 #include "kernels.h"
 
 namespace hymba {
@@ -56,9 +61,41 @@ __device__ __forceinline__ void load8f(const float* p, float* v) {
     v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
 }
 
-template <typename I, typename T>
-__global__ void __launch_bounds__(TPR * RPB, 4)
-fuse_kernel(const I* __restrict__ O, const I* __restrict__ ypre, const I* __restrict__ P, long long ldP, int col_z,
+// Attention output piece c..c+7 of row `row` merged from its head's split partials
+// (layout [row, head, split, dv + 2]: dv sums, then max logit and sum of weights).
+__device__ __forceinline__ void merge8(const float* __restrict__ part, int n_split, int H, int dv,
+                                       long long row, int c, float* o) {
+    const int hd = c / dv, e = c - hd * dv;
+    const float* base = part + ((long long)row * H + hd) * n_split * (dv + 2);
+    float M = -INFINITY;
+    for (int s = 0; s < n_split; ++s) M = fmaxf(M, base[s * (dv + 2) + dv]);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) o[i] = 0.f;
+    float den = 0.f;
+    if (M != -INFINITY) {
+        for (int s = 0; s < n_split; ++s) {
+            const float* ps = base + s * (dv + 2);
+            const float w = exp2f(ps[dv] - M);
+            den = fmaf(w, ps[dv + 1], den);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const float2 v = *reinterpret_cast<const float2*>(ps + e + 2 * i);
+                o[2 * i] = fmaf(w, v.x, o[2 * i]);
+                o[2 * i + 1] = fmaf(w, v.y, o[2 * i + 1]);
+            }
+        }
+    }
+    const float inv = den > 0.f ? 1.f / den : 0.f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) o[i] *= inv;
+}
+
+// (the decode variant runs one block per sequence, so it asks for no more than one
+// block per SM and keeps its merge temporaries in registers)
+template <typename I, typename T, bool SPLIT>
+__global__ void __launch_bounds__(TPR * RPB, SPLIT ? 1 : 4)
+fuse_kernel(const I* __restrict__ O, const float* __restrict__ part, int n_split, int H,
+            const I* __restrict__ ypre, const I* __restrict__ P, long long ldP, int col_z,
             const float* __restrict__ g_attn, const float* __restrict__ g_ssm, const float* __restrict__ beta1,
             const float* __restrict__ beta2, T* __restrict__ U, int rows, int di, float eps, int* len_inc) {
     griddep_sync();
@@ -75,7 +112,10 @@ fuse_kernel(const I* __restrict__ O, const I* __restrict__ ypre, const I* __rest
         if (live && vi < nvec) {
             const int c = vi * 8;
             float z[8];
-            load8<I>(O + row * di + c, o[k]);
+            if constexpr (SPLIT)
+                merge8(part, n_split, H, di / H, row, c, o[k]);
+            else
+                load8<I>(O + row * di + c, o[k]);
             load8<I>(ypre + row * di + c, y[k]);
             load8<I>(P + row * ldP + col_z + c, z);
 #pragma unroll
@@ -126,23 +166,34 @@ fuse_kernel(const I* __restrict__ O, const I* __restrict__ ypre, const I* __rest
 }  // namespace
 
 template <typename I, typename T>
-int launch_fuse(const Ctx& ctx, const I* O, const I* ypre, const I* P, long long ldP, int col_z,
-                const float* g_attn, const float* g_ssm, const float* beta1, const float* beta2, T* U, int rows,
-                int di, float eps, int* len_inc) {
+int launch_fuse(const Ctx& ctx, const I* O, const float* part, int n_split, int H, const I* ypre, const I* P,
+                long long ldP, int col_z, const float* g_attn, const float* g_ssm, const float* beta1,
+                const float* beta2, T* U, int rows, int di, float eps, int* len_inc) {
     if (rows <= 0) return HYMBA_OK;
     if (di % 8 || di > VMAX * 8 * TPR || col_z % 8 || ldP % 8) return HYMBA_ERR_UNSUPPORTED;
-    auto kern = fuse_kernel<I, T>;
-    HYMBA_LAUNCH(ctx, "fuse", kern, ceil_div(rows, RPB), TPR * RPB, 0, O, ypre, P, ldP, col_z, g_attn, g_ssm,
-                 beta1, beta2, U, rows, di, eps, len_inc);
+    if (part) {
+        // pieces of 8 never straddle a head; 8-byte loads of the partial sums
+        if (H <= 0 || n_split <= 0 || di % H || (di / H) % 8 || (reinterpret_cast<uintptr_t>(part) & 7))
+            return HYMBA_ERR_UNSUPPORTED;
+        auto kern = fuse_kernel<I, T, true>;
+        HYMBA_LAUNCH(ctx, "fuse", kern, ceil_div(rows, RPB), TPR * RPB, 0, O, part, n_split, H, ypre, P, ldP,
+                     col_z, g_attn, g_ssm, beta1, beta2, U, rows, di, eps, len_inc);
+        return HYMBA_OK;
+    }
+    auto kern = fuse_kernel<I, T, false>;
+    HYMBA_LAUNCH(ctx, "fuse", kern, ceil_div(rows, RPB), TPR * RPB, 0, O, part, n_split, H, ypre, P, ldP, col_z,
+                 g_attn, g_ssm, beta1, beta2, U, rows, di, eps, len_inc);
     return HYMBA_OK;
 }
 
-template int launch_fuse<float, float>(const Ctx&, const float*, const float*, const float*, long long, int,
-                                       const float*, const float*, const float*, const float*, float*, int, int,
-                                       float, int*);
-template int launch_fuse<f16, bf16>(const Ctx&, const f16*, const f16*, const f16*, long long, int, const float*,
-                                    const float*, const float*, const float*, bf16*, int, int, float, int*);
-template int launch_fuse<f16, f16>(const Ctx&, const f16*, const f16*, const f16*, long long, int, const float*,
-                                   const float*, const float*, const float*, f16*, int, int, float, int*);
+template int launch_fuse<float, float>(const Ctx&, const float*, const float*, int, int, const float*,
+                                       const float*, long long, int, const float*, const float*, const float*,
+                                       const float*, float*, int, int, float, int*);
+template int launch_fuse<f16, bf16>(const Ctx&, const f16*, const float*, int, int, const f16*, const f16*,
+                                    long long, int, const float*, const float*, const float*, const float*,
+                                    bf16*, int, int, float, int*);
+template int launch_fuse<f16, f16>(const Ctx&, const f16*, const float*, int, int, const f16*, const f16*,
+                                   long long, int, const float*, const float*, const float*, const float*,
+                                   f16*, int, int, float, int*);
 
 }  // namespace hymba

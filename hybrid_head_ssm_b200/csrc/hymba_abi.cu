@@ -330,7 +330,7 @@ static int prefill_impl(const Ctx& ctx, const hymba_layer_cfg* c, const hymba_la
                                           st ? st->conv : nullptr, B, Tp, di)))
         return rc;
     // 5. gate, norms, beta, average --------------------------------------------------
-    if ((rc = launch_fuse<I, TA>(ctx, O, ypre, P, pl.ldP, k.z, w->norm_attn_w, w->norm_ssm_w, w->beta1,
+    if ((rc = launch_fuse<I, TA>(ctx, O, nullptr, 0, 0, ypre, P, pl.ldP, k.z, w->norm_attn_w, w->norm_ssm_w, w->beta1,
                                  w->beta2, U, (int)rows, di, c->rms_eps, nullptr)))
         return rc;
     // 6. output projection (+ residual) -------------------------------------------------
@@ -362,23 +362,12 @@ static int decode_impl(const Ctx& ctx, const hymba_layer_cfg* c, const hymba_lay
     const int H = c->n_q_heads, G = c->n_kv_heads, dh = c->head_dim, dv = c->v_head_dim;
     const int pos_offset = c->is_kv_producer ? 0 : -1;
     I* P = reinterpret_cast<I*>(ws + pl.P);
-    float* delta = reinterpret_cast<float*>(ws + pl.delta);
-    I* O = reinterpret_cast<I*>(ws + pl.O);
     I* ypre = reinterpret_cast<I*>(ws + pl.ypre);
     T* U = reinterpret_cast<T*>(ws + pl.U);
-    I* wdt = reinterpret_cast<I*>(ws + pl.wdt);
     float* part = reinterpret_cast<float*>(ws + pl.part);
     I* k_cache = static_cast<I*>(kv->k_cache);
     I* v_cache = static_cast<I*>(kv->v_cache);
     int rc;
-    const T* x;
-    if constexpr (std::is_same<TIO, T>::value) {
-        x = x_io;
-    } else {
-        T* xc = reinterpret_cast<T*>(ws + pl.xcv);
-        if ((rc = launch_pad_copy<TIO, T>(ctx, x_io, B, d, xc, d))) return rc;
-        x = xc;
-    }
     EpiArgs<I> ep = epi_base<I>(EPI_INPROJ, B, k.n_in);
     ep.row_mode = ROWS_DECODE;
     ep.B = B; ep.Tu = 1; ep.Tp = 1; ep.n_meta = m;
@@ -390,24 +379,34 @@ static int decode_impl(const Ctx& ctx, const hymba_layer_cfg* c, const hymba_lay
     ep.pos = kv->len; ep.pos_offset = pos_offset;
     ep.n_meta_ring = kv->cache_cap - m;
     ep.rope_base = c->rope_base;
-    // RoPE table of the new positions and the padded 16-bit W_dt, one launch
+    // RoPE table of the new positions and, for a fp32 residual stream, the new rows in
+    // the layer's type: one launch
     float2* rope = reinterpret_cast<float2*>(ws + pl.rope);
-    if ((rc = launch_decode_prep<T, I>(ctx, rope, kv->len, pos_offset, B, dh, c->rope_base,
-                                       static_cast<const T*>(w->w_dt), di, c->dt_rank, wdt, pl.rpad)))
-        return rc;
+    const T* x;
+    if constexpr (std::is_same<TIO, T>::value) {
+        x = x_io;
+        rc = launch_decode_prep<T, T>(ctx, rope, kv->len, pos_offset, B, dh, c->rope_base, nullptr, 0, 0,
+                                      nullptr, 0);
+    } else {
+        T* xc = reinterpret_cast<T*>(ws + pl.xcv);
+        rc = launch_decode_prep<TIO, T>(ctx, rope, kv->len, pos_offset, B, dh, c->rope_base, x_io, B, d, xc, d);
+        x = xc;
+    }
+    if (rc) return rc;
     ep.rope = rope;
     if ((rc = gemm<T, I>(ctx, "gemm_in_proj_decode", x, d, static_cast<const T*>(w->w_in), d, B, k.n_in, d, ep))) return rc;
-    EpiArgs<I> ed = epi_base<I>(EPI_DELTA, B, di);
-    ed.delta = delta; ed.b_dt = w->b_dt;
-    if ((rc = gemm<I, I>(ctx, "gemm_dt_proj_decode", P + k.dtl, pl.ldP, wdt, pl.rpad, B, di, c->dt_rank, ed))) return rc;
+    // split-KV attention, left as partials that the fusion kernel merges
     if ((rc = launch_attn_decode<I>(ctx, P, pl.ldP, k_cache, v_cache, kv->cache_cap, kv->len, pos_offset,
-                                    part, pl.n_split, O, B, H, G, dv, m, c->window)))
+                                    part, pl.n_split, nullptr, B, H, G, dv, m, c->window)))
         return rc;
-    if ((rc = launch_ssm_decode<I>(ctx, P, pl.ldP, k.x, k.Bc, k.Cc, delta, w->conv_w, w->conv_b, w->A_log,
-                                   w->D, st->h, st->conv, ypre, B, di)))
+    // SSM step with the Delta projection of the new rows folded in
+    if ((rc = launch_ssm_decode<I, T>(ctx, P, pl.ldP, k.x, k.Bc, k.Cc, k.dtl, static_cast<const T*>(w->w_dt),
+                                      w->b_dt, c->dt_rank, w->conv_w, w->conv_b, w->A_log, w->D, st->h,
+                                      st->conv, ypre, B, di)))
         return rc;
-    if ((rc = launch_fuse<I, T>(ctx, O, ypre, P, pl.ldP, k.z, w->norm_attn_w, w->norm_ssm_w, w->beta1,
-                                w->beta2, U, B, di, c->rms_eps, c->is_kv_producer ? kv->len : nullptr)))
+    if ((rc = launch_fuse<I, T>(ctx, nullptr, part, pl.n_split, H, ypre, P, pl.ldP, k.z, w->norm_attn_w,
+                                w->norm_ssm_w, w->beta1, w->beta2, U, B, di, c->rms_eps,
+                                c->is_kv_producer ? kv->len : nullptr)))
         return rc;
     EpiArgs<TIO> eo = epi_base<TIO>(EPI_OUT, B, d);
     eo.y = y;

@@ -41,10 +41,13 @@ int launch_conv_scan_prefill(const Ctx& ctx, const T* P, long long ldP, int col_
                              float* h_out, float* conv_out, int B, int Tp, int di);
 
 // RMSNorm of both branches, SiLU(z) gate, beta scaling and average; one row per block.
+// The attention branch is O [rows, di], or, when `part` is given, the decode
+// attention's split partials [rows, H, n_split, di/H + 2] merged on the fly (O unused).
 template <typename I, typename T>
-int launch_fuse(const Ctx& ctx, const I* O, const I* ypre, const I* P, long long ldP, int col_z,
-                const float* g_attn, const float* g_ssm, const float* beta1, const float* beta2,
-                T* U, int rows, int di, float eps, int* len_inc);
+int launch_fuse(const Ctx& ctx, const I* O, const float* part, int n_split, int H, const I* ypre,
+                const I* P, long long ldP, int col_z, const float* g_attn, const float* g_ssm,
+                const float* beta1, const float* beta2, T* U, int rows, int di, float eps,
+                int* len_inc);
 
 
 // The RoPE table and the zero-padded 16-bit copy of W_dt [rows, cols] -> [rows, ld_dst],
@@ -53,8 +56,10 @@ template <typename TS, typename TD>
 int launch_prefill_prep(const Ctx& ctx, float2* tab, int Tp, int dh, float base, const TS* w, int rows, int cols,
                         TD* wdst, int ld_dst);
 
-// The RoPE table of a decode step's new positions ([B, dh/2] (cos, sin)) and the
-// zero-padded 16-bit copy of W_dt, in one launch.
+// The RoPE table of a decode step's new positions ([B, dh/2] (cos, sin)) and a copy
+// of the [rows, cols] matrix w converted to TD into [rows, ld_dst] (zero-padded; the
+// decode step's input rows when they arrive in another type; rows = 0: none), in one
+// launch.
 template <typename TS, typename TD>
 int launch_decode_prep(const Ctx& ctx, float2* tab, const int* len, int pos_offset, int B, int dh, float base,
                        const TS* w, int rows, int cols, TD* wdst, int ld_dst);
@@ -70,19 +75,21 @@ int launch_cache_fill(const Ctx& ctx, const T* k_seq, const T* v_seq, int seq_ca
                       int n_meta, int Tp);
 
 // Decode attention: one query per (sequence, head) over the cache; split over keys,
-// partial results in `part` [B, H, n_split, dv + 2] fp32, then combined into O.
+// partial results in `part` [B, H, n_split, dv + 2] fp32, then combined into O
+// (O == nullptr: left as partials for the fusion kernel to merge).
 template <typename T>
 int launch_attn_decode(const Ctx& ctx, const T* P, long long ldP, const T* k_cache,
                        const T* v_cache, int cache_cap, const int* len, int pos_offset,
                        float* part, int n_split, T* O, int B, int H, int G, int dv, int n_meta,
                        int window);
 
-// One SSM decode step per (sequence, channel): conv-state shift, conv, SiLU, scan
-// step on h in place, y_pre = C.h + D xc.
-template <typename T>
-int launch_ssm_decode(const Ctx& ctx, const T* P, long long ldP, int col_x, int col_B,
-                      int col_C, const float* delta, const float* conv_w, const float* conv_b,
-                      const float* A_log, const float* D, float* h, float* conv, T* ypre, int B,
-                      int di);
+// One SSM decode step per (sequence, channel): Delta = softplus(dt_low W_dt^T + b_dt)
+// from the projection row's dt_low columns, conv-state shift, conv, SiLU, scan step on
+// h in place, y_pre = C.h + D xc. W_dt is [di, dt_rank] in the layer's weight type.
+template <typename T, typename TW>
+int launch_ssm_decode(const Ctx& ctx, const T* P, long long ldP, int col_x, int col_B, int col_C,
+                      int col_dtl, const TW* w_dt, const float* b_dt, int dt_rank,
+                      const float* conv_w, const float* conv_b, const float* A_log, const float* D,
+                      float* h, float* conv, T* ypre, int B, int di);
 
 }  // namespace hymba

@@ -38,7 +38,7 @@ __global__ void prefill_prep_kernel(float2* tab, int Tp, int half, int dh, float
 // The small inputs of a decode step in one launch: blocks [0, nb_rope) fill the RoPE
 // table of each sequence's new position (len[b] + pos_offset; rows without a valid
 // position get the identity rotation, their outputs are never written), the rest copy
-// W_dt into its zero-padded 16-bit form.
+// the step's input rows into the layer's compute type when they arrive in another.
 template <typename TS, typename TD>
 __global__ void decode_prep_kernel(float2* tab, const int* len, int pos_offset, int B, int half, int dh, float base,
                                    int nb_rope, const TS* w, int rows, int cols, TD* wdst, int ld_dst) {
@@ -131,8 +131,10 @@ template int launch_prefill_prep<float, float>(const Ctx&, float2*, int, int, fl
 template int launch_prefill_prep<bf16, f16>(const Ctx&, float2*, int, int, float, const bf16*, int, int, f16*, int);
 template int launch_decode_prep<float, float>(const Ctx&, float2*, const int*, int, int, int, float, const float*,
                                               int, int, float*, int);
-template int launch_decode_prep<bf16, f16>(const Ctx&, float2*, const int*, int, int, int, float, const bf16*, int, int,
-                                           f16*, int);
+template int launch_decode_prep<bf16, bf16>(const Ctx&, float2*, const int*, int, int, int, float, const bf16*, int,
+                                            int, bf16*, int);
+template int launch_decode_prep<float, bf16>(const Ctx&, float2*, const int*, int, int, int, float, const float*, int,
+                                             int, bf16*, int);
 template int launch_cache_fill<float>(const Ctx&, const float*, const float*, int, float*, float*,
                                       int, int*, int, int, int, int, int, int);
 template int launch_cache_fill<f16>(const Ctx&, const f16*, const f16*, int, f16*, f16*, int,

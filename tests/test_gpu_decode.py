@@ -92,9 +92,12 @@ def test_tiny_f32_pair_decode_matches_oracle(window):
     assert g.hy.hymba_get_device_status(None) == 0
 
 
-def test_bf16_small_pair_decode_matches_oracle():
+@pytest.mark.parametrize("dt_rank", [24, 130, 264])
+def test_bf16_small_pair_decode_matches_oracle(dt_rank):
+    """The decode SSM step stages W_dt with wide loads for an even dt_rank <= 128 (24)
+    and with its general loop otherwise: one pass (130) or two (264)."""
     base = synth.hymba15_layer_cfg(window=24).with_(d_model=256, n_q_heads=5, n_kv_heads=1,
-                                                    d_inner=640, dt_rank=24, n_meta=8)
+                                                    d_inner=640, dt_rank=dt_rank, n_meta=8)
     ca, cb = base, base.with_(is_kv_producer=0)
     wa = synth.layer_weights(ca, 71)
     wb = synth.layer_weights(cb, 72)

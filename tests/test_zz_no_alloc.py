@@ -1,8 +1,9 @@
 """hymba_attn_decode_static: the decode attention for callers that cannot allocate
 device memory (no workspace argument; its scratch is a fixed device array inside the
-library). Checked against the attention output that hymba_mixer_decode leaves in its
-workspace for the same query and cache, on two calls in a row (the second call
-reuses the array the first one left behind).
+library). Checked against the attention of hymba_mixer_decode for the same query and
+cache: the mixer leaves its split-KV partials in its workspace, merged here on the host
+by the softmax rescaling rule, on two calls in a row (the second call reuses the array
+the first one left behind).
 
 This file is named to be collected last, so that a run stopping at the first
 failure has already run every other test."""
@@ -42,8 +43,21 @@ def _decoded_layer(cfg, B, T0, cache_cap, seed):
     ldp = lay["ldP"]
     # the query rows (after RoPE) sit in the projection block of the workspace
     q = ws[lay["P"]:lay["P"] + B * ldp * esz].view(mdt).view(B, ldp)
-    o_ref = ws[lay["O"]:lay["O"] + B * H * dv * esz].view(mdt).view(B, H * dv).float().cpu().numpy()
+    ns = lay["n_split"]
+    n_part = B * H * ns * (dv + 2)
+    part = ws[lay["part"]:lay["part"] + n_part * 4].view(torch.float32).view(B, H, ns, dv + 2)
+    o_ref = _merge_splits(part.double().cpu().numpy()).reshape(B, H * dv)
     return dict(layer=layer, kv=kv, q=q, ldp=ldp, o_ref=o_ref, mdt=mdt)
+
+
+def _merge_splits(part):
+    """Softmax over the union of the key splits from per-split partials [..., dv + 2]:
+    dv unnormalised sums of p v, then the split's max logit (base-2 domain) and its sum
+    of p. Each split is rescaled by 2^(m_s - max m) before the sums are divided."""
+    num, m, l = part[..., :-2], part[..., -2], part[..., -1]
+    M = m.max(axis=-1, keepdims=True)
+    w = np.where(np.isfinite(m), np.exp2(m - M), 0.0)
+    return (w[..., None] * num).sum(axis=-2) / (w * l).sum(axis=-1)[..., None]
 
 
 @pytest.mark.parametrize("kind", ["bf16_hymba15_ring", "f32_tiny_global"])
