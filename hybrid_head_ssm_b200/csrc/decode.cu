@@ -7,6 +7,7 @@
 // Cache layout: k_cache [B, G, cap, dh], v_cache [B, G, cap, dv]; position p < n_meta
 // in slot p, position p >= n_meta in slot n_meta + (p - n_meta) mod (cap - n_meta).
 #include "kernels.h"
+#include "tc.cuh"
 
 namespace hymba {
 
@@ -41,6 +42,13 @@ __device__ __forceinline__ void load_row8(const T* p, float* v) {
         v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
         v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
     }
+}
+
+// An fp16 pair (the raw bits of two f16) as two floats.
+__device__ __forceinline__ float2 x2float(uint32_t v) {
+    __half2 h;
+    memcpy(&h, &v, 4);
+    return __half22float2(h);
 }
 
 constexpr int KGROUPS = 8;  // key groups of the PV phase (128 threads = 8 groups x 16 pieces of 8)
@@ -205,6 +213,213 @@ attn_decode_kernel(const T* __restrict__ P, long long ldP, const T* __restrict__
     }
 }
 
+// ---------------------------------------------------------------------------
+// 16-bit K/V: the split's K and V rows staged in shared memory by bulk async copies
+// ---------------------------------------------------------------------------
+constexpr int BK_NST = 2;                      // stages
+constexpr int BK_STAGE = 16384;                // bytes per stage
+constexpr int BK_TK = BK_STAGE / (DH * 2);     // keys per K tile (128)
+constexpr int BK_TV = BK_STAGE / (128 * 2);    // keys per V tile (64)
+
+// Queue the bulk copies of one tile: the block-local keys [a, e) of the split, rows of
+// row_bytes, into dst in key order. The keys map to cache slots in at most three
+// contiguous runs (meta slots, then the ring up to its end, then from its start), one
+// copy per run; the tile's byte count is announced on `bar` first.
+__device__ __forceinline__ void bk_issue_tile(unsigned char* dst, const unsigned char* src, int row_bytes, int a,
+                                              int e, int k0, int meta_n, int lo, int n_meta, int cap, int ring,
+                                              uint64_t* bar) {
+    tc::mbar_arrive_expect_tx(bar, (uint32_t)((e - a) * row_bytes));
+    const int t0 = a;
+    while (a < e) {
+        const int idx = k0 + a;
+        int slot, run;
+        if (idx < meta_n) {
+            slot = idx;
+            run = min(e - a, meta_n - idx);
+        } else {
+            const int j = lo + (idx - meta_n);
+            slot = n_meta + (j - n_meta) % ring;
+            run = min(e - a, cap - slot);
+        }
+        tc::bulk_load(dst + (size_t)(a - t0) * row_bytes, src + (size_t)slot * row_bytes, (uint32_t)(run * row_bytes),
+                      bar);
+        a += run;
+    }
+}
+
+// One block per (key split, KV head, sequence) serves the R query heads of the KV head,
+// as attn_decode_kernel, with the split's K rows (128-key tiles) and then V rows
+// (64-key tiles) streamed through a two-stage shared-memory ring by bulk async copies:
+// the copies keep enough bytes in flight without holding them in registers. Scores:
+// eight lanes per key, each with its 8 dimensions of the R queries in registers, one
+// conflict-free 16-byte shared load per key, joined by three shuffles per head. P V:
+// warp w takes keys w, w + 4, ... of a tile, lane l elements 4l .. 4l + 3 of the V row.
+template <int R>
+__global__ void __launch_bounds__(128, R <= 6 ? 5 : 4)
+attn_decode_bulk_kernel(const f16* __restrict__ P, long long ldP, const f16* __restrict__ k_cache,
+                        const f16* __restrict__ v_cache, int cap, const int* __restrict__ len, int pos_offset,
+                        float* __restrict__ part, int n_split, int H, int G, int n_meta, int window, int max_chunk,
+                        int* status) {
+    griddep_sync();
+    constexpr int DV = 128;
+    static_assert(R >= 1 && R <= 8, "query heads per KV head");
+    static_assert(4 * R * DV * 4 <= BK_NST * BK_STAGE, "the reduction buffer reuses the stages");
+    extern __shared__ __align__(128) unsigned char bk_smem[];
+    __shared__ int bk_never;  // stays 0: the waits below give up on their own clock only
+    unsigned char* stages = bk_smem;
+    float (*ps)[8] = reinterpret_cast<float (*)[8]>(bk_smem + BK_NST * BK_STAGE);
+    float* stat = reinterpret_cast<float*>(bk_smem + BK_NST * BK_STAGE + (size_t)max_chunk * 32);
+    uint64_t* full = reinterpret_cast<uint64_t*>(stat + 16);
+    float* red = reinterpret_cast<float*>(stages);
+    const int s = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int p = len[b] + pos_offset;
+    const int ring = cap - n_meta;
+    int meta_n, lo;
+    const bool span_ok = decode_span(p, n_meta, window, ring, &meta_n, &lo);
+    if (!span_ok && s == 0 && g == 0 && tid == 0) set_status(status, HYMBA_ERR_DEVICE_RANGE);
+    const int L = span_ok ? meta_n + (p + 1 - lo) : 0;
+    const int chunk = (L + n_split - 1) / n_split;
+    const int k0 = min(L, s * chunk), k1 = min(L, k0 + chunk);
+    const int nk = k1 - k0;
+    const long long kvbase = ((long long)b * G + g) * cap;
+    const unsigned char* kbase = reinterpret_cast<const unsigned char*>(k_cache + kvbase * DH);
+    const unsigned char* vbase = reinterpret_cast<const unsigned char*>(v_cache + kvbase * DV);
+    const int nkt = (nk + BK_TK - 1) / BK_TK;
+    const int nitems = nk > 0 ? nkt + (nk + BK_TV - 1) / BK_TV : 0;
+    auto issue = [&](int i) {
+        unsigned char* dst = stages + (i % BK_NST) * BK_STAGE;
+        if (i < nkt)
+            bk_issue_tile(dst, kbase, DH * 2, i * BK_TK, min(nk, (i + 1) * BK_TK), k0, meta_n, lo, n_meta, cap, ring,
+                          &full[i % BK_NST]);
+        else
+            bk_issue_tile(dst, vbase, DV * 2, (i - nkt) * BK_TV, min(nk, (i - nkt + 1) * BK_TV), k0, meta_n, lo,
+                          n_meta, cap, ring, &full[i % BK_NST]);
+    };
+    if (tid == 0) {
+        bk_never = 0;
+        for (int i = 0; i < BK_NST; ++i) tc::mbar_init(&full[i], 1);
+        tc::fence_mbar_init();
+        for (int i = 0; i < min(BK_NST, nitems); ++i) issue(i);
+    }
+    // this lane's 8 dimensions of the R queries, scaled by log2(e) / sqrt(64)
+    const int ch = lane & 7, kl = lane >> 3;
+    float2 qr[R][4];
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+        float qv[8];
+        load_row8<f16>(P + (long long)b * ldP + (g * R + r) * DH + 8 * ch, qv);
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+            qr[r][i] = make_float2(qv[2 * i] * (LOG2E * 0.125f), qv[2 * i + 1] * (LOG2E * 0.125f));
+    }
+    float2 acc[R][2];
+#pragma unroll
+    for (int r = 0; r < R; ++r) acc[r][0] = acc[r][1] = make_float2(0.f, 0.f);
+    __syncthreads();
+    bool ok = true;
+    for (int i = 0; i < nitems; ++i) {
+        const int st = i % BK_NST;
+        if (ok) ok = tc::mbar_wait(&full[st], (uint32_t)((i / BK_NST) & 1), &bk_never);
+        const unsigned char* sp = stages + st * BK_STAGE;
+        if (i < nkt) {
+            const int base = i * BK_TK, n = min(nk - base, BK_TK);
+            for (int pass = 0; pass * 16 < n; ++pass) {
+                const int kt = pass * 16 + warp * 4 + kl;
+                const bool valid = kt < n;
+                float2 a2[R];
+#pragma unroll
+                for (int r = 0; r < R; ++r) a2[r] = make_float2(0.f, 0.f);
+                if (valid) {
+                    const uint4 u = *reinterpret_cast<const uint4*>(sp + kt * (DH * 2) + ch * 16);
+                    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+                    for (int i2 = 0; i2 < 4; ++i2) {
+                        const float2 kf = x2float(w[i2]);
+#pragma unroll
+                        for (int r = 0; r < R; ++r) a2[r] = __ffma2_rn(qr[r][i2], kf, a2[r]);
+                    }
+                }
+                float v = 0.f;
+#pragma unroll
+                for (int r = 0; r < R; ++r) {
+                    float a = a2[r].x + a2[r].y;
+                    a += __shfl_xor_sync(0xffffffffu, a, 1);
+                    a += __shfl_xor_sync(0xffffffffu, a, 2);
+                    a += __shfl_xor_sync(0xffffffffu, a, 4);
+                    if (ch == r) v = a;
+                }
+                if (valid && ch < R) ps[base + kt][ch] = v;
+            }
+        } else {
+            const int base = (i - nkt) * BK_TV, n = min(nk - base, BK_TV);
+#pragma unroll 2
+            for (int kv = warp; kv < n; kv += 4) {
+                const uint2 u = *reinterpret_cast<const uint2*>(sp + kv * (DV * 2) + lane * 8);
+                const float2 v0 = x2float(u.x), v1 = x2float(u.y);
+                const float4 pa = *reinterpret_cast<const float4*>(&ps[base + kv][0]);
+                float4 pb = make_float4(0.f, 0.f, 0.f, 0.f);
+                if constexpr (R > 4) pb = *reinterpret_cast<const float4*>(&ps[base + kv][4]);
+                const float pw[8] = {pa.x, pa.y, pa.z, pa.w, pb.x, pb.y, pb.z, pb.w};
+#pragma unroll
+                for (int r = 0; r < R; ++r) {
+                    const float2 pr = make_float2(pw[r], pw[r]);
+                    acc[r][0] = __ffma2_rn(pr, v0, acc[r][0]);
+                    acc[r][1] = __ffma2_rn(pr, v1, acc[r][1]);
+                }
+            }
+        }
+        // the stage is free once every warp is past this barrier
+        if (__syncthreads_or(!ok)) {
+            if (tid == 0) {
+                tc::record_timeout(status, 3, i, st);
+                // let the copies already queued land before the block's memory is released
+                for (int q = i; q < min(nitems, i + BK_NST); ++q)
+                    tc::mbar_wait(&full[q % BK_NST], (uint32_t)((q / BK_NST) & 1), &bk_never);
+            }
+            return;
+        }
+        if (tid == 0 && i + BK_NST < nitems) issue(i + BK_NST);
+        if (i == nkt - 1) {
+            // every score of the split is in: per-head max and sum, warp w heads w, w + 4
+            for (int r = warp; r < R; r += 4) {
+                float mx = -INFINITY;
+                for (int kk = lane; kk < nk; kk += 32) mx = fmaxf(mx, ps[kk][r]);
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+                float sum = 0.f;
+                for (int kk = lane; kk < nk; kk += 32) {
+                    const float e = exp2f(ps[kk][r] - mx);
+                    ps[kk][r] = e;
+                    sum += e;
+                }
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+                if (lane == 0) { stat[2 * r] = mx; stat[2 * r + 1] = sum; }
+            }
+            __syncthreads();
+        }
+    }
+    // the four warps' P V sums meet in the stage memory (every copy has landed)
+#pragma unroll
+    for (int r = 0; r < R; ++r)
+        *reinterpret_cast<float4*>(&red[(warp * R + r) * DV + 4 * lane]) =
+            make_float4(acc[r][0].x, acc[r][0].y, acc[r][1].x, acc[r][1].y);
+    __syncthreads();
+    for (int i = tid; i < R * DV; i += blockDim.x) {
+        const int r = i / DV, e = i % DV;
+        float sum = 0.f;
+#pragma unroll
+        for (int w = 0; w < 4; ++w) sum += red[(w * R + r) * DV + e];
+        part[(((long long)b * H + g * R + r) * n_split + s) * (DV + 2) + e] = sum;
+    }
+    if (tid < R) {
+        float* o = part + (((long long)b * H + g * R + tid) * n_split + s) * (DV + 2) + DV;
+        o[0] = nk > 0 ? stat[2 * tid] : -INFINITY;
+        o[1] = nk > 0 ? stat[2 * tid + 1] : 0.f;
+    }
+}
+
 template <typename T, int DV>
 __global__ void __launch_bounds__(DV)
 attn_decode_combine_kernel(const float* __restrict__ part, int n_split, T* __restrict__ O, int H) {
@@ -244,11 +459,6 @@ __device__ __forceinline__ float2 wunpack(uint32_t v) {
 __device__ __forceinline__ float2 wpack(float lo, float hi) { return make_float2(lo, hi); }
 __device__ __forceinline__ uint32_t wpack(bf16 lo, bf16 hi) {
     return (uint32_t)__bfloat16_as_ushort(lo) | ((uint32_t)__bfloat16_as_ushort(hi) << 16);
-}
-__device__ __forceinline__ float2 x2float(uint32_t v) {  // an fp16 pair
-    __half2 h;
-    memcpy(&h, &v, 4);
-    return __half22float2(h);
 }
 
 // One decode step of the selective SSM for (sequence b, channel c), with the Delta
@@ -483,6 +693,31 @@ int launch_attn_decode(const Ctx& ctx, const T* P, long long ldP, const T* k_cac
     if ((reinterpret_cast<uintptr_t>(P) | reinterpret_cast<uintptr_t>(k_cache) | reinterpret_cast<uintptr_t>(v_cache)) & 15 ||
         ldP % (16 / (long long)sizeof(T)))
         return HYMBA_ERR_UNSUPPORTED;
+    if constexpr (std::is_same<T, f16>::value) {
+        // K/V rows staged by bulk copies: 16-byte aligned rows (64 and 128 fp16)
+        const int max_chunk = (cache_cap + n_split - 1) / n_split;
+        const size_t smem = (size_t)BK_NST * BK_STAGE + (size_t)max_chunk * 32 + 16 * sizeof(float) +
+                            BK_NST * sizeof(uint64_t);
+        void (*kb)(const f16*, long long, const f16*, const f16*, int, const int*, int, float*, int, int, int, int,
+                   int, int, int*);
+        switch (H / G) {
+            case 1: kb = attn_decode_bulk_kernel<1>; break;
+            case 2: kb = attn_decode_bulk_kernel<2>; break;
+            case 3: kb = attn_decode_bulk_kernel<3>; break;
+            case 4: kb = attn_decode_bulk_kernel<4>; break;
+            case 5: kb = attn_decode_bulk_kernel<5>; break;
+            case 6: kb = attn_decode_bulk_kernel<6>; break;
+            case 7: kb = attn_decode_bulk_kernel<7>; break;
+            default: kb = attn_decode_bulk_kernel<8>; break;
+        }
+        HYMBA_LAUNCH(ctx, "attn_decode", kb, grid, 128, smem, P, ldP, k_cache, v_cache, cache_cap, len, pos_offset,
+                     part, n_split, H, G, n_meta, window, max_chunk, ctx.status);
+        if (!O) return HYMBA_OK;  // the caller merges the splits itself
+        dim3 g2(H, B);
+        auto k2 = attn_decode_combine_kernel<T, 128>;
+        HYMBA_LAUNCH(ctx, "attn_decode_combine", k2, g2, 128, 0, part, n_split, O, H);
+        return HYMBA_OK;
+    }
     void (*k1)(const T*, long long, const T*, const T*, int, const int*, int, float*, int, int, int, int, int, int*);
     switch (H / G) {
         case 1: k1 = attn_decode_kernel<T, 128, 1>; break;
