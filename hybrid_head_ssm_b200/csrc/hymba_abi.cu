@@ -154,7 +154,9 @@ static size_t take(size_t* cur, size_t bytes) {
     return off;
 }
 
-static int decode_splits(int cache_cap) { return ceil_div(cache_cap > 0 ? cache_cap : 1, 256); }
+// 128-key splits: the 16-bit decode attention streams each split through its shared
+// memory ring in one K tile and two V tiles, and more, shorter blocks fill the waves
+static int decode_splits(int cache_cap) { return ceil_div(cache_cap > 0 ? cache_cap : 1, 128); }
 
 static Plan plan(const hymba_layer_cfg* c, int B, int T, int mode) {
     Plan p;
