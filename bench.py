@@ -20,9 +20,9 @@ import hashlib
 import json
 import os
 import statistics
-import threading
 import subprocess
 import sys
+import tempfile
 import time
 
 import numpy as np
@@ -110,14 +110,14 @@ class Clocks:
     setting is touched), polled about every millisecond by a separate process so that
     the polling does not compete with this one; only the samples taken while the timed
     region is open (wall clock) are reported. The samples go to
-    gpurun_out/clocks_rank<i>.csv."""
+    <clocks_dir>/clocks_rank<i>.csv (`--clocks-dir`, default the system temp directory)."""
 
     REASONS = (("hw_slowdown", 0x8), ("hw_thermal_slowdown", 0x40), ("sw_thermal_slowdown", 0x20),
                ("sw_power_cap", 0x4))
 
-    def __init__(self, cuda_index: int):
+    def __init__(self, cuda_index: int, clocks_dir: str = ""):
         self.cuda_index = cuda_index
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{cuda_index}.csv")
+        self.path = os.path.join(clocks_dir or tempfile.gettempdir(), f"clocks_rank{cuda_index}.csv")
         self.stop_path = self.path + ".stop"
         self.proc = None
         self.t0 = self.t1 = None
@@ -290,6 +290,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--clocks-dir", default="",
+                    help="where the NVML clock samples are written (default: the system temp directory)")
     ap.add_argument("--no-decode", action="store_true")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
@@ -335,7 +337,7 @@ def main():
     def step(xin=None, yout=None):
         rt.prefill(layer, x if xin is None else xin, T, kv, y if yout is None else yout, ws, None, 0)
 
-    clocks = Clocks(local)
+    clocks = Clocks(local, args.clocks_dir)
     clocks.start()
     for _ in range(args.warmup):
         step()

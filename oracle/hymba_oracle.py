@@ -27,7 +27,7 @@ the order the pages give the steps. Sources, cited by page title and section:
   RoPE, sliding-window attention in most layers with 3 full-attention layers,
   KV shared between pairs of layers.
 
-Readings taken where the pages are silent (each is listed in the design doc):
+Readings taken where the pages are silent:
 
 * Fusion of the two branches: each branch is RMS-normalised over its full
   width, scaled per channel by beta1 / beta2, and the two are averaged before
