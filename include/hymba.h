@@ -255,8 +255,9 @@ int hymba_get_device_status(void* stream);
 
 /* Where the first bounded device wait that ran out gave up (after a call reported
  * HYMBA_ERR_DEVICE_TIMEOUT): out[0] 1 if a record exists, out[1..3] the block index
- * (x, y, z), out[4] the role (0 TMA producer, 1 MMA issuer, 2 epilogue/softmax), out[5]
- * the step (k-block or key block), out[6] the barrier. Synchronises the device and
+ * (x, y, z), out[4] the role (0 TMA producer, 1 MMA issuer, 2 epilogue/softmax, 3 decode
+ * attention waiting for its bulk copies), out[5] the step (k-block, key block or copy
+ * tile), out[6] the barrier (or stage). Synchronises the device and
  * clears the record. Requires n >= 7. */
 int hymba_get_device_diag(int32_t* out, int n);
 
@@ -268,7 +269,11 @@ int hymba_get_device_diag(int32_t* out, int n);
  * [rows, d_inner] dtype (before the SiLU(z) gate), out[6] of the fused U [rows,
  * d_inner] dtype, out[7] of the RoPE table, out[8] of the decode split partials,
  * out[9] the decode split count. rows = B * (n_meta + T) for prefill, B for decode
- * (where T is the cache_cap of the KV cache). Requires n >= 10. */
+ * (where T is the cache_cap of the KV cache). A decode step writes neither Delta (it
+ * stays in the SSM step's registers) nor O: its attention stays as the split partials
+ * [B, n_q_heads, splits, v_head_dim + 2] fp32 (per split: the unnormalised sum of
+ * p v, the split's max logit in base 2, the sum of p), which the fusion merges.
+ * Requires n >= 10. */
 int hymba_workspace_layout(const hymba_layer_cfg* cfg, int B, int T, int mode, int64_t* out, int n);
 
 /* Static description of a status code. */
