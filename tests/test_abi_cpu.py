@@ -68,6 +68,10 @@ def test_workspace_layout_is_consistent(hy):
     assert len(set(offs)) == 5
     dec = hy.workspace_layout(c, 64, 1152, hy.HYMBA_MODE_DECODE)
     assert dec["n_split"] >= 1 and dec["part"] > 0
+    # every split holds at most 256 keys (the decode attention's score buffer), and the
+    # partials [B, H, splits, v_head_dim + 2] fp32 fit the last segment
+    assert -(-1152 // dec["n_split"]) <= 256
+    assert dec["total"] - dec["part"] >= 64 * cfg.n_q_heads * dec["n_split"] * (cfg.v_head_dim + 2) * 4
 
 
 def test_invalid_configs_rejected(hy):
@@ -109,6 +113,39 @@ def test_prefill_argument_errors_before_any_launch(hy):
     rc = hy.hymba_mixer_prefill(ctypes.byref(c), ctypes.byref(wf), 1 << 24, 1, 10, 0, (1 << 24) + 64,
                                 ctypes.byref(kvf), None, 1 << 30, 1 << 40, None)
     assert rc == hy.HYMBA_ERR_INVALID_ARG
+
+
+def test_decode_argument_errors_before_any_launch(hy):
+    """Every argument check of hymba_mixer_decode runs before the device is touched
+    (fake host addresses, never dereferenced)."""
+    cfg = synth.tiny_layer_cfg().with_(window=8)
+    c = hy.cfg_struct(cfg)
+    fake = 1 << 20
+    wf = hy.hymba_layer_weights(*([fake] * 13))
+    B = 2
+    kv = hy.kv_struct(cfg, B)
+    kv.k_cache = kv.v_cache = kv.len = fake
+    kv.cache_cap = cfg.n_meta + 8
+    st = hy.hymba_ssm_state(fake, fake)
+    need = hy.hymba_workspace_bytes(ctypes.byref(c), B, kv.cache_cap, hy.HYMBA_MODE_DECODE)
+    assert need > 0
+
+    def call(cfg_s=c, x=1 << 24, flags=0, kv_s=kv, st_s=st, ws=1 << 30, ws_bytes=need, b=B):
+        return hy.hymba_mixer_decode(ctypes.byref(cfg_s), ctypes.byref(wf), x, b, flags, 1 << 26,
+                                     ctypes.byref(kv_s), ctypes.byref(st_s), ws, ws_bytes, None)
+
+    assert call(ws_bytes=need - 256) == hy.HYMBA_ERR_WORKSPACE_TOO_SMALL
+    assert call(x=None) == hy.HYMBA_ERR_INVALID_ARG
+    assert call(b=0) == hy.HYMBA_ERR_INVALID_ARG
+    assert call(st_s=hy.hymba_ssm_state(None, fake)) == hy.HYMBA_ERR_INVALID_ARG
+    assert call(ws=(1 << 30) + 64) == hy.HYMBA_ERR_INVALID_ARG           # not 256-byte aligned
+    assert call(flags=hy.HYMBA_IO_F32) == hy.HYMBA_ERR_INVALID_ARG       # fp32 layer
+    assert call(flags=1 << 12) == hy.HYMBA_ERR_INVALID_ARG               # unknown flag
+    short = hy.kv_struct(cfg, B)
+    short.k_cache = short.v_cache = short.len = fake
+    short.cache_cap = cfg.n_meta                                          # no ring slot
+    assert call(kv_s=short) == hy.HYMBA_ERR_INVALID_ARG
+    assert call(cfg_s=hy.cfg_struct(cfg.with_(head_dim=48))) == hy.HYMBA_ERR_UNSUPPORTED
 
 
 def test_kv_share_rules(hy):
