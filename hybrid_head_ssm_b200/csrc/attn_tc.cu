@@ -411,13 +411,8 @@ int launch_attn_prefill_tc(const Ctx& ctx, const f16* P, long long ldP, const f1
         !tc::make_tmap_3d(&tv, v_seq, false, (uint64_t)B * G, Tp, DV, DV, (uint64_t)kcap * DV, KBLK))
         return HYMBA_ERR_UNSUPPORTED;
     const size_t smem = sizeof(AttnSmem) + 1024;
-    static bool attr_set = false;
-    if (!attr_set) {
-        if (cudaFuncSetAttribute(attn_prefill_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
-            cudaSuccess)
-            return HYMBA_ERR_CUDA;
-        attr_set = true;
-    }
+    static std::atomic<unsigned long long> smem_set{0};
+    if (!smem_opt_in_once(smem_set, attn_prefill_tc_kernel, smem, ctx)) return HYMBA_ERR_CUDA;
     dim3 grid(ceil_div(Tp, QT), H, B);
     HYMBA_LAUNCH(ctx, "attn_prefill", attn_prefill_tc_kernel, grid, NTHREADS, smem, tq, tk, tv, O, Tp, H, G,
                  n_meta, window, ctx.status);

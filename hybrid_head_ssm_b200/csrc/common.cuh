@@ -5,6 +5,7 @@
 #include <cuda_fp16.h>
 #include <stdint.h>
 
+#include <atomic>
 #include <utility>
 
 #include "../../include/hymba.h"
@@ -21,6 +22,7 @@ struct Ctx {
     cudaStream_t stream;
     int* status;   // device status word of the current device
     int sm_count;
+    int device;    // current device (0..63)
 };
 
 // records the start event when tracing covers this kernel
@@ -57,6 +59,20 @@ static inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 b
             ::hymba::launch_pdl(kernel, dim3(grid), dim3(block), (size_t)(smem), (ctx).stream, __VA_ARGS__); \
         if (::hymba::trace_after((ctx), (name)) || launch_err_ != cudaSuccess) return HYMBA_ERR_CUDA; \
     } while (0)
+
+// Opt `kernel` in to `smem` bytes of dynamic shared memory on the context's device, once
+// per device: the attribute belongs to the device's context, so a process driving several
+// GPUs sets it on each. `done` is the caller's mask of devices already set; threads that
+// race here both set the same value.
+template <typename K>
+static inline bool smem_opt_in_once(std::atomic<unsigned long long>& done, K kernel, size_t smem, const Ctx& ctx) {
+    const unsigned long long bit = 1ull << ctx.device;
+    if (done.load(std::memory_order_acquire) & bit) return true;
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+        return false;
+    done.fetch_or(bit, std::memory_order_release);
+    return true;
+}
 
 static inline int ceil_div(long long a, long long b) { return (int)((a + b - 1) / b); }
 static inline long long round_up(long long a, long long b) { return (a + b - 1) / b * b; }

@@ -252,12 +252,8 @@ int launch_bn(const Ctx& ctx, const char* name, const TA* A, long long lda, cons
     }
     const size_t smem = sizeof(GemmSmem<BN, STAGES>) + 1024;
     auto kern = gemm_tc_kernel<TA, TO, BN, STAGES>;
-    static bool attr_set = false;
-    if (!attr_set) {
-        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
-            return HYMBA_ERR_CUDA;
-        attr_set = true;
-    }
+    static std::atomic<unsigned long long> smem_set{0};
+    if (!smem_opt_in_once(smem_set, kern, smem, ctx)) return HYMBA_ERR_CUDA;
     const int tiles = ((M0 + BM - 1) / BM + (M + BM - 1) / BM) * ((N + BN - 1) / BN);
     const int slots = ctx.sm_count * (STAGES == 2 ? 2 : 1);
     const int grid = tiles < slots ? tiles : slots;

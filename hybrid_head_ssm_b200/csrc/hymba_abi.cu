@@ -44,6 +44,7 @@ static int current_ctx(cudaStream_t stream, Ctx* ctx) {
     ctx->stream = stream;
     ctx->status = g_status_ptr[dev];
     ctx->sm_count = g_sm_count[dev];
+    ctx->device = dev;
     return HYMBA_OK;
 }
 

@@ -342,12 +342,8 @@ int launch_conv_scan_prefill(const Ctx& ctx, const T* P, long long ldP, int col_
     dim3 grid(di / CPB, B);
     const size_t smem = sizeof(Smem<T>);
     auto kern = conv_scan_prefill_kernel<T>;
-    static bool attr_set = false;
-    if (!attr_set) {
-        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
-            return HYMBA_ERR_CUDA;
-        attr_set = true;
-    }
+    static std::atomic<unsigned long long> smem_set{0};
+    if (!smem_opt_in_once(smem_set, kern, smem, ctx)) return HYMBA_ERR_CUDA;
     HYMBA_LAUNCH(ctx, "conv_scan_prefill", kern, grid, NTH, smem, P, ldP, col_x, col_B, col_C, delta, conv_w, conv_b,
                  A_log, D, ypre, h_out, conv_out, Tp, di);
     return HYMBA_OK;
