@@ -38,3 +38,13 @@ def assert_close(got, ref, cfg, what="", max_abs=None, rel_l2=None):
 
 def to_np(t):
     return t.float().cpu().numpy().astype(np.float64)
+
+
+def merge_split_partials(part):
+    """Softmax over the union of the key splits from per-split partials [..., dv + 2]:
+    dv unnormalised sums of p v, then the split's max logit (base-2 domain) and its sum
+    of p. Each split is rescaled by 2^(m_s - max m) before the sums are divided."""
+    num, m, l = part[..., :-2], part[..., -2], part[..., -1]
+    M = m.max(axis=-1, keepdims=True)
+    w = np.where(np.isfinite(m), np.exp2(m - M), 0.0)
+    return (w[..., None] * num).sum(axis=-2) / (w * l).sum(axis=-1)[..., None]

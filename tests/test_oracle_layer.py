@@ -58,6 +58,36 @@ def test_decode_by_decode_equals_prefill_pair(window):
     np.testing.assert_allclose(conva, ra["conv"], rtol=0, atol=1e-12)
 
 
+def test_decode_resumes_from_a_state_snapshot():
+    """The decode state is the cache (meta block, ring, len), h and the conv state and
+    nothing else: decoding on from a copy of them gives the same outputs, bit for bit,
+    as decoding on from the originals."""
+    import copy
+    ca, cb, wa, wb = _pair(8, seed=41)
+    B, T, T0, T1 = 2, 24, 6, 13
+    x = synth.layer_input(ca, B, T, 43)
+    pa = oracle.mixer_prefill(ca, wa, x[:, :T0], residual=True)
+    pb = oracle.mixer_prefill(cb, wb, pa["y"], kv_shared=(pa["k"], pa["v"]), residual=True, x_has_meta=True)
+    cache = oracle.cache_from_prefill(ca, pa["k"], pa["v"], ca.n_meta + 8)
+    st = [pa["h"].copy(), pa["conv"].copy(), pb["h"].copy(), pb["conv"].copy()]
+
+    def run(cache, st, t0, t1):
+        out = []
+        for t in range(t0, t1):
+            ya = oracle.mixer_decode(ca, wa, x[:, t], cache, st[0], st[1], residual=True)
+            out.append(oracle.mixer_decode(cb, wb, ya, cache, st[2], st[3], residual=True))
+        return out
+
+    run(cache, st, T0, T1)
+    snap_cache, snap_st = copy.deepcopy(cache), [a.copy() for a in st]
+    first = run(cache, st, T1, T)
+    again = run(snap_cache, snap_st, T1, T)
+    for a, b in zip(first, again):
+        assert np.array_equal(a, b)
+    for a, b in zip(st, snap_st):
+        assert np.array_equal(a, b)
+
+
 def test_ring_slots_closed_form():
     """Meta positions keep slots 0..m-1; position p >= m goes to m + (p - m) mod R."""
     m, R = 3, 4

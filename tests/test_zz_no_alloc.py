@@ -13,7 +13,7 @@ import numpy as np
 import pytest
 
 import synth
-from gpu_helpers import BF16_MAX_ABS, BF16_REL_L2, errors, torch_cuda
+from gpu_helpers import BF16_MAX_ABS, BF16_REL_L2, errors, merge_split_partials, torch_cuda
 
 pytestmark = pytest.mark.gpu
 
@@ -46,18 +46,8 @@ def _decoded_layer(cfg, B, T0, cache_cap, seed):
     ns = lay["n_split"]
     n_part = B * H * ns * (dv + 2)
     part = ws[lay["part"]:lay["part"] + n_part * 4].view(torch.float32).view(B, H, ns, dv + 2)
-    o_ref = _merge_splits(part.double().cpu().numpy()).reshape(B, H * dv)
+    o_ref = merge_split_partials(part.double().cpu().numpy()).reshape(B, H * dv)
     return dict(layer=layer, kv=kv, q=q, ldp=ldp, o_ref=o_ref, mdt=mdt)
-
-
-def _merge_splits(part):
-    """Softmax over the union of the key splits from per-split partials [..., dv + 2]:
-    dv unnormalised sums of p v, then the split's max logit (base-2 domain) and its sum
-    of p. Each split is rescaled by 2^(m_s - max m) before the sums are divided."""
-    num, m, l = part[..., :-2], part[..., -2], part[..., -1]
-    M = m.max(axis=-1, keepdims=True)
-    w = np.where(np.isfinite(m), np.exp2(m - M), 0.0)
-    return (w[..., None] * num).sum(axis=-2) / (w * l).sum(axis=-1)[..., None]
 
 
 @pytest.mark.parametrize("kind", ["bf16_hymba15_ring", "f32_tiny_global"])
