@@ -50,13 +50,15 @@ def peaks():
 
 def kernel_traffic(name, workload):
     """DRAM bytes per launch of a kernel from the committed ncu record (profiles/), or
-    None when there is none for this workload or the kernel's source changed since."""
+    None when there is none for this workload or the kernel's device code changed since
+    (the record hashes the source file up to the kernel's host launcher)."""
     try:
         rec = json.load(open(os.path.join(ROOT, "profiles", "dram_traffic.json"))).get(name)
         if not rec or rec.get("workload") != workload:
             return None
         src = open(os.path.join(ROOT, rec["kernel_source"]), "rb").read()
-        if hashlib.sha1(src).hexdigest() != rec["kernel_source_sha1"]:
+        end = src.find(rec["device_code_until"].encode())
+        if end < 0 or hashlib.sha1(src[:end]).hexdigest() != rec["device_code_sha1"]:
             return None
         return rec["bytes_per_launch"]
     except (OSError, ValueError, KeyError):
