@@ -51,9 +51,15 @@ and Delta-large limits, a hand-worked single step, brute-force per-query softmax
 loops, window >= T equals full causal, meta visibility, GQA equals repeated KV,
 RoPE relative invariance, conv impulse response and causality, RMSNorm scale
 invariance, beta2 = 0, decode-by-decode equals prefill (across ring wrap), and the
-pages' printed cache sizes. The whole-layer composition of these steps (the order
-of the projection blocks, the fusion reading) has no page value to check against:
-parity for it is unpinned beyond the invariants above.
+pages' printed cache sizes, RMSNorm's epsilon inside the square root, and the
+decode-state byte count against the arrays a decode step actually carries.
+
+Parity unpinned (no page value can check it, and none of the pins above would
+notice a change of it): the order of the row blocks of the fused projection
+[Q | K | V | x | z | B | C | dt_low] is a layout reading, not arithmetic (B and C
+sit before dt_low so that their columns start on 16-byte boundaries); and the
+whole-layer composition of the pinned steps (the fusion reading) has no page value
+to check against beyond the invariants above.
 """
 from __future__ import annotations
 
@@ -141,17 +147,15 @@ def attention(q: np.ndarray, k: np.ndarray, v: np.ndarray, mask: np.ndarray) -> 
 # Mamba branch
 # ----------------------------------------------------------------------------
 
-def causal_conv(x: np.ndarray, w: np.ndarray, b: np.ndarray,
-                history: Optional[np.ndarray] = None) -> np.ndarray:
+def causal_conv(x: np.ndarray, w: np.ndarray, b: np.ndarray) -> np.ndarray:
     """Depthwise causal conv: out[t, c] = b[c] + sum_k w[c, k] * x[t - (K-1) + k, c].
 
-    x [L, C]; w [C, K]; inputs before t = 0 come from `history` [C, K] (its last
-    K-1 columns, oldest first) or are zero.
+    x [L, C]; w [C, K]; inputs before t = 0 are zero (the sequence starts at the
+    first meta row; a decode step carries its own conv state instead).
     """
     L, C = x.shape
     K = w.shape[1]
-    pad = np.zeros((K - 1, C)) if history is None else history[:, 1:].T.astype(np.float64)
-    xp = np.concatenate([pad, x], axis=0)
+    xp = np.concatenate([np.zeros((K - 1, C)), x], axis=0)
     out = np.tile(b.astype(np.float64), (L, 1))
     for k in range(K):
         out += w[:, k][None, :] * xp[k:k + L]
@@ -367,12 +371,12 @@ def ssm_state_bytes(n_layers: int, channels: int, d_state: int, batch: int, dtyp
 
 
 def layer_cache_bytes(cfg, batch: int, max_T: int) -> int:
-    """Decode cache of one producer layer: KV slots (meta + ring or full history) of
-    2-byte elements for a bf16 layer (4 for fp32), fp32 SSM state, fp32 conv state
-    and the int32 lengths."""
+    """Decode cache of one layer for sequences of up to max_T positions, meta rows
+    included: for a producer, KV slots (the meta slots + a ring of `window` slots, or
+    one slot per position for a global layer) of 2-byte elements for a bf16 layer (4
+    for fp32); then the fp32 SSM state, fp32 conv state and the int32 lengths."""
     esz = 2 if cfg.dtype == 1 else 4
-    span = cfg.window if cfg.window > 0 else max_T
-    cap = cfg.n_meta + span
+    cap = cfg.n_meta + cfg.window if cfg.window > 0 else max_T
     kv = batch * cfg.n_kv_heads * cap * (cfg.head_dim + cfg.v_head_dim) * esz if cfg.is_kv_producer else 0
     return (kv + ssm_state_bytes(1, cfg.d_inner, cfg.d_state, batch, 4)
             + batch * cfg.d_inner * cfg.d_conv * 4 + batch * 4)

@@ -173,4 +173,46 @@ def test_layer_cache_bytes_formula():
     conv = B * 3200 * 4 * 4
     assert oracle.layer_cache_bytes(cfg, B, 4096 + 128) == kv + h + conv + B * 4
     g = cfg.with_(window=0)
-    assert oracle.layer_cache_bytes(g, B, 5000) == B * 5 * (128 + 5000) * 192 * 2 + h + conv + B * 4
+    assert oracle.layer_cache_bytes(g, B, 5000) == B * 5 * 5000 * 192 * 2 + h + conv + B * 4
+
+
+def test_rmsnorm_epsilon_sits_inside_the_square_root():
+    """RMS(a) = gain * a / sqrt(mean(a^2) + eps): with mean(a^2) = 1 and eps = 3 the
+    divisor is sqrt(4) = 2 exactly, where eps outside the root would give 1 + 3 = 4
+    and eps dropped would give 1."""
+    a = np.array([[1.0, -1.0, 1.0, -1.0]])
+    got = oracle.rms_norm(a, np.ones(4), 3.0)
+    np.testing.assert_array_equal(got, a / 2.0)
+    # a second closed form: mean(a^2) = 12.5 for a = (3, 4) doubled over 4 columns;
+    # eps = 3.5 makes the divisor sqrt(16) = 4
+    b = np.array([[3.0, 4.0, -3.0, -4.0]])
+    np.testing.assert_array_equal(oracle.rms_norm(b, np.full(4, 2.0), 3.5), 2.0 * b / 4.0)
+
+
+@pytest.mark.parametrize("window,producer", [(8, 1), (0, 1), (8, 0)])
+def test_layer_cache_bytes_counts_the_decode_state_arrays(window, producer):
+    """The decode-state size equals the elements of the arrays that one decode step
+    reads and writes, counted from the arrays themselves: the cache a prefill leaves
+    (producer only; meta slots + ring, or the whole history for a global layer), the
+    SSM state h, the conv state and the lengths, at 2 bytes per K/V element for a
+    bf16 layer (4 for fp32) and 4 bytes for the fp32 states and int32 lengths."""
+    for dtype in (synth.F32, synth.BF16):
+        cfg = synth.tiny_layer_cfg().with_(window=window, is_kv_producer=producer, dtype=dtype)
+        B, T = 2, 21
+        w = synth.layer_weights(cfg, 61)
+        x = synth.layer_input(cfg, B, T, 61)
+        max_T = cfg.n_meta + T
+        kv_src = None
+        if not producer:
+            p = oracle.mixer_prefill(cfg.with_(is_kv_producer=1), synth.layer_weights(cfg.with_(is_kv_producer=1), 62), x)
+            kv_src = (p["k"], p["v"])
+        r = oracle.mixer_prefill(cfg, w, x, kv_shared=kv_src)
+        cap = cfg.n_meta + (window if window > 0 else T)
+        kv_elems = 0
+        if producer:
+            cache = oracle.cache_from_prefill(cfg, r["k"], r["v"], cap)
+            kv_elems = cache["k"].size + cache["v"].size
+            assert cache["len"].size == B
+        esz = 2 if dtype == synth.BF16 else 4
+        counted = kv_elems * esz + r["h"].size * 4 + r["conv"].size * 4 + B * 4
+        assert oracle.layer_cache_bytes(cfg, B, max_T) == counted
