@@ -23,26 +23,32 @@ namespace hymba {
 __device__ int g_status_word[8];
 
 static std::mutex g_mu;
-static int* g_status_ptr[64];
+// Per device: the status word's device address and the SM count, published together.
+// A reader that sees the pointer (acquire) also sees the SM count written before it
+// (release), so no caller can launch with a zero grid.
+static std::atomic<int*> g_status_ptr[64];
 static int g_sm_count[64];
 
 static int current_ctx(cudaStream_t stream, Ctx* ctx) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return HYMBA_ERR_CUDA;
-    if (!g_status_ptr[dev]) {
+    int* status = g_status_ptr[dev].load(std::memory_order_acquire);
+    if (!status) {
         std::lock_guard<std::mutex> lk(g_mu);
-        if (!g_status_ptr[dev]) {
+        status = g_status_ptr[dev].load(std::memory_order_relaxed);
+        if (!status) {
             void* p = nullptr;
             if (cudaGetSymbolAddress(&p, g_status_word) != cudaSuccess) return HYMBA_ERR_CUDA;
             int sms = 0;
-            if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+            if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0)
                 return HYMBA_ERR_CUDA;
             g_sm_count[dev] = sms;
-            g_status_ptr[dev] = static_cast<int*>(p);
+            status = static_cast<int*>(p);
+            g_status_ptr[dev].store(status, std::memory_order_release);
         }
     }
     ctx->stream = stream;
-    ctx->status = g_status_ptr[dev];
+    ctx->status = status;
     ctx->sm_count = g_sm_count[dev];
     ctx->device = dev;
     return HYMBA_OK;
@@ -559,10 +565,12 @@ uint64_t hymba_ssm_state_bytes(int n_layers, int channels, int d_state, int batc
 size_t hymba_cache_bytes(const hymba_layer_cfg* cfg, int B, int max_T) {
     if (check_cfg(cfg) || B <= 0 || max_T <= 0) return 0;
     const int esz = cfg->dtype == HYMBA_BF16 ? 2 : 4;
-    const int span = cfg->window > 0 ? cfg->window : max_T;
+    // slots: the meta block + a window-long ring, or one slot per position (meta
+    // included in max_T) for a global layer
+    const int slots = cfg->window > 0 ? cfg->n_meta + cfg->window : max_T;
     size_t kv = 0;
     if (cfg->is_kv_producer)
-        kv = hymba_kv_bytes(1, cfg->n_kv_heads, cfg->head_dim, cfg->v_head_dim, cfg->n_meta + span, B, esz);
+        kv = hymba_kv_bytes(1, cfg->n_kv_heads, cfg->head_dim, cfg->v_head_dim, slots, B, esz);
     return kv + hymba_ssm_state_bytes(1, cfg->d_inner, cfg->d_state, B, 4) +
            (size_t)B * cfg->d_inner * cfg->d_conv * 4 + (size_t)B * 4;
 }

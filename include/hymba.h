@@ -204,8 +204,8 @@ int hymba_kv_share(const hymba_kv* producer, const hymba_layer_cfg* consumer_cfg
 size_t hymba_workspace_bytes(const hymba_layer_cfg* cfg, int B, int T, int mode);
 
 /* Decode-state bytes of one layer for B sequences of up to max_T positions (meta
- * included): KV slots (producer only; n_meta + window, or n_meta + max_T when
- * global) * (head_dim + v_head_dim) * element size (2 for bf16 layers, whose K/V are
+ * included): KV slots (producer only; n_meta + window, or max_T when global)
+ * * (head_dim + v_head_dim) * element size (2 for bf16 layers, whose K/V are
  * fp16; 4 for fp32) * n_kv_heads * B, plus the fp32 SSM state, the fp32 conv state
  * and the int32 lengths. */
 size_t hymba_cache_bytes(const hymba_layer_cfg* cfg, int B, int max_T);
