@@ -35,6 +35,9 @@ Readings taken where the pages are silent:
   widths, so the V head dim is d_inner / n_q_heads.
 * One input projection yields [Q | K | V | x | z | B | C | dt_low] in that order.
   A consumer (KV-sharing secondary) layer has no K, V rows.
+* A consumer's affine adaptation of the shared K, V acts on the K that is shared
+  (after RoPE) and on V, per KV head and dimension, with its own scale and bias
+  for each; a consumer without those weights shares K and V unchanged.
 * RoPE is rotate-half with theta_i = base^(-2i/head_dim); meta tokens take
   positions 0..m-1 and user token t takes m + t; K is kept after RoPE.
 * Key j is visible to query i iff j <= i and (j < m or i - j < W); W <= 0 is
@@ -143,6 +146,25 @@ def attention(q: np.ndarray, k: np.ndarray, v: np.ndarray, mask: np.ndarray) -> 
     return out
 
 
+def adapt_shared_kv(k: np.ndarray, v: np.ndarray, w: Dict[str, np.ndarray], G: int, dh: int, dv: int):
+    """The secondary layer's head-specific affine adaptation of shared K and V
+    ([Hymba Guide] "Cross-Layer KV Cache Sharing", section 1: K~ = K * w_scale + b_bias,
+    elementwise, per KV head; V takes the same form with its own scale and bias).
+
+    k [G, L, dh], v [G, L, dv]; w["kv_scale"], w["kv_bias"] [G*dh + G*dv]: the G K
+    vectors (dh each) first, then the G V vectors (dv each). Without those weights the
+    layer shares K and V unchanged.
+    """
+    if w.get("kv_scale") is None:
+        return k, v
+    s = np.asarray(w["kv_scale"], dtype=np.float64)
+    b = np.asarray(w["kv_bias"], dtype=np.float64)
+    nk = G * dh
+    ks, kb = s[:nk].reshape(G, 1, dh), b[:nk].reshape(G, 1, dh)
+    vs, vb = s[nk:].reshape(G, 1, dv), b[nk:].reshape(G, 1, dv)
+    return k * ks + kb, v * vs + vb
+
+
 # ----------------------------------------------------------------------------
 # Mamba branch
 # ----------------------------------------------------------------------------
@@ -220,7 +242,7 @@ def split_projection(cfg, p: np.ndarray) -> Dict[str, np.ndarray]:
 
 
 def _f64(w: Dict[str, np.ndarray]) -> Dict[str, np.ndarray]:
-    return {k: np.asarray(v, dtype=np.float64) for k, v in w.items()}
+    return {k: (None if v is None else np.asarray(v, dtype=np.float64)) for k, v in w.items()}
 
 
 def mixer_prefill_row(cfg, w: Dict[str, np.ndarray], x: np.ndarray,
@@ -252,9 +274,11 @@ def mixer_prefill_row(cfg, w: Dict[str, np.ndarray], x: np.ndarray,
         v = blocks["v"].reshape(Tp, G, dv).transpose(1, 0, 2)
     else:
         k, v = (np.asarray(a, dtype=np.float64) for a in kv_shared)
+    # a secondary layer adapts the shared K, V ([Hymba Guide] Cross-Layer KV Cache Sharing)
+    ka, va = (k, v) if cfg.is_kv_producer else adapt_shared_kv(k, v, w, G, dh, dv)
     # attention heads: causal GQA over the meta prefix + window
     mask = visibility_mask(pos, pos, m, cfg.window)
-    o = attention(q, k, v, mask).transpose(1, 0, 2).reshape(Tp, H * dv)
+    o = attention(q, ka, va, mask).transpose(1, 0, 2).reshape(Tp, H * dv)
     # Mamba heads: conv, Delta, scan, gate
     xc = silu(causal_conv(blocks["x"], w["conv_w"], w["conv_b"]))
     delta = softplus(blocks["dtl"] @ w["w_dt"].T + w["b_dt"])
@@ -340,6 +364,8 @@ def mixer_decode(cfg, w, x_t: np.ndarray, cache: dict, h: np.ndarray, conv: np.n
         slots = [ring_slot(j, m, ring) for j in vis]
         kk = cache["k"][b][:, slots]
         vv = cache["v"][b][:, slots]
+        if not cfg.is_kv_producer:
+            kk, vv = adapt_shared_kv(kk, vv, w, G, dh, dv)
         o = attention(q, kk, vv, np.ones((1, len(vis)), dtype=bool)).transpose(1, 0, 2).reshape(1, H * dv)
         # Mamba step: shift the conv state, conv, Delta, one scan step
         conv[b] = np.concatenate([conv[b][:, 1:], blocks["x"].T], axis=1)

@@ -174,3 +174,15 @@ def perturbed_weights(w: Dict[str, np.ndarray], cfg: LayerCfg, seed: int,
 
 def workload(name: str) -> dict:
     return dict(WORKLOADS[name])
+
+
+def affine_kv(cfg: LayerCfg, seed: int, spread: float = 0.5) -> Dict[str, np.ndarray]:
+    """Weights of a secondary layer's affine adaptation of shared K and V, as two
+    [G*dh + G*dv] fp32 vectors (the G K vectors, then the G V vectors): scales
+    ~ Uniform[1 - spread, 1 + spread], biases ~ N(0, 0.1^2). The pages give no
+    initialisation; these keep every term of the transform visible in a test."""
+    G, dh, dv = cfg.n_kv_heads, cfg.head_dim, cfg.v_head_dim
+    g = _rng(seed, 11)
+    n = G * (dh + dv)
+    return {"kv_scale": g.uniform(1.0 - spread, 1.0 + spread, size=n).astype(np.float32),
+            "kv_bias": (g.standard_normal(n) * 0.1).astype(np.float32)}

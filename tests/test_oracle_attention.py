@@ -146,3 +146,81 @@ def test_rope_scores_depend_on_relative_position_only():
     x = g.standard_normal((5, dh))
     np.testing.assert_allclose(np.linalg.norm(oracle.rope(x, np.arange(5) * 11, 10000.0), axis=1),
                                np.linalg.norm(x, axis=1), rtol=1e-13)
+
+
+# ---------------------------------------------------------------------------
+# affine adaptation of shared K, V by a secondary layer ("Hymba Guide",
+# Cross-Layer KV Cache Sharing, section 1: K~ = K * w_scale + b_bias)
+# ---------------------------------------------------------------------------
+
+def _affine(G, dh, dv, ks, kb, vs, vb):
+    return {"kv_scale": np.concatenate([np.ravel(ks), np.ravel(vs)]),
+            "kv_bias": np.concatenate([np.ravel(kb), np.ravel(vb)])}
+
+
+def test_affine_kv_hand_worked_one_head():
+    """One query, two keys, dh = 4, dv = 2. Scale ln 3 on K's first dimension makes the
+    scores (ln 3, 0), so the weights are (3/4, 1/4); V scaled by (2, 1) and shifted by
+    (0, 5) gives rows (2, 5) and (0, 6), so the output is (1.5, 5.25)."""
+    q = np.array([[[2.0, 0.0, 0.0, 0.0]]])
+    k = np.array([[[1.0, 0.0, 0.0, 0.0], [0.0, 0.0, 0.0, 0.0]]])
+    v = np.array([[[1.0, 0.0], [0.0, 1.0]]])
+    w = _affine(1, 4, 2, [np.log(3.0), 1.0, 1.0, 1.0], np.zeros(4), [2.0, 1.0], [0.0, 5.0])
+    ka, va = oracle.adapt_shared_kv(k, v, w, 1, 4, 2)
+    o = oracle.attention(q, ka, va, np.ones((1, 2), dtype=bool))
+    np.testing.assert_allclose(o[0, 0], [1.5, 5.25], rtol=1e-14)
+
+
+def test_affine_kv_identity_is_plain_sharing():
+    """Scale 1 and bias 0 reproduce plain sharing bit for bit, and no weights at all
+    leave K and V untouched."""
+    g = np.random.default_rng(81)
+    G, dh, dv = 2, 64, 128
+    k, v = g.standard_normal((G, 9, dh)), g.standard_normal((G, 9, dv))
+    w = _affine(G, dh, dv, np.ones(G * dh), np.zeros(G * dh), np.ones(G * dv), np.zeros(G * dv))
+    ka, va = oracle.adapt_shared_kv(k, v, w, G, dh, dv)
+    assert np.array_equal(ka, k) and np.array_equal(va, v)
+    kb, vb = oracle.adapt_shared_kv(k, v, {}, G, dh, dv)
+    assert kb is k and vb is v
+
+
+def test_affine_kv_per_head_layout():
+    """kv_scale / kv_bias hold the G K vectors first, then the G V vectors. With KV head
+    1's K scale 0 its queries see equal scores (a plain mean of its adapted V rows),
+    while KV head 0 keeps its softmax; V head 1 is shifted by its own bias only."""
+    g = np.random.default_rng(82)
+    G, H, dh, dv, L = 2, 4, 8, 6, 5
+    q = g.standard_normal((H, 1, dh))
+    k = g.standard_normal((G, L, dh))
+    v = g.standard_normal((G, L, dv))
+    vb1 = g.standard_normal(dv)
+    w = _affine(G, dh, dv, np.concatenate([np.ones(dh), np.zeros(dh)]), np.zeros(G * dh),
+                np.ones(G * dv), np.concatenate([np.zeros(dv), vb1]))
+    ka, va = oracle.adapt_shared_kv(k, v, w, G, dh, dv)
+    o = oracle.attention(q, ka, va, np.ones((1, L), dtype=bool))
+    for h in range(2):  # group 0: plain attention
+        s = q[h, 0] @ k[0].T / np.sqrt(dh)
+        p = np.exp(s - s.max())
+        np.testing.assert_allclose(o[h, 0], (p / p.sum()) @ v[0], rtol=1e-12)
+    for h in range(2, 4):  # group 1: uniform weights over V + its bias
+        np.testing.assert_allclose(o[h, 0], v[1].mean(axis=0) + vb1, rtol=1e-12)
+
+
+def test_affine_kv_key_bias_cancels_and_value_affine_commutes():
+    """Two identities of softmax attention that a kernel may rely on: a key bias adds
+    q . b to every score of a query (softmax is shift invariant, so it drops out), and
+    since the weights sum to 1, attention over V * s + b equals (attention over V) * s + b."""
+    g = np.random.default_rng(83)
+    G, H, dh, dv, L = 1, 3, 16, 8, 11
+    q = g.standard_normal((H, L, dh))
+    k = g.standard_normal((G, L, dh))
+    v = g.standard_normal((G, L, dv))
+    mask = oracle.visibility_mask(np.arange(L), np.arange(L), 2, 4)
+    ks, vs, vb = 1.0 + 0.3 * g.standard_normal(dh), 1.0 + 0.3 * g.standard_normal(dv), g.standard_normal(dv)
+    w_nob = _affine(G, dh, dv, ks, np.zeros(dh), vs, np.zeros(dv))
+    w_bias = _affine(G, dh, dv, ks, 5.0 * g.standard_normal(dh), vs, vb)
+    a0 = oracle.attention(q, *oracle.adapt_shared_kv(k, v, w_nob, G, dh, dv), mask)
+    a1 = oracle.attention(q, *oracle.adapt_shared_kv(k, v, w_bias, G, dh, dv), mask)
+    np.testing.assert_allclose(a1, a0 + vb, rtol=1e-10, atol=1e-12)
+    plain = oracle.attention(q * ks, k, v, mask)  # the key scale moved onto the query
+    np.testing.assert_allclose(a0, plain * vs, rtol=1e-10, atol=1e-12)

@@ -216,3 +216,29 @@ def test_layer_cache_bytes_counts_the_decode_state_arrays(window, producer):
         esz = 2 if dtype == synth.BF16 else 4
         counted = kv_elems * esz + r["h"].size * 4 + r["conv"].size * 4 + B * 4
         assert oracle.layer_cache_bytes(cfg, B, max_T) == counted
+
+
+@pytest.mark.parametrize("window", [8, 0])
+def test_decode_equals_prefill_with_affine_shared_kv(window):
+    """A consumer that adapts the shared K, V ("Hymba Guide", Cross-Layer KV Cache
+    Sharing) decodes as it prefills: the adaptation acts on the cached K, V the same way
+    in both paths (the ring of 8 slots wraps several times)."""
+    ca, cb, wa, wb = _pair(window, seed=71)
+    wb = dict(wb, **synth.affine_kv(cb, 71))
+    B, T, T0 = 2, 26, 9
+    m = ca.n_meta
+    x = synth.layer_input(ca, B, T, 72)
+    ra = oracle.mixer_prefill(ca, wa, x, residual=True)
+    rb = oracle.mixer_prefill(cb, wb, ra["y"], kv_shared=(ra["k"], ra["v"]), residual=True, x_has_meta=True)
+    plain = oracle.mixer_prefill(cb, _pair(window, seed=71)[3], ra["y"], kv_shared=(ra["k"], ra["v"]),
+                                 residual=True, x_has_meta=True)
+    assert np.abs(rb["y"] - plain["y"]).max() > 1e-3  # the adaptation changes the output
+    pa = oracle.mixer_prefill(ca, wa, x[:, :T0], residual=True)
+    pb = oracle.mixer_prefill(cb, wb, pa["y"], kv_shared=(pa["k"], pa["v"]), residual=True, x_has_meta=True)
+    cap = m + (window if window > 0 else T)
+    cache = oracle.cache_from_prefill(ca, pa["k"], pa["v"], cap)
+    ha, conva, hb, convb = pa["h"].copy(), pa["conv"].copy(), pb["h"].copy(), pb["conv"].copy()
+    for t in range(T0, T):
+        ya = oracle.mixer_decode(ca, wa, x[:, t], cache, ha, conva, residual=True)
+        yb = oracle.mixer_decode(cb, wb, ya, cache, hb, convb, residual=True)
+        np.testing.assert_allclose(yb, rb["y"][:, m + t], rtol=1e-10, atol=1e-10)
