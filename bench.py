@@ -1,11 +1,16 @@
 """Benchmark of the B200 Hymba hybrid-head mixer.
 
-One step = one hymba_mixer_prefill of the Hymba-1.5B-shaped SWA layer (B=1, T=2048
-user tokens + 128 meta tokens, window 1024, bf16): the fused projection with RoPE
-and K/V write, Delta projection, meta+window GQA attention, conv + selective scan,
-fusion epilogue and output projection. The decode step of the KV-sharing layer pair
-(B=64, 1024-slot ring + 128 meta, fp32 state [64, 3200, 16]) is timed the same way
-and reported under "decode".
+Headline step: one prefill of the 32-layer mixer stack (Hymba-1.5B layer shape,
+d_model 1600, B=8 sequences of T=4096 user tokens + 128 meta tokens, layers 0, 15
+and 31 global, the others sliding-window 1024, consecutive layer pairs sharing KV,
+fp32 residual stream between the bf16 layers). Every layer runs the fused
+projection with RoPE and K/V write, the Delta projection, meta+window GQA attention,
+conv + selective scan, the fusion epilogue and the output projection with the
+residual add.
+
+Beside it, under extra keys: the global layer (B=4, T=8192 + 128 meta), the SWA
+layer (B=1, T=2048 + 128 meta) and the decode step of the KV-sharing layer pair
+(B=64, 1024-slot ring + 128 meta, fp32 state [64, 3200, 16]).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
@@ -32,7 +37,8 @@ sys.path.insert(0, ROOT)
 
 import synth  # noqa: E402
 
-WORKLOAD = "hymba15_swa1024_b1_t2048"
+WORKLOAD = "hymba15_stack32_b8_t4096"
+LAYER_WORKLOADS = ("hymba15_global_b4_t8192", "hymba15_swa1024_b1_t2048")
 DECODE_WORKLOAD = "hymba15_decode_pair_b64_p4096"
 
 
@@ -65,12 +71,18 @@ def kernel_traffic(name, workload):
         return None
 
 
-def roofline_entry(name, bound, units, avg_s, pk, sm_count, sm_mhz):
-    """Achieved rate of one kernel against the peak of its bound."""
+def roofline_entry(name, bound, units, avg_s, pk, sm_count, sm_mhz, long_step=False):
+    """Achieved rate of one kernel against the peak of its bound. A tensor-bound kernel
+    is set against the burst bf16 peak when its launches are timed in a short step, and
+    against the sustained one inside a long step (where the power cap sets the clock);
+    both fractions are given."""
     if bound == "tensor":
         ach = units / avg_s / 1e12
-        return {"kernel": name, "bound": "tensor", "achieved": ach, "peak": pk["bf16_sus"], "unit": "TFLOP/s",
-                "frac": ach / pk["bf16_sus"], "peak_kind": f"bf16 dense, sustained, {pk['src']}"}
+        peak = pk["bf16_sus"] if long_step else pk["bf16"]
+        kind = "sustained" if long_step else "burst"
+        return {"kernel": name, "bound": "tensor", "achieved": ach, "peak": peak, "unit": "TFLOP/s",
+                "frac": ach / peak, "frac_burst": ach / pk["bf16"], "frac_sustained": ach / pk["bf16_sus"],
+                "peak_kind": f"bf16 dense, {kind}, {pk['src']}"}
     if bound == "alu":
         ach = units / avg_s / 1e9
         peak = MUFU_PER_CLK_SM * sm_count * sm_mhz * 1e-3
@@ -182,6 +194,8 @@ class Clocks:
                 "reasons": reasons, "samples": len(inside), "source": source}
 
 
+
+
 def visible_pairs(Tp, m, W):
     i = np.arange(Tp)[:, None]
     j = np.arange(Tp)[None, :]
@@ -189,27 +203,40 @@ def visible_pairs(Tp, m, W):
     return int(vis.sum())
 
 
-def prefill_work(cfg, B, T):
-    """Algorithmic FLOPs / bytes per launch of each prefill kernel."""
+def layer_work(cfg, B, T, has_meta, io_f32):
+    """Algorithmic work of each kernel launch of one prefill call, as {name: (bound,
+    units)}: FLOPs for the projections and attention, MUFU results for the scan, bytes
+    for the HBM-bound kernels."""
     m, Tp = cfg.n_meta, cfg.n_meta + T
-    H, G, dh, dv, di, d, r = (cfg.n_q_heads, cfg.n_kv_heads, cfg.head_dim, cfg.v_head_dim,
-                              cfg.d_inner, cfg.d_model, cfg.dt_rank)
+    H, dh, dv, di, d, r = (cfg.n_q_heads, cfg.head_dim, cfg.v_head_dim, cfg.d_inner, cfg.d_model, cfg.dt_rank)
     rows = B * Tp
+    # the in-projection computes the user rows and the meta rows once (or every row
+    # when the input already carries the meta rows)
+    in_rows = rows if has_meta else B * T + m
     pairs = visible_pairs(Tp, m, cfg.window)
-    return {
-        "gemm_in_proj": ("tensor", 2.0 * B * T * cfg.n_in * d),
-        "gemm_in_proj_meta": ("tensor", 2.0 * m * cfg.n_in * d),
+    w = {
+        "gemm_in_proj": ("tensor", 2.0 * in_rows * cfg.n_in * d),
         "gemm_dt_proj": ("tensor", 2.0 * rows * di * r),
         "attn_prefill": ("tensor", 2.0 * B * pairs * H * (dh + dv)),
-        "attn_prefill_simt": ("tensor", 2.0 * B * pairs * H * (dh + dv)),
-        # MUFU operations: 16 state decays exp2(Delta A), and exp2 + reciprocal of the SiLU,
-        # per (row, channel); the kernel's binding limit (its 56 MB of HBM traffic take
-        # 8.5 us at the measured copy rate, the MUFU work 27 us)
+        # MUFU results: 16 state decays exp2(Delta A), and exp2 + reciprocal of the SiLU,
+        # per (row, channel): the scan's binding limit
         "conv_scan_prefill": ("alu", rows * di * 18.0),
         # O, y_pre, z read, U written: 2 B each per (row, channel)
         "fuse": ("hbm", rows * di * 8.0),
         "gemm_out_proj": ("tensor", 2.0 * rows * d * di),
     }
+    if io_f32 and cfg.dtype == synth.BF16:
+        # fp16 copies of the stream rows (fp32 read, fp16 written) and of W_in, W_out
+        # and the meta rows (bf16 read, fp16 written)
+        xrows = rows if has_meta else B * T
+        w["pad_copy"] = ("hbm", xrows * d * 6.0 + (cfg.n_in * d + d * di + (0 if has_meta else m * d)) * 4.0)
+    return w
+
+
+def add_work(total, part):
+    for n, (bound, u) in part.items():
+        total[n] = (bound, total.get(n, (bound, 0.0))[1] + u)
+    return total
 
 
 def decode_work(cfg, B, cap):
@@ -248,123 +275,170 @@ def cpu_cores():
         return os.cpu_count() or 1
 
 
-def oracle_sample(T_sample: int):
-    """Time the CPU oracle on the first T_sample tokens of the workload's sequence."""
-    import oracle
-    wl = synth.workload(WORKLOAD)
+def workload_config(name):
+    wl = synth.workload(name)
     cfg = wl["cfg"]
-    w = synth.layer_weights(cfg, wl["seed"])
-    x = synth.layer_input(cfg, wl["B"], wl["T"], wl["seed"])[:, :T_sample]
+    c = {"workload": name, "B": wl["B"], "T": wl["T"], "n_meta": cfg.n_meta, "d_model": cfg.d_model,
+         "d_inner": cfg.d_inner, "n_q_heads": cfg.n_q_heads, "n_kv_heads": cfg.n_kv_heads,
+         "window": cfg.window, "per_rank_batch": wl["B"]}
+    if wl["kind"] == "stack":
+        c["n_layers"] = wl["n_layers"]
+        c["global_layers"] = list(wl["global_layers"])
+        c["kv_sharing"] = "consecutive layer pairs (2i producer, 2i+1 consumer)"
+        c["residual_stream"] = "fp32"
+    return c
+
+
+# ---------------------------------------------------------------------------
+# the CPU oracle as a baseline
+# ---------------------------------------------------------------------------
+ORACLE_T = 512  # user tokens of the oracle's sample sequence
+
+
+def _stack_cfgs_weights(layers):
+    wl = synth.workload(WORKLOAD)
+    cfgs = synth.stack_layer_cfgs(wl["cfg"], wl["n_layers"], wl["global_layers"])
+    return wl, cfgs, {l: synth.layer_weights(cfgs[l], 1000 * wl["seed"] + l) for l in layers}
+
+
+def _oracle_layers(cfgs, weights, layers, x, has_meta):
+    import oracle
+    h, kv = x, None
+    for i, l in enumerate(layers):
+        c = cfgs[l]
+        r = oracle.mixer_prefill(c, weights[l], h, kv_shared=None if c.is_kv_producer else kv, residual=True,
+                                 x_has_meta=has_meta or i > 0)
+        if c.is_kv_producer:
+            kv = (r["k"], r["v"])
+        h = r["y"]
+    return h
+
+
+def oracle_stack_sample():
+    """The oracle through all 32 layers of the stack on the first ORACLE_T user tokens of
+    sequence 0 (weights drawn before the clock starts). Returns (tokens/s, seconds)."""
+    wl, cfgs, weights = _stack_cfgs_weights(range(wl_layers()))
+    x = synth.layer_input(cfgs[0], 1, wl["T"], wl["seed"])[:, :ORACLE_T]
     t0 = time.perf_counter()
-    oracle.mixer_prefill(cfg, w, x)
+    _oracle_layers(cfgs, weights, list(range(len(cfgs))), x, False)
     dt = time.perf_counter() - t0
-    return x.shape[0] * x.shape[1] / dt, dt
+    return ORACLE_T / dt, dt
+
+
+def wl_layers():
+    return synth.workload(WORKLOAD)["n_layers"]
 
 
 def run_reference(args, rank):
+    """The oracle as the reference arm: each step runs one KV-sharing layer pair of the
+    stack (pairs taken in turn) on one sequence of ORACLE_T user tokens + 128 meta rows;
+    tokens/s of the whole stack = ORACLE_T / (pair time x 16)."""
     if rank != 0:
         return
-    T_sample = 512
-    vals = []
+    n_layers = wl_layers()
+    wl, cfgs, weights = _stack_cfgs_weights(range(n_layers))
+    x = synth.layer_input(cfgs[0], 1, wl["T"], wl["seed"])[:, :ORACLE_T]
+    g = np.random.default_rng([wl["seed"], 91])
+    xm = (g.standard_normal((1, cfgs[0].n_meta + ORACLE_T, cfgs[0].d_model)) * 2.0).astype(np.float32)
+    times = []
     for i in range(args.warmup + args.steps):
-        v, _ = oracle_sample(T_sample)
+        pair = (i % (n_layers // 2)) * 2
+        t0 = time.perf_counter()
+        _oracle_layers(cfgs, weights, [pair, pair + 1], x if pair == 0 else xm, pair > 0)
         if i >= args.warmup:
-            vals.append(v)
-    v = statistics.median(vals)
-    wl = synth.workload(WORKLOAD)
-    sample = f"first {T_sample} of {wl['T']} user tokens of the B=1 sequence (+128 meta rows)"
+            times.append(time.perf_counter() - t0)
+    pair_s = statistics.mean(times)
+    step_s = pair_s * n_layers / 2
+    v = ORACLE_T / step_s
+    sample = (f"one sequence of {ORACLE_T} user tokens + 128 meta rows through one KV-sharing layer pair per "
+              f"step (the 16 pairs in turn), scaled to the 32-layer stack")
     print(json.dumps({
-        "impl": "reference", "metric": "hybrid-head mixer prefill tokens/s", "value": v,
+        "impl": "reference", "metric": "hybrid-head mixer stack prefill tokens/s", "value": v,
         "unit": "tokens/s", "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": 1e3 * T_sample / v, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "f64", "data": "synthetic",
-        "config": {"workload": WORKLOAD, "B": wl["B"], "T": wl["T"], "n_meta": 128, "window": 1024},
+        "ms_per_step": 1e3 * step_s, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f64", "data": "synthetic", "config": workload_config(WORKLOAD),
         "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": cpu_cores(), "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }))
 
 
-def main():
-    ap = argparse.ArgumentParser()
-    ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
-    ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--clocks-dir", default="",
-                    help="where the NVML clock samples are written (default: the system temp directory)")
-    ap.add_argument("--no-decode", action="store_true")
-    args = ap.parse_args()
-    args.warmup = max(args.warmup, 3)
+# ---------------------------------------------------------------------------
+# device workloads
+# ---------------------------------------------------------------------------
+class PrefillWorkload:
+    """A prefill workload on the device: one layer (bf16 input and output) or the
+    32-layer stack (fp32 residual stream, KV shared by layer pairs, in place after the
+    first layer). step(x, y) queues one pass over all its layers on the current stream."""
 
-    rank = int(os.environ.get("RANK", "0"))
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    if args.impl == "reference":
-        return run_reference(args, rank)
+    def __init__(self, name, rank, torch, hy, rt):
+        import ctypes
+        self.name, self.torch, self.hy, self.rt = name, torch, hy, rt
+        wl = synth.workload(name)
+        self.wl = wl
+        self.B, self.T = wl["B"], wl["T"]
+        base = wl["cfg"]
+        self.Tp = base.n_meta + self.T
+        self.stack = wl["kind"] == "stack"
+        if self.stack:
+            self.cfgs = synth.stack_layer_cfgs(base, wl["n_layers"], wl["global_layers"])
+            seeds = [1000 * wl["seed"] + l for l in range(len(self.cfgs))]
+        else:
+            self.cfgs, seeds = [base], [wl["seed"]]
+        self.layers = [rt.DeviceLayer(c, synth.layer_weights(c, s)) for c, s in zip(self.cfgs, seeds)]
+        io_f32 = self.stack
+        x_np = synth.layer_input(base, self.B, self.T, rank_inputs_seed(wl["seed"], rank))
+        self.x = rt.to_device(x_np, base, io_f32=io_f32)
+        del x_np
+        self.y = torch.empty((self.B, self.Tp, base.d_model), dtype=self.x.dtype, device="cuda")
+        self.kv = rt.KV(base.with_(is_kv_producer=1), self.B, seq_cap=self.Tp)
+        self.kvs = []
+        for c, lay in zip(self.cfgs, self.layers):
+            if c.is_kv_producer:
+                self.kvs.append(self.kv.s)
+            else:
+                s = hy.hymba_kv()
+                hy.check(hy.hymba_kv_share(ctypes.byref(self.kv.s), ctypes.byref(lay.c), ctypes.byref(s)))
+                self.kvs.append(s)
+        self.ws = rt.workspace(base.with_(is_kv_producer=1), self.B, self.T, hy.HYMBA_MODE_PREFILL)
+        self.flags = rt.stream_flags(base) if self.stack else 0
+        self.work = {}
+        for i, c in enumerate(self.cfgs):
+            add_work(self.work, layer_work(c, self.B, self.T, has_meta=i > 0, io_f32=io_f32))
+        self.tokens = self.B * self.T
 
-    import ctypes
-    import torch
-    import torch.distributed as dist
-    import hybrid_head_ssm_b200 as hy
-    from hybrid_head_ssm_b200 import runtime as rt
+    def step(self, xin=None, yout=None):
+        x = self.x if xin is None else xin
+        y = self.y if yout is None else yout
+        for i, (lay, kvs) in enumerate(zip(self.layers, self.kvs)):
+            fl = self.flags | (self.hy.HYMBA_X_HAS_META if i > 0 else 0)
+            self.rt.prefill(lay, x if i == 0 else y, self.T, None, y, self.ws, None, fl, kv_struct_override=kvs)
 
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    torch.cuda.set_device(local)
-    if world > 1:
-        import datetime
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
 
-    def barrier():
-        if world > 1:
-            dist.barrier()
-
-    def max_ranks(v):
-        return max_over_ranks(v, world, "cuda")
-
-    pk = peaks()
-    wl = synth.workload(WORKLOAD)
-    cfg, B, T = wl["cfg"], wl["B"], wl["T"]
-    Tp = cfg.n_meta + T
-    w = synth.layer_weights(cfg, wl["seed"])
-    x_np = synth.layer_input(cfg, B, T, rank_inputs_seed(wl["seed"], rank))
-    layer = rt.DeviceLayer(cfg, w)
-    x = rt.to_device(x_np, cfg)
-    y = torch.empty((B, Tp, cfg.d_model), dtype=torch.bfloat16, device="cuda")
-    kv = rt.KV(cfg, B, seq_cap=Tp)
-    ws = rt.workspace(cfg, B, T, hy.HYMBA_MODE_PREFILL)
-    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")  # > 126 MB L2
+def time_prefill(wk, args, torch, hy, barrier, max_ranks, pk, flush, clocks, sm_count, headline):
+    """Warm-up, a traced pass for the per-kernel breakdown, the timed steps (only the
+    dominant kernel bracketed by events) and the end-to-end run with host buffers."""
     stream = torch.cuda.current_stream()
-
-    def step(xin=None, yout=None):
-        rt.prefill(layer, x if xin is None else xin, T, kv, y if yout is None else yout, ws, None, 0)
-
-    clocks = Clocks(local, args.clocks_dir)
-    clocks.start()
     for _ in range(args.warmup):
-        step()
+        wk.step()
     torch.cuda.synchronize()
 
-    work = prefill_work(cfg, B, T)
-
     def run_steps(n, traced_only=None, timed=False):
-        """n steps, L2 flushed before each (outside the step events); returns the step
-        times (ms) and the trace records."""
         if traced_only is not False:
             hy.hymba_trace_enable(1)
             hy.check(hy.hymba_trace_only(traced_only.encode() if traced_only else None))
         ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
         barrier()
         torch.cuda.synchronize()
-        if timed:
+        if timed and clocks:
             clocks.begin()
         for i in range(n):
             flush.fill_(i & 0xFF)
             ev[i][0].record(stream)
-            step()
+            wk.step()
             ev[i][1].record(stream)
         torch.cuda.synchronize()
-        if timed:
+        if timed and clocks:
             clocks.end()
         barrier()
         trace = hy.trace_collect() if traced_only is not False else []
@@ -372,47 +446,56 @@ def main():
         hy.check(hy.hymba_trace_only(None))
         return [a.elapsed_time(b) for a, b in ev], trace
 
-    # ---- per-kernel breakdown (every launch bracketed by events; outside the timed region,
-    # since events between launches serialise the overlap of consecutive kernels)
-    _, trace_all = run_steps(args.steps, traced_only=None)
+    # per-kernel breakdown: every launch bracketed by events, outside the timed region
+    # (events between launches serialise the overlap of consecutive kernels)
+    n_traced = max(1, min(args.steps, 8192 // (12 * len(wk.layers))))
+    _, trace_all = run_steps(n_traced, traced_only=None)
     per = {}
     for name, t in trace_all:
         per.setdefault(name, []).append(t)
     tot_k = max(sum(map(sum, per.values())), 1e-9)
-    kern = {n: {"launches": len(v), "avg_us": 1e3 * sum(v) / len(v), "share": sum(v) / tot_k} for n, v in per.items()}
+    kern = {n: {"launches_per_step": len(v) / n_traced, "us_per_step": 1e3 * sum(v) / n_traced,
+                "share": sum(v) / tot_k} for n, v in per.items()}
     dom = max(per, key=lambda n: sum(per[n]))
 
-    # ---- timed region: K steps; only the dominant kernel is bracketed by events
+    # timed region: K steps, only the dominant kernel's launches bracketed by events
     launches0 = hy.hymba_launch_count()
-    step_ms, trace_dom = run_steps(args.steps, traced_only=dom, timed=True)
-    launches = hy.hymba_launch_count() - launches0
-    clk = clocks.stop()
+    step_ms, trace_dom = run_steps(args.steps, traced_only=dom, timed=headline)
+    launches = (hy.hymba_launch_count() - launches0) / args.steps
     ms = max_ranks(sum(step_ms) / len(step_ms))
-    tokens = B * T * world
-    value = tokens / (ms * 1e-3)
-
-    sm_count = torch.cuda.get_device_properties(local).multi_processor_count
-    sm_mhz = clk["sm_mhz"] if clk else pk["sm_mhz"]
+    long_step = ms > 20.0
+    sm_mhz = pk["sm_mhz"]
+    if headline and clocks:
+        clk = clocks.stop()
+        if clk:
+            sm_mhz = clk["sm_mhz"]
+    else:
+        clk = None
     dom_t = [t for n, t in trace_dom if n == dom]
-    bound, units = work.get(dom, ("hbm", 0.0))
-    roof = roofline_entry(dom, bound, units, sum(dom_t) / len(dom_t) * 1e-3, pk, sm_count, sm_mhz)
-    roof["launches_timed"] = len(dom_t)
-    roof["traffic"] = kernel_traffic(dom, WORKLOAD)
+    bound, units = wk.work.get(dom, ("hbm", 0.0))
+    dom_s_per_step = sum(dom_t) / args.steps * 1e-3
+    roof = roofline_entry(dom, bound, units, dom_s_per_step, pk, sm_count, sm_mhz, long_step)
+    roof["launches_per_step"] = len(dom_t) / args.steps
+    roof["units_per_step"] = units
+    roof["traffic"] = kernel_traffic(dom, wk.name)
     if roof["traffic"] is not None:
         roof["traffic_unit"] = "bytes per launch (ncu dram__bytes_read.sum + dram__bytes_write.sum)"
-    for n, (bd, u) in work.items():
+    for n, (bd, u) in wk.work.items():
         if n in per:
-            r = roofline_entry(n, bd, u, sum(per[n]) / len(per[n]) * 1e-3, pk, sm_count, sm_mhz)
-            kern[n]["achieved"], kern[n]["unit"], kern[n]["frac"] = r["achieved"], r["unit"], r["frac"]
+            r = roofline_entry(n, bd, u, sum(per[n]) / n_traced * 1e-3, pk, sm_count, sm_mhz, long_step)
+            kern[n].update({k: r[k] for k in ("achieved", "unit", "frac", "peak_kind")})
+            for k in ("frac_burst", "frac_sustained"):
+                if k in r:
+                    kern[n][k] = r[k]
 
-    # ---- end to end through the public API with host buffers: each step uploads its
-    # input from pinned host memory, runs the layer and downloads the output; uploads,
+    # end to end through the public API with host buffers: each step uploads its input
+    # from pinned host memory, runs the workload and downloads the output; uploads,
     # compute and downloads go on three streams with two device buffer sets, so step
     # i+1's upload and step i-1's download overlap step i's compute. Timed with device
     # events from the first upload to the last download.
-    x_host = x.cpu().pin_memory()
-    y_host = [torch.empty(y.shape, dtype=y.dtype).pin_memory() for _ in range(2)]
-    xs, ys = [x, torch.empty_like(x)], [y, torch.empty_like(y)]
+    x_host = wk.x.cpu().pin_memory()
+    y_host = [torch.empty(wk.y.shape, dtype=wk.y.dtype).pin_memory() for _ in range(2)]
+    xs, ys = [wk.x, torch.empty_like(wk.x)], [wk.y, torch.empty_like(wk.y)]
     up, down = torch.cuda.Stream(), torch.cuda.Stream()
 
     def e2e_run(n):
@@ -434,7 +517,7 @@ def main():
             stream.wait_event(uploaded[k])
             if used[k]:
                 stream.wait_event(downloaded[k])  # ys[k] of step i-2 is on the host
-            step(xs[k], ys[k])
+            wk.step(xs[k], ys[k])
             computed[k].record(stream)
             with torch.cuda.stream(down):
                 down.wait_event(computed[k])
@@ -446,46 +529,17 @@ def main():
         torch.cuda.synchronize()
         return t_start.elapsed_time(t_end) / n
 
-    e2e_run(args.warmup)
-    e2e_ms_step = max_ranks(e2e_run(args.steps))
-
-    # ---- decode step of the KV-sharing pair (B=64, ring 1024 + 128 meta)
-    dec = None
-    if not args.no_decode:
-        dec = bench_decode(args, torch, hy, rt, max_ranks, barrier, world, pk, flush)
-
-    out = None
-    if rank == 0:
-        cpu = None
-        if world == 1 and not args.no_cpu_baseline:
-            v, dt = oracle_sample(T)
-            cpu = {"value": v, "unit": "tokens/s", "cores": cpu_cores(), "kind": "oracle",
-                   "sample": f"one full sequence of the workload (B=1, T={T} + 128 meta), {dt:.1f} s"}
-        out = {
-            "metric": "hybrid-head mixer prefill tokens/s", "value": value, "unit": "tokens/s",
-            "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-            "data": "synthetic",
-            "config": {"workload": WORKLOAD, "B": B, "T": T, "n_meta": cfg.n_meta, "window": cfg.window,
-                       "d_model": cfg.d_model, "d_inner": cfg.d_inner, "per_rank_batch": B,
-                       "l2": "flushed between steps (256 MB write outside the step events)"},
-            "roofline": roof,
-            "cpu_baseline": cpu,
-            "e2e": {"value": tokens / (e2e_ms_step * 1e-3), "unit": "tokens/s",
-                    "h2d_bytes_per_step": x.numel() * x.element_size(),
-                    "d2h_bytes_per_step": y.numel() * y.element_size()},
-            "gpu_launches": int(launches),
-            "clocks": clk,
-            "kernels": kern,
-            "decode": dec,
-        }
-        print(json.dumps(out))
-    if world > 1:
-        dist.destroy_process_group()
-    return out
+    e2e_run(min(args.warmup, 3))
+    e2e_ms = max_ranks(e2e_run(args.steps))
+    del xs, ys, x_host, y_host
+    return dict(ms=ms, launches=launches, roof=roof, kern=kern, clk=clk, e2e_ms=e2e_ms,
+                h2d=wk.x.numel() * wk.x.element_size(), d2h=wk.y.numel() * wk.y.element_size())
 
 
-def bench_decode(args, torch, hy, rt, max_over_ranks, barrier, world, pk, flush):
+def bench_decode(args, torch, hy, rt, max_ranks, barrier, world, pk, flush):
+    """The decode step of the KV-sharing pair: timed without any tracing, then a traced
+    pass for the per-kernel figures."""
+    import ctypes
     wl = synth.workload(DECODE_WORKLOAD)
     ca = wl["cfg"]
     cb = ca.with_(is_kv_producer=0)
@@ -494,7 +548,6 @@ def bench_decode(args, torch, hy, rt, max_over_ranks, barrier, world, pk, flush)
     lb = rt.DeviceLayer(cb, synth.layer_weights(cb, seed * 1000 + 1))
     cap = ca.n_meta + ca.window
     Tp = ca.n_meta + T
-    import ctypes
     kv = rt.KV(ca, B, seq_cap=Tp, cache_cap=cap)
     kvb = hy.hymba_kv()
     hy.check(hy.hymba_kv_share(ctypes.byref(kv.s), ctypes.byref(lb.c), ctypes.byref(kvb)))
@@ -511,7 +564,6 @@ def bench_decode(args, torch, hy, rt, max_over_ranks, barrier, world, pk, flush)
     ha, hb = torch.empty_like(xt), torch.empty_like(xt)
     wda = rt.workspace(ca, B, cap, hy.HYMBA_MODE_DECODE)
     wdb = rt.workspace(cb, B, cap, hy.HYMBA_MODE_DECODE)
-    len0 = kv.len.clone()
     stream = torch.cuda.current_stream()
 
     def step():
@@ -521,7 +573,6 @@ def bench_decode(args, torch, hy, rt, max_over_ranks, barrier, world, pk, flush)
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
-    hy.hymba_trace_enable(1)
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
     barrier()
     torch.cuda.synchronize()
@@ -532,9 +583,14 @@ def bench_decode(args, torch, hy, rt, max_over_ranks, barrier, world, pk, flush)
         ev[i][1].record(stream)
     torch.cuda.synchronize()
     barrier()
+    ms = max_ranks(sum(a.elapsed_time(b) for a, b in ev) / args.steps)
+    # per-kernel figures from a separate traced pass
+    hy.hymba_trace_enable(1)
+    for i in range(args.steps):
+        flush.fill_(i & 0xFF)
+        step()
     trace = hy.trace_collect()
     hy.hymba_trace_enable(0)
-    ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in ev) / args.steps)
     per = {}
     for name, t in trace:
         per.setdefault(name, []).append(t)
@@ -551,10 +607,101 @@ def bench_decode(args, torch, hy, rt, max_over_ranks, barrier, world, pk, flush)
     step_bytes = (2 * decode_work(ca, B, cap)["attn_decode"][1]
                   + (ca.n_in + cb.n_in) * ca.d_model * 2.0 + 2 * ca.d_model * ca.d_inner * 2.0
                   + 2 * decode_work(ca, B, cap)["ssm_decode"][1])
-    assert kv.len[0].item() >= len0[0].item()
     return {"workload": DECODE_WORKLOAD, "tokens_per_s": B * world / (ms * 1e-3), "ms_per_step": ms,
             "step_bytes": step_bytes, "step_gbs": step_bytes / (ms * 1e-3) / 1e9,
-            "step_frac_hbm": step_bytes / (ms * 1e-3) / 1e9 / pk["hbm"], "kernels": kern}
+            "step_frac_hbm": step_bytes / (ms * 1e-3) / 1e9 / pk["hbm"],
+            "timing": "timed steps untraced; per-kernel figures from a separate traced pass", "kernels": kern}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--clocks-dir", default="",
+                    help="where the NVML clock samples are written (default: the system temp directory)")
+    ap.add_argument("--no-extra", action="store_true", help="time only the headline workload")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if args.impl == "reference":
+        return run_reference(args, rank)
+
+    import torch
+    import torch.distributed as dist
+    import hybrid_head_ssm_b200 as hy
+    from hybrid_head_ssm_b200 import runtime as rt
+
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_ranks(v):
+        return max_over_ranks(v, world, "cuda")
+
+    pk = peaks()
+    sm_count = torch.cuda.get_device_properties(local).multi_processor_count
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")  # > 126 MB L2
+
+    clocks = Clocks(local, args.clocks_dir)
+    clocks.start()
+    wk = PrefillWorkload(WORKLOAD, rank, torch, hy, rt)
+    head = time_prefill(wk, args, torch, hy, barrier, max_ranks, pk, flush, clocks, sm_count, headline=True)
+    del wk
+    torch.cuda.empty_cache()
+    tokens = synth.workload(WORKLOAD)["B"] * synth.workload(WORKLOAD)["T"] * world
+
+    extra = {}
+    if not args.no_extra:
+        for name in LAYER_WORKLOADS:
+            w2 = PrefillWorkload(name, rank, torch, hy, rt)
+            r = time_prefill(w2, args, torch, hy, barrier, max_ranks, pk, flush, None, sm_count, headline=False)
+            extra[name] = {"tokens_per_s": w2.tokens * world / (r["ms"] * 1e-3), "ms_per_step": r["ms"],
+                           "e2e_tokens_per_s": w2.tokens * world / (r["e2e_ms"] * 1e-3), "roofline": r["roof"],
+                           "kernels": r["kern"], "gpu_launches_per_step": r["launches"]}
+            del w2
+            torch.cuda.empty_cache()
+        extra[DECODE_WORKLOAD] = bench_decode(args, torch, hy, rt, max_ranks, barrier, world, pk, flush)
+
+    out = None
+    if rank == 0:
+        cpu = None
+        if world == 1 and not args.no_cpu_baseline:
+            v, dt = oracle_stack_sample()
+            cpu = {"value": v, "unit": "tokens/s", "cores": cpu_cores(), "kind": "oracle",
+                   "sample": f"sequence 0, first {ORACLE_T} user tokens + 128 meta rows through all "
+                             f"{wl_layers()} layers, {dt:.1f} s"}
+        out = {
+            "metric": "hybrid-head mixer stack prefill tokens/s", "value": tokens / (head["ms"] * 1e-3),
+            "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": head["ms"], "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16", "data": "synthetic",
+            "config": dict(workload_config(WORKLOAD),
+                           l2="inputs larger than L2 (weights 1.3 GB, stream 216 MB); 256 MB written between steps"),
+            "roofline": head["roof"],
+            "cpu_baseline": cpu,
+            "e2e": {"value": tokens / (head["e2e_ms"] * 1e-3), "unit": "tokens/s",
+                    "h2d_bytes_per_step": head["h2d"], "d2h_bytes_per_step": head["d2h"]},
+            "gpu_launches": int(round(head["launches"] * args.steps)),
+            "gpu_launches_per_step": head["launches"],
+            "clocks": head["clk"],
+            "kernels": head["kern"],
+            "extra": extra,
+        }
+        print(json.dumps(out))
+    if world > 1:
+        dist.destroy_process_group()
+    return out
 
 
 if __name__ == "__main__":

@@ -54,7 +54,8 @@ class hymba_layer_cfg(ctypes.Structure):
 
 class hymba_layer_weights(ctypes.Structure):
     _fields_ = [(n, _vp) for n in ("w_in", "w_dt", "b_dt", "conv_w", "conv_b", "A_log", "D",
-                                   "norm_attn_w", "norm_ssm_w", "beta1", "beta2", "w_out", "meta")]
+                                   "norm_attn_w", "norm_ssm_w", "beta1", "beta2", "w_out", "meta",
+                                   "kv_scale", "kv_bias")]
 
 
 class hymba_kv(ctypes.Structure):

@@ -19,13 +19,14 @@ constexpr int MAX_CHUNK = 256;  // keys per split
 constexpr float LOG2E = 1.4426950408889634f;
 
 // Visible key list of the query at position p: meta positions [0, min(n_meta, p+1)),
-// then positions [lo, p]. Returns false when the ring cannot hold the span.
+// then the n_win positions [lo, p] (none while p is inside the meta block). Returns
+// false when the ring cannot hold the span.
 __device__ __forceinline__ bool decode_span(int p, int n_meta, int window, int ring, int* meta_n,
-                                            int* lo) {
+                                            int* lo, int* n_win) {
     *meta_n = min(n_meta, p + 1);
     *lo = window > 0 ? max(n_meta, p - window + 1) : n_meta;
-    const int span = p + 1 - *lo;
-    return p >= 0 && span <= ring;
+    *n_win = max(0, p + 1 - *lo);
+    return p >= 0 && *n_win <= ring;
 }
 
 // 8 consecutive elements of a K or V row as fp32 (one or two 16-byte loads).
@@ -76,10 +77,10 @@ attn_decode_kernel(const T* __restrict__ P, long long ldP, const T* __restrict__
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int p = len[b] + pos_offset;
     const int ring = cap - n_meta;
-    int meta_n, lo;
-    const bool ok = decode_span(p, n_meta, window, ring, &meta_n, &lo);
+    int meta_n, lo, n_win;
+    const bool ok = decode_span(p, n_meta, window, ring, &meta_n, &lo, &n_win);
     if (!ok && s == 0 && g == 0 && tid == 0) set_status(status, HYMBA_ERR_DEVICE_RANGE);
-    const int L = ok ? meta_n + (p + 1 - lo) : 0;
+    const int L = ok ? meta_n + n_win : 0;
     const int chunk = (L + n_split - 1) / n_split;
     const int k0 = min(L, s * chunk), k1 = min(L, k0 + chunk);
     const int nk = k1 - k0;
@@ -275,10 +276,10 @@ attn_decode_bulk_kernel(const f16* __restrict__ P, long long ldP, const f16* __r
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int p = len[b] + pos_offset;
     const int ring = cap - n_meta;
-    int meta_n, lo;
-    const bool span_ok = decode_span(p, n_meta, window, ring, &meta_n, &lo);
+    int meta_n, lo, n_win;
+    const bool span_ok = decode_span(p, n_meta, window, ring, &meta_n, &lo, &n_win);
     if (!span_ok && s == 0 && g == 0 && tid == 0) set_status(status, HYMBA_ERR_DEVICE_RANGE);
-    const int L = span_ok ? meta_n + (p + 1 - lo) : 0;
+    const int L = span_ok ? meta_n + n_win : 0;
     const int chunk = (L + n_split - 1) / n_split;
     const int k0 = min(L, s * chunk), k1 = min(L, k0 + chunk);
     const int nk = k1 - k0;

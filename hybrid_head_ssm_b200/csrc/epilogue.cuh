@@ -36,6 +36,8 @@ struct EpiArgs {
     int pos_offset;        // decode: 0 for a producer (appends), -1 for a consumer
     int n_meta_ring;       // decode: ring length (cache_cap - n_meta)
     float rope_base;       // decode: angles computed on the fly
+    const float* q_scale;  // consumer with an adapted shared K: [G, dh] scales applied to the
+                           // queries of each KV head's group after RoPE (NULL: none)
     // EPI_DELTA
     float* delta;          // [M, N] fp32
     const float* b_dt;
@@ -188,6 +190,18 @@ __device__ __forceinline__ RunDst epi_prepare64(const EpiArgs<T>& e, int r, int 
             }
         } else {
             rope_run64(v, e.rope + (long long)t * 32);
+        }
+        if (e.q_scale && c0 < qw) {
+            // q . (k * s) = (q * s) . k: the K scale of the query's KV head moves onto q
+            const float4* s4 = reinterpret_cast<const float4*>(e.q_scale + (c0 / e.dh) / (e.H / e.G) * e.dh);
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+                const float4 f = s4[j];
+                v[4 * j] *= f.x;
+                v[4 * j + 1] *= f.y;
+                v[4 * j + 2] *= f.z;
+                v[4 * j + 3] *= f.w;
+            }
         }
     }
     d.count = b1 - b0;

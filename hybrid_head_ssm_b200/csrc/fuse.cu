@@ -97,7 +97,8 @@ __global__ void __launch_bounds__(TPR * RPB, SPLIT ? 1 : 4)
 fuse_kernel(const I* __restrict__ O, const float* __restrict__ part, int n_split, int H,
             const I* __restrict__ ypre, const I* __restrict__ P, long long ldP, int col_z,
             const float* __restrict__ g_attn, const float* __restrict__ g_ssm, const float* __restrict__ beta1,
-            const float* __restrict__ beta2, T* __restrict__ U, int rows, int di, float eps, int* len_inc) {
+            const float* __restrict__ beta2, const float* __restrict__ v_scale, const float* __restrict__ v_bias,
+            int rep, T* __restrict__ U, int rows, int di, float eps, int* len_inc) {
     griddep_sync();
     __shared__ float red[RPB][TPR / 32][2];
     const int sub = threadIdx.x / TPR, t = threadIdx.x % TPR;
@@ -116,6 +117,17 @@ fuse_kernel(const I* __restrict__ O, const float* __restrict__ part, int n_split
                 merge8(part, n_split, H, di / H, row, c, o[k]);
             else
                 load8<I>(O + row * di + c, o[k]);
+            if (v_scale) {
+                // a consumer's adapted shared V: attention over V * s + b is the attention
+                // output * s + b (the softmax weights sum to 1)
+                const int dv = di / H, hd = c / dv;
+                const int idx = (hd / rep) * dv + (c - hd * dv);
+                float vs[8], vb[8];
+                load8f(v_scale + idx, vs);
+                load8f(v_bias + idx, vb);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) o[k][i] = fmaf(o[k][i], vs[i], vb[i]);
+            }
             load8<I>(ypre + row * di + c, y[k]);
             load8<I>(P + row * ldP + col_z + c, z);
 #pragma unroll
@@ -166,34 +178,38 @@ fuse_kernel(const I* __restrict__ O, const float* __restrict__ part, int n_split
 }  // namespace
 
 template <typename I, typename T>
-int launch_fuse(const Ctx& ctx, const I* O, const float* part, int n_split, int H, const I* ypre, const I* P,
-                long long ldP, int col_z, const float* g_attn, const float* g_ssm, const float* beta1,
-                const float* beta2, T* U, int rows, int di, float eps, int* len_inc) {
+int launch_fuse(const Ctx& ctx, const I* O, const float* part, int n_split, int H, int G, const I* ypre,
+                const I* P, long long ldP, int col_z, const float* g_attn, const float* g_ssm, const float* beta1,
+                const float* beta2, const float* v_scale, const float* v_bias, T* U, int rows, int di, float eps,
+                int* len_inc) {
     if (rows <= 0) return HYMBA_OK;
     if (di % 8 || di > VMAX * 8 * TPR || col_z % 8 || ldP % 8) return HYMBA_ERR_UNSUPPORTED;
+    // pieces of 8 never straddle a head
+    if (H <= 0 || G <= 0 || H % G || di % H || (di / H) % 8) return HYMBA_ERR_UNSUPPORTED;
+    if ((v_scale == nullptr) != (v_bias == nullptr) ||
+        ((reinterpret_cast<uintptr_t>(v_scale) | reinterpret_cast<uintptr_t>(v_bias)) & 15))
+        return HYMBA_ERR_UNSUPPORTED;
     if (part) {
-        // pieces of 8 never straddle a head; 8-byte loads of the partial sums
-        if (H <= 0 || n_split <= 0 || di % H || (di / H) % 8 || (reinterpret_cast<uintptr_t>(part) & 7))
-            return HYMBA_ERR_UNSUPPORTED;
+        // 8-byte loads of the partial sums
+        if (n_split <= 0 || (reinterpret_cast<uintptr_t>(part) & 7)) return HYMBA_ERR_UNSUPPORTED;
         auto kern = fuse_kernel<I, T, true>;
         HYMBA_LAUNCH(ctx, "fuse", kern, ceil_div(rows, RPB), TPR * RPB, 0, O, part, n_split, H, ypre, P, ldP,
-                     col_z, g_attn, g_ssm, beta1, beta2, U, rows, di, eps, len_inc);
+                     col_z, g_attn, g_ssm, beta1, beta2, v_scale, v_bias, H / G, U, rows, di, eps, len_inc);
         return HYMBA_OK;
     }
     auto kern = fuse_kernel<I, T, false>;
     HYMBA_LAUNCH(ctx, "fuse", kern, ceil_div(rows, RPB), TPR * RPB, 0, O, part, n_split, H, ypre, P, ldP, col_z,
-                 g_attn, g_ssm, beta1, beta2, U, rows, di, eps, len_inc);
+                 g_attn, g_ssm, beta1, beta2, v_scale, v_bias, H / G, U, rows, di, eps, len_inc);
     return HYMBA_OK;
 }
 
-template int launch_fuse<float, float>(const Ctx&, const float*, const float*, int, int, const float*,
-                                       const float*, long long, int, const float*, const float*, const float*,
-                                       const float*, float*, int, int, float, int*);
-template int launch_fuse<f16, bf16>(const Ctx&, const f16*, const float*, int, int, const f16*, const f16*,
-                                    long long, int, const float*, const float*, const float*, const float*,
-                                    bf16*, int, int, float, int*);
-template int launch_fuse<f16, f16>(const Ctx&, const f16*, const float*, int, int, const f16*, const f16*,
-                                   long long, int, const float*, const float*, const float*, const float*,
-                                   f16*, int, int, float, int*);
+
+#define HYMBA_FUSE_INST(I, T)                                                                              \
+    template int launch_fuse<I, T>(const Ctx&, const I*, const float*, int, int, int, const I*, const I*, long long, \
+                                   int, const float*, const float*, const float*, const float*, const float*,       \
+                                   const float*, T*, int, int, float, int*);
+HYMBA_FUSE_INST(float, float)
+HYMBA_FUSE_INST(f16, bf16)
+HYMBA_FUSE_INST(f16, f16)
 
 }  // namespace hymba

@@ -236,6 +236,14 @@ static EpiArgs<T> epi_base(int kind, int M, int N) {
     return e;
 }
 
+// The V half of a consumer's affine adaptation of the shared K/V (NULL: plain sharing).
+static const float* vscale(const hymba_layer_cfg* c, const hymba_layer_weights* w) {
+    return (!c->is_kv_producer && w->kv_scale) ? w->kv_scale + c->n_kv_heads * c->head_dim : nullptr;
+}
+static const float* vbias(const hymba_layer_cfg* c, const hymba_layer_weights* w) {
+    return (!c->is_kv_producer && w->kv_bias) ? w->kv_bias + c->n_kv_heads * c->head_dim : nullptr;
+}
+
 // T: the layer's I/O and weight type (fp32 or bf16). I: its intermediate type
 // (fp32, or fp16 for bf16 layers: the projection, K/V, attention output and y_pre are
 // held in fp16, which has the same width as bf16 and a finer mantissa).
@@ -300,6 +308,7 @@ static int prefill_impl(const Ctx& ctx, const hymba_layer_cfg* c, const hymba_la
     ep.kcap = kv->seq_cap;
     ep.H = H; ep.G = G; ep.dh = dh; ep.dv = dv;
     ep.rope = rope;
+    ep.q_scale = c->is_kv_producer ? nullptr : w->kv_scale;
     if (has_meta) {
         ep.row_mode = ROWS_DIRECT; ep.M = (int)rows;
         if ((rc = gemm<TA, I>(ctx, "gemm_in_proj", x, d, W_in, d, (int)rows, k.n_in, d, ep))) return rc;
@@ -339,8 +348,9 @@ static int prefill_impl(const Ctx& ctx, const hymba_layer_cfg* c, const hymba_la
                                           st ? st->conv : nullptr, B, Tp, di)))
         return rc;
     // 5. gate, norms, beta, average --------------------------------------------------
-    if ((rc = launch_fuse<I, TA>(ctx, O, nullptr, 0, 0, ypre, P, pl.ldP, k.z, w->norm_attn_w, w->norm_ssm_w, w->beta1,
-                                 w->beta2, U, (int)rows, di, c->rms_eps, nullptr)))
+    if ((rc = launch_fuse<I, TA>(ctx, O, nullptr, 0, H, G, ypre, P, pl.ldP, k.z, w->norm_attn_w, w->norm_ssm_w,
+                                 w->beta1, w->beta2, vscale(c, w), vbias(c, w), U, (int)rows, di, c->rms_eps,
+                                 nullptr)))
         return rc;
     // 6. output projection (+ residual) -------------------------------------------------
     EpiArgs<TIO> eo = epi_base<TIO>(EPI_OUT, (int)rows, d);
@@ -388,6 +398,7 @@ static int decode_impl(const Ctx& ctx, const hymba_layer_cfg* c, const hymba_lay
     ep.pos = kv->len; ep.pos_offset = pos_offset;
     ep.n_meta_ring = kv->cache_cap - m;
     ep.rope_base = c->rope_base;
+    ep.q_scale = c->is_kv_producer ? nullptr : w->kv_scale;
     // RoPE table of the new positions and, for a fp32 residual stream, the new rows in
     // the layer's type: one launch
     float2* rope = reinterpret_cast<float2*>(ws + pl.rope);
@@ -413,9 +424,9 @@ static int decode_impl(const Ctx& ctx, const hymba_layer_cfg* c, const hymba_lay
                                       w->b_dt, c->dt_rank, w->conv_w, w->conv_b, w->A_log, w->D, st->h,
                                       st->conv, ypre, B, di)))
         return rc;
-    if ((rc = launch_fuse<I, T>(ctx, nullptr, part, pl.n_split, H, ypre, P, pl.ldP, k.z, w->norm_attn_w,
-                                w->norm_ssm_w, w->beta1, w->beta2, U, B, di, c->rms_eps,
-                                c->is_kv_producer ? kv->len : nullptr)))
+    if ((rc = launch_fuse<I, T>(ctx, nullptr, part, pl.n_split, H, G, ypre, P, pl.ldP, k.z, w->norm_attn_w,
+                                w->norm_ssm_w, w->beta1, w->beta2, vscale(c, w), vbias(c, w), U, B, di,
+                                c->rms_eps, c->is_kv_producer ? kv->len : nullptr)))
         return rc;
     EpiArgs<TIO> eo = epi_base<TIO>(EPI_OUT, B, d);
     eo.y = y;
@@ -429,6 +440,11 @@ static int check_weights(const hymba_layer_cfg* c, const hymba_layer_weights* w)
         !w->norm_attn_w || !w->norm_ssm_w || !w->beta1 || !w->beta2 || !w->w_out)
         return HYMBA_ERR_INVALID_ARG;
     if (c->n_meta > 0 && !w->meta) return HYMBA_ERR_INVALID_ARG;
+    // the affine adaptation of shared K/V: consumers only, both vectors or neither,
+    // 16-byte aligned (read as float4)
+    if ((w->kv_scale == nullptr) != (w->kv_bias == nullptr)) return HYMBA_ERR_INVALID_ARG;
+    if (w->kv_scale && c->is_kv_producer) return HYMBA_ERR_INVALID_ARG;
+    if (((uintptr_t)w->kv_scale | (uintptr_t)w->kv_bias) & 15) return HYMBA_ERR_INVALID_ARG;
     return HYMBA_OK;
 }
 

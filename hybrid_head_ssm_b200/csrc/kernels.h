@@ -43,11 +43,13 @@ int launch_conv_scan_prefill(const Ctx& ctx, const T* P, long long ldP, int col_
 // RMSNorm of both branches, SiLU(z) gate, beta scaling and average; one row per block.
 // The attention branch is O [rows, di], or, when `part` is given, the decode
 // attention's split partials [rows, H, n_split, di/H + 2] merged on the fly (O unused).
+// A consumer's adapted shared V (v_scale, v_bias [G, dv], both or neither) is applied
+// to the attention output before its norm.
 template <typename I, typename T>
-int launch_fuse(const Ctx& ctx, const I* O, const float* part, int n_split, int H, const I* ypre,
+int launch_fuse(const Ctx& ctx, const I* O, const float* part, int n_split, int H, int G, const I* ypre,
                 const I* P, long long ldP, int col_z, const float* g_attn, const float* g_ssm,
-                const float* beta1, const float* beta2, T* U, int rows, int di, float eps,
-                int* len_inc);
+                const float* beta1, const float* beta2, const float* v_scale, const float* v_bias, T* U,
+                int rows, int di, float eps, int* len_inc);
 
 
 // The RoPE table and the zero-padded 16-bit copy of W_dt [rows, cols] -> [rows, ld_dst],

@@ -17,7 +17,8 @@ from . import (HYMBA_BF16, HYMBA_MODE_DECODE, HYMBA_MODE_PREFILL, check, cfg_str
 
 BIG = ("w_in", "w_dt", "w_out", "meta")
 NAMES = ("w_in", "w_dt", "b_dt", "conv_w", "conv_b", "A_log", "D", "norm_attn_w", "norm_ssm_w",
-         "beta1", "beta2", "w_out", "meta")
+         "beta1", "beta2", "w_out", "meta", "kv_scale", "kv_bias")
+OPTIONAL = ("kv_scale", "kv_bias")  # a consumer's affine adaptation of the shared K/V
 
 
 def act_dtype(cfg):
@@ -38,6 +39,9 @@ class DeviceLayer:
         adt = act_dtype(cfg)
         self.t = {}
         for n in NAMES:
+            a = w.get(n)
+            if a is None and n in OPTIONAL:
+                continue
             a = w[n]
             dt = adt if n in BIG else torch.float32
             self.t[n] = torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).to(device=device, dtype=dt)

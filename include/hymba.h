@@ -122,6 +122,18 @@ typedef struct hymba_layer_weights {
     const float* beta2;       /* [d_inner] */
     const void*  w_out;       /* [d_model, d_inner]     dtype */
     const void*  meta;        /* [n_meta, d_model]      dtype */
+    /* Consumer layers only (NULL for a producer, and NULL for plain sharing): the
+     * head-specific affine adaptation of the shared K and V ("Hymba Guide",
+     * Cross-Layer KV Cache Sharing, section 1: K~ = K * w_scale + b_bias, and V~ the
+     * same with its own scale and bias), elementwise per KV head on the K held in the
+     * cache (after RoPE). Both [n_kv_heads*head_dim + n_kv_heads*v_head_dim] fp32: the
+     * K vectors of the KV heads, then their V vectors. Both or neither. No K/V copy is
+     * made: the K scale is applied to the queries instead (q . (k * s) = (q * s) . k),
+     * the K bias adds the same q . b to every score of a query and so leaves the softmax
+     * unchanged, and the V transform is applied to the attention output (its weights
+     * sum to 1). */
+    const float* kv_scale;
+    const float* kv_bias;
 } hymba_layer_weights;
 
 /* K/V of one producer layer and of the consumers that share it ("Hymba Guide",

@@ -204,3 +204,31 @@ def test_hymba15_decode_pair_b64_sampled_rows():
         mx, rl = assert_close(ya[b:b + 1], ra, ca, f"producer row {b}")
         mx2, rl2 = assert_close(yb[b:b + 1], rb, cb, f"consumer row {b}")
         print(f"decode pair row {b}: A {mx:.3e}/{rl:.3e}, B {mx2:.3e}/{rl2:.3e}")
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_pair_decode_with_affine_shared_kv(dtype):
+    """Decode through a pair whose consumer adapts the shared K/V: the query scale and
+    the V transform act in the decode path as in the oracle's literal adaptation of the
+    cached K, V (window 8 / 24 rings that wrap)."""
+    if dtype == "f32":
+        base = synth.tiny_layer_cfg().with_(window=8)
+        B, T0, steps, seed = 2, 10, 12, 81
+    else:
+        base = synth.hymba15_layer_cfg(window=24).with_(d_model=256, n_q_heads=5, n_kv_heads=1, d_inner=640,
+                                                        dt_rank=24, n_meta=8)
+        B, T0, steps, seed = 3, 30, 12, 82
+    ca, cb = base, base.with_(is_kv_producer=0)
+    wa = synth.layer_weights(ca, seed)
+    wb = dict(synth.perturbed_weights(synth.layer_weights(cb, seed + 1), cb, seed + 1), **synth.affine_kv(cb, seed))
+    x = synth.layer_input(ca, B, T0 + steps, seed + 2)
+    cap = ca.n_meta + ca.window
+    g = _Pair(ca, cb, wa, wb, B, T0, cap)
+    g.prefill(x[:, :T0])
+    o = _oracle_pair(ca, cb, wa, wb, x[:, :T0], cap)
+    for t in range(T0, T0 + steps):
+        ya, yb = g.step(x[:, t])
+        ra = oracle.mixer_decode(ca, wa, x[:, t], o["cache"], o["ha"], o["ca"], residual=True)
+        rb = oracle.mixer_decode(cb, wb, ra, o["cache"], o["hb"], o["cb"], residual=True)
+        assert_close(to_np(yb), rb, cb, f"consumer step {t}")
+    assert g.hy.hymba_get_device_status(None) == 0

@@ -202,3 +202,41 @@ def test_prefill_fills_decode_ring_bit_exact():
         s = oracle.ring_slot(p, cfg.n_meta, 8)
         assert torch.equal(kc[:, :, s], ks[:, :, p]) and torch.equal(vc[:, :, s], vs[:, :, p]), p
     assert kv.len.cpu().tolist() == [Tp, Tp]
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_consumer_with_affine_shared_kv(dtype):
+    """A consumer that adapts the shared K and V ("Hymba Guide", Cross-Layer KV Cache
+    Sharing: K~ = K * w_scale + b_bias per KV head, V likewise) reads the GPU producer's
+    K/V; its output and attention stage match the oracle's literal adaptation."""
+    if dtype == "f32":
+        base = synth.tiny_layer_cfg().with_(window=24)
+        B, T = 2, 90
+    else:
+        base = synth.hymba15_layer_cfg(window=40).with_(d_model=256, n_q_heads=5, n_kv_heads=1, d_inner=640,
+                                                        dt_rank=24, n_meta=8)
+        B, T = 2, 133
+    cp, cc = base, base.with_(is_kv_producer=0)
+    wp = synth.layer_weights(cp, 41)
+    wc = dict(synth.perturbed_weights(synth.layer_weights(cc, 42), cc, 42), **synth.affine_kv(cc, 43))
+    x = synth.layer_input(cp, B, T, 44)
+    refp = oracle.mixer_prefill(cp, wp, x)
+    refc = oracle.mixer_prefill(cc, wc, x, kv_shared=(refp["k"], refp["v"]))
+    rp = _run_prefill(cp, wp, x)
+    rc = _run_prefill(cc, wc, x, kv_from=rp["kv"])
+    mx, rl = assert_close(to_np(rc["y"]), refc["y"], cc, "consumer y with adapted K/V")
+    print(f"affine shared KV consumer ({dtype}): max abs {mx:.3e}, rel L2 {rl:.3e}")
+    import torch
+    from hybrid_head_ssm_b200 import runtime as rt
+    lay = rc["lay"]
+    o = to_np(_ws_view(rc["ws"], lay["O"], (B, cc.n_meta + T, cc.n_q_heads * cc.v_head_dim), rt.mid_dtype(cc)))
+    # the workspace holds the attention before the V adaptation (applied in the fusion)
+    nk, rep = cc.n_kv_heads * cc.head_dim, cc.n_q_heads // cc.n_kv_heads
+    vs = np.repeat(wc["kv_scale"][nk:].reshape(cc.n_kv_heads, cc.v_head_dim), rep, axis=0).ravel()
+    vb = np.repeat(wc["kv_bias"][nk:].reshape(cc.n_kv_heads, cc.v_head_dim), rep, axis=0).ravel()
+    o_ref = (refc["o_attn"] - vb) / vs  # per query head h, the V adaptation of its KV head
+    assert_close(o, o_ref, cc, "attention output (before the V adaptation)",
+                 max_abs=1e-4 if cc.dtype == 0 else 2e-2)
+    with pytest.raises(Exception):
+        # a producer may not carry the adaptation
+        _run_prefill(cp, dict(wp, **synth.affine_kv(cp, 45)), x)

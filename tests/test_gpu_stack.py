@@ -2,18 +2,26 @@
 global, consecutive pairs sharing KV, fp32 residual stream between the bf16 layers),
 run at full size through the C ABI.
 
-The stack's own arithmetic sets how far any bf16 implementation can stay from the
-fp64 oracle end to end: the oracle run twice, once on an input perturbed by 1e-6
-(relative), ends 1.6e-4 apart in relative L2 and 7e-3 in max abs after 32 layers
-(about 1.17x growth per layer). A bf16 tensor-core layer rounds its operands at the
-1e-3 level, so the 32-layer output cannot meet the per-output bound end to end.
-Parity at the contract's tolerance is therefore checked per KV-sharing pair, at the
-stack's full size, on seeded inputs with the activation scale of that depth; the
-end-to-end run is checked for a sane, bounded deviation and reported.
+The oracle runs the whole stack once on sequence 0 over a prefix of its positions
+(outputs at a position depend only on earlier positions, so the GPU's full-size
+outputs there are exact samples of the full computation). That run gives the stack's
+own residual stream entering every layer.
 
-The oracle recomputes sequence 0 over a prefix of the positions: outputs at a
-position depend only on earlier positions, so the GPU's full-size outputs there are
-exact samples of the full computation."""
+* Every KV-sharing pair (2k, 2k+1), all 16 of them, is checked at the contract's
+  tolerance: the GPU runs the pair at full size with sequence 0's prefix rows set to
+  the oracle's stream at depth 2k (the other rows are Gaussian with that stream's rms;
+  pair 0 takes the workload's own input), and its outputs on the prefix rows are
+  compared with the oracle's stream at depths 2k+1 and 2k+2.
+* The end-to-end run (all 32 layers on the workload input) cannot meet the per-output
+  bound: the stack amplifies any deviation (measured below from the oracle alone, by
+  running it again on an input perturbed by 1e-3 relative, which is the size of one
+  bf16 operand rounding). Its bound is derived from that amplification and the
+  per-layer errors measured on the pairs: a deviation e_l introduced at layer l reaches
+  the output multiplied by a(L) / a(l), where a(l) is the oracle's own growth of a
+  perturbation from the input to depth l; so the end-to-end relative L2 must stay
+  within sum_l e_l * a(L) / a(l) (with a factor 2 for the direction of the
+  perturbation, which a single probe does not fix).
+"""
 import ctypes
 
 import numpy as np
@@ -21,37 +29,67 @@ import pytest
 
 import oracle
 import synth
-from gpu_helpers import assert_close, errors, to_np, torch_cuda
+from gpu_helpers import BF16_MAX_ABS, BF16_REL_L2, errors, to_np, torch_cuda
 
 pytestmark = pytest.mark.gpu
 
 WL = "hymba15_stack32_b8_t4096"
 T_PREFIX = 1536  # 1664 rows: past the 1024 window, so the sliding window is exercised
-# rms of the residual stream entering layer 0, 14, 30 of the stack (fp64 oracle)
-DEPTH_RMS = {0: 1.0, 14: 2.84, 30: 4.01}
+PERTURB = 1e-3
 
 
 def _layer_weights(wl, l, cfg):
     return synth.layer_weights(cfg, 1000 * wl["seed"] + l)
 
 
-def run_layers_gpu(wl, cfgs, first, h_np, has_meta):
-    """Run layers first, first+1, ... of cfgs in place on h (fp32 stream); returns the
-    output after every layer."""
+def _oracle_stack(wl, cfgs, weights, x_row, ref=None):
+    """The oracle's stream entering every layer and after the last: [L + 1] arrays of
+    [n_meta + T_PREFIX, d_model] (entry 0 is the user input with the meta rows); or,
+    given ref (such a list), the relative L2 distance from it at every depth."""
+    h = x_row[None]
+    kv = None
+    s0 = np.concatenate([weights[0]["meta"].astype(np.float64), x_row.astype(np.float64)], axis=0)
+    out = [s0 if ref is None else errors(s0, ref[0])[1]]
+    for l, cfg in enumerate(cfgs):
+        r = oracle.mixer_prefill(cfg, weights[l], h, kv_shared=None if cfg.is_kv_producer else kv, residual=True,
+                                 x_has_meta=l > 0)
+        if cfg.is_kv_producer:
+            kv = (r["k"], r["v"])
+        h = r["y"]
+        out.append(h[0].copy() if ref is None else errors(h[0], ref[l + 1])[1])
+    return out
+
+
+@pytest.fixture(scope="module")
+def stack_ref():
+    wl = synth.workload(WL)
+    cfgs = synth.stack_layer_cfgs(wl["cfg"], wl["n_layers"], wl["global_layers"])
+    weights = [_layer_weights(wl, l, c) for l, c in enumerate(cfgs)]
+    x = synth.layer_input(wl["cfg"], wl["B"], wl["T"], wl["seed"])
+    streams = _oracle_stack(wl, cfgs, weights, x[0, :T_PREFIX])
+    # the oracle's own sensitivity: the same stack on the input perturbed by PERTURB
+    g = np.random.default_rng([wl["seed"], 99])
+    xp = x[0, :T_PREFIX].astype(np.float64)
+    xp = xp + PERTURB * np.sqrt(np.mean(xp * xp)) * g.standard_normal(xp.shape)
+    growth = _oracle_stack(wl, cfgs, weights, xp, ref=streams)  # relative L2 at each depth
+    return dict(wl=wl, cfgs=cfgs, weights=weights, x=x, streams=streams, growth=np.array(growth))
+
+
+def _run_gpu(wl, cfgs, weights, first, h_np, has_meta):
+    """Layers first.. of cfgs in place on the fp32 stream h; the prefix rows of
+    sequence 0 after every layer."""
     torch = torch_cuda()
     import hybrid_head_ssm_b200 as hy
     from hybrid_head_ssm_b200 import runtime as rt
     B = h_np.shape[0]
-    m = cfgs[0].n_meta
-    T = wl["T"]
+    m, T = cfgs[0].n_meta, wl["T"]
     Tp = m + T
     h = rt.to_device(h_np, cfgs[0], io_f32=True)
     out = h if has_meta else torch.empty((B, Tp, cfgs[0].d_model), dtype=torch.float32, device="cuda")
     ws = rt.workspace(cfgs[0].with_(is_kv_producer=1), B, T, hy.HYMBA_MODE_PREFILL)
     kv, outs = None, []
     for i, cfg in enumerate(cfgs):
-        l = first + i
-        layer = rt.DeviceLayer(cfg, _layer_weights(wl, l, cfg))
+        layer = rt.DeviceLayer(cfg, weights[first + i])
         fl = rt.stream_flags(cfg) | (hy.HYMBA_X_HAS_META if (has_meta or i > 0) else 0)
         if cfg.is_kv_producer:
             kv = rt.KV(cfg, B, seq_cap=Tp)
@@ -59,8 +97,7 @@ def run_layers_gpu(wl, cfgs, first, h_np, has_meta):
         else:
             kvs = hy.hymba_kv()
             hy.check(hy.hymba_kv_share(ctypes.byref(kv.s), ctypes.byref(layer.c), ctypes.byref(kvs)))
-        src = h if i == 0 else out
-        rt.prefill(layer, src, T, kv, out, ws, None, fl, kv_struct_override=kvs)
+        rt.prefill(layer, h if i == 0 else out, T, kv, out, ws, None, fl, kv_struct_override=kvs)
         torch.cuda.synchronize()
         outs.append(to_np(out[0, :m + T_PREFIX]))
         del layer
@@ -68,52 +105,51 @@ def run_layers_gpu(wl, cfgs, first, h_np, has_meta):
     return outs
 
 
-def run_layers_oracle(wl, cfgs, first, h_row, has_meta):
-    kv, outs = None, []
-    h = h_row[None]
-    for i, cfg in enumerate(cfgs):
-        r = oracle.mixer_prefill(cfg, _layer_weights(wl, first + i, cfg), h,
-                                 kv_shared=None if cfg.is_kv_producer else kv, residual=True,
-                                 x_has_meta=has_meta or i > 0)
-        if cfg.is_kv_producer:
-            kv = (r["k"], r["v"])
-        h = r["y"]
-        outs.append(h[0])
-    return outs
+@pytest.fixture(scope="module")
+def pair_errors(stack_ref):
+    """Runs the 16 KV-sharing pairs on the GPU; (max abs, rel L2) per layer."""
+    wl, cfgs, weights, streams = stack_ref["wl"], stack_ref["cfgs"], stack_ref["weights"], stack_ref["streams"]
+    B, T, m, d = wl["B"], wl["T"], wl["cfg"].n_meta, wl["cfg"].d_model
+    errs = {}
+    for first in range(0, wl["n_layers"], 2):
+        if first == 0:
+            h, has_meta = stack_ref["x"], False
+        else:
+            s = streams[first]
+            g = np.random.default_rng([wl["seed"], 77, first])
+            h = (g.standard_normal((B, m + T, d)) * np.sqrt(np.mean(s * s))).astype(np.float32)
+            h[0, :m + T_PREFIX] = s
+            has_meta = True
+        got = _run_gpu(wl, cfgs[first:first + 2], weights, first, h, has_meta)
+        for i in range(2):
+            errs[first + i] = errors(got[i], streams[first + i + 1])
+    return errs
 
 
-@pytest.mark.parametrize("first", [0, 14, 30])
-def test_stack32_pair_at_full_size(first):
-    """Layers (first, first+1) of the stack: a KV-sharing producer/consumer pair, B=8,
-    T=4096, on a seeded input with the residual stream's scale at that depth."""
-    wl = synth.workload(WL)
-    cfgs = synth.stack_layer_cfgs(wl["cfg"], wl["n_layers"], wl["global_layers"])[first:first + 2]
-    B, T, m = wl["B"], wl["T"], wl["cfg"].n_meta
-    if first == 0:
-        h = synth.layer_input(wl["cfg"], B, T, wl["seed"])
-        has_meta = False
-    else:
-        g = np.random.default_rng([wl["seed"], 77, first])
-        h = (g.standard_normal((B, m + T, wl["cfg"].d_model)) * DEPTH_RMS[first]).astype(np.float32)
-        has_meta = True
-    got = run_layers_gpu(wl, cfgs, first, h, has_meta)
-    ref = run_layers_oracle(wl, cfgs, first, h[0, :(T_PREFIX if first == 0 else m + T_PREFIX)], has_meta)
-    for i in range(2):
-        mx, rl = assert_close(got[i], ref[i], wl["cfg"], f"layer {first + i}")
-        print(f"stack layer {first + i} (full size, sequence 0, {m + T_PREFIX} rows): max abs {mx:.3e}, rel L2 {rl:.3e}")
+def test_stack32_every_pair_at_full_size(pair_errors):
+    """All 16 KV-sharing pairs, each fed the oracle's own stream at its depth, within
+    max abs 2e-2 and relative L2 5e-3 on every output."""
+    bad = []
+    for l, (mx, rl) in sorted(pair_errors.items()):
+        print(f"stack layer {l} (pair input from the oracle's stream): max abs {mx:.3e}, rel L2 {rl:.3e}")
+        if not (mx <= BF16_MAX_ABS and rl <= BF16_REL_L2):
+            bad.append((l, mx, rl))
+    assert not bad, bad
 
 
-def test_stack32_end_to_end_deviation_is_bounded():
-    """All 32 layers end to end: every output finite, and the deviation from the fp64
-    oracle within the growth the oracle itself shows (rel L2 below 1, printed)."""
-    wl = synth.workload(WL)
-    cfgs = synth.stack_layer_cfgs(wl["cfg"], wl["n_layers"], wl["global_layers"])
-    x = synth.layer_input(wl["cfg"], wl["B"], wl["T"], wl["seed"])
-    got = run_layers_gpu(wl, cfgs, 0, x, False)
-    ref = run_layers_oracle(wl, cfgs, 0, x[0, :T_PREFIX], False)
-    for l in (0, 1, 3, 7, 15, 31):
-        mx, rl = errors(got[l], ref[l])
-        print(f"stack end to end after layer {l}: max abs {mx:.3e}, rel L2 {rl:.3e}")
+def test_stack32_end_to_end_within_the_propagated_bound(stack_ref, pair_errors):
+    """All 32 layers end to end on the workload input: at every depth the relative L2
+    from the oracle stays within twice sum_l e_l a(depth) / a(l), e_l the per-layer
+    errors measured on the pairs and a(.) the oracle's own growth of a perturbation."""
+    wl, cfgs, weights, streams, growth = (stack_ref[k] for k in ("wl", "cfgs", "weights", "streams", "growth"))
+    got = _run_gpu(wl, cfgs, weights, 0, stack_ref["x"], False)
     assert all(np.isfinite(g).all() for g in got)
-    mx, rl = errors(got[-1], ref[-1])
-    assert rl < 1.0, rl
+    a = growth / growth[0]  # a[l]: growth of an input perturbation up to depth l
+    e = np.array([pair_errors[l][1] for l in range(wl["n_layers"])])
+    print(f"oracle growth of a {PERTURB:g} input perturbation after 32 layers: x{a[-1]:.1f}")
+    for depth in range(1, wl["n_layers"] + 1):
+        mx, rl = errors(got[depth - 1], streams[depth])
+        bound = 2.0 * float(np.sum(e[:depth] * a[depth] / a[1:depth + 1]))
+        if depth in (1, 2, 4, 8, 16, 24, 32):
+            print(f"stack end to end after layer {depth - 1}: max abs {mx:.3e}, rel L2 {rl:.3e} (bound {bound:.3e})")
+        assert rl <= bound, (depth, rl, bound)

@@ -50,16 +50,26 @@ def _decoded_layer(cfg, B, T0, cache_cap, seed):
     return dict(layer=layer, kv=kv, q=q, ldp=ldp, o_ref=o_ref, mdt=mdt)
 
 
-@pytest.mark.parametrize("kind", ["bf16_hymba15_ring", "f32_tiny_global"])
+@pytest.mark.parametrize("kind", ["bf16_hymba15_ring", "f32_tiny_global", "bf16_hymba15_wrapped_5splits",
+                                  "f32_tiny_global_3splits"])
 def test_static_decode_attention_matches_mixer_decode(kind):
+    """One split (80-slot caches) and several: the 1.5B ring of 1024 + 128 meta slots
+    after 1500 prompt tokens (wrapped; 5 splits of 256 keys here, 9 of 128 in the
+    mixer) and a global fp32 cache of 616 slots (3 splits)."""
     torch = torch_cuda()
     import hybrid_head_ssm_b200 as hy
     if kind == "bf16_hymba15_ring":
         cfg = synth.hymba15_layer_cfg(window=64).with_(n_meta=16)
         B, T0, cap = 16, 150, 16 + 64
-    else:
+    elif kind == "f32_tiny_global":
         cfg = synth.tiny_layer_cfg().with_(window=0)
         B, T0, cap = 3, 40, 16 + 64
+    elif kind == "bf16_hymba15_wrapped_5splits":
+        cfg = synth.hymba15_layer_cfg(window=1024)
+        B, T0, cap = 8, 1500, 128 + 1024
+    else:
+        cfg = synth.tiny_layer_cfg().with_(window=0)
+        B, T0, cap = 2, 520, 16 + 600
     r = _decoded_layer(cfg, B, T0, cap, seed=5)
     H, dv = cfg.n_q_heads, cfg.v_head_dim
     for call in range(2):
@@ -90,3 +100,14 @@ def test_static_decode_attention_rejects_requests_beyond_its_scratch():
                                      ctypes.byref(kv), 1 << 30, B, None)
     assert rc == hy.HYMBA_ERR_SCRATCH_LIMIT
     assert "scratch" in hy.hymba_strerror(rc).decode()
+
+
+def test_static_decode_attention_visible_set_bit_exact():
+    """The allocation-free entry point attends to exactly the visible cache slots
+    (K = 0, one-hot V; see test_gpu_visibility): the 1.5B ring of 1024 + 128 slots
+    before and after it wraps (5 splits of 256 keys), and a short window."""
+    from test_gpu_visibility import _decode_visibility
+    cfg = synth.hymba15_layer_cfg(1024)
+    _decode_visibility(cfg, 8, 128 + 1024, (1, 300, 128 + 1024, 128 + 4096 + 1), 31, static=True)
+    small = cfg.with_(d_model=256, n_q_heads=5, n_kv_heads=1, d_inner=640, dt_rank=24, n_meta=16, window=7)
+    _decode_visibility(small, 3, 16 + 7, (5, 23, 61), 32, static=True)
