@@ -31,8 +31,11 @@ Readings taken where the pages are silent:
 
 * Fusion of the two branches: each branch is RMS-normalised over its full
   width, scaled per channel by beta1 / beta2, and the two are averaged before
-  W_o. The [Hymba Guide] formula concatenates instead; averaging needs equal
-  widths, so the V head dim is d_inner / n_q_heads.
+  W_o; averaging needs equal widths, so the V head dim is d_inner / n_q_heads.
+  The [Hymba Guide] formula concatenates instead: that variant (cfg.fusion = 1)
+  places the same normalised, beta-scaled branches side by side, Mamba first, with
+  the V head dim equal to the Q/K head dim, and W_o takes d_inner + n_q_heads *
+  v_head_dim inputs.
 * One input projection yields [Q | K | V | x | z | B | C | dt_low] in that order.
   A consumer (KV-sharing secondary) layer has no K, V rows.
 * A consumer's affine adaptation of the shared K, V acts on the K that is shared
@@ -221,6 +224,22 @@ def fuse(o_attn: np.ndarray, y_ssm: np.ndarray, w: Dict[str, np.ndarray], eps: f
     return (w["beta1"].astype(np.float64) * a + w["beta2"].astype(np.float64) * s) / 2.0
 
 
+def fuse_concat(o_attn: np.ndarray, y_ssm: np.ndarray, w: Dict[str, np.ndarray], eps: float) -> np.ndarray:
+    """U = Concat[beta2 * RMS(ssm), beta1 * RMS(attn)] ([Hymba Guide] "Parallel Hybrid-Head
+    Layer Formulation": y = W_o(Concat[MambaHeads(x), AttentionHeads(x)]), the Mamba heads
+    first). Each branch keeps its RMSNorm and beta scaling; the branches are placed side
+    by side instead of averaged, so they may differ in width (ssm [L, d_inner], attn
+    [L, n_q_heads * v_head_dim]) and W_o takes both widths."""
+    a = rms_norm(o_attn, w["norm_attn_w"].astype(np.float64), eps) * w["beta1"].astype(np.float64)
+    s = rms_norm(y_ssm, w["norm_ssm_w"].astype(np.float64), eps) * w["beta2"].astype(np.float64)
+    return np.concatenate([s, a], axis=-1)
+
+
+def fuse_layer(cfg, o_attn, y_ssm, w, eps):
+    """The layer's fusion: the beta-average, or the concatenation when cfg.fusion == 1."""
+    return fuse_concat(o_attn, y_ssm, w, eps) if getattr(cfg, "fusion", 0) == 1 else fuse(o_attn, y_ssm, w, eps)
+
+
 # ----------------------------------------------------------------------------
 # the layer
 # ----------------------------------------------------------------------------
@@ -286,7 +305,7 @@ def mixer_prefill_row(cfg, w: Dict[str, np.ndarray], x: np.ndarray,
     y_pre, h = selective_scan(xc, delta, A, blocks["B"], blocks["C"], w["D"])
     y_ssm = y_pre * silu(blocks["z"])
     # fusion and the shared output projection
-    u = fuse(o, y_ssm, w, cfg.rms_eps)
+    u = fuse_layer(cfg, o, y_ssm, w, cfg.rms_eps)
     y = u @ w["w_out"].T
     if residual:
         y = y + xh
@@ -374,7 +393,7 @@ def mixer_decode(cfg, w, x_t: np.ndarray, cache: dict, h: np.ndarray, conv: np.n
         A = -np.exp(w["A_log"])
         y_pre, h[b] = selective_scan(xc, delta, A, blocks["B"], blocks["C"], w["D"], h[b])
         y_ssm = y_pre * silu(blocks["z"])
-        u = fuse(o, y_ssm, w, cfg.rms_eps)
+        u = fuse_layer(cfg, o, y_ssm, w, cfg.rms_eps)
         y[b] = (u @ w["w_out"].T)[0] + (x_t[b] if residual else 0.0)
     return y
 

@@ -43,6 +43,12 @@ class LayerCfg:
     dtype: int             # F32 or BF16 (activations and big weights)
     rope_base: float = 10000.0
     rms_eps: float = 1e-6
+    fusion: int = 0        # 0: beta-average of the two branches; 1: concatenation [Mamba | Attention]
+
+    @property
+    def u_width(self) -> int:
+        """Width of the fused branches (the input of W_o)."""
+        return self.d_inner + self.n_q_heads * self.v_head_dim if self.fusion == 1 else self.d_inner
 
     @property
     def n_in(self) -> int:
@@ -145,7 +151,7 @@ def layer_weights(cfg: LayerCfg, seed: int) -> Dict[str, np.ndarray]:
         "norm_ssm_w": np.ones(di, np.float32),
         "beta1": np.ones(H * dv, np.float32),
         "beta2": np.ones(di, np.float32),
-        "w_out": to_storage(_normal(_rng(seed, 6), (d, di), 1.0 / di), cfg.dtype),
+        "w_out": to_storage(_normal(_rng(seed, 6), (d, cfg.u_width), 1.0 / cfg.u_width), cfg.dtype),
         "meta": to_storage(_normal(_rng(seed, 7), (cfg.n_meta, d), 0.02), cfg.dtype),
     }
     return w

@@ -242,3 +242,79 @@ def test_decode_equals_prefill_with_affine_shared_kv(window):
         ya = oracle.mixer_decode(ca, wa, x[:, t], cache, ha, conva, residual=True)
         yb = oracle.mixer_decode(cb, wb, ya, cache, hb, convb, residual=True)
         np.testing.assert_allclose(yb, rb["y"][:, m + t], rtol=1e-10, atol=1e-10)
+
+
+def test_ragged_decode_batch_equals_each_sequence_prefilled():
+    """Sequences of one decode batch may sit at different positions: each keeps its own
+    length, ring slot and state ("51cto" Hymba-1.5B article, section 4, notes that the
+    released code wants batch 1 for generation because padded meta tokens and the
+    sliding window do not mix; a per-sequence position needs no padding). Three
+    sequences prefilled alone with 5, 13 and 22 tokens (window 8: rings at different
+    phases of their wrap) and then decoded together equal each sequence prefilled at
+    its final length."""
+    ca, cb, wa, wb = _pair(8, seed=91)
+    m, cap = ca.n_meta, ca.n_meta + 8
+    lens, steps = (5, 13, 22), 9
+    B = len(lens)
+    x = synth.layer_input(ca, B, max(lens) + steps, 92)
+    caches, hs = [], []
+    for b, T0 in enumerate(lens):
+        pa = oracle.mixer_prefill(ca, wa, x[b:b + 1, :T0], residual=True)
+        pb = oracle.mixer_prefill(cb, wb, pa["y"], kv_shared=(pa["k"], pa["v"]), residual=True, x_has_meta=True)
+        caches.append(oracle.cache_from_prefill(ca, pa["k"], pa["v"], cap))
+        hs.append((pa["h"], pa["conv"], pb["h"], pb["conv"]))
+    cache = {k: np.concatenate([c[k] for c in caches]) for k in ("k", "v", "len")}
+    ha, conva, hb, convb = (np.concatenate([h[i] for h in hs]) for i in range(4))
+    for s in range(steps):
+        xt = np.stack([x[b, lens[b] + s] for b in range(B)])
+        ya = oracle.mixer_decode(ca, wa, xt, cache, ha, conva, residual=True)
+        yb = oracle.mixer_decode(cb, wb, ya, cache, hb, convb, residual=True)
+        for b, T0 in enumerate(lens):
+            ra = oracle.mixer_prefill(ca, wa, x[b:b + 1, :T0 + s + 1], residual=True)
+            rb = oracle.mixer_prefill(cb, wb, ra["y"], kv_shared=(ra["k"], ra["v"]), residual=True, x_has_meta=True)
+            np.testing.assert_allclose(yb[b], rb["y"][0, -1], rtol=1e-10, atol=1e-10)
+    assert list(cache["len"]) == [m + T0 + steps for T0 in lens]
+
+
+def _concat_cfg():
+    """The tiny layer with the concat fusion ("Hymba Guide", Parallel Hybrid-Head Layer
+    Formulation: y = W_o(Concat[MambaHeads(x), AttentionHeads(x)])), V head dim = 64."""
+    return synth.tiny_layer_cfg().with_(fusion=1, v_head_dim=64)
+
+
+def test_concat_fusion_is_the_sum_of_the_two_partial_products():
+    """W_o applied to [Mamba | Attention] equals W_o's first d_inner columns applied to
+    the normalised Mamba branch plus its last H * dv columns applied to the normalised
+    attention branch; widths d_inner + H * dv."""
+    cfg = _concat_cfg()
+    w = synth.perturbed_weights(synth.layer_weights(cfg, 101), cfg, 101)
+    x = synth.layer_input(cfg, 1, 30, 101)
+    r = oracle.mixer_prefill(cfg, w, x)
+    di, hv = cfg.d_inner, cfg.n_q_heads * cfg.v_head_dim
+    assert r["u"].shape[-1] == di + hv == w["w_out"].shape[1]
+    s = oracle.rms_norm(r["y_ssm"], w["norm_ssm_w"].astype(np.float64), cfg.rms_eps) * w["beta2"]
+    a = oracle.rms_norm(r["o_attn"], w["norm_attn_w"].astype(np.float64), cfg.rms_eps) * w["beta1"]
+    wo = w["w_out"].astype(np.float64)
+    np.testing.assert_allclose(r["y"], s @ wo[:, :di].T + a @ wo[:, di:].T, rtol=1e-10, atol=1e-12)
+
+
+def test_concat_with_equal_halves_is_twice_the_average():
+    """With equal branch widths and W_o = [W | W], the concatenation gives 2 * the
+    beta-average through W: both fusions share the per-branch norm and beta scaling."""
+    base = synth.tiny_layer_cfg()
+    cat = base.with_(fusion=1)  # v_head_dim 128: H * dv = d_inner
+    w = synth.perturbed_weights(synth.layer_weights(base, 102), base, 102)
+    wc = dict(w, w_out=np.concatenate([w["w_out"], w["w_out"]], axis=1))
+    x = synth.layer_input(base, 1, 25, 102)
+    ra = oracle.mixer_prefill(base, w, x)
+    rc = oracle.mixer_prefill(cat, wc, x)
+    np.testing.assert_allclose(rc["y"], 2.0 * ra["y"], rtol=1e-10, atol=1e-12)
+
+
+def test_concat_beta1_zero_drops_attention():
+    cfg = _concat_cfg()
+    w = synth.layer_weights(cfg, 103)
+    w = dict(w, beta1=np.zeros_like(w["beta1"]))
+    x = synth.layer_input(cfg, 1, 20, 103)
+    r = oracle.mixer_prefill(cfg, w, x)
+    assert np.all(r["u"][..., cfg.d_inner:] == 0.0)
