@@ -42,7 +42,7 @@ LAYER_WORKLOADS = ("hymba15_global_b4_t8192", "hymba15_swa1024_b1_t2048")
 DECODE_WORKLOAD = "hymba15_decode_pair_b64_p4096"
 
 
-MUFU_PER_CLK_SM = 16  # exp2 / rcp results per clock per SM (4 per SM sub-partition)
+MUFU_PER_CLK_SM = 16  # nominal exp2 / rcp results per clock per SM (4 per SM sub-partition)
 
 
 def peaks():
@@ -85,10 +85,12 @@ def roofline_entry(name, bound, units, avg_s, pk, sm_count, sm_mhz, long_step=Fa
                 "peak_kind": f"bf16 dense, {kind}, {pk['src']}"}
     if bound == "alu":
         ach = units / avg_s / 1e9
-        peak = MUFU_PER_CLK_SM * sm_count * sm_mhz * 1e-3
+        rate = pk.get("mufu_per_clk_sm") or MUFU_PER_CLK_SM
+        src = "measured by hymba_probe_unit_rates" if pk.get("mufu_per_clk_sm") else "nominal"
+        peak = rate * sm_count * sm_mhz * 1e-3
         return {"kernel": name, "bound": "alu", "achieved": ach, "peak": peak, "unit": "G MUFU op/s",
                 "frac": ach / peak,
-                "peak_kind": f"{MUFU_PER_CLK_SM} MUFU results per clock per SM x {sm_count} SMs x {sm_mhz:.0f} MHz "
+                "peak_kind": f"{rate:.2f} exp2 results per clock per SM ({src}) x {sm_count} SMs x {sm_mhz:.0f} MHz "
                              "(SM clock sampled in the timed region)"}
     ach = units / avg_s / 1e9
     return {"kernel": name, "bound": "hbm", "achieved": ach, "peak": pk["hbm"], "unit": "GB/s",
@@ -651,6 +653,8 @@ def main():
 
     pk = peaks()
     sm_count = torch.cuda.get_device_properties(local).multi_processor_count
+    rates = hy.unit_rates()  # exp2 and FMA results per clock per SM, measured on this GPU
+    pk["mufu_per_clk_sm"] = rates["ex2_f32"]
     flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")  # > 126 MB L2
 
     clocks = Clocks(local, args.clocks_dir)
@@ -695,6 +699,7 @@ def main():
             "gpu_launches": int(round(head["launches"] * args.steps)),
             "gpu_launches_per_step": head["launches"],
             "clocks": head["clk"],
+            "unit_rates_per_clk_sm": rates,
             "kernels": head["kern"],
             "extra": extra,
         }

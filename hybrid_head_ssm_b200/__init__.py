@@ -39,6 +39,8 @@ HYMBA_F16 = 2
 HYMBA_X_HAS_META = 1
 HYMBA_ADD_RESIDUAL = 2
 HYMBA_IO_F32 = 4
+HYMBA_FUSION_AVERAGE = 0
+HYMBA_FUSION_CONCAT = 1
 HYMBA_MODE_PREFILL = 0
 HYMBA_MODE_DECODE = 1
 
@@ -49,7 +51,7 @@ class hymba_layer_cfg(ctypes.Structure):
     _fields_ = [("d_model", _i32), ("n_q_heads", _i32), ("n_kv_heads", _i32), ("head_dim", _i32),
                 ("v_head_dim", _i32), ("d_inner", _i32), ("d_state", _i32), ("d_conv", _i32),
                 ("dt_rank", _i32), ("n_meta", _i32), ("window", _i32), ("is_kv_producer", _i32),
-                ("dtype", _i32), ("rope_base", _f32), ("rms_eps", _f32)]
+                ("dtype", _i32), ("rope_base", _f32), ("rms_eps", _f32), ("fusion", _i32)]
 
 
 class hymba_layer_weights(ctypes.Structure):
@@ -93,6 +95,9 @@ _sig = {
     "hymba_launch_count": (ctypes.c_uint64, []),
     "hymba_attn_decode_static": (ctypes.c_int, [_P(hymba_layer_cfg), _vp, ctypes.c_int64, _P(hymba_kv), _vp,
                                                 ctypes.c_int, _vp]),
+    "hymba_probe_unit_rates": (ctypes.c_int, [_P(ctypes.c_double), ctypes.c_int, _vp]),
+    "hymba_debug_set_wait_limit": (ctypes.c_int, [ctypes.c_longlong]),
+    "hymba_debug_stalled_wait": (ctypes.c_int, [_vp]),
 }
 EXPORTS = tuple(_sig)
 
@@ -119,6 +124,13 @@ def workspace_layout(cfg: hymba_layer_cfg, B: int, T: int, mode: int) -> dict:
     check(hymba_workspace_layout(ctypes.byref(cfg), B, T, mode, out, 10))
     keys = ("total", "P", "ldP", "delta", "O", "ypre", "U", "rope", "part", "n_split")
     return dict(zip(keys, list(out)))
+
+
+def unit_rates():
+    """Measured exp2 (fp32, fp16 pairs) and fp32 FMA results per clock per SM."""
+    out = (ctypes.c_double * 3)()
+    check(hymba_probe_unit_rates(out, 3, current_stream_ptr()))
+    return {"ex2_f32": out[0], "ex2_f16x2": out[1], "ffma_f32": out[2]}
 
 
 def device_diag():

@@ -52,7 +52,10 @@ __device__ __forceinline__ float2 x2float(uint32_t v) {
     return __half22float2(h);
 }
 
-constexpr int KGROUPS = 8;  // key groups of the PV phase (128 threads = 8 groups x 16 pieces of 8)
+// PV phase of the register-streaming kernel: 128 threads = (DV / 8 pieces of 8 V elements)
+// x (128 / (DV / 8) key groups)
+template <int DV>
+constexpr int kgroups() { return 128 / (DV / 8); }
 
 // One block per (key split, KV head, sequence) serves the R query heads of the KV head.
 // Scores: four lanes per key, each holding its 16 dimensions of the R queries in
@@ -67,7 +70,9 @@ attn_decode_kernel(const T* __restrict__ P, long long ldP, const T* __restrict__
                    int pos_offset, float* __restrict__ part, int n_split, int H, int G,
                    int n_meta, int window, int* status) {
     griddep_sync();
-    static_assert(DV == 16 * 8, "PV phase covers a V row with 16 pieces of 8");
+    static_assert(DV == 64 || DV == 128, "V head dim");
+    constexpr int KGROUPS = kgroups<DV>();
+    constexpr int PIECES = DV / 8;
     static_assert(R >= 1 && R <= 8, "query heads per KV head");
     __shared__ __align__(16) float ps[MAX_CHUNK][8];
     __shared__ int slots[MAX_CHUNK];
@@ -157,7 +162,7 @@ attn_decode_kernel(const T* __restrict__ P, long long ldP, const T* __restrict__
     __syncthreads();
     // P V: thread (key group kg, piece eb) adds keys kg, kg + 8, ... for V elements eb*8..+7
     {
-        const int eb = tid % 16, kg = tid / 16;
+        const int eb = tid % PIECES, kg = tid / PIECES;
         float2 acc[R][4];
 #pragma unroll
         for (int r = 0; r < R; ++r)
@@ -220,7 +225,6 @@ attn_decode_kernel(const T* __restrict__ P, long long ldP, const T* __restrict__
 constexpr int BK_NST = 2;                      // stages
 constexpr int BK_STAGE = 16384;                // bytes per stage
 constexpr int BK_TK = BK_STAGE / (DH * 2);     // keys per K tile (128)
-constexpr int BK_TV = BK_STAGE / (128 * 2);    // keys per V tile (64)
 
 // Queue the bulk copies of one tile: the block-local keys [a, e) of the split, rows of
 // row_bytes, into dst in key order. The keys map to cache slots in at most three
@@ -255,14 +259,16 @@ __device__ __forceinline__ void bk_issue_tile(unsigned char* dst, const unsigned
 // eight lanes per key, each with its 8 dimensions of the R queries in registers, one
 // conflict-free 16-byte shared load per key, joined by three shuffles per head. P V:
 // warp w takes keys w, w + 4, ... of a tile, lane l elements 4l .. 4l + 3 of the V row.
-template <int R>
+template <int R, int DV>
 __global__ void __launch_bounds__(128, R <= 6 ? 5 : 4)
 attn_decode_bulk_kernel(const f16* __restrict__ P, long long ldP, const f16* __restrict__ k_cache,
                         const f16* __restrict__ v_cache, int cap, const int* __restrict__ len, int pos_offset,
                         float* __restrict__ part, int n_split, int H, int G, int n_meta, int window, int max_chunk,
                         int* status) {
     griddep_sync();
-    constexpr int DV = 128;
+    static_assert(DV == 64 || DV == 128, "V head dim");
+    constexpr int BK_TV = BK_STAGE / (DV * 2);  // keys per V tile
+    constexpr int EPL = DV / 32;                // V elements per lane in the PV phase
     static_assert(R >= 1 && R <= 8, "query heads per KV head");
     static_assert(4 * R * DV * 4 <= BK_NST * BK_STAGE, "the reduction buffer reuses the stages");
     extern __shared__ __align__(128) unsigned char bk_smem[];
@@ -314,14 +320,17 @@ attn_decode_bulk_kernel(const f16* __restrict__ P, long long ldP, const f16* __r
         for (int i = 0; i < 4; ++i)
             qr[r][i] = make_float2(qv[2 * i] * (LOG2E * 0.125f), qv[2 * i + 1] * (LOG2E * 0.125f));
     }
-    float2 acc[R][2];
+    float2 acc[R][EPL / 2];
 #pragma unroll
-    for (int r = 0; r < R; ++r) acc[r][0] = acc[r][1] = make_float2(0.f, 0.f);
+    for (int r = 0; r < R; ++r)
+#pragma unroll
+        for (int x = 0; x < EPL / 2; ++x) acc[r][x] = make_float2(0.f, 0.f);
     __syncthreads();
     bool ok = true;
+    const long long wlim = tc::wait_limit(status);
     for (int i = 0; i < nitems; ++i) {
         const int st = i % BK_NST;
-        if (ok) ok = tc::mbar_wait(&full[st], (uint32_t)((i / BK_NST) & 1), &bk_never);
+        if (ok) ok = tc::mbar_wait(&full[st], (uint32_t)((i / BK_NST) & 1), &bk_never, wlim);
         const unsigned char* sp = stages + st * BK_STAGE;
         if (i < nkt) {
             const int base = i * BK_TK, n = min(nk - base, BK_TK);
@@ -356,8 +365,14 @@ attn_decode_bulk_kernel(const f16* __restrict__ P, long long ldP, const f16* __r
             const int base = (i - nkt) * BK_TV, n = min(nk - base, BK_TV);
 #pragma unroll 2
             for (int kv = warp; kv < n; kv += 4) {
-                const uint2 u = *reinterpret_cast<const uint2*>(sp + kv * (DV * 2) + lane * 8);
-                const float2 v0 = x2float(u.x), v1 = x2float(u.y);
+                float2 vv[EPL / 2];
+                if constexpr (EPL == 4) {
+                    const uint2 u = *reinterpret_cast<const uint2*>(sp + kv * (DV * 2) + lane * 8);
+                    vv[0] = x2float(u.x);
+                    vv[1] = x2float(u.y);
+                } else {
+                    vv[0] = x2float(*reinterpret_cast<const uint32_t*>(sp + kv * (DV * 2) + lane * 4));
+                }
                 const float4 pa = *reinterpret_cast<const float4*>(&ps[base + kv][0]);
                 float4 pb = make_float4(0.f, 0.f, 0.f, 0.f);
                 if constexpr (R > 4) pb = *reinterpret_cast<const float4*>(&ps[base + kv][4]);
@@ -365,8 +380,8 @@ attn_decode_bulk_kernel(const f16* __restrict__ P, long long ldP, const f16* __r
 #pragma unroll
                 for (int r = 0; r < R; ++r) {
                     const float2 pr = make_float2(pw[r], pw[r]);
-                    acc[r][0] = __ffma2_rn(pr, v0, acc[r][0]);
-                    acc[r][1] = __ffma2_rn(pr, v1, acc[r][1]);
+#pragma unroll
+                    for (int x = 0; x < EPL / 2; ++x) acc[r][x] = __ffma2_rn(pr, vv[x], acc[r][x]);
                 }
             }
         }
@@ -404,8 +419,11 @@ attn_decode_bulk_kernel(const f16* __restrict__ P, long long ldP, const f16* __r
     // the four warps' P V sums meet in the stage memory (every copy has landed)
 #pragma unroll
     for (int r = 0; r < R; ++r)
-        *reinterpret_cast<float4*>(&red[(warp * R + r) * DV + 4 * lane]) =
-            make_float4(acc[r][0].x, acc[r][0].y, acc[r][1].x, acc[r][1].y);
+        if constexpr (EPL == 4)
+            *reinterpret_cast<float4*>(&red[(warp * R + r) * DV + 4 * lane]) =
+                make_float4(acc[r][0].x, acc[r][0].y, acc[r][1].x, acc[r][1].y);
+        else
+            *reinterpret_cast<float2*>(&red[(warp * R + r) * DV + 2 * lane]) = acc[r][0];
     __syncthreads();
     for (int i = tid; i < R * DV; i += blockDim.x) {
         const int r = i / DV, e = i % DV;
@@ -680,6 +698,60 @@ ssm_decode_kernel(const T* __restrict__ P, long long ldP, int col_x, int col_B, 
     }
 }
 
+
+template <int DV>
+static void (*bulk_kernel(int R))(const f16*, long long, const f16*, const f16*, int, const int*, int, float*, int,
+                                  int, int, int, int, int, int*) {
+    switch (R) {
+        case 1: return attn_decode_bulk_kernel<1, DV>;
+        case 2: return attn_decode_bulk_kernel<2, DV>;
+        case 3: return attn_decode_bulk_kernel<3, DV>;
+        case 4: return attn_decode_bulk_kernel<4, DV>;
+        case 5: return attn_decode_bulk_kernel<5, DV>;
+        case 6: return attn_decode_bulk_kernel<6, DV>;
+        case 7: return attn_decode_bulk_kernel<7, DV>;
+        default: return attn_decode_bulk_kernel<8, DV>;
+    }
+}
+
+template <typename T, int DV>
+static void (*stream_kernel(int R))(const T*, long long, const T*, const T*, int, const int*, int, float*, int, int,
+                                    int, int, int, int*) {
+    switch (R) {
+        case 1: return attn_decode_kernel<T, DV, 1>;
+        case 2: return attn_decode_kernel<T, DV, 2>;
+        case 3: return attn_decode_kernel<T, DV, 3>;
+        case 4: return attn_decode_kernel<T, DV, 4>;
+        case 5: return attn_decode_kernel<T, DV, 5>;
+        case 6: return attn_decode_kernel<T, DV, 6>;
+        case 7: return attn_decode_kernel<T, DV, 7>;
+        default: return attn_decode_kernel<T, DV, 8>;
+    }
+}
+
+template <typename T, int DV>
+static int attn_decode_dv(const Ctx& ctx, const T* P, long long ldP, const T* k_cache, const T* v_cache,
+                          int cache_cap, const int* len, int pos_offset, float* part, int n_split, T* O, int B,
+                          int H, int G, int n_meta, int window) {
+    dim3 grid(n_split, G, B);
+    if constexpr (std::is_same<T, f16>::value) {
+        // K/V rows staged by bulk copies: 16-byte aligned rows (64 and DV fp16)
+        const int max_chunk = (cache_cap + n_split - 1) / n_split;
+        const size_t smem = (size_t)BK_NST * BK_STAGE + (size_t)max_chunk * 32 + 16 * sizeof(float) +
+                            BK_NST * sizeof(uint64_t);
+        HYMBA_LAUNCH(ctx, "attn_decode", bulk_kernel<DV>(H / G), grid, 128, smem, P, ldP, k_cache, v_cache,
+                     cache_cap, len, pos_offset, part, n_split, H, G, n_meta, window, max_chunk, ctx.status);
+    } else {
+        HYMBA_LAUNCH(ctx, "attn_decode", (stream_kernel<T, DV>(H / G)), grid, 128, 0, P, ldP, k_cache, v_cache,
+                     cache_cap, len, pos_offset, part, n_split, H, G, n_meta, window, ctx.status);
+    }
+    if (!O) return HYMBA_OK;  // the caller merges the splits itself
+    dim3 g2(H, B);
+    auto k2 = attn_decode_combine_kernel<T, DV>;
+    HYMBA_LAUNCH(ctx, "attn_decode_combine", k2, g2, DV, 0, part, n_split, O, H);
+    return HYMBA_OK;
+}
+
 }  // namespace
 
 template <typename T>
@@ -687,56 +759,17 @@ int launch_attn_decode(const Ctx& ctx, const T* P, long long ldP, const T* k_cac
                        const T* v_cache, int cache_cap, const int* len, int pos_offset,
                        float* part, int n_split, T* O, int B, int H, int G, int dv, int n_meta,
                        int window) {
-    if (H / G > MAX_R || dv != 128) return HYMBA_ERR_UNSUPPORTED;
+    if (H / G > MAX_R || (dv != 128 && dv != 64)) return HYMBA_ERR_UNSUPPORTED;
     if ((cache_cap + n_split - 1) / n_split > MAX_CHUNK) return HYMBA_ERR_INVALID_ARG;
-    dim3 grid(n_split, G, B);
     // 16-byte loads of q, K and V rows
     if ((reinterpret_cast<uintptr_t>(P) | reinterpret_cast<uintptr_t>(k_cache) | reinterpret_cast<uintptr_t>(v_cache)) & 15 ||
         ldP % (16 / (long long)sizeof(T)))
         return HYMBA_ERR_UNSUPPORTED;
-    if constexpr (std::is_same<T, f16>::value) {
-        // K/V rows staged by bulk copies: 16-byte aligned rows (64 and 128 fp16)
-        const int max_chunk = (cache_cap + n_split - 1) / n_split;
-        const size_t smem = (size_t)BK_NST * BK_STAGE + (size_t)max_chunk * 32 + 16 * sizeof(float) +
-                            BK_NST * sizeof(uint64_t);
-        void (*kb)(const f16*, long long, const f16*, const f16*, int, const int*, int, float*, int, int, int, int,
-                   int, int, int*);
-        switch (H / G) {
-            case 1: kb = attn_decode_bulk_kernel<1>; break;
-            case 2: kb = attn_decode_bulk_kernel<2>; break;
-            case 3: kb = attn_decode_bulk_kernel<3>; break;
-            case 4: kb = attn_decode_bulk_kernel<4>; break;
-            case 5: kb = attn_decode_bulk_kernel<5>; break;
-            case 6: kb = attn_decode_bulk_kernel<6>; break;
-            case 7: kb = attn_decode_bulk_kernel<7>; break;
-            default: kb = attn_decode_bulk_kernel<8>; break;
-        }
-        HYMBA_LAUNCH(ctx, "attn_decode", kb, grid, 128, smem, P, ldP, k_cache, v_cache, cache_cap, len, pos_offset,
-                     part, n_split, H, G, n_meta, window, max_chunk, ctx.status);
-        if (!O) return HYMBA_OK;  // the caller merges the splits itself
-        dim3 g2(H, B);
-        auto k2 = attn_decode_combine_kernel<T, 128>;
-        HYMBA_LAUNCH(ctx, "attn_decode_combine", k2, g2, 128, 0, part, n_split, O, H);
-        return HYMBA_OK;
-    }
-    void (*k1)(const T*, long long, const T*, const T*, int, const int*, int, float*, int, int, int, int, int, int*);
-    switch (H / G) {
-        case 1: k1 = attn_decode_kernel<T, 128, 1>; break;
-        case 2: k1 = attn_decode_kernel<T, 128, 2>; break;
-        case 3: k1 = attn_decode_kernel<T, 128, 3>; break;
-        case 4: k1 = attn_decode_kernel<T, 128, 4>; break;
-        case 5: k1 = attn_decode_kernel<T, 128, 5>; break;
-        case 6: k1 = attn_decode_kernel<T, 128, 6>; break;
-        case 7: k1 = attn_decode_kernel<T, 128, 7>; break;
-        default: k1 = attn_decode_kernel<T, 128, 8>; break;
-    }
-    HYMBA_LAUNCH(ctx, "attn_decode", k1, grid, 128, 0, P, ldP, k_cache, v_cache, cache_cap, len,
-                 pos_offset, part, n_split, H, G, n_meta, window, ctx.status);
-    if (!O) return HYMBA_OK;  // the caller merges the splits itself
-    dim3 g2(H, B);
-    auto k2 = attn_decode_combine_kernel<T, 128>;
-    HYMBA_LAUNCH(ctx, "attn_decode_combine", k2, g2, 128, 0, part, n_split, O, H);
-    return HYMBA_OK;
+    if (dv == 128)
+        return attn_decode_dv<T, 128>(ctx, P, ldP, k_cache, v_cache, cache_cap, len, pos_offset, part, n_split, O, B,
+                                      H, G, n_meta, window);
+    return attn_decode_dv<T, 64>(ctx, P, ldP, k_cache, v_cache, cache_cap, len, pos_offset, part, n_split, O, B, H,
+                                 G, n_meta, window);
 }
 
 template <typename T, typename TW>

@@ -92,9 +92,11 @@ __device__ __forceinline__ void merge8(const float* __restrict__ part, int n_spl
 
 // (the decode variant runs one block per sequence, so it asks for no more than one
 // block per SM and keeps its merge temporaries in registers)
-template <typename I, typename T, bool SPLIT>
+// CONCAT: U = [beta2 * RMS(Y) | beta1 * RMS(O)] (d_inner + H * dv wide) instead of the
+// average (O and Y of equal width d_inner).
+template <typename I, typename T, bool SPLIT, bool CONCAT>
 __global__ void __launch_bounds__(TPR * RPB, SPLIT ? 1 : 4)
-fuse_kernel(const I* __restrict__ O, const float* __restrict__ part, int n_split, int H,
+fuse_kernel(const I* __restrict__ O, const float* __restrict__ part, int n_split, int H, int dv,
             const I* __restrict__ ypre, const I* __restrict__ P, long long ldP, int col_z,
             const float* __restrict__ g_attn, const float* __restrict__ g_ssm, const float* __restrict__ beta1,
             const float* __restrict__ beta2, const float* __restrict__ v_scale, const float* __restrict__ v_bias,
@@ -104,23 +106,23 @@ fuse_kernel(const I* __restrict__ O, const float* __restrict__ part, int n_split
     const int sub = threadIdx.x / TPR, t = threadIdx.x % TPR;
     const long long row = (long long)blockIdx.x * RPB + sub;
     const bool live = row < rows;
-    const int nvec = di / 8;
+    const int hv = H * dv;                 // attention branch width
+    const int nvo = hv / 8, nvy = di / 8;  // pieces of 8 per branch
     float o[VMAX][8], y[VMAX][8];
     float ss_o = 0.f, ss_y = 0.f;
 #pragma unroll
     for (int k = 0; k < VMAX; ++k) {
         const int vi = t + k * TPR;
-        if (live && vi < nvec) {
+        if (live && vi < nvo) {
             const int c = vi * 8;
-            float z[8];
             if constexpr (SPLIT)
-                merge8(part, n_split, H, di / H, row, c, o[k]);
+                merge8(part, n_split, H, dv, row, c, o[k]);
             else
-                load8<I>(O + row * di + c, o[k]);
+                load8<I>(O + row * hv + c, o[k]);
             if (v_scale) {
                 // a consumer's adapted shared V: attention over V * s + b is the attention
                 // output * s + b (the softmax weights sum to 1)
-                const int dv = di / H, hd = c / dv;
+                const int hd = c / dv;
                 const int idx = (hd / rep) * dv + (c - hd * dv);
                 float vs[8], vb[8];
                 load8f(v_scale + idx, vs);
@@ -128,12 +130,17 @@ fuse_kernel(const I* __restrict__ O, const float* __restrict__ part, int n_split
 #pragma unroll
                 for (int i = 0; i < 8; ++i) o[k][i] = fmaf(o[k][i], vs[i], vb[i]);
             }
+#pragma unroll
+            for (int i = 0; i < 8; ++i) ss_o = fmaf(o[k][i], o[k][i], ss_o);
+        }
+        if (live && vi < nvy) {
+            const int c = vi * 8;
+            float z[8];
             load8<I>(ypre + row * di + c, y[k]);
             load8<I>(P + row * ldP + col_z + c, z);
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
                 y[k][i] *= z[i] / (1.0f + __expf(-z[i]));
-                ss_o = fmaf(o[k][i], o[k][i], ss_o);
                 ss_y = fmaf(y[k][i], y[k][i], ss_y);
             }
         }
@@ -155,21 +162,45 @@ fuse_kernel(const I* __restrict__ O, const float* __restrict__ part, int n_split
         ss_o += red[sub][w][0];
         ss_y += red[sub][w][1];
     }
-    const float ro = 0.5f / sqrtf(ss_o / di + eps);
-    const float ry = 0.5f / sqrtf(ss_y / di + eps);
+    // the average halves both branches; the concatenation keeps them whole
+    const float half = CONCAT ? 1.0f : 0.5f;
+    const float ro = half / sqrtf(ss_o / hv + eps);
+    const float ry = half / sqrtf(ss_y / di + eps);
 #pragma unroll
     for (int k = 0; k < VMAX; ++k) {
         const int vi = t + k * TPR;
-        if (live && vi < nvec) {
-            const int c = vi * 8;
-            float ga[8], gs[8], b1[8], b2[8], u[8];
-            load8f(g_attn + c, ga);
-            load8f(g_ssm + c, gs);
-            load8f(beta1 + c, b1);
-            load8f(beta2 + c, b2);
+        if constexpr (CONCAT) {
+            const long long ldu = di + hv;
+            if (live && vi < nvy) {
+                const int c = vi * 8;
+                float gs[8], b2[8], u[8];
+                load8f(g_ssm + c, gs);
+                load8f(beta2 + c, b2);
 #pragma unroll
-            for (int i = 0; i < 8; ++i) u[i] = b1[i] * ga[i] * o[k][i] * ro + b2[i] * gs[i] * y[k][i] * ry;
-            store8<T>(U + row * di + c, u);
+                for (int i = 0; i < 8; ++i) u[i] = b2[i] * gs[i] * y[k][i] * ry;
+                store8<T>(U + row * ldu + c, u);
+            }
+            if (live && vi < nvo) {
+                const int c = vi * 8;
+                float ga[8], b1[8], u[8];
+                load8f(g_attn + c, ga);
+                load8f(beta1 + c, b1);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) u[i] = b1[i] * ga[i] * o[k][i] * ro;
+                store8<T>(U + row * ldu + di + c, u);
+            }
+        } else {
+            if (live && vi < nvy) {
+                const int c = vi * 8;
+                float ga[8], gs[8], b1[8], b2[8], u[8];
+                load8f(g_attn + c, ga);
+                load8f(g_ssm + c, gs);
+                load8f(beta1 + c, b1);
+                load8f(beta2 + c, b2);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) u[i] = b1[i] * ga[i] * o[k][i] * ro + b2[i] * gs[i] * y[k][i] * ry;
+                store8<T>(U + row * di + c, u);
+            }
         }
     }
     if (len_inc && live && t == 0) len_inc[row] += 1;
@@ -177,37 +208,49 @@ fuse_kernel(const I* __restrict__ O, const float* __restrict__ part, int n_split
 
 }  // namespace
 
-template <typename I, typename T>
-int launch_fuse(const Ctx& ctx, const I* O, const float* part, int n_split, int H, int G, const I* ypre,
-                const I* P, long long ldP, int col_z, const float* g_attn, const float* g_ssm, const float* beta1,
-                const float* beta2, const float* v_scale, const float* v_bias, T* U, int rows, int di, float eps,
-                int* len_inc) {
-    if (rows <= 0) return HYMBA_OK;
-    if (di % 8 || di > VMAX * 8 * TPR || col_z % 8 || ldP % 8) return HYMBA_ERR_UNSUPPORTED;
-    // pieces of 8 never straddle a head
-    if (H <= 0 || G <= 0 || H % G || di % H || (di / H) % 8) return HYMBA_ERR_UNSUPPORTED;
-    if ((v_scale == nullptr) != (v_bias == nullptr) ||
-        ((reinterpret_cast<uintptr_t>(v_scale) | reinterpret_cast<uintptr_t>(v_bias)) & 15))
-        return HYMBA_ERR_UNSUPPORTED;
+template <typename I, typename T, bool CONCAT>
+static int fuse_variant(const Ctx& ctx, const I* O, const float* part, int n_split, int H, int dv, int G,
+                        const I* ypre, const I* P, long long ldP, int col_z, const float* g_attn, const float* g_ssm,
+                        const float* beta1, const float* beta2, const float* v_scale, const float* v_bias, T* U,
+                        int rows, int di, float eps, int* len_inc) {
     if (part) {
-        // 8-byte loads of the partial sums
-        if (n_split <= 0 || (reinterpret_cast<uintptr_t>(part) & 7)) return HYMBA_ERR_UNSUPPORTED;
-        auto kern = fuse_kernel<I, T, true>;
-        HYMBA_LAUNCH(ctx, "fuse", kern, ceil_div(rows, RPB), TPR * RPB, 0, O, part, n_split, H, ypre, P, ldP,
+        auto kern = fuse_kernel<I, T, true, CONCAT>;
+        HYMBA_LAUNCH(ctx, "fuse", kern, ceil_div(rows, RPB), TPR * RPB, 0, O, part, n_split, H, dv, ypre, P, ldP,
                      col_z, g_attn, g_ssm, beta1, beta2, v_scale, v_bias, H / G, U, rows, di, eps, len_inc);
-        return HYMBA_OK;
+    } else {
+        auto kern = fuse_kernel<I, T, false, CONCAT>;
+        HYMBA_LAUNCH(ctx, "fuse", kern, ceil_div(rows, RPB), TPR * RPB, 0, O, part, n_split, H, dv, ypre, P, ldP,
+                     col_z, g_attn, g_ssm, beta1, beta2, v_scale, v_bias, H / G, U, rows, di, eps, len_inc);
     }
-    auto kern = fuse_kernel<I, T, false>;
-    HYMBA_LAUNCH(ctx, "fuse", kern, ceil_div(rows, RPB), TPR * RPB, 0, O, part, n_split, H, ypre, P, ldP, col_z,
-                 g_attn, g_ssm, beta1, beta2, v_scale, v_bias, H / G, U, rows, di, eps, len_inc);
     return HYMBA_OK;
 }
 
+template <typename I, typename T>
+int launch_fuse(const Ctx& ctx, const I* O, const float* part, int n_split, int H, int G, int dv, bool concat,
+                const I* ypre, const I* P, long long ldP, int col_z, const float* g_attn, const float* g_ssm,
+                const float* beta1, const float* beta2, const float* v_scale, const float* v_bias, T* U, int rows,
+                int di, float eps, int* len_inc) {
+    if (rows <= 0) return HYMBA_OK;
+    const int hv = H * dv;
+    if (di % 8 || di > VMAX * 8 * TPR || hv > VMAX * 8 * TPR || col_z % 8 || ldP % 8) return HYMBA_ERR_UNSUPPORTED;
+    // pieces of 8 never straddle a head
+    if (H <= 0 || G <= 0 || H % G || dv % 8 || (!concat && hv != di)) return HYMBA_ERR_UNSUPPORTED;
+    if ((v_scale == nullptr) != (v_bias == nullptr) ||
+        ((reinterpret_cast<uintptr_t>(v_scale) | reinterpret_cast<uintptr_t>(v_bias)) & 15))
+        return HYMBA_ERR_UNSUPPORTED;
+    // 8-byte loads of the partial sums
+    if (part && (n_split <= 0 || (reinterpret_cast<uintptr_t>(part) & 7))) return HYMBA_ERR_UNSUPPORTED;
+    if (concat)
+        return fuse_variant<I, T, true>(ctx, O, part, n_split, H, dv, G, ypre, P, ldP, col_z, g_attn, g_ssm, beta1,
+                                        beta2, v_scale, v_bias, U, rows, di, eps, len_inc);
+    return fuse_variant<I, T, false>(ctx, O, part, n_split, H, dv, G, ypre, P, ldP, col_z, g_attn, g_ssm, beta1,
+                                     beta2, v_scale, v_bias, U, rows, di, eps, len_inc);
+}
 
-#define HYMBA_FUSE_INST(I, T)                                                                              \
-    template int launch_fuse<I, T>(const Ctx&, const I*, const float*, int, int, int, const I*, const I*, long long, \
-                                   int, const float*, const float*, const float*, const float*, const float*,       \
-                                   const float*, T*, int, int, float, int*);
+#define HYMBA_FUSE_INST(I, T)                                                                                  \
+    template int launch_fuse<I, T>(const Ctx&, const I*, const float*, int, int, int, int, bool, const I*, const I*, \
+                                   long long, int, const float*, const float*, const float*, const float*,          \
+                                   const float*, const float*, T*, int, int, float, int*);
 HYMBA_FUSE_INST(float, float)
 HYMBA_FUSE_INST(f16, bf16)
 HYMBA_FUSE_INST(f16, f16)

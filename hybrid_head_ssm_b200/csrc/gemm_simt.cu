@@ -83,6 +83,7 @@ INST(f16, f16)
 INST(bf16, bf16)
 INST(bf16, float)
 INST(f16, float)
+INST(f16, bf16)
 #undef INST
 
 }  // namespace hymba

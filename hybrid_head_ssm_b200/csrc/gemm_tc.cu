@@ -96,6 +96,21 @@ __device__ __forceinline__ void fail(volatile int* abort, int* status, int role,
     tc::record_timeout(status, role, step, bar);
 }
 
+// Tile order: groups of GM row blocks, each walked column block by column block (row
+// blocks fastest), so the CTAs in flight share a few A row panels and a run of B
+// column panels, and both stay in L2 while they are reused (a plain row-fastest order
+// streams the whole A once per column block, which no longer fits in L2 for long
+// batches).
+constexpr int GM = 8;
+__device__ __forceinline__ void tile_coords(int tile, int num_m, int num_n, int* m_blk, int* n_blk) {
+    const int group = tile / (GM * num_n);
+    const int first_m = group * GM;
+    const int gsize = min(GM, num_m - first_m);
+    const int local = tile - group * GM * num_n;
+    *m_blk = first_m + local % gsize;
+    *n_blk = local / gsize;
+}
+
 template <typename TA, typename TO, int BN, int STAGES>
 __global__ void __launch_bounds__(NUM_THREADS, STAGES == 2 ? 2 : 1)
 gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
@@ -140,6 +155,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     griddep_sync();
     const uint32_t tmem = s.tmem_base;
     volatile int* abort = &s.abort;
+    const long long wlim = tc::wait_limit(status);
 
     if (warp == 0) {
         // ---------------- TMA producer ----------------
@@ -148,11 +164,12 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
             int issued_phase[STAGES];
             for (int i = 0; i < STAGES; ++i) issued_phase[i] = -1;
             for (int tile = blockIdx.x; tile < num_tiles && !*abort; tile += gridDim.x) {
-                const int m_blk = tile % num_m, n_blk = tile / num_m;
+                int m_blk, n_blk;
+                tile_coords(tile, num_m, num_n, &m_blk, &n_blk);
                 for (int kb = 0; kb < nk; ++kb, ++it) {
                     const int st = it % STAGES;
                     const uint32_t ph = (it / STAGES) & 1;
-                    if (!tc::mbar_wait(&s.empty[st], ph ^ 1, abort)) { fail(abort, status, 0, kb, 1); break; }
+                    if (!tc::mbar_wait(&s.empty[st], ph ^ 1, abort, wlim)) { fail(abort, status, 0, kb, 1); break; }
                     tc::mbar_arrive_expect_tx(&s.full[st], (BM + BN) * BK * 2);
                     if (m_blk < num_m0) tc::tma_load_2d(s.a[st], &tmA0, &s.full[st], kb * BK, m_blk * BM);
                     else tc::tma_load_2d(s.a[st], &tmA, &s.full[st], kb * BK, (m_blk - num_m0) * BM);
@@ -174,14 +191,14 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
             for (int tile = blockIdx.x; tile < num_tiles && !*abort; tile += gridDim.x, ++tcount) {
                 const int buf = tcount & 1;
                 const uint32_t tph = (tcount >> 1) & 1;
-                if (!tc::mbar_wait(&s.tempty[buf], tph ^ 1, abort)) { fail(abort, status, 1, tcount, 4); break; }
+                if (!tc::mbar_wait(&s.tempty[buf], tph ^ 1, abort, wlim)) { fail(abort, status, 1, tcount, 4); break; }
                 tc::tc_fence_after();
                 const uint32_t d = tmem + buf * BN;
                 bool ok = true;
                 for (int kb = 0; kb < nk; ++kb, ++it) {
                     const int st = it % STAGES;
                     const uint32_t ph = (it / STAGES) & 1;
-                    if (!tc::mbar_wait(&s.full[st], ph, abort)) { fail(abort, status, 1, kb, 2); ok = false; break; }
+                    if (!tc::mbar_wait(&s.full[st], ph, abort, wlim)) { fail(abort, status, 1, kb, 2); ok = false; break; }
                     tc::tc_fence_after();
                     const uint32_t a0 = tc::smem_u32(s.a[st]), b0 = tc::smem_u32(s.b[st]);
 #pragma unroll
@@ -206,9 +223,10 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
             const int buf = tcount & 1;
             const uint32_t tph = (tcount >> 1) & 1;
             // tcgen05.ld is warp-collective: the whole warp decides together
-            if (!__all_sync(0xffffffffu, tc::mbar_wait(&s.tfull[buf], tph, abort))) { fail(abort, status, 2, tcount, 3); break; }
+            if (!__all_sync(0xffffffffu, tc::mbar_wait(&s.tfull[buf], tph, abort, wlim))) { fail(abort, status, 2, tcount, 3); break; }
             tc::tc_fence_after();
-            const int m_blk = tile % num_m, n_blk = tile / num_m;
+            int m_blk, n_blk;
+            tile_coords(tile, num_m, num_n, &m_blk, &n_blk);
             const int row = m_blk * BM + q * 32 + lane;
 #pragma unroll 1
             for (int j = 0; j < BN / 64; ++j) {
@@ -311,6 +329,7 @@ INST(f16, f16)
 INST(bf16, bf16)
 INST(bf16, float)
 INST(f16, float)
+INST(f16, bf16)
 #undef INST
 
 }  // namespace hymba

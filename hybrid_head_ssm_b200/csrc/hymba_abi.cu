@@ -19,8 +19,9 @@ namespace hymba {
 // device status word (one per device that loads the library)
 // ---------------------------------------------------------------------------
 // [0]: status code; [1..7]: where the first timed-out wait gave up (flag, block
-// x, y, z, role, step, barrier), for diagnosis.
-__device__ int g_status_word[8];
+// x, y, z, role, step, barrier), for diagnosis; [8..9]: the limit in cycles of the
+// kernels' progress waits (0: the default), set by hymba_debug_set_wait_limit.
+__device__ __align__(8) int g_status_word[10];
 
 static std::mutex g_mu;
 // Per device: the status word's device address and the SM count, published together.
@@ -125,9 +126,18 @@ static int check_cfg(const hymba_layer_cfg* c) {
     if (c->head_dim != 64 || c->d_state != 16 || c->d_conv != 4) return HYMBA_ERR_UNSUPPORTED;
     if (c->n_q_heads % c->n_kv_heads) return HYMBA_ERR_UNSUPPORTED;
     if (c->n_q_heads / c->n_kv_heads > 8) return HYMBA_ERR_UNSUPPORTED;
-    if (c->v_head_dim * c->n_q_heads != c->d_inner || c->v_head_dim != 128) return HYMBA_ERR_UNSUPPORTED;
-    if (c->d_model % 64 || c->d_inner % 64) return HYMBA_ERR_UNSUPPORTED;
+    if (c->fusion != HYMBA_FUSION_AVERAGE && c->fusion != HYMBA_FUSION_CONCAT) return HYMBA_ERR_INVALID_ARG;
+    if (c->v_head_dim != 128 && c->v_head_dim != 64) return HYMBA_ERR_UNSUPPORTED;
+    const int hv = c->v_head_dim * c->n_q_heads;
+    if (c->fusion == HYMBA_FUSION_AVERAGE && hv != c->d_inner) return HYMBA_ERR_UNSUPPORTED;
+    if (c->d_model % 64 || c->d_inner % 64 || hv % 64) return HYMBA_ERR_UNSUPPORTED;
+    if (c->d_inner > 4096 || hv > 4096) return HYMBA_ERR_UNSUPPORTED;
     return HYMBA_OK;
+}
+
+// Width of the fused branches, the input of W_o.
+static int u_width(const hymba_layer_cfg* c) {
+    return c->fusion == HYMBA_FUSION_CONCAT ? c->d_inner + c->n_q_heads * c->v_head_dim : c->d_inner;
 }
 
 struct Cols {
@@ -180,15 +190,18 @@ static Plan plan(const hymba_layer_cfg* c, int B, int T, int mode) {
     p.delta = take(&cur, rows * di * sizeof(float));
     p.O = take(&cur, rows * (size_t)c->n_q_heads * c->v_head_dim * esz);
     p.ypre = take(&cur, rows * di * esz);
-    p.U = take(&cur, rows * di * esz);
+    p.U = take(&cur, rows * u_width(c) * esz);
     p.wdt = take(&cur, (size_t)di * p.rpad * esz);
     if (c->dtype == HYMBA_BF16) {
         p.xcv = take(&cur, rows * c->d_model * 2);  // 16-bit copy of an fp32 input
         if (mode == HYMBA_MODE_PREFILL) {
-            // fp16 copies of the projection weights for fp32-stream calls
+            // fp16 copies of the projection weights for fp32-stream calls (and of W_out
+            // for the concat fusion)
             p.win16 = take(&cur, (size_t)k.n_in * c->d_model * 2);
             p.meta16 = take(&cur, (size_t)c->n_meta * c->d_model * 2);
-            p.wout16 = take(&cur, (size_t)c->d_model * di * 2);
+            p.wout16 = take(&cur, (size_t)c->d_model * u_width(c) * 2);
+        } else if (c->fusion == HYMBA_FUSION_CONCAT) {
+            p.wout16 = take(&cur, (size_t)c->d_model * u_width(c) * 2);
         }
     }
     if (mode == HYMBA_MODE_DECODE) {
@@ -261,7 +274,7 @@ static int prefill_impl(const Ctx& ctx, const hymba_layer_cfg* c, const hymba_la
     using TA = typename std::conditional<kF16Ops, f16, T>::type;
     const Plan pl = plan(c, B, T_, HYMBA_MODE_PREFILL);
     const Cols k = columns(c);
-    const int m = c->n_meta, Tp = m + T_, d = c->d_model, di = c->d_inner;
+    const int m = c->n_meta, Tp = m + T_, d = c->d_model, di = c->d_inner, uw = u_width(c);
     const int H = c->n_q_heads, G = c->n_kv_heads, dh = c->head_dim, dv = c->v_head_dim;
     const long long rows = (long long)B * Tp;
     const bool has_meta = flags & HYMBA_X_HAS_META;
@@ -287,7 +300,7 @@ static int prefill_impl(const Ctx& ctx, const hymba_layer_cfg* c, const hymba_la
         if ((rc = launch_pad_copy<T, TA>(ctx, static_cast<const T*>(w->w_in), k.n_in, d, wi, d))) return rc;
         if (m > 0 && !has_meta && (rc = launch_pad_copy<T, TA>(ctx, static_cast<const T*>(w->meta), m, d, mt, d)))
             return rc;
-        if ((rc = launch_pad_copy<T, TA>(ctx, static_cast<const T*>(w->w_out), d, di, wo, di))) return rc;
+        if ((rc = launch_pad_copy<T, TA>(ctx, static_cast<const T*>(w->w_out), d, uw, wo, uw))) return rc;
         x = xc; W_in = wi; meta = mt; W_out = wo;
     } else {
         x = x_io;
@@ -335,24 +348,36 @@ static int prefill_impl(const Ctx& ctx, const hymba_layer_cfg* c, const hymba_la
             if ((rc = gemm<TA, I>(ctx, "gemm_in_proj", x, d, W_in, d, B * T_, k.n_in, d, ep))) return rc;
         }
     }
-    // 2. Delta = softplus(dt_low W_dt^T + b_dt) ------------------------------------
-    EpiArgs<I> ed = epi_base<I>(EPI_DELTA, (int)rows, di);
-    ed.delta = delta; ed.b_dt = w->b_dt;
-    if ((rc = gemm<I, I>(ctx, "gemm_dt_proj", P + k.dtl, pl.ldP, wdt, pl.rpad, (int)rows, di, c->dt_rank, ed))) return rc;
+    // 2. Delta = softplus(dt_low W_dt^T + b_dt), or inside the scan (step 4) when the
+    // batch is wide enough for the one-thread-per-channel scan ------------------------
+    const bool fold = std::is_same<I, f16>::value && scan_wide_applies(B, di, c->dt_rank, ctx.sm_count);
+    if (!fold) {
+        EpiArgs<I> ed = epi_base<I>(EPI_DELTA, (int)rows, di);
+        ed.delta = delta; ed.b_dt = w->b_dt;
+        if ((rc = gemm<I, I>(ctx, "gemm_dt_proj", P + k.dtl, pl.ldP, wdt, pl.rpad, (int)rows, di, c->dt_rank, ed)))
+            return rc;
+    }
     // 3. attention heads ---------------------------------------------------------
     if ((rc = attn_prefill<I>(ctx, P, pl.ldP, k_seq, v_seq, kv->seq_cap, O, B, Tp, H, G, dv, m, c->window)))
         return rc;
     // 4. Mamba heads ---------------------------------------------------------------
-    if ((rc = launch_conv_scan_prefill<I>(ctx, P, pl.ldP, k.x, k.Bc, k.Cc, delta, w->conv_w, w->conv_b,
-                                          w->A_log, w->D, ypre, st ? st->h : nullptr,
-                                          st ? st->conv : nullptr, B, Tp, di)))
+    bool scanned = false;
+    if constexpr (std::is_same<I, f16>::value) {
+        if (fold) {
+            if ((rc = launch_conv_scan_wide(ctx, P, pl.ldP, k.x, k.Bc, k.dtl, c->dt_rank, wdt, pl.rpad, w->b_dt,
+                                            w->conv_w, w->conv_b, w->A_log, w->D, ypre, st ? st->h : nullptr,
+                                            st ? st->conv : nullptr, B, Tp, di)))
+                return rc;
+            scanned = true;
+        }
+    }
+    if (!scanned && (rc = launch_conv_scan_prefill<I>(ctx, P, pl.ldP, k.x, k.Bc, k.Cc, delta, w->conv_w, w->conv_b,
+                                                      w->A_log, w->D, ypre, st ? st->h : nullptr,
+                                                      st ? st->conv : nullptr, B, Tp, di)))
         return rc;
-    // 5. gate, norms, beta, average --------------------------------------------------
-    if ((rc = launch_fuse<I, TA>(ctx, O, nullptr, 0, H, G, ypre, P, pl.ldP, k.z, w->norm_attn_w, w->norm_ssm_w,
-                                 w->beta1, w->beta2, vscale(c, w), vbias(c, w), U, (int)rows, di, c->rms_eps,
-                                 nullptr)))
-        return rc;
+    // 5. gate, norms, beta, average (or concatenation) ----------------------------------
     // 6. output projection (+ residual) -------------------------------------------------
+    const bool concat = c->fusion == HYMBA_FUSION_CONCAT;
     EpiArgs<TIO> eo = epi_base<TIO>(EPI_OUT, (int)rows, d);
     eo.y = y; eo.B = B; eo.Tu = T_; eo.Tp = Tp; eo.n_meta = m;
     if (flags & HYMBA_ADD_RESIDUAL) {
@@ -361,7 +386,29 @@ static int prefill_impl(const Ctx& ctx, const hymba_layer_cfg* c, const hymba_la
         eo.res_meta = w->meta;
         eo.res_meta_bf16 = std::is_same<T, bf16>::value;
     }
-    if ((rc = gemm<TA, TIO>(ctx, "gemm_out_proj", U, di, W_out, di, (int)rows, d, di, eo))) return rc;
+    bool projected = false;
+    if constexpr (std::is_same<TA, bf16>::value) {
+        if (concat) {
+            // the concatenated branches are not halved, so U is twice as large as the
+            // average's: U and W_out go to the tensor cores in fp16 (8x finer than bf16)
+            f16* U16 = reinterpret_cast<f16*>(ws + pl.U);
+            f16* wo16 = reinterpret_cast<f16*>(ws + pl.wout16);
+            if ((rc = launch_pad_copy<T, f16>(ctx, static_cast<const T*>(w->w_out), d, uw, wo16, uw))) return rc;
+            if ((rc = launch_fuse<I, f16>(ctx, O, nullptr, 0, H, G, dv, true, ypre, P, pl.ldP, k.z, w->norm_attn_w,
+                                          w->norm_ssm_w, w->beta1, w->beta2, vscale(c, w), vbias(c, w), U16,
+                                          (int)rows, di, c->rms_eps, nullptr)))
+                return rc;
+            if ((rc = gemm<f16, TIO>(ctx, "gemm_out_proj", U16, uw, wo16, uw, (int)rows, d, uw, eo))) return rc;
+            projected = true;
+        }
+    }
+    if (!projected) {
+        if ((rc = launch_fuse<I, TA>(ctx, O, nullptr, 0, H, G, dv, concat, ypre, P, pl.ldP, k.z, w->norm_attn_w,
+                                     w->norm_ssm_w, w->beta1, w->beta2, vscale(c, w), vbias(c, w), U, (int)rows, di,
+                                     c->rms_eps, nullptr)))
+            return rc;
+        if ((rc = gemm<TA, TIO>(ctx, "gemm_out_proj", U, uw, W_out, uw, (int)rows, d, uw, eo))) return rc;
+    }
     // 7. decode cache of a producer ------------------------------------------------------
     if (c->is_kv_producer && kv->k_cache) {
         if ((rc = launch_cache_fill<I>(ctx, k_seq, v_seq, kv->seq_cap, static_cast<I*>(kv->k_cache),
@@ -377,7 +424,7 @@ static int decode_impl(const Ctx& ctx, const hymba_layer_cfg* c, const hymba_lay
                        char* ws) {
     const Plan pl = plan(c, B, kv->cache_cap, HYMBA_MODE_DECODE);
     const Cols k = columns(c);
-    const int m = c->n_meta, d = c->d_model, di = c->d_inner;
+    const int m = c->n_meta, d = c->d_model, di = c->d_inner, uw = u_width(c);
     const int H = c->n_q_heads, G = c->n_kv_heads, dh = c->head_dim, dv = c->v_head_dim;
     const int pos_offset = c->is_kv_producer ? 0 : -1;
     I* P = reinterpret_cast<I*>(ws + pl.P);
@@ -424,14 +471,30 @@ static int decode_impl(const Ctx& ctx, const hymba_layer_cfg* c, const hymba_lay
                                       w->b_dt, c->dt_rank, w->conv_w, w->conv_b, w->A_log, w->D, st->h,
                                       st->conv, ypre, B, di)))
         return rc;
-    if ((rc = launch_fuse<I, T>(ctx, nullptr, part, pl.n_split, H, G, ypre, P, pl.ldP, k.z, w->norm_attn_w,
-                                w->norm_ssm_w, w->beta1, w->beta2, vscale(c, w), vbias(c, w), U, B, di,
-                                c->rms_eps, c->is_kv_producer ? kv->len : nullptr)))
-        return rc;
+    const bool concat = c->fusion == HYMBA_FUSION_CONCAT;
     EpiArgs<TIO> eo = epi_base<TIO>(EPI_OUT, B, d);
     eo.y = y;
     if (flags & HYMBA_ADD_RESIDUAL) { eo.res_mode = 1; eo.res_x = x_io; }
-    if ((rc = gemm<T, TIO>(ctx, "gemm_out_proj_decode", U, di, static_cast<const T*>(w->w_out), di, B, d, di, eo))) return rc;
+    if constexpr (std::is_same<T, bf16>::value) {
+        if (concat) {
+            // as in the prefill: the concatenation's U and W_out in fp16
+            f16* U16 = reinterpret_cast<f16*>(ws + pl.U);
+            f16* wo16 = reinterpret_cast<f16*>(ws + pl.wout16);
+            if ((rc = launch_pad_copy<T, f16>(ctx, static_cast<const T*>(w->w_out), d, uw, wo16, uw))) return rc;
+            if ((rc = launch_fuse<I, f16>(ctx, nullptr, part, pl.n_split, H, G, dv, true, ypre, P, pl.ldP, k.z,
+                                          w->norm_attn_w, w->norm_ssm_w, w->beta1, w->beta2, vscale(c, w),
+                                          vbias(c, w), U16, B, di, c->rms_eps,
+                                          c->is_kv_producer ? kv->len : nullptr)))
+                return rc;
+            return gemm<f16, TIO>(ctx, "gemm_out_proj_decode", U16, uw, wo16, uw, B, d, uw, eo);
+        }
+    }
+    if ((rc = launch_fuse<I, T>(ctx, nullptr, part, pl.n_split, H, G, dv, concat, ypre, P, pl.ldP, k.z,
+                                w->norm_attn_w, w->norm_ssm_w, w->beta1, w->beta2, vscale(c, w), vbias(c, w), U, B,
+                                di, c->rms_eps, c->is_kv_producer ? kv->len : nullptr)))
+        return rc;
+    if ((rc = gemm<T, TIO>(ctx, "gemm_out_proj_decode", U, uw, static_cast<const T*>(w->w_out), uw, B, d, uw, eo)))
+        return rc;
     return HYMBA_OK;
 }
 
@@ -612,6 +675,16 @@ int hymba_get_device_diag(int32_t* out, int n) {
     const int zero[7] = {0};
     if (cudaMemcpy(ctx.status + 1, zero, sizeof(zero), cudaMemcpyHostToDevice) != cudaSuccess) return HYMBA_ERR_CUDA;
     for (int i = 0; i < 7; ++i) out[i] = v[i];
+    return HYMBA_OK;
+}
+
+int hymba_debug_set_wait_limit(long long cycles) {
+    if (cycles < 0) return HYMBA_ERR_INVALID_ARG;
+    Ctx ctx;
+    if (current_ctx(nullptr, &ctx)) return HYMBA_ERR_CUDA;
+    if (cudaDeviceSynchronize() != cudaSuccess) return HYMBA_ERR_CUDA;
+    if (cudaMemcpy(ctx.status + 8, &cycles, sizeof(cycles), cudaMemcpyHostToDevice) != cudaSuccess)
+        return HYMBA_ERR_CUDA;
     return HYMBA_OK;
 }
 

@@ -33,21 +33,32 @@ int launch_attn_prefill_tc(const Ctx& ctx, const f16* P, long long ldP, const f1
                            const f16* v_seq, int kcap, f16* O, int B, int Tp, int H, int G,
                            int dv, int n_meta, int window);
 
-// Depthwise causal conv + SiLU + selective scan over the T' rows of every sequence.
+// Depthwise causal conv + SiLU + selective scan over the T' rows of every sequence,
+// Delta from `delta` [rows, di] fp32.
 template <typename T>
 int launch_conv_scan_prefill(const Ctx& ctx, const T* P, long long ldP, int col_x, int col_B,
                              int col_C, const float* delta, const float* conv_w,
                              const float* conv_b, const float* A_log, const float* D, T* ypre,
                              float* h_out, float* conv_out, int B, int Tp, int di);
 
-// RMSNorm of both branches, SiLU(z) gate, beta scaling and average; one row per block.
-// The attention branch is O [rows, di], or, when `part` is given, the decode
-// attention's split partials [rows, H, n_split, di/H + 2] merged on the fly (O unused).
+// The same for 16-bit intermediates with Delta computed in the kernel (dt_rank <= 128, a
+// multiple of 4), one thread per channel pair and state half: for batches where
+// B * d_inner fills the GPU (scan_wide_applies).
+bool scan_wide_applies(int B, int di, int dt_rank, int sm_count);
+int launch_conv_scan_wide(const Ctx& ctx, const f16* P, long long ldP, int col_x, int col_B, int col_dt, int dt_rank,
+                          const f16* wdt, int ld_wdt, const float* b_dt, const float* conv_w, const float* conv_b,
+                          const float* A_log, const float* D, f16* ypre, float* h_out, float* conv_out, int B, int Tp,
+                          int di);
+
+// RMSNorm of both branches, SiLU(z) gate, beta scaling and average (U [rows, di]) or
+// concatenation (U [rows, di + H*dv] = [Mamba | attention]); one row per block.
+// The attention branch is O [rows, H*dv], or, when `part` is given, the decode
+// attention's split partials [rows, H, n_split, dv + 2] merged on the fly (O unused).
 // A consumer's adapted shared V (v_scale, v_bias [G, dv], both or neither) is applied
 // to the attention output before its norm.
 template <typename I, typename T>
-int launch_fuse(const Ctx& ctx, const I* O, const float* part, int n_split, int H, int G, const I* ypre,
-                const I* P, long long ldP, int col_z, const float* g_attn, const float* g_ssm,
+int launch_fuse(const Ctx& ctx, const I* O, const float* part, int n_split, int H, int G, int dv, bool concat,
+                const I* ypre, const I* P, long long ldP, int col_z, const float* g_attn, const float* g_ssm,
                 const float* beta1, const float* beta2, const float* v_scale, const float* v_bias, T* U,
                 int rows, int di, float eps, int* len_inc);
 

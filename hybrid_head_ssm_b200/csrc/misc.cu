@@ -1,7 +1,11 @@
 // Small data-movement kernels around the mixer: the RoPE angle table with the padded
 // W_dt copy of a prefill, zero-padded weight copies for TMA-aligned strides, and the
-// decode-cache fill after a prefill.
+// decode-cache fill after a prefill; and the stalled wait that exercises the failure
+// path of the bounded waits.
+#include <algorithm>
+
 #include "kernels.h"
+#include "tc.cuh"
 
 namespace hymba {
 
@@ -14,6 +18,49 @@ __global__ void pad_copy_kernel(const TS* src, int rows, int cols, TD* dst, int 
     if (idx >= (long long)rows * ld_dst) return;
     const int r = (int)(idx / ld_dst), c = (int)(idx % ld_dst);
     dst[idx] = from_f<TD>(c < cols ? to_f(src[(long long)r * cols + c]) : 0.f);
+}
+
+// Eight elements of a row as fp32 (one or two 16-byte loads).
+template <typename TS>
+__device__ __forceinline__ void load8_any(const TS* p, float* v) {
+    if constexpr (sizeof(TS) == 4) {
+        const float4 a = __ldg(reinterpret_cast<const float4*>(p));
+        const float4 b = __ldg(reinterpret_cast<const float4*>(p) + 1);
+        v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+        v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+    } else {
+        const uint4 u = __ldg(reinterpret_cast<const uint4*>(p));
+        const TS* h = reinterpret_cast<const TS*>(&u);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) v[i] = to_f(h[i]);
+    }
+}
+
+// The same copy, eight elements per thread and iteration with 16-byte accesses (cols and
+// ld_dst multiples of 8, both rows 16-byte aligned), grid-stride over the 8-element
+// pieces of the destination. HBM-bound: it moves (sizeof(TS) + 2) bytes per element.
+template <typename TS, typename TD>
+__global__ void __launch_bounds__(256) pad_copy8_kernel(const TS* __restrict__ src, int rows, int cols,
+                                                        TD* __restrict__ dst, int ld_dst) {
+    griddep_sync();
+    const int per_row = ld_dst / 8;
+    const long long n = (long long)rows * per_row;
+    for (long long v = (long long)blockIdx.x * blockDim.x + threadIdx.x; v < n; v += (long long)gridDim.x * blockDim.x) {
+        const int r = (int)(v / per_row), c = (int)(v - (long long)r * per_row) * 8;
+        float x[8];
+        if (c < cols) {
+            load8_any<TS>(src + (long long)r * cols + c, x);
+        } else {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) x[i] = 0.f;
+        }
+        uint4 o;
+        o.x = pack2<TD>(x[0], x[1]);
+        o.y = pack2<TD>(x[2], x[3]);
+        o.z = pack2<TD>(x[4], x[5]);
+        o.w = pack2<TD>(x[6], x[7]);
+        *reinterpret_cast<uint4*>(dst + (long long)r * ld_dst + c) = o;
+    }
 }
 
 // The two small inputs of a prefill in one launch: blocks [0, nb_rope) fill the RoPE
@@ -85,6 +132,15 @@ __global__ void cache_fill_kernel(const T* k_seq, const T* v_seq, int seq_cap, T
 template <typename TS, typename TD>
 int launch_pad_copy(const Ctx& ctx, const TS* src, int rows, int cols, TD* dst, int ld_dst) {
     const long long n = (long long)rows * ld_dst;
+    if constexpr (sizeof(TD) == 2) {
+        if (cols % 8 == 0 && ld_dst % 8 == 0 && ((reinterpret_cast<uintptr_t>(src) | reinterpret_cast<uintptr_t>(dst)) & 15) == 0) {
+            auto kern = pad_copy8_kernel<TS, TD>;
+            const long long pieces = n / 8;
+            const int grid = (int)std::min<long long>(ceil_div(pieces, 256), (long long)ctx.sm_count * 8);
+            HYMBA_LAUNCH(ctx, "pad_copy", kern, grid, 256, 0, src, rows, cols, dst, ld_dst);
+            return HYMBA_OK;
+        }
+    }
     auto kern = pad_copy_kernel<TS, TD>;
     HYMBA_LAUNCH(ctx, "pad_copy", kern, ceil_div(n, 256), 256, 0, src, rows, cols, dst, ld_dst);
     return HYMBA_OK;
@@ -141,3 +197,33 @@ template int launch_cache_fill<f16>(const Ctx&, const f16*, const f16*, int, f16
                                     int*, int, int, int, int, int, int);
 
 }  // namespace hymba
+
+namespace hymba {
+namespace {
+
+// One thread waits on an mbarrier that nothing arrives on, with the progress-wait limit
+// the tensor-core kernels use: the wait runs out and records HYMBA_ERR_DEVICE_TIMEOUT
+// (role 4) the way theirs do, and the block returns with nothing in flight.
+__global__ void stalled_wait_kernel(int* status) {
+    __shared__ uint64_t bar;
+    if (threadIdx.x == 0) {
+        tc::mbar_init(&bar, 1);
+        tc::fence_mbar_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        int zero = 0;
+        if (!tc::mbar_wait(&bar, 0, &zero, tc::wait_limit(status))) tc::record_timeout(status, 4, 0, 0);
+    }
+}
+
+}  // namespace
+}  // namespace hymba
+
+extern "C" int hymba_debug_stalled_wait(void* stream) {
+    hymba::Ctx ctx;
+    int rc = hymba::launch_context(static_cast<cudaStream_t>(stream), &ctx);
+    if (rc) return rc;
+    HYMBA_LAUNCH(ctx, "stalled_wait", hymba::stalled_wait_kernel, 1, 32, 0, ctx.status);
+    return HYMBA_OK;
+}

@@ -93,9 +93,19 @@ __device__ __forceinline__ void record_timeout(int* status, int role, int step, 
     }
 }
 
-// Bounded wait on an mbarrier phase. Returns false on timeout or when another role
-// of the block already aborted (*abort != 0).
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
+// The limit of the waits that wait for progress (not of the drains before exit): words
+// 8-9 of the device status word, set by hymba_debug_set_wait_limit; 0 means the default.
+__device__ __forceinline__ long long wait_limit(const int* status) {
+    if (!status) return kWaitLimitCycles;
+    const long long v = *reinterpret_cast<const volatile long long*>(status + 8);
+    return v > 0 ? v : kWaitLimitCycles;
+}
+
+// Bounded wait on an mbarrier phase. Returns false after `limit` cycles or when another
+// role of the block already aborted (*abort != 0). The drains a block runs before it
+// exits (copies and MMAs it issued) keep the default limit.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                          long long limit = kWaitLimitCycles) {
     long long t0 = 0;
     for (uint32_t i = 0;; ++i) {
         if (mbar_try_wait(bar, parity)) return true;
@@ -103,7 +113,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
             if (*abort) return false;
             const long long now = clock64();
             if (t0 == 0) t0 = now;
-            else if (now - t0 > kWaitLimitCycles) return false;
+            else if (now - t0 > limit) return false;
         }
     }
 }

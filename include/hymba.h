@@ -77,15 +77,22 @@ extern "C" {
                                   between stacked layers (the projection operand X^ is
                                   rounded to bf16 inside; the residual add is fp32) */
 
+/* fusion of the two head families (hymba_layer_cfg.fusion) */
+#define HYMBA_FUSION_AVERAGE 0  /* U = (beta1 RMSNorm(O) + beta2 RMSNorm(Y)) / 2, d_inner wide */
+#define HYMBA_FUSION_CONCAT  1  /* U = [beta2 RMSNorm(Y) | beta1 RMSNorm(O)], d_inner + H*dv wide */
+
 /* workspace modes */
 #define HYMBA_MODE_PREFILL 0
 #define HYMBA_MODE_DECODE  1
 
-/* Shape and numerics of one mixer layer. The V head dim must equal
- * d_inner / n_q_heads so that the two branches can be averaged (the concat
- * formula of the Hymba Guide has no such constraint; averaging does).
- * Supported: head_dim == 64; v_head_dim % 64 == 0; n_q_heads % n_kv_heads == 0;
- * d_model, d_inner % 64 == 0; d_state == 16; d_conv == 4. */
+/* Shape and numerics of one mixer layer. With HYMBA_FUSION_AVERAGE the V head dim
+ * must equal d_inner / n_q_heads so that the two branches can be averaged; with
+ * HYMBA_FUSION_CONCAT ("Hymba Guide", Parallel Hybrid-Head Layer Formulation:
+ * y = W_o(Concat[MambaHeads(x), AttentionHeads(x)])) the branches are placed side by
+ * side, Mamba first, and W_o takes d_inner + n_q_heads * v_head_dim inputs.
+ * Supported: head_dim == 64; v_head_dim 64 or 128; n_q_heads % n_kv_heads == 0 with at
+ * most 8 query heads per KV head; d_model, d_inner and n_q_heads * v_head_dim multiples
+ * of 64, at most 4096; d_state == 16; d_conv == 4. */
 typedef struct hymba_layer_cfg {
     int32_t d_model;
     int32_t n_q_heads;
@@ -102,6 +109,7 @@ typedef struct hymba_layer_cfg {
     int32_t dtype;           /* HYMBA_F32 or HYMBA_BF16 */
     float   rope_base;
     float   rms_eps;
+    int32_t fusion;          /* HYMBA_FUSION_AVERAGE or HYMBA_FUSION_CONCAT */
 } hymba_layer_cfg;
 
 /* Weights of one layer (device pointers, caller-owned, read only). Big matrices
@@ -120,7 +128,7 @@ typedef struct hymba_layer_weights {
     const float* norm_ssm_w;  /* [d_inner]              RMSNorm gain of the SSM branch */
     const float* beta1;       /* [n_q_heads*v_head_dim] */
     const float* beta2;       /* [d_inner] */
-    const void*  w_out;       /* [d_model, d_inner]     dtype */
+    const void*  w_out;       /* [d_model, u] dtype: u = d_inner (average) or d_inner + n_q_heads*v_head_dim (concat) */
     const void*  meta;        /* [n_meta, d_model]      dtype */
     /* Consumer layers only (NULL for a producer, and NULL for plain sharing): the
      * head-specific affine adaptation of the shared K and V ("Hymba Guide",
@@ -191,8 +199,12 @@ int hymba_mixer_prefill(const hymba_layer_cfg* cfg, const hymba_layer_weights* w
                         hymba_kv* kv, hymba_ssm_state* st,
                         void* workspace, size_t ws_bytes, void* stream);
 
-/* One decode step: one new token per sequence, all B sequences at the same position
- * len[b] (producer) or len[b]-1 (consumer).
+/* One decode step: one new token per sequence; sequence b's token sits at position
+ * len[b] (producer) or len[b]-1 (consumer). The sequences of a batch may be at
+ * different positions: each keeps its own length, ring slot and state, so a batch of
+ * sequences of different lengths decodes together with no padding (the 51cto
+ * Hymba-1.5B article, section 4, notes that padded meta tokens and the sliding
+ * window kept the released code at batch 1 for generation).
  *   x_t: device [B, d_model]; y_t: device [B, d_model] (may equal x_t); fp32 with
  *   HYMBA_IO_F32, else dtype. Flags: HYMBA_ADD_RESIDUAL, HYMBA_IO_F32.
  *   kv must hold a decode cache (k_cache, len); st is updated in place. A cache
@@ -268,15 +280,29 @@ int hymba_get_device_status(void* stream);
 /* Where the first bounded device wait that ran out gave up (after a call reported
  * HYMBA_ERR_DEVICE_TIMEOUT): out[0] 1 if a record exists, out[1..3] the block index
  * (x, y, z), out[4] the role (0 TMA producer, 1 MMA issuer, 2 epilogue/softmax, 3 decode
- * attention waiting for its bulk copies), out[5] the step (k-block, key block or copy
- * tile), out[6] the barrier (or stage). Synchronises the device and
- * clears the record. Requires n >= 7. */
+ * attention waiting for its bulk copies, 4 hymba_debug_stalled_wait), out[5] the step
+ * (k-block, key block or copy tile), out[6] the barrier (or stage). Synchronises the
+ * device and clears the record. Requires n >= 7. */
 int hymba_get_device_diag(int32_t* out, int n);
+
+/* Failure-path testing. Every device wait of the library that waits for progress
+ * (an mbarrier phase a copy, an MMA or another role completes) gives up after a limit
+ * of SM clock cycles (default 2e8, about 0.1 s), records HYMBA_ERR_DEVICE_TIMEOUT and
+ * where it happened, and its block then waits (with the default limit) for the copies
+ * and MMAs it already issued before it exits, so the context stays usable.
+ * hymba_debug_set_wait_limit sets that limit for the current device (0 restores the
+ * default; synchronises the device first). hymba_debug_stalled_wait queues one block
+ * that waits, with that limit, on an mbarrier nothing arrives on: the wait runs out and
+ * the status word then reads HYMBA_ERR_DEVICE_TIMEOUT, role 4. */
+int hymba_debug_set_wait_limit(long long cycles);
+int hymba_debug_stalled_wait(void* stream);
 
 /* Layout of the workspace of one call, for callers that inspect the stage outputs
  * after a prefill (tests do): out[0] total bytes, out[1] byte offset of the
  * projection P [rows, ld_p] dtype (columns Q | (K V, unused) | x | z | B | C | dt_low),
- * out[2] ld_p in elements, out[3] offset of Delta [rows, d_inner] fp32, out[4] of the
+ * out[2] ld_p in elements, out[3] offset of Delta [rows, d_inner] fp32 (not written
+ * when a bf16 prefill computes Delta inside its scan kernel: dt_rank <= 128 and a
+ * multiple of 4, and B * d_inner / 64 at least twice the SM count), out[4] of the
  * attention output O [rows, n_q_heads*v_head_dim] dtype, out[5] of y_pre = C.h + D xc
  * [rows, d_inner] dtype (before the SiLU(z) gate), out[6] of the fused U [rows,
  * d_inner] dtype, out[7] of the RoPE table, out[8] of the decode split partials,
@@ -309,6 +335,15 @@ int hymba_trace_only(const char* name);
 
 /* Number of kernels the library has queued since load (all entry points). */
 uint64_t hymba_launch_count(void);
+
+/* Measurement: throughput of the units that bound the library's CUDA-core kernels on
+ * the current device, in results per clock per SM of the slowest SM (one 1024-thread
+ * block per SM, 8 independent dependency chains per thread, timed with clock64):
+ * out[0] exp2 in fp32 (ex2.approx.f32, the MUFU unit: the scan's state decays and the
+ * softmax's exponentials), out[1] exp2 on fp16 pairs (ex2.approx.f16x2, counted per
+ * half), out[2] fp32 FMA results of packed FFMA2 (two per instruction). Synchronises
+ * `stream`; uses a fixed device array of the library (no allocation). Requires n >= 3. */
+int hymba_probe_unit_rates(double* out, int n, void* stream);
 
 #ifdef __cplusplus
 }

@@ -77,10 +77,24 @@ def test_workspace_layout_is_consistent(hy):
 def test_invalid_configs_rejected(hy):
     base = synth.tiny_layer_cfg()
     for bad in (base.with_(head_dim=32), base.with_(d_state=8), base.with_(n_kv_heads=3),
-                base.with_(v_head_dim=64), base.with_(dtype=7), base.with_(d_model=0)):
+                base.with_(v_head_dim=64), base.with_(dtype=7), base.with_(d_model=0), base.with_(fusion=2),
+                base.with_(fusion=1, v_head_dim=96)):
         c = hy.cfg_struct(bad)
         assert hy.hymba_workspace_bytes(ctypes.byref(c), 1, 10, 0) == 0
         assert hy.hymba_cache_bytes(ctypes.byref(c), 1, 10) == 0
+
+
+def test_concat_fusion_workspace_holds_the_wider_u(hy):
+    """The concat fusion's U is d_inner + H * dv wide (the input of W_o); its 64-wide V
+    heads need not add up to d_inner."""
+    cat = synth.hymba15_layer_cfg(1024).with_(fusion=1, v_head_dim=64)
+    lc = hy.workspace_layout(hy.cfg_struct(cat), 2, 100, hy.HYMBA_MODE_PREFILL)
+    rows = 2 * (cat.n_meta + 100)
+    assert cat.u_width == 3200 + 25 * 64
+    order = sorted((lc[k], k) for k in ("P", "delta", "O", "ypre", "U", "rope"))
+    nxt = {k: order[i + 1][0] for i, (_, k) in enumerate(order[:-1])}
+    assert lc["total"] - lc["U"] >= rows * cat.u_width * 2  # U is the last of the exposed blocks
+    assert nxt["O"] - lc["O"] >= rows * 25 * 64 * 2
 
 
 def test_prefill_argument_errors_before_any_launch(hy):
@@ -97,7 +111,7 @@ def test_prefill_argument_errors_before_any_launch(hy):
     assert rc == hy.HYMBA_ERR_UNSUPPORTED
     # all pointers "present" (fake host addresses, never dereferenced) but workspace too small
     fake = 1 << 20
-    wf = hy.hymba_layer_weights(*([fake] * 13))
+    wf = hy.hymba_layer_weights(*([fake] * 13))  # no affine shared-KV vectors
     kvf = hy.kv_struct(cfg, 1)
     kvf.k_seq = kvf.v_seq = fake
     kvf.seq_cap = cfg.n_meta + 10

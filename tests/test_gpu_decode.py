@@ -232,3 +232,102 @@ def test_pair_decode_with_affine_shared_kv(dtype):
         rb = oracle.mixer_decode(cb, wb, ra, o["cache"], o["hb"], o["cb"], residual=True)
         assert_close(to_np(yb), rb, cb, f"consumer step {t}")
     assert g.hy.hymba_get_device_status(None) == 0
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_ragged_decode_batch(dtype):
+    """One decode batch whose sequences sit at different positions (prompts of 5, 13 and
+    22 tokens prefilled one by one into their slices of the shared cache and state; the
+    8-slot rings at different phases of their wrap): each sequence's outputs match the
+    oracle's decode of that sequence, with no padding."""
+    torch = torch_cuda()
+    import hybrid_head_ssm_b200 as hy
+    from hybrid_head_ssm_b200 import runtime as rt
+    if dtype == "f32":
+        base = synth.tiny_layer_cfg().with_(window=8)
+    else:
+        base = synth.hymba15_layer_cfg(window=8).with_(d_model=256, n_q_heads=5, n_kv_heads=1, d_inner=640,
+                                                       dt_rank=24, n_meta=8)
+    ca, cb = base, base.with_(is_kv_producer=0)
+    wa = synth.perturbed_weights(synth.layer_weights(ca, 93), ca, 93)
+    wb = synth.perturbed_weights(synth.layer_weights(cb, 94), cb, 94)
+    lens, steps = (5, 13, 22), 9
+    B, m, cap = len(lens), ca.n_meta, ca.n_meta + 8
+    x = synth.layer_input(ca, B, max(lens) + steps, 95)
+    la, lb = rt.DeviceLayer(ca, wa), rt.DeviceLayer(cb, wb)
+    fl = rt.stream_flags(ca)
+    io = torch.float32 if (fl & hy.HYMBA_IO_F32 or ca.dtype == 0) else rt.act_dtype(ca)
+    kv = rt.KV(ca, B, cache_cap=cap)
+    sa, sb = rt.State(ca, B), rt.State(cb, B)
+    caches, hs = [], []
+    for b, T0 in enumerate(lens):
+        # sequence b alone (B = 1) into its slice of the batch's cache and state
+        Tp = m + T0
+        kseq = torch.empty((1, ca.n_kv_heads, Tp, ca.head_dim), dtype=rt.mid_dtype(ca), device="cuda")
+        vseq = torch.empty((1, ca.n_kv_heads, Tp, ca.v_head_dim), dtype=rt.mid_dtype(ca), device="cuda")
+        kvs = hy.kv_struct(ca, 1, kseq, vseq, kv.k_cache[b:b + 1], kv.v_cache[b:b + 1], kv.len[b:b + 1])
+        kvc = hy.hymba_kv()
+        hy.check(hy.hymba_kv_share(ctypes.byref(kvs), ctypes.byref(lb.c), ctypes.byref(kvc)))
+        xb = rt.to_device(x[b:b + 1, :T0], ca, io_f32=io == torch.float32)
+        ya = torch.empty((1, Tp, ca.d_model), dtype=io, device="cuda")
+        yb = torch.empty_like(ya)
+        ws = rt.workspace(ca, 1, T0, hy.HYMBA_MODE_PREFILL)
+        sta = hy.state_struct(sa.h[b:b + 1], sa.conv[b:b + 1])
+        stb = hy.state_struct(sb.h[b:b + 1], sb.conv[b:b + 1])
+        hy.check(hy.hymba_mixer_prefill(ctypes.byref(la.c), ctypes.byref(la.s), xb.data_ptr(), 1, T0, fl,
+                                        ya.data_ptr(), ctypes.byref(kvs), ctypes.byref(sta), ws.data_ptr(),
+                                        ws.numel(), hy.current_stream_ptr()))
+        hy.check(hy.hymba_mixer_prefill(ctypes.byref(lb.c), ctypes.byref(lb.s), ya.data_ptr(), 1, T0,
+                                        fl | hy.HYMBA_X_HAS_META, yb.data_ptr(), ctypes.byref(kvc),
+                                        ctypes.byref(stb), ws.data_ptr(), ws.numel(), hy.current_stream_ptr()))
+        pa = oracle.mixer_prefill(ca, wa, x[b:b + 1, :T0], residual=True)
+        pb = oracle.mixer_prefill(cb, wb, pa["y"], kv_shared=(pa["k"], pa["v"]), residual=True, x_has_meta=True)
+        caches.append(oracle.cache_from_prefill(ca, pa["k"], pa["v"], cap))
+        hs.append((pa["h"], pa["conv"], pb["h"], pb["conv"]))
+    torch.cuda.synchronize()
+    assert kv.len.cpu().tolist() == [m + T0 for T0 in lens]
+    cache = {k: np.concatenate([c[k] for c in caches]) for k in ("k", "v", "len")}
+    ha, conva, hb, convb = (np.concatenate([h[i] for h in hs]) for i in range(4))
+    kvb = hy.hymba_kv()
+    hy.check(hy.hymba_kv_share(ctypes.byref(kv.s), ctypes.byref(lb.c), ctypes.byref(kvb)))
+    wda = rt.workspace(ca, B, cap, hy.HYMBA_MODE_DECODE)
+    wdb = rt.workspace(cb, B, cap, hy.HYMBA_MODE_DECODE)
+    for s in range(steps):
+        xt_np = np.stack([x[b, lens[b] + s] for b in range(B)])
+        xt = rt.to_device(xt_np, ca, io_f32=io == torch.float32)
+        ya, yb = torch.empty_like(xt), torch.empty_like(xt)
+        rt.decode(la, xt, kv.s, sa, ya, wda, fl)
+        rt.decode(lb, ya, kvb, sb, yb, wdb, fl)
+        ra = oracle.mixer_decode(ca, wa, xt_np, cache, ha, conva, residual=True)
+        rb = oracle.mixer_decode(cb, wb, ra, cache, hb, convb, residual=True)
+        assert_close(to_np(yb), rb, cb, f"ragged batch, step {s}")
+    assert kv.len.cpu().tolist() == [m + T0 + steps for T0 in lens]
+    assert hy.hymba_get_device_status(None) == 0
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_pair_decode_with_concat_fusion(dtype):
+    """Decode through a KV-sharing pair with the concat fusion and 64-wide V heads: the
+    decode attention's 64-wide partials, their merge and the wider W_o."""
+    if dtype == "f32":
+        base = synth.tiny_layer_cfg().with_(window=8, fusion=1, v_head_dim=64)
+        B, T0, steps, seed = 2, 10, 10, 121
+    else:
+        base = synth.hymba15_layer_cfg(window=24).with_(d_model=256, n_q_heads=5, n_kv_heads=1, d_inner=640,
+                                                        dt_rank=24, n_meta=8, fusion=1, v_head_dim=64)
+        B, T0, steps, seed = 3, 30, 10, 122
+    ca, cb = base, base.with_(is_kv_producer=0)
+    wa = synth.perturbed_weights(synth.layer_weights(ca, seed), ca, seed)
+    wb = synth.perturbed_weights(synth.layer_weights(cb, seed + 1), cb, seed + 1)
+    x = synth.layer_input(ca, B, T0 + steps, seed + 2)
+    cap = ca.n_meta + ca.window
+    g = _Pair(ca, cb, wa, wb, B, T0, cap)
+    g.prefill(x[:, :T0])
+    o = _oracle_pair(ca, cb, wa, wb, x[:, :T0], cap)
+    for t in range(T0, T0 + steps):
+        ya, yb = g.step(x[:, t])
+        ra = oracle.mixer_decode(ca, wa, x[:, t], o["cache"], o["ha"], o["ca"], residual=True)
+        rb = oracle.mixer_decode(cb, wb, ra, o["cache"], o["hb"], o["cb"], residual=True)
+        assert_close(to_np(ya), ra, ca, f"producer step {t}")
+        assert_close(to_np(yb), rb, cb, f"consumer step {t}")
+    assert g.hy.hymba_get_device_status(None) == 0

@@ -47,13 +47,14 @@ def _ws_view(ws, off, shape, dtype):
     return ws[off:off + n * esz].view(dtype).view(*shape)
 
 
-def _check_stages(cfg, r, ref, B, Tp):
+def _check_stages(cfg, r, ref, B, Tp, delta_written=True):
     import torch
     from hybrid_head_ssm_b200 import runtime as rt
     lay, ws = r["lay"], r["ws"]
     mdt = rt.mid_dtype(cfg)
     di, H, dv = cfg.d_inner, cfg.n_q_heads, cfg.v_head_dim
-    delta = to_np(_ws_view(ws, lay["delta"], (B, Tp, di), torch.float32))
+    # a wide bf16 batch computes Delta inside the scan kernel (no Delta tensor)
+    delta = to_np(_ws_view(ws, lay["delta"], (B, Tp, di), torch.float32)) if delta_written else None
     o = to_np(_ws_view(ws, lay["O"], (B, Tp, H * dv), mdt))
     u = to_np(_ws_view(ws, lay["U"], (B, Tp, di), rt.act_dtype(cfg)))
     ypre = to_np(_ws_view(ws, lay["ypre"], (B, Tp, di), mdt))
@@ -61,7 +62,8 @@ def _check_stages(cfg, r, ref, B, Tp):
     zc = cfg.n_q_heads * cfg.head_dim + (cfg.n_kv_heads * (cfg.head_dim + cfg.v_head_dim) if cfg.is_kv_producer else 0) + di
     z = P[:, :, zc:zc + di]
     tol = dict(max_abs=1e-4 if cfg.dtype == 0 else 6e-2, rel_l2=5e-3)
-    assert_close(delta, ref["delta"], cfg, "Delta", max_abs=tol["max_abs"])
+    if delta is not None:
+        assert_close(delta, ref["delta"], cfg, "Delta", max_abs=tol["max_abs"])
     assert_close(ypre * oracle.silu(z), ref["y_ssm"], cfg, "gated SSM output", max_abs=1e-4 if cfg.dtype == 0 else 2.5e-1,
                  rel_l2=5e-3)
     assert_close(o, ref["o_attn"], cfg, "attention output", **tol)
@@ -240,3 +242,55 @@ def test_consumer_with_affine_shared_kv(dtype):
     with pytest.raises(Exception):
         # a producer may not carry the adaptation
         _run_prefill(cp, dict(wp, **synth.affine_kv(cp, 45)), x)
+
+
+@pytest.mark.parametrize("case", ["f32_tiny", "bf16_small", "bf16_hymba15"])
+def test_concat_fusion_layer(case):
+    """The concat fusion ("Hymba Guide", Parallel Hybrid-Head Layer Formulation:
+    y = W_o(Concat[MambaHeads(x), AttentionHeads(x)])) with V head dim 64 = the Q/K
+    head dim: attention output H * 64 wide, U = [Mamba | attention], W_o over both."""
+    if case == "f32_tiny":
+        cfg = synth.tiny_layer_cfg().with_(fusion=1, v_head_dim=64, window=24)
+        B, T = 2, 90
+    elif case == "bf16_small":
+        cfg = synth.hymba15_layer_cfg(window=40).with_(d_model=256, n_q_heads=5, n_kv_heads=1, d_inner=640,
+                                                       dt_rank=24, n_meta=8, fusion=1, v_head_dim=64)
+        B, T = 2, 133
+    else:
+        cfg = synth.hymba15_layer_cfg(window=1024).with_(fusion=1, v_head_dim=64)
+        B, T = 1, 1500
+    w = synth.perturbed_weights(synth.layer_weights(cfg, 111), cfg, 111)
+    x = synth.layer_input(cfg, B, T, 112)
+    ref = oracle.mixer_prefill(cfg, w, x)
+    r = _run_prefill(cfg, w, x)
+    mx, rl = assert_close(to_np(r["y"]), ref["y"], cfg, "y (concat fusion)")
+    print(f"concat fusion {case}: max abs {mx:.3e}, rel L2 {rl:.3e}")
+    from hybrid_head_ssm_b200 import runtime as rt
+    lay = r["lay"]
+    Tp = cfg.n_meta + T
+    o = to_np(_ws_view(r["ws"], lay["O"], (B, Tp, cfg.n_q_heads * cfg.v_head_dim), rt.mid_dtype(cfg)))
+    assert_close(o, ref["o_attn"], cfg, "attention output (dv 64)", max_abs=1e-4 if cfg.dtype == 0 else 2e-2)
+    # a consumer of the concat producer's 64-wide V
+    cc = cfg.with_(is_kv_producer=0)
+    wc = synth.perturbed_weights(synth.layer_weights(cc, 113), cc, 113)
+    refc = oracle.mixer_prefill(cc, wc, x, kv_shared=(ref["k"], ref["v"]))
+    rc = _run_prefill(cc, wc, x, kv_from=r["kv"])
+    assert_close(to_np(rc["y"]), refc["y"], cc, "consumer y (concat fusion)")
+
+
+def test_bf16_many_sequences_use_the_wide_scan():
+    """A batch wide enough (B * d_inner / 64 >= 2 * SMs) for the one-thread-per-channel
+    scan (with Delta computed inside it): 30 sequences of a small bf16 layer with a
+    ragged last chunk (8 meta + 70 rows); y, the final SSM state and the conv state."""
+    cfg = synth.hymba15_layer_cfg(window=24).with_(d_model=256, n_q_heads=5, n_kv_heads=1, d_inner=640,
+                                                   dt_rank=24, n_meta=8)
+    w = synth.perturbed_weights(synth.layer_weights(cfg, 141), cfg, 141)
+    B, T = 30, 70
+    x = synth.layer_input(cfg, B, T, 142)
+    ref = oracle.mixer_prefill(cfg, w, x)
+    r = _run_prefill(cfg, w, x)
+    mx, rl = assert_close(to_np(r["y"]), ref["y"], cfg, "y (wide scan)")
+    print(f"wide scan batch: max abs {mx:.3e}, rel L2 {rl:.3e}")
+    _check_stages(cfg, r, ref, B, cfg.n_meta + T, delta_written=False)
+    assert_close(to_np(r["st"].h), ref["h"], cfg, "final SSM state", max_abs=5e-2)
+    assert_close(to_np(r["st"].conv), ref["conv"], cfg, "conv state", max_abs=2e-2)
