@@ -48,6 +48,10 @@ Readings taken where the pages are silent:
 * The Mamba branch: depthwise causal conv (zero history before the first meta
   row) + bias, SiLU; Delta = softplus(dt_low W_dt^T + b_dt); A = -exp(A_log);
   y = (C_t . h_t + D x_t) * SiLU(z_t) with x_t the conv output.
+* The block around the mixer ([51cto] section 2 gives the MLP intermediate size 5504
+  and nothing else): pre-norm residual blocks, h + Mixer(RMSNorm(h)) then
+  h + MLP(RMSNorm(h)), each RMSNorm with its own gain, and a SiLU-gated MLP
+  W_down (SiLU(W_gate n) * W_up n) as in the Llama-family blocks the model builds on.
 * The decode cache holds the meta block in slots 0..m-1 and the non-meta
   positions in a ring: position p >= m lives in slot m + (p - m) mod R, R = cap - m.
   The conv state holds the last d_conv pre-conv inputs, oldest first.
@@ -322,6 +326,46 @@ def mixer_prefill(cfg, w, x: np.ndarray, kv_shared=None, residual: bool = False,
         sh = None if kv_shared is None else (kv_shared[0][b], kv_shared[1][b])
         rows.append(mixer_prefill_row(cfg, w, x[b], sh, residual, x_has_meta))
     return {key: np.stack([r[key] for r in rows]) for key in rows[0] if rows[0][key] is not None}
+
+
+# ----------------------------------------------------------------------------
+# the Hymba block around the mixer ([51cto] section 2: MLP intermediate size 5504)
+# ----------------------------------------------------------------------------
+
+def mlp(h: np.ndarray, w: Dict[str, np.ndarray], eps: float) -> np.ndarray:
+    """The block's pre-norm MLP with its residual: n = RMSNorm(h) * g,
+    h + W_down (SiLU(W_gate n) * (W_up n)). h [L, d]; w_gate, w_up [d_ff, d]; w_down [d, d_ff]."""
+    w = _f64(w)
+    n = rms_norm(h.astype(np.float64), w["norm_w"], eps)
+    a = silu(n @ w["w_gate"].T) * (n @ w["w_up"].T)
+    return h + a @ w["w_down"].T
+
+
+def block_prefill_row(cfg, w_mixer, w_mlp, h: np.ndarray, kv_shared=None):
+    """One Hymba block on one sequence's stream h [T', d] (meta rows included):
+    h1 = h + Mixer(RMSNorm(h) * g_pre), then h2 = MLP(h1) with its own pre-norm.
+    Returns the mixer's dict with y = h2 (and h1)."""
+    n = rms_norm(h.astype(np.float64), np.asarray(w_mixer["pre_norm_w"], dtype=np.float64), cfg.rms_eps)
+    r = mixer_prefill_row(cfg, w_mixer, n, kv_shared, residual=False, x_has_meta=True)
+    h1 = h + r["y"]
+    r = dict(r, h1=h1, y=mlp(h1, w_mlp, cfg.rms_eps))
+    return r
+
+
+def block_prefill(cfg, w_mixer, w_mlp, h: np.ndarray, kv_shared=None):
+    """Batched block_prefill_row, h [B, T', d]."""
+    rows = []
+    for b in range(h.shape[0]):
+        sh = None if kv_shared is None else (kv_shared[0][b], kv_shared[1][b])
+        rows.append(block_prefill_row(cfg, w_mixer, w_mlp, h[b], sh))
+    return {key: np.stack([r[key] for r in rows]) for key in rows[0] if rows[0][key] is not None}
+
+
+def block_decode(cfg, w_mixer, w_mlp, h_t: np.ndarray, cache: dict, hs: np.ndarray, conv: np.ndarray):
+    """One decode step of the block: h_t [B, d] -> MLP(h_t + Mixer(RMSNorm(h_t) * g_pre))."""
+    n = rms_norm(h_t.astype(np.float64), np.asarray(w_mixer["pre_norm_w"], dtype=np.float64), cfg.rms_eps)
+    h1 = h_t + mixer_decode(cfg, w_mixer, n, cache, hs, conv, residual=False)
+    return mlp(h1, w_mlp, cfg.rms_eps)
 
 
 # ----------------------------------------------------------------------------

@@ -192,3 +192,21 @@ def affine_kv(cfg: LayerCfg, seed: int, spread: float = 0.5) -> Dict[str, np.nda
     n = G * (dh + dv)
     return {"kv_scale": g.uniform(1.0 - spread, 1.0 + spread, size=n).astype(np.float32),
             "kv_bias": (g.standard_normal(n) * 0.1).astype(np.float32)}
+
+
+def mlp_weights(d_model: int, d_ff: int, dtype: int, seed: int) -> Dict[str, np.ndarray]:
+    """The block's MLP: W_gate, W_up [d_ff, d_model] ~ N(0, 1/d_model), W_down [d_model, d_ff]
+    ~ N(0, 1/d_ff) (storage-exact), and its pre-norm gain (1)."""
+    return {"norm_w": np.ones(d_model, np.float32),
+            "w_gate": to_storage(_normal(_rng(seed, 21), (d_ff, d_model), 1.0 / d_model), dtype),
+            "w_up": to_storage(_normal(_rng(seed, 22), (d_ff, d_model), 1.0 / d_model), dtype),
+            "w_down": to_storage(_normal(_rng(seed, 23), (d_model, d_ff), 1.0 / d_ff), dtype)}
+
+
+def with_pre_norm(w: Dict[str, np.ndarray], cfg: LayerCfg, seed: int = 0, scale: float = 0.0) -> Dict[str, np.ndarray]:
+    """A copy of the mixer weights with the block's pre-mixer RMSNorm gain (1, or 1 + N(0, scale^2))."""
+    g = np.ones(cfg.d_model) + (_rng(seed, 24).standard_normal(cfg.d_model) * scale if scale else 0.0)
+    return dict(w, pre_norm_w=g.astype(np.float32))
+
+
+HYMBA15_D_FF = 5504  # MLP intermediate size of Hymba-1.5B (51cto article, section 2)

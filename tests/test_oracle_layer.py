@@ -318,3 +318,67 @@ def test_concat_beta1_zero_drops_attention():
     x = synth.layer_input(cfg, 1, 20, 103)
     r = oracle.mixer_prefill(cfg, w, x)
     assert np.all(r["u"][..., cfg.d_inner:] == 0.0)
+
+
+# ---------------------------------------------------------------------------
+# the block around the mixer: pre-norm residual mixer, pre-norm SiLU-gated MLP
+# ("51cto" Hymba-1.5B article, section 2: MLP intermediate size 5504)
+# ---------------------------------------------------------------------------
+
+def test_mlp_hand_worked():
+    """d = 2, d_ff = 1: n = RMSNorm(h) = h / rms(h) = (1, 1) for h = (3, 3); gate row
+    (ln 3, 0) gives SiLU(ln 3) = ln 3 * 3/4; up row (2, 0) gives 2; down column (1, -1)."""
+    h = np.array([[3.0, 3.0]])
+    w = {"norm_w": np.ones(2), "w_gate": np.array([[np.log(3.0), 0.0]]), "w_up": np.array([[2.0, 0.0]]),
+         "w_down": np.array([[1.0], [-1.0]])}
+    a = np.log(3.0) * 0.75 * 2.0
+    np.testing.assert_allclose(oracle.mlp(h, w, 0.0), [[3.0 + a, 3.0 - a]], rtol=1e-14)
+
+
+def test_mlp_zero_down_is_identity_and_scale_invariant_branch():
+    g = np.random.default_rng(111)
+    w = synth.mlp_weights(32, 48, synth.F32, 111)
+    h = g.standard_normal((5, 32))
+    np.testing.assert_array_equal(oracle.mlp(h, dict(w, w_down=np.zeros_like(w["w_down"])), 1e-6), h)
+    # the branch sees RMSNorm(h): scaling h scales only the residual part
+    branch = oracle.mlp(h, w, 0.0) - h
+    np.testing.assert_allclose(oracle.mlp(7.0 * h, w, 0.0) - 7.0 * h, branch, rtol=1e-12, atol=1e-12)
+
+
+def test_block_is_two_pre_norm_residual_steps():
+    """block(h) = MLP(h + mixer(RMSNorm(h) g)); with W_out = 0 and W_down = 0 it is the
+    identity, and the mixer inside sees the normalised stream (scaling h leaves the
+    mixer's output unchanged)."""
+    cfg = synth.tiny_layer_cfg().with_(rms_eps=0.0)  # exact scale invariance of the norms
+    wm = synth.with_pre_norm(synth.layer_weights(cfg, 112), cfg, 112, scale=0.3)
+    wf = synth.mlp_weights(cfg.d_model, 96, cfg.dtype, 113)
+    g = np.random.default_rng(114)
+    h = g.standard_normal((1, cfg.n_meta + 20, cfg.d_model))
+    r = oracle.block_prefill(cfg, wm, wf, h)
+    np.testing.assert_allclose(r["y"][0], oracle.mlp(r["h1"][0], wf, cfg.rms_eps), rtol=1e-12)
+    zero = oracle.block_prefill(cfg, dict(wm, w_out=np.zeros_like(wm["w_out"])),
+                                dict(wf, w_down=np.zeros_like(wf["w_down"])), h)
+    np.testing.assert_array_equal(zero["y"], h)
+    r3 = oracle.block_prefill(cfg, wm, wf, 3.0 * h)
+    np.testing.assert_allclose(r3["h1"] - 3.0 * h, r["h1"] - h, rtol=1e-9, atol=1e-9)
+
+
+def test_block_decode_equals_block_prefill():
+    """A KV-sharing pair of blocks decodes as it prefills (window 8 ring wrapping)."""
+    ca, cb, wa, wb = _pair(8, seed=115)
+    wa, wb = synth.with_pre_norm(wa, ca, 115, 0.3), synth.with_pre_norm(wb, cb, 116, 0.3)
+    fa, fb = synth.mlp_weights(ca.d_model, 64, ca.dtype, 117), synth.mlp_weights(cb.d_model, 64, cb.dtype, 118)
+    B, T, T0 = 2, 22, 9
+    m = ca.n_meta
+    g = np.random.default_rng(119)
+    h = g.standard_normal((B, m + T, ca.d_model))
+    ra = oracle.block_prefill(ca, wa, fa, h)
+    rb = oracle.block_prefill(cb, wb, fb, ra["y"], kv_shared=(ra["k"], ra["v"]))
+    pa = oracle.block_prefill(ca, wa, fa, h[:, :m + T0])
+    pb = oracle.block_prefill(cb, wb, fb, pa["y"], kv_shared=(pa["k"], pa["v"]))
+    cache = oracle.cache_from_prefill(ca, pa["k"], pa["v"], m + 8)
+    ha, conva, hb, convb = pa["h"].copy(), pa["conv"].copy(), pb["h"].copy(), pb["conv"].copy()
+    for t in range(T0, T):
+        ya = oracle.block_decode(ca, wa, fa, h[:, m + t], cache, ha, conva)
+        yb = oracle.block_decode(cb, wb, fb, ya, cache, hb, convb)
+        np.testing.assert_allclose(yb, rb["y"][:, m + t], rtol=1e-10, atol=1e-10)
