@@ -54,21 +54,44 @@ def peaks():
     return dict(hbm=6650.0, bf16=1590.0, bf16_sus=1400.0, sm_mhz=1965.0, src="fallback")
 
 
+TRAFFIC_HEADERS = ("hybrid_head_ssm_b200/csrc/common.cuh", "hybrid_head_ssm_b200/csrc/tc.cuh",
+                   "hybrid_head_ssm_b200/csrc/kernels.h", "hybrid_head_ssm_b200/csrc/epilogue.cuh",
+                   "include/hymba.h")
+
+
+def sources_sha1(sources):
+    """sha1 over the kernel's source file and every header it includes."""
+    h = hashlib.sha1()
+    for rel in sources:
+        h.update(rel.encode())
+        h.update(open(os.path.join(ROOT, rel), "rb").read())
+    return h.hexdigest()
+
+
 def kernel_traffic(name, workload):
     """DRAM bytes per launch of a kernel from the committed ncu record (profiles/), or
-    None when there is none for this workload or the kernel's device code changed since
-    (the record hashes the source file up to the kernel's host launcher)."""
+    None when there is none for this workload or the kernel's source (its file and the
+    headers it includes) changed since the counters were taken."""
     try:
         rec = json.load(open(os.path.join(ROOT, "profiles", "dram_traffic.json"))).get(name)
         if not rec or rec.get("workload") != workload:
             return None
-        src = open(os.path.join(ROOT, rec["kernel_source"]), "rb").read()
-        end = src.find(rec["device_code_until"].encode())
-        if end < 0 or hashlib.sha1(src[:end]).hexdigest() != rec["device_code_sha1"]:
+        if sources_sha1(rec["sources"]) != rec["sources_sha1"]:
             return None
         return rec["bytes_per_launch"]
     except (OSError, ValueError, KeyError):
         return None
+
+
+def record_traffic(name, workload, source, bytes_per_launch, counters, summary):
+    """Write the committed record of a kernel's measured DRAM traffic (ncu
+    dram__bytes_read.sum + dram__bytes_write.sum per launch), keyed on its sources."""
+    path = os.path.join(ROOT, "profiles", "dram_traffic.json")
+    recs = json.load(open(path)) if os.path.exists(path) else {}
+    sources = [source] + list(TRAFFIC_HEADERS)
+    recs[name] = {"bytes_per_launch": bytes_per_launch, "counters": counters, "workload": workload,
+                  "summary": summary, "sources": sources, "sources_sha1": sources_sha1(sources)}
+    json.dump(recs, open(path, "w"), indent=2)
 
 
 def roofline_entry(name, bound, units, avg_s, pk, sm_count, sm_mhz, long_step=False):
@@ -373,17 +396,19 @@ class PrefillWorkload:
     32-layer stack (fp32 residual stream, KV shared by layer pairs, in place after the
     first layer). step(x, y) queues one pass over all its layers on the current stream."""
 
-    def __init__(self, name, rank, torch, hy, rt):
+    def __init__(self, name, rank, torch, hy, rt, shrink=None):
         import ctypes
         self.name, self.torch, self.hy, self.rt = name, torch, hy, rt
         wl = synth.workload(name)
+        if shrink:
+            wl.update(shrink)  # a profiling-size case of the same workload
         self.wl = wl
         self.B, self.T = wl["B"], wl["T"]
         base = wl["cfg"]
         self.Tp = base.n_meta + self.T
         self.stack = wl["kind"] == "stack"
         if self.stack:
-            self.cfgs = synth.stack_layer_cfgs(base, wl["n_layers"], wl["global_layers"])
+            self.cfgs = synth.stack_layer_cfgs(base, wl["n_layers"], wl["global_layers"])[:wl["n_layers"]]
             seeds = [1000 * wl["seed"] + l for l in range(len(self.cfgs))]
         else:
             self.cfgs, seeds = [base], [wl["seed"]]
@@ -546,6 +571,8 @@ def bench_decode(args, torch, hy, rt, max_ranks, barrier, world, pk, flush):
     ca = wl["cfg"]
     cb = ca.with_(is_kv_producer=0)
     B, T, seed = wl["B"], wl["T"], wl["seed"]
+    if args.decode_prompt > 0:
+        T = args.decode_prompt
     la = rt.DeviceLayer(ca, synth.layer_weights(ca, seed * 1000))
     lb = rt.DeviceLayer(cb, synth.layer_weights(cb, seed * 1000 + 1))
     cap = ca.n_meta + ca.window
@@ -625,7 +652,21 @@ def main():
     ap.add_argument("--clocks-dir", default="",
                     help="where the NVML clock samples are written (default: the system temp directory)")
     ap.add_argument("--no-extra", action="store_true", help="time only the headline workload")
+    ap.add_argument("--only", default="", choices=["", "stack", "global", "swa", "decode"],
+                    help="run one workload alone and print its figures (for profiling runs)")
+    ap.add_argument("--decode-prompt", type=int, default=0,
+                    help="prompt length of the decode pair's prefill (default: the workload's 4096)")
+    ap.add_argument("--small", action="store_true",
+                    help="with --only: the profiling-size case of the workload (stack: 2 layers, T=1024; "
+                         "global: B=1; decode: a 1100-token prompt), a few GB on the device at most")
+    ap.add_argument("--record-traffic", nargs=6, metavar=("KERNEL", "WORKLOAD", "SOURCE", "BYTES", "COUNTERS",
+                                                          "SUMMARY"),
+                    help="write the DRAM traffic record of a kernel measured by ncu and exit")
     args = ap.parse_args()
+    if args.record_traffic:
+        k, wl, src, nb, counters, summary = args.record_traffic
+        record_traffic(k, wl, src, int(nb), counters, summary)
+        return None
     args.warmup = max(args.warmup, 3)
 
     rank = int(os.environ.get("RANK", "0"))
@@ -656,6 +697,27 @@ def main():
     rates = hy.unit_rates()  # exp2 and FMA results per clock per SM, measured on this GPU
     pk["mufu_per_clk_sm"] = rates["ex2_f32"]
     flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")  # > 126 MB L2
+
+    if args.only:
+        # one workload alone, for profiling runs: no headline line
+        if args.only == "decode":
+            if args.small and args.decode_prompt <= 0:
+                args.decode_prompt = 1100
+            r = bench_decode(args, torch, hy, rt, max_ranks, barrier, world, pk, flush)
+        else:
+            name = {"stack": WORKLOAD, "global": LAYER_WORKLOADS[0], "swa": LAYER_WORKLOADS[1]}[args.only]
+            shrink = None
+            if args.small:
+                shrink = {"stack": dict(T=1024, n_layers=2), "global": dict(B=1), "swa": {}}[args.only]
+            w1 = PrefillWorkload(name, rank, torch, hy, rt, shrink)
+            r = time_prefill(w1, args, torch, hy, barrier, max_ranks, pk, flush, None, sm_count, headline=False)
+            r = {"workload": name, "ms_per_step": r["ms"], "tokens_per_s": w1.tokens * world / (r["ms"] * 1e-3),
+                 "kernels": r["kern"]}
+        if rank == 0:
+            print(json.dumps({"only": args.only, **r}))
+        if world > 1:
+            dist.destroy_process_group()
+        return r
 
     clocks = Clocks(local, args.clocks_dir)
     clocks.start()

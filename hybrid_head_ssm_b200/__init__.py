@@ -39,6 +39,7 @@ HYMBA_F16 = 2
 HYMBA_X_HAS_META = 1
 HYMBA_ADD_RESIDUAL = 2
 HYMBA_IO_F32 = 4
+HYMBA_PRE_NORM = 8
 HYMBA_FUSION_AVERAGE = 0
 HYMBA_FUSION_CONCAT = 1
 HYMBA_MODE_PREFILL = 0
@@ -57,7 +58,7 @@ class hymba_layer_cfg(ctypes.Structure):
 class hymba_layer_weights(ctypes.Structure):
     _fields_ = [(n, _vp) for n in ("w_in", "w_dt", "b_dt", "conv_w", "conv_b", "A_log", "D",
                                    "norm_attn_w", "norm_ssm_w", "beta1", "beta2", "w_out", "meta",
-                                   "kv_scale", "kv_bias")]
+                                   "kv_scale", "kv_bias", "pre_norm_w")]
 
 
 class hymba_kv(ctypes.Structure):
@@ -65,6 +66,10 @@ class hymba_kv(ctypes.Structure):
                 ("len", _vp), ("cache_cap", _i32), ("batch", _i32), ("n_meta", _i32),
                 ("n_kv_heads", _i32), ("head_dim", _i32), ("v_head_dim", _i32), ("dtype", _i32),
                 ("window", _i32)]
+
+
+class hymba_mlp_weights(ctypes.Structure):
+    _fields_ = [(n, _vp) for n in ("norm_w", "w_gate", "w_up", "w_down")]
 
 
 class hymba_ssm_state(ctypes.Structure):
@@ -79,6 +84,9 @@ _sig = {
     "hymba_mixer_decode": (ctypes.c_int, [_P(hymba_layer_cfg), _P(hymba_layer_weights), _vp, ctypes.c_int,
                                           ctypes.c_int, _vp, _P(hymba_kv), _P(hymba_ssm_state), _vp, _sz, _vp]),
     "hymba_kv_share": (ctypes.c_int, [_P(hymba_kv), _P(hymba_layer_cfg), _P(hymba_kv)]),
+    "hymba_mlp": (ctypes.c_int, [_P(hymba_layer_cfg), ctypes.c_int, _P(hymba_mlp_weights), _vp, ctypes.c_longlong,
+                                 _vp, _sz, _vp]),
+    "hymba_mlp_workspace_bytes": (_sz, [_P(hymba_layer_cfg), ctypes.c_int, ctypes.c_longlong]),
     "hymba_workspace_bytes": (_sz, [_P(hymba_layer_cfg), ctypes.c_int, ctypes.c_int, ctypes.c_int]),
     "hymba_workspace_layout": (ctypes.c_int, [_P(hymba_layer_cfg), ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                               _P(ctypes.c_int64), ctypes.c_int]),

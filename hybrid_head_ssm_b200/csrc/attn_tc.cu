@@ -21,8 +21,11 @@
 //               tile's MMAs run under the other tile's softmax;
 //   warps 2-3   idle after setup;
 //   warps 4-7   softmax of tile A, warps 8-11 of tile B: one thread per query row
-//               (TMEM lane), 128 scores in registers: scale and mask, row max, P =
-//               2^(s - m) in fp32 (MUFU ex2), row sum in fp32, P packed to fp16 pairs
+//               (TMEM lane), 128 scores in registers (four TMEM loads in flight, one wait):
+//               scale and mask, row max, P = 2^(s - m) in fp32 (MUFU ex2; with the MMAs
+//               of the other tile running meanwhile the exponentials are not the limit:
+//               moving a quarter of them to an FMA-pipe polynomial measured no faster),
+//               row sum in fp32, P packed to fp16 pairs
 //               and stored to TMEM with tcgen05.st. O is rescaled in TMEM only when the
 //               running max grows by more than 2^8 (P then stays below 2^8, far inside
 //               fp16). At the end O / l is written in fp16.
@@ -135,27 +138,6 @@ __device__ __forceinline__ void mma_f16_ts(uint32_t tmem_d, uint32_t tmem_a, uin
         "setp.ne.b32 p, %4, 0;\n\t"
         "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}"
         ::"r"(tmem_d), "r"(tmem_a), "l"(bdesc), "r"(idesc), "r"(accumulate));
-}
-
-// 2^x on the FMA pipe for a pair of arguments x <= 16 (or -inf), Cody-Waite style:
-// x = j + f with j = round(x) (the magic constant 1.5 * 2^23 leaves j in the low mantissa
-// bits) and f in [-1/2, 1/2]; 2^f from the degree-3 polynomial with the least relative
-// error on that interval (coefficients fitted by Lawson's iteratively reweighted least
-// squares; relative error 7.5e-5, below the half-ulp of the fp16 P it feeds); 2^j added
-// to the exponent field. Arguments are clamped at -125 so that the exponent stays
-// normal: 2^-125 rounds to 0 in fp16 and is negligible in the fp32 row sum.
-constexpr float EXP2_C0 = 0.99992812f, EXP2_C1 = 0.69326097f, EXP2_C2 = 0.24261054f, EXP2_C3 = 0.05517132f;
-__device__ __forceinline__ float2 exp2_poly2(float2 x) {
-    x = make_float2(fmaxf(x.x, -125.f), fmaxf(x.y, -125.f));
-    const float2 magic = make_float2(12582912.f, 12582912.f);
-    const float2 t = __fadd2_rn(x, magic);
-    const float2 f = __fadd2_rn(x, __fadd2_rn(magic, make_float2(-t.x, -t.y)));
-    float2 p = __ffma2_rn(make_float2(EXP2_C3, EXP2_C3), f, make_float2(EXP2_C2, EXP2_C2));
-    p = __ffma2_rn(p, f, make_float2(EXP2_C1, EXP2_C1));
-    p = __ffma2_rn(p, f, make_float2(EXP2_C0, EXP2_C0));
-    const int jx = __float_as_int(t.x) - 0x4B400000, jy = __float_as_int(t.y) - 0x4B400000;
-    return make_float2(__int_as_float(__float_as_int(p.x) + (jx << 23)),
-                       __int_as_float(__float_as_int(p.y) + (jy << 23)));
 }
 
 // 32 lanes x 64 consecutive 32-bit columns from registers (thread t writes lane base + t).
@@ -444,8 +426,7 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
 #pragma unroll
             for (int c = 0; c < 64; ++c) {
                 const float2 x = __ffma2_rn(make_float2(sv[2 * c], sv[2 * c + 1]), sc2, nmu2);
-                // three pairs in four on the MUFU unit, the fourth on the FMA pipe
-                const float2 p = (c & 3) == 3 ? exp2_poly2(x) : make_float2(fast_exp2(x.x), fast_exp2(x.y));
+                const float2 p = make_float2(fast_exp2(x.x), fast_exp2(x.y));
                 l4[c & 3] = __fadd2_rn(l4[c & 3], p);
                 pk[c] = pack_f16x2(p.x, p.y);
             }

@@ -7,7 +7,7 @@
 
 namespace hymba {
 
-enum EpiKind { EPI_INPROJ = 0, EPI_DELTA = 1, EPI_OUT = 2 };
+enum EpiKind { EPI_INPROJ = 0, EPI_DELTA = 1, EPI_OUT = 2, EPI_GLU = 3 };
 
 // How GEMM row r maps to rows of the layer's T' = n_meta + T rows per sequence.
 enum RowMode {
@@ -47,6 +47,8 @@ struct EpiArgs {
     const T* res_x;
     const void* res_meta;  // [n_meta, N] of the layer's weight type
     int res_meta_bf16;     // 1: res_meta is bf16; 0: it has type T
+    // EPI_GLU: y = SiLU(gate) * (this GEMM's result), gate [M, N] of type T
+    const T* glu_gate;
     // in-projection GEMMs that also cover the meta rows: GEMM rows [0, meta_pad) are
     // meta rows (valid below meta_M, written for every sequence), the rest follow
     // row_mode after subtracting meta_pad
@@ -145,6 +147,19 @@ __device__ __forceinline__ RunDst epi_prepare64(const EpiArgs<T>& e, int r, int 
         d.p = reinterpret_cast<char*>(e.delta + (long long)r * e.N + c0);
         d.count = 1;
         d.nbytes = n * 4;
+        return d;
+    }
+    if (e.kind == EPI_GLU) {
+        // the gated MLP: SiLU of the gate projection (same row and columns) times this one
+        float gv[64];
+#pragma unroll
+        for (int j = 0; j < 64; ++j) gv[j] = 0.f;
+        add_residual64(gv, e.glu_gate + (long long)r * e.N + c0, n);
+#pragma unroll
+        for (int j = 0; j < 64; ++j) v[j] *= silu_f(gv[j]);
+        d.p = reinterpret_cast<char*>(e.y + (long long)r * e.N + c0);
+        d.count = 1;
+        d.nbytes = n * (int)sizeof(T);
         return d;
     }
     if (e.kind == EPI_OUT) {

@@ -192,8 +192,10 @@ static Plan plan(const hymba_layer_cfg* c, int B, int T, int mode) {
     p.ypre = take(&cur, rows * di * esz);
     p.U = take(&cur, rows * u_width(c) * esz);
     p.wdt = take(&cur, (size_t)di * p.rpad * esz);
+    // the projection's copy of the input rows: converted to 16 bits (fp32 stream of a
+    // bf16 layer) or RMS-normalised (HYMBA_PRE_NORM)
+    p.xcv = take(&cur, rows * c->d_model * esz);
     if (c->dtype == HYMBA_BF16) {
-        p.xcv = take(&cur, rows * c->d_model * 2);  // 16-bit copy of an fp32 input
         if (mode == HYMBA_MODE_PREFILL) {
             // fp16 copies of the projection weights for fp32-stream calls (and of W_out
             // for the concat fusion)
@@ -290,20 +292,30 @@ static int prefill_impl(const Ctx& ctx, const hymba_layer_cfg* c, const hymba_la
     int rc;
 
     const TA *x, *W_in, *meta, *W_out;
+    const bool pre_norm = flags & HYMBA_PRE_NORM;
+    TA* xn = reinterpret_cast<TA*>(ws + pl.xcv);
     if constexpr (kF16Ops) {
-        TA* xc = reinterpret_cast<TA*>(ws + pl.xcv);
         TA* wi = reinterpret_cast<TA*>(ws + pl.win16);
         TA* mt = reinterpret_cast<TA*>(ws + pl.meta16);
         TA* wo = reinterpret_cast<TA*>(ws + pl.wout16);
         const int xrows = B * (has_meta ? Tp : T_);
-        if ((rc = launch_pad_copy<TIO, TA>(ctx, x_io, xrows, d, xc, d))) return rc;
+        if (pre_norm) {
+            if ((rc = launch_rmsnorm_rows<TIO, TA>(ctx, x_io, w->pre_norm_w, xn, xrows, d, c->rms_eps))) return rc;
+        } else if ((rc = launch_pad_copy<TIO, TA>(ctx, x_io, xrows, d, xn, d))) {
+            return rc;
+        }
         if ((rc = launch_pad_copy<T, TA>(ctx, static_cast<const T*>(w->w_in), k.n_in, d, wi, d))) return rc;
         if (m > 0 && !has_meta && (rc = launch_pad_copy<T, TA>(ctx, static_cast<const T*>(w->meta), m, d, mt, d)))
             return rc;
         if ((rc = launch_pad_copy<T, TA>(ctx, static_cast<const T*>(w->w_out), d, uw, wo, uw))) return rc;
-        x = xc; W_in = wi; meta = mt; W_out = wo;
+        x = xn; W_in = wi; meta = mt; W_out = wo;
     } else {
         x = x_io;
+        if (pre_norm) {
+            if ((rc = launch_rmsnorm_rows<TIO, TA>(ctx, x_io, w->pre_norm_w, xn, (long long)B * Tp, d, c->rms_eps)))
+                return rc;
+            x = xn;
+        }
         W_in = static_cast<const T*>(w->w_in);
         meta = static_cast<const T*>(w->meta);
         W_out = static_cast<const T*>(w->w_out);
@@ -450,12 +462,18 @@ static int decode_impl(const Ctx& ctx, const hymba_layer_cfg* c, const hymba_lay
     // the layer's type: one launch
     float2* rope = reinterpret_cast<float2*>(ws + pl.rope);
     const T* x;
-    if constexpr (std::is_same<TIO, T>::value) {
+    T* xc = reinterpret_cast<T*>(ws + pl.xcv);
+    if (flags & HYMBA_PRE_NORM) {
+        // the block's pre-norm: the projection reads RMSNorm(x) * g, the residual is x
+        if ((rc = launch_rmsnorm_rows<TIO, T>(ctx, x_io, w->pre_norm_w, xc, B, d, c->rms_eps))) return rc;
+        rc = launch_decode_prep<T, T>(ctx, rope, kv->len, pos_offset, B, dh, c->rope_base, nullptr, 0, 0,
+                                      nullptr, 0);
+        x = xc;
+    } else if constexpr (std::is_same<TIO, T>::value) {
         x = x_io;
         rc = launch_decode_prep<T, T>(ctx, rope, kv->len, pos_offset, B, dh, c->rope_base, nullptr, 0, 0,
                                       nullptr, 0);
     } else {
-        T* xc = reinterpret_cast<T*>(ws + pl.xcv);
         rc = launch_decode_prep<TIO, T>(ctx, rope, kv->len, pos_offset, B, dh, c->rope_base, x_io, B, d, xc, d);
         x = xc;
     }
@@ -520,6 +538,69 @@ static int check_kv_shape(const hymba_layer_cfg* c, const hymba_kv* kv, int B) {
     return HYMBA_OK;
 }
 
+// ---------------------------------------------------------------------------
+// the block's MLP: h += W_down (SiLU(W_gate n) * (W_up n)), n = RMSNorm(h) * g
+// ---------------------------------------------------------------------------
+struct MlpPlan {
+    size_t total = 0, n = 0, gate = 0, act = 0, wg = 0, wu = 0, wd = 0;
+};
+
+static MlpPlan mlp_plan(const hymba_layer_cfg* c, int d_ff, long long rows) {
+    MlpPlan p;
+    const size_t esz = c->dtype == HYMBA_BF16 ? 2 : 4;  // fp16 operands for bf16 layers
+    size_t cur = 0;
+    p.n = take(&cur, rows * c->d_model * esz);
+    p.gate = take(&cur, rows * (size_t)d_ff * esz);
+    p.act = take(&cur, rows * (size_t)d_ff * esz);
+    if (c->dtype == HYMBA_BF16) {
+        p.wg = take(&cur, (size_t)d_ff * c->d_model * 2);
+        p.wu = take(&cur, (size_t)d_ff * c->d_model * 2);
+        p.wd = take(&cur, (size_t)c->d_model * d_ff * 2);
+    }
+    p.total = cur;
+    return p;
+}
+
+// T: the layer's weight type; TA: the operand type (fp16 for bf16 weights, converted per
+// call; fp32 for fp32 layers, CUDA-core GEMMs)
+template <typename T, typename TA>
+static int mlp_impl(const Ctx& ctx, const hymba_layer_cfg* c, int d_ff, const hymba_mlp_weights* w, float* h,
+                    long long rows, char* ws) {
+    const MlpPlan pl = mlp_plan(c, d_ff, rows);
+    const int d = c->d_model;
+    TA* n = reinterpret_cast<TA*>(ws + pl.n);
+    TA* gate = reinterpret_cast<TA*>(ws + pl.gate);
+    TA* act = reinterpret_cast<TA*>(ws + pl.act);
+    const TA *Wg, *Wu, *Wd;
+    int rc;
+    if constexpr (std::is_same<T, TA>::value) {
+        Wg = static_cast<const TA*>(w->w_gate);
+        Wu = static_cast<const TA*>(w->w_up);
+        Wd = static_cast<const TA*>(w->w_down);
+    } else {
+        TA* wg = reinterpret_cast<TA*>(ws + pl.wg);
+        TA* wu = reinterpret_cast<TA*>(ws + pl.wu);
+        TA* wd = reinterpret_cast<TA*>(ws + pl.wd);
+        if ((rc = launch_pad_copy<T, TA>(ctx, static_cast<const T*>(w->w_gate), d_ff, d, wg, d))) return rc;
+        if ((rc = launch_pad_copy<T, TA>(ctx, static_cast<const T*>(w->w_up), d_ff, d, wu, d))) return rc;
+        if ((rc = launch_pad_copy<T, TA>(ctx, static_cast<const T*>(w->w_down), d, d_ff, wd, d_ff))) return rc;
+        Wg = wg; Wu = wu; Wd = wd;
+    }
+    if ((rc = launch_rmsnorm_rows<float, TA>(ctx, h, w->norm_w, n, rows, d, c->rms_eps))) return rc;
+    EpiArgs<TA> eg = epi_base<TA>(EPI_OUT, (int)rows, d_ff);
+    eg.y = gate;
+    if ((rc = gemm<TA, TA>(ctx, "gemm_mlp_gate", n, d, Wg, d, (int)rows, d_ff, d, eg))) return rc;
+    EpiArgs<TA> eu = epi_base<TA>(EPI_GLU, (int)rows, d_ff);
+    eu.y = act;
+    eu.glu_gate = gate;
+    if ((rc = gemm<TA, TA>(ctx, "gemm_mlp_up", n, d, Wu, d, (int)rows, d_ff, d, eu))) return rc;
+    EpiArgs<float> ed = epi_base<float>(EPI_OUT, (int)rows, d);
+    ed.y = h;
+    ed.res_mode = 1;
+    ed.res_x = h;  // in place: each output element is read, then written, by one thread
+    return gemm<TA, float>(ctx, "gemm_mlp_down", act, d_ff, Wd, d_ff, (int)rows, d, d_ff, ed);
+}
+
 }  // namespace hymba
 
 using namespace hymba;
@@ -548,7 +629,9 @@ int hymba_mixer_prefill(const hymba_layer_cfg* cfg, const hymba_layer_weights* w
     int rc = check_cfg(cfg);
     if (rc) return rc;
     if ((rc = check_weights(cfg, w))) return rc;
-    if (!x || !y || !kv || !workspace || B <= 0 || T <= 0 || (flags & ~7)) return HYMBA_ERR_INVALID_ARG;
+    if (!x || !y || !kv || !workspace || B <= 0 || T <= 0 || (flags & ~15)) return HYMBA_ERR_INVALID_ARG;
+    // the block's pre-norm acts on a stream that already holds the meta rows
+    if ((flags & HYMBA_PRE_NORM) && (!(flags & HYMBA_X_HAS_META) || !w->pre_norm_w)) return HYMBA_ERR_INVALID_ARG;
     if ((flags & HYMBA_IO_F32) && cfg->dtype != HYMBA_BF16) return HYMBA_ERR_INVALID_ARG;
     if ((uintptr_t)workspace & 255) return HYMBA_ERR_INVALID_ARG;
     if (!kv->k_seq || !kv->v_seq) return HYMBA_ERR_INVALID_ARG;
@@ -590,8 +673,9 @@ int hymba_mixer_decode(const hymba_layer_cfg* cfg, const hymba_layer_weights* w,
     if (rc) return rc;
     if ((rc = check_weights(cfg, w))) return rc;
     if (!x_t || !y_t || !kv || !st || !st->h || !st->conv || !workspace || B <= 0 ||
-        (flags & ~(HYMBA_ADD_RESIDUAL | HYMBA_IO_F32)))
+        (flags & ~(HYMBA_ADD_RESIDUAL | HYMBA_IO_F32 | HYMBA_PRE_NORM)))
         return HYMBA_ERR_INVALID_ARG;
+    if ((flags & HYMBA_PRE_NORM) && !w->pre_norm_w) return HYMBA_ERR_INVALID_ARG;
     if ((flags & HYMBA_IO_F32) && cfg->dtype != HYMBA_BF16) return HYMBA_ERR_INVALID_ARG;
     if ((uintptr_t)workspace & 255) return HYMBA_ERR_INVALID_ARG;
     if (!kv->k_cache || !kv->v_cache || !kv->len || kv->cache_cap <= cfg->n_meta) return HYMBA_ERR_INVALID_ARG;
@@ -676,6 +760,28 @@ int hymba_get_device_diag(int32_t* out, int n) {
     if (cudaMemcpy(ctx.status + 1, zero, sizeof(zero), cudaMemcpyHostToDevice) != cudaSuccess) return HYMBA_ERR_CUDA;
     for (int i = 0; i < 7; ++i) out[i] = v[i];
     return HYMBA_OK;
+}
+
+size_t hymba_mlp_workspace_bytes(const hymba_layer_cfg* cfg, int d_ff, long long rows) {
+    if (check_cfg(cfg) || d_ff <= 0 || rows <= 0) return 0;
+    return mlp_plan(cfg, d_ff, rows).total;
+}
+
+int hymba_mlp(const hymba_layer_cfg* cfg, int d_ff, const hymba_mlp_weights* w, float* h, long long rows,
+              void* workspace, size_t ws_bytes, void* stream) {
+    int rc = check_cfg(cfg);
+    if (rc) return rc;
+    if (!w || !w->norm_w || !w->w_gate || !w->w_up || !w->w_down || !h || !workspace || rows <= 0 || d_ff <= 0 ||
+        rows > 0x7fffffffLL)
+        return HYMBA_ERR_INVALID_ARG;
+    if (d_ff % 64) return HYMBA_ERR_UNSUPPORTED;
+    if (((uintptr_t)workspace & 255) || ((uintptr_t)h & 15)) return HYMBA_ERR_INVALID_ARG;
+    if (ws_bytes < mlp_plan(cfg, d_ff, rows).total) return HYMBA_ERR_WORKSPACE_TOO_SMALL;
+    Ctx ctx;
+    if ((rc = current_ctx(static_cast<cudaStream_t>(stream), &ctx))) return rc;
+    char* ws = static_cast<char*>(workspace);
+    if (cfg->dtype == HYMBA_BF16) return mlp_impl<bf16, f16>(ctx, cfg, d_ff, w, h, rows, ws);
+    return mlp_impl<float, float>(ctx, cfg, d_ff, w, h, rows, ws);
 }
 
 int hymba_debug_set_wait_limit(long long cycles) {

@@ -77,6 +77,11 @@ template <typename TS, typename TD>
 int launch_decode_prep(const Ctx& ctx, float2* tab, const int* len, int pos_offset, int B, int dh, float base,
                        const TS* w, int rows, int cols, TD* wdst, int ld_dst);
 
+// dst [rows, cols] = g * src / sqrt(mean(src^2) + eps) per row (cols <= 4096, a
+// multiple of 8; 16-byte aligned rows).
+template <typename TS, typename TD>
+int launch_rmsnorm_rows(const Ctx& ctx, const TS* src, const float* g, TD* dst, long long rows, int cols, float eps);
+
 // Copy a [rows, cols] matrix into a zero-padded [rows, ld_dst] one of type TD.
 template <typename TS, typename TD>
 int launch_pad_copy(const Ctx& ctx, const TS* src, int rows, int cols, TD* dst, int ld_dst);

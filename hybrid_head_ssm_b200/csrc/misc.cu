@@ -227,3 +227,93 @@ extern "C" int hymba_debug_stalled_wait(void* stream) {
     HYMBA_LAUNCH(ctx, "stalled_wait", hymba::stalled_wait_kernel, 1, 32, 0, ctx.status);
     return HYMBA_OK;
 }
+
+namespace hymba {
+namespace {
+
+// Row RMSNorm with gain into another type: dst[r, c] = g[c] * src[r, c] / sqrt(mean_c
+// src[r, c]^2 + eps). One row per 256-thread block, pieces of 8 elements (16-byte
+// accesses when the element type allows), the row held in registers between the sum of
+// squares and the output (cols <= 4096).
+template <typename TS, typename TD>
+__global__ void __launch_bounds__(256) rmsnorm_rows_kernel(const TS* __restrict__ src, const float* __restrict__ g,
+                                                           TD* __restrict__ dst, int rows, int cols, float eps) {
+    griddep_sync();
+    __shared__ float red[8];
+    const long long r = blockIdx.x;
+    const int t = threadIdx.x;
+    const int npc = cols / 8;
+    float v[2][8];
+    float ss = 0.f;
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+        const int pc = t + k * 256;
+        if (pc < npc) {
+            const TS* p = src + r * cols + 8 * pc;
+            if constexpr (sizeof(TS) == 4) {
+                const float4 a = *reinterpret_cast<const float4*>(p);
+                const float4 b = *reinterpret_cast<const float4*>(p + 4);
+                v[k][0] = a.x; v[k][1] = a.y; v[k][2] = a.z; v[k][3] = a.w;
+                v[k][4] = b.x; v[k][5] = b.y; v[k][6] = b.z; v[k][7] = b.w;
+            } else {
+                const uint4 u = *reinterpret_cast<const uint4*>(p);
+                const TS* h = reinterpret_cast<const TS*>(&u);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) v[k][i] = to_f(h[i]);
+            }
+#pragma unroll
+            for (int i = 0; i < 8; ++i) ss = fmaf(v[k][i], v[k][i], ss);
+        }
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+    if ((t & 31) == 0) red[t >> 5] = ss;
+    __syncthreads();
+    ss = 0.f;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) ss += red[w];
+    const float inv = 1.0f / sqrtf(ss / cols + eps);
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+        const int pc = t + k * 256;
+        if (pc < npc) {
+            const float4 ga = *reinterpret_cast<const float4*>(g + 8 * pc);
+            const float4 gb = *reinterpret_cast<const float4*>(g + 8 * pc + 4);
+            const float gg[8] = {ga.x, ga.y, ga.z, ga.w, gb.x, gb.y, gb.z, gb.w};
+            TD* q = dst + r * cols + 8 * pc;
+            if constexpr (sizeof(TD) == 4) {
+                *reinterpret_cast<float4*>(q) = make_float4(gg[0] * v[k][0] * inv, gg[1] * v[k][1] * inv,
+                                                            gg[2] * v[k][2] * inv, gg[3] * v[k][3] * inv);
+                *reinterpret_cast<float4*>(q + 4) = make_float4(gg[4] * v[k][4] * inv, gg[5] * v[k][5] * inv,
+                                                                gg[6] * v[k][6] * inv, gg[7] * v[k][7] * inv);
+            } else {
+                uint4 o;
+                o.x = pack2<TD>(gg[0] * v[k][0] * inv, gg[1] * v[k][1] * inv);
+                o.y = pack2<TD>(gg[2] * v[k][2] * inv, gg[3] * v[k][3] * inv);
+                o.z = pack2<TD>(gg[4] * v[k][4] * inv, gg[5] * v[k][5] * inv);
+                o.w = pack2<TD>(gg[6] * v[k][6] * inv, gg[7] * v[k][7] * inv);
+                *reinterpret_cast<uint4*>(q) = o;
+            }
+        }
+    }
+}
+
+}  // namespace
+
+template <typename TS, typename TD>
+int launch_rmsnorm_rows(const Ctx& ctx, const TS* src, const float* g, TD* dst, long long rows, int cols, float eps) {
+    if (rows <= 0) return HYMBA_OK;
+    if (cols % 8 || cols > 4096 || rows > 0x7fffffffLL ||
+        ((reinterpret_cast<uintptr_t>(src) | reinterpret_cast<uintptr_t>(dst) | reinterpret_cast<uintptr_t>(g)) & 15))
+        return HYMBA_ERR_UNSUPPORTED;
+    auto kern = rmsnorm_rows_kernel<TS, TD>;
+    HYMBA_LAUNCH(ctx, "rmsnorm", kern, (unsigned)rows, 256, 0, src, g, dst, (int)rows, cols, eps);
+    return HYMBA_OK;
+}
+
+template int launch_rmsnorm_rows<float, float>(const Ctx&, const float*, const float*, float*, long long, int, float);
+template int launch_rmsnorm_rows<float, f16>(const Ctx&, const float*, const float*, f16*, long long, int, float);
+template int launch_rmsnorm_rows<bf16, bf16>(const Ctx&, const bf16*, const float*, bf16*, long long, int, float);
+template int launch_rmsnorm_rows<float, bf16>(const Ctx&, const float*, const float*, bf16*, long long, int, float);
+
+}  // namespace hymba

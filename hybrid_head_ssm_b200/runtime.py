@@ -17,8 +17,9 @@ from . import (HYMBA_BF16, HYMBA_MODE_DECODE, HYMBA_MODE_PREFILL, check, cfg_str
 
 BIG = ("w_in", "w_dt", "w_out", "meta")
 NAMES = ("w_in", "w_dt", "b_dt", "conv_w", "conv_b", "A_log", "D", "norm_attn_w", "norm_ssm_w",
-         "beta1", "beta2", "w_out", "meta", "kv_scale", "kv_bias")
-OPTIONAL = ("kv_scale", "kv_bias")  # a consumer's affine adaptation of the shared K/V
+         "beta1", "beta2", "w_out", "meta", "kv_scale", "kv_bias", "pre_norm_w")
+# a consumer's affine adaptation of the shared K/V; the block's pre-mixer norm gain
+OPTIONAL = ("kv_scale", "kv_bias", "pre_norm_w")
 
 
 def act_dtype(cfg):
@@ -101,3 +102,34 @@ def stream_flags(cfg) -> int:
     """Flags of a layer inside a residual stack: fp32 residual stream for bf16 layers."""
     from . import HYMBA_ADD_RESIDUAL, HYMBA_IO_F32
     return HYMBA_ADD_RESIDUAL | (HYMBA_IO_F32 if cfg.dtype == HYMBA_BF16 else 0)
+
+
+class DeviceMLP:
+    """The block MLP's weights in device memory and their C struct."""
+
+    def __init__(self, cfg, w: Dict[str, np.ndarray], device="cuda"):
+        from . import hymba_mlp_weights
+        self.cfg = cfg
+        self.c = cfg_struct(cfg)
+        self.d_ff = w["w_gate"].shape[0]
+        adt = act_dtype(cfg)
+        self.t = {n: torch.from_numpy(np.ascontiguousarray(w[n], dtype=np.float32)).to(
+            device=device, dtype=torch.float32 if n == "norm_w" else adt) for n in ("norm_w", "w_gate", "w_up", "w_down")}
+        self.s = hymba_mlp_weights(*[self.t[n].data_ptr() for n in ("norm_w", "w_gate", "w_up", "w_down")])
+
+
+def mlp_workspace(mlp: DeviceMLP, rows: int, device="cuda") -> torch.Tensor:
+    from . import hymba_mlp_workspace_bytes
+    n = hymba_mlp_workspace_bytes(ctypes.byref(mlp.c), mlp.d_ff, rows)
+    if n == 0:
+        raise ValueError("invalid MLP configuration")
+    return torch.empty(n, dtype=torch.uint8, device=device)
+
+
+def mlp(m: DeviceMLP, h: torch.Tensor, ws: torch.Tensor) -> None:
+    """h += MLP(RMSNorm(h)) in place on every row of the fp32 stream h."""
+    from . import hymba_mlp
+    assert h.dtype == torch.float32 and h.is_contiguous()
+    rows = h.numel() // m.cfg.d_model
+    check(hymba_mlp(ctypes.byref(m.c), m.d_ff, ctypes.byref(m.s), h.data_ptr(), rows, ws.data_ptr(), ws.numel(),
+                    current_stream_ptr()))

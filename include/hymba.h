@@ -76,6 +76,9 @@ extern "C" {
 #define HYMBA_IO_F32        4  /* bf16 layer with fp32 x, y: a residual stream kept in fp32
                                   between stacked layers (the projection operand X^ is
                                   rounded to bf16 inside; the residual add is fp32) */
+#define HYMBA_PRE_NORM      8  /* the block's pre-norm: the mixer reads RMSNorm(x) * pre_norm_w
+                                  while the residual (HYMBA_ADD_RESIDUAL) stays x; prefill
+                                  requires HYMBA_X_HAS_META (the stream holds the meta rows) */
 
 /* fusion of the two head families (hymba_layer_cfg.fusion) */
 #define HYMBA_FUSION_AVERAGE 0  /* U = (beta1 RMSNorm(O) + beta2 RMSNorm(Y)) / 2, d_inner wide */
@@ -142,6 +145,8 @@ typedef struct hymba_layer_weights {
      * sum to 1). */
     const float* kv_scale;
     const float* kv_bias;
+    /* [d_model] fp32 gain of the block's pre-mixer RMSNorm (HYMBA_PRE_NORM; else unused) */
+    const float* pre_norm_w;
 } hymba_layer_weights;
 
 /* K/V of one producer layer and of the consumers that share it ("Hymba Guide",
@@ -214,6 +219,26 @@ int hymba_mixer_decode(const hymba_layer_cfg* cfg, const hymba_layer_weights* w,
                        const void* x_t, int B, int flags, void* y_t,
                        hymba_kv* kv, hymba_ssm_state* st,
                        void* workspace, size_t ws_bytes, void* stream);
+
+/* The MLP of the Hymba block around the mixer (the 51cto Hymba-1.5B article, section 2,
+ * gives its intermediate size, 5504; the form is the Llama-family pre-norm SiLU-gated
+ * MLP): h += W_down (SiLU(W_gate n) * (W_up n)) with n = RMSNorm(h) * norm_w, on every
+ * row of the fp32 residual stream h [rows, d_model] in place. A block is
+ *   hymba_mixer_prefill/decode(... HYMBA_PRE_NORM | HYMBA_ADD_RESIDUAL ...), then hymba_mlp.
+ * Weights (device, caller-owned) of the layer's dtype: w_gate, w_up [d_ff, d_model],
+ * w_down [d_model, d_ff]; norm_w [d_model] fp32. d_ff a multiple of 64. A bf16 layer's
+ * GEMMs take fp16 operands (the weights converted per call into the workspace); an
+ * fp32 layer's run on CUDA cores. Workspace: hymba_mlp_workspace_bytes, 256-byte aligned. */
+typedef struct hymba_mlp_weights {
+    const float* norm_w;
+    const void*  w_gate;
+    const void*  w_up;
+    const void*  w_down;
+} hymba_mlp_weights;
+
+int hymba_mlp(const hymba_layer_cfg* cfg, int d_ff, const hymba_mlp_weights* w, float* h, long long rows,
+              void* workspace, size_t ws_bytes, void* stream);
+size_t hymba_mlp_workspace_bytes(const hymba_layer_cfg* cfg, int d_ff, long long rows);
 
 /* Cross-layer KV sharing: fill *consumer_out with the producer's buffers (pointer
  * copies, no device work, no new memory). Fails with HYMBA_ERR_KV_INCOMPATIBLE
