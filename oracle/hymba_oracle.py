@@ -48,6 +48,11 @@ Readings taken where the pages are silent:
 * The Mamba branch: depthwise causal conv (zero history before the first meta
   row) + bias, SiLU; Delta = softplus(dt_low W_dt^T + b_dt); A = -exp(A_log);
   y = (C_t . h_t + D x_t) * SiLU(z_t) with x_t the conv output.
+* The SSD form of the Mamba heads ([Lecture 04] section 3 names it without
+  formulas; cfg.ssm_heads > 0): the channels split into ssm_heads heads of
+  d_inner / ssm_heads consecutive channels; W_dt, b_dt and A_log have one entry per
+  head, so Delta_t and A are scalars per head shared by its channels and all states;
+  conv, B_t, C_t, D and the gate are as in the selective form.
 * The block around the mixer ([51cto] section 2 gives the MLP intermediate size 5504
   and nothing else): pre-norm residual blocks, h + Mixer(RMSNorm(h)) then
   h + MLP(RMSNorm(h)), each RMSNorm with its own gain, and a SiLU-gated MLP
@@ -212,6 +217,26 @@ def selective_scan(xc: np.ndarray, delta: np.ndarray, A: np.ndarray, Bm: np.ndar
     return y, h
 
 
+def ssm_params(cfg, w: Dict[str, np.ndarray], dtl: np.ndarray) -> Tuple[np.ndarray, np.ndarray]:
+    """Delta [L, d_inner] and A [d_inner, N] of the scan from the dt_low rows [L, r].
+
+    Delta = softplus(dt_low W_dt^T + b_dt) and A = -exp(A_log). In the selective form
+    (cfg.ssm_heads == 0) both are per channel, A per (channel, state). In the SSD form
+    ([Lecture 04] section 3: Mamba-2 makes A a scalar times the identity and adds a
+    multi-head structure) W_dt, b_dt and A_log have one entry per SSM head: the head's
+    Delta_t and scalar A serve its d_inner / ssm_heads consecutive channels and all N
+    states, so the same recurrence applies with those values repeated.
+    """
+    delta = softplus(dtl @ w["w_dt"].T + w["b_dt"])
+    A = -np.exp(w["A_log"])
+    nh = getattr(cfg, "ssm_heads", 0)
+    if nh > 0:
+        P = cfg.d_inner // nh
+        delta = np.repeat(delta, P, axis=-1)
+        A = np.repeat(A, P)[:, None] * np.ones((1, cfg.d_state))
+    return delta, A
+
+
 # ----------------------------------------------------------------------------
 # fusion
 # ----------------------------------------------------------------------------
@@ -304,8 +329,7 @@ def mixer_prefill_row(cfg, w: Dict[str, np.ndarray], x: np.ndarray,
     o = attention(q, ka, va, mask).transpose(1, 0, 2).reshape(Tp, H * dv)
     # Mamba heads: conv, Delta, scan, gate
     xc = silu(causal_conv(blocks["x"], w["conv_w"], w["conv_b"]))
-    delta = softplus(blocks["dtl"] @ w["w_dt"].T + w["b_dt"])
-    A = -np.exp(w["A_log"])
+    delta, A = ssm_params(cfg, w, blocks["dtl"])
     y_pre, h = selective_scan(xc, delta, A, blocks["B"], blocks["C"], w["D"])
     y_ssm = y_pre * silu(blocks["z"])
     # fusion and the shared output projection
@@ -433,8 +457,7 @@ def mixer_decode(cfg, w, x_t: np.ndarray, cache: dict, h: np.ndarray, conv: np.n
         # Mamba step: shift the conv state, conv, Delta, one scan step
         conv[b] = np.concatenate([conv[b][:, 1:], blocks["x"].T], axis=1)
         xc = silu(w["conv_b"] + np.sum(w["conv_w"] * conv[b], axis=1))[None, :]
-        delta = softplus(blocks["dtl"] @ w["w_dt"].T + w["b_dt"])
-        A = -np.exp(w["A_log"])
+        delta, A = ssm_params(cfg, w, blocks["dtl"])
         y_pre, h[b] = selective_scan(xc, delta, A, blocks["B"], blocks["C"], w["D"], h[b])
         y_ssm = y_pre * silu(blocks["z"])
         u = fuse_layer(cfg, o, y_ssm, w, cfg.rms_eps)

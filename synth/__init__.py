@@ -11,8 +11,10 @@ the distributions are those of the synthetic workloads):
 
 * X ~ N(0, 1); projection weights ~ N(0, 1/fan_in) (the second argument of N is a
   variance); meta tokens ~ N(0, 0.02).
-* A_log = log(u), u ~ Uniform[1, 16] continuous, iid per (channel, state).
-* dt bias b = softplus^-1(dt), dt = exp(Uniform[ln 1e-3, ln 1e-1]) per channel.
+* A_log = log(u), u ~ Uniform[1, 16] continuous, iid per (channel, state) (per SSM
+  head in the SSD form).
+* dt bias b = softplus^-1(dt), dt = exp(Uniform[ln 1e-3, ln 1e-1]) per channel (per
+  SSM head in the SSD form).
 * conv taps ~ N(0, 1/d_conv), conv bias 0; D = 1; RMSNorm gains 1; beta1 = beta2 = 1.
 """
 from __future__ import annotations
@@ -44,6 +46,13 @@ class LayerCfg:
     rope_base: float = 10000.0
     rms_eps: float = 1e-6
     fusion: int = 0        # 0: beta-average of the two branches; 1: concatenation [Mamba | Attention]
+    ssm_heads: int = 0     # 0: A per (channel, state), Delta per channel; > 0: SSD form, A a scalar
+                           # per SSM head and Delta per head (head dim d_inner / ssm_heads)
+
+    @property
+    def n_dt(self) -> int:
+        """Rows of W_dt (and entries of b_dt): one per channel, or one per SSM head."""
+        return self.ssm_heads if self.ssm_heads > 0 else self.d_inner
 
     @property
     def u_width(self) -> int:
@@ -124,7 +133,8 @@ def layer_weights(cfg: LayerCfg, seed: int) -> Dict[str, np.ndarray]:
     """Random-init weights of one mixer layer, as float32 arrays of storage-exact values.
 
     Big matrices follow the [out, in] convention: w_in [n_in, d_model],
-    w_dt [d_inner, dt_rank], w_out [d_model, d_inner].
+    w_dt [n_dt, dt_rank], w_out [d_model, d_inner]. A_log is [d_inner, d_state], or
+    [ssm_heads] in the SSD form.
     """
     d, di, N, r = cfg.d_model, cfg.d_inner, cfg.d_state, cfg.dt_rank
     H, G, dh, dv = cfg.n_q_heads, cfg.n_kv_heads, cfg.head_dim, cfg.v_head_dim
@@ -138,14 +148,16 @@ def layer_weights(cfg: LayerCfg, seed: int) -> Dict[str, np.ndarray]:
             continue
         rows.append(blk)
     w_in = np.concatenate(rows, axis=0)
-    dt = np.exp(_rng(seed, 2).uniform(np.log(1e-3), np.log(1e-1), size=di))
+    nd = cfg.n_dt
+    dt = np.exp(_rng(seed, 2).uniform(np.log(1e-3), np.log(1e-1), size=nd))
+    a_shape = (cfg.ssm_heads,) if cfg.ssm_heads > 0 else (di, N)
     w = {
         "w_in": to_storage(w_in, cfg.dtype),
-        "w_dt": to_storage(_normal(_rng(seed, 3), (di, r), 1.0 / r), cfg.dtype),
+        "w_dt": to_storage(_normal(_rng(seed, 3), (nd, r), 1.0 / r), cfg.dtype),
         "b_dt": np.log(np.expm1(dt)).astype(np.float32),
         "conv_w": _normal(_rng(seed, 4), (di, cfg.d_conv), 1.0 / cfg.d_conv).astype(np.float32),
         "conv_b": np.zeros(di, np.float32),
-        "A_log": np.log(_rng(seed, 5).uniform(1.0, 16.0, size=(di, N))).astype(np.float32),
+        "A_log": np.log(_rng(seed, 5).uniform(1.0, 16.0, size=a_shape)).astype(np.float32),
         "D": np.ones(di, np.float32),
         "norm_attn_w": np.ones(H * dv, np.float32),
         "norm_ssm_w": np.ones(di, np.float32),
