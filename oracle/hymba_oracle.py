@@ -337,8 +337,11 @@ def mixer_prefill_row(cfg, w: Dict[str, np.ndarray], x: np.ndarray,
     y = u @ w["w_out"].T
     if residual:
         y = y + xh
+    # the decode conv state: the last d_conv pre-conv inputs, oldest first, with the zero
+    # history before the first row when the sequence is shorter than the conv
     K = cfg.d_conv
-    conv_state = blocks["x"][Tp - K:].T.copy() if Tp >= K else None
+    xpad = np.concatenate([np.zeros((K, di)), blocks["x"]], axis=0)
+    conv_state = xpad[-K:].T.copy()
     return dict(y=y, k=k, v=v, h=h, conv=conv_state, o_attn=o, y_ssm=y_ssm, u=u, delta=delta)
 
 

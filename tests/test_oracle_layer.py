@@ -382,3 +382,22 @@ def test_block_decode_equals_block_prefill():
         ya = oracle.block_decode(ca, wa, fa, h[:, m + t], cache, ha, conva)
         yb = oracle.block_decode(cb, wb, fb, ya, cache, hb, convb)
         np.testing.assert_allclose(yb, rb["y"][:, m + t], rtol=1e-10, atol=1e-10)
+
+
+def test_decode_after_a_prefill_shorter_than_the_conv():
+    """A prefill of fewer rows than the conv width (no meta rows, 2 tokens) leaves a conv
+    state whose missing history is zero, so decoding on from it equals prefilling the
+    whole sequence (the zero history before the first row of the prefill)."""
+    cfg = synth.tiny_layer_cfg().with_(n_meta=0, window=8)
+    w = synth.perturbed_weights(synth.layer_weights(cfg, 41), cfg, 41)
+    B, T, T0 = 2, 9, 2
+    x = synth.layer_input(cfg, B, T, 42)
+    ref = oracle.mixer_prefill(cfg, w, x, residual=True)
+    pre = oracle.mixer_prefill(cfg, w, x[:, :T0], residual=True)
+    assert pre["conv"].shape == (B, cfg.d_inner, cfg.d_conv)
+    np.testing.assert_array_equal(pre["conv"][:, :, :cfg.d_conv - T0], 0.0)
+    cache = oracle.cache_from_prefill(cfg, pre["k"], pre["v"], cfg.window)
+    h, conv = pre["h"].copy(), pre["conv"].copy()
+    for t in range(T0, T):
+        y = oracle.mixer_decode(cfg, w, x[:, t], cache, h, conv, residual=True)
+        np.testing.assert_allclose(y, ref["y"][:, t], rtol=1e-10, atol=1e-10)
