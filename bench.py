@@ -38,7 +38,7 @@ sys.path.insert(0, ROOT)
 import synth  # noqa: E402
 
 WORKLOAD = "hymba15_stack32_b8_t4096"
-LAYER_WORKLOADS = ("hymba15_global_b4_t8192", "hymba15_swa1024_b1_t2048")
+LAYER_WORKLOADS = ("hymba15_global_b4_t8192", "hymba15_swa1024_b1_t2048", "hymba15_ssd_swa1024_b8_t4096")
 DECODE_WORKLOAD = "hymba15_decode_pair_b64_p4096"
 
 
@@ -239,17 +239,25 @@ def layer_work(cfg, B, T, has_meta, io_f32):
     # when the input already carries the meta rows)
     in_rows = rows if has_meta else B * T + m
     pairs = visible_pairs(Tp, m, cfg.window)
+    nh = getattr(cfg, "ssm_heads", 0)
     w = {
         "gemm_in_proj": ("tensor", 2.0 * in_rows * cfg.n_in * d),
-        "gemm_dt_proj": ("tensor", 2.0 * rows * di * r),
+        "gemm_dt_proj": ("tensor", 2.0 * rows * (nh if nh > 0 else di) * r),
         "attn_prefill": ("tensor", 2.0 * B * pairs * H * (dh + dv)),
+    }
+    if nh > 0:
+        # SSD form: x read and y_pre written (2 B each per (row, channel)), B and C (64 B)
+        # and the heads' Delta (4 B each) per row
+        w["ssd_scan_prefill"] = ("hbm", rows * (4.0 * di + 64.0 + 4.0 * nh))
+    else:
         # MUFU results: 16 state decays exp2(Delta A), and exp2 + reciprocal of the SiLU,
         # per (row, channel): the scan's binding limit
-        "conv_scan_prefill": ("alu", rows * di * 18.0),
+        w["conv_scan_prefill"] = ("alu", rows * di * 18.0)
+    w.update({
         # O, y_pre, z read, U written: 2 B each per (row, channel)
         "fuse": ("hbm", rows * di * 8.0),
         "gemm_out_proj": ("tensor", 2.0 * rows * d * di),
-    }
+    })
     if io_f32 and cfg.dtype == synth.BF16:
         # fp16 copies of the stream rows (fp32 read, fp16 written) and of W_in, W_out
         # and the meta rows (bf16 read, fp16 written)
@@ -652,7 +660,7 @@ def main():
     ap.add_argument("--clocks-dir", default="",
                     help="where the NVML clock samples are written (default: the system temp directory)")
     ap.add_argument("--no-extra", action="store_true", help="time only the headline workload")
-    ap.add_argument("--only", default="", choices=["", "stack", "global", "swa", "decode"],
+    ap.add_argument("--only", default="", choices=["", "stack", "global", "swa", "ssd", "decode"],
                     help="run one workload alone and print its figures (for profiling runs)")
     ap.add_argument("--decode-prompt", type=int, default=0,
                     help="prompt length of the decode pair's prefill (default: the workload's 4096)")
@@ -705,10 +713,12 @@ def main():
                 args.decode_prompt = 1100
             r = bench_decode(args, torch, hy, rt, max_ranks, barrier, world, pk, flush)
         else:
-            name = {"stack": WORKLOAD, "global": LAYER_WORKLOADS[0], "swa": LAYER_WORKLOADS[1]}[args.only]
+            name = {"stack": WORKLOAD, "global": LAYER_WORKLOADS[0], "swa": LAYER_WORKLOADS[1],
+                    "ssd": LAYER_WORKLOADS[2]}[args.only]
             shrink = None
             if args.small:
-                shrink = {"stack": dict(T=1024, n_layers=2), "global": dict(B=1), "swa": {}}[args.only]
+                shrink = {"stack": dict(T=1024, n_layers=2), "global": dict(B=1), "swa": {},
+                          "ssd": dict(T=1024)}[args.only]
             w1 = PrefillWorkload(name, rank, torch, hy, rt, shrink)
             r = time_prefill(w1, args, torch, hy, barrier, max_ranks, pk, flush, None, sm_count, headline=False)
             r = {"workload": name, "ms_per_step": r["ms"], "tokens_per_s": w1.tokens * world / (r["ms"] * 1e-3),

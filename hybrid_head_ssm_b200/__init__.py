@@ -52,7 +52,8 @@ class hymba_layer_cfg(ctypes.Structure):
     _fields_ = [("d_model", _i32), ("n_q_heads", _i32), ("n_kv_heads", _i32), ("head_dim", _i32),
                 ("v_head_dim", _i32), ("d_inner", _i32), ("d_state", _i32), ("d_conv", _i32),
                 ("dt_rank", _i32), ("n_meta", _i32), ("window", _i32), ("is_kv_producer", _i32),
-                ("dtype", _i32), ("rope_base", _f32), ("rms_eps", _f32), ("fusion", _i32)]
+                ("dtype", _i32), ("rope_base", _f32), ("rms_eps", _f32), ("fusion", _i32),
+                ("ssm_heads", _i32)]
 
 
 class hymba_layer_weights(ctypes.Structure):

@@ -497,7 +497,7 @@ ssm_decode_kernel(const T* __restrict__ P, long long ldP, int col_x, int col_B, 
                   int wide, const float* __restrict__ conv_w, const float* __restrict__ conv_b,
                   const float* __restrict__ A_log, const float* __restrict__ Dp,
                   float* __restrict__ h, float* __restrict__ conv, T* __restrict__ ypre, int B,
-                  int di) {
+                  int di, int hp) {
     griddep_sync();
     using Slot = typename WSlot<TW>::type;
     constexpr int NS = 16, KC = 4;
@@ -598,12 +598,13 @@ ssm_decode_kernel(const T* __restrict__ P, long long ldP, int col_x, int col_B, 
             if (q0) __syncthreads();
             for (int cc = warp; cc < SSM_CH; cc += SSM_WARPS) {
                 const int ch = c0 + cc;
+                const long long wrow = hp > 0 ? ch / hp : ch;  // SSD form: the head's row
                 for (int q = lane; q < nq; q += 32) {
                     const int j = 2 * (q0 + q);
                     TW lo = wz, hi = wz;
                     if (ch < di) {
-                        lo = w_dt[(long long)ch * r + j];
-                        if (j + 1 < r) hi = w_dt[(long long)ch * r + j + 1];
+                        lo = w_dt[wrow * r + j];
+                        if (j + 1 < r) hi = w_dt[wrow * r + j + 1];
                     }
                     Ws[cc * RS + q] = wpack(lo, hi);
                 }
@@ -632,15 +633,22 @@ ssm_decode_kernel(const T* __restrict__ P, long long ldP, int col_x, int col_B, 
     if (!cok) return;
     // per-channel constants, shared by the thread's sequences
     const float4 w4 = *reinterpret_cast<const float4*>(conv_w + (long long)c * KC);
-    const float cb = conv_b[c], bdt = b_dt[c], Dc = Dp[c];
+    const float cb = conv_b[c], bdt = b_dt[hp > 0 ? c / hp : c], Dc = Dp[c];
     float Ae[NS];  // -exp(A_log) log2(e): exp(Delta A) = exp2(Delta Ae)
+    if (hp > 0) {
+        // SSD form: one A per head, for every state
+        const float a = -fast_exp2(A_log[c / hp] * LOG2E) * LOG2E;
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
-        const float4 a4 = *reinterpret_cast<const float4*>(A_log + (long long)c * NS + 4 * k);
-        Ae[4 * k] = -fast_exp2(a4.x * LOG2E) * LOG2E;
-        Ae[4 * k + 1] = -fast_exp2(a4.y * LOG2E) * LOG2E;
-        Ae[4 * k + 2] = -fast_exp2(a4.z * LOG2E) * LOG2E;
-        Ae[4 * k + 3] = -fast_exp2(a4.w * LOG2E) * LOG2E;
+        for (int n = 0; n < NS; ++n) Ae[n] = a;
+    } else {
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const float4 a4 = *reinterpret_cast<const float4*>(A_log + (long long)c * NS + 4 * k);
+            Ae[4 * k] = -fast_exp2(a4.x * LOG2E) * LOG2E;
+            Ae[4 * k + 1] = -fast_exp2(a4.y * LOG2E) * LOG2E;
+            Ae[4 * k + 2] = -fast_exp2(a4.z * LOG2E) * LOG2E;
+            Ae[4 * k + 3] = -fast_exp2(a4.w * LOG2E) * LOG2E;
+        }
     }
 #pragma unroll
     for (int u = 0; u < SSM_RPT; ++u) {
@@ -776,9 +784,9 @@ template <typename T, typename TW>
 int launch_ssm_decode(const Ctx& ctx, const T* P, long long ldP, int col_x, int col_B, int col_C,
                       int col_dtl, const TW* w_dt, const float* b_dt, int dt_rank,
                       const float* conv_w, const float* conv_b, const float* A_log, const float* D,
-                      float* h, float* conv, T* ypre, int B, int di) {
+                      float* h, float* conv, T* ypre, int B, int di, int hp) {
     if (B <= 0) return HYMBA_OK;
-    if (dt_rank <= 0) return HYMBA_ERR_INVALID_ARG;
+    if (dt_rank <= 0 || hp < 0 || (hp > 0 && di % hp)) return HYMBA_ERR_INVALID_ARG;
     // 16-byte loads: the B/C columns of every projection row, conv taps, A_log and conv state
     constexpr int V = 16 / (int)sizeof(T);
     if (ldP % V || col_B % V || col_C % V || (reinterpret_cast<uintptr_t>(conv_w) & 15) ||
@@ -793,13 +801,13 @@ int launch_ssm_decode(const Ctx& ctx, const T* P, long long ldP, int col_x, int 
     // one-pass wide staging: 16-bit W_dt with even dt_rank <= 128 (so the block's run of
     // 32 rows is 16-byte aligned and a whole number of 16-byte pieces, d_inner being a
     // multiple of 32), 4-byte dt_low pairs
-    const int wide = sizeof(TW) == 2 && dt_rank % 2 == 0 && npairs <= SSM_PAIRS && di % SSM_CH == 0 &&
+    const int wide = hp == 0 && sizeof(TW) == 2 && dt_rank % 2 == 0 && npairs <= SSM_PAIRS && di % SSM_CH == 0 &&
                      (reinterpret_cast<uintptr_t>(w_dt) & 15) == 0 && col_dtl % 2 == 0 &&
                      SSM_CH * npairs / 4 <= SSM_WLD * SSM_WARPS * 32 && SSM_ROWS * npairs <= SSM_XLD * SSM_WARPS * 32;
     dim3 grid(ceil_div(di, SSM_CH), ceil_div(B, SSM_ROWS));
     HYMBA_LAUNCH(ctx, "ssm_decode", (ssm_decode_kernel<T, TW>), grid, SSM_WARPS * 32, smem, P, ldP, col_x,
                  col_B, col_C, col_dtl, w_dt, b_dt, dt_rank, wide, conv_w, conv_b, A_log, D, h, conv, ypre, B,
-                 di);
+                 di, hp);
     return HYMBA_OK;
 }
 
@@ -811,9 +819,9 @@ template int launch_attn_decode<f16>(const Ctx&, const f16*, long long, const f1
                                      int, int);
 template int launch_ssm_decode<float, float>(const Ctx&, const float*, long long, int, int, int, int,
                                              const float*, const float*, int, const float*, const float*,
-                                             const float*, const float*, float*, float*, float*, int, int);
+                                             const float*, const float*, float*, float*, float*, int, int, int);
 template int launch_ssm_decode<f16, bf16>(const Ctx&, const f16*, long long, int, int, int, int,
                                           const bf16*, const float*, int, const float*, const float*,
-                                          const float*, const float*, float*, float*, f16*, int, int);
+                                          const float*, const float*, float*, float*, f16*, int, int, int);
 
 }  // namespace hymba

@@ -206,6 +206,182 @@ fuse_kernel(const I* __restrict__ O, const float* __restrict__ part, int n_split
     if (len_inc && live && t == 0) len_inc[row] += 1;
 }
 
+// An 8-element piece of an input row as loaded (16-bit: one 16-byte word; fp32: two).
+template <typename I>
+struct Piece {
+    uint4 v[sizeof(I) / 2];
+};
+
+template <typename I>
+__device__ __forceinline__ void load_piece(Piece<I>& p, const I* src) {
+#pragma unroll
+    for (int i = 0; i < (int)(sizeof(I) / 2); ++i) p.v[i] = reinterpret_cast<const uint4*>(src)[i];
+}
+
+template <typename I>
+__device__ __forceinline__ void unpack_piece(const Piece<I>& p, float* v) {
+    if constexpr (sizeof(I) == 2) {
+        const I* h = reinterpret_cast<const I*>(&p.v[0]);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) v[i] = to_f(h[i]);
+    } else {
+        const float* f = reinterpret_cast<const float*>(&p.v[0]);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) v[i] = f[i];
+    }
+}
+
+template <typename I>
+__device__ __forceinline__ void pack_piece(Piece<I>& p, const float* v) {
+    if constexpr (sizeof(I) == 2) {
+        p.v[0] = make_uint4(pack2<I>(v[0], v[1]), pack2<I>(v[2], v[3]), pack2<I>(v[4], v[5]), pack2<I>(v[6], v[7]));
+    } else {
+        p.v[0] = make_uint4(__float_as_uint(v[0]), __float_as_uint(v[1]), __float_as_uint(v[2]), __float_as_uint(v[3]));
+        p.v[1] = make_uint4(__float_as_uint(v[4]), __float_as_uint(v[5]), __float_as_uint(v[6]), __float_as_uint(v[7]));
+    }
+}
+
+// Prefill fusion, persistent over rows: block b takes rows b, b + grid, ... and loads the
+// next row's pieces into registers before working on the current one, so every block
+// keeps a row of loads in flight through its reductions and stores (a row kernel that
+// loads, reduces and stores in turn leaves HBM idle while it reduces). The per-channel
+// factors beta * gain (halved for the average) are formed once per block in shared
+// memory. The gated Mamba branch is kept between the two passes in the intermediate
+// type (fp16 for 16-bit layers: the normalised result is written as bf16 or fp16).
+template <typename I, typename T, bool CONCAT>
+__global__ void __launch_bounds__(TPR, 3)
+fuse_rows_kernel(const I* __restrict__ O, int H, int dv, const I* __restrict__ ypre, const I* __restrict__ P,
+                 long long ldP, int col_z, const float* __restrict__ g_attn, const float* __restrict__ g_ssm,
+                 const float* __restrict__ beta1, const float* __restrict__ beta2, const float* __restrict__ v_scale,
+                 const float* __restrict__ v_bias, int rep, T* __restrict__ U, long long rows, int di, float eps) {
+    constexpr bool PF = sizeof(I) == 2;  // prefetch the next row (16-bit inputs: few registers per piece)
+    extern __shared__ float fac[];        // [hv] attention factors, then [di] Mamba factors
+    __shared__ float red[2][TPR / 32][2];
+    griddep_sync();
+    const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
+    const int hv = H * dv, nvo = hv / 8, nvy = di / 8;
+    const float half = CONCAT ? 1.0f : 0.5f;  // the average halves both branches
+    for (int c = t; c < hv; c += TPR) fac[c] = half * beta1[c] * g_attn[c];
+    for (int c = t; c < di; c += TPR) fac[hv + c] = half * beta2[c] * g_ssm[c];
+    __syncthreads();
+    const long long ldu = CONCAT ? (long long)di + hv : di;
+
+    Piece<I> po[VMAX], py[VMAX], pz[VMAX];
+    auto load_row = [&](long long r, Piece<I>* a, Piece<I>* b, Piece<I>* z) {
+#pragma unroll
+        for (int k = 0; k < VMAX; ++k) {
+            const int vi = t + k * TPR;
+            if (vi < nvo) load_piece<I>(a[k], O + r * hv + vi * 8);
+            if (vi < nvy) {
+                load_piece<I>(b[k], ypre + r * di + vi * 8);
+                load_piece<I>(z[k], P + r * ldP + col_z + vi * 8);
+            }
+        }
+    };
+    long long row = blockIdx.x;
+    if (PF && row < rows) load_row(row, po, py, pz);
+    for (int it = 0; row < rows; ++it, row += gridDim.x) {
+        Piece<I> no[VMAX], ny[VMAX], nz[VMAX];
+        const long long nrow = row + gridDim.x;
+        if (PF) {
+            if (nrow < rows) load_row(nrow, no, ny, nz);
+        } else {
+            load_row(row, po, py, pz);
+        }
+        // pass 1: the consumer's V transform, the gate, both sums of squares
+        float ss_o = 0.f, ss_y = 0.f;
+#pragma unroll
+        for (int k = 0; k < VMAX; ++k) {
+            const int vi = t + k * TPR;
+            if (vi < nvo) {
+                float o[8];
+                unpack_piece<I>(po[k], o);
+                if (v_scale) {
+                    // attention over V * s + b is the attention output * s + b (weights sum to 1)
+                    const int c = vi * 8, hd = c / dv;
+                    const int idx = (hd / rep) * dv + (c - hd * dv);
+                    float vs[8], vb[8];
+                    load8f(v_scale + idx, vs);
+                    load8f(v_bias + idx, vb);
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) o[i] = fmaf(o[i], vs[i], vb[i]);
+                    pack_piece<I>(po[k], o);
+                    unpack_piece<I>(po[k], o);  // normalise what is kept
+                }
+#pragma unroll
+                for (int i = 0; i < 8; ++i) ss_o = fmaf(o[i], o[i], ss_o);
+            }
+            if (vi < nvy) {
+                float y[8], z[8];
+                unpack_piece<I>(py[k], y);
+                unpack_piece<I>(pz[k], z);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) y[i] *= z[i] / (1.0f + __expf(-z[i]));
+                pack_piece<I>(py[k], y);
+                unpack_piece<I>(py[k], y);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) ss_y = fmaf(y[i], y[i], ss_y);
+            }
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) {
+            ss_o += __shfl_xor_sync(0xffffffffu, ss_o, off);
+            ss_y += __shfl_xor_sync(0xffffffffu, ss_y, off);
+        }
+        if (lane == 0) {
+            red[it & 1][warp][0] = ss_o;
+            red[it & 1][warp][1] = ss_y;
+        }
+        __syncthreads();  // (the other buffer was last read before the previous barrier)
+        ss_o = 0.f;
+        ss_y = 0.f;
+#pragma unroll
+        for (int w = 0; w < TPR / 32; ++w) {
+            ss_o += red[it & 1][w][0];
+            ss_y += red[it & 1][w][1];
+        }
+        const float ro = rsqrtf(ss_o / hv + eps);
+        const float ry = rsqrtf(ss_y / di + eps);
+        // pass 2: scale, combine, store
+#pragma unroll
+        for (int k = 0; k < VMAX; ++k) {
+            const int vi = t + k * TPR;
+            const int c = vi * 8;
+            if constexpr (CONCAT) {
+                if (vi < nvy) {
+                    float y[8], u[8];
+                    unpack_piece<I>(py[k], y);
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) u[i] = fac[hv + c + i] * y[i] * ry;
+                    store8<T>(U + row * ldu + c, u);
+                }
+                if (vi < nvo) {
+                    float o[8], u[8];
+                    unpack_piece<I>(po[k], o);
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) u[i] = fac[c + i] * o[i] * ro;
+                    store8<T>(U + row * ldu + di + c, u);
+                }
+            } else if (vi < nvy) {
+                float o[8], y[8], u[8];
+                unpack_piece<I>(po[k], o);
+                unpack_piece<I>(py[k], y);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) u[i] = fmaf(fac[c + i] * ro, o[i], fac[hv + c + i] * ry * y[i]);
+                store8<T>(U + row * ldu + c, u);
+            }
+        }
+        if (PF) {
+#pragma unroll
+            for (int k = 0; k < VMAX; ++k) {
+                po[k] = no[k];
+                py[k] = ny[k];
+                pz[k] = nz[k];
+            }
+        }
+    }
+}
+
 }  // namespace
 
 template <typename I, typename T, bool CONCAT>
@@ -218,9 +394,13 @@ static int fuse_variant(const Ctx& ctx, const I* O, const float* part, int n_spl
         HYMBA_LAUNCH(ctx, "fuse", kern, ceil_div(rows, RPB), TPR * RPB, 0, O, part, n_split, H, dv, ypre, P, ldP,
                      col_z, g_attn, g_ssm, beta1, beta2, v_scale, v_bias, H / G, U, rows, di, eps, len_inc);
     } else {
-        auto kern = fuse_kernel<I, T, false, CONCAT>;
-        HYMBA_LAUNCH(ctx, "fuse", kern, ceil_div(rows, RPB), TPR * RPB, 0, O, part, n_split, H, dv, ypre, P, ldP,
-                     col_z, g_attn, g_ssm, beta1, beta2, v_scale, v_bias, H / G, U, rows, di, eps, len_inc);
+        auto kern = fuse_rows_kernel<I, T, CONCAT>;
+        const size_t smem = (size_t)(H * dv + di) * sizeof(float);
+        static std::atomic<unsigned long long> smem_set{0};
+        if (smem > 48 * 1024 && !smem_opt_in_once(smem_set, kern, smem, ctx)) return HYMBA_ERR_CUDA;
+        const int grid = (int)std::min<long long>(rows, 3LL * (ctx.sm_count > 0 ? ctx.sm_count : 148));
+        HYMBA_LAUNCH(ctx, "fuse", kern, grid, TPR, smem, O, H, dv, ypre, P, ldP, col_z, g_attn, g_ssm, beta1, beta2,
+                     v_scale, v_bias, H / G, U, (long long)rows, di, eps);
     }
     return HYMBA_OK;
 }

@@ -132,8 +132,19 @@ static int check_cfg(const hymba_layer_cfg* c) {
     if (c->fusion == HYMBA_FUSION_AVERAGE && hv != c->d_inner) return HYMBA_ERR_UNSUPPORTED;
     if (c->d_model % 64 || c->d_inner % 64 || hv % 64) return HYMBA_ERR_UNSUPPORTED;
     if (c->d_inner > 4096 || hv > 4096) return HYMBA_ERR_UNSUPPORTED;
+    if (c->ssm_heads < 0 || (c->ssm_heads > 0 && c->d_inner % c->ssm_heads)) return HYMBA_ERR_INVALID_ARG;
+    if (c->ssm_heads > 0) {
+        const int hp = c->d_inner / c->ssm_heads;
+        if (hp % 8) return HYMBA_ERR_UNSUPPORTED;
+        if (c->dtype == HYMBA_BF16 && !ssd_scan_applies(c->d_inner, c->ssm_heads)) return HYMBA_ERR_UNSUPPORTED;
+    }
     return HYMBA_OK;
 }
+
+// Rows of W_dt: one per channel, or one per SSM head in the SSD form.
+static int n_dt(const hymba_layer_cfg* c) { return c->ssm_heads > 0 ? c->ssm_heads : c->d_inner; }
+// Channels per SSM head (0: the selective form).
+static int ssm_hp(const hymba_layer_cfg* c) { return c->ssm_heads > 0 ? c->d_inner / c->ssm_heads : 0; }
 
 // Width of the fused branches, the input of W_o.
 static int u_width(const hymba_layer_cfg* c) {
@@ -321,7 +332,7 @@ static int prefill_impl(const Ctx& ctx, const hymba_layer_cfg* c, const hymba_la
         W_out = static_cast<const T*>(w->w_out);
     }
     // RoPE table and the padded 16-bit W_dt of step 2, one launch
-    if ((rc = launch_prefill_prep<T, I>(ctx, rope, Tp, dh, c->rope_base, static_cast<const T*>(w->w_dt), di,
+    if ((rc = launch_prefill_prep<T, I>(ctx, rope, Tp, dh, c->rope_base, static_cast<const T*>(w->w_dt), n_dt(c),
                                         c->dt_rank, wdt, pl.rpad)))
         return rc;
     // 1. fused input projection (+ RoPE, K/V scatter) ------------------------------
@@ -362,11 +373,14 @@ static int prefill_impl(const Ctx& ctx, const hymba_layer_cfg* c, const hymba_la
     }
     // 2. Delta = softplus(dt_low W_dt^T + b_dt), or inside the scan (step 4) when the
     // batch is wide enough for the one-thread-per-channel scan ------------------------
-    const bool fold = std::is_same<I, f16>::value && scan_wide_applies(B, di, c->dt_rank, ctx.sm_count);
+    const bool fold = std::is_same<I, f16>::value && c->ssm_heads == 0 &&
+                      scan_wide_applies(B, di, c->dt_rank, ctx.sm_count);
     if (!fold) {
-        EpiArgs<I> ed = epi_base<I>(EPI_DELTA, (int)rows, di);
+        // [rows, n_dt]: per channel, or per SSM head in the SSD form
+        EpiArgs<I> ed = epi_base<I>(EPI_DELTA, (int)rows, n_dt(c));
         ed.delta = delta; ed.b_dt = w->b_dt;
-        if ((rc = gemm<I, I>(ctx, "gemm_dt_proj", P + k.dtl, pl.ldP, wdt, pl.rpad, (int)rows, di, c->dt_rank, ed)))
+        if ((rc = gemm<I, I>(ctx, "gemm_dt_proj", P + k.dtl, pl.ldP, wdt, pl.rpad, (int)rows, n_dt(c), c->dt_rank,
+                             ed)))
             return rc;
     }
     // 3. attention heads ---------------------------------------------------------
@@ -375,7 +389,14 @@ static int prefill_impl(const Ctx& ctx, const hymba_layer_cfg* c, const hymba_la
     // 4. Mamba heads ---------------------------------------------------------------
     bool scanned = false;
     if constexpr (std::is_same<I, f16>::value) {
-        if (fold) {
+        if (c->ssm_heads > 0) {
+            // SSD form: chunked matmuls on the tensor cores
+            if ((rc = launch_ssd_scan(ctx, P, pl.ldP, k.x, k.Bc, delta, n_dt(c), w->conv_w, w->conv_b, w->A_log,
+                                      w->D, ypre, st ? st->h : nullptr, st ? st->conv : nullptr, B, Tp, di,
+                                      c->ssm_heads)))
+                return rc;
+            scanned = true;
+        } else if (fold) {
             if ((rc = launch_conv_scan_wide(ctx, P, pl.ldP, k.x, k.Bc, k.dtl, c->dt_rank, wdt, pl.rpad, w->b_dt,
                                             w->conv_w, w->conv_b, w->A_log, w->D, ypre, st ? st->h : nullptr,
                                             st ? st->conv : nullptr, B, Tp, di)))
@@ -385,7 +406,7 @@ static int prefill_impl(const Ctx& ctx, const hymba_layer_cfg* c, const hymba_la
     }
     if (!scanned && (rc = launch_conv_scan_prefill<I>(ctx, P, pl.ldP, k.x, k.Bc, k.Cc, delta, w->conv_w, w->conv_b,
                                                       w->A_log, w->D, ypre, st ? st->h : nullptr,
-                                                      st ? st->conv : nullptr, B, Tp, di)))
+                                                      st ? st->conv : nullptr, B, Tp, di, ssm_hp(c))))
         return rc;
     // 5. gate, norms, beta, average (or concatenation) ----------------------------------
     // 6. output projection (+ residual) -------------------------------------------------
@@ -487,7 +508,7 @@ static int decode_impl(const Ctx& ctx, const hymba_layer_cfg* c, const hymba_lay
     // SSM step with the Delta projection of the new rows folded in
     if ((rc = launch_ssm_decode<I, T>(ctx, P, pl.ldP, k.x, k.Bc, k.Cc, k.dtl, static_cast<const T*>(w->w_dt),
                                       w->b_dt, c->dt_rank, w->conv_w, w->conv_b, w->A_log, w->D, st->h,
-                                      st->conv, ypre, B, di)))
+                                      st->conv, ypre, B, di, ssm_hp(c))))
         return rc;
     const bool concat = c->fusion == HYMBA_FUSION_CONCAT;
     EpiArgs<TIO> eo = epi_base<TIO>(EPI_OUT, B, d);

@@ -34,12 +34,13 @@ int launch_attn_prefill_tc(const Ctx& ctx, const f16* P, long long ldP, const f1
                            int dv, int n_meta, int window);
 
 // Depthwise causal conv + SiLU + selective scan over the T' rows of every sequence,
-// Delta from `delta` [rows, di] fp32.
+// Delta from `delta` [rows, di] fp32; hp > 0 (the SSD form, hp channels per head, a
+// multiple of 8): `delta` [rows, di / hp] and A_log [di / hp], one value per head.
 template <typename T>
 int launch_conv_scan_prefill(const Ctx& ctx, const T* P, long long ldP, int col_x, int col_B,
                              int col_C, const float* delta, const float* conv_w,
                              const float* conv_b, const float* A_log, const float* D, T* ypre,
-                             float* h_out, float* conv_out, int B, int Tp, int di);
+                             float* h_out, float* conv_out, int B, int Tp, int di, int hp);
 
 // The same for 16-bit intermediates with Delta computed in the kernel (dt_rank <= 128, a
 // multiple of 4), one thread per channel pair and state half: for batches where
@@ -49,6 +50,13 @@ int launch_conv_scan_wide(const Ctx& ctx, const f16* P, long long ldP, int col_x
                           const f16* wdt, int ld_wdt, const float* b_dt, const float* conv_w, const float* conv_b,
                           const float* A_log, const float* D, f16* ypre, float* h_out, float* conv_out, int B, int Tp,
                           int di);
+
+// conv + SiLU and the SSD-form scan (scalar A and Delta per SSM head of 64 channels) as
+// chunked tensor-core matmuls, fp16 operands; delta [rows, ld_delta] per head.
+bool ssd_scan_applies(int di, int ssm_heads);
+int launch_ssd_scan(const Ctx& ctx, const f16* P, long long ldP, int col_x, int col_B, const float* delta,
+                    int ld_delta, const float* conv_w, const float* conv_b, const float* A_log, const float* D,
+                    f16* ypre, float* h_out, float* conv_out, int B, int Tp, int di, int ssm_heads);
 
 // RMSNorm of both branches, SiLU(z) gate, beta scaling and average (U [rows, di]) or
 // concatenation (U [rows, di + H*dv] = [Mamba | attention]); one row per block.
@@ -108,6 +116,6 @@ template <typename T, typename TW>
 int launch_ssm_decode(const Ctx& ctx, const T* P, long long ldP, int col_x, int col_B, int col_C,
                       int col_dtl, const TW* w_dt, const float* b_dt, int dt_rank,
                       const float* conv_w, const float* conv_b, const float* A_log, const float* D,
-                      float* h, float* conv, T* ypre, int B, int di);
+                      float* h, float* conv, T* ypre, int B, int di, int hp);
 
 }  // namespace hymba

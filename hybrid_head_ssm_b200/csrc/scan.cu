@@ -103,8 +103,8 @@ __device__ __forceinline__ void load8x2(const T* p, float2* v) {
 // zeroed when unpacked).
 template <typename T>
 __device__ __forceinline__ void stage_chunk(Raw<T>& r, int h, const T* P, long long ldP, int col_x, int col_B,
-                                            int col_C, const float* delta, int di, int c0, long long row0, int t0,
-                                            int Tp) {
+                                            int col_C, const float* delta, int di, int hp, int c0, long long row0,
+                                            int t0, int Tp) {
     constexpr int XV = CPB * (int)sizeof(T) / 16;
     constexpr int DV = CPB * 4 / 16;
     constexpr int BV = 16 * (int)sizeof(T) / 16;
@@ -115,12 +115,23 @@ __device__ __forceinline__ void stage_chunk(Raw<T>& r, int h, const T* P, long l
         cp_async16(reinterpret_cast<char*>(&r.x[rr + KC - 1][0]) + 16 * k,
                    reinterpret_cast<const char*>(P + row * ldP + col_x + c0) + 16 * k);
     }
+    if (hp > 0) {
+        // SSD form: one Delta per row for the block's head ([rows, di / hp])
+        for (int j = h; j < TC; j += NHELP) {
+            const long long row = row0 + min(t0 + j, Tp - 1);
+            asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(
+                             static_cast<uint32_t>(__cvta_generic_to_shared(&r.d[j][0]))),
+                         "l"(delta + row * (di / hp) + c0 / hp)
+                         : "memory");
+        }
+    } else {
 #pragma unroll
-    for (int j = h; j < TC * DV; j += NHELP) {
-        const int rr = j / DV, k = j % DV;
-        const long long row = row0 + min(t0 + rr, Tp - 1);
-        cp_async16(reinterpret_cast<char*>(&r.d[rr][0]) + 16 * k,
-                   reinterpret_cast<const char*>(delta + row * di + c0) + 16 * k);
+        for (int j = h; j < TC * DV; j += NHELP) {
+            const int rr = j / DV, k = j % DV;
+            const long long row = row0 + min(t0 + rr, Tp - 1);
+            cp_async16(reinterpret_cast<char*>(&r.d[rr][0]) + 16 * k,
+                       reinterpret_cast<const char*>(delta + row * di + c0) + 16 * k);
+        }
     }
 #pragma unroll
     for (int j = h; j < TC * BV; j += NHELP) {
@@ -137,7 +148,7 @@ __device__ __forceinline__ void stage_chunk(Raw<T>& r, int h, const T* P, long l
 // 4 * (h & 1) .. +3: conv + SiLU, the (Delta, Delta*xc) pairs, D xc and the B/C quads
 // into operand buffer `buf`.
 template <typename T>
-__device__ __forceinline__ void unpack_chunk(Smem<T>& sm, const Raw<T>& r, int buf, int h, int nt) {
+__device__ __forceinline__ void unpack_chunk(Smem<T>& sm, const Raw<T>& r, int buf, int h, int nt, int hp) {
     const int t = h >> 1, hf = h & 1;
     float2 acc[2] = {sm.w2[KC][2 * hf], sm.w2[KC][2 * hf + 1]};
 #pragma unroll
@@ -147,7 +158,8 @@ __device__ __forceinline__ void unpack_chunk(Smem<T>& sm, const Raw<T>& r, int b
 #pragma unroll
         for (int j = 0; j < 2; ++j) acc[j] = __ffma2_rn(sm.w2[q][2 * hf + j], hf ? xv[2 + j] : xv[j], acc[j]);
     }
-    const float4 dq = *reinterpret_cast<const float4*>(&r.d[t][4 * hf]);
+    const float4 dq = hp > 0 ? make_float4(r.d[t][0], r.d[t][0], r.d[t][0], r.d[t][0])
+                             : *reinterpret_cast<const float4*>(&r.d[t][4 * hf]);
     const float keep = t < nt ? 1.f : 0.f;
     const float2 dl[2] = {make_float2(dq.x * keep, dq.y * keep), make_float2(dq.z * keep, dq.w * keep)};
     float2 xdv[2];
@@ -207,7 +219,7 @@ __global__ void __launch_bounds__(NTH)
 conv_scan_prefill_kernel(const T* __restrict__ P, long long ldP, int col_x, int col_B, int col_C, const float* __restrict__ delta,
             const float* __restrict__ conv_w, const float* __restrict__ conv_b, const float* __restrict__ A_log,
             const float* __restrict__ Dp, T* __restrict__ ypre, float* __restrict__ h_out,
-            float* __restrict__ conv_out, int Tp, int di) {
+            float* __restrict__ conv_out, int Tp, int di, int hp) {
     griddep_sync();
     extern __shared__ __align__(16) uint8_t smem_raw[];
     Smem<T>& sm = *reinterpret_cast<Smem<T>*>(smem_raw);
@@ -231,8 +243,8 @@ conv_scan_prefill_kernel(const T* __restrict__ P, long long ldP, int col_x, int 
     // prologue (helpers): stage chunks 0 and 1, zero halo of chunk 0
     if (!scanner) {
         if (h < (KC - 1) * CPB) sm.raw[0].x[h / CPB][h % CPB] = from_f<T>(0.f);
-        stage_chunk<T>(sm.raw[0], h, P, ldP, col_x, col_B, col_C, delta, di, c0, row0, 0, Tp);
-        if (nchunk > 1) stage_chunk<T>(sm.raw[1], h, P, ldP, col_x, col_B, col_C, delta, di, c0, row0, TC, Tp);
+        stage_chunk<T>(sm.raw[0], h, P, ldP, col_x, col_B, col_C, delta, di, hp, c0, row0, 0, Tp);
+        if (nchunk > 1) stage_chunk<T>(sm.raw[1], h, P, ldP, col_x, col_B, col_C, delta, di, hp, c0, row0, TC, Tp);
         cp_async_commit();
         cp_async_wait0();
     }
@@ -244,15 +256,21 @@ conv_scan_prefill_kernel(const T* __restrict__ P, long long ldP, int col_x, int 
 #pragma unroll
             for (int i = 0; i < CPB * (int)sizeof(T) / 16; ++i) dst[i] = src[i];
         }
-        unpack_chunk<T>(sm, sm.raw[0], 0, h, nt_of(0));
+        unpack_chunk<T>(sm, sm.raw[0], 0, h, nt_of(0), hp);
     }
     __syncthreads();  // chunk 0 unpacked, chunk 1's halo in place
 
     const int cl = tid / TPC, p = tid % TPC;
     float2 A2 = make_float2(0.f, 0.f), hs = make_float2(0.f, 0.f);
-    if (scanner)
-        A2 = make_float2(-expf(A_log[(long long)(c0 + cl) * 16 + 2 * p]) * LOG2E,
-                         -expf(A_log[(long long)(c0 + cl) * 16 + 2 * p + 1]) * LOG2E);
+    if (scanner) {
+        if (hp > 0) {  // SSD form: one A per head, for every state
+            const float a = -expf(A_log[(c0 + cl) / hp]) * LOG2E;
+            A2 = make_float2(a, a);
+        } else {
+            A2 = make_float2(-expf(A_log[(long long)(c0 + cl) * 16 + 2 * p]) * LOG2E,
+                             -expf(A_log[(long long)(c0 + cl) * 16 + 2 * p + 1]) * LOG2E);
+        }
+    }
     for (int k = 0; k < nchunk; ++k) {
         const int buf = k & 1;
         if (scanner) {
@@ -301,7 +319,7 @@ conv_scan_prefill_kernel(const T* __restrict__ P, long long ldP, int col_x, int 
         } else {
             // stage k+2, halo of k+2, unpack k+1, reduce k-1
             if (k + 2 < nchunk)
-                stage_chunk<T>(sm.raw[(k + 2) % NRAW], h, P, ldP, col_x, col_B, col_C, delta, di, c0, row0,
+                stage_chunk<T>(sm.raw[(k + 2) % NRAW], h, P, ldP, col_x, col_B, col_C, delta, di, hp, c0, row0,
                                (k + 2) * TC, Tp);
             cp_async_commit();
             if (k + 2 < nchunk && h < KC - 1) {
@@ -313,7 +331,7 @@ conv_scan_prefill_kernel(const T* __restrict__ P, long long ldP, int col_x, int 
             // reduce k-1 before unpacking k+1 into the same buffers (each helper reads and
             // then rewrites only its own row and channels of xd)
             if (k >= 1) reduce_chunk<T>(sm, buf ^ 1, h, nt_of(k - 1), ypre, row0, (k - 1) * TC, di, c0);
-            if (k + 1 < nchunk) unpack_chunk<T>(sm, sm.raw[(k + 1) % NRAW], buf ^ 1, h, nt_of(k + 1));
+            if (k + 1 < nchunk) unpack_chunk<T>(sm, sm.raw[(k + 1) % NRAW], buf ^ 1, h, nt_of(k + 1), hp);
             if (k + 1 == nchunk && conv_out && h < KC * CPB) {
                 // conv state: the last KC inputs of the sequence, oldest first
                 const int q = h / CPB, cc = h % CPB;
@@ -337,23 +355,26 @@ conv_scan_prefill_kernel(const T* __restrict__ P, long long ldP, int col_x, int 
 template <typename T>
 int launch_conv_scan_prefill(const Ctx& ctx, const T* P, long long ldP, int col_x, int col_B, int col_C,
                              const float* delta, const float* conv_w, const float* conv_b, const float* A_log,
-                             const float* D, T* ypre, float* h_out, float* conv_out, int B, int Tp, int di) {
-    if (di % CPB || (col_x % 8) || (col_B % 8) || (col_C % 8) || (ldP % 8)) return HYMBA_ERR_UNSUPPORTED;
+                             const float* D, T* ypre, float* h_out, float* conv_out, int B, int Tp, int di,
+                             int hp) {
+    if (di % CPB || (col_x % 8) || (col_B % 8) || (col_C % 8) || (ldP % 8) || hp < 0 ||
+        (hp > 0 && (hp % CPB || di % hp)))
+        return HYMBA_ERR_UNSUPPORTED;
     dim3 grid(di / CPB, B);
     const size_t smem = sizeof(Smem<T>);
     auto kern = conv_scan_prefill_kernel<T>;
     static std::atomic<unsigned long long> smem_set{0};
     if (!smem_opt_in_once(smem_set, kern, smem, ctx)) return HYMBA_ERR_CUDA;
     HYMBA_LAUNCH(ctx, "conv_scan_prefill", kern, grid, NTH, smem, P, ldP, col_x, col_B, col_C, delta, conv_w, conv_b,
-                 A_log, D, ypre, h_out, conv_out, Tp, di);
+                 A_log, D, ypre, h_out, conv_out, Tp, di, hp);
     return HYMBA_OK;
 }
 
 template int launch_conv_scan_prefill<float>(const Ctx&, const float*, long long, int, int, int, const float*,
                                              const float*, const float*, const float*, const float*, float*, float*,
-                                             float*, int, int, int);
+                                             float*, int, int, int, int);
 template int launch_conv_scan_prefill<f16>(const Ctx&, const f16*, long long, int, int, int, const float*,
                                            const float*, const float*, const float*, const float*, f16*, float*,
-                                           float*, int, int, int);
+                                           float*, int, int, int, int);
 
 }  // namespace hymba

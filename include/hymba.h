@@ -113,6 +113,15 @@ typedef struct hymba_layer_cfg {
     float   rope_base;
     float   rms_eps;
     int32_t fusion;          /* HYMBA_FUSION_AVERAGE or HYMBA_FUSION_CONCAT */
+    /* 0: the selective form, A per (channel, state) and Delta per channel. > 0: the SSD
+     * form ("Lecture 04 - Beyond the Dense Transformer", section 3: Mamba-2 makes A a
+     * scalar times the identity and gives the SSM a multi-head structure): the channels
+     * split into ssm_heads heads of d_inner / ssm_heads consecutive channels, and
+     * W_dt, b_dt and A_log hold one entry per head (Delta_t and A shared by the head's
+     * channels and all states). The head width must be a multiple of 8, and exactly 64
+     * for HYMBA_BF16 (whose prefill computes the chunked matmul form on the tensor
+     * cores); otherwise HYMBA_ERR_UNSUPPORTED. */
+    int32_t ssm_heads;
 } hymba_layer_cfg;
 
 /* Weights of one layer (device pointers, caller-owned, read only). Big matrices
@@ -121,11 +130,11 @@ typedef struct hymba_layer_cfg {
  * dt_low (B and C first so that their columns start on 16-byte boundaries). */
 typedef struct hymba_layer_weights {
     const void*  w_in;        /* [n_in, d_model]        dtype */
-    const void*  w_dt;        /* [d_inner, dt_rank]     dtype */
-    const float* b_dt;        /* [d_inner] */
+    const void*  w_dt;        /* [n_dt, dt_rank]        dtype; n_dt = d_inner, or ssm_heads in the SSD form */
+    const float* b_dt;        /* [n_dt] */
     const float* conv_w;      /* [d_inner, d_conv]      tap d_conv-1 meets the newest input */
     const float* conv_b;      /* [d_inner] */
-    const float* A_log;       /* [d_inner, d_state]     A = -exp(A_log) */
+    const float* A_log;       /* [d_inner, d_state]     A = -exp(A_log); [ssm_heads] in the SSD form */
     const float* D;           /* [d_inner] */
     const float* norm_attn_w; /* [n_q_heads*v_head_dim] RMSNorm gain of the attention branch */
     const float* norm_ssm_w;  /* [d_inner]              RMSNorm gain of the SSM branch */

@@ -93,6 +93,10 @@ WORKLOADS: Dict[str, dict] = {
     # decode step of a KV-sharing layer pair: B=64, prompt 4096 + 128 meta, ring 1024
     "hymba15_decode_pair_b64_p4096": dict(kind="decode_pair", cfg=hymba15_layer_cfg(1024), B=64,
                                           T=4096, seed=3),
+    # the SWA layer with the Mamba heads in the SSD form (50 heads of 64 channels), at the
+    # stack's batch: B=8, T=4096 + 128 meta
+    "hymba15_ssd_swa1024_b8_t4096": dict(kind="prefill", cfg=hymba15_layer_cfg(1024).with_(ssm_heads=50), B=8,
+                                         T=4096, seed=5),
     # 32-layer mixer stack: B=8, T=4096 + 128 meta; layers 0/15/31 global; pairs share KV
     "hymba15_stack32_b8_t4096": dict(kind="stack", cfg=hymba15_layer_cfg(1024), B=8, T=4096,
                                      seed=4, n_layers=32, global_layers=(0, 15, 31)),

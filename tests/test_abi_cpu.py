@@ -78,10 +78,20 @@ def test_invalid_configs_rejected(hy):
     base = synth.tiny_layer_cfg()
     for bad in (base.with_(head_dim=32), base.with_(d_state=8), base.with_(n_kv_heads=3),
                 base.with_(v_head_dim=64), base.with_(dtype=7), base.with_(d_model=0), base.with_(fusion=2),
-                base.with_(fusion=1, v_head_dim=96)):
+                base.with_(fusion=1, v_head_dim=96), base.with_(ssm_heads=-1), base.with_(ssm_heads=3),
+                base.with_(ssm_heads=128), synth.hymba15_layer_cfg(1024).with_(ssm_heads=25)):
         c = hy.cfg_struct(bad)
         assert hy.hymba_workspace_bytes(ctypes.byref(c), 1, 10, 0) == 0
         assert hy.hymba_cache_bytes(ctypes.byref(c), 1, 10) == 0
+
+
+def test_ssd_form_configs_accepted(hy):
+    """The SSD form: any head width that is a multiple of 8 for fp32, 64 for bf16 (the
+    tensor-core chunk kernel's width)."""
+    for ok in (synth.tiny_layer_cfg().with_(ssm_heads=4), synth.tiny_layer_cfg().with_(ssm_heads=64),
+               synth.hymba15_layer_cfg(1024).with_(ssm_heads=50)):
+        c = hy.cfg_struct(ok)
+        assert hy.hymba_workspace_bytes(ctypes.byref(c), 1, 10, 0) > 0
 
 
 def test_concat_fusion_workspace_holds_the_wider_u(hy):

@@ -67,7 +67,7 @@ def _check_stages(cfg, r, ref, B, Tp, delta_written=True):
     assert_close(ypre * oracle.silu(z), ref["y_ssm"], cfg, "gated SSM output", max_abs=1e-4 if cfg.dtype == 0 else 2.5e-1,
                  rel_l2=5e-3)
     assert_close(o, ref["o_attn"], cfg, "attention output", **tol)
-    assert_close(u, ref["u"], cfg, "fused U", max_abs=2e-4 if cfg.dtype == 0 else 1.5e-1, rel_l2=5e-3)
+    assert_close(u, ref["u"], cfg, "fused U", max_abs=1e-4 if cfg.dtype == 0 else 1.5e-1, rel_l2=5e-3)
 
 
 @pytest.mark.parametrize("perturb", [False, True])
@@ -137,7 +137,7 @@ def test_tiny_f32_kv_share_and_residual_stack():
     rt.prefill(lb, yb, 40, ga["kv"], yb, ws, None, hy.HYMBA_X_HAS_META | hy.HYMBA_ADD_RESIDUAL,
                kv_struct_override=kvs)  # in place: y == x
     torch.cuda.synchronize()
-    assert_close(to_np(yb), rb["y"], cb, "consumer y (in place)", max_abs=2e-4)
+    assert_close(to_np(yb), rb["y"], cb, "consumer y (in place)")
 
 
 def test_bf16_hymba15_swa_layer():
@@ -278,14 +278,16 @@ def test_concat_fusion_layer(case):
     assert_close(to_np(rc["y"]), refc["y"], cc, "consumer y (concat fusion)")
 
 
-def test_bf16_many_sequences_use_the_wide_scan():
-    """A batch wide enough (B * d_inner / 64 >= 2 * SMs) for the one-thread-per-channel
-    scan (with Delta computed inside it): 30 sequences of a small bf16 layer with a
-    ragged last chunk (8 meta + 70 rows); y, the final SSM state and the conv state."""
+@pytest.mark.parametrize("T", [70, 10, 24])
+def test_bf16_many_sequences_use_the_wide_scan(T):
+    """A batch wide enough (B * d_inner / 64 >= 2 * SMs) for the wide scan (two threads
+    per channel, Delta computed inside it): 30 sequences of a small bf16 layer with 8 meta
+    rows + T: a ragged last chunk (78 rows), one short chunk (18), exactly one chunk (32);
+    y, the final SSM state and the conv state."""
     cfg = synth.hymba15_layer_cfg(window=24).with_(d_model=256, n_q_heads=5, n_kv_heads=1, d_inner=640,
                                                    dt_rank=24, n_meta=8)
     w = synth.perturbed_weights(synth.layer_weights(cfg, 141), cfg, 141)
-    B, T = 30, 70
+    B = 30
     x = synth.layer_input(cfg, B, T, 142)
     ref = oracle.mixer_prefill(cfg, w, x)
     r = _run_prefill(cfg, w, x)
