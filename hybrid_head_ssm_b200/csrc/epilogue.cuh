@@ -49,6 +49,9 @@ struct EpiArgs {
     int res_meta_bf16;     // 1: res_meta is bf16; 0: it has type T
     // EPI_GLU: y = SiLU(gate) * (this GEMM's result), gate [M, N] of type T
     const T* glu_gate;
+    // EPI_OUT into fp32 with accumulate = 1: the run is added to y (red.global.add) instead
+    // of stored, no residual (split-K partial sums; y holds the residual beforehand)
+    int accumulate;
     // in-projection GEMMs that also cover the meta rows: GEMM rows [0, meta_pad) are
     // meta rows (valid below meta_M, written for every sequence), the rest follow
     // row_mode after subtracting meta_pad
@@ -105,6 +108,7 @@ struct RunDst {
     int count;
     int nbytes;
     int esz;
+    int add;   // fp32 runs only: accumulate into the destination
 };
 
 // Everything the epilogue does to one run except the store: bias + softplus (Delta),
@@ -114,7 +118,7 @@ template <typename T>
 __device__ __forceinline__ RunDst epi_prepare64(const EpiArgs<T>& e, int r, int c0, float* v) {
     // the element size depends on the launch only (the staged store relies on it being
     // the same in every lane, rows without output included)
-    RunDst d{nullptr, 0, 0, 0, e.kind == EPI_DELTA ? 4 : (int)sizeof(T)};
+    RunDst d{nullptr, 0, 0, 0, e.kind == EPI_DELTA ? 4 : (int)sizeof(T), 0};
     int mode = e.row_mode, M = e.M;
     if (e.meta_pad > 0) {
         if (r < e.meta_pad) {
@@ -163,6 +167,13 @@ __device__ __forceinline__ RunDst epi_prepare64(const EpiArgs<T>& e, int r, int 
         return d;
     }
     if (e.kind == EPI_OUT) {
+        if (e.accumulate) {
+            d.p = reinterpret_cast<char*>(e.y + (long long)r * e.N + c0);
+            d.count = 1;
+            d.nbytes = n * (int)sizeof(T);
+            d.add = 1;
+            return d;
+        }
         if (e.res_mode == 1) {
             add_residual64(v, e.res_x + (long long)r * e.N + c0, n);
         } else if (e.res_mode == 2) {
@@ -250,6 +261,10 @@ __device__ void epi_run64(const EpiArgs<T>& e, int r, int c0, float* v) {
     const RunDst d = epi_prepare64<T>(e, r, c0, v);
     for (int b = 0; b < d.count; ++b) {
         char* p = d.p + b * d.stride;
+        if (d.add) {
+            for (int j = 0; j < d.nbytes / 4; ++j) atomicAdd(reinterpret_cast<float*>(p) + j, v[j]);
+            continue;
+        }
         if (d.esz == 4) store_run<float>(reinterpret_cast<float*>(p), v, d.nbytes / 4);
         else store_run<T>(reinterpret_cast<T*>(p), v, d.nbytes / (int)sizeof(T));
     }
@@ -298,6 +313,20 @@ __device__ __forceinline__ void epi_store_staged(const RunDst& d, const float* v
                 const bool vec = off + 16 <= ri.nbytes && ((reinterpret_cast<uintptr_t>(ri.p) | (uintptr_t)ri.stride) & 15) == 0;
                 for (int b = 0; b < ri.count; ++b) {
                     char* dst = ri.p + b * ri.stride + off;
+                    if (ri.add) {
+                        // split-K partial sums of an fp32 output
+                        if (vec) {
+                            asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(dst),
+                                         "f"(__uint_as_float(val.x)), "f"(__uint_as_float(val.y)),
+                                         "f"(__uint_as_float(val.z)), "f"(__uint_as_float(val.w))
+                                         : "memory");
+                        } else {
+                            const float* src = reinterpret_cast<const float*>(&val);
+                            for (int k = 0; 4 * k < min(16, ri.nbytes - off); ++k)
+                                atomicAdd(reinterpret_cast<float*>(dst) + k, src[k]);
+                        }
+                        continue;
+                    }
                     if (vec) {
                         *reinterpret_cast<uint4*>(dst) = val;
                     } else {

@@ -61,33 +61,66 @@ __device__ __forceinline__ void load8f(const float* p, float* v) {
     v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
 }
 
-// Attention output piece c..c+7 of row `row` merged from its head's split partials
-// (layout [row, head, split, dv + 2]: dv sums, then max logit and sum of weights).
+// Merge weights of a row's split partials (layout [row, head, split, dv + 2]: dv sums,
+// then the split's max logit and sum of weights): w[head][s] = exp2(m_s - M) / den with
+// M = max_s m_s and den = sum_s exp2(m_s - M) l_s, formed once per (row, head) by the
+// block into shared memory (zero for a head that saw no key).
+__device__ __forceinline__ void merge_weights(const float* __restrict__ part, int n_split, int H, int dv,
+                                              long long row, float* wts, int t, int nthreads) {
+    // one warp per head, one lane per split (in rounds of 32 splits)
+    const int warp = t >> 5, lane = t & 31, nwarps = nthreads >> 5;
+    for (int hd = warp; hd < H; hd += nwarps) {
+        const float* base = part + ((long long)row * H + hd) * n_split * (dv + 2) + dv;
+        float M = -INFINITY;
+        for (int s = lane; s < n_split; s += 32) M = fmaxf(M, base[s * (dv + 2)]);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+        float den = 0.f;
+        for (int s = lane; s < n_split; s += 32) {
+            const float w = M != -INFINITY ? exp2f(base[s * (dv + 2)] - M) : 0.f;
+            wts[hd * n_split + s] = w;
+            den = fmaf(w, base[s * (dv + 2) + 1], den);
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
+        const float inv = den > 0.f ? 1.f / den : 0.f;
+        for (int s = lane; s < n_split; s += 32) wts[hd * n_split + s] *= inv;
+    }
+}
+
+// Attention output piece c..c+7 of row `row`: the weighted sum of its head's split
+// partials (the loads of four splits in flight at a time).
 __device__ __forceinline__ void merge8(const float* __restrict__ part, int n_split, int H, int dv,
-                                       long long row, int c, float* o) {
+                                       long long row, int c, const float* wts, float* o) {
     const int hd = c / dv, e = c - hd * dv;
-    const float* base = part + ((long long)row * H + hd) * n_split * (dv + 2);
-    float M = -INFINITY;
-    for (int s = 0; s < n_split; ++s) M = fmaxf(M, base[s * (dv + 2) + dv]);
+    const float* base = part + ((long long)row * H + hd) * n_split * (dv + 2) + e;
+    const float* w = wts + hd * n_split;
 #pragma unroll
     for (int i = 0; i < 8; ++i) o[i] = 0.f;
-    float den = 0.f;
-    if (M != -INFINITY) {
-        for (int s = 0; s < n_split; ++s) {
-            const float* ps = base + s * (dv + 2);
-            const float w = exp2f(ps[dv] - M);
-            den = fmaf(w, ps[dv + 1], den);
+    int s = 0;
+    for (; s + 4 <= n_split; s += 4) {
+        float4 v[4][2];
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const float2 v = *reinterpret_cast<const float2*>(ps + e + 2 * i);
-                o[2 * i] = fmaf(w, v.x, o[2 * i]);
-                o[2 * i + 1] = fmaf(w, v.y, o[2 * i + 1]);
-            }
+        for (int u = 0; u < 4; ++u) {
+            const float* ps = base + (s + u) * (dv + 2);
+            v[u][0] = make_float4(ps[0], ps[1], ps[2], ps[3]);
+            v[u][1] = make_float4(ps[4], ps[5], ps[6], ps[7]);
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const float wu = w[s + u];
+            o[0] = fmaf(wu, v[u][0].x, o[0]); o[1] = fmaf(wu, v[u][0].y, o[1]);
+            o[2] = fmaf(wu, v[u][0].z, o[2]); o[3] = fmaf(wu, v[u][0].w, o[3]);
+            o[4] = fmaf(wu, v[u][1].x, o[4]); o[5] = fmaf(wu, v[u][1].y, o[5]);
+            o[6] = fmaf(wu, v[u][1].z, o[6]); o[7] = fmaf(wu, v[u][1].w, o[7]);
         }
     }
-    const float inv = den > 0.f ? 1.f / den : 0.f;
+    for (; s < n_split; ++s) {
+        const float* ps = base + s * (dv + 2);
+        const float wu = w[s];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) o[i] *= inv;
+        for (int i = 0; i < 8; ++i) o[i] = fmaf(wu, ps[i], o[i]);
+    }
 }
 
 // (the decode variant runs one block per sequence, so it asks for no more than one
@@ -100,12 +133,18 @@ fuse_kernel(const I* __restrict__ O, const float* __restrict__ part, int n_split
             const I* __restrict__ ypre, const I* __restrict__ P, long long ldP, int col_z,
             const float* __restrict__ g_attn, const float* __restrict__ g_ssm, const float* __restrict__ beta1,
             const float* __restrict__ beta2, const float* __restrict__ v_scale, const float* __restrict__ v_bias,
-            int rep, T* __restrict__ U, int rows, int di, float eps, int* len_inc) {
+            int rep, T* __restrict__ U, int rows, int di, float eps, int* len_inc, float* __restrict__ y_init,
+            const float* __restrict__ y_res, int d_model) {
     griddep_sync();
     __shared__ float red[RPB][TPR / 32][2];
+    extern __shared__ float merge_wts[];  // SPLIT: [H, n_split] merge weights of the row
     const int sub = threadIdx.x / TPR, t = threadIdx.x % TPR;
     const long long row = (long long)blockIdx.x * RPB + sub;
     const bool live = row < rows;
+    if constexpr (SPLIT) {
+        if (live) merge_weights(part, n_split, H, dv, row, merge_wts, t, TPR);
+        __syncthreads();
+    }
     const int hv = H * dv;                 // attention branch width
     const int nvo = hv / 8, nvy = di / 8;  // pieces of 8 per branch
     float o[VMAX][8], y[VMAX][8];
@@ -116,7 +155,7 @@ fuse_kernel(const I* __restrict__ O, const float* __restrict__ part, int n_split
         if (live && vi < nvo) {
             const int c = vi * 8;
             if constexpr (SPLIT)
-                merge8(part, n_split, H, dv, row, c, o[k]);
+                merge8(part, n_split, H, dv, row, c, merge_wts, o[k]);
             else
                 load8<I>(O + row * hv + c, o[k]);
             if (v_scale) {
@@ -204,6 +243,19 @@ fuse_kernel(const I* __restrict__ O, const float* __restrict__ part, int n_split
         }
     }
     if (len_inc && live && t == 0) len_inc[row] += 1;
+    // the output projection that follows adds its split-K partial sums to y: y starts as
+    // the residual (or zero), unless y is the residual itself
+    if (y_init && live && y_init != y_res)
+        for (int c = t; c < d_model; c += TPR)
+            y_init[row * d_model + c] = y_res ? y_res[row * d_model + c] : 0.f;
+}
+
+constexpr int RT = 512;                 // prefill fusion: threads per row (one 8-channel piece each)
+
+__device__ __forceinline__ void cp_async16_own(void* dst, const void* src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(static_cast<uint32_t>(__cvta_generic_to_shared(dst))),
+                 "l"(src)
+                 : "memory");
 }
 
 // An 8-element piece of an input row as loaded (16-bit: one 16-byte word; fp32: two).
@@ -241,86 +293,91 @@ __device__ __forceinline__ void pack_piece(Piece<I>& p, const float* v) {
     }
 }
 
-// Prefill fusion, persistent over rows: block b takes rows b, b + grid, ... and loads the
-// next row's pieces into registers before working on the current one, so every block
-// keeps a row of loads in flight through its reductions and stores (a row kernel that
-// loads, reduces and stores in turn leaves HBM idle while it reduces). The per-channel
-// factors beta * gain (halved for the average) are formed once per block in shared
-// memory. The gated Mamba branch is kept between the two passes in the intermediate
-// type (fp16 for 16-bit layers: the normalised result is written as bf16 or fp16).
+// Prefill fusion, persistent over rows: block b takes rows b, b + grid, ... and each
+// thread copies its own pieces of the next three rows (O, y_pre, z: 16-byte cp.async into
+// a four-slot shared-memory ring that only it reads) before working on the current one, so
+// every block keeps three rows of loads in flight through its reductions and stores (a row
+// kernel that loads, reduces and stores in turn leaves HBM idle while it reduces). The
+// per-channel factors beta * gain (halved for the average) of a thread's columns are
+// formed once, in registers; the gated Mamba branch stays in fp32 between the passes.
+// One piece of 8 channels per thread and branch (widths up to 8 * RT).
+constexpr int RSLOT = 4;  // ring slots: the current row and three in flight
+
 template <typename I, typename T, bool CONCAT>
-__global__ void __launch_bounds__(TPR, 3)
+__global__ void __launch_bounds__(RT, 1)
 fuse_rows_kernel(const I* __restrict__ O, int H, int dv, const I* __restrict__ ypre, const I* __restrict__ P,
                  long long ldP, int col_z, const float* __restrict__ g_attn, const float* __restrict__ g_ssm,
                  const float* __restrict__ beta1, const float* __restrict__ beta2, const float* __restrict__ v_scale,
                  const float* __restrict__ v_bias, int rep, T* __restrict__ U, long long rows, int di, float eps) {
-    constexpr bool PF = sizeof(I) == 2;  // prefetch the next row (16-bit inputs: few registers per piece)
-    extern __shared__ float fac[];        // [hv] attention factors, then [di] Mamba factors
-    __shared__ float red[2][TPR / 32][2];
+    constexpr int PW = sizeof(I) / 2;  // 16-byte words per piece
+    extern __shared__ uint4 ring[];    // [RSLOT][3 arrays][PW][RT]
+    __shared__ float red[2][RT / 32][2];
     griddep_sync();
     const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
     const int hv = H * dv, nvo = hv / 8, nvy = di / 8;
+    const int c = t * 8;
+    const bool has_o = t < nvo, has_y = t < nvy;
     const float half = CONCAT ? 1.0f : 0.5f;  // the average halves both branches
-    for (int c = t; c < hv; c += TPR) fac[c] = half * beta1[c] * g_attn[c];
-    for (int c = t; c < di; c += TPR) fac[hv + c] = half * beta2[c] * g_ssm[c];
-    __syncthreads();
-    const long long ldu = CONCAT ? (long long)di + hv : di;
-
-    Piece<I> po[VMAX], py[VMAX], pz[VMAX];
-    auto load_row = [&](long long r, Piece<I>* a, Piece<I>* b, Piece<I>* z) {
+    // this thread's columns are the same in every row: their factors stay in registers
+    float fa[8], fs[8];
 #pragma unroll
-        for (int k = 0; k < VMAX; ++k) {
-            const int vi = t + k * TPR;
-            if (vi < nvo) load_piece<I>(a[k], O + r * hv + vi * 8);
-            if (vi < nvy) {
-                load_piece<I>(b[k], ypre + r * di + vi * 8);
-                load_piece<I>(z[k], P + r * ldP + col_z + vi * 8);
+    for (int i = 0; i < 8; ++i) {
+        fa[i] = has_o ? half * beta1[c + i] * g_attn[c + i] : 0.f;
+        fs[i] = has_y ? half * beta2[c + i] * g_ssm[c + i] : 0.f;
+    }
+    const int vidx = has_o ? (c / dv / rep) * dv + (c % dv) : 0;  // a consumer's V transform entries
+    const long long ldu = CONCAT ? (long long)di + hv : di;
+    auto slot = [&](int sl, int arr, int w) -> uint4* { return ring + ((sl * 3 + arr) * PW + w) * RT + t; };
+    auto issue = [&](long long r, int sl) {
+        if (r < rows) {
+#pragma unroll
+            for (int w = 0; w < PW; ++w) {
+                if (has_o) cp_async16_own(slot(sl, 0, w), O + r * hv + c + 8 / PW * w);
+                if (has_y) {
+                    cp_async16_own(slot(sl, 1, w), ypre + r * di + c + 8 / PW * w);
+                    cp_async16_own(slot(sl, 2, w), P + r * ldP + col_z + c + 8 / PW * w);
+                }
             }
         }
+        asm volatile("cp.async.commit_group;" ::: "memory");
+    };
+    auto fetch = [&](int sl, int arr, float* v) {
+        Piece<I> pc;
+#pragma unroll
+        for (int w = 0; w < PW; ++w) pc.v[w] = *slot(sl, arr, w);
+        unpack_piece<I>(pc, v);
     };
     long long row = blockIdx.x;
-    if (PF && row < rows) load_row(row, po, py, pz);
+    for (int k = 0; k < RSLOT - 1; ++k) issue(row + (long long)k * gridDim.x, k);
     for (int it = 0; row < rows; ++it, row += gridDim.x) {
-        Piece<I> no[VMAX], ny[VMAX], nz[VMAX];
-        const long long nrow = row + gridDim.x;
-        if (PF) {
-            if (nrow < rows) load_row(nrow, no, ny, nz);
-        } else {
-            load_row(row, po, py, pz);
-        }
+        const int sl = it % RSLOT;
+        issue(row + (long long)(RSLOT - 1) * gridDim.x, (it + RSLOT - 1) % RSLOT);
+        // this thread's copies of `row` have landed (the RSLOT - 1 later groups may still fly)
+        asm volatile("cp.async.wait_group %0;" ::"n"(RSLOT - 1) : "memory");
         // pass 1: the consumer's V transform, the gate, both sums of squares
+        float o[8], yg[8];
         float ss_o = 0.f, ss_y = 0.f;
+        if (has_o) {
+            fetch(sl, 0, o);
+            if (v_scale) {
+                // attention over V * s + b is the attention output * s + b (weights sum to 1)
+                float vs[8], vb[8];
+                load8f(v_scale + vidx, vs);
+                load8f(v_bias + vidx, vb);
 #pragma unroll
-        for (int k = 0; k < VMAX; ++k) {
-            const int vi = t + k * TPR;
-            if (vi < nvo) {
-                float o[8];
-                unpack_piece<I>(po[k], o);
-                if (v_scale) {
-                    // attention over V * s + b is the attention output * s + b (weights sum to 1)
-                    const int c = vi * 8, hd = c / dv;
-                    const int idx = (hd / rep) * dv + (c - hd * dv);
-                    float vs[8], vb[8];
-                    load8f(v_scale + idx, vs);
-                    load8f(v_bias + idx, vb);
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) o[i] = fmaf(o[i], vs[i], vb[i]);
-                    pack_piece<I>(po[k], o);
-                    unpack_piece<I>(po[k], o);  // normalise what is kept
-                }
-#pragma unroll
-                for (int i = 0; i < 8; ++i) ss_o = fmaf(o[i], o[i], ss_o);
+                for (int i = 0; i < 8; ++i) o[i] = fmaf(o[i], vs[i], vb[i]);
             }
-            if (vi < nvy) {
-                float y[8], z[8];
-                unpack_piece<I>(py[k], y);
-                unpack_piece<I>(pz[k], z);
 #pragma unroll
-                for (int i = 0; i < 8; ++i) y[i] *= z[i] / (1.0f + __expf(-z[i]));
-                pack_piece<I>(py[k], y);
-                unpack_piece<I>(py[k], y);
+            for (int i = 0; i < 8; ++i) ss_o = fmaf(o[i], o[i], ss_o);
+        }
+        if (has_y) {
+            float z[8];
+            fetch(sl, 1, yg);
+            fetch(sl, 2, z);
 #pragma unroll
-                for (int i = 0; i < 8; ++i) ss_y = fmaf(y[i], y[i], ss_y);
+            for (int i = 0; i < 8; ++i) {
+                yg[i] *= __fdividef(z[i], 1.0f + __expf(-z[i]));
+                ss_y = fmaf(yg[i], yg[i], ss_y);
             }
         }
 #pragma unroll
@@ -336,50 +393,34 @@ fuse_rows_kernel(const I* __restrict__ O, int H, int dv, const I* __restrict__ y
         ss_o = 0.f;
         ss_y = 0.f;
 #pragma unroll
-        for (int w = 0; w < TPR / 32; ++w) {
+        for (int w = 0; w < RT / 32; ++w) {
             ss_o += red[it & 1][w][0];
             ss_y += red[it & 1][w][1];
         }
         const float ro = rsqrtf(ss_o / hv + eps);
         const float ry = rsqrtf(ss_y / di + eps);
         // pass 2: scale, combine, store
+        if constexpr (CONCAT) {
+            if (has_y) {
+                float u[8];
 #pragma unroll
-        for (int k = 0; k < VMAX; ++k) {
-            const int vi = t + k * TPR;
-            const int c = vi * 8;
-            if constexpr (CONCAT) {
-                if (vi < nvy) {
-                    float y[8], u[8];
-                    unpack_piece<I>(py[k], y);
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) u[i] = fac[hv + c + i] * y[i] * ry;
-                    store8<T>(U + row * ldu + c, u);
-                }
-                if (vi < nvo) {
-                    float o[8], u[8];
-                    unpack_piece<I>(po[k], o);
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) u[i] = fac[c + i] * o[i] * ro;
-                    store8<T>(U + row * ldu + di + c, u);
-                }
-            } else if (vi < nvy) {
-                float o[8], y[8], u[8];
-                unpack_piece<I>(po[k], o);
-                unpack_piece<I>(py[k], y);
-#pragma unroll
-                for (int i = 0; i < 8; ++i) u[i] = fmaf(fac[c + i] * ro, o[i], fac[hv + c + i] * ry * y[i]);
+                for (int i = 0; i < 8; ++i) u[i] = fs[i] * yg[i] * ry;
                 store8<T>(U + row * ldu + c, u);
             }
-        }
-        if (PF) {
+            if (has_o) {
+                float u[8];
 #pragma unroll
-            for (int k = 0; k < VMAX; ++k) {
-                po[k] = no[k];
-                py[k] = ny[k];
-                pz[k] = nz[k];
+                for (int i = 0; i < 8; ++i) u[i] = fa[i] * o[i] * ro;
+                store8<T>(U + row * ldu + di + c, u);
             }
+        } else if (has_y) {
+            float u[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) u[i] = fmaf(fa[i] * ro, o[i], fs[i] * ry * yg[i]);
+            store8<T>(U + row * ldu + c, u);
         }
     }
+    asm volatile("cp.async.wait_group 0;" ::: "memory");
 }
 
 }  // namespace
@@ -388,18 +429,22 @@ template <typename I, typename T, bool CONCAT>
 static int fuse_variant(const Ctx& ctx, const I* O, const float* part, int n_split, int H, int dv, int G,
                         const I* ypre, const I* P, long long ldP, int col_z, const float* g_attn, const float* g_ssm,
                         const float* beta1, const float* beta2, const float* v_scale, const float* v_bias, T* U,
-                        int rows, int di, float eps, int* len_inc) {
+                        int rows, int di, float eps, int* len_inc, float* y_init, const float* y_res, int d_model) {
     if (part) {
         auto kern = fuse_kernel<I, T, true, CONCAT>;
-        HYMBA_LAUNCH(ctx, "fuse", kern, ceil_div(rows, RPB), TPR * RPB, 0, O, part, n_split, H, dv, ypre, P, ldP,
-                     col_z, g_attn, g_ssm, beta1, beta2, v_scale, v_bias, H / G, U, rows, di, eps, len_inc);
-    } else {
-        auto kern = fuse_rows_kernel<I, T, CONCAT>;
-        const size_t smem = (size_t)(H * dv + di) * sizeof(float);
+        const size_t smem = (size_t)H * n_split * sizeof(float);
         static std::atomic<unsigned long long> smem_set{0};
         if (smem > 48 * 1024 && !smem_opt_in_once(smem_set, kern, smem, ctx)) return HYMBA_ERR_CUDA;
-        const int grid = (int)std::min<long long>(rows, 3LL * (ctx.sm_count > 0 ? ctx.sm_count : 148));
-        HYMBA_LAUNCH(ctx, "fuse", kern, grid, TPR, smem, O, H, dv, ypre, P, ldP, col_z, g_attn, g_ssm, beta1, beta2,
+        HYMBA_LAUNCH(ctx, "fuse", kern, ceil_div(rows, RPB), TPR * RPB, smem, O, part, n_split, H, dv, ypre, P, ldP,
+                     col_z, g_attn, g_ssm, beta1, beta2, v_scale, v_bias, H / G, U, rows, di, eps, len_inc, y_init,
+                     y_res, d_model);
+    } else {
+        auto kern = fuse_rows_kernel<I, T, CONCAT>;
+        const size_t smem = (size_t)RSLOT * 3 * RT * sizeof(I) * 8;
+        static std::atomic<unsigned long long> smem_set{0};
+        if (!smem_opt_in_once(smem_set, kern, smem, ctx)) return HYMBA_ERR_CUDA;
+        const int grid = (int)std::min<long long>(rows, ctx.sm_count > 0 ? ctx.sm_count : 148);
+        HYMBA_LAUNCH(ctx, "fuse", kern, grid, RT, smem, O, H, dv, ypre, P, ldP, col_z, g_attn, g_ssm, beta1, beta2,
                      v_scale, v_bias, H / G, U, (long long)rows, di, eps);
     }
     return HYMBA_OK;
@@ -409,8 +454,9 @@ template <typename I, typename T>
 int launch_fuse(const Ctx& ctx, const I* O, const float* part, int n_split, int H, int G, int dv, bool concat,
                 const I* ypre, const I* P, long long ldP, int col_z, const float* g_attn, const float* g_ssm,
                 const float* beta1, const float* beta2, const float* v_scale, const float* v_bias, T* U, int rows,
-                int di, float eps, int* len_inc) {
+                int di, float eps, int* len_inc, float* y_init, const float* y_res, int d_model) {
     if (rows <= 0) return HYMBA_OK;
+    if (y_init && (!part || d_model <= 0)) return HYMBA_ERR_UNSUPPORTED;
     const int hv = H * dv;
     if (di % 8 || di > VMAX * 8 * TPR || hv > VMAX * 8 * TPR || col_z % 8 || ldP % 8) return HYMBA_ERR_UNSUPPORTED;
     // pieces of 8 never straddle a head
@@ -422,15 +468,16 @@ int launch_fuse(const Ctx& ctx, const I* O, const float* part, int n_split, int 
     if (part && (n_split <= 0 || (reinterpret_cast<uintptr_t>(part) & 7))) return HYMBA_ERR_UNSUPPORTED;
     if (concat)
         return fuse_variant<I, T, true>(ctx, O, part, n_split, H, dv, G, ypre, P, ldP, col_z, g_attn, g_ssm, beta1,
-                                        beta2, v_scale, v_bias, U, rows, di, eps, len_inc);
+                                        beta2, v_scale, v_bias, U, rows, di, eps, len_inc, y_init, y_res, d_model);
     return fuse_variant<I, T, false>(ctx, O, part, n_split, H, dv, G, ypre, P, ldP, col_z, g_attn, g_ssm, beta1,
-                                     beta2, v_scale, v_bias, U, rows, di, eps, len_inc);
+                                     beta2, v_scale, v_bias, U, rows, di, eps, len_inc, y_init, y_res, d_model);
 }
 
 #define HYMBA_FUSE_INST(I, T)                                                                                  \
     template int launch_fuse<I, T>(const Ctx&, const I*, const float*, int, int, int, int, bool, const I*, const I*, \
                                    long long, int, const float*, const float*, const float*, const float*,          \
-                                   const float*, const float*, T*, int, int, float, int*);
+                                   const float*, const float*, T*, int, int, float, int*, float*, const float*, \
+                                   int);
 HYMBA_FUSE_INST(float, float)
 HYMBA_FUSE_INST(f16, bf16)
 HYMBA_FUSE_INST(f16, f16)

@@ -68,6 +68,7 @@ template <typename TA, typename TO>
 int launch_gemm_simt(const Ctx& ctx, const char* name, const TA* A, long long lda, const TA* Bw, long long ldb,
                      int M, int N, int K, const EpiArgs<TO>& e) {
     if (M <= 0 || N <= 0) return HYMBA_OK;
+    if (e.accumulate) return HYMBA_ERR_UNSUPPORTED;  // split-K partial sums run on the tensor-core GEMM
     dim3 grid(ceil_div(N, TN), ceil_div(M, TM));
     auto kern = gemm_simt_kernel<TA, TO>;
     HYMBA_LAUNCH(ctx, name, kern, grid, 256, 0, A, lda, Bw, ldb, M, N, K, e);

@@ -14,6 +14,8 @@
 // The accumulator is double-buffered in TMEM so the epilogue of one tile overlaps the
 // MMAs of the next. Every mbarrier wait is bounded; on timeout the CTA records
 // HYMBA_ERR_DEVICE_TIMEOUT, drains what it issued and exits.
+#include <algorithm>
+
 #include "kernels.h"
 #include "tc.cuh"
 
@@ -114,7 +116,8 @@ __device__ __forceinline__ void tile_coords(int tile, int num_m, int num_n, int*
 template <typename TA, typename TO, int BN, int STAGES>
 __global__ void __launch_bounds__(NUM_THREADS, STAGES == 2 ? 2 : 1)
 gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-               const __grid_constant__ CUtensorMap tmA0, int M0, int M, int N, int K, EpiArgs<TO> e, int* status) {
+               const __grid_constant__ CUtensorMap tmA0, int M0, int M, int N, int K, int ksplit, EpiArgs<TO> e,
+               int* status) {
     extern __shared__ uint8_t smem_raw[];
     GemmSmem<BN, STAGES>& s = *reinterpret_cast<GemmSmem<BN, STAGES>*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                         ~static_cast<uintptr_t>(1023));
@@ -125,7 +128,14 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     // rest from A (M rows); the epilogue tells them apart by row index (EpiArgs::meta_pad)
     const int num_m0 = (M0 + BM - 1) / BM;
     const int num_m = num_m0 + (M + BM - 1) / BM, num_n = (N + BN - 1) / BN;
-    const int num_tiles = num_m * num_n, nk = (K + BK - 1) / BK;
+    // split-K: tile index = output tile * ksplit + split; split s covers k-blocks
+    // [s nk / ksplit, (s + 1) nk / ksplit) and adds its partial sum to the output
+    const int num_tiles = num_m * num_n * ksplit, nk = (K + BK - 1) / BK;
+    auto krange = [&](int tile, int* kb0, int* kb1) {
+        const int sp = tile % ksplit;
+        *kb0 = sp * nk / ksplit;
+        *kb1 = (sp + 1) * nk / ksplit;
+    };
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < STAGES; ++i) {
@@ -164,9 +174,10 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
             int issued_phase[STAGES];
             for (int i = 0; i < STAGES; ++i) issued_phase[i] = -1;
             for (int tile = blockIdx.x; tile < num_tiles && !*abort; tile += gridDim.x) {
-                int m_blk, n_blk;
-                tile_coords(tile, num_m, num_n, &m_blk, &n_blk);
-                for (int kb = 0; kb < nk; ++kb, ++it) {
+                int m_blk, n_blk, kb0, kb1;
+                tile_coords(tile / ksplit, num_m, num_n, &m_blk, &n_blk);
+                krange(tile, &kb0, &kb1);
+                for (int kb = kb0; kb < kb1; ++kb, ++it) {
                     const int st = it % STAGES;
                     const uint32_t ph = (it / STAGES) & 1;
                     if (!tc::mbar_wait(&s.empty[st], ph ^ 1, abort, wlim)) { fail(abort, status, 0, kb, 1); break; }
@@ -195,7 +206,9 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
                 tc::tc_fence_after();
                 const uint32_t d = tmem + buf * BN;
                 bool ok = true;
-                for (int kb = 0; kb < nk; ++kb, ++it) {
+                int kb0, kb1;
+                krange(tile, &kb0, &kb1);
+                for (int kb = kb0; kb < kb1; ++kb, ++it) {
                     const int st = it % STAGES;
                     const uint32_t ph = (it / STAGES) & 1;
                     if (!tc::mbar_wait(&s.full[st], ph, abort, wlim)) { fail(abort, status, 1, kb, 2); ok = false; break; }
@@ -204,7 +217,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
 #pragma unroll
                     for (int kk = 0; kk < BK / 16; ++kk)
                         tc::mma_f16_ss(d, tc::sdesc_k_sw128(a0 + kk * 32), tc::sdesc_k_sw128(b0 + kk * 32), IDESC,
-                                       (kb | kk) != 0);
+                                       (kb != kb0 || kk != 0));
                     tc::mma_commit(&s.empty[st]);
                 }
                 if (!ok) break;
@@ -226,7 +239,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
             if (!__all_sync(0xffffffffu, tc::mbar_wait(&s.tfull[buf], tph, abort, wlim))) { fail(abort, status, 2, tcount, 3); break; }
             tc::tc_fence_after();
             int m_blk, n_blk;
-            tile_coords(tile, num_m, num_n, &m_blk, &n_blk);
+            tile_coords(tile / ksplit, num_m, num_n, &m_blk, &n_blk);
             const int row = m_blk * BM + q * 32 + lane;
 #pragma unroll 1
             for (int j = 0; j < BN / 64; ++j) {
@@ -258,7 +271,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
 
 template <typename TA, typename TO, int BN, int STAGES>
 int launch_bn(const Ctx& ctx, const char* name, const TA* A, long long lda, const TA* Bw, long long ldb, int M,
-              int N, int K, const EpiArgs<TO>& e, const TA* A0, int M0) {
+              int N, int K, const EpiArgs<TO>& e, const TA* A0, int M0, int ksplit) {
     constexpr bool kBF16 = std::is_same<TA, bf16>::value;
     CUtensorMap ta, tb, ta0;
     if (!tc::make_tmap_2d(&ta, A, kBF16, M, K, lda, BM)) return HYMBA_ERR_UNSUPPORTED;
@@ -272,13 +285,13 @@ int launch_bn(const Ctx& ctx, const char* name, const TA* A, long long lda, cons
     auto kern = gemm_tc_kernel<TA, TO, BN, STAGES>;
     static std::atomic<unsigned long long> smem_set{0};
     if (!smem_opt_in_once(smem_set, kern, smem, ctx)) return HYMBA_ERR_CUDA;
-    const int tiles = ((M0 + BM - 1) / BM + (M + BM - 1) / BM) * ((N + BN - 1) / BN);
+    const int tiles = ((M0 + BM - 1) / BM + (M + BM - 1) / BM) * ((N + BN - 1) / BN) * ksplit;
     const int slots = ctx.sm_count * (STAGES == 2 ? 2 : 1);
     const int grid = tiles < slots ? tiles : slots;
     EpiArgs<TO> e2 = e;
     e2.meta_pad = ((M0 + BM - 1) / BM) * BM;
     e2.meta_M = M0;
-    HYMBA_LAUNCH(ctx, name, kern, grid, NUM_THREADS, smem, ta, tb, ta0, M0, M, N, K, e2, ctx.status);
+    HYMBA_LAUNCH(ctx, name, kern, grid, NUM_THREADS, smem, ta, tb, ta0, M0, M, N, K, ksplit, e2, ctx.status);
     return HYMBA_OK;
 }
 
@@ -306,18 +319,27 @@ int launch_gemm_tc(const Ctx& ctx, const char* name, const TA* A, long long lda,
                    int M, int N, int K, const EpiArgs<TO>& e, const TA* A0, int M0) {
     if (M <= 0 || N <= 0) return HYMBA_OK;
     if (M0 > 0 && (!A0 || ((uintptr_t)A0 & 15))) return HYMBA_ERR_INVALID_ARG;
-    switch (pick_bn(M + M0, N, ctx.sm_count > 0 ? ctx.sm_count : 148)) {
-        case 256: return launch_bn<TA, TO, 256, 4>(ctx, name, A, lda, Bw, ldb, M, N, K, e, A0, M0);
+    const int sms = ctx.sm_count > 0 ? ctx.sm_count : 148;
+    if (e.accumulate) {
+        // split-K into an fp32 output that holds the rest of the sum: 64-wide tiles, and
+        // as many splits as fill the SMs (a few rows x a long K, the decode projections)
+        if (sizeof(TO) != 4 || e.kind != EPI_OUT || M0 > 0) return HYMBA_ERR_INVALID_ARG;
+        const int tiles = ((M + BM - 1) / BM) * ((N + 63) / 64), nk = (K + BK - 1) / BK;
+        const int ksplit = std::max(1, std::min(nk, sms / std::max(1, tiles)));
+        return launch_bn<TA, TO, 64, 4>(ctx, name, A, lda, Bw, ldb, M, N, K, e, A0, M0, ksplit);
+    }
+    switch (pick_bn(M + M0, N, sms)) {
+        case 256: return launch_bn<TA, TO, 256, 4>(ctx, name, A, lda, Bw, ldb, M, N, K, e, A0, M0, 1);
         case 128:
-            if (K <= 2 * BK) return launch_bn<TA, TO, 128, 2>(ctx, name, A, lda, Bw, ldb, M, N, K, e, A0, M0);
-            return launch_bn<TA, TO, 128, 4>(ctx, name, A, lda, Bw, ldb, M, N, K, e, A0, M0);
+            if (K <= 2 * BK) return launch_bn<TA, TO, 128, 2>(ctx, name, A, lda, Bw, ldb, M, N, K, e, A0, M0, 1);
+            return launch_bn<TA, TO, 128, 4>(ctx, name, A, lda, Bw, ldb, M, N, K, e, A0, M0, 1);
         default:
-            if (K <= 2 * BK) return launch_bn<TA, TO, 64, 2>(ctx, name, A, lda, Bw, ldb, M, N, K, e, A0, M0);
+            if (K <= 2 * BK) return launch_bn<TA, TO, 64, 2>(ctx, name, A, lda, Bw, ldb, M, N, K, e, A0, M0, 1);
             // one row block streaming a long K (decode): a deeper ring keeps more weight
             // tiles in flight per CTA
             if (M + M0 <= BM && K > 4 * BK)
-                return launch_bn<TA, TO, 64, 8>(ctx, name, A, lda, Bw, ldb, M, N, K, e, A0, M0);
-            return launch_bn<TA, TO, 64, 4>(ctx, name, A, lda, Bw, ldb, M, N, K, e, A0, M0);
+                return launch_bn<TA, TO, 64, 8>(ctx, name, A, lda, Bw, ldb, M, N, K, e, A0, M0, 1);
+            return launch_bn<TA, TO, 64, 4>(ctx, name, A, lda, Bw, ldb, M, N, K, e, A0, M0, 1);
     }
 }
 

@@ -228,13 +228,23 @@ static Plan plan(const hymba_layer_cfg* c, int B, int T, int mode) {
 // ---------------------------------------------------------------------------
 // dispatch: tcgen05 for 16-bit operands, CUDA cores for fp32
 // ---------------------------------------------------------------------------
+// Whether gemm() takes the tensor-core path for these operands.
+template <typename TA>
+static bool tc_gemm_ok(const TA* A, long long lda, const TA* W, long long ldw) {
+#ifdef HYMBA_WITH_TCGEN05
+    return sizeof(TA) == 2 && ((uintptr_t)A & 15) == 0 && ((uintptr_t)W & 15) == 0 && lda % 8 == 0 && ldw % 8 == 0;
+#else
+    (void)A; (void)lda; (void)W; (void)ldw;
+    return false;
+#endif
+}
+
 template <typename TA, typename TO>
 static int gemm(const Ctx& ctx, const char* name, const TA* A, long long lda, const TA* W, long long ldw,
                 int M, int N, int K, const EpiArgs<TO>& e) {
 #ifdef HYMBA_WITH_TCGEN05
     if constexpr (sizeof(TA) == 2) {
-        if (((uintptr_t)A & 15) == 0 && ((uintptr_t)W & 15) == 0 && lda % 8 == 0 && ldw % 8 == 0)
-            return launch_gemm_tc<TA, TO>(ctx, name, A, lda, W, ldw, M, N, K, e);
+        if (tc_gemm_ok(A, lda, W, ldw)) return launch_gemm_tc<TA, TO>(ctx, name, A, lda, W, ldw, M, N, K, e);
     }
 #endif
     return launch_gemm_simt<TA, TO>(ctx, name, A, lda, W, ldw, M, N, K, e);
@@ -514,23 +524,42 @@ static int decode_impl(const Ctx& ctx, const hymba_layer_cfg* c, const hymba_lay
     EpiArgs<TIO> eo = epi_base<TIO>(EPI_OUT, B, d);
     eo.y = y;
     if (flags & HYMBA_ADD_RESIDUAL) { eo.res_mode = 1; eo.res_x = x_io; }
+    // The out-projection of a decode step is a few rows against a long K: with an fp32
+    // output it is split over K across the SMs, each split adding its partial sum to y,
+    // which the fusion kernel first sets to the residual (or zero).
+    float* y_init = nullptr;
+    const float* y_res = nullptr;
+    auto plan_split = [&](bool tc_path) {
+        if constexpr (std::is_same<TIO, float>::value) {
+            if (tc_path) {
+                eo.accumulate = 1;
+                y_init = y;
+                y_res = eo.res_mode == 1 ? x_io : nullptr;
+                eo.res_mode = 0;
+            }
+        } else {
+            (void)tc_path;
+        }
+    };
     if constexpr (std::is_same<T, bf16>::value) {
         if (concat) {
             // as in the prefill: the concatenation's U and W_out in fp16
             f16* U16 = reinterpret_cast<f16*>(ws + pl.U);
             f16* wo16 = reinterpret_cast<f16*>(ws + pl.wout16);
             if ((rc = launch_pad_copy<T, f16>(ctx, static_cast<const T*>(w->w_out), d, uw, wo16, uw))) return rc;
+            plan_split(tc_gemm_ok<f16>(U16, uw, wo16, uw));
             if ((rc = launch_fuse<I, f16>(ctx, nullptr, part, pl.n_split, H, G, dv, true, ypre, P, pl.ldP, k.z,
                                           w->norm_attn_w, w->norm_ssm_w, w->beta1, w->beta2, vscale(c, w),
                                           vbias(c, w), U16, B, di, c->rms_eps,
-                                          c->is_kv_producer ? kv->len : nullptr)))
+                                          c->is_kv_producer ? kv->len : nullptr, y_init, y_res, d)))
                 return rc;
             return gemm<f16, TIO>(ctx, "gemm_out_proj_decode", U16, uw, wo16, uw, B, d, uw, eo);
         }
     }
+    plan_split(tc_gemm_ok<T>(U, uw, static_cast<const T*>(w->w_out), uw));
     if ((rc = launch_fuse<I, T>(ctx, nullptr, part, pl.n_split, H, G, dv, concat, ypre, P, pl.ldP, k.z,
                                 w->norm_attn_w, w->norm_ssm_w, w->beta1, w->beta2, vscale(c, w), vbias(c, w), U, B,
-                                di, c->rms_eps, c->is_kv_producer ? kv->len : nullptr)))
+                                di, c->rms_eps, c->is_kv_producer ? kv->len : nullptr, y_init, y_res, d)))
         return rc;
     if ((rc = gemm<T, TIO>(ctx, "gemm_out_proj_decode", U, uw, static_cast<const T*>(w->w_out), uw, B, d, uw, eo)))
         return rc;

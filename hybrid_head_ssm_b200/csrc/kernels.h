@@ -60,6 +60,8 @@ int launch_ssd_scan(const Ctx& ctx, const f16* P, long long ldP, int col_x, int 
 
 // RMSNorm of both branches, SiLU(z) gate, beta scaling and average (U [rows, di]) or
 // concatenation (U [rows, di + H*dv] = [Mamba | attention]); one row per block.
+// Decode only: y_init [rows, d_model] is set to y_res (or zero) for a split-K output
+// projection that adds its partial sums to it.
 // The attention branch is O [rows, H*dv], or, when `part` is given, the decode
 // attention's split partials [rows, H, n_split, dv + 2] merged on the fly (O unused).
 // A consumer's adapted shared V (v_scale, v_bias [G, dv], both or neither) is applied
@@ -68,7 +70,8 @@ template <typename I, typename T>
 int launch_fuse(const Ctx& ctx, const I* O, const float* part, int n_split, int H, int G, int dv, bool concat,
                 const I* ypre, const I* P, long long ldP, int col_z, const float* g_attn, const float* g_ssm,
                 const float* beta1, const float* beta2, const float* v_scale, const float* v_bias, T* U,
-                int rows, int di, float eps, int* len_inc);
+                int rows, int di, float eps, int* len_inc, float* y_init = nullptr, const float* y_res = nullptr,
+                int d_model = 0);
 
 
 // The RoPE table and the zero-padded 16-bit copy of W_dt [rows, cols] -> [rows, ld_dst],

@@ -5,32 +5,40 @@
 //     h_t = exp(Delta_t A) h_{t-1} + (Delta_t B_t) xc_t,   y_t = C_t . h_t + D xc_t
 // with A = -exp(A_log) per (channel, state), the state in fp32 registers.
 //
-// The work per (row, channel) is fixed by the method: 16 exponentials of the state decays
-// (plus the SiLU's and softplus's), which run on the 16-per-clock MUFU unit, and about 48
-// fp32 instructions around them. The kernel is laid out so that little else is issued:
-// one thread per channel holds all 16 states as fp32 pairs (packed FMUL2 / FFMA2 on two
-// states at a time, B_t and C_t read as fp32 quads that the whole warp shares), runs the
-// conv of its channel with the last three inputs in registers, and stores y of its
-// channel (a warp writes 32 consecutive channels). The decays of step t+1 depend only on
-// Delta_{t+1}, so they are computed while step t's state update runs: the exponentials
-// of one step overlap the FMA chain of the previous one.
+// The work per (row, channel) is set by the method: 16 exponentials of the state decays
+// on the 16-per-clock MUFU unit (plus the SiLU's and the softplus's) and about 48 fp32
+// instructions around them. Everything that does not depend on the state is done for a
+// whole chunk of rows in parallel before the recurrence runs, so the recurrence issues
+// little besides its own arithmetic.
 //
-// One block of 64 threads per (64-channel group, sequence). Rows are walked in chunks of
-// 32; cp.async stages chunk k+1 (x, dt_low, B, C) while chunk k is worked on. Per chunk,
-// before the recurrence: Delta from warp-level tensor-core MMAs (m16n8k16, fp16 dt_low
-// rows x the W_dt rows of the warp's 32 channels, which stay in registers, fp32
-// accumulate) plus softplus, written to shared memory in conflict-free 8-byte pairs, and
-// B and C converted to fp32. This kernel is used when B * d_inner is large enough to fill
-// the GPU; smaller batches use the kernel that splits a channel's states over 8 threads
-// (scan.cu).
+// One block of 128 threads per (64-channel group, sequence). Rows are walked in chunks of
+// 32; cp.async stages chunk k+1 (x with a three-row halo, dt_low, B, C) while chunk k is
+// worked on in three phases separated by block barriers:
+//   A1: Delta of the chunk from warp-level tensor-core MMAs (m16n8k16, fp16 dt_low rows x
+//       the W_dt rows of the warp's 16 channels, which stay in registers, fp32
+//       accumulate) plus a branch-free softplus, stored in conflict-free 8-byte pairs;
+//       B and C converted to fp32;
+//   A2: conv + SiLU of every (row, channel), stored with Delta as the pairs
+//       (Delta, Delta xc) the recurrence consumes, and D xc;
+//   B:  the recurrence. Thread (channel c, half s) holds states 8s .. 8s+7 of c as four
+//       fp32 pairs: per row one 8-byte load of (Delta, Delta xc), B_t and C_t of its half
+//       as fp32 quads shared by the warp, four (FMUL2, 2 ex2, FMUL2, FFMA2, FFMA2) groups,
+//       and the next row's decays computed ahead so the exponentials overlap the FMA
+//       chain; the halves add their partial C.h with one shuffle and half 0 stores y.
+// Two threads per channel keep enough warps per SM to hide the latencies; this kernel is
+// used when B * d_inner fills the GPU. Smaller batches use the kernel that splits a
+// channel's states over 8 threads (scan.cu).
 #include "kernels.h"
 
 namespace hymba {
 
 namespace {
 
-constexpr int WCH = 64;            // channels per block = threads per block
+constexpr int WCH = 64;            // channels per block
+constexpr int WTH = 128;           // threads per block: 64 channels x 2 state halves
 constexpr int WTC = 32;            // rows per chunk
+constexpr int WHALO = 3;           // conv history rows staged before each chunk
+constexpr int WXR = WTC + WHALO;   // staged x rows per chunk
 constexpr int WRMAX = 128;         // dt_rank <= WRMAX
 constexpr int WKS = WRMAX / 16;    // MMA k-steps at most
 constexpr int WDLD = WRMAX + 8;    // staged dt_low row stride (fp16): conflict-free ldmatrix rows
@@ -38,16 +46,18 @@ constexpr int WDD = WCH + 8;       // Delta row stride (fp32): conflict-free 8-b
 constexpr float WLOG2E = 1.4426950408889634f;
 
 struct WideSmem {
-    alignas(16) f16 x[2][WTC][WCH];        // pre-conv inputs of the block's channels
+    alignas(16) f16 x[2][WXR][WCH];        // pre-conv inputs of the block's channels, rows t0-3 ..
     alignas(16) f16 dtl[2][WTC][WDLD];     // dt_low rows
     alignas(16) f16 bc[2][WTC][32];        // B (16) then C (16) of each row, as staged
     alignas(16) float bcf[WTC][32];        // the same in fp32, current chunk
     alignas(16) float dlt[WTC][WDD];       // Delta of the current chunk
+    alignas(16) float2 dd[WTC][WCH];       // (Delta, Delta xc)
+    alignas(16) float dx[WTC][WCH];        // D xc
 };
 
-__device__ __forceinline__ void cp16(void* dst, const void* src) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(static_cast<uint32_t>(__cvta_generic_to_shared(dst))),
-                 "l"(src)
+__device__ __forceinline__ void cp16(void* dst, const void* src, bool zero = false) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(static_cast<uint32_t>(__cvta_generic_to_shared(dst))),
+                 "l"(src), "r"(zero ? 0 : 16)
                  : "memory");
 }
 __device__ __forceinline__ void cp8(void* dst, const void* src) {
@@ -90,29 +100,31 @@ __device__ __forceinline__ float softplus_bf(float u) {
     return fmaxf(u, 0.0f) + (e < 9.765625e-4f ? series : lg);
 }
 
-// Stage rows t0 .. t0+WTC-1 of sequence b (rows past Tp repeat the last one; they are
-// never scanned): x of the block's channels, dt_low (r_dt values in 8-byte pieces), B, C.
+// Stage rows t0 .. t0+WTC-1 of sequence b into buffer buf: x of the block's channels with
+// the WHALO rows before t0 (zeros before the first row), dt_low (r_dt values in 8-byte
+// pieces), B and C. Rows past Tp repeat the last one; they are never scanned.
 __device__ __forceinline__ void stage(WideSmem& sm, int buf, int tid, const f16* P, long long ldP, int col_x,
                                      int col_B, int col_dt, int r_dt, int c0, long long row0, int t0, int Tp) {
-    for (int j = tid; j < WTC * (WCH / 8); j += WCH) {
+    for (int j = tid; j < WXR * (WCH / 8); j += WTH) {
         const int rr = j / (WCH / 8), k = j % (WCH / 8);
-        const long long row = row0 + min(t0 + rr, Tp - 1);
-        cp16(&sm.x[buf][rr][8 * k], P + row * ldP + col_x + c0 + 8 * k);
+        const int t = t0 - WHALO + rr;
+        const long long row = row0 + min(max(t, 0), Tp - 1);
+        cp16(&sm.x[buf][rr][8 * k], P + row * ldP + col_x + c0 + 8 * k, t < 0);
     }
-    for (int j = tid; j < WTC * 4; j += WCH) {  // B and C: 32 fp16 = 4 pieces of 16 bytes
-        const int rr = j / 4, k = j % 4;
+    {
+        const int rr = tid / 4, k = tid % 4;  // B and C: 32 fp16 = 4 pieces of 16 bytes per row
         const long long row = row0 + min(t0 + rr, Tp - 1);
         cp16(&sm.bc[buf][rr][8 * k], P + row * ldP + col_B + 8 * k);
     }
     const int pieces = r_dt / 4;
-    for (int j = tid; j < WTC * pieces; j += WCH) {
+    for (int j = tid; j < WTC * pieces; j += WTH) {
         const int rr = j / pieces, k = j - rr * pieces;
         const long long row = row0 + min(t0 + rr, Tp - 1);
         cp8(&sm.dtl[buf][rr][4 * k], P + row * ldP + col_dt + 4 * k);
     }
 }
 
-__global__ void __launch_bounds__(WCH, 3)
+__global__ void __launch_bounds__(WTH, 3)
 conv_scan_wide_kernel(const f16* __restrict__ P, long long ldP, int col_x, int col_B, int col_dt, int r_dt,
                       const f16* __restrict__ wdt, int ld_wdt, const float* __restrict__ b_dt,
                       const float* __restrict__ conv_w, const float* __restrict__ conv_b,
@@ -128,61 +140,64 @@ conv_scan_wide_kernel(const f16* __restrict__ P, long long ldP, int col_x, int c
     const int ks = (r_dt + 15) / 16;
 
     // zero tails of the dt_low buffers (columns the copies never write, read by the MMAs)
-    for (int j = tid; j < 2 * WTC * (WDLD - r_dt); j += WCH) {
+    for (int j = tid; j < 2 * WTC * (WDLD - r_dt); j += WTH) {
         const int bsel = j / (WTC * (WDLD - r_dt)), rem = j - bsel * WTC * (WDLD - r_dt);
         sm.dtl[bsel][rem / (WDLD - r_dt)][r_dt + rem % (WDLD - r_dt)] = __float2half_rn(0.f);
     }
     stage(sm, 0, tid, P, ldP, col_x, col_B, col_dt, r_dt, c0, row0, 0, Tp);
     cp_commit();
 
-    // Delta MMAs: this lane's B fragments of the warp's 32 channels (n-tiles j = 0..3;
+    // A1 constants: this lane's B fragments of the warp's 16 channels (n-tiles j = 0, 1;
     // W_dt is zero-padded to 16 ks columns) and the bias of its output columns
     // 8 j + 2 (lane % 4), +1
     const int g = lane >> 2, q = lane & 3;
-    uint32_t bfr[WKS][4][2];
+    uint32_t bfr[WKS][2][2];
 #pragma unroll
     for (int st = 0; st < WKS; ++st)
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
+        for (int j = 0; j < 2; ++j) {
             bfr[st][j][0] = bfr[st][j][1] = 0u;
             if (st < ks) {
-                const f16* wr = wdt + (long long)(c0 + warp * 32 + 8 * j + g) * ld_wdt + 16 * st + 2 * q;
+                const f16* wr = wdt + (long long)(c0 + warp * 16 + 8 * j + g) * ld_wdt + 16 * st + 2 * q;
                 bfr[st][j][0] = *reinterpret_cast<const uint32_t*>(wr);
                 bfr[st][j][1] = *reinterpret_cast<const uint32_t*>(wr + 8);
             }
         }
-    float2 bdt[4];
+    float2 bdt[2];
 #pragma unroll
-    for (int j = 0; j < 4; ++j) bdt[j] = *reinterpret_cast<const float2*>(b_dt + c0 + warp * 32 + 8 * j + 2 * q);
+    for (int j = 0; j < 2; ++j)
+        bdt[j] = *reinterpret_cast<const float2*>(b_dt + c0 + warp * 16 + 8 * j + 2 * q);
+    // A2: conv of channel cc over rows rh .. rh+15 of each chunk
+    const int cc = tid & (WCH - 1), rh = (tid / WCH) * (WTC / 2);
+    const float4 w4 = *reinterpret_cast<const float4*>(conv_w + (long long)(c0 + cc) * 4);
+    const float cbias = conv_b[c0 + cc], Dcc = Dp[c0 + cc];
 
-    // this thread's channel: conv taps, D, and A of its 16 states (as exp2 factors)
-    const int c = c0 + tid;
-    const float4 w4 = *reinterpret_cast<const float4*>(conv_w + (long long)c * 4);
-    const float cbias = conv_b[c], Dc = Dp[c];
-    float2 A2[8], h[8];
+    // B: channel cl of the block, states 8 s .. 8 s + 7 as pairs
+    const int cl = warp * 16 + (lane >> 1), s = lane & 1;
+    float2 A2[4], h[4];
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
-        const float4 a4 = *reinterpret_cast<const float4*>(A_log + (long long)c * 16 + 4 * k);
+    for (int k = 0; k < 2; ++k) {
+        const float4 a4 = *reinterpret_cast<const float4*>(A_log + (long long)(c0 + cl) * 16 + 8 * s + 4 * k);
         A2[2 * k] = make_float2(-expf(a4.x) * WLOG2E, -expf(a4.y) * WLOG2E);
         A2[2 * k + 1] = make_float2(-expf(a4.z) * WLOG2E, -expf(a4.w) * WLOG2E);
     }
 #pragma unroll
-    for (int k = 0; k < 8; ++k) h[k] = make_float2(0.f, 0.f);
-    float x1 = 0.f, x2 = 0.f, x3 = 0.f;  // x_{t-1}, x_{t-2}, x_{t-3}
+    for (int k = 0; k < 4; ++k) h[k] = make_float2(0.f, 0.f);
 
     for (int kc = 0; kc < nchunk; ++kc) {
         const int buf = kc & 1;
         cp_wait0();
-        __syncthreads();  // chunk kc staged; everyone is past chunk kc-1
+        __syncthreads();  // chunk kc staged; everyone is past chunk kc-1's phase B
         if (kc + 1 < nchunk) stage(sm, buf ^ 1, tid, P, ldP, col_x, col_B, col_dt, r_dt, c0, row0, (kc + 1) * WTC, Tp);
         cp_commit();
-        // ---- Delta of the chunk (rows 16 i + g (+8), channels warp*32 + 8 j + 2 q (+1)) ----
+
+        // ---- A1: Delta (rows 16 i + g (+8), channels warp*16 + 8 j + 2 q (+1)), B/C to fp32 ----
         {
-            float acc[2][4][4];
+            float acc[2][2][4];
 #pragma unroll
             for (int i = 0; i < 2; ++i)
 #pragma unroll
-                for (int j = 0; j < 4; ++j)
+                for (int j = 0; j < 2; ++j)
 #pragma unroll
                     for (int e = 0; e < 4; ++e) acc[i][j][e] = 0.f;
 #pragma unroll
@@ -193,15 +208,15 @@ conv_scan_wide_kernel(const f16* __restrict__ P, long long ldP, int col_x, int c
                         uint32_t a[4];
                         ldmatrix_x4(a, &sm.dtl[buf][16 * i + (lane & 15)][16 * st + 8 * (lane >> 4)]);
 #pragma unroll
-                        for (int j = 0; j < 4; ++j) mma16816(acc[i][j], a, bfr[st][j][0], bfr[st][j][1]);
+                        for (int j = 0; j < 2; ++j) mma16816(acc[i][j], a, bfr[st][j][0], bfr[st][j][1]);
                     }
                 }
             }
 #pragma unroll
             for (int i = 0; i < 2; ++i)
 #pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    const int col = warp * 32 + 8 * j + 2 * q;
+                for (int j = 0; j < 2; ++j) {
+                    const int col = warp * 16 + 8 * j + 2 * q;
                     *reinterpret_cast<float2*>(&sm.dlt[16 * i + g][col]) =
                         make_float2(softplus_bf(acc[i][j][0] + bdt[j].x), softplus_bf(acc[i][j][1] + bdt[j].y));
                     *reinterpret_cast<float2*>(&sm.dlt[16 * i + g + 8][col]) =
@@ -209,80 +224,96 @@ conv_scan_wide_kernel(const f16* __restrict__ P, long long ldP, int col_x, int c
                 }
         }
 #pragma unroll
-        for (int j = tid; j < WTC * 32; j += WCH) sm.bcf[j / 32][j % 32] = __half2float(sm.bc[buf][j / 32][j % 32]);
+        for (int j = tid; j < WTC * 32; j += WTH) sm.bcf[j / 32][j % 32] = __half2float(sm.bc[buf][j / 32][j % 32]);
         __syncthreads();
 
-        // ---- the recurrence over the chunk's rows ----
-        const int nt = min(WTC, Tp - kc * WTC);
-        f16* yrow = ypre + (row0 + (long long)kc * WTC) * di + c;
-        // decays of the first row
-        float d = sm.dlt[0][tid];
-        float2 a[8];
+        // ---- A2: conv + SiLU of channel cc, rows rh .. rh+15 (x row t sits at staged row t + WHALO) ----
+        {
+            float x3 = __half2float(sm.x[buf][rh][cc]);
+            float x2 = __half2float(sm.x[buf][rh + 1][cc]);
+            float x1 = __half2float(sm.x[buf][rh + 2][cc]);
 #pragma unroll
-        for (int k = 0; k < 8; ++k) {
-            const float2 ad = __fmul2_rn(make_float2(d, d), A2[k]);
+            for (int t = rh; t < rh + WTC / 2; ++t) {
+                const float xt = __half2float(sm.x[buf][t + WHALO][cc]);
+                const float u = fmaf(w4.w, xt, fmaf(w4.z, x1, fmaf(w4.y, x2, fmaf(w4.x, x3, cbias))));
+                x3 = x2;
+                x2 = x1;
+                x1 = xt;
+                const float xc = u * rcp_fast(1.0f + fast_exp2(-u * WLOG2E));
+                const float d = sm.dlt[t][cc];
+                sm.dd[t][cc] = make_float2(d, d * xc);
+                sm.dx[t][cc] = Dcc * xc;
+            }
+        }
+        __syncthreads();
+
+        // ---- B: the recurrence ----
+        const int nt = min(WTC, Tp - kc * WTC);
+        f16* yrow = ypre + (row0 + (long long)kc * WTC) * di + c0 + cl;
+        float2 dv = sm.dd[0][cl];
+        float2 a[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const float2 ad = __fmul2_rn(make_float2(dv.x, dv.x), A2[k]);
             a[k] = make_float2(fast_exp2(ad.x), fast_exp2(ad.y));
         }
         auto step = [&](int t) {
-            // conv + SiLU of this channel
-            const float xt = __half2float(sm.x[buf][t][tid]);
-            const float u = fmaf(w4.w, xt, fmaf(w4.z, x1, fmaf(w4.y, x2, fmaf(w4.x, x3, cbias))));
-            x3 = x2;
-            x2 = x1;
-            x1 = xt;
-            const float xc = u * rcp_fast(1.0f + fast_exp2(-u * WLOG2E));
-            const float dxc = d * xc;
-            // the next row's decays (independent of this row's state update)
-            const float dn = t + 1 < WTC ? sm.dlt[t + 1][tid] : 0.f;
-            float2 an[8];
+            // the next row's decays first: they depend only on its Delta
+            const float2 dn = sm.dd[min(t + 1, WTC - 1)][cl];
+            float2 an[4];
 #pragma unroll
-            for (int k = 0; k < 8; ++k) {
-                const float2 ad = __fmul2_rn(make_float2(dn, dn), A2[k]);
+            for (int k = 0; k < 4; ++k) {
+                const float2 ad = __fmul2_rn(make_float2(dn.x, dn.x), A2[k]);
                 an[k] = make_float2(fast_exp2(ad.x), fast_exp2(ad.y));
             }
-            const float4* bq = reinterpret_cast<const float4*>(&sm.bcf[t][0]);
-            const float2 xx = make_float2(dxc, dxc);
-            float2 y0 = make_float2(0.f, 0.f), y1 = make_float2(0.f, 0.f);
+            const float4 b0 = *reinterpret_cast<const float4*>(&sm.bcf[t][8 * s]);
+            const float4 b1 = *reinterpret_cast<const float4*>(&sm.bcf[t][8 * s + 4]);
+            const float4 q0 = *reinterpret_cast<const float4*>(&sm.bcf[t][16 + 8 * s]);
+            const float4 q1 = *reinterpret_cast<const float4*>(&sm.bcf[t][16 + 8 * s + 4]);
+            const float2 xx = make_float2(dv.y, dv.y);
+            h[0] = __ffma2_rn(a[0], h[0], __fmul2_rn(xx, make_float2(b0.x, b0.y)));
+            h[1] = __ffma2_rn(a[1], h[1], __fmul2_rn(xx, make_float2(b0.z, b0.w)));
+            h[2] = __ffma2_rn(a[2], h[2], __fmul2_rn(xx, make_float2(b1.x, b1.y)));
+            h[3] = __ffma2_rn(a[3], h[3], __fmul2_rn(xx, make_float2(b1.z, b1.w)));
+            float2 y0 = __fmul2_rn(make_float2(q0.x, q0.y), h[0]);
+            float2 y1 = __fmul2_rn(make_float2(q0.z, q0.w), h[1]);
+            y0 = __ffma2_rn(make_float2(q1.x, q1.y), h[2], y0);
+            y1 = __ffma2_rn(make_float2(q1.z, q1.w), h[3], y1);
+            const float2 y2 = __fadd2_rn(y0, y1);
+            float ys = y2.x + y2.y;
+            ys += __shfl_xor_sync(0xffffffffu, ys, 1);  // the other half's states
+            if (s == 0) yrow[(long long)t * di] = __float2half_rn(ys + sm.dx[t][cl]);
 #pragma unroll
-            for (int k4 = 0; k4 < 4; ++k4) {
-                const float4 bv = bq[k4], cv = bq[4 + k4];
-                h[2 * k4] = __ffma2_rn(a[2 * k4], h[2 * k4], __fmul2_rn(xx, make_float2(bv.x, bv.y)));
-                h[2 * k4 + 1] = __ffma2_rn(a[2 * k4 + 1], h[2 * k4 + 1], __fmul2_rn(xx, make_float2(bv.z, bv.w)));
-                y0 = __ffma2_rn(make_float2(cv.x, cv.y), h[2 * k4], y0);
-                y1 = __ffma2_rn(make_float2(cv.z, cv.w), h[2 * k4 + 1], y1);
-            }
-            const float2 ys = __fadd2_rn(y0, y1);
-            yrow[(long long)t * di] = __float2half_rn(fmaf(Dc, xc, ys.x + ys.y));
-#pragma unroll
-            for (int k = 0; k < 8; ++k) a[k] = an[k];
-            d = dn;
+            for (int k = 0; k < 4; ++k) a[k] = an[k];
+            dv = dn;
         };
         if (nt == WTC) {
-#pragma unroll 2
+#pragma unroll 4
             for (int t = 0; t < WTC; ++t) step(t);
         } else {
             for (int t = 0; t < nt; ++t) step(t);
         }
-        if (kc + 1 == nchunk && conv_out) {
-            // conv state: the last four inputs of the sequence, oldest first (zeros before
-            // the first row)
-            float x4 = 0.f;
-            if (nt >= 4) x4 = __half2float(sm.x[buf][nt - 4][tid]);
-            else if (kc > 0) x4 = __half2float(sm.x[buf ^ 1][WTC + nt - 4][tid]);  // the previous chunk's rows
-            *reinterpret_cast<float4*>(conv_out + ((long long)b * di + c) * 4) = make_float4(x4, x3, x2, x1);
-        }
+    }
+    if (conv_out && tid < WCH) {
+        // conv state: the last four inputs of the sequence, oldest first (staged rows of
+        // the last chunk; the halo holds zeros before the first row)
+        const int tl = Tp - (nchunk - 1) * WTC + WHALO;  // staged index of row Tp
+        const int lb = (nchunk - 1) & 1;
+        *reinterpret_cast<float4*>(conv_out + ((long long)b * di + c0 + tid) * 4) =
+            make_float4(__half2float(sm.x[lb][tl - 4][tid]), __half2float(sm.x[lb][tl - 3][tid]),
+                        __half2float(sm.x[lb][tl - 2][tid]), __half2float(sm.x[lb][tl - 1][tid]));
     }
     if (h_out) {
-        float* hp = h_out + ((long long)b * di + c) * 16;
+        float* hp = h_out + ((long long)b * di + c0 + cl) * 16 + 8 * s;
 #pragma unroll
-        for (int k = 0; k < 8; ++k) *reinterpret_cast<float2*>(hp + 2 * k) = h[k];
+        for (int k = 0; k < 4; ++k) *reinterpret_cast<float2*>(hp + 2 * k) = h[k];
     }
 }
 
 }  // namespace
 
 bool scan_wide_applies(int B, int di, int dt_rank, int sm_count) {
-    // one thread per channel: the GPU needs a few blocks of 64 per SM
+    // two threads per channel: the GPU needs a few blocks of 128 per SM
     return di % WCH == 0 && dt_rank > 0 && dt_rank <= WRMAX && dt_rank % 4 == 0 &&
            (long long)B * (di / WCH) >= 2LL * sm_count;
 }
@@ -302,7 +333,7 @@ int launch_conv_scan_wide(const Ctx& ctx, const f16* P, long long ldP, int col_x
     const size_t smem = sizeof(WideSmem);
     static std::atomic<unsigned long long> smem_set{0};
     if (!smem_opt_in_once(smem_set, conv_scan_wide_kernel, smem, ctx)) return HYMBA_ERR_CUDA;
-    HYMBA_LAUNCH(ctx, "conv_scan_prefill", conv_scan_wide_kernel, grid, WCH, smem, P, ldP, col_x, col_B, col_dt,
+    HYMBA_LAUNCH(ctx, "conv_scan_prefill", conv_scan_wide_kernel, grid, WTH, smem, P, ldP, col_x, col_B, col_dt,
                  dt_rank, wdt, ld_wdt, b_dt, conv_w, conv_b, A_log, D, ypre, h_out, conv_out, Tp, di);
     return HYMBA_OK;
 }
