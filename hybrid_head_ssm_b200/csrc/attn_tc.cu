@@ -64,7 +64,7 @@ struct AttnSmem {
     uint64_t q_full;
     uint64_t k_full[KST], k_empty[KST];
     uint64_t v_full[VST], v_empty[VST];
-    uint64_t s_full[2], pv_done[2], o_done[2], drain[2];
+    uint64_t s_full[2], p_full[2], pv_done[2], o_done[2], drain;
     uint32_t tmem_base;
     int abort;
 };
@@ -191,10 +191,11 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
         }
         for (int t = 0; t < 2; ++t) {
             tc::mbar_init(&s.s_full[t], 1);
+            tc::mbar_init(&s.p_full[t], QT);
             tc::mbar_init(&s.pv_done[t], 1);
             tc::mbar_init(&s.o_done[t], 1);
-            tc::mbar_init(&s.drain[t], 1);
         }
+        tc::mbar_init(&s.drain, 1);
         s.abort = 0;
         tc::fence_mbar_init();
         tc::prefetch_tmap(&tmQ);
@@ -256,6 +257,99 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
                     for (int i = 0; i < VST; ++i)
                         if (last_phase[i] >= 0) tc::mbar_wait(&s.v_full[i], (uint32_t)last_phase[i], &zero);
             }
+        } else if (warp == 1) {
+            // ---------------- MMA issuer ----------------
+            if (tc::elect_one()) {
+                bool ok = tc::mbar_wait(&s.q_full, 0, abort, wlim);
+                if (!ok) fail(abort, status, 1, 0, 0);
+                const int n_t[2] = {blk.count(0), blk.count(1)};
+                int jS[2] = {blk.nth(0, 0), blk.nth(1, 0)};  // union block of each tile's next S
+                int jP[2] = {jS[0], jS[1]};                  // ... and of its next PV
+                int uS[2] = {0, 0}, uP[2] = {0, 0};
+                // S_t(u) = Q_t K_j^T; frees the K stage (two commits when the other tile
+                // skips block j)
+                auto issue_s = [&](int t) -> bool {
+                    const int j = jS[t];
+                    const int kst = j % KST;
+                    if (!tc::mbar_wait(&s.k_full[kst], (j / KST) & 1, abort, wlim)) { fail(abort, status, 1, j, 2); return false; }
+                    tc::tc_fence_after();
+                    const uint32_t qa = tc::smem_u32(s.q[t]);
+                    const uint32_t ka = tc::smem_u32(s.k[kst]);
+                    const uint32_t sd = tmem + TM_S + t * 128;
+#pragma unroll
+                    for (int kk = 0; kk < DH / 16; ++kk)
+                        tc::mma_f16_ss(sd, tc::sdesc_k_sw128(qa + kk * 32), tc::sdesc_k_sw128(ka + kk * 32), IDESC_S,
+                                       kk > 0);
+                    tc::mma_commit(&s.s_full[t]);
+                    tc::mma_commit(&s.k_empty[kst]);
+                    if (blk.users(j) == 1) tc::mma_commit(&s.k_empty[kst]);
+                    ++uS[t];
+                    int nj = jS[t] + 1;
+                    while (nj < nblk && !blk.uses(t, nj)) ++nj;
+                    jS[t] = uS[t] < n_t[t] ? nj : -1;
+                    return true;
+                };
+                // O_t += P_t V_j, P_t read from TMEM (the tile's S columns)
+                auto issue_pv = [&](int t) -> bool {
+                    const int j = jP[t], u = uP[t];
+                    const int vst = j % VST;
+                    if (!tc::mbar_wait(&s.p_full[t], u & 1, abort, wlim)) { fail(abort, status, 1, j, 4 + t); return false; }
+                    if (!tc::mbar_wait(&s.v_full[vst], (j / VST) & 1, abort, wlim)) { fail(abort, status, 1, j, 10); return false; }
+                    tc::tc_fence_after();
+                    const uint32_t va = tc::smem_u32(s.v[vst][0]);
+                    const uint32_t pa = tmem + TM_S + t * 128;
+#pragma unroll
+                    for (int kk = 0; kk < KBLK / 16; ++kk)
+                        mma_f16_ts(tmem + TM_O + t * 128, pa + kk * 8, tc::sdesc_mn_sw128(va + kk * 2048, KBLK * 128),
+                                   IDESC_PV, (u > 0 || kk > 0));
+                    tc::mma_commit(&s.pv_done[t]);
+                    tc::mma_commit(&s.v_empty[vst]);
+                    if (blk.users(j) == 1) tc::mma_commit(&s.v_empty[vst]);
+                    ++uP[t];
+                    int nj = jP[t] + 1;
+                    while (nj < nblk && !blk.uses(t, nj)) ++nj;
+                    jP[t] = uP[t] < n_t[t] ? nj : -1;
+                    if (uP[t] == n_t[t]) tc::mma_commit(&s.o_done[t]);
+                    return true;
+                };
+                for (int t = 0; ok && t < 2; ++t)
+                    if (n_t[t] > 0) ok = issue_s(t);
+                // then whatever is ready, tiles in turn: the PV of a tile once its softmax
+                // wrote P, and its next S once that PV completed (S overwrites P)
+                long long t_idle = 0;
+                uint32_t spins = 0;
+                while (ok && (uP[0] < n_t[0] || uP[1] < n_t[1])) {
+                    bool progressed = false;
+                    for (int t = 0; ok && t < 2; ++t) {
+                        if (uP[t] < uS[t] && tc::mbar_test_wait(&s.p_full[t], uP[t] & 1) &&
+                            tc::mbar_test_wait(&s.v_full[jP[t] % VST], (jP[t] / VST) & 1)) {
+                            ok = issue_pv(t);
+                            progressed = true;
+                        }
+                        if (ok && uS[t] < n_t[t] && uS[t] == uP[t] &&
+                            tc::mbar_test_wait(&s.pv_done[t], (uP[t] - 1) & 1) &&
+                            tc::mbar_test_wait(&s.k_full[jS[t] % KST], (jS[t] / KST) & 1)) {
+                            ok = issue_s(t);
+                            progressed = true;
+                        }
+                    }
+                    if (progressed) {
+                        t_idle = 0;
+                    } else if ((++spins & 255) == 0) {
+                        const long long now = clock64();
+                        if (*abort) ok = false;
+                        else if (t_idle == 0) t_idle = now;
+                        else if (now - t_idle > wlim) {
+                            fail(abort, status, 1, uP[0] + uP[1], 11);
+                            ok = false;
+                        }
+                    }
+                }
+                // drain: every MMA issued has completed before the block exits
+                tc::mma_commit(&s.drain);
+                int zero = 0;
+                tc::mbar_wait(&s.drain, 0, &zero);
+            }
         }
     } else {
         setmaxnreg_inc<REG_SOFT>();
@@ -274,59 +368,16 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
         const int wa = window > 0 ? max(n_meta, i - window + 1) : n_meta;
         float m_used = -INFINITY, l = 0.f;
         bool ok = true;
-        // The tile's MMAs are issued by lane 0 of its first softmax warp, right after the
-        // tile's four warps pass a named barrier with P stored: S_t = Q_t K_j^T into the
-        // tile's S columns, O_t += P_t V_j with P_t read from those columns, and the next
-        // S_t once that PV has completed (it overwrites P_t). No polling warp sits between
-        // a softmax step and the MMAs it releases.
-        const bool issuer = q == 0 && lane == 0;
-        const uint32_t sd = tmem + TM_S + t * 128, od = tmem + TM_O + t * 128;
-        auto next_block = [&](int jj) {
-            do { ++jj; } while (jj < nblk && !blk.uses(t, jj));
-            return jj;
-        };
-        auto issue_s = [&](int jb) -> bool {
-            const int kst = jb % KST;
-            if (!tc::mbar_wait(&s.k_full[kst], (jb / KST) & 1, abort, wlim)) { fail(abort, status, 1, jb, 2); return false; }
-            tc::tc_fence_after();
-            const uint32_t qa = tc::smem_u32(s.q[t]);
-            const uint32_t ka = tc::smem_u32(s.k[kst]);
-#pragma unroll
-            for (int kk = 0; kk < DH / 16; ++kk)
-                tc::mma_f16_ss(sd, tc::sdesc_k_sw128(qa + kk * 32), tc::sdesc_k_sw128(ka + kk * 32), IDESC_S, kk > 0);
-            tc::mma_commit(&s.s_full[t]);
-            // frees the K stage (two commits when the other tile skips block jb)
-            tc::mma_commit(&s.k_empty[kst]);
-            if (blk.users(jb) == 1) tc::mma_commit(&s.k_empty[kst]);
-            return true;
-        };
-        auto issue_pv = [&](int jb, int u) -> bool {
-            const int vst = jb % VST;
-            if (!tc::mbar_wait(&s.v_full[vst], (jb / VST) & 1, abort, wlim)) { fail(abort, status, 1, jb, 10); return false; }
-            tc::tc_fence_after();
-            const uint32_t va = tc::smem_u32(s.v[vst][0]);
-#pragma unroll
-            for (int kk = 0; kk < KBLK / 16; ++kk)
-                mma_f16_ts(od, sd + kk * 8, tc::sdesc_mn_sw128(va + kk * 2048, KBLK * 128), IDESC_PV, (u > 0 || kk > 0));
-            tc::mma_commit(&s.v_empty[vst]);
-            if (blk.users(jb) == 1) tc::mma_commit(&s.v_empty[vst]);
-            return true;
-        };
-        if (issuer && nt > 0) {
-            if (!tc::mbar_wait(&s.q_full, 0, abort, wlim)) fail(abort, status, 1, 0, 0);
-            else issue_s(blk.nth(t, 0));
-        }
         int j = -1;
         for (int u = 0; u < nt; ++u) {
-            j = next_block(j);
+            do { ++j; } while (!blk.uses(t, j));
             // tcgen05.ld/st are warp-collective: every decision that guards them is taken
             // by the whole warp (__all_sync / __any_sync)
-            ok = __all_sync(0xffffffffu, ok && !*abort);
-            if (ok && !__all_sync(0xffffffffu, tc::mbar_wait(&s.s_full[t], u & 1, abort, wlim))) {
+            if (!__all_sync(0xffffffffu, tc::mbar_wait(&s.s_full[t], u & 1, abort, wlim))) {
                 if (lane == 0) fail(abort, status, 2, u, 5);
                 ok = false;
+                break;
             }
-            if (ok) {
             tc::tc_fence_after();
             // the four 32-column loads in flight together, one wait
             uint32_t sr[4][32];
@@ -397,31 +448,8 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
                 tc::tmem_wait_st();
             }
             tc::tc_fence_before();
-            }
-            // every warp of the tile passes the barrier once per block, also after a failed
-            // wait, so that none of them waits at it for good
-            asm volatile("barrier.sync %0, %1;" ::"r"(1 + t), "r"(128) : "memory");
-            if (issuer && ok && !*abort) {
-                tc::tc_fence_after();
-                if (issue_pv(j, u)) {
-                    if (u + 1 < nt) {
-                        tc::mma_commit(&s.pv_done[t]);
-                        // the next S_t overwrites P_t: wait until this PV has read it
-                        if (!tc::mbar_wait(&s.pv_done[t], u & 1, abort, wlim)) fail(abort, status, 1, j, 4 + t);
-                        else issue_s(next_block(j));
-                    } else {
-                        tc::mma_commit(&s.o_done[t]);
-                    }
-                }
-            }
+            tc::mbar_arrive(&s.p_full[t]);
         }
-        if (issuer && nt > 0 && *abort) {
-            // every MMA this thread issued has completed before the block exits
-            int zero = 0;
-            tc::mma_commit(&s.drain[t]);
-            tc::mbar_wait(&s.drain[t], 0, &zero);
-        }
-        ok = __all_sync(0xffffffffu, ok && !*abort);
         if (ok && nt > 0 && __all_sync(0xffffffffu, tc::mbar_wait(&s.o_done[t], 0, abort, wlim))) {
             tc::tc_fence_after();
             const float inv = l > 0.f ? 1.f / l : 0.f;

@@ -210,10 +210,10 @@ attn_decode_kernel(const T* __restrict__ P, long long ldP, const T* __restrict__
         float sum = 0.f;
 #pragma unroll
         for (int k = 0; k < KGROUPS; ++k) sum += red[k][r][e];
-        part[(((long long)b * H + g * R + r) * n_split + s) * (DV + 2) + e] = sum;
+        part[(((long long)b * H + g * R + r) * n_split + s) * (DV + 4) + e] = sum;
     }
     if (tid < R) {
-        float* st = part + (((long long)b * H + g * R + tid) * n_split + s) * (DV + 2) + DV;
+        float* st = part + (((long long)b * H + g * R + tid) * n_split + s) * (DV + 4) + DV;
         st[0] = nk > 0 ? stat[tid][0] : -INFINITY;
         st[1] = nk > 0 ? stat[tid][1] : 0.f;
     }
@@ -430,10 +430,10 @@ attn_decode_bulk_kernel(const f16* __restrict__ P, long long ldP, const f16* __r
         float sum = 0.f;
 #pragma unroll
         for (int w = 0; w < 4; ++w) sum += red[(w * R + r) * DV + e];
-        part[(((long long)b * H + g * R + r) * n_split + s) * (DV + 2) + e] = sum;
+        part[(((long long)b * H + g * R + r) * n_split + s) * (DV + 4) + e] = sum;
     }
     if (tid < R) {
-        float* o = part + (((long long)b * H + g * R + tid) * n_split + s) * (DV + 2) + DV;
+        float* o = part + (((long long)b * H + g * R + tid) * n_split + s) * (DV + 4) + DV;
         o[0] = nk > 0 ? stat[2 * tid] : -INFINITY;
         o[1] = nk > 0 ? stat[2 * tid + 1] : 0.f;
     }
@@ -444,16 +444,16 @@ __global__ void __launch_bounds__(DV)
 attn_decode_combine_kernel(const float* __restrict__ part, int n_split, T* __restrict__ O, int H) {
     griddep_sync();
     const int h = blockIdx.x, b = blockIdx.y, e = threadIdx.x;
-    const float* base = part + ((long long)b * H + h) * n_split * (DV + 2);
+    const float* base = part + ((long long)b * H + h) * n_split * (DV + 4);
     float M = -INFINITY;
-    for (int s = 0; s < n_split; ++s) M = fmaxf(M, base[s * (DV + 2) + DV]);
+    for (int s = 0; s < n_split; ++s) M = fmaxf(M, base[s * (DV + 4) + DV]);
     float num = 0.f, den = 0.f;
     if (M != -INFINITY) {
         for (int s = 0; s < n_split; ++s) {
-            const float ms = base[s * (DV + 2) + DV];
+            const float ms = base[s * (DV + 4) + DV];
             const float w = exp2f(ms - M);
-            num = fmaf(w, base[s * (DV + 2) + e], num);
-            den = fmaf(w, base[s * (DV + 2) + DV + 1], den);
+            num = fmaf(w, base[s * (DV + 4) + e], num);
+            den = fmaf(w, base[s * (DV + 4) + DV + 1], den);
         }
     }
     O[((long long)b * H + h) * DV + e] = from_f<T>(den > 0.f ? num / den : 0.f);

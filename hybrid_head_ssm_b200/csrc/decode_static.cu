@@ -8,7 +8,7 @@
 
 namespace hymba {
 
-// Partial results of the key splits: [B, n_q_heads, n_split, v_head_dim + 2] fp32.
+// Partial results of the key splits: [B, n_q_heads, n_split, v_head_dim + 4] fp32.
 // Every GPU that loads the library holds this array until the process exits.
 static constexpr size_t kStaticScratchBytes = size_t(8) << 20;
 static __device__ __align__(256) float g_decode_scratch[kStaticScratchBytes / sizeof(float)];
@@ -48,7 +48,7 @@ extern "C" int hymba_attn_decode_static(const hymba_layer_cfg* cfg, const void* 
         return HYMBA_ERR_KV_INCOMPATIBLE;
     if (ldq < (int64_t)cfg->n_q_heads * 64) return HYMBA_ERR_INVALID_ARG;
     const int n_split = (kv->cache_cap + 255) / 256;
-    const size_t need = (size_t)B * cfg->n_q_heads * n_split * (cfg->v_head_dim + 2) * sizeof(float);
+    const size_t need = (size_t)B * cfg->n_q_heads * n_split * (cfg->v_head_dim + 4) * sizeof(float);
     if (need > kStaticScratchBytes) return HYMBA_ERR_SCRATCH_LIMIT;
     float* scratch = nullptr;
     int rc = static_scratch(&scratch);

@@ -61,7 +61,7 @@ __device__ __forceinline__ void load8f(const float* p, float* v) {
     v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
 }
 
-// Merge weights of a row's split partials (layout [row, head, split, dv + 2]: dv sums,
+// Merge weights of a row's split partials (layout [row, head, split, dv + 4]: dv sums,
 // then the split's max logit and sum of weights): w[head][s] = exp2(m_s - M) / den with
 // M = max_s m_s and den = sum_s exp2(m_s - M) l_s, formed once per (row, head) by the
 // block into shared memory (zero for a head that saw no key).
@@ -70,16 +70,16 @@ __device__ __forceinline__ void merge_weights(const float* __restrict__ part, in
     // one warp per head, one lane per split (in rounds of 32 splits)
     const int warp = t >> 5, lane = t & 31, nwarps = nthreads >> 5;
     for (int hd = warp; hd < H; hd += nwarps) {
-        const float* base = part + ((long long)row * H + hd) * n_split * (dv + 2) + dv;
+        const float* base = part + ((long long)row * H + hd) * n_split * (dv + 4) + dv;
         float M = -INFINITY;
-        for (int s = lane; s < n_split; s += 32) M = fmaxf(M, base[s * (dv + 2)]);
+        for (int s = lane; s < n_split; s += 32) M = fmaxf(M, base[s * (dv + 4)]);
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
         float den = 0.f;
         for (int s = lane; s < n_split; s += 32) {
-            const float w = M != -INFINITY ? exp2f(base[s * (dv + 2)] - M) : 0.f;
+            const float w = M != -INFINITY ? exp2f(base[s * (dv + 4)] - M) : 0.f;
             wts[hd * n_split + s] = w;
-            den = fmaf(w, base[s * (dv + 2) + 1], den);
+            den = fmaf(w, base[s * (dv + 4) + 1], den);
         }
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
@@ -93,7 +93,7 @@ __device__ __forceinline__ void merge_weights(const float* __restrict__ part, in
 __device__ __forceinline__ void merge8(const float* __restrict__ part, int n_split, int H, int dv,
                                        long long row, int c, const float* wts, float* o) {
     const int hd = c / dv, e = c - hd * dv;
-    const float* base = part + ((long long)row * H + hd) * n_split * (dv + 2) + e;
+    const float* base = part + ((long long)row * H + hd) * n_split * (dv + 4) + e;
     const float* w = wts + hd * n_split;
 #pragma unroll
     for (int i = 0; i < 8; ++i) o[i] = 0.f;
@@ -102,9 +102,10 @@ __device__ __forceinline__ void merge8(const float* __restrict__ part, int n_spl
         float4 v[4][2];
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
-            const float* ps = base + (s + u) * (dv + 2);
-            v[u][0] = make_float4(ps[0], ps[1], ps[2], ps[3]);
-            v[u][1] = make_float4(ps[4], ps[5], ps[6], ps[7]);
+            // records of dv + 4 floats start on 16-byte boundaries
+            const float4* ps = reinterpret_cast<const float4*>(base + (s + u) * (dv + 4));
+            v[u][0] = ps[0];
+            v[u][1] = ps[1];
         }
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
@@ -116,7 +117,7 @@ __device__ __forceinline__ void merge8(const float* __restrict__ part, int n_spl
         }
     }
     for (; s < n_split; ++s) {
-        const float* ps = base + s * (dv + 2);
+        const float* ps = base + s * (dv + 4);
         const float wu = w[s];
 #pragma unroll
         for (int i = 0; i < 8; ++i) o[i] = fmaf(wu, ps[i], o[i]);

@@ -219,7 +219,7 @@ static Plan plan(const hymba_layer_cfg* c, int B, int T, int mode) {
     }
     if (mode == HYMBA_MODE_DECODE) {
         p.n_split = decode_splits(T);
-        p.part = take(&cur, (size_t)B * c->n_q_heads * p.n_split * (c->v_head_dim + 2) * sizeof(float));
+        p.part = take(&cur, (size_t)B * c->n_q_heads * p.n_split * (c->v_head_dim + 4) * sizeof(float));
     }
     p.total = cur;
     return p;

@@ -24,7 +24,7 @@
 //       fp32 pairs: per row one 8-byte load of (Delta, Delta xc), B_t and C_t of its half
 //       as fp32 quads shared by the warp, four (FMUL2, 2 ex2, FMUL2, FFMA2, FFMA2) groups,
 //       and the next row's decays computed ahead so the exponentials overlap the FMA
-//       chain; the halves add their partial C.h with one shuffle and half 0 stores y.
+//       chain; the halves add their partial C.h with one shuffle and both store y.
 // Two threads per channel keep enough warps per SM to hide the latencies; this kernel is
 // used when B * d_inner fills the GPU. Smaller batches use the kernel that splits a
 // channel's states over 8 threads (scan.cu).
@@ -250,7 +250,10 @@ conv_scan_wide_kernel(const f16* __restrict__ P, long long ldP, int col_x, int c
         // ---- B: the recurrence ----
         const int nt = min(WTC, Tp - kc * WTC);
         f16* yrow = ypre + (row0 + (long long)kc * WTC) * di + c0 + cl;
-        float2 dv = sm.dd[0][cl];
+        const float2* ddc = &sm.dd[0][cl];
+        const float* bcs = &sm.bcf[0][8 * s];
+        const float* dxc = &sm.dx[0][cl];
+        float2 dv = ddc[0];
         float2 a[4];
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
@@ -259,17 +262,15 @@ conv_scan_wide_kernel(const f16* __restrict__ P, long long ldP, int col_x, int c
         }
         auto step = [&](int t) {
             // the next row's decays first: they depend only on its Delta
-            const float2 dn = sm.dd[min(t + 1, WTC - 1)][cl];
+            const float2 dn = ddc[min(t + 1, WTC - 1) * WCH];
             float2 an[4];
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
                 const float2 ad = __fmul2_rn(make_float2(dn.x, dn.x), A2[k]);
                 an[k] = make_float2(fast_exp2(ad.x), fast_exp2(ad.y));
             }
-            const float4 b0 = *reinterpret_cast<const float4*>(&sm.bcf[t][8 * s]);
-            const float4 b1 = *reinterpret_cast<const float4*>(&sm.bcf[t][8 * s + 4]);
-            const float4 q0 = *reinterpret_cast<const float4*>(&sm.bcf[t][16 + 8 * s]);
-            const float4 q1 = *reinterpret_cast<const float4*>(&sm.bcf[t][16 + 8 * s + 4]);
+            const float4* bq = reinterpret_cast<const float4*>(bcs + t * 32);
+            const float4 b0 = bq[0], b1 = bq[1], q0 = bq[4], q1 = bq[5];
             const float2 xx = make_float2(dv.y, dv.y);
             h[0] = __ffma2_rn(a[0], h[0], __fmul2_rn(xx, make_float2(b0.x, b0.y)));
             h[1] = __ffma2_rn(a[1], h[1], __fmul2_rn(xx, make_float2(b0.z, b0.w)));
@@ -282,13 +283,15 @@ conv_scan_wide_kernel(const f16* __restrict__ P, long long ldP, int col_x, int c
             const float2 y2 = __fadd2_rn(y0, y1);
             float ys = y2.x + y2.y;
             ys += __shfl_xor_sync(0xffffffffu, ys, 1);  // the other half's states
-            if (s == 0) yrow[(long long)t * di] = __float2half_rn(ys + sm.dx[t][cl]);
+            // both halves hold y and store the same value (no divergent branch per row)
+            yrow[(long long)t * di] = __float2half_rn(ys + dxc[t * WCH]);
 #pragma unroll
             for (int k = 0; k < 4; ++k) a[k] = an[k];
             dv = dn;
         };
         if (nt == WTC) {
-#pragma unroll 4
+            // fully unrolled: every shared-memory address is the base plus a constant
+#pragma unroll
             for (int t = 0; t < WTC; ++t) step(t);
         } else {
             for (int t = 0; t < nt; ++t) step(t);

@@ -296,7 +296,7 @@ uint64_t hymba_ssm_state_bytes(int n_layers, int channels, int d_state, int batc
  *   o:  device [B, n_q_heads * v_head_dim], same element type.
  * The partial results of its key splits live in one file-scope device array of 8 MiB
  * (every GPU that loads the library holds it until the process exits). Requests with
- * B * n_q_heads * ceil(cache_cap / 256) * (v_head_dim + 2) * 4 bytes above that return
+ * B * n_q_heads * ceil(cache_cap / 256) * (v_head_dim + 4) * 4 bytes above that return
  * HYMBA_ERR_SCRATCH_LIMIT and queue no work. The first call on a device looks up the
  * array's device address (with that device current); make that first call before any
  * stream capture. All calls share the one array, and every call writes each partial
@@ -343,8 +343,9 @@ int hymba_debug_stalled_wait(void* stream);
  * out[9] the decode split count. rows = B * (n_meta + T) for prefill, B for decode
  * (where T is the cache_cap of the KV cache). A decode step writes neither Delta (it
  * stays in the SSM step's registers) nor O: its attention stays as the split partials
- * [B, n_q_heads, splits, v_head_dim + 2] fp32 (per split: the unnormalised sum of
- * p v, the split's max logit in base 2, the sum of p), which the fusion merges.
+ * [B, n_q_heads, splits, v_head_dim + 4] fp32 (per split: the unnormalised sum of
+ * p v, the split's max logit in base 2, the sum of p, and two pad words so that each
+ * record starts on a 16-byte boundary), which the fusion merges.
  * Requires n >= 10. */
 int hymba_workspace_layout(const hymba_layer_cfg* cfg, int B, int T, int mode, int64_t* out, int n);
 

@@ -184,8 +184,8 @@ def _decode_visibility(cfg, B, cap, lens, seed, static=False):
                 rt.decode(layer, x, kvs, st, y, ws, 0)
                 torch.cuda.synchronize()
                 assert hy.hymba_get_device_status(None) == 0
-                n = B * H * ns * (dv + 2)
-                part = ws[lay["part"]:lay["part"] + n * 4].view(torch.float32).view(B, H, ns, dv + 2)
+                n = B * H * ns * (dv + 4)  # records: dv sums, max logit, sum of p, two pad words
+                part = ws[lay["part"]:lay["part"] + n * 4].view(torch.float32).view(B, H, ns, dv + 4)
                 part = part.double().cpu().numpy()
                 # p = 1 for every visible key: the split sums of p v are 0/(b+1) one-hot
                 # counts, the split sums of p count the keys; normalise by the total

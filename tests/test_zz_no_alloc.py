@@ -44,9 +44,10 @@ def _decoded_layer(cfg, B, T0, cache_cap, seed):
     # the query rows (after RoPE) sit in the projection block of the workspace
     q = ws[lay["P"]:lay["P"] + B * ldp * esz].view(mdt).view(B, ldp)
     ns = lay["n_split"]
-    n_part = B * H * ns * (dv + 2)
-    part = ws[lay["part"]:lay["part"] + n_part * 4].view(torch.float32).view(B, H, ns, dv + 2)
-    o_ref = merge_split_partials(part.double().cpu().numpy()).reshape(B, H * dv)
+    # records of dv + 4 floats: dv sums, the max logit, the sum of p, two pad words
+    n_part = B * H * ns * (dv + 4)
+    part = ws[lay["part"]:lay["part"] + n_part * 4].view(torch.float32).view(B, H, ns, dv + 4)
+    o_ref = merge_split_partials(part[..., :dv + 2].double().cpu().numpy()).reshape(B, H * dv)
     return dict(layer=layer, kv=kv, q=q, ldp=ldp, o_ref=o_ref, mdt=mdt)
 
 
@@ -88,11 +89,11 @@ def test_static_decode_attention_matches_mixer_decode(kind):
 
 
 def test_static_decode_attention_rejects_requests_beyond_its_scratch():
-    """B * n_q_heads * splits * (v_head_dim + 2) * 4 bytes must fit the fixed 8 MiB."""
+    """B * n_q_heads * splits * (v_head_dim + 4) * 4 bytes must fit the fixed 8 MiB."""
     torch = torch_cuda()
     import hybrid_head_ssm_b200 as hy
     cfg = synth.hymba15_layer_cfg(window=0)
-    B, cap = 64, 128 + 8192  # 33 splits: 64 * 25 * 33 * 130 * 4 bytes > 8 MiB
+    B, cap = 64, 128 + 8192  # 33 splits: 64 * 25 * 33 * 132 * 4 bytes > 8 MiB
     kv = hy.kv_struct(cfg, B)
     kv.k_cache = kv.v_cache = kv.len = 1 << 30  # never dereferenced: the check comes first
     kv.cache_cap = cap
