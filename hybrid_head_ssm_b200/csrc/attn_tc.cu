@@ -129,6 +129,12 @@ __device__ __forceinline__ void setmaxnreg_inc() { asm volatile("setmaxnreg.inc.
 template <uint32_t N>
 __device__ __forceinline__ void setmaxnreg_dec() { asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N)); }
 
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+
 // D[tmem] (+)= A[tmem] * B[smem]: the A operand (M x K, 16-bit, two K elements per
 // 32-bit column) read from tensor memory.
 __device__ __forceinline__ void mma_f16_ts(uint32_t tmem_d, uint32_t tmem_a, uint64_t bdesc, uint32_t idesc,
@@ -395,15 +401,18 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
 #pragma unroll
                 for (int c = 0; c < 128; ++c) sv[c] = (unsigned)(k0 + c - a) < span ? sv[c] : -INFINITY;
             }
+            // row max with three-input max: 8 independent chains over the 128 scores
             float mx8[8];
 #pragma unroll
-            for (int c = 0; c < 8; ++c) mx8[c] = fmaxf(sv[c], sv[c + 8]);
+            for (int c = 0; c < 8; ++c) mx8[c] = fmax3(sv[c], sv[c + 8], sv[c + 16]);
 #pragma unroll
-            for (int c = 16; c < 128; c += 8)
+            for (int c = 24; c + 16 < 128; c += 16)
 #pragma unroll
-                for (int x = 0; x < 8; ++x) mx8[x] = fmaxf(mx8[x], sv[c + x]);
-            const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                                   fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]))) * scale;
+                for (int x = 0; x < 8; ++x) mx8[x] = fmax3(mx8[x], sv[c + x], sv[c + 8 + x]);
+#pragma unroll
+            for (int x = 0; x < 8; ++x) mx8[x] = fmaxf(mx8[x], sv[120 + x]);
+            const float mx = fmax3(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(mx8[3], mx8[4], mx8[5]),
+                                   fmaxf(mx8[6], mx8[7])) * scale;
             // a row whose running max grows by more than 2^8 moves to the new max; its O
             // (PV of the earlier blocks, all completed: this S was issued after the last
             // PV of the tile completed) is scaled in TMEM once P is stored (before the PV
