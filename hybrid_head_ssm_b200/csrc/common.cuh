@@ -52,6 +52,35 @@ static inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 b
     return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
+// As launch_pdl, with the grid divided into thread-block clusters of cluster_x CTAs along x.
+template <typename... KArgs, typename... Args>
+static inline cudaError_t launch_pdl_cluster(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                                             unsigned cluster_x, cudaStream_t stream, Args&&... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = cluster_x;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
+#define HYMBA_LAUNCH_CLUSTER(ctx, name, kernel, grid, block, smem, cluster_x, ...)              \
+    do {                                                                                         \
+        ::hymba::trace_before((ctx), (name));                                                    \
+        const cudaError_t launch_err_ = ::hymba::launch_pdl_cluster(                             \
+            kernel, dim3(grid), dim3(block), (size_t)(smem), (cluster_x), (ctx).stream, __VA_ARGS__); \
+        if (::hymba::trace_after((ctx), (name)) || launch_err_ != cudaSuccess) return HYMBA_ERR_CUDA; \
+    } while (0)
+
 #define HYMBA_LAUNCH(ctx, name, kernel, grid, block, smem, ...)                                  \
     do {                                                                                         \
         ::hymba::trace_before((ctx), (name));                                                    \
@@ -96,6 +125,24 @@ __device__ __forceinline__ void griddep_launch_dependents() { asm volatile("grid
 __device__ __forceinline__ void griddep_sync() {
     griddep_wait();
     griddep_launch_dependents();
+}
+
+// Thread-block cluster primitives: this CTA's rank in its cluster, the cluster-wide
+// barrier (every thread of every CTA arrives; release / acquire order shared-memory
+// accesses across the cluster), and a load from another CTA's shared memory (DSMEM).
+__device__ __forceinline__ uint32_t cluster_rank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+__device__ __forceinline__ void cluster_arrive() { asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory"); }
+__device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory"); }
+__device__ __forceinline__ float ld_cluster_f32(const float* local, uint32_t rank) {
+    uint32_t a = static_cast<uint32_t>(__cvta_generic_to_shared(local)), r;
+    float v;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(rank));
+    asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(r) : "memory");
+    return v;
 }
 
 __device__ __forceinline__ void set_status(int* status, int code) {

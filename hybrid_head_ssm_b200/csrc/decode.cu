@@ -260,25 +260,23 @@ __device__ __forceinline__ void bk_issue_tile(unsigned char* dst, const unsigned
 // conflict-free 16-byte shared load per key, joined by three shuffles per head. P V:
 // warp w takes keys w, w + 4, ... of a tile, lane l elements 4l .. 4l + 3 of the V row.
 template <int R, int DV>
-__global__ void __launch_bounds__(128, R <= 6 ? 5 : 4)
-attn_decode_bulk_kernel(const f16* __restrict__ P, long long ldP, const f16* __restrict__ k_cache,
-                        const f16* __restrict__ v_cache, int cap, const int* __restrict__ len, int pos_offset,
-                        float* __restrict__ part, int n_split, int H, int G, int n_meta, int window, int max_chunk,
-                        int* status) {
+__device__ __forceinline__ void
+attn_decode_bulk_body(const f16* __restrict__ P, long long ldP, const f16* __restrict__ k_cache,
+                      const f16* __restrict__ v_cache, int cap, const int* __restrict__ len, int pos_offset,
+                      float* __restrict__ part, int n_split, int H, int G, int n_meta, int window, int max_chunk,
+                      int* status, int s, int g, int b, unsigned char* bk_smem) {
     griddep_sync();
     static_assert(DV == 64 || DV == 128, "V head dim");
     constexpr int BK_TV = BK_STAGE / (DV * 2);  // keys per V tile
     constexpr int EPL = DV / 32;                // V elements per lane in the PV phase
     static_assert(R >= 1 && R <= 8, "query heads per KV head");
     static_assert(4 * R * DV * 4 <= BK_NST * BK_STAGE, "the reduction buffer reuses the stages");
-    extern __shared__ __align__(128) unsigned char bk_smem[];
     __shared__ int bk_never;  // stays 0: the waits below give up on their own clock only
     unsigned char* stages = bk_smem;
     float (*ps)[8] = reinterpret_cast<float (*)[8]>(bk_smem + BK_NST * BK_STAGE);
     float* stat = reinterpret_cast<float*>(bk_smem + BK_NST * BK_STAGE + (size_t)max_chunk * 32);
     uint64_t* full = reinterpret_cast<uint64_t*>(stat + 16);
     float* red = reinterpret_cast<float*>(stages);
-    const int s = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int p = len[b] + pos_offset;
     const int ring = cap - n_meta;
@@ -439,6 +437,17 @@ attn_decode_bulk_kernel(const f16* __restrict__ P, long long ldP, const f16* __r
     }
 }
 
+template <int R, int DV>
+__global__ void __launch_bounds__(128, R <= 6 ? 5 : 4)
+attn_decode_bulk_kernel(const f16* __restrict__ P, long long ldP, const f16* __restrict__ k_cache,
+                        const f16* __restrict__ v_cache, int cap, const int* __restrict__ len, int pos_offset,
+                        float* __restrict__ part, int n_split, int H, int G, int n_meta, int window, int max_chunk,
+                        int* status) {
+    extern __shared__ __align__(128) unsigned char bk_smem[];
+    attn_decode_bulk_body<R, DV>(P, ldP, k_cache, v_cache, cap, len, pos_offset, part, n_split, H, G, n_meta, window,
+                                 max_chunk, status, blockIdx.x, blockIdx.y, blockIdx.z, bk_smem);
+}
+
 template <typename T, int DV>
 __global__ void __launch_bounds__(DV)
 attn_decode_combine_kernel(const float* __restrict__ part, int n_split, T* __restrict__ O, int H) {
@@ -491,19 +500,18 @@ __device__ __forceinline__ uint32_t wpack(bf16 lo, bf16 hi) {
 // a few wide loads per thread, all in flight together, and the loads of h go out
 // before the dot products.
 template <typename T, typename TW>
-__global__ void __launch_bounds__(SSM_WARPS * 32, 6)
-ssm_decode_kernel(const T* __restrict__ P, long long ldP, int col_x, int col_B, int col_C,
-                  int col_dtl, const TW* __restrict__ w_dt, const float* __restrict__ b_dt, int r,
-                  int wide, const float* __restrict__ conv_w, const float* __restrict__ conv_b,
-                  const float* __restrict__ A_log, const float* __restrict__ Dp,
-                  float* __restrict__ h, float* __restrict__ conv, T* __restrict__ ypre, int B,
-                  int di, int hp) {
+__device__ __forceinline__ void
+ssm_decode_body(const T* __restrict__ P, long long ldP, int col_x, int col_B, int col_C,
+                int col_dtl, const TW* __restrict__ w_dt, const float* __restrict__ b_dt, int r,
+                int wide, const float* __restrict__ conv_w, const float* __restrict__ conv_b,
+                const float* __restrict__ A_log, const float* __restrict__ Dp,
+                float* __restrict__ h, float* __restrict__ conv, T* __restrict__ ypre, int B,
+                int di, int hp, int bx, int by, unsigned char* ssm_smem) {
     griddep_sync();
     using Slot = typename WSlot<TW>::type;
     constexpr int NS = 16, KC = 4;
-    extern __shared__ __align__(16) unsigned char ssm_smem[];
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int c0 = blockIdx.x * SSM_CH, b0 = blockIdx.y * SSM_ROWS;
+    const int c0 = bx * SSM_CH, b0 = by * SSM_ROWS;
     const int c = c0 + lane;
     const bool cok = c < di;
     int bs[SSM_RPT];
@@ -707,6 +715,83 @@ ssm_decode_kernel(const T* __restrict__ P, long long ldP, int col_x, int col_B, 
 }
 
 
+template <typename T, typename TW>
+__global__ void __launch_bounds__(SSM_WARPS * 32, 6)
+ssm_decode_kernel(const T* __restrict__ P, long long ldP, int col_x, int col_B, int col_C,
+                  int col_dtl, const TW* __restrict__ w_dt, const float* __restrict__ b_dt, int r,
+                  int wide, const float* __restrict__ conv_w, const float* __restrict__ conv_b,
+                  const float* __restrict__ A_log, const float* __restrict__ Dp,
+                  float* __restrict__ h, float* __restrict__ conv, T* __restrict__ ypre, int B,
+                  int di, int hp) {
+    extern __shared__ __align__(16) unsigned char ssm_smem[];
+    ssm_decode_body<T, TW>(P, ldP, col_x, col_B, col_C, col_dtl, w_dt, b_dt, r, wide, conv_w, conv_b, A_log, Dp, h,
+                           conv, ypre, B, di, hp, blockIdx.x, blockIdx.y, ssm_smem);
+}
+
+// The decode attention and the SSM step of a layer in one launch (both read only the
+// in-projection's rows and write disjoint outputs): blocks [0, n_ssm) run the SSM step,
+// the rest the attention's (split, KV head, sequence) blocks, so the SSM's loads of the
+// state overlap the attention's stream of the cache.
+struct DecodeAttnArgs {
+    const f16* P;
+    long long ldP;
+    const f16* k_cache;
+    const f16* v_cache;
+    int cap;
+    const int* len;
+    int pos_offset;
+    float* part;
+    int n_split, H, G, n_meta, window, max_chunk;
+};
+template <typename TW>
+struct DecodeSsmArgs {
+    const f16* P;
+    long long ldP;
+    int col_x, col_B, col_C, col_dtl;
+    const TW* w_dt;
+    const float* b_dt;
+    int r, wide;
+    const float *conv_w, *conv_b, *A_log, *D;
+    float *h, *conv;
+    f16* ypre;
+    int B, di, hp, gx;
+};
+
+template <int R, int DV, typename TW>
+__global__ void __launch_bounds__(128, R <= 6 ? 5 : 4)
+decode_attn_ssm_kernel(const DecodeAttnArgs a, const DecodeSsmArgs<TW> m, int n_ssm, int* status) {
+    extern __shared__ __align__(128) unsigned char dsm[];
+    // the SSM blocks are spread evenly through the grid: block bid is the SSM block
+    // floor(bid * n_ssm / n) when that count steps at bid, else attention block
+    // bid - floor(bid * n_ssm / n)
+    const long long n = (long long)gridDim.x, bid = blockIdx.x;
+    const int k0 = (int)(bid * n_ssm / n), k1 = (int)((bid + 1) * n_ssm / n);
+    if (k1 > k0) {
+        ssm_decode_body<f16, TW>(m.P, m.ldP, m.col_x, m.col_B, m.col_C, m.col_dtl, m.w_dt, m.b_dt, m.r, m.wide,
+                                 m.conv_w, m.conv_b, m.A_log, m.D, m.h, m.conv, m.ypre, m.B, m.di, m.hp,
+                                 k0 % m.gx, k0 / m.gx, dsm);
+    } else {
+        const int q = (int)bid - k0;
+        attn_decode_bulk_body<R, DV>(a.P, a.ldP, a.k_cache, a.v_cache, a.cap, a.len, a.pos_offset, a.part, a.n_split,
+                                     a.H, a.G, a.n_meta, a.window, a.max_chunk, status, q % a.n_split,
+                                     (q / a.n_split) % a.G, q / (a.n_split * a.G), dsm);
+    }
+}
+
+template <int DV, typename TW>
+static void (*fused_kernel(int R))(const DecodeAttnArgs, const DecodeSsmArgs<TW>, int, int*) {
+    switch (R) {
+        case 1: return decode_attn_ssm_kernel<1, DV, TW>;
+        case 2: return decode_attn_ssm_kernel<2, DV, TW>;
+        case 3: return decode_attn_ssm_kernel<3, DV, TW>;
+        case 4: return decode_attn_ssm_kernel<4, DV, TW>;
+        case 5: return decode_attn_ssm_kernel<5, DV, TW>;
+        case 6: return decode_attn_ssm_kernel<6, DV, TW>;
+        case 7: return decode_attn_ssm_kernel<7, DV, TW>;
+        default: return decode_attn_ssm_kernel<8, DV, TW>;
+    }
+}
+
 template <int DV>
 static void (*bulk_kernel(int R))(const f16*, long long, const f16*, const f16*, int, const int*, int, float*, int,
                                   int, int, int, int, int, int*) {
@@ -810,6 +895,55 @@ int launch_ssm_decode(const Ctx& ctx, const T* P, long long ldP, int col_x, int 
                  di, hp);
     return HYMBA_OK;
 }
+
+template <typename TW>
+int launch_decode_attn_ssm(const Ctx& ctx, const f16* P, long long ldP, const f16* k_cache, const f16* v_cache,
+                           int cache_cap, const int* len, int pos_offset, float* part, int n_split, int B, int H,
+                           int G, int dv, int n_meta, int window, int col_x, int col_B, int col_C, int col_dtl,
+                           const TW* w_dt, const float* b_dt, int dt_rank, const float* conv_w, const float* conv_b,
+                           const float* A_log, const float* D, float* h, float* conv, f16* ypre, int di, int hp) {
+    // anything outside the shapes both halves take goes to the two separate launches, which
+    // report their own errors
+    if (B <= 0 || dt_rank <= 0 || hp < 0 || (hp > 0 && di % hp) || G <= 0 || H % G || H / G > MAX_R ||
+        (dv != 64 && dv != 128) || n_split <= 0 || (cache_cap + n_split - 1) / n_split > MAX_CHUNK)
+        return HYMBA_ERR_UNSUPPORTED;
+    constexpr int V = 8;  // 16-byte loads of fp16 rows
+    if (ldP % V || col_B % V || col_C % V || (reinterpret_cast<uintptr_t>(conv_w) & 15) ||
+        (reinterpret_cast<uintptr_t>(A_log) & 15) || (reinterpret_cast<uintptr_t>(conv) & 15) ||
+        (reinterpret_cast<uintptr_t>(h) & 15) || (reinterpret_cast<uintptr_t>(P) & 15) ||
+        ((reinterpret_cast<uintptr_t>(k_cache) | reinterpret_cast<uintptr_t>(v_cache)) & 15))
+        return HYMBA_ERR_UNSUPPORTED;
+    using Slot = typename WSlot<TW>::type;
+    const int npairs = (dt_rank + 1) / 2;
+    const int cp = npairs < SSM_PAIRS ? npairs : SSM_PAIRS;
+    const size_t smem_ssm = ((SSM_CH * (size_t)(cp | 1) * sizeof(Slot) + 15) & ~size_t(15)) +
+                            (size_t)SSM_ROWS * cp * sizeof(float2);
+    const int wide = hp == 0 && sizeof(TW) == 2 && dt_rank % 2 == 0 && npairs <= SSM_PAIRS && di % SSM_CH == 0 &&
+                     (reinterpret_cast<uintptr_t>(w_dt) & 15) == 0 && col_dtl % 2 == 0 &&
+                     SSM_CH * npairs / 4 <= SSM_WLD * SSM_WARPS * 32 && SSM_ROWS * npairs <= SSM_XLD * SSM_WARPS * 32;
+    const int max_chunk = (cache_cap + n_split - 1) / n_split;
+    const size_t smem_attn = (size_t)BK_NST * BK_STAGE + (size_t)max_chunk * 32 + 16 * sizeof(float) +
+                             BK_NST * sizeof(uint64_t);
+    const size_t smem = smem_attn > smem_ssm ? smem_attn : smem_ssm;
+    DecodeAttnArgs a{P, ldP, k_cache, v_cache, cache_cap, len, pos_offset, part, n_split, H, G, n_meta, window,
+                     max_chunk};
+    DecodeSsmArgs<TW> m{P, ldP, col_x, col_B, col_C, col_dtl, w_dt, b_dt, dt_rank, wide, conv_w, conv_b, A_log, D,
+                        h, conv, ypre, B, di, hp, ceil_div(di, SSM_CH)};
+    const int n_ssm = m.gx * ceil_div(B, SSM_ROWS);
+    const int n_attn = n_split * G * B;
+    auto kern = dv == 128 ? fused_kernel<128, TW>(H / G) : fused_kernel<64, TW>(H / G);
+    if (smem > 48 * 1024) {
+        static std::atomic<unsigned long long> smem_set{0};
+        if (!smem_opt_in_once(smem_set, kern, smem, ctx)) return HYMBA_ERR_CUDA;
+    }
+    HYMBA_LAUNCH(ctx, "attn_ssm_decode", kern, n_ssm + n_attn, 128, smem, a, m, n_ssm, ctx.status);
+    return HYMBA_OK;
+}
+
+template int launch_decode_attn_ssm<bf16>(const Ctx&, const f16*, long long, const f16*, const f16*, int, const int*,
+                                          int, float*, int, int, int, int, int, int, int, int, int, int, int,
+                                          const bf16*, const float*, int, const float*, const float*, const float*,
+                                          const float*, float*, float*, f16*, int, int);
 
 template int launch_attn_decode<float>(const Ctx&, const float*, long long, const float*,
                                        const float*, int, const int*, int, float*, int, float*,

@@ -5,24 +5,18 @@
 // output projection; normalise-scale-average is the reading used for how they are
 // combined). HBM-bound: per (row, channel) it reads O, y_pre and z and writes U once.
 //
-// One row per 256-thread block; each thread keeps its (at most two) 8-element pieces
-// of the row in registers between the two passes (sums of squares, then the output),
-// moving 8 elements per 16-byte access. Few registers per thread keep many rows in
-// flight per SM, which is what an HBM-bound row kernel needs.
-//
-// Decode variant (SPLIT): the attention output arrives as the split-KV partials of the
-// decode attention (per head and key split: unnormalised sum of p v, the split's
-// max logit and sum of p) and is merged here, piece by piece, with the usual
-// rescaling by exp2(m_s - max_s m_s).
+// Two kernels: the prefill one (persistent over rows, loads of the next rows in flight
+// through each row's reductions) and the decode one (one thread-block cluster per row,
+// merging the split partials of the decode attention); both keep a thread's pieces of a
+// row in registers between the two passes (sums of squares, then the output) and move 8
+// elements per 16-byte access.
 #include "kernels.h"
 
 namespace hymba {
 
 namespace {
 
-constexpr int TPR = 256;                // threads per row
-constexpr int RPB = 1;                  // rows per block
-constexpr int VMAX = 2;                 // 8-element vectors per thread and array (d_inner <= 4096)
+constexpr int kMaxWidth = 4096;         // widest branch (channels) either kernel takes
 
 template <typename I>
 __device__ __forceinline__ void load8(const I* p, float* v) {
@@ -61,128 +55,125 @@ __device__ __forceinline__ void load8f(const float* p, float* v) {
     v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
 }
 
-// Merge weights of a row's split partials (layout [row, head, split, dv + 4]: dv sums,
-// then the split's max logit and sum of weights): w[head][s] = exp2(m_s - M) / den with
-// M = max_s m_s and den = sum_s exp2(m_s - M) l_s, formed once per (row, head) by the
-// block into shared memory (zero for a head that saw no key).
-__device__ __forceinline__ void merge_weights(const float* __restrict__ part, int n_split, int H, int dv,
-                                              long long row, float* wts, int t, int nthreads) {
-    // one warp per head, one lane per split (in rounds of 32 splits)
-    const int warp = t >> 5, lane = t & 31, nwarps = nthreads >> 5;
-    for (int hd = warp; hd < H; hd += nwarps) {
-        const float* base = part + ((long long)row * H + hd) * n_split * (dv + 4) + dv;
-        float M = -INFINITY;
-        for (int s = lane; s < n_split; s += 32) M = fmaxf(M, base[s * (dv + 4)]);
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-        float den = 0.f;
-        for (int s = lane; s < n_split; s += 32) {
-            const float w = M != -INFINITY ? exp2f(base[s * (dv + 4)] - M) : 0.f;
-            wts[hd * n_split + s] = w;
-            den = fmaf(w, base[s * (dv + 4) + 1], den);
-        }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
-        const float inv = den > 0.f ? 1.f / den : 0.f;
-        for (int s = lane; s < n_split; s += 32) wts[hd * n_split + s] *= inv;
-    }
-}
+// Decode fusion: one thread-block cluster of FC CTAs per sequence row. CTA r of the
+// cluster takes pieces [r * po, (r + 1) * po) of the attention branch (po = ceil(pieces /
+// FC)) and likewise of the Mamba branch, one 8-channel piece per thread and branch. The
+// attention pieces arrive as the split partials of the decode attention, layout [row,
+// head, split, dv + 4] (dv sums of p v, then the split's max logit m_s and sum of p l_s),
+// merged with the weights w_s = exp2(m_s - M) / sum_s exp2(m_s - M) l_s, M = max_s m_s.
+// Every load of a thread (its first FSPL split records, y_pre and z, its heads' (m_s, l_s))
+// is issued before the first barrier. The two sums of squares of the row meet across the
+// cluster through distributed shared memory: each CTA publishes its partial sums, and
+// after a cluster barrier reads the other CTAs' from their shared memory.
+constexpr int FC = 8;    // CTAs per row (cluster size)
+constexpr int FT = 64;   // threads per CTA
+constexpr int FSPL = 8;  // split records per piece loaded ahead of the merge weights
+static_assert(FC * FT * 8 >= kMaxWidth, "one piece per thread and branch");
 
-// Attention output piece c..c+7 of row `row`: the weighted sum of its head's split
-// partials (the loads of four splits in flight at a time).
-__device__ __forceinline__ void merge8(const float* __restrict__ part, int n_split, int H, int dv,
-                                       long long row, int c, const float* wts, float* o) {
-    const int hd = c / dv, e = c - hd * dv;
-    const float* base = part + ((long long)row * H + hd) * n_split * (dv + 4) + e;
-    const float* w = wts + hd * n_split;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) o[i] = 0.f;
-    int s = 0;
-    for (; s + 4 <= n_split; s += 4) {
-        float4 v[4][2];
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            // records of dv + 4 floats start on 16-byte boundaries
-            const float4* ps = reinterpret_cast<const float4*>(base + (s + u) * (dv + 4));
-            v[u][0] = ps[0];
-            v[u][1] = ps[1];
-        }
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            const float wu = w[s + u];
-            o[0] = fmaf(wu, v[u][0].x, o[0]); o[1] = fmaf(wu, v[u][0].y, o[1]);
-            o[2] = fmaf(wu, v[u][0].z, o[2]); o[3] = fmaf(wu, v[u][0].w, o[3]);
-            o[4] = fmaf(wu, v[u][1].x, o[4]); o[5] = fmaf(wu, v[u][1].y, o[5]);
-            o[6] = fmaf(wu, v[u][1].z, o[6]); o[7] = fmaf(wu, v[u][1].w, o[7]);
-        }
-    }
-    for (; s < n_split; ++s) {
-        const float* ps = base + s * (dv + 4);
-        const float wu = w[s];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) o[i] = fmaf(wu, ps[i], o[i]);
-    }
-}
-
-// (the decode variant runs one block per sequence, so it asks for no more than one
-// block per SM and keeps its merge temporaries in registers)
-// CONCAT: U = [beta2 * RMS(Y) | beta1 * RMS(O)] (d_inner + H * dv wide) instead of the
-// average (O and Y of equal width d_inner).
-template <typename I, typename T, bool SPLIT, bool CONCAT>
-__global__ void __launch_bounds__(TPR * RPB, SPLIT ? 1 : 4)
-fuse_kernel(const I* __restrict__ O, const float* __restrict__ part, int n_split, int H, int dv,
-            const I* __restrict__ ypre, const I* __restrict__ P, long long ldP, int col_z,
-            const float* __restrict__ g_attn, const float* __restrict__ g_ssm, const float* __restrict__ beta1,
-            const float* __restrict__ beta2, const float* __restrict__ v_scale, const float* __restrict__ v_bias,
-            int rep, T* __restrict__ U, int rows, int di, float eps, int* len_inc, float* __restrict__ y_init,
-            const float* __restrict__ y_res, int d_model) {
+template <typename I, typename T, bool CONCAT>
+__global__ void __launch_bounds__(FT)
+fuse_split_kernel(const float* __restrict__ part, int n_split, int H, int dv, const I* __restrict__ ypre,
+                  const I* __restrict__ P, long long ldP, int col_z, const float* __restrict__ g_attn,
+                  const float* __restrict__ g_ssm, const float* __restrict__ beta1, const float* __restrict__ beta2,
+                  const float* __restrict__ v_scale, const float* __restrict__ v_bias, int rep, T* __restrict__ U,
+                  int di, float eps, int* len_inc, float* __restrict__ y_init, const float* __restrict__ y_res,
+                  int d_model) {
     griddep_sync();
-    __shared__ float red[RPB][TPR / 32][2];
-    extern __shared__ float merge_wts[];  // SPLIT: [H, n_split] merge weights of the row
-    const int sub = threadIdx.x / TPR, t = threadIdx.x % TPR;
-    const long long row = (long long)blockIdx.x * RPB + sub;
-    const bool live = row < rows;
-    if constexpr (SPLIT) {
-        if (live) merge_weights(part, n_split, H, dv, row, merge_wts, t, TPR);
-        __syncthreads();
-    }
-    const int hv = H * dv;                 // attention branch width
-    const int nvo = hv / 8, nvy = di / 8;  // pieces of 8 per branch
-    float o[VMAX][8], y[VMAX][8];
-    float ss_o = 0.f, ss_y = 0.f;
+    extern __shared__ float fsm[];  // [nh * n_split] m_s, [nh * n_split] l_s, [nh] M, [nh] 1 / den
+    __shared__ float wsum[FT / 32][2];
+    __shared__ float csum[2];  // this CTA's partial sums of squares, read by the whole cluster
+    __shared__ float tot[2];
+    const int cr = (int)cluster_rank();
+    const long long row = blockIdx.x / FC;
+    const int t = threadIdx.x;
+    const int hv = H * dv, nvo = hv / 8, nvy = di / 8;
+    const int po = (nvo + FC - 1) / FC, py = (nvy + FC - 1) / FC;
+    const int a_lo = min(cr * po, nvo), a_hi = min(a_lo + po, nvo);
+    const int vo = a_lo + t, vy = cr * py + t;
+    const bool has_o = vo < a_hi, has_y = t < py && vy < nvy;
+    // heads of this CTA's attention pieces (pieces never straddle a head)
+    const int h_lo = a_lo * 8 / dv, nh = a_hi > a_lo ? (a_hi * 8 - 1) / dv + 1 - h_lo : 0;
+    float* fm = fsm;
+    float* fl = fsm + nh * n_split;
+    float* hM = fl + nh * n_split;
+    float* hinv = hM + nh;
+    const float* rbase = part + (long long)row * H * n_split * (dv + 4);
+    // issue every load: split records of this piece, y_pre and z, the heads' statistics
+    const int hd = has_o ? vo * 8 / dv : 0, e = has_o ? vo * 8 - hd * dv : 0;
+    const float* pp = rbase + (long long)hd * n_split * (dv + 4) + e;
+    const int npre = min(n_split, FSPL);
+    float4 pv[FSPL][2];
 #pragma unroll
-    for (int k = 0; k < VMAX; ++k) {
-        const int vi = t + k * TPR;
-        if (live && vi < nvo) {
-            const int c = vi * 8;
-            if constexpr (SPLIT)
-                merge8(part, n_split, H, dv, row, c, merge_wts, o[k]);
-            else
-                load8<I>(O + row * hv + c, o[k]);
-            if (v_scale) {
-                // a consumer's adapted shared V: attention over V * s + b is the attention
-                // output * s + b (the softmax weights sum to 1)
-                const int hd = c / dv;
-                const int idx = (hd / rep) * dv + (c - hd * dv);
-                float vs[8], vb[8];
-                load8f(v_scale + idx, vs);
-                load8f(v_bias + idx, vb);
-#pragma unroll
-                for (int i = 0; i < 8; ++i) o[k][i] = fmaf(o[k][i], vs[i], vb[i]);
-            }
-#pragma unroll
-            for (int i = 0; i < 8; ++i) ss_o = fmaf(o[k][i], o[k][i], ss_o);
+    for (int sp = 0; sp < FSPL; ++sp)
+        if (has_o && sp < npre) {
+            const float4* q = reinterpret_cast<const float4*>(pp + (long long)sp * (dv + 4));
+            pv[sp][0] = q[0];
+            pv[sp][1] = q[1];
         }
-        if (live && vi < nvy) {
-            const int c = vi * 8;
-            float z[8];
-            load8<I>(ypre + row * di + c, y[k]);
-            load8<I>(P + row * ldP + col_z + c, z);
+    float y[8], z[8];
+    if (has_y) {
+        load8<I>(ypre + row * di + vy * 8, y);
+        load8<I>(P + row * ldP + col_z + vy * 8, z);
+    }
+    for (int i = t; i < nh * n_split; i += FT) {
+        const int hh = i / n_split, sp = i - hh * n_split;
+        const float2 ml = *reinterpret_cast<const float2*>(rbase + ((long long)(h_lo + hh) * n_split + sp) * (dv + 4) + dv);
+        fm[i] = ml.x;
+        fl[i] = ml.y;
+    }
+    __syncthreads();
+    for (int hh = t; hh < nh; hh += FT) {
+        float M = -INFINITY;
+        for (int sp = 0; sp < n_split; ++sp) M = fmaxf(M, fm[hh * n_split + sp]);
+        float den = 0.f;
+        if (M != -INFINITY)
+            for (int sp = 0; sp < n_split; ++sp) den = fmaf(exp2f(fm[hh * n_split + sp] - M), fl[hh * n_split + sp], den);
+        hM[hh] = M;
+        hinv[hh] = den > 0.f ? 1.f / den : 0.f;
+    }
+    __syncthreads();
+    float o[8];
+    float ss_o = 0.f, ss_y = 0.f;
+    if (has_o) {
+        const int hh = hd - h_lo;
+        const float M = hM[hh], inv = hinv[hh];
+        const float* mrow = fm + hh * n_split;
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                y[k][i] *= z[i] / (1.0f + __expf(-z[i]));
-                ss_y = fmaf(y[k][i], y[k][i], ss_y);
+        for (int i = 0; i < 8; ++i) o[i] = 0.f;
+#pragma unroll
+        for (int sp = 0; sp < FSPL; ++sp)
+            if (sp < npre) {
+                const float w = M != -INFINITY ? exp2f(mrow[sp] - M) * inv : 0.f;
+                o[0] = fmaf(w, pv[sp][0].x, o[0]); o[1] = fmaf(w, pv[sp][0].y, o[1]);
+                o[2] = fmaf(w, pv[sp][0].z, o[2]); o[3] = fmaf(w, pv[sp][0].w, o[3]);
+                o[4] = fmaf(w, pv[sp][1].x, o[4]); o[5] = fmaf(w, pv[sp][1].y, o[5]);
+                o[6] = fmaf(w, pv[sp][1].z, o[6]); o[7] = fmaf(w, pv[sp][1].w, o[7]);
             }
+        for (int sp = npre; sp < n_split; ++sp) {
+            const float4* q = reinterpret_cast<const float4*>(pp + (long long)sp * (dv + 4));
+            const float4 a = q[0], b = q[1];
+            const float w = M != -INFINITY ? exp2f(mrow[sp] - M) * inv : 0.f;
+            o[0] = fmaf(w, a.x, o[0]); o[1] = fmaf(w, a.y, o[1]); o[2] = fmaf(w, a.z, o[2]); o[3] = fmaf(w, a.w, o[3]);
+            o[4] = fmaf(w, b.x, o[4]); o[5] = fmaf(w, b.y, o[5]); o[6] = fmaf(w, b.z, o[6]); o[7] = fmaf(w, b.w, o[7]);
+        }
+        if (v_scale) {
+            // a consumer's adapted shared V: attention over V * s + b is the attention
+            // output * s + b (the softmax weights sum to 1)
+            const int idx = (hd / rep) * dv + e;
+            float vs[8], vb[8];
+            load8f(v_scale + idx, vs);
+            load8f(v_bias + idx, vb);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) o[i] = fmaf(o[i], vs[i], vb[i]);
+        }
+#pragma unroll
+        for (int i = 0; i < 8; ++i) ss_o = fmaf(o[i], o[i], ss_o);
+    }
+    if (has_y) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            y[i] *= z[i] / (1.0f + __expf(-z[i]));
+            ss_y = fmaf(y[i], y[i], ss_y);
         }
     }
 #pragma unroll
@@ -191,64 +182,70 @@ fuse_kernel(const I* __restrict__ O, const float* __restrict__ part, int n_split
         ss_y += __shfl_xor_sync(0xffffffffu, ss_y, off);
     }
     if ((t & 31) == 0) {
-        red[sub][t >> 5][0] = ss_o;
-        red[sub][t >> 5][1] = ss_y;
+        wsum[t >> 5][0] = ss_o;
+        wsum[t >> 5][1] = ss_y;
     }
     __syncthreads();
-    ss_o = 0.f;
-    ss_y = 0.f;
+    if (t < 2) {
+        float v = 0.f;
 #pragma unroll
-    for (int w = 0; w < TPR / 32; ++w) {
-        ss_o += red[sub][w][0];
-        ss_y += red[sub][w][1];
+        for (int w = 0; w < FT / 32; ++w) v += wsum[w][t];
+        csum[t] = v;
     }
+    cluster_arrive();
+    cluster_wait();
+    if (t < 2) {
+        float v = 0.f;
+#pragma unroll
+        for (int r = 0; r < FC; ++r) v += ld_cluster_f32(&csum[t], (uint32_t)r);
+        tot[t] = v;
+    }
+    __syncthreads();
+    // the other CTAs may leave once every CTA has read their sums
+    cluster_arrive();
     // the average halves both branches; the concatenation keeps them whole
     const float half = CONCAT ? 1.0f : 0.5f;
-    const float ro = half / sqrtf(ss_o / hv + eps);
-    const float ry = half / sqrtf(ss_y / di + eps);
+    const float ro = half / sqrtf(tot[0] / hv + eps);
+    const float ry = half / sqrtf(tot[1] / di + eps);
+    if constexpr (CONCAT) {
+        const long long ldu = di + hv;
+        if (has_y) {
+            const int c = vy * 8;
+            float gs[8], b2[8], u[8];
+            load8f(g_ssm + c, gs);
+            load8f(beta2 + c, b2);
 #pragma unroll
-    for (int k = 0; k < VMAX; ++k) {
-        const int vi = t + k * TPR;
-        if constexpr (CONCAT) {
-            const long long ldu = di + hv;
-            if (live && vi < nvy) {
-                const int c = vi * 8;
-                float gs[8], b2[8], u[8];
-                load8f(g_ssm + c, gs);
-                load8f(beta2 + c, b2);
-#pragma unroll
-                for (int i = 0; i < 8; ++i) u[i] = b2[i] * gs[i] * y[k][i] * ry;
-                store8<T>(U + row * ldu + c, u);
-            }
-            if (live && vi < nvo) {
-                const int c = vi * 8;
-                float ga[8], b1[8], u[8];
-                load8f(g_attn + c, ga);
-                load8f(beta1 + c, b1);
-#pragma unroll
-                for (int i = 0; i < 8; ++i) u[i] = b1[i] * ga[i] * o[k][i] * ro;
-                store8<T>(U + row * ldu + di + c, u);
-            }
-        } else {
-            if (live && vi < nvy) {
-                const int c = vi * 8;
-                float ga[8], gs[8], b1[8], b2[8], u[8];
-                load8f(g_attn + c, ga);
-                load8f(g_ssm + c, gs);
-                load8f(beta1 + c, b1);
-                load8f(beta2 + c, b2);
-#pragma unroll
-                for (int i = 0; i < 8; ++i) u[i] = b1[i] * ga[i] * o[k][i] * ro + b2[i] * gs[i] * y[k][i] * ry;
-                store8<T>(U + row * di + c, u);
-            }
+            for (int i = 0; i < 8; ++i) u[i] = b2[i] * gs[i] * y[i] * ry;
+            store8<T>(U + row * ldu + c, u);
         }
+        if (has_o) {
+            const int c = vo * 8;
+            float ga[8], b1[8], u[8];
+            load8f(g_attn + c, ga);
+            load8f(beta1 + c, b1);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) u[i] = b1[i] * ga[i] * o[i] * ro;
+            store8<T>(U + row * ldu + di + c, u);
+        }
+    } else if (has_o && has_y) {
+        // equal widths: a thread holds the same channels of both branches
+        const int c = vy * 8;
+        float ga[8], gs[8], b1[8], b2[8], u[8];
+        load8f(g_attn + c, ga);
+        load8f(g_ssm + c, gs);
+        load8f(beta1 + c, b1);
+        load8f(beta2 + c, b2);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) u[i] = b1[i] * ga[i] * o[i] * ro + b2[i] * gs[i] * y[i] * ry;
+        store8<T>(U + row * di + c, u);
     }
-    if (len_inc && live && t == 0) len_inc[row] += 1;
+    if (len_inc && cr == 0 && t == 0) len_inc[row] += 1;
     // the output projection that follows adds its split-K partial sums to y: y starts as
     // the residual (or zero), unless y is the residual itself
-    if (y_init && live && y_init != y_res)
-        for (int c = t; c < d_model; c += TPR)
+    if (y_init && y_init != y_res)
+        for (int c = cr * FT + t; c < d_model; c += FC * FT)
             y_init[row * d_model + c] = y_res ? y_res[row * d_model + c] : 0.f;
+    cluster_wait();
 }
 
 constexpr int RT = 512;                 // prefill fusion: threads per row (one 8-channel piece each)
@@ -432,13 +429,16 @@ static int fuse_variant(const Ctx& ctx, const I* O, const float* part, int n_spl
                         const float* beta1, const float* beta2, const float* v_scale, const float* v_bias, T* U,
                         int rows, int di, float eps, int* len_inc, float* y_init, const float* y_res, int d_model) {
     if (part) {
-        auto kern = fuse_kernel<I, T, true, CONCAT>;
-        const size_t smem = (size_t)H * n_split * sizeof(float);
+        auto kern = fuse_split_kernel<I, T, CONCAT>;
+        // heads spanned by one CTA's attention pieces: at most ceil(po * 8 / dv) + 1
+        const int po = ceil_div(H * dv / 8, FC);
+        const int nh = std::min(H, ceil_div(po * 8, dv) + 1);
+        const size_t smem = (2 * (size_t)nh * n_split + 2 * (size_t)nh) * sizeof(float);
         static std::atomic<unsigned long long> smem_set{0};
         if (smem > 48 * 1024 && !smem_opt_in_once(smem_set, kern, smem, ctx)) return HYMBA_ERR_CUDA;
-        HYMBA_LAUNCH(ctx, "fuse", kern, ceil_div(rows, RPB), TPR * RPB, smem, O, part, n_split, H, dv, ypre, P, ldP,
-                     col_z, g_attn, g_ssm, beta1, beta2, v_scale, v_bias, H / G, U, rows, di, eps, len_inc, y_init,
-                     y_res, d_model);
+        HYMBA_LAUNCH_CLUSTER(ctx, "fuse", kern, (long long)rows * FC, FT, smem, FC, part, n_split, H, dv, ypre, P,
+                             ldP, col_z, g_attn, g_ssm, beta1, beta2, v_scale, v_bias, H / G, U, di, eps, len_inc,
+                             y_init, y_res, d_model);
     } else {
         auto kern = fuse_rows_kernel<I, T, CONCAT>;
         const size_t smem = (size_t)RSLOT * 3 * RT * sizeof(I) * 8;
@@ -459,14 +459,15 @@ int launch_fuse(const Ctx& ctx, const I* O, const float* part, int n_split, int 
     if (rows <= 0) return HYMBA_OK;
     if (y_init && (!part || d_model <= 0)) return HYMBA_ERR_UNSUPPORTED;
     const int hv = H * dv;
-    if (di % 8 || di > VMAX * 8 * TPR || hv > VMAX * 8 * TPR || col_z % 8 || ldP % 8) return HYMBA_ERR_UNSUPPORTED;
+    if (di % 8 || di > kMaxWidth || hv > kMaxWidth || col_z % 8 || ldP % 8) return HYMBA_ERR_UNSUPPORTED;
     // pieces of 8 never straddle a head
     if (H <= 0 || G <= 0 || H % G || dv % 8 || (!concat && hv != di)) return HYMBA_ERR_UNSUPPORTED;
     if ((v_scale == nullptr) != (v_bias == nullptr) ||
         ((reinterpret_cast<uintptr_t>(v_scale) | reinterpret_cast<uintptr_t>(v_bias)) & 15))
         return HYMBA_ERR_UNSUPPORTED;
-    // 8-byte loads of the partial sums
-    if (part && (n_split <= 0 || (reinterpret_cast<uintptr_t>(part) & 7))) return HYMBA_ERR_UNSUPPORTED;
+    // 16-byte loads of the partial sums; one cluster per row along x
+    if (part && (n_split <= 0 || (reinterpret_cast<uintptr_t>(part) & 15) || (long long)rows * FC > INT32_MAX))
+        return HYMBA_ERR_UNSUPPORTED;
     if (concat)
         return fuse_variant<I, T, true>(ctx, O, part, n_split, H, dv, G, ypre, P, ldP, col_z, g_attn, g_ssm, beta1,
                                         beta2, v_scale, v_bias, U, rows, di, eps, len_inc, y_init, y_res, d_model);

@@ -511,15 +511,26 @@ static int decode_impl(const Ctx& ctx, const hymba_layer_cfg* c, const hymba_lay
     if (rc) return rc;
     ep.rope = rope;
     if ((rc = gemm<T, I>(ctx, "gemm_in_proj_decode", x, d, static_cast<const T*>(w->w_in), d, B, k.n_in, d, ep))) return rc;
-    // split-KV attention, left as partials that the fusion kernel merges
-    if ((rc = launch_attn_decode<I>(ctx, P, pl.ldP, k_cache, v_cache, kv->cache_cap, kv->len, pos_offset,
-                                    part, pl.n_split, nullptr, B, H, G, dv, m, c->window)))
-        return rc;
-    // SSM step with the Delta projection of the new rows folded in
-    if ((rc = launch_ssm_decode<I, T>(ctx, P, pl.ldP, k.x, k.Bc, k.Cc, k.dtl, static_cast<const T*>(w->w_dt),
-                                      w->b_dt, c->dt_rank, w->conv_w, w->conv_b, w->A_log, w->D, st->h,
-                                      st->conv, ypre, B, di, ssm_hp(c))))
-        return rc;
+    // split-KV attention, left as partials that the fusion kernel merges, and the SSM step
+    // with the Delta projection of the new rows folded in: one launch for 16-bit layers
+    bool both = false;
+    if constexpr (std::is_same<I, f16>::value && std::is_same<T, bf16>::value) {
+        rc = launch_decode_attn_ssm<bf16>(ctx, P, pl.ldP, k_cache, v_cache, kv->cache_cap, kv->len, pos_offset, part,
+                                          pl.n_split, B, H, G, dv, m, c->window, k.x, k.Bc, k.Cc, k.dtl,
+                                          static_cast<const bf16*>(w->w_dt), w->b_dt, c->dt_rank, w->conv_w,
+                                          w->conv_b, w->A_log, w->D, st->h, st->conv, ypre, di, ssm_hp(c));
+        if (rc != HYMBA_OK && rc != HYMBA_ERR_UNSUPPORTED) return rc;
+        both = rc == HYMBA_OK;
+    }
+    if (!both) {
+        if ((rc = launch_attn_decode<I>(ctx, P, pl.ldP, k_cache, v_cache, kv->cache_cap, kv->len, pos_offset,
+                                        part, pl.n_split, nullptr, B, H, G, dv, m, c->window)))
+            return rc;
+        if ((rc = launch_ssm_decode<I, T>(ctx, P, pl.ldP, k.x, k.Bc, k.Cc, k.dtl, static_cast<const T*>(w->w_dt),
+                                          w->b_dt, c->dt_rank, w->conv_w, w->conv_b, w->A_log, w->D, st->h,
+                                          st->conv, ypre, B, di, ssm_hp(c))))
+            return rc;
+    }
     const bool concat = c->fusion == HYMBA_FUSION_CONCAT;
     EpiArgs<TIO> eo = epi_base<TIO>(EPI_OUT, B, d);
     eo.y = y;

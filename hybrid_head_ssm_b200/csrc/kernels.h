@@ -115,6 +115,15 @@ int launch_attn_decode(const Ctx& ctx, const T* P, long long ldP, const T* k_cac
 // One SSM decode step per (sequence, channel): Delta = softplus(dt_low W_dt^T + b_dt)
 // from the projection row's dt_low columns, conv-state shift, conv, SiLU, scan step on
 // h in place, y_pre = C.h + D xc. W_dt is [di, dt_rank] in the layer's weight type.
+// The decode attention (split partials) and the SSM step of a layer in one launch
+// (16-bit layers): the same arguments as the two launches above.
+template <typename TW>
+int launch_decode_attn_ssm(const Ctx& ctx, const f16* P, long long ldP, const f16* k_cache, const f16* v_cache,
+                           int cache_cap, const int* len, int pos_offset, float* part, int n_split, int B, int H,
+                           int G, int dv, int n_meta, int window, int col_x, int col_B, int col_C, int col_dtl,
+                           const TW* w_dt, const float* b_dt, int dt_rank, const float* conv_w, const float* conv_b,
+                           const float* A_log, const float* D, float* h, float* conv, f16* ypre, int di, int hp);
+
 template <typename T, typename TW>
 int launch_ssm_decode(const Ctx& ctx, const T* P, long long ldP, int col_x, int col_B, int col_C,
                       int col_dtl, const TW* w_dt, const float* b_dt, int dt_rank,
