@@ -6,8 +6,11 @@
 //
 // Cache layout: k_cache [B, G, cap, dh], v_cache [B, G, cap, dv]; position p < n_meta
 // in slot p, position p >= n_meta in slot n_meta + (p - n_meta) mod (cap - n_meta).
+#include <algorithm>
+
 #include "kernels.h"
 #include "tc.cuh"
+#include "warp_mma.cuh"
 
 namespace hymba {
 
@@ -220,64 +223,54 @@ attn_decode_kernel(const T* __restrict__ P, long long ldP, const T* __restrict__
 }
 
 // ---------------------------------------------------------------------------
-// 16-bit K/V: the split's K and V rows staged in shared memory by bulk async copies
+// 16-bit K/V: the split's K and V rows in shared memory, scores and P V on the tensor
+// cores (warp-level m16n8k16 MMAs, fp16 operands, fp32 accumulators)
 // ---------------------------------------------------------------------------
-constexpr int BK_NST = 2;                      // stages
-constexpr int BK_STAGE = 16384;                // bytes per stage
-constexpr int BK_TK = BK_STAGE / (DH * 2);     // keys per K tile (128)
-
-// Queue the bulk copies of one tile: the block-local keys [a, e) of the split, rows of
-// row_bytes, into dst in key order. The keys map to cache slots in at most three
-// contiguous runs (meta slots, then the ring up to its end, then from its start), one
-// copy per run; the tile's byte count is announced on `bar` first.
-__device__ __forceinline__ void bk_issue_tile(unsigned char* dst, const unsigned char* src, int row_bytes, int a,
-                                              int e, int k0, int meta_n, int lo, int n_meta, int cap, int ring,
-                                              uint64_t* bar) {
-    tc::mbar_arrive_expect_tx(bar, (uint32_t)((e - a) * row_bytes));
-    const int t0 = a;
-    while (a < e) {
-        const int idx = k0 + a;
-        int slot, run;
-        if (idx < meta_n) {
-            slot = idx;
-            run = min(e - a, meta_n - idx);
-        } else {
-            const int j = lo + (idx - meta_n);
-            slot = n_meta + (j - n_meta) % ring;
-            run = min(e - a, cap - slot);
-        }
-        tc::bulk_load(dst + (size_t)(a - t0) * row_bytes, src + (size_t)slot * row_bytes, (uint32_t)(run * row_bytes),
-                      bar);
-        a += run;
-    }
+// Shared memory of one block for splits of up to max_chunk keys: K [NKP][64] and
+// V [NKP][DV] fp16 rows (16-byte chunks XOR-swizzled by the row's low three bits, so
+// that the eight rows an ldmatrix reads fall in eight different bank groups), P as two
+// fp16 parts [2][8 heads][NKP + 8], the slot of every key, and the per-warp partial
+// maxima and sums. NKP = max_chunk rounded up to 64.
+__host__ __device__ constexpr int mma_nkp(int max_chunk) { return (max_chunk + 63) / 64 * 64; }
+__host__ __device__ constexpr size_t mma_smem_bytes(int max_chunk, int dv) {
+    return (size_t)mma_nkp(max_chunk) * (DH + dv) * 2 + 2 * 8 * ((size_t)mma_nkp(max_chunk) + 8) * 2 +
+           (size_t)mma_nkp(max_chunk) * 4 + 2 * 4 * 8 * 4;
 }
 
-// One block per (key split, KV head, sequence) serves the R query heads of the KV head,
-// as attn_decode_kernel, with the split's K rows (128-key tiles) and then V rows
-// (64-key tiles) streamed through a two-stage shared-memory ring by bulk async copies:
-// the copies keep enough bytes in flight without holding them in registers. Scores:
-// eight lanes per key, each with its 8 dimensions of the R queries in registers, one
-// conflict-free 16-byte shared load per key, joined by three shuffles per head. P V:
-// warp w takes keys w, w + 4, ... of a tile, lane l elements 4l .. 4l + 3 of the V row.
+// One block (four warps) per (key split, KV head, sequence) serves the R <= 8 query
+// heads of the KV head. Every K and V row of the split is requested up front by 16-byte
+// asynchronous copies (K, then V, as two commit groups), so the block's whole share of
+// the cache is in flight while it waits. Scores S^T = K q^T: the 16-key tiles of K are
+// the MMA's A operand (ldmatrix), the R queries (padded to 8) its B operand, held in
+// registers for the block's life; warp w takes key tiles w, w + 4, ... The split's
+// max per head meets across the warps in shared memory. p = exp2(s - max) enters P V as
+// two fp16 parts, p = p_hi + p_lo (p_hi = p rounded to fp16, p_lo the rounded remainder),
+// two MMAs against the same V fragment, so the weights keep about 22 bits (a single
+// fp16 rounding of p costs up to 2^-11 of every weight). P V: O^T = V^T P^T, V^T 16-row
+// tiles by transposing ldmatrix, P^T from shared memory; warp w takes the V columns
+// [w DV / 4, (w + 1) DV / 4) over all keys, so no reduction across warps.
 template <int R, int DV>
 __device__ __forceinline__ void
-attn_decode_bulk_body(const f16* __restrict__ P, long long ldP, const f16* __restrict__ k_cache,
-                      const f16* __restrict__ v_cache, int cap, const int* __restrict__ len, int pos_offset,
-                      float* __restrict__ part, int n_split, int H, int G, int n_meta, int window, int max_chunk,
-                      int* status, int s, int g, int b, unsigned char* bk_smem) {
+attn_decode_mma_body(const f16* __restrict__ P, long long ldP, const f16* __restrict__ k_cache,
+                     const f16* __restrict__ v_cache, int cap, const int* __restrict__ len, int pos_offset,
+                     float* __restrict__ part, int n_split, int H, int G, int n_meta, int window, int max_chunk,
+                     int* status, int s, int g, int b, unsigned char* smem) {
     griddep_sync();
     static_assert(DV == 64 || DV == 128, "V head dim");
-    constexpr int BK_TV = BK_STAGE / (DV * 2);  // keys per V tile
-    constexpr int EPL = DV / 32;                // V elements per lane in the PV phase
     static_assert(R >= 1 && R <= 8, "query heads per KV head");
-    static_assert(4 * R * DV * 4 <= BK_NST * BK_STAGE, "the reduction buffer reuses the stages");
-    __shared__ int bk_never;  // stays 0: the waits below give up on their own clock only
-    unsigned char* stages = bk_smem;
-    float (*ps)[8] = reinterpret_cast<float (*)[8]>(bk_smem + BK_NST * BK_STAGE);
-    float* stat = reinterpret_cast<float*>(bk_smem + BK_NST * BK_STAGE + (size_t)max_chunk * 32);
-    uint64_t* full = reinterpret_cast<uint64_t*>(stat + 16);
-    float* red = reinterpret_cast<float*>(stages);
+    constexpr int VCH = DV / 8;         // 16-byte chunks per V row
+    constexpr int MTW = DV / 64;        // 16-column V^T tiles per warp
+    const int NKP = mma_nkp(max_chunk);
+    const int PST = NKP + 8;            // fp16 elements per P row (bank-conflict-free B loads)
+    unsigned char* Ks = smem;
+    unsigned char* Vs = smem + (size_t)NKP * DH * 2;
+    f16* Ps = reinterpret_cast<f16*>(Vs + (size_t)NKP * DV * 2);
+    f16* Pl = Ps + 8 * PST;
+    int* slots = reinterpret_cast<int*>(Pl + 8 * PST);
+    float* red = reinterpret_cast<float*>(slots + NKP);  // [2][4 warps][8 heads]
+    float* Os = reinterpret_cast<float*>(Ks);            // [R][DV + 4] once K is no longer read
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int gq = lane >> 2, tq = lane & 3;            // MMA fragment row group and column pair
     const int p = len[b] + pos_offset;
     const int ring = cap - n_meta;
     int meta_n, lo, n_win;
@@ -287,165 +280,184 @@ attn_decode_bulk_body(const f16* __restrict__ P, long long ldP, const f16* __res
     const int chunk = (L + n_split - 1) / n_split;
     const int k0 = min(L, s * chunk), k1 = min(L, k0 + chunk);
     const int nk = k1 - k0;
+    const int nkt = (nk + 15) / 16;  // 16-key tiles
+    const int nk16 = nkt * 16;
+    float* const rec = part + (((long long)b * H + g * R) * n_split + s) * (DV + 4);
+    const long long rec_head = (long long)n_split * (DV + 4);
+    if (nk == 0) {
+        for (int i = tid; i < R * (DV + 4); i += blockDim.x) {
+            const int r = i / (DV + 4), e = i - r * (DV + 4);
+            rec[r * rec_head + e] = e == DV ? -INFINITY : 0.f;
+        }
+        return;
+    }
+    // cache slot of every key of the split (keys past nk repeat the first, masked below)
+    for (int kk = tid; kk < nk16; kk += blockDim.x) {
+        const int idx = k0 + (kk < nk ? kk : 0);
+        const int j = idx < meta_n ? idx : lo + (idx - meta_n);
+        slots[kk] = j < n_meta ? j : n_meta + (j - n_meta) % ring;
+    }
+    __syncthreads();
     const long long kvbase = ((long long)b * G + g) * cap;
-    const unsigned char* kbase = reinterpret_cast<const unsigned char*>(k_cache + kvbase * DH);
-    const unsigned char* vbase = reinterpret_cast<const unsigned char*>(v_cache + kvbase * DV);
-    const int nkt = (nk + BK_TK - 1) / BK_TK;
-    const int nitems = nk > 0 ? nkt + (nk + BK_TV - 1) / BK_TV : 0;
-    auto issue = [&](int i) {
-        unsigned char* dst = stages + (i % BK_NST) * BK_STAGE;
-        if (i < nkt)
-            bk_issue_tile(dst, kbase, DH * 2, i * BK_TK, min(nk, (i + 1) * BK_TK), k0, meta_n, lo, n_meta, cap, ring,
-                          &full[i % BK_NST]);
-        else
-            bk_issue_tile(dst, vbase, DV * 2, (i - nkt) * BK_TV, min(nk, (i - nkt + 1) * BK_TV), k0, meta_n, lo,
-                          n_meta, cap, ring, &full[i % BK_NST]);
-    };
-    if (tid == 0) {
-        bk_never = 0;
-        for (int i = 0; i < BK_NST; ++i) tc::mbar_init(&full[i], 1);
-        tc::fence_mbar_init();
-        for (int i = 0; i < min(BK_NST, nitems); ++i) issue(i);
+    const unsigned char* kb = reinterpret_cast<const unsigned char*>(k_cache + kvbase * DH);
+    const unsigned char* vb = reinterpret_cast<const unsigned char*>(v_cache + kvbase * DV);
+    {
+        // K: eight threads per 128-byte row, rows tid / 8 + 16 i (the swizzle term is fixed)
+        const int c = tid & 7, r0 = tid >> 3, sw = ((c ^ (r0 & 7)) << 4);
+        for (int r = r0; r < nk16; r += 16)
+            wm::cpa16(Ks + r * (DH * 2) + sw, kb + (long long)slots[r] * (DH * 2) + c * 16);
+        wm::cpa_commit();
+        // V: VCH threads per row
+        constexpr int RPI = 128 / VCH;  // rows per pass
+        const int cv = tid % VCH, rv0 = tid / VCH, swv = ((cv ^ (rv0 & 7)) << 4);
+        for (int r = rv0; r < nk16; r += RPI)
+            wm::cpa16(Vs + r * (DV * 2) + swv, vb + (long long)slots[r] * (DV * 2) + cv * 16);
+        wm::cpa_commit();
     }
-    // this lane's 8 dimensions of the R queries, scaled by log2(e) / sqrt(64)
-    const int ch = lane & 7, kl = lane >> 3;
-    float2 qr[R][4];
+    // B operand of the scores: q^T, lane (gq, tq) holds dims 16 ks + 2 tq (+1, +8, +9) of
+    // query head gq (zero past R)
+    uint32_t qb[4][2];
+    {
+        const uint32_t* qrow = reinterpret_cast<const uint32_t*>(P + (long long)b * ldP + (g * R + gq) * DH);
 #pragma unroll
-    for (int r = 0; r < R; ++r) {
-        float qv[8];
-        load_row8<f16>(P + (long long)b * ldP + (g * R + r) * DH + 8 * ch, qv);
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-            qr[r][i] = make_float2(qv[2 * i] * (LOG2E * 0.125f), qv[2 * i + 1] * (LOG2E * 0.125f));
+        for (int ks = 0; ks < 4; ++ks) {
+            qb[ks][0] = gq < R ? qrow[8 * ks + tq] : 0u;
+            qb[ks][1] = gq < R ? qrow[8 * ks + tq + 4] : 0u;
+        }
     }
-    float2 acc[R][EPL / 2];
-#pragma unroll
-    for (int r = 0; r < R; ++r)
-#pragma unroll
-        for (int x = 0; x < EPL / 2; ++x) acc[r][x] = make_float2(0.f, 0.f);
+    wm::cpa_wait1();
     __syncthreads();
-    bool ok = true;
-    const long long wlim = tc::wait_limit(status);
-    for (int i = 0; i < nitems; ++i) {
-        const int st = i % BK_NST;
-        if (ok) ok = tc::mbar_wait(&full[st], (uint32_t)((i / BK_NST) & 1), &bk_never, wlim);
-        const unsigned char* sp = stages + st * BK_STAGE;
-        if (i < nkt) {
-            const int base = i * BK_TK, n = min(nk - base, BK_TK);
-            for (int pass = 0; pass * 16 < n; ++pass) {
-                const int kt = pass * 16 + warp * 4 + kl;
-                const bool valid = kt < n;
-                float2 a2[R];
+    // scores of the warp's key tiles: c[0..1] keys 16 t + gq, heads 2 tq, 2 tq + 1;
+    // c[2..3] the same heads at key 16 t + gq + 8
+    constexpr int MAXT = MAX_CHUNK / 64;  // key tiles per warp
+    float sc[MAXT][4];
+    const float qk_scale = LOG2E * 0.125f;  // log2(e) / sqrt(64)
+    float mx0 = -INFINITY, mx1 = -INFINITY;
 #pragma unroll
-                for (int r = 0; r < R; ++r) a2[r] = make_float2(0.f, 0.f);
-                if (valid) {
-                    const uint4 u = *reinterpret_cast<const uint4*>(sp + kt * (DH * 2) + ch * 16);
-                    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+    for (int i = 0; i < MAXT; ++i) {
+        const int t = warp + 4 * i;
 #pragma unroll
-                    for (int i2 = 0; i2 < 4; ++i2) {
-                        const float2 kf = x2float(w[i2]);
+        for (int e = 0; e < 4; ++e) sc[i][e] = 0.f;
+        if (t < nkt) {
+            const int row = 16 * t + (lane & 15);
 #pragma unroll
-                        for (int r = 0; r < R; ++r) a2[r] = __ffma2_rn(qr[r][i2], kf, a2[r]);
-                    }
-                }
-                float v = 0.f;
-#pragma unroll
-                for (int r = 0; r < R; ++r) {
-                    float a = a2[r].x + a2[r].y;
-                    a += __shfl_xor_sync(0xffffffffu, a, 1);
-                    a += __shfl_xor_sync(0xffffffffu, a, 2);
-                    a += __shfl_xor_sync(0xffffffffu, a, 4);
-                    if (ch == r) v = a;
-                }
-                if (valid && ch < R) ps[base + kt][ch] = v;
+            for (int ks = 0; ks < 4; ++ks) {
+                uint32_t a[4];
+                wm::ldsm_x4(a, Ks + row * (DH * 2) + (((2 * ks + (lane >> 4)) ^ (row & 7)) << 4));
+                wm::mma_f16(sc[i], a[0], a[1], a[2], a[3], qb[ks][0], qb[ks][1]);
             }
-        } else {
-            const int base = (i - nkt) * BK_TV, n = min(nk - base, BK_TV);
-#pragma unroll 2
-            for (int kv = warp; kv < n; kv += 4) {
-                float2 vv[EPL / 2];
-                if constexpr (EPL == 4) {
-                    const uint2 u = *reinterpret_cast<const uint2*>(sp + kv * (DV * 2) + lane * 8);
-                    vv[0] = x2float(u.x);
-                    vv[1] = x2float(u.y);
-                } else {
-                    vv[0] = x2float(*reinterpret_cast<const uint32_t*>(sp + kv * (DV * 2) + lane * 4));
-                }
-                const float4 pa = *reinterpret_cast<const float4*>(&ps[base + kv][0]);
-                float4 pb = make_float4(0.f, 0.f, 0.f, 0.f);
-                if constexpr (R > 4) pb = *reinterpret_cast<const float4*>(&ps[base + kv][4]);
-                const float pw[8] = {pa.x, pa.y, pa.z, pa.w, pb.x, pb.y, pb.z, pb.w};
-#pragma unroll
-                for (int r = 0; r < R; ++r) {
-                    const float2 pr = make_float2(pw[r], pw[r]);
-#pragma unroll
-                    for (int x = 0; x < EPL / 2; ++x) acc[r][x] = __ffma2_rn(pr, vv[x], acc[r][x]);
-                }
-            }
-        }
-        // the stage is free once every warp is past this barrier
-        if (__syncthreads_or(!ok)) {
-            if (tid == 0) {
-                tc::record_timeout(status, 3, i, st);
-                // let the copies already queued land before the block's memory is released
-                for (int q = i; q < min(nitems, i + BK_NST); ++q)
-                    tc::mbar_wait(&full[q % BK_NST], (uint32_t)((q / BK_NST) & 1), &bk_never);
-            }
-            return;
-        }
-        if (tid == 0 && i + BK_NST < nitems) issue(i + BK_NST);
-        if (i == nkt - 1) {
-            // every score of the split is in: per-head max and sum, warp w heads w, w + 4
-            for (int r = warp; r < R; r += 4) {
-                float mx = -INFINITY;
-                for (int kk = lane; kk < nk; kk += 32) mx = fmaxf(mx, ps[kk][r]);
-#pragma unroll
-                for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-                float sum = 0.f;
-                for (int kk = lane; kk < nk; kk += 32) {
-                    const float e = exp2f(ps[kk][r] - mx);
-                    ps[kk][r] = e;
-                    sum += e;
-                }
-#pragma unroll
-                for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-                if (lane == 0) { stat[2 * r] = mx; stat[2 * r + 1] = sum; }
-            }
-            __syncthreads();
+            const bool v0 = 16 * t + gq < nk, v1 = 16 * t + gq + 8 < nk;
+            sc[i][0] = v0 ? sc[i][0] * qk_scale : -INFINITY;
+            sc[i][1] = v0 ? sc[i][1] * qk_scale : -INFINITY;
+            sc[i][2] = v1 ? sc[i][2] * qk_scale : -INFINITY;
+            sc[i][3] = v1 ? sc[i][3] * qk_scale : -INFINITY;
+            mx0 = fmaxf(mx0, fmaxf(sc[i][0], sc[i][2]));
+            mx1 = fmaxf(mx1, fmaxf(sc[i][1], sc[i][3]));
         }
     }
-    // the four warps' P V sums meet in the stage memory (every copy has landed)
 #pragma unroll
-    for (int r = 0; r < R; ++r)
-        if constexpr (EPL == 4)
-            *reinterpret_cast<float4*>(&red[(warp * R + r) * DV + 4 * lane]) =
-                make_float4(acc[r][0].x, acc[r][0].y, acc[r][1].x, acc[r][1].y);
-        else
-            *reinterpret_cast<float2*>(&red[(warp * R + r) * DV + 2 * lane]) = acc[r][0];
+    for (int o = 4; o < 32; o <<= 1) {
+        mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
+        mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
+    }
+    if (gq == 0) {
+        red[warp * 8 + 2 * tq] = mx0;
+        red[warp * 8 + 2 * tq + 1] = mx1;
+    }
     __syncthreads();
-    for (int i = tid; i < R * DV; i += blockDim.x) {
-        const int r = i / DV, e = i % DV;
-        float sum = 0.f;
+    const float M0 = fmaxf(fmaxf(red[2 * tq], red[8 + 2 * tq]), fmaxf(red[16 + 2 * tq], red[24 + 2 * tq]));
+    const float M1 =
+        fmaxf(fmaxf(red[2 * tq + 1], red[9 + 2 * tq]), fmaxf(red[17 + 2 * tq], red[25 + 2 * tq]));
+    // p = exp2(s - max) (every head sees every key, so the max is finite) as p_hi + p_lo
+    float l0 = 0.f, l1 = 0.f;
 #pragma unroll
-        for (int w = 0; w < 4; ++w) sum += red[(w * R + r) * DV + e];
-        part[(((long long)b * H + g * R + r) * n_split + s) * (DV + 4) + e] = sum;
+    for (int i = 0; i < MAXT; ++i) {
+        const int t = warp + 4 * i;
+        if (t < nkt) {
+            const int key = 16 * t + gq;
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float pe = fast_exp2(sc[i][e] - ((e & 1) ? M1 : M0));
+                const __half hi = __float2half_rn(pe);
+                const __half lo = __float2half_rn(pe - __half2float(hi));
+                const int at = (2 * tq + (e & 1)) * PST + key + ((e & 2) ? 8 : 0);
+                Ps[at] = hi;
+                Pl[at] = lo;
+                if (e & 1) l1 += pe; else l0 += pe;
+            }
+        }
+    }
+#pragma unroll
+    for (int o = 4; o < 32; o <<= 1) {
+        l0 += __shfl_xor_sync(0xffffffffu, l0, o);
+        l1 += __shfl_xor_sync(0xffffffffu, l1, o);
+    }
+    if (gq == 0) {
+        red[32 + warp * 8 + 2 * tq] = l0;
+        red[32 + warp * 8 + 2 * tq + 1] = l1;
+    }
+    wm::cpa_wait0();
+    __syncthreads();
+    // P V over all keys for the warp's V columns
+    float oc[MTW][4];
+#pragma unroll
+    for (int m = 0; m < MTW; ++m)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) oc[m][e] = 0.f;
+    const uint32_t* Pw = reinterpret_cast<const uint32_t*>(Ps) + gq * (PST / 2);
+    const uint32_t* Plw = reinterpret_cast<const uint32_t*>(Pl) + gq * (PST / 2);
+    const int vrow = (lane & 7) + ((lane >> 4) << 3);  // key within the 16-key step
+    const int vch = (lane >> 3) & 1;                   // chunk within the 16-column tile
+    for (int t = 0; t < nkt; ++t) {
+        const uint32_t b0 = Pw[8 * t + tq], b1 = Pw[8 * t + tq + 4];
+        const uint32_t c0 = Plw[8 * t + tq], c1 = Plw[8 * t + tq + 4];
+        const int key = 16 * t + vrow;
+        const unsigned char* vr = Vs + key * (DV * 2);
+#pragma unroll
+        for (int m = 0; m < MTW; ++m) {
+            const int c = 2 * (warp * MTW + m) + vch;
+            uint32_t a[4];
+            wm::ldsm_x4_t(a, vr + ((c ^ (key & 7)) << 4));
+            wm::mma_f16(oc[m], a[0], a[1], a[2], a[3], b0, b1);
+            wm::mma_f16(oc[m], a[0], a[1], a[2], a[3], c0, c1);
+        }
+    }
+    // (Os reuses K, whose last reads came before the two barriers above)
+#pragma unroll
+    for (int m = 0; m < MTW; ++m) {
+        const int col = 16 * (warp * MTW + m) + gq;
+        if (2 * tq < R) {
+            Os[(2 * tq) * (DV + 4) + col] = oc[m][0];
+            Os[(2 * tq) * (DV + 4) + col + 8] = oc[m][2];
+        }
+        if (2 * tq + 1 < R) {
+            Os[(2 * tq + 1) * (DV + 4) + col] = oc[m][1];
+            Os[(2 * tq + 1) * (DV + 4) + col + 8] = oc[m][3];
+        }
+    }
+    __syncthreads();
+    for (int i = tid; i < R * (DV / 4); i += blockDim.x) {
+        const int r = i / (DV / 4), q = i - r * (DV / 4);
+        *reinterpret_cast<float4*>(rec + r * rec_head + 4 * q) =
+            *reinterpret_cast<const float4*>(Os + r * (DV + 4) + 4 * q);
     }
     if (tid < R) {
-        float* o = part + (((long long)b * H + g * R + tid) * n_split + s) * (DV + 4) + DV;
-        o[0] = nk > 0 ? stat[2 * tid] : -INFINITY;
-        o[1] = nk > 0 ? stat[2 * tid + 1] : 0.f;
+        const float mx = fmaxf(fmaxf(red[tid], red[8 + tid]), fmaxf(red[16 + tid], red[24 + tid]));
+        const float sum = red[32 + tid] + red[40 + tid] + red[48 + tid] + red[56 + tid];
+        rec[tid * rec_head + DV] = mx;
+        rec[tid * rec_head + DV + 1] = sum;
     }
 }
 
 template <int R, int DV>
-__global__ void __launch_bounds__(128, R <= 6 ? 5 : 4)
-attn_decode_bulk_kernel(const f16* __restrict__ P, long long ldP, const f16* __restrict__ k_cache,
-                        const f16* __restrict__ v_cache, int cap, const int* __restrict__ len, int pos_offset,
-                        float* __restrict__ part, int n_split, int H, int G, int n_meta, int window, int max_chunk,
-                        int* status) {
-    extern __shared__ __align__(128) unsigned char bk_smem[];
-    attn_decode_bulk_body<R, DV>(P, ldP, k_cache, v_cache, cap, len, pos_offset, part, n_split, H, G, n_meta, window,
-                                 max_chunk, status, blockIdx.x, blockIdx.y, blockIdx.z, bk_smem);
+__global__ void __launch_bounds__(128, 4)
+attn_decode_mma_kernel(const f16* __restrict__ P, long long ldP, const f16* __restrict__ k_cache,
+                       const f16* __restrict__ v_cache, int cap, const int* __restrict__ len, int pos_offset,
+                       float* __restrict__ part, int n_split, int H, int G, int n_meta, int window, int max_chunk,
+                       int* status) {
+    extern __shared__ __align__(128) unsigned char mm_smem[];
+    attn_decode_mma_body<R, DV>(P, ldP, k_cache, v_cache, cap, len, pos_offset, part, n_split, H, G, n_meta, window,
+                                max_chunk, status, blockIdx.x, blockIdx.y, blockIdx.z, mm_smem);
 }
 
 template <typename T, int DV>
@@ -758,7 +770,7 @@ struct DecodeSsmArgs {
 };
 
 template <int R, int DV, typename TW>
-__global__ void __launch_bounds__(128, R <= 6 ? 5 : 4)
+__global__ void __launch_bounds__(128, 4)
 decode_attn_ssm_kernel(const DecodeAttnArgs a, const DecodeSsmArgs<TW> m, int n_ssm, int* status) {
     extern __shared__ __align__(128) unsigned char dsm[];
     // the SSM blocks are spread evenly through the grid: block bid is the SSM block
@@ -772,7 +784,7 @@ decode_attn_ssm_kernel(const DecodeAttnArgs a, const DecodeSsmArgs<TW> m, int n_
                                  k0 % m.gx, k0 / m.gx, dsm);
     } else {
         const int q = (int)bid - k0;
-        attn_decode_bulk_body<R, DV>(a.P, a.ldP, a.k_cache, a.v_cache, a.cap, a.len, a.pos_offset, a.part, a.n_split,
+        attn_decode_mma_body<R, DV>(a.P, a.ldP, a.k_cache, a.v_cache, a.cap, a.len, a.pos_offset, a.part, a.n_split,
                                      a.H, a.G, a.n_meta, a.window, a.max_chunk, status, q % a.n_split,
                                      (q / a.n_split) % a.G, q / (a.n_split * a.G), dsm);
     }
@@ -793,17 +805,17 @@ static void (*fused_kernel(int R))(const DecodeAttnArgs, const DecodeSsmArgs<TW>
 }
 
 template <int DV>
-static void (*bulk_kernel(int R))(const f16*, long long, const f16*, const f16*, int, const int*, int, float*, int,
+static void (*mma_kernel(int R))(const f16*, long long, const f16*, const f16*, int, const int*, int, float*, int,
                                   int, int, int, int, int, int*) {
     switch (R) {
-        case 1: return attn_decode_bulk_kernel<1, DV>;
-        case 2: return attn_decode_bulk_kernel<2, DV>;
-        case 3: return attn_decode_bulk_kernel<3, DV>;
-        case 4: return attn_decode_bulk_kernel<4, DV>;
-        case 5: return attn_decode_bulk_kernel<5, DV>;
-        case 6: return attn_decode_bulk_kernel<6, DV>;
-        case 7: return attn_decode_bulk_kernel<7, DV>;
-        default: return attn_decode_bulk_kernel<8, DV>;
+        case 1: return attn_decode_mma_kernel<1, DV>;
+        case 2: return attn_decode_mma_kernel<2, DV>;
+        case 3: return attn_decode_mma_kernel<3, DV>;
+        case 4: return attn_decode_mma_kernel<4, DV>;
+        case 5: return attn_decode_mma_kernel<5, DV>;
+        case 6: return attn_decode_mma_kernel<6, DV>;
+        case 7: return attn_decode_mma_kernel<7, DV>;
+        default: return attn_decode_mma_kernel<8, DV>;
     }
 }
 
@@ -828,12 +840,15 @@ static int attn_decode_dv(const Ctx& ctx, const T* P, long long ldP, const T* k_
                           int H, int G, int n_meta, int window) {
     dim3 grid(n_split, G, B);
     if constexpr (std::is_same<T, f16>::value) {
-        // K/V rows staged by bulk copies: 16-byte aligned rows (64 and DV fp16)
         const int max_chunk = (cache_cap + n_split - 1) / n_split;
-        const size_t smem = (size_t)BK_NST * BK_STAGE + (size_t)max_chunk * 32 + 16 * sizeof(float) +
-                            BK_NST * sizeof(uint64_t);
-        HYMBA_LAUNCH(ctx, "attn_decode", bulk_kernel<DV>(H / G), grid, 128, smem, P, ldP, k_cache, v_cache,
-                     cache_cap, len, pos_offset, part, n_split, H, G, n_meta, window, max_chunk, ctx.status);
+        const size_t smem = mma_smem_bytes(max_chunk, DV);
+        auto kern = mma_kernel<DV>(H / G);
+        if (smem > 48 * 1024) {
+            static std::atomic<unsigned long long> smem_set[8];
+            if (!smem_opt_in_once(smem_set[H / G - 1], kern, mma_smem_bytes(MAX_CHUNK, DV), ctx)) return HYMBA_ERR_CUDA;
+        }
+        HYMBA_LAUNCH(ctx, "attn_decode", kern, grid, 128, smem, P, ldP, k_cache, v_cache, cache_cap, len, pos_offset,
+                     part, n_split, H, G, n_meta, window, max_chunk, ctx.status);
     } else {
         HYMBA_LAUNCH(ctx, "attn_decode", (stream_kernel<T, DV>(H / G)), grid, 128, 0, P, ldP, k_cache, v_cache,
                      cache_cap, len, pos_offset, part, n_split, H, G, n_meta, window, ctx.status);
@@ -854,8 +869,9 @@ int launch_attn_decode(const Ctx& ctx, const T* P, long long ldP, const T* k_cac
                        int window) {
     if (H / G > MAX_R || (dv != 128 && dv != 64)) return HYMBA_ERR_UNSUPPORTED;
     if ((cache_cap + n_split - 1) / n_split > MAX_CHUNK) return HYMBA_ERR_INVALID_ARG;
-    // 16-byte loads of q, K and V rows
-    if ((reinterpret_cast<uintptr_t>(P) | reinterpret_cast<uintptr_t>(k_cache) | reinterpret_cast<uintptr_t>(v_cache)) & 15 ||
+    // 16-byte loads of q, K and V rows; 16-byte stores of the partial records
+    if ((reinterpret_cast<uintptr_t>(P) | reinterpret_cast<uintptr_t>(k_cache) | reinterpret_cast<uintptr_t>(v_cache) |
+         reinterpret_cast<uintptr_t>(part)) & 15 ||
         ldP % (16 / (long long)sizeof(T)))
         return HYMBA_ERR_UNSUPPORTED;
     if (dv == 128)
@@ -911,7 +927,8 @@ int launch_decode_attn_ssm(const Ctx& ctx, const f16* P, long long ldP, const f1
     if (ldP % V || col_B % V || col_C % V || (reinterpret_cast<uintptr_t>(conv_w) & 15) ||
         (reinterpret_cast<uintptr_t>(A_log) & 15) || (reinterpret_cast<uintptr_t>(conv) & 15) ||
         (reinterpret_cast<uintptr_t>(h) & 15) || (reinterpret_cast<uintptr_t>(P) & 15) ||
-        ((reinterpret_cast<uintptr_t>(k_cache) | reinterpret_cast<uintptr_t>(v_cache)) & 15))
+        ((reinterpret_cast<uintptr_t>(k_cache) | reinterpret_cast<uintptr_t>(v_cache) |
+          reinterpret_cast<uintptr_t>(part)) & 15))
         return HYMBA_ERR_UNSUPPORTED;
     using Slot = typename WSlot<TW>::type;
     const int npairs = (dt_rank + 1) / 2;
@@ -922,8 +939,7 @@ int launch_decode_attn_ssm(const Ctx& ctx, const f16* P, long long ldP, const f1
                      (reinterpret_cast<uintptr_t>(w_dt) & 15) == 0 && col_dtl % 2 == 0 &&
                      SSM_CH * npairs / 4 <= SSM_WLD * SSM_WARPS * 32 && SSM_ROWS * npairs <= SSM_XLD * SSM_WARPS * 32;
     const int max_chunk = (cache_cap + n_split - 1) / n_split;
-    const size_t smem_attn = (size_t)BK_NST * BK_STAGE + (size_t)max_chunk * 32 + 16 * sizeof(float) +
-                             BK_NST * sizeof(uint64_t);
+    const size_t smem_attn = mma_smem_bytes(max_chunk, dv);
     const size_t smem = smem_attn > smem_ssm ? smem_attn : smem_ssm;
     DecodeAttnArgs a{P, ldP, k_cache, v_cache, cache_cap, len, pos_offset, part, n_split, H, G, n_meta, window,
                      max_chunk};
@@ -933,8 +949,10 @@ int launch_decode_attn_ssm(const Ctx& ctx, const f16* P, long long ldP, const f1
     const int n_attn = n_split * G * B;
     auto kern = dv == 128 ? fused_kernel<128, TW>(H / G) : fused_kernel<64, TW>(H / G);
     if (smem > 48 * 1024) {
-        static std::atomic<unsigned long long> smem_set{0};
-        if (!smem_opt_in_once(smem_set, kern, smem, ctx)) return HYMBA_ERR_CUDA;
+        // one opt-in per kernel and device, at the largest size any launch asks for
+        static std::atomic<unsigned long long> smem_set[2][8];
+        const size_t most = std::max(mma_smem_bytes(MAX_CHUNK, dv), smem_ssm);
+        if (!smem_opt_in_once(smem_set[dv == 128][H / G - 1], kern, most, ctx)) return HYMBA_ERR_CUDA;
     }
     HYMBA_LAUNCH(ctx, "attn_ssm_decode", kern, n_ssm + n_attn, 128, smem, a, m, n_ssm, ctx.status);
     return HYMBA_OK;

@@ -67,7 +67,8 @@ __device__ __forceinline__ void load8f(const float* p, float* v) {
 // after a cluster barrier reads the other CTAs' from their shared memory.
 constexpr int FC = 8;    // CTAs per row (cluster size)
 constexpr int FT = 64;   // threads per CTA
-constexpr int FSPL = 8;  // split records per piece loaded ahead of the merge weights
+constexpr int FSPL = 16;  // split records per piece loaded ahead of the merge weights
+constexpr int FYI = 4;    // residual values per thread loaded ahead (y_init)
 static_assert(FC * FT * 8 >= kMaxWidth, "one piece per thread and branch");
 
 template <typename I, typename T, bool CONCAT>
@@ -114,6 +115,22 @@ fuse_split_kernel(const float* __restrict__ part, int n_split, int H, int dv, co
     if (has_y) {
         load8<I>(ypre + row * di + vy * 8, y);
         load8<I>(P + row * ldP + col_z + vy * 8, z);
+    }
+    // the per-channel factors of this thread's pieces and its share of the residual
+    float fa[8], fb[8], fc[8], fd[8];
+    if constexpr (CONCAT) {
+        if (has_y) { load8f(g_ssm + vy * 8, fa); load8f(beta2 + vy * 8, fb); }
+        if (has_o) { load8f(g_attn + vo * 8, fc); load8f(beta1 + vo * 8, fd); }
+    } else if (has_y) {
+        load8f(g_attn + vy * 8, fa); load8f(beta1 + vy * 8, fb);
+        load8f(g_ssm + vy * 8, fc); load8f(beta2 + vy * 8, fd);
+    }
+    const bool init = y_init && y_init != y_res;
+    float yr[FYI];
+#pragma unroll
+    for (int k = 0; k < FYI; ++k) {
+        const int c = cr * FT + t + k * FC * FT;
+        yr[k] = init && y_res && c < d_model ? y_res[row * d_model + c] : 0.f;
     }
     for (int i = t; i < nh * n_split; i += FT) {
         const int hh = i / n_split, sp = i - hh * n_split;
@@ -210,41 +227,36 @@ fuse_split_kernel(const float* __restrict__ part, int n_split, int H, int dv, co
     if constexpr (CONCAT) {
         const long long ldu = di + hv;
         if (has_y) {
-            const int c = vy * 8;
-            float gs[8], b2[8], u[8];
-            load8f(g_ssm + c, gs);
-            load8f(beta2 + c, b2);
+            float u[8];
 #pragma unroll
-            for (int i = 0; i < 8; ++i) u[i] = b2[i] * gs[i] * y[i] * ry;
-            store8<T>(U + row * ldu + c, u);
+            for (int i = 0; i < 8; ++i) u[i] = fb[i] * fa[i] * y[i] * ry;
+            store8<T>(U + row * ldu + vy * 8, u);
         }
         if (has_o) {
-            const int c = vo * 8;
-            float ga[8], b1[8], u[8];
-            load8f(g_attn + c, ga);
-            load8f(beta1 + c, b1);
+            float u[8];
 #pragma unroll
-            for (int i = 0; i < 8; ++i) u[i] = b1[i] * ga[i] * o[i] * ro;
-            store8<T>(U + row * ldu + di + c, u);
+            for (int i = 0; i < 8; ++i) u[i] = fd[i] * fc[i] * o[i] * ro;
+            store8<T>(U + row * ldu + di + vo * 8, u);
         }
     } else if (has_o && has_y) {
         // equal widths: a thread holds the same channels of both branches
-        const int c = vy * 8;
-        float ga[8], gs[8], b1[8], b2[8], u[8];
-        load8f(g_attn + c, ga);
-        load8f(g_ssm + c, gs);
-        load8f(beta1 + c, b1);
-        load8f(beta2 + c, b2);
+        float u[8];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) u[i] = b1[i] * ga[i] * o[i] * ro + b2[i] * gs[i] * y[i] * ry;
-        store8<T>(U + row * di + c, u);
+        for (int i = 0; i < 8; ++i) u[i] = fb[i] * fa[i] * o[i] * ro + fd[i] * fc[i] * y[i] * ry;
+        store8<T>(U + row * di + vy * 8, u);
     }
     if (len_inc && cr == 0 && t == 0) len_inc[row] += 1;
     // the output projection that follows adds its split-K partial sums to y: y starts as
     // the residual (or zero), unless y is the residual itself
-    if (y_init && y_init != y_res)
-        for (int c = cr * FT + t; c < d_model; c += FC * FT)
+    if (init) {
+#pragma unroll
+        for (int k = 0; k < FYI; ++k) {
+            const int c = cr * FT + t + k * FC * FT;
+            if (c < d_model) y_init[row * d_model + c] = yr[k];
+        }
+        for (int c = cr * FT + t + FYI * FC * FT; c < d_model; c += FC * FT)
             y_init[row * d_model + c] = y_res ? y_res[row * d_model + c] : 0.f;
+    }
     cluster_wait();
 }
 

@@ -25,6 +25,7 @@
 // The work is bound by the HBM traffic of x and y (4 bytes per row and channel); the
 // tensor cores do about 330 flops per (row, channel).
 #include "kernels.h"
+#include "warp_mma.cuh"
 
 namespace hymba {
 
@@ -53,40 +54,15 @@ struct SsdSmem {
     alignas(16) float Dv[SP];
 };
 
-__device__ __forceinline__ void cpa16(void* dst, const void* src, bool zero = false) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(static_cast<uint32_t>(__cvta_generic_to_shared(dst))),
-                 "l"(src), "r"(zero ? 0 : 16)
-                 : "memory");
-}
-__device__ __forceinline__ void cpa4(void* dst, const void* src) {
-    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(static_cast<uint32_t>(__cvta_generic_to_shared(dst))),
-                 "l"(src)
-                 : "memory");
-}
-__device__ __forceinline__ void cpa_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-__device__ __forceinline__ void cpa_wait0() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+using wm::cpa16;
+using wm::cpa4;
+using wm::cpa_commit;
+using wm::cpa_wait0;
+using wm::ldsm_x4;
+using wm::ldsm_x4_t;
+using wm::mma_f16;
+using wm::pack_h2;
 
-__device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], const void* p) {
-    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
-                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-                 : "r"(static_cast<uint32_t>(__cvta_generic_to_shared(p))));
-}
-__device__ __forceinline__ void ldsm_x4_t(uint32_t (&r)[4], const void* p) {
-    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
-                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-                 : "r"(static_cast<uint32_t>(__cvta_generic_to_shared(p))));
-}
-__device__ __forceinline__ void mma_f16(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
-                                        uint32_t b0, uint32_t b1) {
-    asm volatile(
-        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
-        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
-        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
-}
-__device__ __forceinline__ uint32_t pack_h2(float lo, float hi) {
-    const __half2 h = __floats2half2_rn(lo, hi);
-    return *reinterpret_cast<const uint32_t*>(&h);
-}
 __device__ __forceinline__ uint32_t scale_h2(uint32_t v, float lo, float hi) {
     const __half2 r = __hmul2(*reinterpret_cast<const __half2*>(&v), __floats2half2_rn(lo, hi));
     return *reinterpret_cast<const uint32_t*>(&r);
