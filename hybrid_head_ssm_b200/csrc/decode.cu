@@ -509,8 +509,10 @@ __device__ __forceinline__ uint32_t wpack(bf16 lo, bf16 hi) {
 // read once for both). The block's 32 rows of W_dt and 8 dt_low rows are staged in
 // shared memory (rows padded to an odd number of slots, so that the per-lane row reads
 // hit distinct banks); with 16-bit operands and an even dt_rank <= 128 the staging is
-// a few wide loads per thread, all in flight together, and the loads of h go out
-// before the dot products.
+// a few wide loads per thread. Every load that does not depend on Delta (the state rows,
+// the conv state, x, the per-channel constants, and the rows' B and C, copied once per
+// block into shared memory) is issued before the staging, so the block waits for one
+// round trip to memory rather than one per stage.
 template <typename T, typename TW>
 __device__ __forceinline__ void
 ssm_decode_body(const T* __restrict__ P, long long ldP, int col_x, int col_B, int col_C,
@@ -533,25 +535,63 @@ ssm_decode_body(const T* __restrict__ P, long long ldP, int col_x, int col_B, in
         bs[u] = b0 + warp + u * SSM_WARPS;
         ok[u] = cok && bs[u] < B;
     }
-    // the state rows: the longest loads, independent of Delta, issued ahead of the dot
-    // products (which run while they are in flight)
-    float hv[SSM_RPT][NS];
-    auto load_h = [&]() {
-#pragma unroll
-        for (int u = 0; u < SSM_RPT; ++u) {
-            const float4* hp = reinterpret_cast<const float4*>(h + ((long long)bs[u] * di + c) * NS);
-#pragma unroll
-            for (int q = 0; q < NS / 4; ++q) {
-                const float4 t = ok[u] ? hp[q] : make_float4(0.f, 0.f, 0.f, 0.f);
-                hv[u][4 * q] = t.x; hv[u][4 * q + 1] = t.y; hv[u][4 * q + 2] = t.z; hv[u][4 * q + 3] = t.w;
-            }
-        }
-    };
     const int npairs = (r + 1) / 2;
     const int cp = min(npairs, SSM_PAIRS);
     const int RS = cp | 1;
     Slot* Ws = reinterpret_cast<Slot*>(ssm_smem);
     float2* xs = reinterpret_cast<float2*>(ssm_smem + ((SSM_CH * RS * sizeof(Slot) + 15) & ~size_t(15)));
+    // B and C of the block's rows: [SSM_ROWS][2][NS] in the projection's type
+    T* bcs = reinterpret_cast<T*>(xs + SSM_ROWS * cp);
+    {
+        constexpr int CH16 = NS * (int)sizeof(T) / 16;  // 16-byte pieces of one B or C row
+        if (tid < SSM_ROWS * 2 * CH16) {
+            const int row = tid / (2 * CH16), w = (tid / CH16) & 1, k = tid % CH16;
+            if (b0 + row < B)
+                wm::cpa16(bcs + (row * 2 + w) * NS + k * (16 / (int)sizeof(T)),
+                          P + (long long)(b0 + row) * ldP + (w ? col_C : col_B) + k * (16 / (int)sizeof(T)));
+        }
+        wm::cpa_commit();
+    }
+    // the state rows, the conv state, x and the per-channel constants
+    float hv[SSM_RPT][NS];
+    float4 cst4[SSM_RPT];
+    float xin[SSM_RPT];
+#pragma unroll
+    for (int u = 0; u < SSM_RPT; ++u) {
+        const long long idx = (long long)bs[u] * di + c;
+        const float4* hp4 = reinterpret_cast<const float4*>(h + idx * NS);
+#pragma unroll
+        for (int q = 0; q < NS / 4; ++q) {
+            const float4 t = ok[u] ? hp4[q] : make_float4(0.f, 0.f, 0.f, 0.f);
+            hv[u][4 * q] = t.x; hv[u][4 * q + 1] = t.y; hv[u][4 * q + 2] = t.z; hv[u][4 * q + 3] = t.w;
+        }
+        cst4[u] = ok[u] ? *reinterpret_cast<const float4*>(conv + idx * KC) : make_float4(0.f, 0.f, 0.f, 0.f);
+        xin[u] = ok[u] ? to_f(P[(long long)bs[u] * ldP + col_x + c]) : 0.f;
+    }
+    float4 w4 = make_float4(0.f, 0.f, 0.f, 0.f);
+    float cb = 0.f, bdt = 0.f, Dc = 0.f;
+    float Ae[NS];  // -exp(A_log) log2(e): exp(Delta A) = exp2(Delta Ae)
+    if (cok) {
+        w4 = *reinterpret_cast<const float4*>(conv_w + (long long)c * KC);
+        cb = conv_b[c];
+        bdt = b_dt[hp > 0 ? c / hp : c];
+        Dc = Dp[c];
+        if (hp > 0) {
+            // SSD form: one A per head, for every state
+            const float a = -fast_exp2(A_log[c / hp] * LOG2E) * LOG2E;
+#pragma unroll
+            for (int n = 0; n < NS; ++n) Ae[n] = a;
+        } else {
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const float4 a4 = *reinterpret_cast<const float4*>(A_log + (long long)c * NS + 4 * k);
+                Ae[4 * k] = -fast_exp2(a4.x * LOG2E) * LOG2E;
+                Ae[4 * k + 1] = -fast_exp2(a4.y * LOG2E) * LOG2E;
+                Ae[4 * k + 2] = -fast_exp2(a4.z * LOG2E) * LOG2E;
+                Ae[4 * k + 3] = -fast_exp2(a4.w * LOG2E) * LOG2E;
+            }
+        }
+    }
     float2 dacc[SSM_RPT];
 #pragma unroll
     for (int u = 0; u < SSM_RPT; ++u) dacc[u] = make_float2(0.f, 0.f);
@@ -599,7 +639,6 @@ ssm_decode_body(const T* __restrict__ P, long long ldP, int col_x, int col_B, in
                 }
             }
             __syncthreads();
-            load_h();
 #pragma unroll 4
             for (int q = 0; q < npairs; ++q) {
                 const float2 wv = wunpack(Ws[lane * RS + q]);
@@ -611,7 +650,6 @@ ssm_decode_body(const T* __restrict__ P, long long ldP, int col_x, int col_B, in
     }
     if (!(sizeof(TW) == 2 && wide)) {
         // general staging: any dt_rank and weight type, in passes of SSM_PAIRS pairs
-        load_h();
         const TW wz = from_f<TW>(0.f);
         for (int q0 = 0; q0 < npairs; q0 += cp) {
             const int nq = min(cp, npairs - q0);
@@ -650,36 +688,18 @@ ssm_decode_body(const T* __restrict__ P, long long ldP, int col_x, int col_B, in
             }
         }
     }
+    wm::cpa_wait0();
+    __syncthreads();  // B and C are in
     if (!cok) return;
-    // per-channel constants, shared by the thread's sequences
-    const float4 w4 = *reinterpret_cast<const float4*>(conv_w + (long long)c * KC);
-    const float cb = conv_b[c], bdt = b_dt[hp > 0 ? c / hp : c], Dc = Dp[c];
-    float Ae[NS];  // -exp(A_log) log2(e): exp(Delta A) = exp2(Delta Ae)
-    if (hp > 0) {
-        // SSD form: one A per head, for every state
-        const float a = -fast_exp2(A_log[c / hp] * LOG2E) * LOG2E;
-#pragma unroll
-        for (int n = 0; n < NS; ++n) Ae[n] = a;
-    } else {
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            const float4 a4 = *reinterpret_cast<const float4*>(A_log + (long long)c * NS + 4 * k);
-            Ae[4 * k] = -fast_exp2(a4.x * LOG2E) * LOG2E;
-            Ae[4 * k + 1] = -fast_exp2(a4.y * LOG2E) * LOG2E;
-            Ae[4 * k + 2] = -fast_exp2(a4.z * LOG2E) * LOG2E;
-            Ae[4 * k + 3] = -fast_exp2(a4.w * LOG2E) * LOG2E;
-        }
-    }
 #pragma unroll
     for (int u = 0; u < SSM_RPT; ++u) {
         if (!ok[u]) continue;
         const long long idx = (long long)bs[u] * di + c;
-        const T* prow = P + (long long)bs[u] * ldP;
         const float d = softplus_fast(dacc[u].x + dacc[u].y + bdt);
         // shift the new input into the conv state (oldest first), then convolve
         float4* cst = reinterpret_cast<float4*>(conv + idx * KC);
-        const float4 c4 = *cst;
-        const float cs[KC] = {c4.y, c4.z, c4.w, to_f(prow[col_x + c])};
+        const float4 c4 = cst4[u];
+        const float cs[KC] = {c4.y, c4.z, c4.w, xin[u]};
         float acc = cb;
         acc = fmaf(w4.x, cs[0], acc);
         acc = fmaf(w4.y, cs[1], acc);
@@ -688,35 +708,13 @@ ssm_decode_body(const T* __restrict__ P, long long ldP, int col_x, int col_B, in
         *cst = make_float4(cs[0], cs[1], cs[2], cs[3]);
         const float xc = silu_f(acc);
         const float dx = d * xc;
-        float Bv[NS], Cv[NS];
-        if constexpr (sizeof(T) == 2) {
-#pragma unroll
-            for (int k = 0; k < 2; ++k) {
-                const uint4 ub = *reinterpret_cast<const uint4*>(prow + col_B + 8 * k);
-                const uint4 uc = *reinterpret_cast<const uint4*>(prow + col_C + 8 * k);
-                const T* hb = reinterpret_cast<const T*>(&ub);
-                const T* hc = reinterpret_cast<const T*>(&uc);
-#pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    Bv[8 * k + i] = to_f(hb[i]);
-                    Cv[8 * k + i] = to_f(hc[i]);
-                }
-            }
-        } else {
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                const float4 fb = *reinterpret_cast<const float4*>(prow + col_B + 4 * k);
-                const float4 fc = *reinterpret_cast<const float4*>(prow + col_C + 4 * k);
-                Bv[4 * k] = fb.x; Bv[4 * k + 1] = fb.y; Bv[4 * k + 2] = fb.z; Bv[4 * k + 3] = fb.w;
-                Cv[4 * k] = fc.x; Cv[4 * k + 1] = fc.y; Cv[4 * k + 2] = fc.z; Cv[4 * k + 3] = fc.w;
-            }
-        }
+        const T* Bs = bcs + (warp + u * SSM_WARPS) * 2 * NS;  // this row's B, then C
         float y = 0.f;
 #pragma unroll
         for (int n = 0; n < NS; ++n) {
             const float a = fast_exp2(d * Ae[n]);
-            hv[u][n] = fmaf(a, hv[u][n], dx * Bv[n]);
-            y = fmaf(Cv[n], hv[u][n], y);
+            hv[u][n] = fmaf(a, hv[u][n], dx * to_f(Bs[n]));
+            y = fmaf(to_f(Bs[NS + n]), hv[u][n], y);
         }
         float4* hp = reinterpret_cast<float4*>(h + idx * NS);
 #pragma unroll
@@ -728,7 +726,7 @@ ssm_decode_body(const T* __restrict__ P, long long ldP, int col_x, int col_B, in
 
 
 template <typename T, typename TW>
-__global__ void __launch_bounds__(SSM_WARPS * 32, 6)
+__global__ void __launch_bounds__(SSM_WARPS * 32, 4)
 ssm_decode_kernel(const T* __restrict__ P, long long ldP, int col_x, int col_B, int col_C,
                   int col_dtl, const TW* __restrict__ w_dt, const float* __restrict__ b_dt, int r,
                   int wide, const float* __restrict__ conv_w, const float* __restrict__ conv_b,
@@ -898,7 +896,7 @@ int launch_ssm_decode(const Ctx& ctx, const T* P, long long ldP, int col_x, int 
     const int npairs = (dt_rank + 1) / 2;
     const int cp = npairs < SSM_PAIRS ? npairs : SSM_PAIRS;
     const size_t smem = ((SSM_CH * (size_t)(cp | 1) * sizeof(Slot) + 15) & ~size_t(15)) +
-                        (size_t)SSM_ROWS * cp * sizeof(float2);
+                        (size_t)SSM_ROWS * cp * sizeof(float2) + (size_t)SSM_ROWS * 2 * 16 * sizeof(T);
     // one-pass wide staging: 16-bit W_dt with even dt_rank <= 128 (so the block's run of
     // 32 rows is 16-byte aligned and a whole number of 16-byte pieces, d_inner being a
     // multiple of 32), 4-byte dt_low pairs
@@ -934,7 +932,7 @@ int launch_decode_attn_ssm(const Ctx& ctx, const f16* P, long long ldP, const f1
     const int npairs = (dt_rank + 1) / 2;
     const int cp = npairs < SSM_PAIRS ? npairs : SSM_PAIRS;
     const size_t smem_ssm = ((SSM_CH * (size_t)(cp | 1) * sizeof(Slot) + 15) & ~size_t(15)) +
-                            (size_t)SSM_ROWS * cp * sizeof(float2);
+                            (size_t)SSM_ROWS * cp * sizeof(float2) + (size_t)SSM_ROWS * 2 * 16 * sizeof(f16);
     const int wide = hp == 0 && sizeof(TW) == 2 && dt_rank % 2 == 0 && npairs <= SSM_PAIRS && di % SSM_CH == 0 &&
                      (reinterpret_cast<uintptr_t>(w_dt) & 15) == 0 && col_dtl % 2 == 0 &&
                      SSM_CH * npairs / 4 <= SSM_WLD * SSM_WARPS * 32 && SSM_ROWS * npairs <= SSM_XLD * SSM_WARPS * 32;
