@@ -275,11 +275,15 @@ def add_work(total, part):
 def decode_work(cfg, B, cap):
     """Algorithmic HBM bytes per launch of the decode kernels (2-byte K/V, fp32 state)."""
     G, dh, dv, di, r = cfg.n_kv_heads, cfg.head_dim, cfg.v_head_dim, cfg.d_inner, cfg.dt_rank
+    attn = B * G * cap * (dh + dv) * 2.0
+    # h and conv state read + written (fp32), x read, y_pre written per (sequence,
+    # channel); W_dt once and the dt_low rows for the folded Delta projection
+    ssm = B * di * (16 * 4 * 2 + 4 * 4 * 2 + 2 + 2) + di * r * 2.0 + B * r * 2.0
     return {
-        "attn_decode": ("hbm", B * G * cap * (dh + dv) * 2.0),
-        # h and conv state read + written (fp32), x read, y_pre written per (sequence,
-        # channel); W_dt once and the dt_low rows for the folded Delta projection
-        "ssm_decode": ("hbm", B * di * (16 * 4 * 2 + 4 * 4 * 2 + 2 + 2) + di * r * 2.0 + B * r * 2.0),
+        "attn_decode": ("hbm", attn),
+        "ssm_decode": ("hbm", ssm),
+        # 16-bit layers: both in one launch
+        "attn_ssm_decode": ("hbm", attn + ssm),
         "gemm_in_proj_decode": ("hbm", cfg.n_in * cfg.d_model * 2.0),
         "gemm_out_proj_decode": ("hbm", cfg.d_model * di * 2.0),
     }
