@@ -113,12 +113,15 @@ struct RunDst {
 
 // Everything the epilogue does to one run except the store: bias + softplus (Delta),
 // residual (output projection), RoPE (Q and K of the in-projection), and the run's
-// destination. count = 0 when the row has nothing to write.
-template <typename T>
+// destination. count = 0 when the row has nothing to write. KIND >= 0 fixes the
+// epilogue kind at compile time (the kernel then holds that kind's code only);
+// KIND < 0 reads it from e.kind.
+template <typename T, int KIND = -1>
 __device__ __forceinline__ RunDst epi_prepare64(const EpiArgs<T>& e, int r, int c0, float* v) {
+    const int kind = KIND >= 0 ? KIND : e.kind;
     // the element size depends on the launch only (the staged store relies on it being
     // the same in every lane, rows without output included)
-    RunDst d{nullptr, 0, 0, 0, e.kind == EPI_DELTA ? 4 : (int)sizeof(T), 0};
+    RunDst d{nullptr, 0, 0, 0, kind == EPI_DELTA ? 4 : (int)sizeof(T), 0};
     int mode = e.row_mode, M = e.M;
     if (e.meta_pad > 0) {
         if (r < e.meta_pad) {
@@ -130,7 +133,7 @@ __device__ __forceinline__ RunDst epi_prepare64(const EpiArgs<T>& e, int r, int 
     }
     if (r >= M || c0 >= e.N) return d;
     const int n = min(64, e.N - c0);
-    if (e.kind == EPI_DELTA) {
+    if (kind == EPI_DELTA) {
         const float* bias = e.b_dt + c0;
         if (n == 64 && (e.N & 3) == 0) {
             float4 bb[16];
@@ -153,7 +156,7 @@ __device__ __forceinline__ RunDst epi_prepare64(const EpiArgs<T>& e, int r, int 
         d.nbytes = n * 4;
         return d;
     }
-    if (e.kind == EPI_GLU) {
+    if (kind == EPI_GLU) {
         // the gated MLP: SiLU of the gate projection (same row and columns) times this one
         float gv[64];
 #pragma unroll
@@ -166,7 +169,7 @@ __device__ __forceinline__ RunDst epi_prepare64(const EpiArgs<T>& e, int r, int 
         d.nbytes = n * (int)sizeof(T);
         return d;
     }
-    if (e.kind == EPI_OUT) {
+    if (kind == EPI_OUT) {
         if (e.accumulate) {
             d.p = reinterpret_cast<char*>(e.y + (long long)r * e.N + c0);
             d.count = 1;
