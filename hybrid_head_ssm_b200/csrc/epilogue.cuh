@@ -115,15 +115,16 @@ struct RunDst {
 // residual (output projection), RoPE (Q and K of the in-projection), and the run's
 // destination. count = 0 when the row has nothing to write. KIND >= 0 fixes the
 // epilogue kind at compile time (the kernel then holds that kind's code only);
-// KIND < 0 reads it from e.kind.
-template <typename T, int KIND = -1>
+// KIND < 0 reads it from e.kind. DEC fixes the decode form as well: decode rows and no
+// meta rows (in-projection), split-K partial sums (output projection).
+template <typename T, int KIND = -1, bool DEC = false>
 __device__ __forceinline__ RunDst epi_prepare64(const EpiArgs<T>& e, int r, int c0, float* v) {
     const int kind = KIND >= 0 ? KIND : e.kind;
     // the element size depends on the launch only (the staged store relies on it being
     // the same in every lane, rows without output included)
     RunDst d{nullptr, 0, 0, 0, kind == EPI_DELTA ? 4 : (int)sizeof(T), 0};
-    int mode = e.row_mode, M = e.M;
-    if (e.meta_pad > 0) {
+    int mode = DEC ? (int)ROWS_DECODE : e.row_mode, M = e.M;
+    if (!DEC && e.meta_pad > 0) {
         if (r < e.meta_pad) {
             mode = ROWS_META;
             M = e.meta_M;
@@ -170,7 +171,7 @@ __device__ __forceinline__ RunDst epi_prepare64(const EpiArgs<T>& e, int r, int 
         return d;
     }
     if (kind == EPI_OUT) {
-        if (e.accumulate) {
+        if (DEC || e.accumulate) {
             d.p = reinterpret_cast<char*>(e.y + (long long)r * e.N + c0);
             d.count = 1;
             d.nbytes = n * (int)sizeof(T);

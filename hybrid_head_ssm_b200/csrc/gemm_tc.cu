@@ -113,10 +113,10 @@ __device__ __forceinline__ void tile_coords(int tile, int num_m, int num_n, int*
     *n_blk = local / gsize;
 }
 
-// KIND >= 0: the epilogue kind fixed at compile time (the decode projections, whose
-// launches follow kernels that stream far more than L2 holds: a smaller kernel refetches
-// less code); KIND < 0: the kind from the arguments.
-template <typename TA, typename TO, int BN, int STAGES, int KIND = -1>
+// KIND >= 0: the epilogue kind fixed at compile time, and DEC its decode form (the decode
+// projections, whose launches follow kernels that stream far more than L2 holds: a
+// smaller kernel refetches less code); KIND < 0: the kind from the arguments.
+template <typename TA, typename TO, int BN, int STAGES, int KIND = -1, bool DEC = false>
 __global__ void __launch_bounds__(NUM_THREADS, STAGES == 2 ? 2 : 1)
 gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                const __grid_constant__ CUtensorMap tmA0, int M0, int M, int N, int K, int ksplit, EpiArgs<TO> e,
@@ -257,7 +257,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
                     v[i] = __uint_as_float(r0[i]);
                     v[32 + i] = __uint_as_float(r1[i]);
                 }
-                const RunDst d = epi_prepare64<TO, KIND>(e, row, n_blk * BN + j * 64, v);
+                const RunDst d = epi_prepare64<TO, KIND, DEC>(e, row, n_blk * BN + j * 64, v);
                 epi_store_staged<TO>(d, v, s.stage[q], s.info[q], lane);
             }
             tc::tc_fence_before();
@@ -272,7 +272,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     }
 }
 
-template <typename TA, typename TO, int BN, int STAGES, int KIND = -1>
+template <typename TA, typename TO, int BN, int STAGES, int KIND = -1, bool DEC = false>
 int launch_bn(const Ctx& ctx, const char* name, const TA* A, long long lda, const TA* Bw, long long ldb, int M,
               int N, int K, const EpiArgs<TO>& e, const TA* A0, int M0, int ksplit) {
     constexpr bool kBF16 = std::is_same<TA, bf16>::value;
@@ -285,7 +285,7 @@ int launch_bn(const Ctx& ctx, const char* name, const TA* A, long long lda, cons
         ta0 = ta;
     }
     const size_t smem = sizeof(GemmSmem<BN, STAGES>) + 1024;
-    auto kern = gemm_tc_kernel<TA, TO, BN, STAGES, KIND>;
+    auto kern = gemm_tc_kernel<TA, TO, BN, STAGES, KIND, DEC>;
     static std::atomic<unsigned long long> smem_set{0};
     if (!smem_opt_in_once(smem_set, kern, smem, ctx)) return HYMBA_ERR_CUDA;
     const int tiles = ((M0 + BM - 1) / BM + (M + BM - 1) / BM) * ((N + BN - 1) / BN) * ksplit;
@@ -329,7 +329,7 @@ int launch_gemm_tc(const Ctx& ctx, const char* name, const TA* A, long long lda,
         if (sizeof(TO) != 4 || e.kind != EPI_OUT || M0 > 0) return HYMBA_ERR_INVALID_ARG;
         const int tiles = ((M + BM - 1) / BM) * ((N + 63) / 64), nk = (K + BK - 1) / BK;
         const int ksplit = std::max(1, std::min(nk, sms / std::max(1, tiles)));
-        return launch_bn<TA, TO, 64, 4, EPI_OUT>(ctx, name, A, lda, Bw, ldb, M, N, K, e, A0, M0, ksplit);
+        return launch_bn<TA, TO, 64, 4, EPI_OUT, true>(ctx, name, A, lda, Bw, ldb, M, N, K, e, A0, M0, ksplit);
     }
     switch (pick_bn(M + M0, N, sms)) {
         case 256: return launch_bn<TA, TO, 256, 4>(ctx, name, A, lda, Bw, ldb, M, N, K, e, A0, M0, 1);
@@ -341,8 +341,8 @@ int launch_gemm_tc(const Ctx& ctx, const char* name, const TA* A, long long lda,
             // one row block streaming a long K (decode): a deeper ring keeps more weight
             // tiles in flight per CTA
             if (M + M0 <= BM && K > 4 * BK) {
-                if (e.kind == EPI_INPROJ)
-                    return launch_bn<TA, TO, 64, 8, EPI_INPROJ>(ctx, name, A, lda, Bw, ldb, M, N, K, e, A0, M0, 1);
+                if (e.kind == EPI_INPROJ && e.row_mode == ROWS_DECODE && M0 == 0)
+                    return launch_bn<TA, TO, 64, 8, EPI_INPROJ, true>(ctx, name, A, lda, Bw, ldb, M, N, K, e, A0, M0, 1);
                 return launch_bn<TA, TO, 64, 8>(ctx, name, A, lda, Bw, ldb, M, N, K, e, A0, M0, 1);
             }
             return launch_bn<TA, TO, 64, 4>(ctx, name, A, lda, Bw, ldb, M, N, K, e, A0, M0, 1);
