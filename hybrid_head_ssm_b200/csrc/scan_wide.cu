@@ -100,11 +100,25 @@ __device__ __forceinline__ float softplus_bf(float u) {
     return fmaxf(u, 0.0f) + (e < 9.765625e-4f ? series : lg);
 }
 
+// The dt_low pieces (r_dt / 4 per row) a thread copies: j = tid, tid + WTH, ... as (row,
+// piece), the first one and the step, so that each chunk's copies need no division.
+struct DtPieces {
+    int pieces, rr0, k0, drr, dk;
+    __device__ void init(int tid, int r_dt) {
+        pieces = r_dt / 4;
+        rr0 = tid / pieces;
+        k0 = tid - rr0 * pieces;
+        drr = WTH / pieces;
+        dk = WTH - drr * pieces;
+    }
+};
+
 // Stage rows t0 .. t0+WTC-1 of sequence b into buffer buf: x of the block's channels with
 // the WHALO rows before t0 (zeros before the first row), dt_low (r_dt values in 8-byte
 // pieces), B and C. Rows past Tp repeat the last one; they are never scanned.
 __device__ __forceinline__ void stage(WideSmem& sm, int buf, int tid, const f16* P, long long ldP, int col_x,
-                                     int col_B, int col_dt, int r_dt, int c0, long long row0, int t0, int Tp) {
+                                     int col_B, int col_dt, const DtPieces& dp, int c0, long long row0, int t0,
+                                     int Tp) {
     for (int j = tid; j < WXR * (WCH / 8); j += WTH) {
         const int rr = j / (WCH / 8), k = j % (WCH / 8);
         const int t = t0 - WHALO + rr;
@@ -116,11 +130,15 @@ __device__ __forceinline__ void stage(WideSmem& sm, int buf, int tid, const f16*
         const long long row = row0 + min(t0 + rr, Tp - 1);
         cp16(&sm.bc[buf][rr][8 * k], P + row * ldP + col_B + 8 * k);
     }
-    const int pieces = r_dt / 4;
-    for (int j = tid; j < WTC * pieces; j += WTH) {
-        const int rr = j / pieces, k = j - rr * pieces;
+    for (int rr = dp.rr0, k = dp.k0; rr < WTC;) {
         const long long row = row0 + min(t0 + rr, Tp - 1);
         cp8(&sm.dtl[buf][rr][4 * k], P + row * ldP + col_dt + 4 * k);
+        rr += dp.drr;
+        k += dp.dk;
+        if (k >= dp.pieces) {
+            k -= dp.pieces;
+            ++rr;
+        }
     }
 }
 
@@ -144,7 +162,9 @@ conv_scan_wide_kernel(const f16* __restrict__ P, long long ldP, int col_x, int c
         const int bsel = j / (WTC * (WDLD - r_dt)), rem = j - bsel * WTC * (WDLD - r_dt);
         sm.dtl[bsel][rem / (WDLD - r_dt)][r_dt + rem % (WDLD - r_dt)] = __float2half_rn(0.f);
     }
-    stage(sm, 0, tid, P, ldP, col_x, col_B, col_dt, r_dt, c0, row0, 0, Tp);
+    DtPieces dp;
+    dp.init(tid, r_dt);
+    stage(sm, 0, tid, P, ldP, col_x, col_B, col_dt, dp, c0, row0, 0, Tp);
     cp_commit();
 
     // A1 constants: this lane's B fragments of the warp's 16 channels (n-tiles j = 0, 1;
@@ -188,7 +208,7 @@ conv_scan_wide_kernel(const f16* __restrict__ P, long long ldP, int col_x, int c
         const int buf = kc & 1;
         cp_wait0();
         __syncthreads();  // chunk kc staged; everyone is past chunk kc-1's phase B
-        if (kc + 1 < nchunk) stage(sm, buf ^ 1, tid, P, ldP, col_x, col_B, col_dt, r_dt, c0, row0, (kc + 1) * WTC, Tp);
+        if (kc + 1 < nchunk) stage(sm, buf ^ 1, tid, P, ldP, col_x, col_B, col_dt, dp, c0, row0, (kc + 1) * WTC, Tp);
         cp_commit();
 
         // ---- A1: Delta (rows 16 i + g (+8), channels warp*16 + 8 j + 2 q (+1)), B/C to fp32 ----
