@@ -313,10 +313,11 @@ int hymba_get_device_status(void* stream);
 
 /* Where the first bounded device wait that ran out gave up (after a call reported
  * HYMBA_ERR_DEVICE_TIMEOUT): out[0] 1 if a record exists, out[1..3] the block index
- * (x, y, z), out[4] the role (0 TMA producer, 1 MMA issuer, 2 epilogue/softmax, 3 decode
- * attention waiting for its bulk copies, 4 hymba_debug_stalled_wait), out[5] the step
- * (k-block, key block or copy tile), out[6] the barrier (or stage). Synchronises the
- * device and clears the record. Requires n >= 7. */
+ * (x, y, z), out[4] the role (0 TMA producer, 1 MMA issuer, 2 epilogue/softmax,
+ * 4 hymba_debug_stalled_wait; 3 is not used: the decode attention's copies are waited
+ * for by the hardware's own copy-group wait, which always ends), out[5] the step (k-block
+ * or key block), out[6] the barrier (or stage). Synchronises the device and clears the
+ * record. Requires n >= 7. */
 int hymba_get_device_diag(int32_t* out, int n);
 
 /* Failure-path testing. Every device wait of the library that waits for progress
