@@ -18,8 +18,9 @@
 //       the W_dt rows of the warp's 16 channels, which stay in registers, fp32
 //       accumulate) plus a branch-free softplus, stored in conflict-free 8-byte pairs;
 //       B and C converted to fp32;
-//   A2: conv + SiLU of every (row, channel), stored with Delta as the pairs
-//       (Delta, Delta xc) the recurrence consumes, and D xc;
+//   A2: conv + SiLU of every (row, channel), two adjacent channels per thread as fp32
+//       pairs (FFMA2), stored with Delta as the pairs (Delta, Delta xc) the recurrence
+//       consumes, and D xc;
 //   B:  the recurrence. Thread (channel c, half s) holds states 8s .. 8s+7 of c as four
 //       fp32 pairs: per row one 8-byte load of (Delta, Delta xc), B_t and C_t of its half
 //       as fp32 quads shared by the warp, four (FMUL2, 2 ex2, FMUL2, FFMA2, FFMA2) groups,
@@ -187,10 +188,20 @@ conv_scan_wide_kernel(const f16* __restrict__ P, long long ldP, int col_x, int c
 #pragma unroll
     for (int j = 0; j < 2; ++j)
         bdt[j] = *reinterpret_cast<const float2*>(b_dt + c0 + warp * 16 + 8 * j + 2 * q);
-    // A2: conv of channel cc over rows rh .. rh+15 of each chunk
-    const int cc = tid & (WCH - 1), rh = (tid / WCH) * (WTC / 2);
-    const float4 w4 = *reinterpret_cast<const float4*>(conv_w + (long long)(c0 + cc) * 4);
-    const float cbias = conv_b[c0 + cc], Dcc = Dp[c0 + cc];
+    // A2: conv of channels 2 cp, 2 cp + 1 over rows rh .. rh+7 of each chunk
+    constexpr int A2R = WTC / (WTH / (WCH / 2));  // rows per thread: 8
+    const int cp = tid & (WCH / 2 - 1), rh = (tid / (WCH / 2)) * A2R;
+    float2 w2[4];  // tap k of the two channels
+    {
+        const float4 wa = *reinterpret_cast<const float4*>(conv_w + (long long)(c0 + 2 * cp) * 4);
+        const float4 wb = *reinterpret_cast<const float4*>(conv_w + (long long)(c0 + 2 * cp + 1) * 4);
+        w2[0] = make_float2(wa.x, wb.x);
+        w2[1] = make_float2(wa.y, wb.y);
+        w2[2] = make_float2(wa.z, wb.z);
+        w2[3] = make_float2(wa.w, wb.w);
+    }
+    const float2 cb2 = *reinterpret_cast<const float2*>(conv_b + c0 + 2 * cp);
+    const float2 D2 = *reinterpret_cast<const float2*>(Dp + c0 + 2 * cp);
 
     // B: channel cl of the block, states 8 s .. 8 s + 7 as pairs
     const int cl = warp * 16 + (lane >> 1), s = lane & 1;
@@ -247,22 +258,31 @@ conv_scan_wide_kernel(const f16* __restrict__ P, long long ldP, int col_x, int c
         for (int j = tid; j < WTC * 32; j += WTH) sm.bcf[j / 32][j % 32] = __half2float(sm.bc[buf][j / 32][j % 32]);
         __syncthreads();
 
-        // ---- A2: conv + SiLU of channel cc, rows rh .. rh+15 (x row t sits at staged row t + WHALO) ----
+        // ---- A2: conv + SiLU of channels 2 cp, 2 cp + 1, rows rh .. rh+7 (x row t sits at
+        // staged row t + WHALO) ----
         {
-            float x3 = __half2float(sm.x[buf][rh][cc]);
-            float x2 = __half2float(sm.x[buf][rh + 1][cc]);
-            float x1 = __half2float(sm.x[buf][rh + 2][cc]);
+            const float2 nl2 = make_float2(-WLOG2E, -WLOG2E), one2 = make_float2(1.f, 1.f);
+            auto xpair = [&](int row) {
+                return __half22float2(*reinterpret_cast<const __half2*>(&sm.x[buf][row][2 * cp]));
+            };
+            float2 x3 = xpair(rh), x2 = xpair(rh + 1), x1 = xpair(rh + 2);
 #pragma unroll
-            for (int t = rh; t < rh + WTC / 2; ++t) {
-                const float xt = __half2float(sm.x[buf][t + WHALO][cc]);
-                const float u = fmaf(w4.w, xt, fmaf(w4.z, x1, fmaf(w4.y, x2, fmaf(w4.x, x3, cbias))));
+            for (int t = rh; t < rh + A2R; ++t) {
+                const float2 xt = xpair(t + WHALO);
+                float2 u = __ffma2_rn(w2[0], x3, cb2);
+                u = __ffma2_rn(w2[1], x2, u);
+                u = __ffma2_rn(w2[2], x1, u);
+                u = __ffma2_rn(w2[3], xt, u);
                 x3 = x2;
                 x2 = x1;
                 x1 = xt;
-                const float xc = u * rcp_fast(1.0f + fast_exp2(-u * WLOG2E));
-                const float d = sm.dlt[t][cc];
-                sm.dd[t][cc] = make_float2(d, d * xc);
-                sm.dx[t][cc] = Dcc * xc;
+                const float2 ne = __fmul2_rn(u, nl2);
+                const float2 den = __fadd2_rn(make_float2(fast_exp2(ne.x), fast_exp2(ne.y)), one2);
+                const float2 xc = __fmul2_rn(u, make_float2(rcp_fast(den.x), rcp_fast(den.y)));
+                const float2 d = *reinterpret_cast<const float2*>(&sm.dlt[t][2 * cp]);
+                const float2 dxc = __fmul2_rn(d, xc);
+                *reinterpret_cast<float4*>(&sm.dd[t][2 * cp]) = make_float4(d.x, dxc.x, d.y, dxc.y);
+                *reinterpret_cast<float2*>(&sm.dx[t][2 * cp]) = __fmul2_rn(D2, xc);
             }
         }
         __syncthreads();
