@@ -92,13 +92,20 @@ __device__ __forceinline__ void mma16816(float (&c)[4], const uint32_t (&a)[4], 
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
+// softplus of a pair (two adjacent channels), the arithmetic on fp32 pairs:
 // softplus(u) = max(u, 0) + log(1 + e), e = exp(-|u|), branch-free: the series
 // e - e^2/2 + e^3/3 where 1 + e would drop e's low bits (e < 2^-10), the MUFU log2 above.
-__device__ __forceinline__ float softplus_bf(float u) {
-    const float e = fast_exp2(-fabsf(u) * WLOG2E);
-    const float series = e * (1.0f - e * (0.5f - e * (1.0f / 3.0f)));
-    const float lg = lg2_fast(1.0f + e) * 0.69314718055994531f;
-    return fmaxf(u, 0.0f) + (e < 9.765625e-4f ? series : lg);
+__device__ __forceinline__ float2 softplus_bf2(float2 u) {
+    const float2 na = __fmul2_rn(make_float2(fabsf(u.x), fabsf(u.y)), make_float2(-WLOG2E, -WLOG2E));
+    const float2 e = make_float2(fast_exp2(na.x), fast_exp2(na.y));
+    // e (1 - e (1/2 - e / 3)) = e (1 + e (e / 3 - 1/2))
+    const float2 a = __ffma2_rn(e, make_float2(1.0f / 3.0f, 1.0f / 3.0f), make_float2(-0.5f, -0.5f));
+    const float2 series = __fmul2_rn(e, __ffma2_rn(e, a, make_float2(1.f, 1.f)));
+    const float2 ope = __fadd2_rn(e, make_float2(1.f, 1.f));
+    const float2 lg = __fmul2_rn(make_float2(lg2_fast(ope.x), lg2_fast(ope.y)),
+                                 make_float2(0.69314718055994531f, 0.69314718055994531f));
+    return __fadd2_rn(make_float2(fmaxf(u.x, 0.0f), fmaxf(u.y, 0.0f)),
+                      make_float2(e.x < 9.765625e-4f ? series.x : lg.x, e.y < 9.765625e-4f ? series.y : lg.y));
 }
 
 // The dt_low pieces (r_dt / 4 per row) a thread copies: j = tid, tid + WTH, ... as (row,
@@ -249,9 +256,9 @@ conv_scan_wide_kernel(const f16* __restrict__ P, long long ldP, int col_x, int c
                 for (int j = 0; j < 2; ++j) {
                     const int col = warp * 16 + 8 * j + 2 * q;
                     *reinterpret_cast<float2*>(&sm.dlt[16 * i + g][col]) =
-                        make_float2(softplus_bf(acc[i][j][0] + bdt[j].x), softplus_bf(acc[i][j][1] + bdt[j].y));
+                        softplus_bf2(__fadd2_rn(make_float2(acc[i][j][0], acc[i][j][1]), bdt[j]));
                     *reinterpret_cast<float2*>(&sm.dlt[16 * i + g + 8][col]) =
-                        make_float2(softplus_bf(acc[i][j][2] + bdt[j].x), softplus_bf(acc[i][j][3] + bdt[j].y));
+                        softplus_bf2(__fadd2_rn(make_float2(acc[i][j][2], acc[i][j][3]), bdt[j]));
                 }
         }
 #pragma unroll
