@@ -739,9 +739,9 @@ ssm_decode_kernel(const T* __restrict__ P, long long ldP, int col_x, int col_B, 
 }
 
 // The decode attention and the SSM step of a layer in one launch (both read only the
-// in-projection's rows and write disjoint outputs): blocks [0, n_ssm) run the SSM step,
-// the rest the attention's (split, KV head, sequence) blocks, so the SSM's loads of the
-// state overlap the attention's stream of the cache.
+// in-projection's rows and write disjoint outputs): n_ssm blocks, spread evenly through
+// the grid, run the SSM step and the rest the attention's (split, KV head, sequence)
+// blocks, so the SSM's loads of the state overlap the attention's stream of the cache.
 struct DecodeAttnArgs {
     const f16* P;
     long long ldP;
